@@ -1,0 +1,246 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) quantized Mixture-of-Experts FFN layer.
+ *
+ * The layer (GLM-5.2 colibri page "Show HN: getting GLM-5.2 running on my slow
+ * compute", section "What's implemented"; OLMoE page "I ran a 7B
+ * Mixture-of-Experts LLM in a language I built", section "Mixture-of-Experts"):
+ *
+ *   logits  = x . W_r^T                                (fp32 router)
+ *   idx, w  = top-k of softmax(logits)                 (optionally renormalised)
+ *             or DeepSeek-V3-style sigmoid noaux_tc:   s = sigmoid(logits),
+ *             select on s + bias, w = s / sum_sel(s) * routed_scaling_factor
+ *   q_x     = Q8_0-style int8 activations              (group-32 fp16 scales, or
+ *                                                      one fp32 scale per token)
+ *   g, u    = dequant-on-use int8 / packed-int4 expert matmuls (integer dots)
+ *   h       = silu(g) * u, re-quantized like q_x      (SwiGLU)
+ *   y_e     = down projection of h
+ *   y       = sum_j w_j * y_{e_j} + FFN_shared(x)      (shared expert optional)
+ *
+ * with batch-union grouping ("Batch-union MoE" on the GLM page): the (token,
+ * slot) pairs are grouped by expert so every selected expert's weights are
+ * streamed from HBM once per call, whatever the number of tokens routed to it.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named x, y, logits, idx, w, q, scales, workspace, blob data are
+ *     DEVICE pointers owned by the caller; struct arguments themselves
+ *     (moe_expert_blob, moe_route_cfg) live in host memory and are read during
+ *     the call only.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream). Argument and shape checks happen on the host
+ *     before anything is enqueued and return synchronously; nothing is
+ *     enqueued when a call returns an error.
+ *   - The library never allocates device memory and never synchronizes,
+ *     except moe_read_device_status, which synchronizes `stream`.
+ *   - Inputs must be finite. Results for NaN or Inf inputs are unspecified.
+ *   - Supported shapes: hidden H and expert intermediate I multiples of 128;
+ *     1 <= top_k <= min(E, 32); E <= 1024; T >= 0 (T = 0 is a no-op).
+ *
+ * Numerics. Every step that decides an integer (quantized codes, top-k
+ * selection) runs a fixed fp32 operation sequence, so results are bit-exact
+ * across runs and against a CPU implementation of the same sequence:
+ *   - quantization: d = amax / Q (fp32 division, Q = 127 int8 or 7 int4),
+ *     stored as fp32 (per row / per token) or rounded to fp16 (group of 32);
+ *     q = clamp(round_half_away(v / stored_d), -Q, Q); q = 0 if stored_d = 0;
+ *   - router logits: per 32-element chunk an fma chain from +0 in ascending
+ *     index, chunk partials added in ascending chunk order;
+ *   - exp: Cody-Waite reduction by ln 2 with a degree-7 Taylor polynomial,
+ *     argument clamped to [-87, 88]; sigmoid s = 1 / (1 + exp(-L));
+ *   - expert row value: exact int32 dot per group of 32, then
+ *     acc = fma((float)I_g, c_g, acc) over ascending groups from +0, where c_g
+ *     is the product of the two group scales (both group-32) or the scale that
+ *     varies by group, and the per-row / per-token scale multiplies the end;
+ *     per-row weights with per-token activations form one group (the row);
+ *   - SwiGLU h = (g / (1 + exp(-g))) * u.
+ * The down projection and the weighted combine are fp32 in an unspecified
+ * order (fp32 atomic adds into y); their rounding differs from run to run by
+ * a few ulp.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum value */
+  MOE_ERR_UNSUPPORTED = 2,   /* shape or format combination outside the supported set */
+  MOE_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+  MOE_ERR_CUDA = 4,          /* a CUDA launch or copy failed (cudaGetLastError) */
+  MOE_ERR_DEVICE_CHECK = 5,  /* a kernel found an out-of-range index at run time */
+  MOE_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up */
+} moe_status;
+
+/* Expert weight code type. Packed int4: two's-complement nibbles, two per byte. */
+enum { MOE_W_INT8 = 0, MOE_W_INT4 = 1 };
+/* Weight scale granularity: one fp32 per row, or one fp16 per 32 values of a row. */
+enum { MOE_SCALE_ROW_F32 = 0, MOE_SCALE_G32_F16 = 1 };
+/* Activation quantization: one fp32 scale per token, or Q8_0-style fp16 per 32. */
+enum { MOE_ACT_TOKEN_F32 = 0, MOE_ACT_G32_F16 = 1 };
+/* Router scoring. */
+enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID_NOAUX_TC = 1 };
+
+/* moe_route_cfg.flags */
+#define MOE_FLAG_DEBUG 1u          /* also keep gate/up stage values and per-pair down values
+                                      in the workspace (see moe_layer_debug_views) */
+#define MOE_FLAG_FORCE_GEMV 2u     /* run every expert on the weight-streaming (GEMV) path */
+
+/* A set of E quantized experts of one layer (or the single shared expert, E = 1).
+ *
+ * `data` (device, 256-byte aligned, caller-owned) holds `bytes` >= moe_expert_blob_bytes().
+ * Byte layout, four regions each starting at a multiple of 256 bytes from `data`:
+ *   R0 gate/up codes: for each expert e, for each s in [0, I/128): a block of
+ *      256 rows -- rows 0..127 are gate rows 128s..128s+127, rows 128..255 the
+ *      up rows of the same intermediate indices -- stored as [KB/16][256][16]:
+ *      16-byte piece p of row r at (p * 256 + r) * 16. KB = H (int8) or H/2
+ *      (int4; element 2j in the low nibble of byte j).
+ *   R1 down codes: for each e, for each s in [0, H/128): rows 128s..128s+127 of
+ *      the [H][I] down matrix stored [KBd/16][128][16], KBd = I or I/2.
+ *   R2 gate/up scales: for each e, each 256-row block: fp16 [H/32][256]
+ *      (group-major) or fp32 [256].
+ *   R3 down scales: for each e, each 128-row block: fp16 [I/32][128] or fp32 [128].
+ * Padding bytes between regions are zero. */
+typedef struct {
+  int32_t wtype;      /* MOE_W_INT8 | MOE_W_INT4 */
+  int32_t wscale;     /* MOE_SCALE_ROW_F32 | MOE_SCALE_G32_F16 */
+  int32_t n_experts;  /* E */
+  int32_t hidden;     /* H */
+  int32_t inter;      /* I */
+  int32_t reserved;
+  void* data;         /* device */
+  size_t bytes;
+} moe_expert_blob;
+
+typedef struct {
+  int32_t score;                /* MOE_SCORE_* */
+  int32_t top_k;
+  int32_t renormalize;          /* softmax: weights over the selected experts sum to 1;
+                                   sigmoid: weights = s / sum of selected s */
+  float routed_scaling_factor;  /* multiplies every routing weight (1.0 for plain softmax) */
+  int32_t act;                  /* MOE_ACT_* (applies to x and to h) */
+  uint32_t flags;               /* MOE_FLAG_* */
+} moe_route_cfg;
+
+/* Version of this ABI (MOE_ABI_VERSION). */
+MOE_API int32_t moe_abi_version(void);
+
+/* Human-readable name of a status code (static string). */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Bytes a blob of this format needs; 0 if the shape or format is unsupported. */
+MOE_API size_t moe_expert_blob_bytes(int32_t wtype, int32_t wscale, int32_t n_experts, int32_t hidden,
+                             int32_t inter);
+
+/* Quantize fp32 expert weights into `out` (GLM page, "Quantization kernels: int8 / packed
+ * int4 ... per-row scales, dequant-on-use"; group size 32 from the mtlm-7m-base card).
+ *   w_gate_up [E][2I][H] fp32: rows 0..I-1 the gate projection, I..2I-1 the up projection;
+ *   w_down    [E][H][I] fp32.
+ * out->wtype, wscale, n_experts, hidden, inter, data and bytes are set by the caller;
+ * the blob is fully rewritten (padding zeroed). Errors: INVALID_ARG (null), UNSUPPORTED
+ * (shape), WORKSPACE (out->bytes too small). */
+MOE_API moe_status moe_quantize_experts(const float* w_gate_up, const float* w_down,
+                                const moe_expert_blob* out, void* stream);
+
+/* Q8_0-style activation quantization (GLM page, "Integer-dot kernels (Q8_0-style int8
+ * activations ...)").  x [T][H] fp32 -> q [T][H] int8 and `scales`: fp16 [T][H/32]
+ * (MOE_ACT_G32_F16) or fp32 [T] (MOE_ACT_TOKEN_F32). H multiple of 32. */
+MOE_API moe_status moe_quantize_activations(const float* x, int32_t T, int32_t H, int32_t act,
+                                    int8_t* q, void* scales, void* stream);
+
+/* Router logits [T][E] = x [T][H] . router_w [E][H]^T in the fixed fp32 order above. */
+MOE_API moe_status moe_router_logits(const float* x, const float* router_w, int32_t T, int32_t E,
+                             int32_t H, float* logits, void* stream);
+
+/* Top-k selection and routing weights from logits [T][E] (GLM page: "DeepSeek-V3-style
+ * sigmoid router (noaux_tc, routed_scaling_factor)"; OLMoE page: "top-8 of 64").
+ * bias [E] (sigmoid mode only, may be NULL = zeros) shifts the selection key, never the
+ * weights. idx [T][k] int32 in descending key order (ties: lower expert index first),
+ * w [T][k] fp32. */
+MOE_API moe_status moe_route_topk(const float* logits, const float* bias, int32_t T, int32_t E,
+                          const moe_route_cfg* cfg, int32_t* idx, float* w, void* stream);
+
+/* Workspace bytes moe_permute needs for (T, k, E). */
+MOE_API size_t moe_permute_workspace_bytes(int32_t T, int32_t k, int32_t E);
+
+/* Batch-union grouping (GLM page, "Batch-union MoE"): offsets [E+1] (offsets[e] = first
+ * position of expert e) and perm [T*k], the pair indices t*k+j sorted by (expert, t).
+ * idx values must lie in [0, E); out-of-range values set MOE_ERR_DEVICE_CHECK in the
+ * workspace status word and are dropped. */
+MOE_API moe_status moe_permute(const int32_t* idx, int32_t T, int32_t k, int32_t E, int32_t* offsets,
+                       int32_t* perm, void* workspace, size_t ws_bytes, void* stream);
+
+/* Workspace bytes moe_layer_forward needs; 0 if the arguments are unsupported. */
+MOE_API size_t moe_layer_workspace_bytes(int32_t T, const moe_expert_blob* experts,
+                                 const moe_expert_blob* shared, const moe_route_cfg* cfg);
+
+/* The whole layer: y [T][H] fp32 (overwritten) from x [T][H] fp32.
+ *   router_w [E][H] fp32; router_bias [E] fp32 or NULL (sigmoid mode only);
+ *   experts: the routed experts; shared: NULL or one expert (n_experts = 1) with the same
+ *   hidden size, wtype and wscale as `experts` and its own intermediate size.
+ * workspace: device buffer of ws_bytes >= moe_layer_workspace_bytes(); it holds every
+ * intermediate (quantized x, logits, routing, grouping, quantized h) and the device status
+ * word. Calls that share a workspace must be ordered on one stream. */
+MOE_API moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
+                             const float* router_bias, const moe_expert_blob* experts,
+                             const moe_expert_blob* shared, const moe_route_cfg* cfg, float* y,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Byte offsets, inside a moe_layer_forward workspace, of the intermediates of the last
+ * call with the same (T, experts, shared, cfg). -1 = not kept for this configuration.
+ * Pair rows are in grouped order: row r of q_h / s_h / gate / up / y_pair belongs to the
+ * (token, slot) pair perm[r]; shared-expert rows follow as rows T*k + t. */
+typedef struct {
+  int64_t status;       /* int32 device status word (moe_status value) */
+  int64_t q_x;          /* int8 [T][H] */
+  int64_t s_x;          /* fp16 [T][H/32] or fp32 [T] */
+  int64_t logits;       /* fp32 [T][E] */
+  int64_t idx;          /* int32 [T][k] */
+  int64_t w;            /* fp32 [T][k] */
+  int64_t offsets;      /* int32 [E+1] */
+  int64_t perm;         /* int32 [T*k] */
+  int64_t n_active;     /* int32: number of distinct experts selected */
+  int64_t act_expert;   /* int32 [n_active] distinct experts, ascending */
+  int64_t q_h;          /* int8 [T*k][I] then [T][I_shared] */
+  int64_t s_h;          /* fp16 [T*k][I/32] then [T][I_s/32], or fp32 [T*k] then [T] */
+  int64_t gate;         /* MOE_FLAG_DEBUG: fp32 [T*k][I] then [T][I_s] */
+  int64_t up;           /* MOE_FLAG_DEBUG: fp32, same shape */
+  int64_t y_pair;       /* MOE_FLAG_DEBUG: fp32 [T*k][H] then [T][H]: expert outputs before
+                           the combine */
+  int64_t total;        /* == moe_layer_workspace_bytes() */
+} moe_debug_views;
+
+MOE_API moe_status moe_layer_debug_views(int32_t T, const moe_expert_blob* experts,
+                                 const moe_expert_blob* shared, const moe_route_cfg* cfg,
+                                 moe_debug_views* out);
+
+/* Per-group exact int32 dots of sampled expert rows against given int8 activation rows, read
+ * through the blob layout (the integer-dot step of the GLM page's "Integer-dot kernels").
+ *   which 0: gate/up rows (logical row r in [0, 2I) of [2I][H]), K = H;
+ *   which 1: down rows (r in [0, H) of [H][I]), K = I.
+ * expert [n], row [n]: int32; act [n][K] int8; dots [n][K/32] int32. */
+MOE_API moe_status moe_expert_group_dots(const moe_expert_blob* blob, int32_t which, int32_t n,
+                                 const int32_t* expert, const int32_t* row, const int8_t* act,
+                                 int32_t* dots, void* stream);
+
+/* Reads and clears the device status word of a moe_layer_forward / moe_permute workspace.
+ * Synchronizes `stream`. Returns MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT as
+ * recorded by the kernels, or MOE_ERR_CUDA if the copy fails. */
+MOE_API moe_status moe_read_device_status(void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

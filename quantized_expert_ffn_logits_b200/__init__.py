@@ -1,0 +1,299 @@
+"""Python binding of the B200 quantized MoE FFN layer (include/moe_b200.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels of
+``_lib/libmoe_b200.so``; torch supplies device memory and the current stream.
+The entry points keep the C names. Importing this package fails loudly when the
+shared library is missing: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_lib", "libmoe_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"CUDA library not built: {LIB_PATH} (run quantized_expert_ffn_logits_b200/build.py)")
+
+_lib = C.CDLL(LIB_PATH)
+
+# ---------------------------------------------------------------- constants
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, 1, 2, 3
+MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT = 4, 5, 6
+MOE_W_INT8, MOE_W_INT4 = 0, 1
+MOE_SCALE_ROW_F32, MOE_SCALE_G32_F16 = 0, 1
+MOE_ACT_TOKEN_F32, MOE_ACT_G32_F16 = 0, 1
+MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID_NOAUX_TC = 0, 1
+MOE_FLAG_DEBUG, MOE_FLAG_FORCE_GEMV = 1, 2
+
+WTYPES = {"int8": MOE_W_INT8, "int4": MOE_W_INT4}
+WSCALES = {"row_f32": MOE_SCALE_ROW_F32, "g32_f16": MOE_SCALE_G32_F16}
+ACTS = {"token_f32": MOE_ACT_TOKEN_F32, "g32_f16": MOE_ACT_G32_F16}
+SCORES = {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID_NOAUX_TC}
+
+
+class moe_expert_blob(C.Structure):
+    _fields_ = [("wtype", C.c_int32), ("wscale", C.c_int32), ("n_experts", C.c_int32),
+                ("hidden", C.c_int32), ("inter", C.c_int32), ("reserved", C.c_int32),
+                ("data", C.c_void_p), ("bytes", C.c_size_t)]
+
+
+class moe_route_cfg(C.Structure):
+    _fields_ = [("score", C.c_int32), ("top_k", C.c_int32), ("renormalize", C.c_int32),
+                ("routed_scaling_factor", C.c_float), ("act", C.c_int32), ("flags", C.c_uint32)]
+
+
+class moe_debug_views(C.Structure):
+    _fields_ = [(n, C.c_int64) for n in ("status", "q_x", "s_x", "logits", "idx", "w", "offsets",
+                                          "perm", "n_active", "act_expert", "q_h", "s_h", "gate",
+                                          "up", "y_pair", "total")]
+
+
+_vp, _i32, _sz = C.c_void_p, C.c_int32, C.c_size_t
+_PB, _PC = C.POINTER(moe_expert_blob), C.POINTER(moe_route_cfg)
+_SIGS = {
+    "moe_abi_version": (_i32, []),
+    "moe_status_string": (C.c_char_p, [_i32]),
+    "moe_expert_blob_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
+    "moe_quantize_experts": (_i32, [_vp, _vp, _PB, _vp]),
+    "moe_quantize_activations": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_router_logits": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp]),
+    "moe_route_topk": (_i32, [_vp, _vp, _i32, _i32, _PC, _vp, _vp, _vp]),
+    "moe_permute_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "moe_layer_workspace_bytes": (_sz, [_i32, _PB, _PB, _PC]),
+    "moe_layer_forward": (_i32, [_vp, _i32, _vp, _vp, _PB, _PB, _PC, _vp, _vp, _sz, _vp]),
+    "moe_layer_debug_views": (_i32, [_i32, _PB, _PB, _PC, C.POINTER(moe_debug_views)]),
+    "moe_expert_group_dots": (_i32, [_PB, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "moe_read_device_status": (_i32, [_vp, _sz, _vp]),
+}
+EXPORTS = tuple(_SIGS)
+for _name, (_res, _args) in _SIGS.items():
+    _fn = getattr(_lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {moe_status_string(status)}")
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != MOE_OK:
+        raise MoeError(rc, where)
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t, dtype, name):
+    import torch
+    if t is None:
+        return None
+    if not (t.is_cuda and t.dtype == dtype and t.is_contiguous()):
+        raise ValueError(f"{name}: expected a contiguous CUDA {dtype} tensor, got "
+                         f"{t.dtype} on {t.device} (contiguous={t.is_contiguous()})")
+    return t
+
+
+# ---------------------------------------------------------------- config objects
+@dataclass
+class RouteCfg:
+    score: str = "softmax"
+    top_k: int = 8
+    renormalize: bool = True
+    routed_scaling_factor: float = 1.0
+    act: str = "g32_f16"
+    flags: int = 0
+
+    def struct(self) -> moe_route_cfg:
+        return moe_route_cfg(SCORES[self.score], self.top_k, int(self.renormalize),
+                             float(self.routed_scaling_factor), ACTS[self.act], self.flags)
+
+
+class ExpertBlob:
+    """A quantized expert set in one device byte buffer (layout: include/moe_b200.h)."""
+
+    def __init__(self, wtype: str, wscale: str, n_experts: int, hidden: int, inter: int,
+                 data=None, device=None):
+        import torch
+        self.wtype, self.wscale = wtype, wscale
+        self.n_experts, self.hidden, self.inter = n_experts, hidden, inter
+        nbytes = moe_expert_blob_bytes(WTYPES[wtype], WSCALES[wscale], n_experts, hidden, inter)
+        if nbytes == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "moe_expert_blob_bytes")
+        if data is None:
+            data = torch.empty(nbytes, dtype=torch.uint8, device=device or "cuda")
+        if data.numel() < nbytes:
+            raise ValueError("blob buffer too small")
+        self.data = _dev(data, torch.uint8, "blob")
+        self.nbytes = nbytes
+
+    def struct(self) -> moe_expert_blob:
+        return moe_expert_blob(WTYPES[self.wtype], WSCALES[self.wscale], self.n_experts,
+                               self.hidden, self.inter, 0, self.data.data_ptr(), self.data.numel())
+
+    @classmethod
+    def quantize(cls, w_gate_up, w_down, wtype: str, wscale: str, stream=None) -> "ExpertBlob":
+        """w_gate_up [E][2I][H], w_down [E][H][I] fp32 CUDA tensors -> blob."""
+        E, twoI, H = w_gate_up.shape
+        b = cls(wtype, wscale, E, H, twoI // 2, device=w_gate_up.device)
+        moe_quantize_experts(w_gate_up, w_down, b, stream)
+        return b
+
+
+# ---------------------------------------------------------------- entry points
+def moe_abi_version() -> int:
+    return int(_lib.moe_abi_version())
+
+
+def moe_status_string(status: int) -> str:
+    return _lib.moe_status_string(int(status)).decode()
+
+
+def moe_expert_blob_bytes(wtype: int, wscale: int, n_experts: int, hidden: int, inter: int) -> int:
+    return int(_lib.moe_expert_blob_bytes(wtype, wscale, n_experts, hidden, inter))
+
+
+def moe_quantize_experts(w_gate_up, w_down, blob: ExpertBlob, stream=None) -> None:
+    import torch
+    _dev(w_gate_up, torch.float32, "w_gate_up")
+    _dev(w_down, torch.float32, "w_down")
+    st = blob.struct()
+    _check(_lib.moe_quantize_experts(_ptr(w_gate_up), _ptr(w_down), C.byref(st), _stream(stream)),
+           "moe_quantize_experts")
+
+
+def moe_quantize_activations(x, act: str = "g32_f16", stream=None):
+    import torch
+    _dev(x, torch.float32, "x")
+    T, H = x.shape
+    q = torch.empty((T, H), dtype=torch.int8, device=x.device)
+    if ACTS[act] == MOE_ACT_G32_F16:
+        s = torch.empty((T, H // 32), dtype=torch.float16, device=x.device)
+    else:
+        s = torch.empty((T,), dtype=torch.float32, device=x.device)
+    _check(_lib.moe_quantize_activations(_ptr(x), T, H, ACTS[act], _ptr(q), _ptr(s), _stream(stream)),
+           "moe_quantize_activations")
+    return q, s
+
+
+def moe_router_logits(x, router_w, stream=None):
+    import torch
+    _dev(x, torch.float32, "x")
+    _dev(router_w, torch.float32, "router_w")
+    T, H = x.shape
+    E = router_w.shape[0]
+    out = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    _check(_lib.moe_router_logits(_ptr(x), _ptr(router_w), T, E, H, _ptr(out), _stream(stream)),
+           "moe_router_logits")
+    return out
+
+
+def moe_route_topk(logits, bias, cfg: RouteCfg, stream=None):
+    import torch
+    _dev(logits, torch.float32, "logits")
+    _dev(bias, torch.float32, "bias")
+    T, E = logits.shape
+    idx = torch.empty((T, cfg.top_k), dtype=torch.int32, device=logits.device)
+    w = torch.empty((T, cfg.top_k), dtype=torch.float32, device=logits.device)
+    st = cfg.struct()
+    _check(_lib.moe_route_topk(_ptr(logits), _ptr(bias), T, E, C.byref(st), _ptr(idx), _ptr(w),
+                               _stream(stream)), "moe_route_topk")
+    return idx, w
+
+
+def moe_permute(idx, n_experts: int, stream=None):
+    import torch
+    _dev(idx, torch.int32, "idx")
+    T, k = idx.shape
+    nb = int(_lib.moe_permute_workspace_bytes(T, k, n_experts))
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device=idx.device)
+    offsets = torch.empty(n_experts + 1, dtype=torch.int32, device=idx.device)
+    perm = torch.empty(T * k, dtype=torch.int32, device=idx.device)
+    _check(_lib.moe_permute(_ptr(idx), T, k, n_experts, _ptr(offsets), _ptr(perm), _ptr(ws),
+                            ws.numel(), _stream(stream)), "moe_permute")
+    return offsets, perm, ws
+
+
+def moe_layer_workspace_bytes(T: int, experts: ExpertBlob, shared: ExpertBlob | None,
+                              cfg: RouteCfg) -> int:
+    e = experts.struct()
+    s = shared.struct() if shared is not None else None
+    c = cfg.struct()
+    return int(_lib.moe_layer_workspace_bytes(T, C.byref(e), C.byref(s) if s else None, C.byref(c)))
+
+
+def moe_layer_forward(x, router_w, router_bias, experts: ExpertBlob, shared: ExpertBlob | None,
+                      cfg: RouteCfg, y=None, workspace=None, stream=None):
+    """y [T][H] = MoE FFN layer(x [T][H]). Returns (y, workspace)."""
+    import torch
+    _dev(x, torch.float32, "x")
+    _dev(router_w, torch.float32, "router_w")
+    _dev(router_bias, torch.float32, "router_bias")
+    T, H = x.shape
+    if y is None:
+        y = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    _dev(y, torch.float32, "y")
+    nb = moe_layer_workspace_bytes(T, experts, shared, cfg)
+    if nb == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(nb, dtype=torch.uint8, device=x.device)
+    _dev(workspace, torch.uint8, "workspace")
+    e = experts.struct()
+    s = shared.struct() if shared is not None else None
+    c = cfg.struct()
+    _check(_lib.moe_layer_forward(_ptr(x), T, _ptr(router_w), _ptr(router_bias), C.byref(e),
+                                  C.byref(s) if s else None, C.byref(c), _ptr(y), _ptr(workspace),
+                                  workspace.numel(), _stream(stream)), "moe_layer_forward")
+    return y, workspace
+
+
+def moe_layer_debug_views(T: int, experts: ExpertBlob, shared: ExpertBlob | None,
+                          cfg: RouteCfg) -> dict:
+    e = experts.struct()
+    s = shared.struct() if shared is not None else None
+    c = cfg.struct()
+    v = moe_debug_views()
+    _check(_lib.moe_layer_debug_views(T, C.byref(e), C.byref(s) if s else None, C.byref(c),
+                                      C.byref(v)), "moe_layer_debug_views")
+    return {n: getattr(v, n) for n, _ in moe_debug_views._fields_}
+
+
+def moe_expert_group_dots(blob: ExpertBlob, which: int, expert, row, act, stream=None):
+    import torch
+    _dev(expert, torch.int32, "expert")
+    _dev(row, torch.int32, "row")
+    _dev(act, torch.int8, "act")
+    n, K = act.shape
+    dots = torch.empty((n, K // 32), dtype=torch.int32, device=act.device)
+    b = blob.struct()
+    _check(_lib.moe_expert_group_dots(C.byref(b), which, n, _ptr(expert), _ptr(row), _ptr(act),
+                                      _ptr(dots), _stream(stream)), "moe_expert_group_dots")
+    return dots
+
+
+def moe_read_device_status(workspace, stream=None) -> int:
+    return int(_lib.moe_read_device_status(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def workspace_view(workspace, offset: int, dtype, shape):
+    """A typed tensor view of a region of a layer workspace (for inspecting intermediates)."""
+    import torch
+    n = 1
+    for d in shape:
+        n *= d
+    nbytes = n * torch.empty((), dtype=dtype).element_size()
+    return workspace[offset:offset + nbytes].view(dtype).view(*shape)

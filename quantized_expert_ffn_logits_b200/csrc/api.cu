@@ -1,0 +1,455 @@
+// api.cu -- the C ABI (include/moe_b200.h): argument checks, workspace layout and
+// the launch sequence of the layer forward.
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/moe_b200.h"
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+using moe::BlobView;
+
+inline int64_t al256(int64_t v) { return (v + 255) & ~int64_t(255); }
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+struct BlobOffsets {
+  int64_t gu_w, dn_w, gu_s, dn_s, total;
+};
+
+bool blob_offsets(int32_t wtype, int32_t wscale, int32_t E, int32_t H, int32_t I, BlobOffsets& o) {
+  if ((wtype != MOE_W_INT8 && wtype != MOE_W_INT4) ||
+      (wscale != MOE_SCALE_ROW_F32 && wscale != MOE_SCALE_G32_F16))
+    return false;
+  if (E < 1 || E > 1024 || H < 128 || I < 128 || H % 128 || I % 128) return false;
+  const int64_t kb_gu = wtype == MOE_W_INT8 ? H : H / 2;
+  const int64_t kb_dn = wtype == MOE_W_INT8 ? I : I / 2;
+  const int64_t s_gu = wscale == MOE_SCALE_G32_F16 ? (int64_t)(H / 32) * 2 : 4;
+  const int64_t s_dn = wscale == MOE_SCALE_G32_F16 ? (int64_t)(I / 32) * 2 : 4;
+  o.gu_w = 0;
+  o.dn_w = al256(o.gu_w + (int64_t)E * 2 * I * kb_gu);
+  o.gu_s = al256(o.dn_w + (int64_t)E * H * kb_dn);
+  o.dn_s = al256(o.gu_s + (int64_t)E * 2 * I * s_gu);
+  o.total = al256(o.dn_s + (int64_t)E * H * s_dn);
+  return true;
+}
+
+moe_status check_blob(const moe_expert_blob* b, BlobOffsets& o) {
+  if (!b || !b->data) return MOE_ERR_INVALID_ARG;
+  if (!blob_offsets(b->wtype, b->wscale, b->n_experts, b->hidden, b->inter, o))
+    return MOE_ERR_UNSUPPORTED;
+  if (!aligned(b->data, 256)) return MOE_ERR_INVALID_ARG;
+  if ((int64_t)b->bytes < o.total) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+BlobView view(const moe_expert_blob* b, const BlobOffsets& o) {
+  const uint8_t* d = static_cast<const uint8_t*>(b->data);
+  BlobView v;
+  v.gu_w = d + o.gu_w;
+  v.dn_w = d + o.dn_w;
+  v.gu_s = d + o.gu_s;
+  v.dn_s = d + o.dn_s;
+  v.E = b->n_experts;
+  v.H = b->hidden;
+  v.I = b->inter;
+  v.wbits = b->wtype == MOE_W_INT8 ? 8 : 4;
+  v.wg32 = b->wscale == MOE_SCALE_G32_F16;
+  return v;
+}
+
+moe_status check_cfg(const moe_route_cfg* c, int32_t E) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID_NOAUX_TC) return MOE_ERR_INVALID_ARG;
+  if (c->act != MOE_ACT_TOKEN_F32 && c->act != MOE_ACT_G32_F16) return MOE_ERR_INVALID_ARG;
+  if (c->top_k < 1 || c->top_k > 32 || c->top_k > E) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// Workspace of one layer forward: every region starts at a multiple of 256 bytes.
+struct Layout {
+  int64_t status, qx, sx, logits, idx, w, offsets, perm, n_active, act_expert, act_begin;
+  int64_t masks, base, qh, sh, hbuf, dbg_gate, dbg_up, dbg_y, total;
+  int64_t qh_sh, sh_sh, hbuf_sh, dbg_gate_sh, dbg_up_sh, dbg_y_sh;   // shared-expert rows
+};
+
+Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k, int32_t ag32,
+              bool debug) {
+  Layout L;
+  int64_t o = 0;
+  auto take = [&](int64_t bytes) {
+    const int64_t at = o;
+    o = al256(o + (bytes > 0 ? bytes : 0));
+    return at;
+  };
+  const int64_t P = (int64_t)T * k;
+  const int64_t C = (T + 31) / 32;
+  L.status = take(256);
+  L.qx = take((int64_t)T * H);
+  L.sx = take(ag32 ? (int64_t)T * (H / 32) * 2 : (int64_t)T * 4);
+  L.logits = take((int64_t)T * E * 4);
+  L.idx = take(P * 4);
+  L.w = take(P * 4);
+  L.offsets = take((int64_t)(E + 1) * 4);
+  L.perm = take(P * 4);
+  L.n_active = take(4);
+  L.act_expert = take((int64_t)(E + 1) * 4);
+  L.act_begin = take((int64_t)(E + 2) * 4);
+  L.masks = take(T > 1 ? C * E * 4 : 0);
+  L.base = take(T > 1 ? C * E * 4 : 0);
+  const int64_t rows_h = P * I + (int64_t)T * Is;
+  L.qh = take(rows_h);
+  L.qh_sh = L.qh + P * I;
+  if (ag32) {
+    L.sh = take((P * (I / 32) + (int64_t)T * (Is / 32)) * 2);
+    L.sh_sh = L.sh + P * (I / 32) * 2;
+  } else {
+    L.sh = take((P + T) * 4);
+    L.sh_sh = L.sh + P * 4;
+  }
+  if (!ag32) {
+    L.hbuf = take(rows_h * 4);
+    L.hbuf_sh = L.hbuf + P * I * 4;
+  } else {
+    L.hbuf = L.hbuf_sh = -1;
+  }
+  if (debug) {
+    L.dbg_gate = take(rows_h * 4);
+    L.dbg_gate_sh = L.dbg_gate + P * I * 4;
+    L.dbg_up = take(rows_h * 4);
+    L.dbg_up_sh = L.dbg_up + P * I * 4;
+    L.dbg_y = take((P + T) * H * 4);
+    L.dbg_y_sh = L.dbg_y + P * H * 4;
+  } else {
+    L.dbg_gate = L.dbg_up = L.dbg_y = -1;
+    L.dbg_gate_sh = L.dbg_up_sh = L.dbg_y_sh = -1;
+  }
+  L.total = o;
+  return L;
+}
+
+struct LayerPlan {
+  BlobOffsets eo, so;
+  int32_t Is;
+  Layout L;
+};
+
+moe_status plan_layer(int32_t T, const moe_expert_blob* experts, const moe_expert_blob* shared,
+                      const moe_route_cfg* cfg, LayerPlan& p) {
+  if (T < 0) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_blob(experts, p.eo);
+  if (s != MOE_OK) return s;
+  s = check_cfg(cfg, experts->n_experts);
+  if (s != MOE_OK) return s;
+  p.Is = 0;
+  if (shared) {
+    s = check_blob(shared, p.so);
+    if (s != MOE_OK) return s;
+    if (shared->n_experts != 1 || shared->hidden != experts->hidden ||
+        shared->wtype != experts->wtype || shared->wscale != experts->wscale)
+      return MOE_ERR_UNSUPPORTED;
+    p.Is = shared->inter;
+  }
+  p.L = layout(T, experts->n_experts, experts->hidden, experts->inter, p.Is, cfg->top_k,
+               cfg->act == MOE_ACT_G32_F16, (cfg->flags & MOE_FLAG_DEBUG) != 0);
+  return MOE_OK;
+}
+
+moe_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_DEVICE_CHECK: return "MOE_ERR_DEVICE_CHECK";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+size_t moe_expert_blob_bytes(int32_t wtype, int32_t wscale, int32_t n_experts, int32_t hidden,
+                             int32_t inter) {
+  BlobOffsets o;
+  if (!blob_offsets(wtype, wscale, n_experts, hidden, inter, o)) return 0;
+  return (size_t)o.total;
+}
+
+moe_status moe_quantize_experts(const float* w_gate_up, const float* w_down,
+                                const moe_expert_blob* out, void* stream) {
+  if (!w_gate_up || !w_down) return MOE_ERR_INVALID_ARG;
+  BlobOffsets o;
+  const moe_status s = check_blob(out, o);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(out->data, 0, (size_t)o.total, st) != cudaSuccess) return MOE_ERR_CUDA;
+  const BlobView b = view(out, o);
+  uint8_t* d = static_cast<uint8_t*>(out->data);
+  moe::launch_quantize_experts(w_gate_up, w_down, b, d + o.gu_w, d + o.dn_w, d + o.gu_s,
+                               d + o.dn_s, st);
+  return launch_status();
+}
+
+moe_status moe_quantize_activations(const float* x, int32_t T, int32_t H, int32_t act, int8_t* q,
+                                    void* scales, void* stream) {
+  if (T < 0 || H <= 0 || H % 32) return T < 0 ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED;
+  if (act != MOE_ACT_TOKEN_F32 && act != MOE_ACT_G32_F16) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !q || !scales) return MOE_ERR_INVALID_ARG;
+  moe::launch_quantize_act(x, T, H, act == MOE_ACT_G32_F16, q, scales, nullptr, nullptr,
+                           static_cast<cudaStream_t>(stream));
+  return launch_status();
+}
+
+moe_status moe_router_logits(const float* x, const float* router_w, int32_t T, int32_t E,
+                             int32_t H, float* logits, void* stream) {
+  if (T < 0 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (H <= 0 || H % 32) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!x || !router_w || !logits || !aligned(x, 16) || !aligned(router_w, 16))
+    return MOE_ERR_INVALID_ARG;
+  moe::launch_router_logits(x, router_w, T, E, H, logits, static_cast<cudaStream_t>(stream));
+  return launch_status();
+}
+
+moe_status moe_route_topk(const float* logits, const float* bias, int32_t T, int32_t E,
+                          const moe_route_cfg* cfg, int32_t* idx, float* w, void* stream) {
+  if (T < 0 || E < 1 || E > 1024) return E > 1024 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
+  const moe_status s = check_cfg(cfg, E);
+  if (s != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  if (!logits || !idx || !w) return MOE_ERR_INVALID_ARG;
+  moe::launch_topk(logits, cfg->score == MOE_SCORE_SIGMOID_NOAUX_TC ? bias : nullptr, T, E,
+                   cfg->top_k, cfg->score, cfg->renormalize != 0, cfg->routed_scaling_factor, idx,
+                   w, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+  return launch_status();
+}
+
+size_t moe_permute_workspace_bytes(int32_t T, int32_t k, int32_t E) {
+  if (T < 0 || k < 1 || E < 1 || E > 1024) return 0;
+  const int64_t C = (T + 31) / 32;
+  return (size_t)(256 + al256(C * E * 4) * 2 + 256 + al256((int64_t)(E + 1) * 4) +
+                  al256((int64_t)(E + 2) * 4));
+}
+
+moe_status moe_permute(const int32_t* idx, int32_t T, int32_t k, int32_t E, int32_t* offsets,
+                       int32_t* perm, void* workspace, size_t ws_bytes, void* stream) {
+  if (T < 0 || k < 1 || E < 1) return MOE_ERR_INVALID_ARG;
+  if (E > 1024 || k > 32 || k > E) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (!idx || !offsets || !perm || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < moe_permute_workspace_bytes(T, k, E)) return MOE_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const int64_t C = (T + 31) / 32;
+  int64_t o = 256;
+  uint32_t* masks = reinterpret_cast<uint32_t*>(ws + o);
+  o += al256(C * E * 4);
+  int32_t* base = reinterpret_cast<int32_t*>(ws + o);
+  o += al256(C * E * 4);
+  moe::Grouping g;
+  g.offsets = offsets;
+  g.perm = perm;
+  g.n_active = reinterpret_cast<int32_t*>(ws + o);
+  o += 256;
+  g.act_expert = reinterpret_cast<int32_t*>(ws + o);
+  o += al256((int64_t)(E + 1) * 4);
+  g.act_begin = reinterpret_cast<int32_t*>(ws + o);
+  moe::launch_permute(idx, T, k, E, g, masks, base, reinterpret_cast<int*>(ws), 1,
+                      static_cast<cudaStream_t>(stream));
+  return launch_status();
+}
+
+size_t moe_layer_workspace_bytes(int32_t T, const moe_expert_blob* experts,
+                                 const moe_expert_blob* shared, const moe_route_cfg* cfg) {
+  LayerPlan p;
+  if (!experts || !cfg) return 0;
+  // sizes only: a blob without data is fine here
+  moe_expert_blob e = *experts;
+  if (!e.data) e.data = reinterpret_cast<void*>(256);
+  moe_expert_blob sh;
+  if (shared) {
+    sh = *shared;
+    if (!sh.data) sh.data = reinterpret_cast<void*>(256);
+  }
+  e.bytes = e.bytes ? e.bytes : (size_t)-1;
+  if (shared) sh.bytes = sh.bytes ? sh.bytes : (size_t)-1;
+  if (plan_layer(T, &e, shared ? &sh : nullptr, cfg, p) != MOE_OK) return 0;
+  return (size_t)p.L.total;
+}
+
+moe_status moe_layer_debug_views(int32_t T, const moe_expert_blob* experts,
+                                 const moe_expert_blob* shared, const moe_route_cfg* cfg,
+                                 moe_debug_views* out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  const size_t total = moe_layer_workspace_bytes(T, experts, shared, cfg);
+  if (total == 0) return MOE_ERR_UNSUPPORTED;
+  const int32_t Is = shared ? shared->inter : 0;
+  const Layout L = layout(T, experts->n_experts, experts->hidden, experts->inter, Is, cfg->top_k,
+                          cfg->act == MOE_ACT_G32_F16, (cfg->flags & MOE_FLAG_DEBUG) != 0);
+  out->status = L.status;
+  out->q_x = L.qx;
+  out->s_x = L.sx;
+  out->logits = L.logits;
+  out->idx = L.idx;
+  out->w = L.w;
+  out->offsets = L.offsets;
+  out->perm = L.perm;
+  out->n_active = L.n_active;
+  out->act_expert = L.act_expert;
+  out->q_h = L.qh;
+  out->s_h = L.sh;
+  out->gate = L.dbg_gate;
+  out->up = L.dbg_up;
+  out->y_pair = L.dbg_y;
+  out->total = L.total;
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
+                             const float* router_bias, const moe_expert_blob* experts,
+                             const moe_expert_blob* shared, const moe_route_cfg* cfg, float* y,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  LayerPlan p;
+  moe_status s = plan_layer(T, experts, shared, cfg, p);
+  if (s != MOE_OK) return s;
+  if (T == 0) return MOE_OK;
+  if (!x || !router_w || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(router_w, 16) || !aligned(y, 16)) return MOE_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256)) return MOE_ERR_INVALID_ARG;
+  if (ws_bytes < (size_t)p.L.total) return MOE_ERR_WORKSPACE;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const Layout& L = p.L;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  auto at = [&](int64_t off) -> void* { return off < 0 ? nullptr : ws + off; };
+  const int32_t E = experts->n_experts, H = experts->hidden, I = experts->inter, k = cfg->top_k;
+  const int ag32 = cfg->act == MOE_ACT_G32_F16;
+  int* status = static_cast<int*>(at(L.status));
+  const BlobView bv = view(experts, p.eo);
+
+  // 1. Q8_0 activations (also zeroes y and the status word)
+  moe::launch_quantize_act(x, T, H, ag32, static_cast<int8_t*>(at(L.qx)), at(L.sx), y, status, st);
+  // 2. router logits
+  float* logits = static_cast<float*>(at(L.logits));
+  moe::launch_router_logits(x, router_w, T, E, H, logits, st);
+  // 3. top-k selection, weights and batch-union grouping
+  moe::Grouping g;
+  g.offsets = static_cast<int32_t*>(at(L.offsets));
+  g.perm = static_cast<int32_t*>(at(L.perm));
+  g.n_active = static_cast<int32_t*>(at(L.n_active));
+  g.act_expert = static_cast<int32_t*>(at(L.act_expert));
+  g.act_begin = static_cast<int32_t*>(at(L.act_begin));
+  int32_t* idx = static_cast<int32_t*>(at(L.idx));
+  float* wts = static_cast<float*>(at(L.w));
+  moe::launch_topk(logits, cfg->score == MOE_SCORE_SIGMOID_NOAUX_TC ? router_bias : nullptr, T, E,
+                   k, cfg->score, cfg->renormalize != 0, cfg->routed_scaling_factor, idx, wts,
+                   T == 1 ? &g : nullptr, status, st);
+  if (T > 1)
+    moe::launch_permute(idx, T, k, E, g, static_cast<uint32_t*>(at(L.masks)),
+                        static_cast<int32_t*>(at(L.base)), status, 0, st);
+
+  // 4. gate/up + SwiGLU (+ h quantization for group-32 activations)
+  moe::ExpertArgs ra;
+  std::memset(&ra, 0, sizeof(ra));
+  ra.b = bv;
+  ra.qa = static_cast<const int8_t*>(at(L.qx));
+  ra.sa = at(L.sx);
+  ra.ag32 = ag32;
+  ra.n_active = g.n_active;
+  ra.act_expert = g.act_expert;
+  ra.act_begin = g.act_begin;
+  ra.perm = g.perm;
+  ra.wts = wts;
+  ra.T = T;
+  ra.k = k;
+  ra.max_active = (int)((int64_t)T * k < E ? (int64_t)T * k : E);
+  ra.qh = static_cast<int8_t*>(at(L.qh));
+  ra.sh = static_cast<__half*>(at(L.sh));
+  ra.hbuf = static_cast<float*>(at(L.hbuf));
+  ra.dbg_a = static_cast<float*>(at(L.dbg_gate));
+  ra.dbg_b = static_cast<float*>(at(L.dbg_up));
+  ra.y = y;
+  ra.status = status;
+  moe::launch_gateup(ra, st);
+
+  moe::ExpertArgs sa;
+  if (shared) {
+    sa = ra;
+    sa.b = view(shared, p.so);
+    sa.n_active = nullptr;
+    sa.act_expert = nullptr;
+    sa.act_begin = nullptr;
+    sa.perm = nullptr;
+    sa.max_active = 1;
+    sa.qh = static_cast<int8_t*>(at(L.qh_sh));
+    sa.sh = static_cast<__half*>(at(L.sh_sh));
+    sa.hbuf = static_cast<float*>(at(L.hbuf_sh));
+    sa.dbg_a = static_cast<float*>(at(L.dbg_gate_sh));
+    sa.dbg_b = static_cast<float*>(at(L.dbg_up_sh));
+    moe::launch_gateup(sa, st);
+  }
+  if (!ag32) {
+    moe::launch_quantize_rows_token(static_cast<const float*>(at(L.hbuf)), T * k, I,
+                                    static_cast<int8_t*>(at(L.qh)), static_cast<float*>(at(L.sh)), st);
+    if (shared)
+      moe::launch_quantize_rows_token(static_cast<const float*>(at(L.hbuf_sh)), T, p.Is,
+                                      static_cast<int8_t*>(at(L.qh_sh)),
+                                      static_cast<float*>(at(L.sh_sh)), st);
+  }
+
+  // 5. down projection + weighted combine into y
+  moe::ExpertArgs rd = ra;
+  rd.qa = static_cast<const int8_t*>(at(L.qh));
+  rd.sa = at(L.sh);
+  rd.dbg_a = static_cast<float*>(at(L.dbg_y));
+  rd.dbg_b = nullptr;
+  moe::launch_down(rd, st);
+  if (shared) {
+    moe::ExpertArgs sd = sa;
+    sd.qa = static_cast<const int8_t*>(at(L.qh_sh));
+    sd.sa = at(L.sh_sh);
+    sd.dbg_a = static_cast<float*>(at(L.dbg_y_sh));
+    sd.dbg_b = nullptr;
+    moe::launch_down(sd, st);
+  }
+  (void)H;
+  return launch_status();
+}
+
+moe_status moe_expert_group_dots(const moe_expert_blob* blob, int32_t which, int32_t n,
+                                 const int32_t* expert, const int32_t* row, const int8_t* act,
+                                 int32_t* dots, void* stream) {
+  BlobOffsets o;
+  const moe_status s = check_blob(blob, o);
+  if (s != MOE_OK) return s;
+  if ((which != 0 && which != 1) || n < 0) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (!expert || !row || !act || !dots || !aligned(act, 16)) return MOE_ERR_INVALID_ARG;
+  moe::launch_group_dots(view(blob, o), which, n, expert, row, act, dots,
+                         static_cast<cudaStream_t>(stream));
+  return launch_status();
+}
+
+moe_status moe_read_device_status(void* workspace, size_t ws_bytes, void* stream) {
+  if (!workspace || ws_bytes < 4) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  return static_cast<moe_status>(h);
+}
+
+}  // extern "C"

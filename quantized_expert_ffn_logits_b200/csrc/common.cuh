@@ -1,0 +1,152 @@
+// common.cuh -- device helpers shared by the kernels of the B200 MoE FFN layer.
+//
+// Every helper that takes part in a decision that yields an integer (a
+// quantized code, a top-k selection) is written with explicit round-to-nearest
+// intrinsics (__fmaf_rn, __fmul_rn, __fadd_rn, __fdiv_rn) so that nvcc cannot
+// contract or reorder it: these sequences are the numerical contract stated
+// in include/moe_b200.h.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+constexpr int kStatusDeviceCheck = 5;
+constexpr int kStatusTimeout = 6;
+
+// ------------------------------------------------------------------ exp & co.
+// exp(a) in fp32: Cody-Waite reduction a = n ln2 + r with ln 2 split into a
+// 24-bit head and its fp32-rounded tail, degree-7 Taylor polynomial (1/k!
+// rounded to fp32) in Horner form, then scaling by 2^n built in the exponent
+// field. The argument is clamped to [-87, 88] so 2^n stays a normal number.
+__device__ __forceinline__ float cexp(float a) {
+  a = fminf(fmaxf(a, -87.0f), 88.0f);
+  const float kf = rintf(__fmul_rn(a, 0x1.715476p+0f));   // log2(e)
+  float r = __fmaf_rn(-kf, 0x1.62e43p-1f, a);              // ln2 head
+  r = __fmaf_rn(-kf, -0x1.05c61p-29f, r);                  // ln2 tail
+  float p = 0x1.a01a02p-13f;                               // 1/7!
+  p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);                    // 1/6!
+  p = __fmaf_rn(p, r, 0x1.111112p-7f);                     // 1/5!
+  p = __fmaf_rn(p, r, 0x1.555556p-5f);                     // 1/4!
+  p = __fmaf_rn(p, r, 0x1.555556p-3f);                     // 1/3!
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  const int n = (int)kf;
+  return __fmul_rn(p, __int_as_float((n + 127) << 23));
+}
+
+__device__ __forceinline__ float csigmoid(float L) {
+  return __fdiv_rn(1.0f, __fadd_rn(1.0f, cexp(-L)));
+}
+
+// SwiGLU: h = (g / (1 + exp(-g))) * u.
+__device__ __forceinline__ float cswiglu(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, cexp(-g))), u);
+}
+
+// ---------------------------------------------------------------- quantization
+__device__ __forceinline__ float f16_round(float d) { return __half2float(__float2half_rn(d)); }
+
+// Code of v under stored scale s: round half away from zero, clamp to [-qmax, qmax].
+__device__ __forceinline__ int quant_code(float v, float s, float qmax) {
+  if (s == 0.0f) return 0;
+  float r = roundf(__fdiv_rn(v, s));
+  r = fminf(fmaxf(r, -qmax), qmax);
+  return (int)r;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ void set_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+// --------------------------------------------------------------- integer dots
+// Signed x signed 4-way byte dot.
+__device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {
+  return __dp4a((int)a, (int)b, c);
+}
+
+// Unsigned (a) x signed (b) 4-way byte dot.
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// One group of 32 int8 weights (two 16-byte pieces) against 32 int8 activations.
+__device__ __forceinline__ int group_dot_i8(const uint4& w0, const uint4& w1, const uint4& x0,
+                                            const uint4& x1) {
+  int d = dp4a_ss(w0.x, x0.x, 0);
+  d = dp4a_ss(w0.y, x0.y, d);
+  d = dp4a_ss(w0.z, x0.z, d);
+  d = dp4a_ss(w0.w, x0.w, d);
+  d = dp4a_ss(w1.x, x1.x, d);
+  d = dp4a_ss(w1.y, x1.y, d);
+  d = dp4a_ss(w1.z, x1.z, d);
+  d = dp4a_ss(w1.w, x1.w, d);
+  return d;
+}
+
+// One group of 32 packed int4 weights (one 16-byte piece, element 2j in the low
+// nibble of byte j) against activations stored de-interleaved per 8 elements:
+// xe.* hold elements {0,2,4,6} and xo.* elements {1,3,5,7} of each 8-element
+// word. Nibbles are read as unsigned n ^ 8 = q + 8, so the dot is corrected by
+// 8 * (sum of the group's activations), xsum.
+__device__ __forceinline__ int group_dot_i4(const uint4& w, const uint4& xe, const uint4& xo,
+                                            int xsum) {
+  const uint32_t m = 0x0F0F0F0Fu;
+  uint32_t v0 = w.x ^ 0x88888888u, v1 = w.y ^ 0x88888888u;
+  uint32_t v2 = w.z ^ 0x88888888u, v3 = w.w ^ 0x88888888u;
+  int d = dp4a_us(v0 & m, xe.x, 0);
+  d = dp4a_us((v0 >> 4) & m, xo.x, d);
+  d = dp4a_us(v1 & m, xe.y, d);
+  d = dp4a_us((v1 >> 4) & m, xo.y, d);
+  d = dp4a_us(v2 & m, xe.z, d);
+  d = dp4a_us((v2 >> 4) & m, xo.z, d);
+  d = dp4a_us(v3 & m, xe.w, d);
+  d = dp4a_us((v3 >> 4) & m, xo.w, d);
+  return d - 8 * xsum;
+}
+
+// 8 activation bytes x0..x7 -> (x0 x2 x4 x6), (x1 x3 x5 x7).
+__device__ __forceinline__ void deinterleave8(uint32_t lo, uint32_t hi, uint32_t& even,
+                                              uint32_t& odd) {
+  even = __byte_perm(lo, hi, 0x6420);
+  odd = __byte_perm(lo, hi, 0x7531);
+}
+
+// ------------------------------------------------------------------ layouts
+// Views of one expert blob (layout documented in include/moe_b200.h).
+struct BlobView {
+  const uint8_t* gu_w;  // R0 gate/up codes
+  const uint8_t* dn_w;  // R1 down codes
+  const uint8_t* gu_s;  // R2 gate/up scales
+  const uint8_t* dn_s;  // R3 down scales
+  int E, H, I;
+  int wbits;            // 8 or 4
+  int wg32;             // 1: fp16 group-32 scales, 0: fp32 per row
+};
+
+__host__ __device__ __forceinline__ int kbytes(int K, int wbits) { return wbits == 8 ? K : K / 2; }
+
+}  // namespace moe

@@ -1,0 +1,72 @@
+// kernels.cuh -- launch wrappers of the device kernels (host-side declarations).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+// ---- quantize.cu
+void launch_quantize_experts(const float* w_gu, const float* w_dn, const BlobView& b,
+                             uint8_t* gu_w, uint8_t* dn_w, uint8_t* gu_s, uint8_t* dn_s,
+                             cudaStream_t st);
+// y_zero (optional): output rows to zero; status (optional): status word to reset.
+void launch_quantize_act(const float* x, int T, int H, int g32, int8_t* q, void* scales,
+                         float* y_zero, int* status, cudaStream_t st);
+void launch_quantize_rows_token(const float* h, int rows, int K, int8_t* q, float* scales,
+                                cudaStream_t st);
+
+// ---- router.cu
+void launch_router_logits(const float* x, const float* wr, int T, int E, int H, float* logits,
+                          cudaStream_t st);
+
+struct Grouping {            // batch-union grouping outputs (all device pointers)
+  int32_t* offsets;          // [E+1]
+  int32_t* perm;             // [T*k]
+  int32_t* n_active;         // [1]
+  int32_t* act_expert;       // [E]
+  int32_t* act_begin;        // [E+1]
+};
+
+void launch_topk(const float* logits, const float* bias, int T, int E, int k, int score,
+                 int renorm, float rsf, int32_t* idx, float* w, const Grouping* single_token,
+                 int* status, cudaStream_t st);
+// masks/base: scratch [ceil(T/32)][E] each.
+// reset_status: clear the status word first (stand-alone use).
+void launch_permute(const int32_t* idx, int T, int k, int E, const Grouping& g, uint32_t* masks,
+                    int32_t* base, int* status, int reset_status, cudaStream_t st);
+
+// ---- expert_gemv.cu
+struct ExpertArgs {
+  BlobView b;
+  // activation rows: gate/up reads q_x rows (one per token); down reads q_h rows (one per slot)
+  const int8_t* qa;
+  const void* sa;            // fp16 [rows][K/32] or fp32 [rows]
+  int ag32;
+  // grouping: routed experts when act_expert != nullptr, else one expert (index 0) applied
+  // to slots [0, T) where slot t is token t
+  const int32_t* n_active;
+  const int32_t* act_expert;
+  const int32_t* act_begin;
+  const int32_t* perm;
+  const float* wts;          // routing weights [T*k] (down, routed)
+  int T, k;
+  int max_active;            // grid bound on active experts
+  // outputs
+  int8_t* qh;                // gate/up, g32 act: [slots][I] codes
+  __half* sh;                // gate/up, g32 act: [slots][I/32]
+  float* hbuf;               // gate/up, token act: [slots][I] fp32 h
+  float* dbg_a;              // gate/up: gate values [slots][I]; down: pair values [slots][H]
+  float* dbg_b;              // gate/up: up values
+  float* y;                  // down: [T][H] accumulated
+  int* status;
+};
+
+void launch_gateup(const ExpertArgs& a, cudaStream_t st);
+void launch_down(const ExpertArgs& a, cudaStream_t st);
+void launch_group_dots(const BlobView& b, int which, int n, const int32_t* expert,
+                       const int32_t* row, const int8_t* act, int32_t* dots, cudaStream_t st);
+
+}  // namespace moe

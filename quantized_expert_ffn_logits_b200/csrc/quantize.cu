@@ -1,0 +1,179 @@
+// quantize.cu -- expert weight and activation quantization kernels.
+//
+// Symmetric quantization with stored-scale codes (GLM-5.2 colibri page, "What's
+// implemented": "Quantization kernels: int8 / packed int4 / packed int2,
+// per-row scales, dequant-on-use"; Q8_0-style int8 activations from the same
+// section; group size 32 from the mtlm-7m-base card, "Files").
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+// One warp per weight row. Rows [0, E*2I) are gate/up rows (logical [E][2I][H]),
+// rows [E*2I, E*2I + E*H) are down rows (logical [E][H][I]). Codes and scales are
+// written straight into the blob's tiled layout.
+__global__ void __launch_bounds__(256) k_quantize_experts(const float* __restrict__ w_gu,
+                                                          const float* __restrict__ w_dn,
+                                                          BlobView b, uint8_t* gu_w, uint8_t* dn_w,
+                                                          uint8_t* gu_s, uint8_t* dn_s) {
+  const int lane = threadIdx.x & 31;
+  const int64_t n_gu = (int64_t)b.E * 2 * b.I;
+  const int64_t n_rows = n_gu + (int64_t)b.E * b.H;
+  const float qmax = b.wbits == 8 ? 127.0f : 7.0f;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t R = warp0; R < n_rows; R += nwarps) {
+    const float* src;
+    int K, rows_per_block, piece_stride;
+    uint8_t* dst;     // byte 0 of this row's piece 0 in the tiled code region
+    uint8_t* sdst;    // this row's scale slot (g32: group 0, next group at +rows_per_block)
+    if (R < n_gu) {
+      const int e = (int)(R / (2 * b.I));
+      const int lr = (int)(R % (2 * b.I));
+      const int half = lr >= b.I;
+      const int i = lr - half * b.I;
+      K = b.H;
+      rows_per_block = 256;
+      const int kb = kbytes(K, b.wbits);
+      const int r = half * 128 + (i & 127);
+      const int64_t blk = (int64_t)e * 2 * b.I + (int64_t)(i >> 7) * 256;  // first row of block
+      src = w_gu + R * (int64_t)K;
+      dst = gu_w + blk * kb + (int64_t)r * 16;
+      sdst = b.wg32 ? gu_s + (blk * (K / 32) + r) * 2 : gu_s + (blk + r) * 4;
+    } else {
+      const int64_t R2 = R - n_gu;
+      const int e = (int)(R2 / b.H);
+      const int n = (int)(R2 % b.H);
+      K = b.I;
+      rows_per_block = 128;
+      const int kb = kbytes(K, b.wbits);
+      const int r = n & 127;
+      const int64_t blk = (int64_t)e * b.H + (int64_t)(n >> 7) * 128;
+      src = w_dn + R2 * (int64_t)K;
+      dst = dn_w + blk * kb + (int64_t)r * 16;
+      sdst = b.wg32 ? dn_s + (blk * (K / 32) + r) * 2 : dn_s + (blk + r) * 4;
+    }
+    piece_stride = rows_per_block * 16;
+    const int G = K / 32;
+    float s_row = 0.0f;
+    if (!b.wg32) {
+      float amax = 0.0f;
+      for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(src[k]));
+      amax = warp_max(amax);
+      s_row = __fdiv_rn(amax, qmax);
+      if (lane == 0) *reinterpret_cast<float*>(sdst) = s_row;
+    }
+    for (int g = 0; g < G; ++g) {
+      const float v = src[32 * g + lane];
+      float s = s_row;
+      if (b.wg32) {
+        const float amax = warp_max(fabsf(v));
+        s = f16_round(__fdiv_rn(amax, qmax));
+        if (lane == 0)
+          reinterpret_cast<__half*>(sdst)[(int64_t)g * rows_per_block] = __float2half_rn(s);
+      }
+      const int q = quant_code(v, s, qmax);
+      if (b.wbits == 8) {
+        const int byte = 32 * g + lane;
+        dst[(int64_t)(byte >> 4) * piece_stride + (byte & 15)] = (uint8_t)(int8_t)q;
+      } else {
+        const int hi = __shfl_down_sync(0xffffffffu, q, 1);
+        if ((lane & 1) == 0) {
+          const int byte = 16 * g + (lane >> 1);
+          dst[(int64_t)(byte >> 4) * piece_stride + (byte & 15)] =
+              (uint8_t)((q & 15) | ((hi & 15) << 4));
+        }
+      }
+    }
+  }
+}
+
+// One CTA per token. g32: a warp per group of 32; token mode: one fp32 scale over
+// the row. Optionally zeroes the token's output row (the layer accumulates y).
+__global__ void __launch_bounds__(256) k_quantize_act(const float* __restrict__ x, int T, int H,
+                                                      int g32, int8_t* __restrict__ q,
+                                                      void* scales, float* y_zero, int* status) {
+  const int t = blockIdx.x;
+  if (t >= T) return;
+  if (status && t == 0 && threadIdx.x == 0) *status = 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const float* xr = x + (int64_t)t * H;
+  int8_t* qr = q + (int64_t)t * H;
+  if (y_zero) {
+    float4* yr = reinterpret_cast<float4*>(y_zero + (int64_t)t * H);
+    for (int k = threadIdx.x; k < H / 4; k += blockDim.x) yr[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  if (g32) {
+    __half* sr = reinterpret_cast<__half*>(scales) + (int64_t)t * (H / 32);
+    for (int g = warp; g < H / 32; g += nw) {
+      const float v = xr[32 * g + lane];
+      const float s = f16_round(__fdiv_rn(warp_max(fabsf(v)), 127.0f));
+      qr[32 * g + lane] = (int8_t)quant_code(v, s, 127.0f);
+      if (lane == 0) sr[g] = __float2half_rn(s);
+    }
+  } else {
+    __shared__ float red[32];
+    float amax = 0.0f;
+    for (int k = threadIdx.x; k < H; k += blockDim.x) amax = fmaxf(amax, fabsf(xr[k]));
+    amax = warp_max(amax);
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    if (warp == 0) {
+      float v = lane < nw ? red[lane] : 0.0f;
+      v = warp_max(v);
+      if (lane == 0) red[0] = v;
+    }
+    __syncthreads();
+    const float s = __fdiv_rn(red[0], 127.0f);
+    for (int k = threadIdx.x; k < H; k += blockDim.x) qr[k] = (int8_t)quant_code(xr[k], s, 127.0f);
+    if (threadIdx.x == 0) reinterpret_cast<float*>(scales)[t] = s;
+  }
+}
+
+// Token-mode quantization of h (one fp32 scale per (token, expert) over I).
+__global__ void __launch_bounds__(256) k_quantize_rows_token(const float* __restrict__ h, int rows,
+                                                             int K, int8_t* __restrict__ q,
+                                                             float* __restrict__ scales) {
+  const int r = blockIdx.x;
+  if (r >= rows) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const float* hr = h + (int64_t)r * K;
+  __shared__ float red[32];
+  float amax = 0.0f;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) amax = fmaxf(amax, fabsf(hr[k]));
+  amax = warp_max(amax);
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+  if (warp == 0) {
+    float v = lane < nw ? red[lane] : 0.0f;
+    v = warp_max(v);
+    if (lane == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float s = __fdiv_rn(red[0], 127.0f);
+  for (int k = threadIdx.x; k < K; k += blockDim.x) q[(int64_t)r * K + k] = (int8_t)quant_code(hr[k], s, 127.0f);
+  if (threadIdx.x == 0) scales[r] = s;
+}
+
+void launch_quantize_experts(const float* w_gu, const float* w_dn, const BlobView& b,
+                             uint8_t* gu_w, uint8_t* dn_w, uint8_t* gu_s, uint8_t* dn_s,
+                             cudaStream_t st) {
+  const int64_t rows = (int64_t)b.E * (2 * b.I + b.H);
+  int64_t blocks = (rows + 7) / 8;
+  if (blocks > 148 * 64) blocks = 148 * 64;
+  k_quantize_experts<<<(unsigned)blocks, 256, 0, st>>>(w_gu, w_dn, b, gu_w, dn_w, gu_s, dn_s);
+}
+
+void launch_quantize_act(const float* x, int T, int H, int g32, int8_t* q, void* scales,
+                         float* y_zero, int* status, cudaStream_t st) {
+  if (T <= 0) return;
+  k_quantize_act<<<T, 256, 0, st>>>(x, T, H, g32, q, scales, y_zero, status);
+}
+
+void launch_quantize_rows_token(const float* h, int rows, int K, int8_t* q, float* scales,
+                                cudaStream_t st) {
+  if (rows <= 0) return;
+  k_quantize_rows_token<<<rows, 256, 0, st>>>(h, rows, K, q, scales);
+}
+
+}  // namespace moe

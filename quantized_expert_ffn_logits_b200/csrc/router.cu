@@ -1,0 +1,351 @@
+// router.cu -- router logits, warp-level top-k selection and batch-union grouping.
+//
+// Router: "DeepSeek-V3-style sigmoid router (noaux_tc, routed_scaling_factor)"
+// (GLM-5.2 colibri page, "What's implemented") or softmax top-k ("top-8 of 64
+// experts/layer", OLMoE page, "Mixture-of-Experts"). Grouping: "Batch-union MoE:
+// in prefill (and MTP verification), each unique expert of the batch is read
+// once and applied to every position that routes to it" (GLM page).
+#include <cfloat>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace moe {
+
+// ------------------------------------------------------------------ logits
+// Small T: one CTA per (expert, block of TT tokens). Thread c owns 32-element
+// chunk c: the expert's 32 weights stay in registers, each token's chunk partial
+// is one fma chain; partials are then added in chunk order by one thread per token.
+template <int TT>
+__global__ void __launch_bounds__(256) k_router_small(const float* __restrict__ x,
+                                                      const float* __restrict__ wr, int T, int E,
+                                                      int H, float* __restrict__ logits) {
+  extern __shared__ float part[];  // [TT][C]
+  const int e = blockIdx.x;
+  const int t0 = blockIdx.y * TT;
+  const int C = H / 32;
+  const float* wrow = wr + (int64_t)e * H;
+  for (int c = threadIdx.x; c < C; c += blockDim.x) {
+    float4 w4[8];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) w4[v] = __ldg(reinterpret_cast<const float4*>(wrow + 32 * c) + v);
+    for (int tt = 0; tt < TT && t0 + tt < T; ++tt) {
+      const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)(t0 + tt) * H + 32 * c);
+      float acc = 0.0f;
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const float4 xv = __ldg(xr + v);
+        acc = __fmaf_rn(xv.x, w4[v].x, acc);
+        acc = __fmaf_rn(xv.y, w4[v].y, acc);
+        acc = __fmaf_rn(xv.z, w4[v].z, acc);
+        acc = __fmaf_rn(xv.w, w4[v].w, acc);
+      }
+      part[tt * C + c] = acc;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < TT && t0 + (int)threadIdx.x < T) {
+    const float* p = part + threadIdx.x * C;
+    float total = 0.0f;
+    for (int c = 0; c < C; ++c) total = __fadd_rn(total, p[c]);
+    logits[(int64_t)(t0 + threadIdx.x) * E + e] = total;
+  }
+}
+
+// Large T: 64x64 output tile per CTA, each thread a 4x4 register tile. The K loop
+// walks the 32-element chunks in order; within a chunk every output runs its own
+// fma chain from +0 and is then added to the output's running total.
+__global__ void __launch_bounds__(256) k_router_tiled(const float* __restrict__ x,
+                                                      const float* __restrict__ wr, int T, int E,
+                                                      int H, float* __restrict__ logits) {
+  __shared__ __align__(16) float xs[32][68];
+  __shared__ __align__(16) float ws[32][68];
+  const int tb = blockIdx.y * 64, eb = blockIdx.x * 64;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  float total[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) total[i][j] = 0.0f;
+  for (int c = 0; c < H / 32; ++c) {
+    for (int l = threadIdx.x; l < 64 * 32; l += 256) {
+      const int rr = l >> 5, kk = l & 31;
+      const int t = tb + rr, e = eb + rr;
+      xs[kk][rr] = t < T ? x[(int64_t)t * H + 32 * c + kk] : 0.0f;
+      ws[kk][rr] = e < E ? wr[(int64_t)e * H + 32 * c + kk] : 0.0f;
+    }
+    __syncthreads();
+    float part[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[i][j] = 0.0f;
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) part[i][j] = __fmaf_rn(av[i], bv[j], part[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) total[i][j] = __fadd_rn(total[i][j], part[i][j]);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = tb + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = eb + tx * 4 + j;
+      if (e < E) logits[(int64_t)t * E + e] = total[i][j];
+    }
+  }
+}
+
+void launch_router_logits(const float* x, const float* wr, int T, int E, int H, float* logits,
+                          cudaStream_t st) {
+  if (T <= 0) return;
+  if (T <= 32) {
+    constexpr int TT = 8;
+    const int C = H / 32;
+    dim3 grid(E, (T + TT - 1) / TT);
+    const int threads = C >= 256 ? 256 : ((C + 31) / 32) * 32;
+    k_router_small<TT><<<grid, threads, TT * C * sizeof(float), st>>>(x, wr, T, E, H, logits);
+  } else {
+    dim3 grid((E + 63) / 64, (T + 63) / 64);
+    k_router_tiled<<<grid, 256, 0, st>>>(x, wr, T, E, H, logits);
+  }
+}
+
+// ------------------------------------------------------------------- top-k
+// One warp per token; lane l holds the keys of experts l, l+32, ... (NE per lane).
+// k rounds of a warp arg-max (larger key wins, equal keys go to the lower expert).
+template <int NE>
+__global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits,
+                                              const float* __restrict__ bias, int T, int E, int k,
+                                              int score, int renorm, float rsf,
+                                              int32_t* __restrict__ idx, float* __restrict__ w,
+                                              Grouping g1, int single, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const float* Lt = logits + (int64_t)t * E;
+  float key[NE], lg[NE];
+#pragma unroll
+  for (int m = 0; m < NE; ++m) {
+    const int e = lane + 32 * m;
+    lg[m] = e < E ? Lt[e] : 0.0f;
+    if (e >= E) key[m] = -FLT_MAX;
+    else if (score == 0) key[m] = lg[m];
+    else key[m] = __fadd_rn(csigmoid(lg[m]), bias ? bias[e] : 0.0f);
+  }
+  uint32_t taken = 0;
+  int my_e = 0;
+  for (int j = 0; j < k; ++j) {
+    float bk = -FLT_MAX;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int m = 0; m < NE; ++m) {
+      const int e = lane + 32 * m;
+      if (e < E && !((taken >> m) & 1u) && (key[m] > bk || be == 0x7fffffff)) {
+        bk = key[m];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ok > bk || (ok == bk && oe < be)) {
+        bk = ok;
+        be = oe;
+      }
+    }
+    if (be < E && (be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == j) my_e = be;
+  }
+  const bool sel = lane < k;
+  if (sel && (my_e < 0 || my_e >= E)) set_status(status, kStatusDeviceCheck);
+  const float myL = sel ? Lt[min(max(my_e, 0), E - 1)] : 0.0f;
+  float wv;
+  if (score == 0) {
+    const float Lmax = __shfl_sync(0xffffffffu, myL, 0);
+    const float ex = sel ? cexp(myL - Lmax) : 0.0f;
+    float den;
+    if (renorm) {
+      den = warp_sum(ex);
+    } else {
+      float s = 0.0f;
+#pragma unroll
+      for (int m = 0; m < NE; ++m)
+        if (lane + 32 * m < E) s += cexp(lg[m] - Lmax);
+      den = warp_sum(s);
+    }
+    wv = ex / den * rsf;
+  } else {
+    const float s = sel ? csigmoid(myL) : 0.0f;
+    const float den = renorm ? warp_sum(s) : 1.0f;
+    wv = s / den * rsf;
+  }
+  if (sel) {
+    idx[(int64_t)t * k + lane] = my_e;
+    w[(int64_t)t * k + lane] = wv;
+  }
+  if (single) {
+    // One token: the grouping is the k selected experts in ascending order.
+    int rank = 0;
+    for (int i = 0; i < k; ++i) rank += __shfl_sync(0xffffffffu, my_e, i) < my_e;
+    if (sel) {
+      g1.act_expert[rank] = my_e;
+      g1.act_begin[rank] = rank;
+      g1.perm[rank] = lane;
+    }
+    if (lane == 0) {
+      g1.act_begin[k] = k;
+      *g1.n_active = k;
+      g1.offsets[E] = k;
+    }
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      int cnt = 0;
+      for (int i = 0; i < k; ++i) cnt += __shfl_sync(0xffffffffu, my_e, i) < e;
+      if (e < E) g1.offsets[e] = cnt;
+    }
+  }
+}
+
+void launch_topk(const float* logits, const float* bias, int T, int E, int k, int score,
+                 int renorm, float rsf, int32_t* idx, float* w, const Grouping* single_token,
+                 int* status, cudaStream_t st) {
+  if (T <= 0) return;
+  const int blocks = (T + 7) / 8;
+  Grouping g{};
+  if (single_token) g = *single_token;
+  const int single = single_token != nullptr;
+#define MOE_TOPK_CASE(N)                                                                    \
+  k_topk<N><<<blocks, 256, 0, st>>>(logits, bias, T, E, k, score, renorm, rsf, idx, w, g, \
+                                    single, status)
+  if (E <= 32) MOE_TOPK_CASE(1);
+  else if (E <= 64) MOE_TOPK_CASE(2);
+  else if (E <= 128) MOE_TOPK_CASE(4);
+  else if (E <= 256) MOE_TOPK_CASE(8);
+  else if (E <= 512) MOE_TOPK_CASE(16);
+  else MOE_TOPK_CASE(32);
+#undef MOE_TOPK_CASE
+}
+
+// ----------------------------------------------------------------- grouping
+// Stable counting sort of the T*k (token, slot) pairs by expert, one CTA.
+//   A: per 32-token chunk c, masks[c][e] = bit set of the chunk's tokens routed to e;
+//   B: per expert, base[c][e] = pairs of e in chunks before c;
+//   C: exclusive scan over experts -> offsets, list of distinct experts;
+//   D: pos = offsets[e] + base[c][e] + (tokens of the chunk before this one routed to e).
+__global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ idx, int T, int k,
+                                                  int E, Grouping g, uint32_t* masks,
+                                                  int32_t* base, int* status, int reset_status) {
+  __shared__ int32_t off_s[1024];
+  __shared__ int32_t wsum[32], fsum[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (reset_status && tid == 0 && status) *status = 0;
+  __syncthreads();
+  const int C = (T + 31) / 32;
+  for (int c = warp; c < C; c += 32) {
+    uint32_t* mrow = masks + (int64_t)c * E;
+    for (int e = lane; e < E; e += 32) mrow[e] = 0u;
+    __syncwarp();
+    const int t = 32 * c + lane;
+    if (t < T) {
+      for (int j = 0; j < k; ++j) {
+        const int e = idx[(int64_t)t * k + j];
+        if (e < 0 || e >= E) set_status(status, kStatusDeviceCheck);
+        else atomicOr(&mrow[e], 1u << lane);
+      }
+    }
+  }
+  __syncthreads();
+  int v = 0;
+  if (tid < E) {
+    int run = 0;
+    for (int c = 0; c < C; ++c) {
+      const uint32_t m = __ldcg(masks + (int64_t)c * E + tid);
+      base[(int64_t)c * E + tid] = run;
+      run += __popc(m);
+    }
+    v = run;
+  }
+  const int f = (tid < E && v > 0) ? 1 : 0;
+  int incl = v, inclf = f;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int a = __shfl_up_sync(0xffffffffu, incl, o);
+    const int b = __shfl_up_sync(0xffffffffu, inclf, o);
+    if (lane >= o) {
+      incl += a;
+      inclf += b;
+    }
+  }
+  if (lane == 31) {
+    wsum[warp] = incl;
+    fsum[warp] = inclf;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int a = wsum[lane], b = fsum[lane];
+    int ia = a, ib = b;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, ia, o);
+      const int y = __shfl_up_sync(0xffffffffu, ib, o);
+      if (lane >= o) {
+        ia += x;
+        ib += y;
+      }
+    }
+    wsum[lane] = ia - a;
+    fsum[lane] = ib - b;
+  }
+  __syncthreads();
+  incl += wsum[warp];
+  inclf += fsum[warp];
+  if (tid < E) {
+    const int excl = incl - v;
+    off_s[tid] = excl;
+    g.offsets[tid] = excl;
+    if (f) {
+      g.act_expert[inclf - 1] = tid;
+      g.act_begin[inclf - 1] = excl;
+    }
+    if (tid == E - 1) {
+      g.offsets[E] = incl;
+      *g.n_active = inclf;
+      g.act_begin[inclf] = incl;
+    }
+  }
+  __syncthreads();
+  for (int c = warp; c < C; c += 32) {
+    const int t = 32 * c + lane;
+    if (t >= T) continue;
+    for (int j = 0; j < k; ++j) {
+      const int e = idx[(int64_t)t * k + j];
+      if (e < 0 || e >= E) continue;
+      const uint32_t m = __ldcg(masks + (int64_t)c * E + e);
+      const int pos = off_s[e] + __ldcg(base + (int64_t)c * E + e) + __popc(m & ((1u << lane) - 1u));
+      g.perm[pos] = t * k + j;
+    }
+  }
+}
+
+void launch_permute(const int32_t* idx, int T, int k, int E, const Grouping& g, uint32_t* masks,
+                    int32_t* base, int* status, int reset_status, cudaStream_t st) {
+  if (T <= 0) return;
+  k_permute<<<1, 1024, 0, st>>>(idx, T, k, E, g, masks, base, status, reset_status);
+}
+
+}  // namespace moe

@@ -1,0 +1,115 @@
+"""Shared helpers of the tests: build one workload on the GPU (through the C ABI) and on
+the CPU oracle from the same seeded inputs, and compare."""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle as O
+import synth as S
+
+REL_L2 = 1e-5      # layer output: relative L2 error bound
+MAX_ABS = 1e-4     # layer output: max |error| relative to max |y_ref|
+
+
+def wbits(cfg):
+    return 8 if cfg.wtype == "int8" else 4
+
+
+def wg32(cfg):
+    return cfg.wscale == "g32_f16"
+
+
+def ag32(cfg):
+    return cfg.act == "g32_f16"
+
+
+def route_cfg(cfg, flags=0):
+    import quantized_expert_ffn_logits_b200 as M
+    return M.RouteCfg(score=cfg.score, top_k=cfg.top_k, renormalize=cfg.renormalize,
+                      routed_scaling_factor=cfg.rsf, act=cfg.act, flags=flags)
+
+
+def gpu_layer(case: S.Case, device="cuda"):
+    """Expert blobs, router weight, bias and x of a case, on the device."""
+    import torch
+    import quantized_expert_ffn_logits_b200 as M
+    c = case.cfg
+    gu = torch.empty((c.E, 2 * c.I, c.H), dtype=torch.float32, device=device)
+    dn = torch.empty((c.E, c.H, c.I), dtype=torch.float32, device=device)
+    case.gate_up_gpu(gu)
+    case.down_gpu(dn)
+    blob = M.ExpertBlob.quantize(gu, dn, c.wtype, c.wscale)
+    del gu, dn
+    shared = None
+    if c.shared_I:
+        sgu = torch.empty((1, 2 * c.shared_I, c.H), dtype=torch.float32, device=device)
+        sdn = torch.empty((1, c.H, c.shared_I), dtype=torch.float32, device=device)
+        case.shared_gate_up_gpu(sgu)
+        case.shared_down_gpu(sdn)
+        shared = M.ExpertBlob.quantize(sgu, sdn, c.wtype, c.wscale)
+        del sgu, sdn
+    wr = torch.from_numpy(case.router_w()).to(device)
+    b = case.bias()
+    bias = torch.from_numpy(b).to(device) if b is not None else None
+    x = torch.from_numpy(case.x()).to(device)
+    return dict(blob=blob, shared=shared, wr=wr, bias=bias, x=x)
+
+
+def oracle_experts(case: S.Case, experts=None):
+    """Oracle-quantized routed experts (all, or the listed ones in that order) and shared."""
+    c = case.cfg
+    ids = range(c.E) if experts is None else experts
+    ex = O.QExperts.quantize(np.stack([case.gate_up(e) for e in ids]),
+                             np.stack([case.down(e) for e in ids]), wbits(c), wg32(c))
+    sh = None
+    if c.shared_I:
+        sh = O.QExperts.quantize(case.shared_gate_up()[None], case.shared_down()[None], wbits(c), wg32(c))
+    return ex, sh
+
+
+def oracle_layer(case: S.Case, union=False):
+    c = case.cfg
+    ex, sh = oracle_experts(case)
+    return O.layer_forward(case.x(), case.router_w(), case.bias(), ex, sh, c.score, c.top_k,
+                           c.renormalize, c.rsf, ag32(c), union=union)
+
+
+def oracle_tokens(case: S.Case, tokens):
+    """Per-token oracle for selected tokens only, regenerating just the experts they use.
+    Returns dict(y [n][H], idx, w, ye {(t, j): fp64 [H]}, qh/sh/gate/up per pair)."""
+    c = case.cfg
+    x = case.x()
+    L = O.router_logits(x[tokens], case.router_w())
+    idx, w = O.route(L, case.bias(), c.score, c.top_k, c.renormalize, c.rsf)
+    qx, sx = O.quantize_act(x[tokens], ag32(c))
+    need = sorted(set(int(e) for e in idx.reshape(-1)))
+    y = np.zeros((len(tokens), c.H))
+    pairs = {}
+    for e in need:
+        ex = O.QExperts.quantize(case.gate_up(e)[None], case.down(e)[None], wbits(c), wg32(c))
+        for n, t in enumerate(tokens):
+            for j in range(c.top_k):
+                if idx[n, j] == e:
+                    r = O.expert_ffn(ex, 0, qx[n], sx[n], ag32(c))
+                    pairs[(n, j)] = r
+                    y[n] += w[n, j] * r["ye"]
+        del ex
+    if c.shared_I:
+        sh = O.QExperts.quantize(case.shared_gate_up()[None], case.shared_down()[None], wbits(c), wg32(c))
+        for n in range(len(tokens)):
+            y[n] += O.expert_ffn(sh, 0, qx[n], sx[n], ag32(c))["ye"]
+    return dict(y=y, idx=idx, w=w, logits=L, qx=qx, sx=sx, pairs=pairs)
+
+
+def assert_close_y(got, ref, what="y"):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    den = np.linalg.norm(ref)
+    rel = np.linalg.norm(got - ref) / den if den > 0 else np.linalg.norm(got)
+    mabs = np.max(np.abs(got - ref)) if got.size else 0.0
+    scale = np.max(np.abs(ref)) if ref.size else 1.0
+    assert rel <= REL_L2, f"{what}: rel-L2 {rel:.3e} > {REL_L2}"
+    assert mabs <= MAX_ABS * scale, f"{what}: max-abs {mabs:.3e} > {MAX_ABS} * {scale:.3e}"
+    return rel, mabs
