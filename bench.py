@@ -1,0 +1,549 @@
+#!/usr/bin/env python
+"""Throughput of the B200 quantized MoE FFN layer.
+
+One step = one full layer forward (router logits, top-k, Q8_0 activation
+quantization, batch-union grouping, gate/up + SwiGLU, down + weighted combine)
+on a fresh batch of synthetic tokens. Consecutive steps rotate over several
+layer replicas (distinct expert weights), so the expert bytes a step touches are
+never left in L2 by the previous steps. The timed region replays a CUDA graph of
+the steps (launch overhead removed), bracketed by a barrier and a device
+synchronize on both sides; multi-GPU runs are weak-scaled (each rank its own
+tokens and replicas, no data-path collective) and report the max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload olmoe_int8:1]
+  python bench.py --impl reference ...   (the CPU oracle as the reference arm)
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth as S  # noqa: E402
+
+METRIC = "MoE-layer tok/s (decode b=1, prefill 4k); HBM GB/s and int8 TC % of peak"
+DEFAULT_WORKLOAD = "olmoe_int8:1"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------- helpers
+def parse_workload(spec: str):
+    name, _, t = spec.partition(":")
+    cfg = S.CONFIGS[name]
+    T = int(t) if t else cfg.tokens[0]
+    return cfg, T
+
+
+def workload_desc(cfg, T):
+    return (f"{cfg.name} T={T}: H{cfg.H} E{cfg.E} I{cfg.I} top-{cfg.top_k} {cfg.score}"
+            f"{' renorm' if cfg.renormalize else ''}{f' rsf {cfg.rsf}' if cfg.rsf != 1 else ''}, "
+            f"{cfg.wtype} {cfg.wscale} experts, {cfg.act} activations"
+            f"{f', shared I{cfg.shared_I}' if cfg.shared_I else ''}")
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def blob_row_bytes(cfg, K, I_rows):
+    kb = K if cfg.wtype == "int8" else K // 2
+    sb = (K // 32) * 2 if cfg.wscale == "g32_f16" else 4
+    return I_rows * (kb + sb)
+
+
+def gateup_bytes(cfg, T, n_active):
+    """Algorithmic bytes of the gate/up stage: each unique expert's gate/up codes+scales once,
+    the shared expert's, q_x read and q_h (+ scales) written."""
+    P = T * cfg.top_k
+    b = n_active * blob_row_bytes(cfg, cfg.H, 2 * cfg.I)
+    if cfg.shared_I:
+        b += blob_row_bytes(cfg, cfg.H, 2 * cfg.shared_I)
+    b += T * cfg.H + (T * (cfg.H // 32) * 2 if cfg.act == "g32_f16" else T * 4)
+    b += P * cfg.I + (P * (cfg.I // 32) * 2 if cfg.act == "g32_f16" else P * 4)
+    if cfg.shared_I:
+        b += T * cfg.shared_I
+    return b
+
+
+def layer_bytes(cfg, T, n_active):
+    """Algorithmic bytes of one layer forward: unique experts' blobs (gate/up and down), the
+    shared expert, the router weight, x in and y out (fp32)."""
+    b = n_active * (blob_row_bytes(cfg, cfg.H, 2 * cfg.I) + blob_row_bytes(cfg, cfg.I, cfg.H))
+    if cfg.shared_I:
+        b += blob_row_bytes(cfg, cfg.H, 2 * cfg.shared_I) + blob_row_bytes(cfg, cfg.shared_I, cfg.H)
+    b += cfg.E * cfg.H * 4 + 2 * T * cfg.H * 4
+    return b
+
+
+def layer_int_ops(cfg, T):
+    return 2 * (T * cfg.top_k * 3 * cfg.H * cfg.I + T * 3 * cfg.H * cfg.shared_I)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 20 ms while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.samples = []
+        self.proc = None
+        self.window = None
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20"]
+        if gpu_id:
+            cmd += ["-i", gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.perf_counter(), line.strip()))
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "nvidia-smi unavailable"}
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        t0, t1 = self.window if self.window else (0, float("inf"))
+        inside = [s for ts, s in self.samples if t0 <= ts <= t1]
+        note = "samples inside the timed region"
+        if not inside and self.samples:
+            # region shorter than one sampling period: keep the samples bracketing it
+            near = sorted(self.samples, key=lambda p: min(abs(p[0] - t0), abs(p[0] - t1)))[:2]
+            inside = [s for _, s in near]
+            note = "timed region shorter than the 20 ms sampling period: nearest samples"
+        sm, mx, reasons = [], [], set()
+        for s in inside:
+            f = [v.strip() for v in s.split(",")]
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except (ValueError, IndexError):
+                continue
+            for name, v in zip(self.REASONS, f[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm), "note": note}
+
+
+# --------------------------------------------------------------------- oracle
+def oracle_sampler(cfg, T, seed_base=7_000_000):
+    """Prepare the oracle for timing on host cores: experts of a token sample, pre-quantized.
+    Returns (run_units(n_units) -> tokens processed, unit description, cores)."""
+    import oracle as O
+    from concurrent.futures import ThreadPoolExecutor
+
+    cores = os.cpu_count() or 1
+    wbits = 8 if cfg.wtype == "int8" else 4
+    wg32 = cfg.wscale == "g32_f16"
+    ag32 = cfg.act == "g32_f16"
+    n_tok = 64
+    case = S.Case.make(cfg, n_tok, seed=seed_base + T)
+    x = case.x()
+    Wr, bias = case.router_w(), case.bias()
+    L = O.router_logits(x, Wr)
+    idx, _ = O.route(L, bias, cfg.score, cfg.top_k, cfg.renormalize, cfg.rsf)
+    experts = {}
+    shared = None
+    if cfg.shared_I:
+        shared = O.QExperts.quantize(case.shared_gate_up()[None], case.shared_down()[None], wbits, wg32)
+    per_tok = cfg.top_k + (1 if shared is not None else 0)
+    pool = ThreadPoolExecutor(cores)
+
+    def ensure(e):
+        if e not in experts:
+            experts[e] = O.QExperts.quantize(case.gate_up(e)[None], case.down(e)[None], wbits, wg32)
+        return experts[e]
+
+    # pre-quantize the experts of the first tokens (input preparation, not timed)
+    for e in sorted(set(int(v) for v in idx[:16].reshape(-1))):
+        ensure(e)
+    cursor = [0]
+
+    def run_units(n_units):
+        """Oracle work for n_units (token, expert) units starting at the cursor: per token the
+        router logits, top-k, activation quantization, its expert FFNs and the combine."""
+        units = []
+        while len(units) < n_units:
+            t = (cursor[0] // per_tok) % 16
+            u = cursor[0] % per_tok
+            units.append((t, u))
+            cursor[0] += 1
+        toks = sorted(set(t for t, _ in units))
+        Lt = O.router_logits(x[toks], Wr)
+        it, wt = O.route(Lt, bias, cfg.score, cfg.top_k, cfg.renormalize, cfg.rsf)
+        qx, sx = O.quantize_act(x[toks], ag32)
+        pos = {t: i for i, t in enumerate(toks)}
+
+        def one(tu):
+            t, u = tu
+            i = pos[t]
+            if u < cfg.top_k:
+                r = O.expert_ffn(experts[int(it[i, u])], 0, qx[i], sx[i], ag32)
+                return i, wt[i, u] * r["ye"]
+            r = O.expert_ffn(shared, 0, qx[i], sx[i], ag32)
+            return i, r["ye"]
+
+        y = np.zeros((len(toks), cfg.H))
+        for i, v in pool.map(one, units):
+            y[i] += v
+        return n_units / per_tok
+
+    desc = (f"(token, expert) units of {cfg.name}: per token its router logits, top-{cfg.top_k}, "
+            f"Q8_0 quantization, {per_tok} expert FFNs (fp64 down) and the combine; "
+            f"16 tokens cycled, {cores} threads over units")
+    return run_units, desc, cores
+
+
+def time_oracle(cfg, T, budget_s=12.0):
+    run_units, desc, cores = oracle_sampler(cfg, T)
+    per_tok = cfg.top_k + (1 if cfg.shared_I else 0)
+    t0 = time.perf_counter()
+    run_units(per_tok)
+    t1 = time.perf_counter() - t0
+    n = max(per_tok, int(budget_s / max(t1, 1e-3)) * per_tok)
+    n = min(n, 64 * per_tok)
+    t0 = time.perf_counter()
+    toks = run_units(n)
+    el = time.perf_counter() - t0
+    return {"value": toks / el, "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "sample": f"{toks:g} tokens = {n} {desc}; {el:.1f} s"}
+
+
+def reference_arm(args, cfg, T):
+    """The oracle as the reference implementation, on host cores: K timed steps, each a
+    bounded sample of the workload (whole (token, expert) units), so the run stays short."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    run_units, desc, cores = oracle_sampler(cfg, T)
+    per_tok = cfg.top_k + (1 if cfg.shared_I else 0)
+    t0 = time.perf_counter()
+    run_units(1)
+    t_unit = max(time.perf_counter() - t0, 1e-4)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    units = int(max(1, min(per_tok * T, budget / t_unit)))
+    for _ in range(args.warmup):
+        run_units(units)
+    t0 = time.perf_counter()
+    toks = 0.0
+    for _ in range(args.steps):
+        toks += run_units(units)
+    el = time.perf_counter() - t0
+    value = toks / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tok/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg, T), "T": T,
+                   "step": f"{units} (token, expert) units per step = {units / per_tok:g} tokens"},
+        "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{args.steps} steps of {units} {desc}"},
+        "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- GPU arm
+def gpu_arm(args, cfg, T):
+    import torch
+    import torch.distributed as dist
+    import quantized_expert_ffn_logits_b200 as M
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    R = args.replicas
+    rcfg = M.RouteCfg(score=cfg.score, top_k=cfg.top_k, renormalize=cfg.renormalize,
+                      routed_scaling_factor=cfg.rsf, act=cfg.act)
+    layers, n_active_of = [], []
+    for r in range(R):
+        case = S.Case.make(cfg, T, replica=1000 * rank + r)
+        gu = torch.empty((cfg.E, 2 * cfg.I, cfg.H), dtype=torch.float32, device=dev)
+        case.gate_up_gpu(gu)
+        dn = torch.empty((cfg.E, cfg.H, cfg.I), dtype=torch.float32, device=dev)
+        case.down_gpu(dn)
+        blob = M.ExpertBlob.quantize(gu, dn, cfg.wtype, cfg.wscale)
+        del gu, dn
+        shared = None
+        if cfg.shared_I:
+            sgu = torch.empty((1, 2 * cfg.shared_I, cfg.H), dtype=torch.float32, device=dev)
+            sdn = torch.empty((1, cfg.H, cfg.shared_I), dtype=torch.float32, device=dev)
+            case.shared_gate_up_gpu(sgu)
+            case.shared_down_gpu(sdn)
+            shared = M.ExpertBlob.quantize(sgu, sdn, cfg.wtype, cfg.wscale)
+            del sgu, sdn
+        wr = torch.from_numpy(case.router_w()).to(dev)
+        b = case.bias()
+        bias = torch.from_numpy(b).to(dev) if b is not None else None
+        layers.append(M.Layer(T, blob, shared, rcfg, wr, bias))
+    torch.cuda.synchronize()
+    # distinct token batches, resident in HBM before timing
+    G = max(1, min(args.steps, args.period))
+    xs = []
+    for s in range(G):
+        xc = S.Case.make(cfg, T, seed=90_000_000 + 1_000_000 * rank + s)
+        xs.append(torch.from_numpy(xc.x()).to(dev))
+    y = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
+    # distinct experts per step (for the algorithmic byte counts)
+    for s in range(G):
+        lay = layers[s % R]
+        idx, _ = M.moe_route_topk(M.moe_router_logits(xs[s], lay.router_w), lay.router_bias, rcfg)
+        n_active_of.append(int(torch.unique(idx).numel()))
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    # warm-up (eager)
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            layers[s % R](xs[s % G], y, stream)
+    stream.synchronize()
+
+    # one graph period of G steps with stage events around every step (torch events used
+    # as plain cudaEvent_t handles; recorded once eagerly so the handles exist)
+    nst = len(M.MOE_STAGES)
+    evs = []
+    with torch.cuda.stream(stream):
+        for s in range(G):
+            e = M.moe_stage_events()
+            pair = []
+            for i in range(nst):
+                b_ev = torch.cuda.Event(enable_timing=True, external=True)
+                e_ev = torch.cuda.Event(enable_timing=True, external=True)
+                b_ev.record(stream)
+                e_ev.record(stream)
+                e.begin[i] = b_ev.cuda_event
+                e.end[i] = e_ev.cuda_event
+                pair.append((b_ev, e_ev))
+            evs.append((e, pair))
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for s in range(G):
+            layers[s % R](xs[s], y, stream, events=evs[s][0])
+    rem = args.steps % G
+    graph_rem = None
+    if rem:
+        graph_rem = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_rem, stream=stream):
+            for s in range(rem):
+                layers[s % R](xs[s], y, stream)
+    # one untimed replay
+    with torch.cuda.stream(stream):
+        graph.replay()
+    stream.synchronize()
+
+    # ------------------------------------------------------------ timed region
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(gpu_id)
+    time.sleep(0.1)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")
+    w0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(args.steps // G):
+            graph.replay()
+        if graph_rem is not None:
+            graph_rem.replay()
+        end.record(stream)
+    stream.synchronize()
+    w1 = time.perf_counter()
+    torch.cuda.nvtx.range_pop()
+    barrier()
+    clocks.mark(w0, w1)
+    clk = clocks.stop()
+    ms = start.elapsed_time(end)
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # per-stage device times of the last graph period (inside the timed region)
+    stage_ms = {n: [] for n in M.MOE_STAGES}
+    if args.steps >= G:
+        for s in range(G):
+            for i, n in enumerate(M.MOE_STAGES):
+                b_ev, e_ev = evs[s][1][i]
+                stage_ms[n].append(b_ev.elapsed_time(e_ev))
+    stage_us = {n: (1e3 * statistics.mean(v) if v else None) for n, v in stage_ms.items()}
+
+    value = world * T * args.steps / (ms_max / 1e3)
+    peaks, peak_src = load_peaks()
+    n_act = float(np.mean(n_active_of))
+    # dominant kernel: gate/up (weight streaming, HBM-bound)
+    gu_us = stage_us["gate_up"]
+    gu_bytes = float(np.mean([gateup_bytes(cfg, T, a) for a in n_active_of]))
+    roof = None
+    if gu_us:
+        ach = gu_bytes / (gu_us * 1e-6) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic_from_profiles(cfg, T),
+                "kernel": "k_gateup (gate/up + SwiGLU + h quantization)",
+                "bytes_per_launch": int(gu_bytes), "us_per_launch": round(gu_us, 3),
+                "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6.65 TB/s"}
+    lb = float(np.mean([layer_bytes(cfg, T, a) for a in n_active_of]))
+    step_s = ms_max / 1e3 / args.steps
+    layer = {"bytes_per_step": int(lb), "gbs": round(lb / step_s / 1e9, 1),
+             "frac_hbm": round(lb / step_s / 1e9 / peaks["hbm_gbs"], 4),
+             "int8_tops": round(layer_int_ops(cfg, T) / step_s / 1e12, 2),
+             "distinct_experts_per_step": round(n_act, 2),
+             "stage_us": {k: (round(v, 3) if v is not None else None) for k, v in stage_us.items()}}
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if not args.no_e2e:
+        ne = min(args.steps, args.e2e_steps)
+        xh = [torch.from_numpy(S.Case.make(cfg, T, seed=95_000_000 + s).x()).pin_memory() for s in range(min(ne, 64))]
+        yh = torch.empty((T, cfg.H), dtype=torch.float32).pin_memory()
+        xd = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
+        with torch.cuda.stream(stream):
+            for s in range(3):
+                xd.copy_(xh[s % len(xh)], non_blocking=True)
+                layers[s % R](xd, y, stream)
+                yh.copy_(y, non_blocking=True)
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for s in range(ne):
+                xd.copy_(xh[s % len(xh)], non_blocking=True)
+                layers[s % R](xd, y, stream)
+                yh.copy_(y, non_blocking=True)
+            e1.record(stream)
+        stream.synchronize()
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": world * T * ne / (float(te.item()) / 1e3), "unit": "tok/s",
+               "h2d_bytes_per_step": T * cfg.H * 4, "d2h_bytes_per_step": T * cfg.H * 4,
+               "steps": ne, "path": "Layer.__call__ (moe_layer_forward) eager, pinned host x in / y out"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle(cfg, T)
+
+    launches = layers[0].kernels * args.steps
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic",
+        "config": {"workload": workload_desc(cfg, T), "T": T, "replicas": R,
+                   "l2": f"inputs larger than L2: {R} layer replicas rotate "
+                         f"({R * layers[0].experts.nbytes / 1e9:.2f} GB of expert blobs)",
+                   "graph": f"CUDA graph of {G} steps replayed", "accumulate": "int32 dots, fp32 scales",
+                   "parallelism": f"dp{world} (weak: independent tokens per GPU)"},
+        "roofline": roof,
+        "layer": layer,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    del graph, graph_rem
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def traffic_from_profiles(cfg, T):
+    """DRAM bytes per launch of the gate/up kernel from the committed ncu summary, if it was
+    taken on this workload with the current kernel source; else None."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "k_gateup_traffic.json")
+    src = os.path.join(ROOT, "quantized_expert_ffn_logits_b200", "csrc", "expert_gemv.cu")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if d.get("source_sha256_16") != h or d.get("workload") != f"{cfg.name}:{T}":
+            return None
+        return d.get("dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    help="config[:T], config one of " + ", ".join(S.CONFIG_ORDER))
+    ap.add_argument("--replicas", type=int, default=8, help="layer replicas rotated per step")
+    ap.add_argument("--period", type=int, default=256, help="steps per captured graph")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    cfg, T = parse_workload(args.workload)
+    if args.impl == "reference":
+        return reference_arm(args, cfg, T)
+    return gpu_arm(args, cfg, T)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -197,6 +197,40 @@ MOE_API moe_status moe_layer_forward(const float* x, int32_t T, const float* rou
                              const moe_expert_blob* shared, const moe_route_cfg* cfg, float* y,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* Stages of moe_layer_forward, in launch order. */
+enum {
+  MOE_STAGE_QUANT_X = 0,   /* activation quantization (also zeroes y) */
+  MOE_STAGE_ROUTER = 1,    /* router logits */
+  MOE_STAGE_TOPK = 2,      /* top-k selection and weights (grouping too when T = 1) */
+  MOE_STAGE_GROUP = 3,     /* batch-union grouping (T > 1) */
+  MOE_STAGE_GATE_UP = 4,   /* gate/up + SwiGLU (+ h quantization for group-32 activations) */
+  MOE_STAGE_QUANT_H = 5,   /* h quantization (per-token activation scales only) */
+  MOE_STAGE_DOWN = 6,      /* down projection + weighted combine */
+  MOE_STAGE_COUNT = 7
+};
+
+/* Caller-created CUDA events (cudaEvent_t, may be NULL) recorded on `stream` just before
+ * the first and just after the last kernel of each stage; a stage that launches nothing
+ * records both events back to back. Inside stream capture they are recorded as external
+ * event nodes, so cudaEventElapsedTime works on them after the graph runs. */
+typedef struct {
+  void* begin[MOE_STAGE_COUNT];
+  void* end[MOE_STAGE_COUNT];
+} moe_stage_events;
+
+/* moe_layer_forward with per-stage event records (profiling). */
+MOE_API moe_status moe_layer_forward_timed(const float* x, int32_t T, const float* router_w,
+                                           const float* router_bias,
+                                           const moe_expert_blob* experts,
+                                           const moe_expert_blob* shared,
+                                           const moe_route_cfg* cfg, float* y, void* workspace,
+                                           size_t ws_bytes, void* stream,
+                                           const moe_stage_events* events);
+
+/* Number of kernels one moe_layer_forward call with these arguments launches. */
+MOE_API int32_t moe_layer_kernel_count(int32_t T, const moe_expert_blob* experts,
+                                       const moe_expert_blob* shared, const moe_route_cfg* cfg);
+
 /* Byte offsets, inside a moe_layer_forward workspace, of the intermediates of the last
  * call with the same (T, experts, shared, cfg). -1 = not kept for this configuration.
  * Pair rows are in grouped order: row r of q_h / s_h / gate / up / y_pair belongs to the

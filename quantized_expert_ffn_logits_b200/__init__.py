@@ -51,6 +51,13 @@ class moe_debug_views(C.Structure):
                                           "up", "y_pair", "total")]
 
 
+MOE_STAGES = ("quant_x", "router", "topk", "group", "gate_up", "quant_h", "down")
+
+
+class moe_stage_events(C.Structure):
+    _fields_ = [("begin", C.c_void_p * len(MOE_STAGES)), ("end", C.c_void_p * len(MOE_STAGES))]
+
+
 _vp, _i32, _sz = C.c_void_p, C.c_int32, C.c_size_t
 _PB, _PC = C.POINTER(moe_expert_blob), C.POINTER(moe_route_cfg)
 _SIGS = {
@@ -65,6 +72,9 @@ _SIGS = {
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
     "moe_layer_workspace_bytes": (_sz, [_i32, _PB, _PB, _PC]),
     "moe_layer_forward": (_i32, [_vp, _i32, _vp, _vp, _PB, _PB, _PC, _vp, _vp, _sz, _vp]),
+    "moe_layer_forward_timed": (_i32, [_vp, _i32, _vp, _vp, _PB, _PB, _PC, _vp, _vp, _sz, _vp,
+                                       C.POINTER(moe_stage_events)]),
+    "moe_layer_kernel_count": (_i32, [_i32, _PB, _PB, _PC]),
     "moe_layer_debug_views": (_i32, [_i32, _PB, _PB, _PC, C.POINTER(moe_debug_views)]),
     "moe_expert_group_dots": (_i32, [_PB, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "moe_read_device_status": (_i32, [_vp, _sz, _vp]),
@@ -259,6 +269,50 @@ def moe_layer_forward(x, router_w, router_bias, experts: ExpertBlob, shared: Exp
                                   C.byref(s) if s else None, C.byref(c), _ptr(y), _ptr(workspace),
                                   workspace.numel(), _stream(stream)), "moe_layer_forward")
     return y, workspace
+
+
+def moe_layer_kernel_count(T: int, experts: ExpertBlob, shared: ExpertBlob | None,
+                           cfg: RouteCfg) -> int:
+    e = experts.struct()
+    s = shared.struct() if shared is not None else None
+    c = cfg.struct()
+    return int(_lib.moe_layer_kernel_count(T, C.byref(e), C.byref(s) if s else None, C.byref(c)))
+
+
+class Layer:
+    """A prepared layer call: the C structs and the workspace are built once, so each call
+    is one ctypes call into moe_layer_forward (or moe_layer_forward_timed with events)."""
+
+    def __init__(self, T: int, experts: ExpertBlob, shared: ExpertBlob | None, cfg: RouteCfg,
+                 router_w, router_bias=None, workspace=None):
+        import torch
+        self.T, self.experts, self.shared, self.cfg = T, experts, shared, cfg
+        self.router_w = _dev(router_w, torch.float32, "router_w")
+        self.router_bias = _dev(router_bias, torch.float32, "router_bias")
+        self._e = experts.struct()
+        self._s = shared.struct() if shared is not None else None
+        self._c = cfg.struct()
+        nb = moe_layer_workspace_bytes(T, experts, shared, cfg)
+        if nb == 0:
+            raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
+        self.workspace = workspace if workspace is not None else torch.empty(
+            nb, dtype=torch.uint8, device=router_w.device)
+        self._args = (self.router_w.data_ptr(), _ptr(self.router_bias), C.byref(self._e),
+                      C.byref(self._s) if self._s is not None else None, C.byref(self._c))
+        self.kernels = moe_layer_kernel_count(T, experts, shared, cfg)
+
+    def __call__(self, x, y, stream=None, events: moe_stage_events | None = None):
+        rw, rb, e, s, c = self._args
+        st = _stream(stream)
+        if events is None:
+            rc = _lib.moe_layer_forward(x.data_ptr(), self.T, rw, rb, e, s, c, y.data_ptr(),
+                                        self.workspace.data_ptr(), self.workspace.numel(), st)
+        else:
+            rc = _lib.moe_layer_forward_timed(x.data_ptr(), self.T, rw, rb, e, s, c, y.data_ptr(),
+                                              self.workspace.data_ptr(), self.workspace.numel(), st,
+                                              C.byref(events))
+        _check(rc, "moe_layer_forward")
+        return y
 
 
 def moe_layer_debug_views(T: int, experts: ExpertBlob, shared: ExpertBlob | None,

@@ -317,10 +317,29 @@ moe_status moe_layer_debug_views(int32_t T, const moe_expert_blob* experts,
   return MOE_OK;
 }
 
-moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
-                             const float* router_bias, const moe_expert_blob* experts,
-                             const moe_expert_blob* shared, const moe_route_cfg* cfg, float* y,
-                             void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+struct StageMarks {
+  const moe_stage_events* ev;
+  cudaStream_t st;
+  bool capturing;
+  cudaError_t err = cudaSuccess;
+  void mark(void* e) {
+    if (!e) return;
+    cudaError_t r = capturing ? cudaEventRecordWithFlags(static_cast<cudaEvent_t>(e), st, cudaEventRecordExternal)
+                              : cudaEventRecord(static_cast<cudaEvent_t>(e), st);
+    if (r != cudaSuccess) err = r;
+  }
+  void begin(int s) { if (ev) mark(ev->begin[s]); }
+  void end(int s) { if (ev) mark(ev->end[s]); }
+};
+
+moe_status forward_impl(const float* x, int32_t T, const float* router_w, const float* router_bias,
+                        const moe_expert_blob* experts, const moe_expert_blob* shared,
+                        const moe_route_cfg* cfg, float* y, void* workspace, size_t ws_bytes,
+                        void* stream, const moe_stage_events* events) {
   LayerPlan p;
   moe_status s = plan_layer(T, experts, shared, cfg, p);
   if (s != MOE_OK) return s;
@@ -331,6 +350,12 @@ moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
   if (ws_bytes < (size_t)p.L.total) return MOE_ERR_WORKSPACE;
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  StageMarks mk{events, st, false};
+  if (events) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+    mk.capturing = cs == cudaStreamCaptureStatusActive;
+  }
   const Layout& L = p.L;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto at = [&](int64_t off) -> void* { return off < 0 ? nullptr : ws + off; };
@@ -340,10 +365,14 @@ moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
   const BlobView bv = view(experts, p.eo);
 
   // 1. Q8_0 activations (also zeroes y and the status word)
+  mk.begin(MOE_STAGE_QUANT_X);
   moe::launch_quantize_act(x, T, H, ag32, static_cast<int8_t*>(at(L.qx)), at(L.sx), y, status, st);
+  mk.end(MOE_STAGE_QUANT_X);
   // 2. router logits
   float* logits = static_cast<float*>(at(L.logits));
+  mk.begin(MOE_STAGE_ROUTER);
   moe::launch_router_logits(x, router_w, T, E, H, logits, st);
+  mk.end(MOE_STAGE_ROUTER);
   // 3. top-k selection, weights and batch-union grouping
   moe::Grouping g;
   g.offsets = static_cast<int32_t*>(at(L.offsets));
@@ -353,12 +382,16 @@ moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
   g.act_begin = static_cast<int32_t*>(at(L.act_begin));
   int32_t* idx = static_cast<int32_t*>(at(L.idx));
   float* wts = static_cast<float*>(at(L.w));
+  mk.begin(MOE_STAGE_TOPK);
   moe::launch_topk(logits, cfg->score == MOE_SCORE_SIGMOID_NOAUX_TC ? router_bias : nullptr, T, E,
                    k, cfg->score, cfg->renormalize != 0, cfg->routed_scaling_factor, idx, wts,
                    T == 1 ? &g : nullptr, status, st);
+  mk.end(MOE_STAGE_TOPK);
+  mk.begin(MOE_STAGE_GROUP);
   if (T > 1)
     moe::launch_permute(idx, T, k, E, g, static_cast<uint32_t*>(at(L.masks)),
                         static_cast<int32_t*>(at(L.base)), status, 0, st);
+  mk.end(MOE_STAGE_GROUP);
 
   // 4. gate/up + SwiGLU (+ h quantization for group-32 activations)
   moe::ExpertArgs ra;
@@ -382,6 +415,7 @@ moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
   ra.dbg_b = static_cast<float*>(at(L.dbg_up));
   ra.y = y;
   ra.status = status;
+  mk.begin(MOE_STAGE_GATE_UP);
   moe::launch_gateup(ra, st);
 
   moe::ExpertArgs sa;
@@ -400,6 +434,8 @@ moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
     sa.dbg_b = static_cast<float*>(at(L.dbg_up_sh));
     moe::launch_gateup(sa, st);
   }
+  mk.end(MOE_STAGE_GATE_UP);
+  mk.begin(MOE_STAGE_QUANT_H);
   if (!ag32) {
     moe::launch_quantize_rows_token(static_cast<const float*>(at(L.hbuf)), T * k, I,
                                     static_cast<int8_t*>(at(L.qh)), static_cast<float*>(at(L.sh)), st);
@@ -408,8 +444,10 @@ moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
                                       static_cast<int8_t*>(at(L.qh_sh)),
                                       static_cast<float*>(at(L.sh_sh)), st);
   }
+  mk.end(MOE_STAGE_QUANT_H);
 
   // 5. down projection + weighted combine into y
+  mk.begin(MOE_STAGE_DOWN);
   moe::ExpertArgs rd = ra;
   rd.qa = static_cast<const int8_t*>(at(L.qh));
   rd.sa = at(L.sh);
@@ -424,8 +462,43 @@ moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
     sd.dbg_b = nullptr;
     moe::launch_down(sd, st);
   }
-  (void)H;
+  mk.end(MOE_STAGE_DOWN);
+  if (mk.err != cudaSuccess) return MOE_ERR_CUDA;
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
+                             const float* router_bias, const moe_expert_blob* experts,
+                             const moe_expert_blob* shared, const moe_route_cfg* cfg, float* y,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  return forward_impl(x, T, router_w, router_bias, experts, shared, cfg, y, workspace, ws_bytes,
+                      stream, nullptr);
+}
+
+moe_status moe_layer_forward_timed(const float* x, int32_t T, const float* router_w,
+                                   const float* router_bias, const moe_expert_blob* experts,
+                                   const moe_expert_blob* shared, const moe_route_cfg* cfg,
+                                   float* y, void* workspace, size_t ws_bytes, void* stream,
+                                   const moe_stage_events* events) {
+  return forward_impl(x, T, router_w, router_bias, experts, shared, cfg, y, workspace, ws_bytes,
+                      stream, events);
+}
+
+int32_t moe_layer_kernel_count(int32_t T, const moe_expert_blob* experts,
+                               const moe_expert_blob* shared, const moe_route_cfg* cfg) {
+  if (moe_layer_workspace_bytes(T, experts, shared, cfg) == 0) return -1;
+  if (T == 0) return 0;
+  const int sh = shared ? 1 : 0;
+  int n = 3;                                   // quantize x, router logits, top-k
+  n += T > 1;                                  // grouping
+  n += 1 + sh;                                 // gate/up
+  if (cfg->act != MOE_ACT_G32_F16) n += 1 + sh;   // h quantization
+  n += 1 + sh;                                 // down
+  return n;
 }
 
 moe_status moe_expert_group_dots(const moe_expert_blob* blob, int32_t which, int32_t n,
