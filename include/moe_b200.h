@@ -181,6 +181,23 @@ MOE_API size_t moe_permute_workspace_bytes(int32_t T, int32_t k, int32_t E);
 MOE_API moe_status moe_permute(const int32_t* idx, int32_t T, int32_t k, int32_t E, int32_t* offsets,
                        int32_t* perm, void* workspace, size_t ws_bytes, void* stream);
 
+/* moe_permute without a workspace argument and without allocating. (The pages have no
+ * counterpart: this exists for callers that can neither allocate device memory nor pass a
+ * scratch buffer -- code running during CUDA graph capture, serving loops whose memory is
+ * fully owned by a framework allocator, plugin hosts that hand an operator only its tensors.)
+ * Scratch is a 1 MiB array compiled into the library as a device global, so every GPU that
+ * loads the library holds it until the process exits; a grouping whose scratch need,
+ * moe_permute_workspace_bytes(T, k, E), exceeds 1 MiB returns MOE_ERR_WORKSPACE (for example
+ * T = 4096 with E = 512 fits, T = 8192 with E = 1024 does not). The first call on each device
+ * looks up the array's device address (cudaGetSymbolAddress); make that first call before
+ * any stream capture on that device. All calls share the one array: calls that may overlap
+ * on the GPU (different streams without ordering, several host threads) race and corrupt
+ * each other's results; order them on one stream. Out-of-range expert ids are dropped, as in
+ * moe_permute; the device status word that records them is not readable through this entry
+ * point. Other errors and arguments as moe_permute. */
+MOE_API moe_status moe_permute_no_alloc(const int32_t* idx, int32_t T, int32_t k, int32_t E,
+                                        int32_t* offsets, int32_t* perm, void* stream);
+
 /* Workspace bytes moe_layer_forward needs; 0 if the arguments are unsupported. */
 MOE_API size_t moe_layer_workspace_bytes(int32_t T, const moe_expert_blob* experts,
                                  const moe_expert_blob* shared, const moe_route_cfg* cfg);

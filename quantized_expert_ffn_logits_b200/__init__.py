@@ -70,6 +70,7 @@ _SIGS = {
     "moe_route_topk": (_i32, [_vp, _vp, _i32, _i32, _PC, _vp, _vp, _vp]),
     "moe_permute_workspace_bytes": (_sz, [_i32, _i32, _i32]),
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_no_alloc": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_layer_workspace_bytes": (_sz, [_i32, _PB, _PB, _PC]),
     "moe_layer_forward": (_i32, [_vp, _i32, _vp, _vp, _PB, _PB, _PC, _vp, _vp, _sz, _vp]),
     "moe_layer_forward_timed": (_i32, [_vp, _i32, _vp, _vp, _PB, _PB, _PC, _vp, _vp, _sz, _vp,
@@ -235,6 +236,19 @@ def moe_permute(idx, n_experts: int, stream=None):
     _check(_lib.moe_permute(_ptr(idx), T, k, n_experts, _ptr(offsets), _ptr(perm), _ptr(ws),
                             ws.numel(), _stream(stream)), "moe_permute")
     return offsets, perm, ws
+
+
+def moe_permute_no_alloc(idx, n_experts: int, stream=None):
+    """moe_permute with the library's fixed 1 MiB device scratch (no workspace, no allocation
+    inside the library; see include/moe_b200.h for the limits)."""
+    import torch
+    _dev(idx, torch.int32, "idx")
+    T, k = idx.shape
+    offsets = torch.empty(n_experts + 1, dtype=torch.int32, device=idx.device)
+    perm = torch.empty(T * k, dtype=torch.int32, device=idx.device)
+    _check(_lib.moe_permute_no_alloc(_ptr(idx), T, k, n_experts, _ptr(offsets), _ptr(perm),
+                                     _stream(stream)), "moe_permute_no_alloc")
+    return offsets, perm
 
 
 def moe_layer_workspace_bytes(T: int, experts: ExpertBlob, shared: ExpertBlob | None,
