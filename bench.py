@@ -347,8 +347,11 @@ def gpu_arm(args, cfg, T):
             layers[s % R](xs[s % G], y, stream)
     stream.synchronize()
 
-    # one graph period of G steps with stage events around every step (torch events used
-    # as plain cudaEvent_t handles; recorded once eagerly so the handles exist)
+    # Graphs: `graph_ev` = one period of G steps with every stage bracketed by CUDA events
+    # (external event nodes; they cut the programmatic edges around them, so this period
+    # runs slower), `graph` = G steps without events, `graph_rem` = the remainder. The timed
+    # region replays `graph` for the first K - G steps and `graph_ev` for the last G, so the
+    # per-launch stage durations are read live from inside the timed region.
     nst = len(M.MOE_STAGES)
     evs = []
     with torch.cuda.stream(stream):
@@ -365,20 +368,27 @@ def gpu_arm(args, cfg, T):
                 pair.append((b_ev, e_ev))
             evs.append((e, pair))
     stream.synchronize()
+    graph_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ev, stream=stream):
+        for s in range(G):
+            layers[s % R](xs[s], y, stream, events=evs[s][0])
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for s in range(G):
-            layers[s % R](xs[s], y, stream, events=evs[s][0])
-    rem = args.steps % G
+            layers[s % R](xs[s], y, stream)
+    n_main, rem = divmod(args.steps - G, G)
     graph_rem = None
     if rem:
         graph_rem = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph_rem, stream=stream):
             for s in range(rem):
                 layers[s % R](xs[s], y, stream)
-    # one untimed replay
+    # one untimed replay of each
     with torch.cuda.stream(stream):
         graph.replay()
+        graph_ev.replay()
+        if graph_rem is not None:
+            graph_rem.replay()
     stream.synchronize()
 
     # ------------------------------------------------------------ timed region
@@ -396,10 +406,11 @@ def gpu_arm(args, cfg, T):
     w0 = time.perf_counter()
     with torch.cuda.stream(stream):
         start.record(stream)
-        for _ in range(args.steps // G):
+        for _ in range(n_main):
             graph.replay()
         if graph_rem is not None:
             graph_rem.replay()
+        graph_ev.replay()
         end.record(stream)
     stream.synchronize()
     w1 = time.perf_counter()
@@ -415,7 +426,7 @@ def gpu_arm(args, cfg, T):
 
     # per-stage device times of the last graph period (inside the timed region)
     stage_ms = {n: [] for n in M.MOE_STAGES}
-    if args.steps >= G:
+    if True:
         for s in range(G):
             for i, n in enumerate(M.MOE_STAGES):
                 b_ev, e_ev = evs[s][1][i]
@@ -489,7 +500,7 @@ def gpu_arm(args, cfg, T):
         "config": {"workload": workload_desc(cfg, T), "T": T, "replicas": R,
                    "l2": f"inputs larger than L2: {R} layer replicas rotate "
                          f"({R * layers[0].experts.nbytes / 1e9:.2f} GB of expert blobs)",
-                   "graph": f"CUDA graph of {G} steps replayed", "accumulate": "int32 dots, fp32 scales",
+                   "graph": f"CUDA graphs of {G} steps; the last {G} timed steps carry per-stage event nodes", "accumulate": "int32 dots, fp32 scales",
                    "parallelism": f"dp{world} (weak: independent tokens per GPU)"},
         "roofline": roof,
         "layer": layer,
@@ -498,7 +509,7 @@ def gpu_arm(args, cfg, T):
         "gpu_launches": launches,
         "clocks": clk,
     }
-    del graph, graph_rem
+    del graph, graph_rem, graph_ev
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:

@@ -136,6 +136,10 @@ typedef struct {
 /* Version of this ABI (MOE_ABI_VERSION). */
 MOE_API int32_t moe_abi_version(void);
 
+/* Description of the last MOE_ERR_CUDA returned on the calling host thread (which call
+ * failed and the CUDA error text); "" if none. Valid until the thread's next failing call. */
+MOE_API const char* moe_last_error(void);
+
 /* Human-readable name of a status code (static string). */
 MOE_API const char* moe_status_string(moe_status s);
 
@@ -207,8 +211,16 @@ MOE_API size_t moe_layer_workspace_bytes(int32_t T, const moe_expert_blob* exper
  *   experts: the routed experts; shared: NULL or one expert (n_experts = 1) with the same
  *   hidden size, wtype and wscale as `experts` and its own intermediate size.
  * workspace: device buffer of ws_bytes >= moe_layer_workspace_bytes(); it holds every
- * intermediate (quantized x, logits, routing, grouping, quantized h) and the device status
- * word. Calls that share a workspace must be ordered on one stream. */
+ * intermediate (quantized x, logits, routing, grouping, quantized h) and, in its first 256
+ * bytes, a control block (device status word, routing ticket counter). The control block must
+ * be zero before the workspace is first used (allocate it zeroed, e.g. cudaMemset once); the
+ * library leaves it consistent after every call. Calls that share a workspace must be ordered
+ * on one stream.
+ * Launch sequence: for T <= 32 one routing kernel (activation quantization, logits, top-k and
+ * grouping; the last CTA to finish its logit does the selection), then one gate/up kernel and
+ * one down kernel, each covering the routed and the shared experts; larger T routes through
+ * four kernels. Kernels use programmatic dependent launch, so under stream capture the graph
+ * gets programmatic edges. */
 MOE_API moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
                              const float* router_bias, const moe_expert_blob* experts,
                              const moe_expert_blob* shared, const moe_route_cfg* cfg, float* y,
@@ -285,7 +297,10 @@ MOE_API moe_status moe_expert_group_dots(const moe_expert_blob* blob, int32_t wh
                                  const int32_t* expert, const int32_t* row, const int8_t* act,
                                  int32_t* dots, void* stream);
 
-/* Reads and clears the device status word of a moe_layer_forward / moe_permute workspace.
+/* The control block's int32 words [2] and [3] record the first bounded wait that gave up
+ * during the last call (MOE_ERR_TIMEOUT): [2] = kernel (1 gate/up, 2 down) | role (1 producer,
+ * 2 consumer) << 4 | pipeline stage << 8, [3] = the CTA index; both 0 otherwise.
+ * Reads and clears the device status word of a moe_layer_forward / moe_permute workspace.
  * Synchronizes `stream`. Returns MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT as
  * recorded by the kernels, or MOE_ERR_CUDA if the copy fails. */
 MOE_API moe_status moe_read_device_status(void* workspace, size_t ws_bytes, void* stream);

@@ -63,6 +63,7 @@ _PB, _PC = C.POINTER(moe_expert_blob), C.POINTER(moe_route_cfg)
 _SIGS = {
     "moe_abi_version": (_i32, []),
     "moe_status_string": (C.c_char_p, [_i32]),
+    "moe_last_error": (C.c_char_p, []),
     "moe_expert_blob_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "moe_quantize_experts": (_i32, [_vp, _vp, _PB, _vp]),
     "moe_quantize_activations": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp]),
@@ -90,7 +91,10 @@ for _name, (_res, _args) in _SIGS.items():
 class MoeError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {moe_status_string(status)}")
+        detail = ""
+        if status == MOE_ERR_CUDA:
+            detail = " [" + _lib.moe_last_error().decode() + "]"
+        super().__init__(f"{where}: {moe_status_string(status)}{detail}")
 
 
 def _check(rc: int, where: str) -> None:
@@ -274,7 +278,7 @@ def moe_layer_forward(x, router_w, router_bias, experts: ExpertBlob, shared: Exp
     if nb == 0:
         raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
     if workspace is None:
-        workspace = torch.empty(nb, dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(nb, dtype=torch.uint8, device=x.device)   # control block zeroed
     _dev(workspace, torch.uint8, "workspace")
     e = experts.struct()
     s = shared.struct() if shared is not None else None
@@ -309,8 +313,8 @@ class Layer:
         nb = moe_layer_workspace_bytes(T, experts, shared, cfg)
         if nb == 0:
             raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
-        self.workspace = workspace if workspace is not None else torch.empty(
-            nb, dtype=torch.uint8, device=router_w.device)
+        self.workspace = workspace if workspace is not None else torch.zeros(
+            nb, dtype=torch.uint8, device=router_w.device)   # control block zeroed
         self._args = (self.router_w.data_ptr(), _ptr(self.router_bias), C.byref(self._e),
                       C.byref(self._s) if self._s is not None else None, C.byref(self._c))
         self.kernels = moe_layer_kernel_count(T, experts, shared, cfg)

@@ -1,6 +1,7 @@
 // api.cu -- the C ABI (include/moe_b200.h): argument checks, workspace layout and
 // the launch sequence of the layer forward.
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 
 #include "../../include/moe_b200.h"
@@ -12,6 +13,9 @@ namespace {
 using moe::BlobView;
 
 inline int64_t al256(int64_t v) { return (v + 255) & ~int64_t(255); }
+
+// Batches up to this many tokens take the single-launch routing kernel.
+constexpr int32_t kFusedRouteMaxT = 32;
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 struct BlobOffsets {
@@ -156,8 +160,16 @@ moe_status plan_layer(int32_t T, const moe_expert_blob* experts, const moe_exper
   return MOE_OK;
 }
 
+thread_local char g_last_error[256] = "";
+
+moe_status cuda_fail(const char* where, cudaError_t e) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e), (int)e);
+  return MOE_ERR_CUDA;
+}
+
 moe_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : cuda_fail("launch", e);
 }
 
 }  // namespace
@@ -165,6 +177,8 @@ moe_status launch_status() {
 extern "C" {
 
 int32_t moe_abi_version(void) { return MOE_ABI_VERSION; }
+
+const char* moe_last_error(void) { return g_last_error; }
 
 const char* moe_status_string(moe_status s) {
   switch (s) {
@@ -193,7 +207,8 @@ moe_status moe_quantize_experts(const float* w_gate_up, const float* w_down,
   const moe_status s = check_blob(out, o);
   if (s != MOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(out->data, 0, (size_t)o.total, st) != cudaSuccess) return MOE_ERR_CUDA;
+  const cudaError_t me = cudaMemsetAsync(out->data, 0, (size_t)o.total, st);
+  if (me != cudaSuccess) return cuda_fail("blob memset", me);
   const BlobView b = view(out, o);
   uint8_t* d = static_cast<uint8_t*>(out->data);
   moe::launch_quantize_experts(w_gate_up, w_down, b, d + o.gu_w, d + o.dn_w, d + o.gu_s,
@@ -353,7 +368,8 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   StageMarks mk{events, st, false};
   if (events) {
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return MOE_ERR_CUDA;
+    const cudaError_t ce = cudaStreamIsCapturing(st, &cs);
+    if (ce != cudaSuccess) return cuda_fail("cudaStreamIsCapturing", ce);
     mk.capturing = cs == cudaStreamCaptureStatusActive;
   }
   const Layout& L = p.L;
@@ -364,16 +380,6 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   int* status = static_cast<int*>(at(L.status));
   const BlobView bv = view(experts, p.eo);
 
-  // 1. Q8_0 activations (also zeroes y and the status word)
-  mk.begin(MOE_STAGE_QUANT_X);
-  moe::launch_quantize_act(x, T, H, ag32, static_cast<int8_t*>(at(L.qx)), at(L.sx), y, status, st);
-  mk.end(MOE_STAGE_QUANT_X);
-  // 2. router logits
-  float* logits = static_cast<float*>(at(L.logits));
-  mk.begin(MOE_STAGE_ROUTER);
-  moe::launch_router_logits(x, router_w, T, E, H, logits, st);
-  mk.end(MOE_STAGE_ROUTER);
-  // 3. top-k selection, weights and batch-union grouping
   moe::Grouping g;
   g.offsets = static_cast<int32_t*>(at(L.offsets));
   g.perm = static_cast<int32_t*>(at(L.perm));
@@ -382,18 +388,69 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   g.act_begin = static_cast<int32_t*>(at(L.act_begin));
   int32_t* idx = static_cast<int32_t*>(at(L.idx));
   float* wts = static_cast<float*>(at(L.w));
-  mk.begin(MOE_STAGE_TOPK);
-  moe::launch_topk(logits, cfg->score == MOE_SCORE_SIGMOID_NOAUX_TC ? router_bias : nullptr, T, E,
-                   k, cfg->score, cfg->renormalize != 0, cfg->routed_scaling_factor, idx, wts,
-                   T == 1 ? &g : nullptr, status, st);
-  mk.end(MOE_STAGE_TOPK);
-  mk.begin(MOE_STAGE_GROUP);
-  if (T > 1)
+  float* logits = static_cast<float*>(at(L.logits));
+  const float* bias = cfg->score == MOE_SCORE_SIGMOID_NOAUX_TC ? router_bias : nullptr;
+  cudaError_t err = cudaSuccess;
+  const char* err_where = "";
+  auto keep = [&](cudaError_t e, const char* where) {
+    if (e != cudaSuccess && err == cudaSuccess) {
+      err = e;
+      err_where = where;
+    }
+  };
+
+  if (T <= kFusedRouteMaxT) {
+    // 1-3. activation quantization, router logits, top-k and grouping in one launch
+    moe::RouteArgs r;
+    r.x = x;
+    r.wr = router_w;
+    r.bias = bias;
+    r.T = T;
+    r.E = E;
+    r.H = H;
+    r.k = k;
+    r.score = cfg->score;
+    r.renorm = cfg->renormalize != 0;
+    r.ag32 = ag32;
+    r.rsf = cfg->routed_scaling_factor;
+    r.qx = static_cast<int8_t*>(at(L.qx));
+    r.sx = at(L.sx);
+    r.y = y;
+    r.logits = logits;
+    r.idx = idx;
+    r.w = wts;
+    r.g = g;
+    r.status = status;
+    r.ticket = reinterpret_cast<unsigned*>(ws + L.status + 4);
+    mk.begin(MOE_STAGE_QUANT_X);
+    keep(moe::launch_route_fused(r, st), "routing kernel");
+    mk.end(MOE_STAGE_QUANT_X);
+    for (int sg = MOE_STAGE_ROUTER; sg <= MOE_STAGE_GROUP; ++sg) {
+      mk.begin(sg);
+      mk.end(sg);
+    }
+  } else {
+    // 1. Q8_0 activations (also zeroes y and the status word)
+    mk.begin(MOE_STAGE_QUANT_X);
+    moe::launch_quantize_act(x, T, H, ag32, static_cast<int8_t*>(at(L.qx)), at(L.sx), y, status, st);
+    mk.end(MOE_STAGE_QUANT_X);
+    // 2. router logits
+    mk.begin(MOE_STAGE_ROUTER);
+    moe::launch_router_logits(x, router_w, T, E, H, logits, st);
+    mk.end(MOE_STAGE_ROUTER);
+    // 3. top-k selection and weights, batch-union grouping
+    mk.begin(MOE_STAGE_TOPK);
+    moe::launch_topk(logits, bias, T, E, k, cfg->score, cfg->renormalize != 0,
+                     cfg->routed_scaling_factor, idx, wts, nullptr, status, st);
+    mk.end(MOE_STAGE_TOPK);
+    mk.begin(MOE_STAGE_GROUP);
     moe::launch_permute(idx, T, k, E, g, static_cast<uint32_t*>(at(L.masks)),
                         static_cast<int32_t*>(at(L.base)), status, 0, st);
-  mk.end(MOE_STAGE_GROUP);
+    mk.end(MOE_STAGE_GROUP);
+  }
 
-  // 4. gate/up + SwiGLU (+ h quantization for group-32 activations)
+  // 4. gate/up + SwiGLU (+ h quantization for group-32 activations); routed and shared
+  //    experts in one grid
   moe::ExpertArgs ra;
   std::memset(&ra, 0, sizeof(ra));
   ra.b = bv;
@@ -415,10 +472,8 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   ra.dbg_b = static_cast<float*>(at(L.dbg_up));
   ra.y = y;
   ra.status = status;
-  mk.begin(MOE_STAGE_GATE_UP);
-  moe::launch_gateup(ra, st);
-
   moe::ExpertArgs sa;
+  std::memset(&sa, 0, sizeof(sa));
   if (shared) {
     sa = ra;
     sa.b = view(shared, p.so);
@@ -432,8 +487,9 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     sa.hbuf = static_cast<float*>(at(L.hbuf_sh));
     sa.dbg_a = static_cast<float*>(at(L.dbg_gate_sh));
     sa.dbg_b = static_cast<float*>(at(L.dbg_up_sh));
-    moe::launch_gateup(sa, st);
   }
+  mk.begin(MOE_STAGE_GATE_UP);
+  keep(moe::launch_gateup_tma(ra, shared ? &sa : nullptr, st), "gate/up kernel");
   mk.end(MOE_STAGE_GATE_UP);
   mk.begin(MOE_STAGE_QUANT_H);
   if (!ag32) {
@@ -446,24 +502,24 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   }
   mk.end(MOE_STAGE_QUANT_H);
 
-  // 5. down projection + weighted combine into y
-  mk.begin(MOE_STAGE_DOWN);
+  // 5. down projection + weighted combine into y; routed and shared experts in one grid
   moe::ExpertArgs rd = ra;
   rd.qa = static_cast<const int8_t*>(at(L.qh));
   rd.sa = at(L.sh);
   rd.dbg_a = static_cast<float*>(at(L.dbg_y));
   rd.dbg_b = nullptr;
-  moe::launch_down(rd, st);
+  moe::ExpertArgs sd = sa;
   if (shared) {
-    moe::ExpertArgs sd = sa;
     sd.qa = static_cast<const int8_t*>(at(L.qh_sh));
     sd.sa = at(L.sh_sh);
     sd.dbg_a = static_cast<float*>(at(L.dbg_y_sh));
     sd.dbg_b = nullptr;
-    moe::launch_down(sd, st);
   }
+  mk.begin(MOE_STAGE_DOWN);
+  keep(moe::launch_down_tma(rd, shared ? &sd : nullptr, st), "down kernel");
   mk.end(MOE_STAGE_DOWN);
-  if (mk.err != cudaSuccess) return MOE_ERR_CUDA;
+  if (err != cudaSuccess) return cuda_fail(err_where, err);
+  if (mk.err != cudaSuccess) return cuda_fail("stage event record", mk.err);
   return launch_status();
 }
 
@@ -492,12 +548,10 @@ int32_t moe_layer_kernel_count(int32_t T, const moe_expert_blob* experts,
                                const moe_expert_blob* shared, const moe_route_cfg* cfg) {
   if (moe_layer_workspace_bytes(T, experts, shared, cfg) == 0) return -1;
   if (T == 0) return 0;
-  const int sh = shared ? 1 : 0;
-  int n = 3;                                   // quantize x, router logits, top-k
-  n += T > 1;                                  // grouping
-  n += 1 + sh;                                 // gate/up
-  if (cfg->act != MOE_ACT_G32_F16) n += 1 + sh;   // h quantization
-  n += 1 + sh;                                 // down
+  int n = T <= kFusedRouteMaxT ? 1 : 4;        // routing (fused, or quantize/logits/top-k/grouping)
+  n += 1;                                       // gate/up, routed and shared experts in one grid
+  if (cfg->act != MOE_ACT_G32_F16) n += 1 + (shared ? 1 : 0);   // h quantization
+  n += 1;                                       // down, routed and shared experts in one grid
   return n;
 }
 
@@ -519,9 +573,12 @@ moe_status moe_read_device_status(void* workspace, size_t ws_bytes, void* stream
   if (!workspace || ws_bytes < 4) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t h = 0;
-  if (cudaMemcpyAsync(&h, workspace, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
-  if (cudaMemsetAsync(workspace, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaError_t e = cudaMemcpyAsync(&h, workspace, 4, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail("status copy", e);
+  e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail("status synchronize", e);
+  e = cudaMemsetAsync(workspace, 0, 4, st);
+  if (e != cudaSuccess) return cuda_fail("status clear", e);
   return static_cast<moe_status>(h);
 }
 

@@ -80,6 +80,20 @@ __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Streaming 128-bit load of read-only data (no L1 allocation: weights are read once).
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+  uint4 v;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(p));
+  return v;
+}
+
+// Fire-and-forget prefetch of the line holding p into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // --------------------------------------------------------------- integer dots
 // Signed x signed 4-way byte dot.
 __device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {

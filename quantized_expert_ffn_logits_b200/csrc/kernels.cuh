@@ -64,8 +64,53 @@ struct ExpertArgs {
   int* status;
 };
 
-void launch_gateup(const ExpertArgs& a, cudaStream_t st);
-void launch_down(const ExpertArgs& a, cudaStream_t st);
+// ---- expert_stream.cu: routed experts `r` and (optional) shared expert `s` in one grid each
+cudaError_t launch_gateup_tma(const ExpertArgs& r, const ExpertArgs* s, cudaStream_t st);
+cudaError_t launch_down_tma(const ExpertArgs& r, const ExpertArgs* s, cudaStream_t st);
+
+// ---- route_fused.cu (T <= 32)
+struct RouteArgs {
+  const float* x;
+  const float* wr;
+  const float* bias;      // sigmoid mode only, may be null
+  int T, E, H, k, score, renorm, ag32;
+  float rsf;
+  int8_t* qx;
+  void* sx;
+  float* y;               // zeroed here
+  float* logits;
+  int32_t* idx;
+  float* w;
+  Grouping g;
+  int* status;
+  unsigned* ticket;       // zero between calls; the last CTA resets it
+};
+cudaError_t launch_route_fused(const RouteArgs& r, cudaStream_t st);
+
+#ifdef MOE_NO_PDL
+constexpr bool kUsePdl = false;
+#else
+constexpr bool kUsePdl = true;
+#endif
+
+// Launch with programmatic stream serialization (the kernel calls griddepcontrol.wait
+// before touching its predecessor's outputs).
+template <typename Kern, typename... Args>
+inline cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = kUsePdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 void launch_group_dots(const BlobView& b, int which, int n, const int32_t* expert,
                        const int32_t* row, const int8_t* act, int32_t* dots, cudaStream_t st);
 

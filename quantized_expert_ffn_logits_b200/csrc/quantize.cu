@@ -6,6 +6,7 @@
 // section; group size 32 from the mtlm-7m-base card, "Files").
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tma.cuh"
 
 namespace moe {
 
@@ -93,9 +94,15 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const float* __restric
 __global__ void __launch_bounds__(256) k_quantize_act(const float* __restrict__ x, int T, int H,
                                                       int g32, int8_t* __restrict__ q,
                                                       void* scales, float* y_zero, int* status) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   if (t >= T) return;
-  if (status && t == 0 && threadIdx.x == 0) *status = 0;
+  if (status && t == 0 && threadIdx.x == 0) {
+    status[0] = 0;
+    status[2] = 0;
+    status[3] = 0;
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const float* xr = x + (int64_t)t * H;
   int8_t* qr = q + (int64_t)t * H;
@@ -134,6 +141,8 @@ __global__ void __launch_bounds__(256) k_quantize_act(const float* __restrict__ 
 __global__ void __launch_bounds__(256) k_quantize_rows_token(const float* __restrict__ h, int rows,
                                                              int K, int8_t* __restrict__ q,
                                                              float* __restrict__ scales) {
+  pdl_wait();
+  pdl_trigger();
   const int r = blockIdx.x;
   if (r >= rows) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -167,13 +176,13 @@ void launch_quantize_experts(const float* w_gu, const float* w_dn, const BlobVie
 void launch_quantize_act(const float* x, int T, int H, int g32, int8_t* q, void* scales,
                          float* y_zero, int* status, cudaStream_t st) {
   if (T <= 0) return;
-  k_quantize_act<<<T, 256, 0, st>>>(x, T, H, g32, q, scales, y_zero, status);
+  launch_pdl(k_quantize_act, dim3(T), dim3(256), 0, st, x, T, H, g32, q, scales, y_zero, status);
 }
 
 void launch_quantize_rows_token(const float* h, int rows, int K, int8_t* q, float* scales,
                                 cudaStream_t st) {
   if (rows <= 0) return;
-  k_quantize_rows_token<<<rows, 256, 0, st>>>(h, rows, K, q, scales);
+  launch_pdl(k_quantize_rows_token, dim3(rows), dim3(256), 0, st, h, rows, K, q, scales);
 }
 
 }  // namespace moe

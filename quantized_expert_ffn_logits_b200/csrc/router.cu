@@ -9,6 +9,8 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "tma.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -21,6 +23,8 @@ __global__ void __launch_bounds__(256) k_router_small(const float* __restrict__ 
                                                       const float* __restrict__ wr, int T, int E,
                                                       int H, float* __restrict__ logits) {
   extern __shared__ float part[];  // [TT][C]
+  pdl_wait();
+  pdl_trigger();
   const int e = blockIdx.x;
   const int t0 = blockIdx.y * TT;
   const int C = H / 32;
@@ -60,6 +64,8 @@ __global__ void __launch_bounds__(256) k_router_tiled(const float* __restrict__ 
                                                       int H, float* __restrict__ logits) {
   __shared__ __align__(16) float xs[32][68];
   __shared__ __align__(16) float ws[32][68];
+  pdl_wait();
+  pdl_trigger();
   const int tb = blockIdx.y * 64, eb = blockIdx.x * 64;
   const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
   float total[4][4];
@@ -117,87 +123,30 @@ void launch_router_logits(const float* x, const float* wr, int T, int E, int H, 
     const int C = H / 32;
     dim3 grid(E, (T + TT - 1) / TT);
     const int threads = C >= 256 ? 256 : ((C + 31) / 32) * 32;
-    k_router_small<TT><<<grid, threads, TT * C * sizeof(float), st>>>(x, wr, T, E, H, logits);
+    launch_pdl(k_router_small<TT>, grid, dim3(threads), TT * C * sizeof(float), st, x, wr, T, E, H,
+               logits);
   } else {
     dim3 grid((E + 63) / 64, (T + 63) / 64);
-    k_router_tiled<<<grid, 256, 0, st>>>(x, wr, T, E, H, logits);
+    launch_pdl(k_router_tiled, grid, dim3(256), 0, st, x, wr, T, E, H, logits);
   }
 }
 
 // ------------------------------------------------------------------- top-k
-// One warp per token; lane l holds the keys of experts l, l+32, ... (NE per lane).
-// k rounds of a warp arg-max (larger key wins, equal keys go to the lower expert).
+// One warp per token (warp_topk); for a single token the grouping is written too.
 template <int NE>
 __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits,
                                               const float* __restrict__ bias, int T, int E, int k,
                                               int score, int renorm, float rsf,
                                               int32_t* __restrict__ idx, float* __restrict__ w,
                                               Grouping g1, int single, int* status) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  const float* Lt = logits + (int64_t)t * E;
-  float key[NE], lg[NE];
-#pragma unroll
-  for (int m = 0; m < NE; ++m) {
-    const int e = lane + 32 * m;
-    lg[m] = e < E ? Lt[e] : 0.0f;
-    if (e >= E) key[m] = -FLT_MAX;
-    else if (score == 0) key[m] = lg[m];
-    else key[m] = __fadd_rn(csigmoid(lg[m]), bias ? bias[e] : 0.0f);
-  }
-  uint32_t taken = 0;
-  int my_e = 0;
-  for (int j = 0; j < k; ++j) {
-    float bk = -FLT_MAX;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int m = 0; m < NE; ++m) {
-      const int e = lane + 32 * m;
-      if (e < E && !((taken >> m) & 1u) && (key[m] > bk || be == 0x7fffffff)) {
-        bk = key[m];
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ok > bk || (ok == bk && oe < be)) {
-        bk = ok;
-        be = oe;
-      }
-    }
-    if (be < E && (be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == j) my_e = be;
-  }
+  const int my_e = warp_topk<NE>(logits + (int64_t)t * E, bias, E, k, score, renorm, rsf,
+                                 idx + (int64_t)t * k, w + (int64_t)t * k, status);
   const bool sel = lane < k;
-  if (sel && (my_e < 0 || my_e >= E)) set_status(status, kStatusDeviceCheck);
-  const float myL = sel ? Lt[min(max(my_e, 0), E - 1)] : 0.0f;
-  float wv;
-  if (score == 0) {
-    const float Lmax = __shfl_sync(0xffffffffu, myL, 0);
-    const float ex = sel ? cexp(myL - Lmax) : 0.0f;
-    float den;
-    if (renorm) {
-      den = warp_sum(ex);
-    } else {
-      float s = 0.0f;
-#pragma unroll
-      for (int m = 0; m < NE; ++m)
-        if (lane + 32 * m < E) s += cexp(lg[m] - Lmax);
-      den = warp_sum(s);
-    }
-    wv = ex / den * rsf;
-  } else {
-    const float s = sel ? csigmoid(myL) : 0.0f;
-    const float den = renorm ? warp_sum(s) : 1.0f;
-    wv = s / den * rsf;
-  }
-  if (sel) {
-    idx[(int64_t)t * k + lane] = my_e;
-    w[(int64_t)t * k + lane] = wv;
-  }
   if (single) {
     // One token: the grouping is the k selected experts in ascending order.
     int rank = 0;
@@ -229,9 +178,9 @@ void launch_topk(const float* logits, const float* bias, int T, int E, int k, in
   Grouping g{};
   if (single_token) g = *single_token;
   const int single = single_token != nullptr;
-#define MOE_TOPK_CASE(N)                                                                    \
-  k_topk<N><<<blocks, 256, 0, st>>>(logits, bias, T, E, k, score, renorm, rsf, idx, w, g, \
-                                    single, status)
+#define MOE_TOPK_CASE(N)                                                                     \
+  launch_pdl(k_topk<N>, dim3(blocks), dim3(256), 0, st, logits, bias, T, E, k, score, renorm, rsf, \
+             idx, w, g, single, status)
   if (E <= 32) MOE_TOPK_CASE(1);
   else if (E <= 64) MOE_TOPK_CASE(2);
   else if (E <= 128) MOE_TOPK_CASE(4);
@@ -253,6 +202,8 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
   __shared__ int32_t off_s[1024];
   __shared__ int32_t wsum[32], fsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_trigger();
   if (reset_status && tid == 0 && status) *status = 0;
   __syncthreads();
   const int C = (T + 31) / 32;
@@ -345,7 +296,8 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
 void launch_permute(const int32_t* idx, int T, int k, int E, const Grouping& g, uint32_t* masks,
                     int32_t* base, int* status, int reset_status, cudaStream_t st) {
   if (T <= 0) return;
-  k_permute<<<1, 1024, 0, st>>>(idx, T, k, E, g, masks, base, status, reset_status);
+  launch_pdl(k_permute, dim3(1), dim3(1024), 0, st, idx, T, k, E, g, masks, base, status,
+             reset_status);
 }
 
 }  // namespace moe
