@@ -101,16 +101,21 @@ enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID_NOAUX_TC = 1 };
  *
  * `data` (device, 256-byte aligned, caller-owned) holds `bytes` >= moe_expert_blob_bytes().
  * Byte layout, four regions each starting at a multiple of 256 bytes from `data`:
- *   R0 gate/up codes: for each expert e, for each s in [0, I/128): a block of
- *      256 rows -- rows 0..127 are gate rows 128s..128s+127, rows 128..255 the
- *      up rows of the same intermediate indices -- stored as [KB/16][256][16]:
- *      16-byte piece p of row r at (p * 256 + r) * 16. KB = H (int8) or H/2
- *      (int4; element 2j in the low nibble of byte j).
- *   R1 down codes: for each e, for each s in [0, H/128): rows 128s..128s+127 of
- *      the [H][I] down matrix stored [KBd/16][128][16], KBd = I or I/2.
- *   R2 gate/up scales: for each e, each 256-row block: fp16 [H/32][256]
- *      (group-major) or fp32 [256].
- *   R3 down scales: for each e, each 128-row block: fp16 [I/32][128] or fp32 [128].
+ *   R0 gate/up codes: for each expert e, for each s in [0, I/64): a block of
+ *      128 rows -- rows 0..63 are gate rows 64s..64s+63, rows 64..127 the up
+ *      rows of the same intermediate indices -- stored as [KB/16][128][16]:
+ *      16-byte piece p of row r at (p * 128 + r) * 16. KB = H (int8) or H/2
+ *      (int4; element 2j in the low nibble of byte j). One block's K range is
+ *      one contiguous run, one piece of it 2 KB.
+ *   R1 down codes: the [H][I] matrix of expert e cut along I into slabs of 64
+ *      intermediate indices: for each e, each u in [0, I/64), each b in
+ *      [0, H/128): rows 128b..128b+127, columns 64u..64u+63, stored
+ *      [SB/16][128][16] (SB = 64 bytes int8, 32 bytes int4). One slab (all H
+ *      rows of 64 columns) is one contiguous run.
+ *   R2 gate/up scales: for each e, each 128-row block: fp16 [H/32][128]
+ *      (group-major) or fp32 [128].
+ *   R3 down scales: fp16: for each e, u, b as in R1: [2][128] (the two groups
+ *      of the slab); fp32: [E][H], one per row.
  * Padding bytes between regions are zero. */
 typedef struct {
   int32_t wtype;      /* MOE_W_INT8 | MOE_W_INT4 */

@@ -156,9 +156,11 @@ int orc_pack_int4(const int8_t* q, int64_t N, int K, uint8_t* out) {
 /* The blob byte layout is the one the library's public header documents:
  * four regions (gate/up codes, down codes, gate/up scales, down scales), each
  * starting at a multiple of 256 bytes; codes stored in 16-byte pieces
- * [row-block][piece][row][16 bytes] with 256-row gate/up blocks (128 gate rows
- * then the 128 matching up rows) and 128-row down blocks; scales stored
- * [row-block][group][row] (fp16) or [row-block][row] (fp32). */
+ * [row-block][piece][row][16 bytes] with 128-row gate/up blocks (64 gate rows
+ * then the 64 matching up rows), scales [row-block][group][row] (fp16) or
+ * [row-block][row] (fp32); the down matrix is cut along I into slabs of 64
+ * intermediate indices, each slab [128-row block][piece][row][16 bytes] with
+ * fp16 scales [slab][128-row block][2 groups][row], fp32 scales [expert][row]. */
 
 static uint64_t al256(uint64_t v) { return (v + 255) & ~(uint64_t)255; }
 
@@ -203,34 +205,42 @@ int orc_pack_blob(int E, int H, int I, int wbits, int g32, const int8_t* q_gu, c
   uint8_t* rb = (uint8_t*)malloc(kb_gu > kb_dn ? kb_gu : kb_dn);
   for (int e = 0; e < E; ++e) {
     /* gate/up */
-    for (int sb = 0; sb < I / 128; ++sb)
-      for (int r = 0; r < 256; ++r) {
-        int64_t lr = r < 128 ? 128 * sb + r : (int64_t)I + 128 * sb + (r - 128);
+    for (int sb = 0; sb < I / 64; ++sb)
+      for (int r = 0; r < 128; ++r) {
+        int64_t lr = r < 64 ? 64 * sb + r : (int64_t)I + 64 * sb + (r - 64);
         int64_t grow = (int64_t)e * 2 * I + lr;
         row_bytes(q_gu + grow * H, H, wbits, rb);
-        put_row(blob + off[0] + (uint64_t)e * 2 * I * kb_gu, 256, kb_gu, sb, r, rb);
+        put_row(blob + off[0] + (uint64_t)e * 2 * I * kb_gu, 128, kb_gu, sb, r, rb);
         if (g32) {
-          uint16_t* sr = (uint16_t*)(blob + off[2] + ((uint64_t)e * 2 * I + (uint64_t)sb * 256) * Gg * 2);
-          for (int g = 0; g < Gg; ++g) sr[g * 256 + r] = f16_bits(s_gu[grow * Gg + g]);
+          uint16_t* sr = (uint16_t*)(blob + off[2] + ((uint64_t)e * 2 * I + (uint64_t)sb * 128) * Gg * 2);
+          for (int g = 0; g < Gg; ++g) sr[g * 128 + r] = f16_bits(s_gu[grow * Gg + g]);
         } else {
-          float* sr = (float*)(blob + off[2] + ((uint64_t)e * 2 * I + (uint64_t)sb * 256) * 4);
+          float* sr = (float*)(blob + off[2] + ((uint64_t)e * 2 * I + (uint64_t)sb * 128) * 4);
           sr[r] = s_gu[grow];
         }
       }
-    /* down */
-    for (int sb = 0; sb < H / 128; ++sb)
-      for (int r = 0; r < 128; ++r) {
-        int64_t grow = (int64_t)e * H + 128 * sb + r;
+    /* down: slab (e, u) = all H rows x intermediate indices 64u .. 64u+63, stored as
+       128-row blocks [hb][piece][row][16 bytes]; g32 scales [slab][hb][2][row] */
+    {
+      const int U = I / 64, HB = H / 128;
+      const uint64_t sbytes = kb_dn / U;     /* code bytes of 64 elements: 64 or 32 */
+      for (int n = 0; n < H; ++n) {
+        int64_t grow = (int64_t)e * H + n;
+        int hb = n / 128, r = n % 128;
         row_bytes(q_dn + grow * I, I, wbits, rb);
-        put_row(blob + off[1] + (uint64_t)e * H * kb_dn, 128, kb_dn, sb, r, rb);
-        if (g32) {
-          uint16_t* sr = (uint16_t*)(blob + off[3] + ((uint64_t)e * H + (uint64_t)sb * 128) * Gd * 2);
-          for (int g = 0; g < Gd; ++g) sr[g * 128 + r] = f16_bits(s_dn[grow * Gd + g]);
-        } else {
-          float* sr = (float*)(blob + off[3] + ((uint64_t)e * H + (uint64_t)sb * 128) * 4);
-          sr[r] = s_dn[grow];
+        for (int u = 0; u < U; ++u) {
+          uint64_t slab = ((uint64_t)e * U + u) * HB + hb;
+          uint8_t* base = blob + off[1] + slab * 128 * sbytes;
+          for (uint64_t bb = 0; bb < sbytes; ++bb)
+            base[(bb / 16) * 128 * 16 + (uint64_t)r * 16 + bb % 16] = rb[u * sbytes + bb];
+          if (g32) {
+            uint16_t* sr = (uint16_t*)(blob + off[3] + slab * 2 * 128 * 2);
+            for (int j = 0; j < 2; ++j) sr[j * 128 + r] = f16_bits(s_dn[grow * Gd + 2 * u + j]);
+          }
         }
+        if (!g32) ((float*)(blob + off[3]))[grow] = s_dn[grow];
       }
+    }
   }
   free(rb);
   return 0;

@@ -73,7 +73,7 @@ moe_status check_cfg(const moe_route_cfg* c, int32_t E) {
 
 // Workspace of one layer forward: every region starts at a multiple of 256 bytes.
 struct Layout {
-  int64_t status, qx, sx, logits, idx, w, offsets, perm, n_active, act_expert, act_begin;
+  int64_t status, qx, sx, logits, idx, w, offsets, perm, n_active, act_expert, act_begin, act_rows;
   int64_t masks, base, qh, sh, hbuf, dbg_gate, dbg_up, dbg_y, total;
   int64_t qh_sh, sh_sh, hbuf_sh, dbg_gate_sh, dbg_up_sh, dbg_y_sh;   // shared-expert rows
 };
@@ -100,6 +100,7 @@ Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k,
   L.n_active = take(4);
   L.act_expert = take((int64_t)(E + 1) * 4);
   L.act_begin = take((int64_t)(E + 2) * 4);
+  L.act_rows = take((int64_t)E * 8 * 4);
   L.masks = take(T > 1 ? C * E * 4 : 0);
   L.base = take(T > 1 ? C * E * 4 : 0);
   const int64_t rows_h = P * I + (int64_t)T * Is;
@@ -273,7 +274,7 @@ moe_status moe_permute(const int32_t* idx, int32_t T, int32_t k, int32_t E, int3
   o += al256(C * E * 4);
   int32_t* base = reinterpret_cast<int32_t*>(ws + o);
   o += al256(C * E * 4);
-  moe::Grouping g;
+  moe::Grouping g{};
   g.offsets = offsets;
   g.perm = perm;
   g.n_active = reinterpret_cast<int32_t*>(ws + o);
@@ -380,12 +381,13 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   int* status = static_cast<int*>(at(L.status));
   const BlobView bv = view(experts, p.eo);
 
-  moe::Grouping g;
+  moe::Grouping g{};
   g.offsets = static_cast<int32_t*>(at(L.offsets));
   g.perm = static_cast<int32_t*>(at(L.perm));
   g.n_active = static_cast<int32_t*>(at(L.n_active));
   g.act_expert = static_cast<int32_t*>(at(L.act_expert));
   g.act_begin = static_cast<int32_t*>(at(L.act_begin));
+  g.act_rows = static_cast<int32_t*>(at(L.act_rows));
   int32_t* idx = static_cast<int32_t*>(at(L.idx));
   float* wts = static_cast<float*>(at(L.w));
   float* logits = static_cast<float*>(at(L.logits));
@@ -461,6 +463,7 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   ra.act_expert = g.act_expert;
   ra.act_begin = g.act_begin;
   ra.perm = g.perm;
+  ra.act_rows = g.act_rows;
   ra.wts = wts;
   ra.T = T;
   ra.k = k;
@@ -481,6 +484,7 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     sa.act_expert = nullptr;
     sa.act_begin = nullptr;
     sa.perm = nullptr;
+    sa.act_rows = nullptr;
     sa.max_active = 1;
     sa.qh = static_cast<int8_t*>(at(L.qh_sh));
     sa.sh = static_cast<__half*>(at(L.sh_sh));
@@ -488,20 +492,6 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     sa.dbg_a = static_cast<float*>(at(L.dbg_gate_sh));
     sa.dbg_b = static_cast<float*>(at(L.dbg_up_sh));
   }
-  mk.begin(MOE_STAGE_GATE_UP);
-  keep(moe::launch_gateup_tma(ra, shared ? &sa : nullptr, st), "gate/up kernel");
-  mk.end(MOE_STAGE_GATE_UP);
-  mk.begin(MOE_STAGE_QUANT_H);
-  if (!ag32) {
-    moe::launch_quantize_rows_token(static_cast<const float*>(at(L.hbuf)), T * k, I,
-                                    static_cast<int8_t*>(at(L.qh)), static_cast<float*>(at(L.sh)), st);
-    if (shared)
-      moe::launch_quantize_rows_token(static_cast<const float*>(at(L.hbuf_sh)), T, p.Is,
-                                      static_cast<int8_t*>(at(L.qh_sh)),
-                                      static_cast<float*>(at(L.sh_sh)), st);
-  }
-  mk.end(MOE_STAGE_QUANT_H);
-
   // 5. down projection + weighted combine into y; routed and shared experts in one grid
   moe::ExpertArgs rd = ra;
   rd.qa = static_cast<const int8_t*>(at(L.qh));
@@ -515,9 +505,39 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     sd.dbg_a = static_cast<float*>(at(L.dbg_y_sh));
     sd.dbg_b = nullptr;
   }
-  mk.begin(MOE_STAGE_DOWN);
-  keep(moe::launch_down_tma(rd, shared ? &sd : nullptr, st), "down kernel");
-  mk.end(MOE_STAGE_DOWN);
+  const moe::ExpertArgs* sap = shared ? &sa : nullptr;
+  const moe::ExpertArgs* sdp = shared ? &sd : nullptr;
+  // the down kernels add each unit's share of a pair's down value into the pair's view
+  if (L.dbg_y >= 0)
+    keep(cudaMemsetAsync(ws + L.dbg_y, 0, (size_t)((int64_t)(T * k + T) * H * 4), st), "debug view reset");
+  if (moe::experts_fusable(ra, sap)) {
+    // 4+5 in one persistent grid: per unit (expert, 64 intermediate indices) the gate/up
+    // pass, SwiGLU and h quantization, then the unit's share of the down projection
+    mk.begin(MOE_STAGE_GATE_UP);
+    keep(moe::launch_experts(2, ra, sap, rd, sdp, st), "expert kernel");
+    mk.end(MOE_STAGE_GATE_UP);
+    for (int sg = MOE_STAGE_QUANT_H; sg <= MOE_STAGE_DOWN; ++sg) {
+      mk.begin(sg);
+      mk.end(sg);
+    }
+  } else {
+    mk.begin(MOE_STAGE_GATE_UP);
+    keep(moe::launch_experts(0, ra, sap, rd, sdp, st), "gate/up kernel");
+    mk.end(MOE_STAGE_GATE_UP);
+    mk.begin(MOE_STAGE_QUANT_H);
+    if (!ag32) {
+      moe::launch_quantize_rows_token(static_cast<const float*>(at(L.hbuf)), T * k, I,
+                                      static_cast<int8_t*>(at(L.qh)), static_cast<float*>(at(L.sh)), st);
+      if (shared)
+        moe::launch_quantize_rows_token(static_cast<const float*>(at(L.hbuf_sh)), T, p.Is,
+                                        static_cast<int8_t*>(at(L.qh_sh)),
+                                        static_cast<float*>(at(L.sh_sh)), st);
+    }
+    mk.end(MOE_STAGE_QUANT_H);
+    mk.begin(MOE_STAGE_DOWN);
+    keep(moe::launch_experts(1, ra, sap, rd, sdp, st), "down kernel");
+    mk.end(MOE_STAGE_DOWN);
+  }
   if (err != cudaSuccess) return cuda_fail(err_where, err);
   if (mk.err != cudaSuccess) return cuda_fail("stage event record", mk.err);
   return launch_status();
@@ -549,6 +569,7 @@ int32_t moe_layer_kernel_count(int32_t T, const moe_expert_blob* experts,
   if (moe_layer_workspace_bytes(T, experts, shared, cfg) == 0) return -1;
   if (T == 0) return 0;
   int n = T <= kFusedRouteMaxT ? 1 : 4;        // routing (fused, or quantize/logits/top-k/grouping)
+  if (cfg->act == MOE_ACT_G32_F16) return n + 1;   // gate/up and down of all experts in one grid
   n += 1;                                       // gate/up, routed and shared experts in one grid
   if (cfg->act != MOE_ACT_G32_F16) n += 1 + (shared ? 1 : 0);   // h quantization
   n += 1;                                       // down, routed and shared experts in one grid

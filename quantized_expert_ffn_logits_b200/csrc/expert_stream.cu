@@ -5,17 +5,28 @@
 // "Quantization kernels: ... dequant-on-use"; "Batch-union MoE": every selected expert's
 // weights are streamed once per call, whatever the number of tokens routed to it).
 //
-// Memory design. In the blob the rows of one 16-byte piece are contiguous, so a warp whose
-// lanes own 32 consecutive rows reads 512 contiguous bytes per 128-bit load. A CTA splits
-// its 64 rows' K range over four warps per 32 rows; at start every warp prefetches its whole
-// range into L2 (one prefetch per 512-byte run), so HBM streams the unit at full rate while
-// the warp consumes it in batches of 16 register loads per lane. The exact int32 group dots
-// are parked in shared memory and the ordered fp32 chain of each row runs once all of its
-// groups are in. (Measured on this part: plain streaming loads reach 7.2 TB/s; bulk copies
-// of 512-byte runs stay below 2 TB/s, and a multistage cp.async ring spent more
-// instructions on bookkeeping than it saved.)
+// Work unit = one selected expert x one 128-row block of the blob: gate/up blocks hold 64
+// gate rows and the 64 matching up rows, down blocks 128 output rows. A block's whole K
+// range is one contiguous run in the blob ([piece][128 rows][16 B], 2 KB per piece), so it
+// streams as a handful of large bulk copies. Grid = one persistent CTA per SM (at most
+// one per unit), units taken round-robin; a unit with more tokens than fit one pass is
+// streamed once per pass.
+//
+// CTA = one producer warp + eight consumer warps. The producer's lane 0 walks the CTA's
+// passes and pushes 32 KB chunks (16 pieces) plus the matching group scales into a
+// four-stage shared-memory ring with cp.async.bulk ("full" mbarrier per stage, released
+// on an "empty" mbarrier), and the pass's activation rows into one of two activation
+// buffers right behind the pass's first chunk, so they arrive in stream order instead of
+// queueing behind the weights. A consumer thread owns one row of the block for a set of
+// tokens: per chunk it loads all 16 pieces of its row, forms every group's exact int32 dot
+// (independent dp4a chains) and then runs the ordered fp32 chain over the chunk's groups,
+// acc = fma((float)I_g, c_g, acc) -- groups arrive in ascending order, so nothing is
+// parked. Up to four chunks (128 KB) per SM are in flight. Every wait is bounded: a wait
+// that gives up sets the status word, the consumers skip the rest of their work but keep
+// releasing stages (all warps take the same barriers), and the producer drains its copies
+// before the CTA exits.
+#include <algorithm>
 #include <cstring>
-#include <mutex>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -23,488 +34,794 @@
 
 namespace moe {
 
-constexpr int TMT = 4;   // most token slots per pass over the weights
-constexpr int NQ = 4;    // warps per 32-row group, each one quarter of the groups along K
-constexpr int NT = 32 * 2 * NQ;         // threads per CTA
+constexpr int kRows = 128;                 // rows per unit
+constexpr int kPiece = kRows * 16;         // bytes of one 16-byte column of the unit: 2 KB
+constexpr int kSP = 16;                    // pieces per ring stage (32 KB)
+constexpr int kNS = 4;                     // ring stages
+constexpr int kCW = 8;                     // consumer warps
+constexpr int kNT = 32 * (kCW + 1);        // + the producer warp
+constexpr int kTMP = 8;                    // most tokens per pass over a unit's weights
+constexpr int kSmemMax = 227 * 1024;
 
-// Shared-memory layout of one CTA (64 rows; base aligned to 1024 bytes).
-struct SmemPlan {
-  int xs, sx, xsum, idot, sw, ubuf, rows, total;
+// Shared-memory plan (offsets from a 1024-aligned base). Activation buffer b holds tm rows
+// of K codes, then (g32 activations) tm rows of G fp16 scales.
+struct RingPlan {
+  int ring, sring, bars, abuf, abytes, ascale, xsum, sxf, idot, ubuf, hq, info, total;
 };
 
-__host__ __device__ inline SmemPlan smem_plan(int K, int tm, int wg32) {
-  SmemPlan p;
+__host__ __device__ inline RingPlan ring_plan(int K, int tm) {
+  RingPlan p;
   const int G = K / 32;
   int o = 0;
-  p.xs = o;
-  o += tm * K;
-  p.sx = o;
-  o += tm * G * 4;
-  p.xsum = o;
-  o += tm * G * 4;
-  p.idot = o;
-  o += tm * G * 64 * 4;
-  p.sw = o;
-  o += wg32 ? G * 64 * 4 : 0;
-  p.ubuf = o;
-  o += tm * 32 * 4;
-  p.rows = o;
-  o += 4 * TMT * 4;
-  p.total = o + 1024;   // slack for aligning the base to 1024 bytes
+  // every region starts on a 128-byte boundary (128-bit and bulk-copy accesses)
+  auto take = [&](int bytes) {
+    const int at = o;
+    o = (o + bytes + 127) & ~127;
+    return at;
+  };
+  p.ring = take(kNS * kSP * kPiece);            // 128 KB
+  p.sring = take(kNS * kSP * 128 * 2);          // group / row scales of a stage
+  p.bars = take((2 * kNS + 4) * 8);
+  p.ascale = tm * K;                            // offset of the scales inside a buffer
+  p.abytes = (tm * K + tm * G * 2 + 127) & ~127;
+  p.abuf = take(2 * p.abytes);
+  p.xsum = take(2 * tm * G * 4);
+  p.sxf = take(tm * G * 4);                     // scales not copied by the producer, as fp32
+  p.idot = take(2 * 8 * tm * kRows * 4);        // int32 dots of a block of 8 groups, two buffers
+  p.ubuf = take(2 * tm * 64 * 4);               // gate / up stage values of a pass
+  p.hq = take(2 * tm * 64 + 2 * tm * 4 + 2 * tm * 4);   // h codes (+ de-interleaved), scales, sums
+  p.info = take(3 * kTMP * 4 + 16);             // tokens, weights, abort flag
+  p.total = o + 1024;                           // slack for aligning the base
   return p;
 }
 
-// Token slots per pass: up to TMT, as many as the int32 dot buffer budget allows.
-__host__ __device__ inline int pass_tokens(int K, int max_tokens) {
-  const int G = K / 32;
-  int tm = (32 * 1024) / (G * 64 * 4);
-  tm = tm < 1 ? 1 : (tm > TMT ? TMT : tm);
-  return max_tokens < tm ? (max_tokens < 1 ? 1 : max_tokens) : tm;
+// Tokens per pass: up to kTMP, as many as shared memory allows.
+inline int ring_tokens(int K, int max_tokens) {
+  int tm = max_tokens < 1 ? 1 : (max_tokens > kTMP ? kTMP : max_tokens);
+  while (tm > 1 && ring_plan(K, tm).total > kSmemMax) --tm;
+  return tm;
 }
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-// Activation rows of up to tm slots into shared memory (int4 weights: each 8-byte word
-// de-interleaved into even / odd elements, plus per-group sums). Threads [0, nthr).
-template <int WBITS, bool AG32>
-__device__ __forceinline__ void load_acts(const int8_t* __restrict__ qa, const void* sa, int K, int m,
-                                          const int* rows, uint8_t* xs, float* sx, int* xsum,
-                                          int tid, int nthr) {
-  const int G = K / 32;
-  const int words = K / 8;
-  for (int l = tid; l < m * words; l += nthr) {
-    const int tt = l / words, wi = l - tt * words;
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(qa + (int64_t)rows[tt] * K) + wi);
-    uint2 o = v;
-    if (WBITS == 4) deinterleave8(v.x, v.y, o.x, o.y);
-    reinterpret_cast<uint2*>(xs + tt * K)[wi] = o;
-  }
-  for (int l = tid; l < m * G; l += nthr) {
-    const int tt = l / G, g = l - tt * G;
-    if (AG32) sx[tt * G + g] = __half2float(reinterpret_cast<const __half*>(sa)[(int64_t)rows[tt] * G + g]);
-    else if (g == 0) sx[tt] = reinterpret_cast<const float*>(sa)[rows[tt]];
-    if (WBITS == 4) {
-      const uint4* p = reinterpret_cast<const uint4*>(qa + (int64_t)rows[tt] * K + 32 * g);
-      const uint4 a = __ldg(p), b = __ldg(p + 1);
-      int s = __dp4a((int)a.x, 0x01010101, 0);
-      s = __dp4a((int)a.y, 0x01010101, s);
-      s = __dp4a((int)a.z, 0x01010101, s);
-      s = __dp4a((int)a.w, 0x01010101, s);
-      s = __dp4a((int)b.x, 0x01010101, s);
-      s = __dp4a((int)b.y, 0x01010101, s);
-      s = __dp4a((int)b.z, 0x01010101, s);
-      s = __dp4a((int)b.w, 0x01010101, s);
-      xsum[tt * G + g] = s;
-    }
-  }
-}
-
-// The canonical fp32 chain of one row over all groups: acc = fma((float)I_g, c_g, acc) for
-// ascending g from +0, then the per-row / per-token scale.
-template <bool WG32, bool AG32>
-__device__ __forceinline__ float row_chain(const int* idot_t, const float* sw, const float* sx_t, int G,
-                                           int row, float sx_tok, float sw_row) {
-  if (!WG32 && !AG32) {
-    int isum = 0;
-    for (int g = 0; g < G; ++g) isum += idot_t[g * 64 + row];
-    return __fmul_rn(__fmaf_rn(__int2float_rn(isum), sx_tok, 0.0f), sw_row);
-  }
-  float acc = 0.0f;
-  int g = 0;
-  for (; g + 8 <= G; g += 8) {
-    int d[8];
-    float c[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      d[q] = idot_t[(g + q) * 64 + row];
-      if (WG32 && AG32) c[q] = __fmul_rn(sw[(g + q) * 64 + row], sx_t[g + q]);
-      else if (WG32) c[q] = sw[(g + q) * 64 + row];
-      else c[q] = sx_t[g + q];
-    }
-#pragma unroll
-    for (int q = 0; q < 8; ++q) acc = __fmaf_rn(__int2float_rn(d[q]), c[q], acc);
-  }
-  for (; g < G; ++g) {
-    float c;
-    if (WG32 && AG32) c = __fmul_rn(sw[g * 64 + row], sx_t[g]);
-    else if (WG32) c = sw[g * 64 + row];
-    else c = sx_t[g];
-    acc = __fmaf_rn(__int2float_rn(idot_t[g * 64 + row]), c, acc);
-  }
-  if (WG32 && AG32) return acc;
-  if (WG32) return __fmul_rn(acc, sx_tok);
-  return __fmul_rn(acc, sw_row);
-}
+// One work unit as the kernel sees it.
+struct Unit {
+  bool shd;      // the shared expert
+  int ai;        // active-expert index (routed)
+  int e;         // expert
+  int s0, s1;    // slots [s0, s1) routed to it (shared: all tokens)
+  int sub;       // row block inside the expert
+  int rows8[8];  // tokens of slots s0 .. s0+7 (routed gate/up)
+};
 
 // Resolve grid work unit u (routed units first, then the shared expert's); false if idle.
+// Routing data is read through L2 (written by an earlier kernel of the same stream); every
+// load is issued before any is used, so resolving a unit costs one L2 round trip.
 __device__ __forceinline__ bool unit_of(const ExpertArgs& r, const ExpertArgs& s, int has_shared,
-                                        int routed_units, int per_expert_r, int u, bool& shared,
-                                        int& e, int& s0, int& s1, int& sub) {
+                                        int routed_units, int per_expert_r, int u, Unit& U,
+                                        bool want_rows, bool report) {
   if (u < routed_units) {
-    shared = false;
-    const int ai = u / per_expert_r;
-    sub = u - ai * per_expert_r;
-    const int na = *r.n_active;
-    if (ai >= na) return false;
-    e = r.act_expert[ai];
-    s0 = r.act_begin[ai];
-    s1 = r.act_begin[ai + 1];
-    if (e < 0 || e >= r.b.E || s0 < 0 || s0 > s1 || s1 > r.T * r.k) {
-      if (threadIdx.x == 0) set_status(r.status, kStatusDeviceCheck);
+    U.shd = false;
+    U.ai = u / per_expert_r;
+    U.sub = u - U.ai * per_expert_r;
+    const int na = __ldcg(r.n_active);
+    U.e = __ldcg(r.act_expert + U.ai);
+    U.s0 = __ldcg(r.act_begin + U.ai);
+    U.s1 = __ldcg(r.act_begin + U.ai + 1);
+    if (want_rows) {
+      const int4 lo = __ldcg(reinterpret_cast<const int4*>(r.act_rows) + 2 * U.ai);
+      const int4 hi = __ldcg(reinterpret_cast<const int4*>(r.act_rows) + 2 * U.ai + 1);
+      U.rows8[0] = lo.x;
+      U.rows8[1] = lo.y;
+      U.rows8[2] = lo.z;
+      U.rows8[3] = lo.w;
+      U.rows8[4] = hi.x;
+      U.rows8[5] = hi.y;
+      U.rows8[6] = hi.z;
+      U.rows8[7] = hi.w;
+    }
+    if (U.ai >= na) return false;
+    if (U.e < 0 || U.e >= r.b.E || U.s0 < 0 || U.s0 > U.s1 || U.s1 > r.T * r.k) {
+      if (report) set_status(r.status, kStatusDeviceCheck);
       return false;
     }
     return true;
   }
   if (!has_shared) return false;
-  shared = true;
-  e = 0;
-  s0 = 0;
-  s1 = s.T;
-  sub = u - routed_units;
+  U.shd = true;
+  U.ai = 0;
+  U.e = 0;
+  U.s0 = 0;
+  U.s1 = s.T;
+  U.sub = u - routed_units;
   return true;
 }
 
-// Up to GB groups of a lane's row from global memory (16-byte pieces; piece p at
-// wrow + p * PSTRIDE, group scales at srow[g * SSTRIDE]) -> exact int32 dots against the
-// staged token rows, into idot[(tt * G + g) * 64 + row]; scales into sw[g * 64 + row].
-// Strides are compile-time so every load uses an immediate offset; full batches with one
-// token (the decode case) take a straight-line path.
-template <int WBITS, bool WG32, int PSTRIDE, int SSTRIDE>
-struct Batch {
-  static constexpr int PPG = WBITS == 8 ? 2 : 1;
-  static constexpr int GB = WBITS == 8 ? 8 : 16;     // 16 pieces = 16 loads in flight per lane
-  uint4 w[PPG * GB];
-  float sc[GB];
-
-  __device__ __forceinline__ void load(const uint8_t* __restrict__ wrow, const __half* __restrict__ srow,
-                                       int g0, int nb) {
-    const uint8_t* wp = wrow + (int64_t)g0 * PPG * PSTRIDE;
-    const __half* sp = srow + (int64_t)g0 * SSTRIDE;
-    if (nb == GB) {
+// Activation row of slot `slot`: gate/up reads the token's q_x row, down the slot's q_h
+// row. Tokens of a routed unit's first 8 slots come with the unit; later ones from the
+// pair list. A corrupt token or pair index is reported and read as row 0.
+__device__ __forceinline__ int act_row(const ExpertArgs& a, bool gateup, const Unit& U, int slot) {
+  if (!gateup || U.shd) return slot;
+  const int j = slot - U.s0;
+  int t;
+  if (j < 8) {
+    t = U.rows8[0];
 #pragma unroll
-      for (int p = 0; p < PPG * GB; ++p) w[p] = ldg_stream(reinterpret_cast<const uint4*>(wp + p * PSTRIDE));
-      if (WG32) {
-#pragma unroll
-        for (int u = 0; u < GB; ++u) sc[u] = __half2float(sp[u * SSTRIDE]);
-      }
-    } else {
-#pragma unroll
-      for (int p = 0; p < PPG * GB; ++p)
-        if (p < PPG * nb) w[p] = ldg_stream(reinterpret_cast<const uint4*>(wp + p * PSTRIDE));
-      if (WG32) {
-#pragma unroll
-        for (int u = 0; u < GB; ++u)
-          if (u < nb) sc[u] = __half2float(sp[u * SSTRIDE]);
-      }
-    }
+    for (int q = 1; q < 8; ++q)
+      if (j == q) t = U.rows8[q];
+  } else {
+    const int p = __ldcg(a.perm + slot);
+    t = (p >= 0 && p < a.T * a.k) ? p / a.k : -1;
   }
-
-  __device__ __forceinline__ int dot1(int u, const uint8_t* xg, int xs_sum) const {
-    const uint4 x0 = *reinterpret_cast<const uint4*>(xg);
-    const uint4 x1 = *reinterpret_cast<const uint4*>(xg + 16);
-    if (WBITS == 8) return group_dot_i8(w[2 * u], w[2 * u + 1], x0, x1);
-    return group_dot_i4(w[u], make_uint4(x0.x, x0.z, x1.x, x1.z), make_uint4(x0.y, x0.w, x1.y, x1.w), xs_sum);
+  if (t < 0 || t >= a.T) {
+    set_status(a.status, kStatusDeviceCheck);
+    return 0;
   }
+  return t;
+}
 
-  __device__ __forceinline__ void dots(int g0, int nb, int K, int m, int row, const uint8_t* xs,
-                                       const int* xsum, int* idot, float* sw) const {
-    const int G = K / 32;
-    if (nb == GB && m == 1) {
-      const uint8_t* xg = xs + 32 * g0;
-      int* id = idot + g0 * 64 + row;
-      const int* xsm = xsum + g0;
-#pragma unroll
-      for (int u = 0; u < GB; ++u) id[u * 64] = dot1(u, xg + 32 * u, WBITS == 4 ? xsm[u] : 0);
-      if (WG32) {
-#pragma unroll
-        for (int u = 0; u < GB; ++u) sw[(g0 + u) * 64 + row] = sc[u];
-      }
-      return;
-    }
-    if (WG32) {
-#pragma unroll
-      for (int u = 0; u < GB; ++u)
-        if (u < nb) sw[(g0 + u) * 64 + row] = sc[u];
-    }
-    for (int tt = 0; tt < m; ++tt) {
-      const uint8_t* xg = xs + tt * K + 32 * g0;
-      int* id = idot + (tt * G + g0) * 64 + row;
-      const int* xsm = xsum + tt * G + g0;
-#pragma unroll
-      for (int u = 0; u < GB; ++u)
-        if (u < nb) id[u * 64] = dot1(u, xg + 32 * u, WBITS == 4 ? xsm[u] : 0);
-    }
+// Record the first wait that gave up: word 2 = kernel | role << 4 | stage << 8, word 3 = CTA.
+__device__ __forceinline__ void wait_failed(int* status, int kernel, int role, int stage) {
+  if (!status) return;
+  if (atomicCAS(status, 0, kStatusTimeout) == 0) {
+    status[2] = kernel | (role << 4) | (stage << 8);
+    status[3] = (int)blockIdx.x;
   }
+}
+
+struct Ring {
+  uint8_t* ring;
+  uint8_t* sring;
+  uint64_t* full;     // [kNS]
+  uint64_t* empty;    // [kNS]
+  uint64_t* afull;    // [2]
+  uint64_t* aempty;   // [2]
+  uint8_t* abuf;      // [2][abytes]
+  int* xsum;          // [2][tm][G]
+  float* sxf;         // [tm][G] (or [tm] per-token scales)
 };
 
-// L2 prefetch of a lane's pieces [p0, p1) (one instruction per piece covers the warp's 512
-// contiguous bytes) and, for group-32 scales, groups [g0, g1).
-template <int WBITS, bool WG32>
-__device__ __forceinline__ void prefetch_rows(const uint8_t* wrow, int pstride, const __half* srow,
-                                              int sstride, int g0, int g1) {
+// Launch arguments. x[0][*] = gate/up (q_x activations, writes h), x[1][*] = down (reads h,
+// adds into y); [*][0] routed experts, [*][1] the shared expert. Units are (expert,
+// 64 intermediate indices) in every mode: MODE 0 runs the gate/up pass of each unit,
+// MODE 1 its down pass (h from an earlier kernel), MODE 2 both, h staying on chip.
+struct RingArgs {
+  ExpertArgs x[2][2];
+  int has_shared;
+  int units;               // routed units first, then the shared expert's
+  int routed;              // routed units
+  int per;                 // units per routed expert (I / 64)
+  int tm, kmax;
+};
+
+// ------------------------------------------------------------------ producer
+// Lane 0 of the producer warp: every chunk of every pass of every unit of this CTA, in the
+// order the consumers take them. Gate/up pass: the unit's 128 rows over K = H (codes at
+// gu_w + blk * KB, fp16 group scales at gu_s + blk * G * 2, blk = first row of the block),
+// with the pass's activation rows right after the first chunk. Down pass: the unit's slab
+// (all H rows x its 64 columns) in chunks of whole 128-row blocks, with their scales
+// (fp16 [block][2][128] or fp32 per row).
+template <int WBITS, bool WG32, bool AG32, int MODE>
+__device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& R) {
   constexpr int PPG = WBITS == 8 ? 2 : 1;
-  for (int p = g0 * PPG; p < g1 * PPG; ++p) prefetch_l2(wrow + (int64_t)p * pstride);
-  if (WG32)
-    for (int g = g0; g < g1; ++g) prefetch_l2(srow + (int64_t)g * sstride);
-}
-
-// ------------------------------------------------------------------ gate / up
-// CTA = one work unit: one selected expert x 32 intermediate indices = 32 gate rows + the
-// matching 32 up rows (routed units first, then the shared expert's). Eight warps: warps
-// 0..NQ-1 own the gate rows, NQ..2NQ-1 the up rows (one row per lane), warp quarter q takes
-// the q-th quarter of the groups along K. As soon as the unit is known every warp asks L2
-// for its whole K range (and for this unit's 1/(I/32) share of the expert's down
-// projection, which the next kernel reads), then keeps 16 register loads per lane in flight
-// batch by batch; the token rows are staged meanwhile. One warp per (half, token) then runs
-// the ordered row chains, and the gate warps apply SwiGLU and quantize h.
-template <int WBITS, bool WG32, bool AG32>
-__global__ void __launch_bounds__(NT, 2)
-    k_gateup_rows(const __grid_constant__ ExpertArgs ra, const __grid_constant__ ExpertArgs sa,
-                  int has_shared, int routed_units, int tm) {
-  using B = Batch<WBITS, WG32, 256 * 16, 256>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = align1024(smem_raw);
-  const int K = ra.b.H, G = K / 32, KB = kbytes(K, WBITS);
-  const SmemPlan P = smem_plan(K, tm, WG32);
-  uint8_t* xs = base + P.xs;
-  float* sx = reinterpret_cast<float*>(base + P.sx);
-  int* xsum = reinterpret_cast<int*>(base + P.xsum);
-  int* idot = reinterpret_cast<int*>(base + P.idot);
-  float* swb = reinterpret_cast<float*>(base + P.sw);
-  float* ubuf = reinterpret_cast<float*>(base + P.ubuf);
-  int* rows = reinterpret_cast<int*>(base + P.rows);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  pdl_wait();
-  pdl_trigger();
-  bool shd;
-  int e, s0, s1, ib;
-  if (!unit_of(ra, sa, has_shared, routed_units, ra.b.I / 32, blockIdx.x, shd, e, s0, s1, ib)) return;
-  const ExpertArgs& a = shd ? sa : ra;
-  const int I = a.b.I, IB = I / 32;
-  const int64_t blk = (int64_t)e * 2 * I + (int64_t)(ib >> 2) * 256;     // first row of the block
-  const int r_gate = (ib & 3) * 32;
-  const int half = warp / NQ, q = warp % NQ;
-  const int row = half * 32 + lane;
-  const int i = ib * 32 + lane;
-  const uint8_t* wrow = a.b.gu_w + blk * KB + (int64_t)(half * 128 + r_gate + lane) * 16;
-  const __half* srow = reinterpret_cast<const __half*>(a.b.gu_s) + blk * G + half * 128 + r_gate + lane;
-  const int GQ = G / NQ, gq0 = q * GQ;
-
-  // ask L2 for everything this warp will read, then for the down slice of this expert
-  prefetch_rows<WBITS, WG32>(wrow, 256 * 16, srow, 256, gq0 + B::GB, gq0 + GQ);
-  {
-    const int64_t dn_bytes = (int64_t)a.b.H * kbytes(I, WBITS);
-    const int64_t per = dn_bytes / IB;
-    const uint8_t* d0 = a.b.dn_w + (int64_t)e * dn_bytes + (int64_t)ib * per;
-    for (int64_t o = (int64_t)threadIdx.x * 128; o < per; o += (int64_t)NT * 128) prefetch_l2(d0 + o);
-    if (WG32) {
-      const int64_t ds_bytes = (int64_t)a.b.H * (I / 32) * 2;
-      const int64_t sper = ds_bytes / IB;
-      const uint8_t* s0p = a.b.dn_s + (int64_t)e * ds_bytes + (int64_t)ib * sper;
-      for (int64_t o = (int64_t)threadIdx.x * 128; o < sper; o += (int64_t)NT * 128) prefetch_l2(s0p + o);
+  constexpr int PPU = WBITS == 8 ? 4 : 2;   // pieces of a row's 64-column down slice
+  constexpr int NBC = kSP / PPU;            // 128-row down blocks per chunk
+  constexpr int kern = MODE == 1 ? 2 : 1;
+  int* status = A.x[0][0].status;
+  uint32_t c = 0, pidx = 0, nacts = 0;      // chunks, passes, activation copies issued
+  bool ok = true;
+  auto push = [&](const uint8_t* w, uint32_t wbytes, const uint8_t* sc, uint32_t sbytes) -> bool {
+    const int st = c % kNS;
+    if (c >= (uint32_t)kNS && !mbar_wait(&R.empty[st], ((c / kNS) - 1) & 1)) {
+      wait_failed(status, kern, 0, st);
+      return false;
     }
-  }
-
-  for (int c0 = s0; c0 < s1; c0 += tm) {
-    const int m = min(tm, s1 - c0);
-    B bt;
-    bt.load(wrow, srow, gq0, min(B::GB, GQ));      // first batch in flight
-    if (threadIdx.x < m) {
-      const int slot = c0 + threadIdx.x;
-      int r = slot;
-      if (!shd) {
-        const int p = a.perm[slot];
-        const bool okp = p >= 0 && p < a.T * a.k;
-        if (!okp) set_status(a.status, kStatusDeviceCheck);
-        r = okp ? p / a.k : 0;
-      }
-      rows[threadIdx.x] = r;
-    }
-    __syncthreads();
-    load_acts<WBITS, AG32>(a.qa, a.sa, K, m, rows, xs, sx, xsum, threadIdx.x, NT);
-    __syncthreads();
-    for (int g0 = gq0; g0 < gq0 + GQ; g0 += B::GB) {
-      const int nb = min(B::GB, gq0 + GQ - g0);
-      if (g0 != gq0) bt.load(wrow, srow, g0, nb);
-      bt.dots(g0, nb, K, m, row, xs, xsum, idot, swb);
-    }
-    __syncthreads();
-    // row chains: warp w -> (half w / tm, token w % tm)
-    float v = 0.0f;
-    const int ch_half = warp / tm, ch_tt = warp % tm;
-    const bool chain = warp < 2 * tm && ch_tt < m;
-    if (chain) {
-      const int crow = ch_half * 32 + lane;
-      const float swr =
-          WG32 ? 0.0f : reinterpret_cast<const float*>(a.b.gu_s)[blk + ch_half * 128 + r_gate + lane];
-      v = row_chain<WG32, AG32>(idot + ch_tt * G * 64, swb, sx + ch_tt * G, G, crow, sx[ch_tt], swr);
-      if (a.dbg_a) (ch_half == 0 ? a.dbg_a : a.dbg_b)[(int64_t)(c0 + ch_tt) * I + i] = v;
-      if (ch_half == 1) ubuf[ch_tt * 32 + lane] = v;
-    }
-    __syncthreads();
-    if (chain && ch_half == 0) {
-      const int slot = c0 + ch_tt;
-      const float h = cswiglu(v, ubuf[ch_tt * 32 + lane]);
-      if (AG32) {
-        const float sc = f16_round(__fdiv_rn(warp_max(fabsf(h)), 127.0f));
-        a.qh[(int64_t)slot * I + i] = (int8_t)quant_code(h, sc, 127.0f);
-        if (lane == 0) a.sh[(int64_t)slot * IB + ib] = __float2half_rn(sc);
-      } else {
-        a.hbuf[(int64_t)slot * I + i] = h;
-      }
-    }
-    __syncthreads();
-  }
-}
-
-// -------------------------------------------------------------------- down
-// CTA = one selected expert x 64 output rows (two row warps of 32; NQ warps per row warp
-// split the groups along K; rows of a piece are contiguous). Same load scheme as gate/up.
-// Chains per (row warp, token); the weighted value is added into y with an fp32 atomic.
-template <int WBITS, bool WG32, bool AG32>
-__global__ void __launch_bounds__(NT, 2)
-    k_down_rows(const __grid_constant__ ExpertArgs ra, const __grid_constant__ ExpertArgs sa,
-                int has_shared, int routed_units, int tm) {
-  using B = Batch<WBITS, WG32, 128 * 16, 128>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = align1024(smem_raw);
-  const int H = ra.b.H;
-  const int Kmax = has_shared && sa.b.I > ra.b.I ? sa.b.I : ra.b.I;
-  const SmemPlan P = smem_plan(Kmax, tm, WG32);
-  uint8_t* xs = base + P.xs;
-  float* sx = reinterpret_cast<float*>(base + P.sx);
-  int* xsum = reinterpret_cast<int*>(base + P.xsum);
-  int* idot = reinterpret_cast<int*>(base + P.idot);
-  float* swb = reinterpret_cast<float*>(base + P.sw);
-  int* rows = reinterpret_cast<int*>(base + P.rows);
-  int* toks = rows + TMT;
-  float* wts = reinterpret_cast<float*>(toks + TMT);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  pdl_wait();
-  pdl_trigger();
-  bool shd;
-  int e, s0, s1, hb;
-  if (!unit_of(ra, sa, has_shared, routed_units, H / 64, blockIdx.x, shd, e, s0, s1, hb)) return;
-  const ExpertArgs& a = shd ? sa : ra;
-  const int K = a.b.I, G = K / 32, KB = kbytes(K, WBITS);
-  const int64_t blk = (int64_t)e * H + (int64_t)(hb >> 1) * 128;
-  const int r0 = (hb & 1) * 64;
-  const int rw = warp / NQ, q = warp % NQ;
-  const int row = rw * 32 + lane;
-  const uint8_t* wrow = a.b.dn_w + blk * KB + (int64_t)(r0 + row) * 16;
-  const __half* srow = reinterpret_cast<const __half*>(a.b.dn_s) + blk * G + r0 + row;
-  const int GQ = G / NQ, gq0 = q * GQ;
-  prefetch_rows<WBITS, WG32>(wrow, 128 * 16, srow, 128, gq0 + B::GB, gq0 + GQ);
-
-  for (int c0 = s0; c0 < s1; c0 += tm) {
-    const int m = min(tm, s1 - c0);
-    B bt;
-    bt.load(wrow, srow, gq0, min(B::GB, GQ));
-    if (threadIdx.x < m) {
-      const int slot = c0 + threadIdx.x;
-      rows[threadIdx.x] = slot;
-      if (!shd) {
-        int p = a.perm[slot];
-        if (p < 0 || p >= a.T * a.k) {
-          set_status(a.status, kStatusDeviceCheck);
-          p = 0;
+    mbar_arrive_expect_tx(&R.full[st], wbytes + sbytes);
+    bulk_load(R.ring + st * (kSP * kPiece), w, wbytes, &R.full[st]);
+    if (sbytes) bulk_load(R.sring + st * (kSP * 256), sc, sbytes, &R.full[st]);
+    ++c;
+    return true;
+  };
+  for (int u = blockIdx.x; u < A.units && ok; u += gridDim.x) {
+    Unit U;
+    if (!unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, false)) continue;
+    const ExpertArgs& g = A.x[0][U.shd ? 1 : 0];
+    const ExpertArgs& d = A.x[1][U.shd ? 1 : 0];
+    for (int c0 = U.s0; c0 < U.s1 && ok; c0 += A.tm, ++pidx) {
+      const int m = min(A.tm, U.s1 - c0);
+      if (MODE != 1) {
+        const int K = g.b.H, KB = kbytes(K, WBITS), NP = KB / 16, G = K / 32;
+        const bool copy_scales = AG32 && (G % 8) == 0;
+        const int64_t blk = (int64_t)U.e * 2 * g.b.I + (int64_t)U.sub * kRows;
+        const uint8_t* wsrc = g.b.gu_w + blk * KB;
+        const uint8_t* ssrc = g.b.gu_s + blk * G * 2;
+        for (int p0 = 0; p0 < NP && ok; p0 += kSP) {
+          const int np = min(kSP, NP - p0);
+          ok = push(wsrc + (int64_t)p0 * kPiece, (uint32_t)np * kPiece,
+                    ssrc + (int64_t)(p0 / PPG) * 256, WG32 ? (uint32_t)(np / PPG) * 256 : 0u);
+          if (!ok || p0 != 0) continue;
+          // this pass's activation rows, behind its first chunk
+          const int b = pidx & 1;
+          if (pidx >= 2 && !mbar_wait(&R.aempty[b], ((pidx >> 1) - 1) & 1)) {
+            wait_failed(status, kern, 3, b);
+            ok = false;
+            break;
+          }
+          uint8_t* dst = R.abuf + b * P.abytes;
+          const uint32_t bytes = (uint32_t)(m * K + (copy_scales ? m * G * 2 : 0));
+          mbar_arrive_expect_tx(&R.afull[b], bytes);
+          ++nacts;
+          for (int tt = 0; tt < m; ++tt) {
+            const int row = act_row(g, true, U, c0 + tt);
+            bulk_load(dst + tt * K, g.qa + (int64_t)row * K, (uint32_t)K, &R.afull[b]);
+            if (copy_scales)
+              bulk_load(dst + P.ascale + tt * G * 2,
+                        reinterpret_cast<const uint8_t*>(g.sa) + (int64_t)row * G * 2, (uint32_t)(G * 2),
+                        &R.afull[b]);
+          }
         }
-        toks[threadIdx.x] = p / a.k;
-        wts[threadIdx.x] = a.wts[p];
-      } else {
-        toks[threadIdx.x] = slot;
-        wts[threadIdx.x] = 1.0f;
+      }
+      if (MODE != 0 && ok) {
+        const int HB = d.b.H / kRows;
+        const int64_t slab0 = ((int64_t)U.e * (d.b.I / 64) + U.sub) * HB;   // first 128-row block
+        const uint8_t* wsrc = d.b.dn_w + slab0 * PPU * kPiece;
+        const uint8_t* ssrc = WG32 ? d.b.dn_s + slab0 * 512 : d.b.dn_s + (int64_t)U.e * d.b.H * 4;
+        for (int hb0 = 0; hb0 < HB && ok; hb0 += NBC) {
+          const int nb = min(NBC, HB - hb0);
+          ok = push(wsrc + (int64_t)hb0 * PPU * kPiece, (uint32_t)(nb * PPU * kPiece), ssrc + (int64_t)hb0 * 512,
+                    (uint32_t)nb * 512);
+        }
       }
     }
-    __syncthreads();
-    load_acts<WBITS, AG32>(a.qa, a.sa, K, m, rows, xs, sx, xsum, threadIdx.x, NT);
-    __syncthreads();
-    for (int g0 = gq0; g0 < gq0 + GQ; g0 += B::GB) {
-      const int nb = min(B::GB, gq0 + GQ - g0);
-      if (g0 != gq0) bt.load(wrow, srow, g0, nb);
-      bt.dots(g0, nb, K, m, row, xs, xsum, idot, swb);
+  }
+  // drain: no copy may still be writing into this CTA's shared memory when it exits
+  const uint32_t c0 = c > (uint32_t)kNS ? c - kNS : 0;
+  for (uint32_t dd = c0; dd < c; ++dd)
+    if (!mbar_wait(&R.full[dd % kNS], (dd / kNS) & 1)) {
+      wait_failed(status, kern, 2, dd % kNS);
+      break;
     }
-    __syncthreads();
-    const int ch_rw = warp / tm, ch_tt = warp % tm;
-    if (warp < 2 * tm && ch_tt < m) {
-      const int crow = ch_rw * 32 + lane;
-      const float swr = WG32 ? 0.0f : reinterpret_cast<const float*>(a.b.dn_s)[blk + r0 + crow];
-      const float v = row_chain<WG32, AG32>(idot + ch_tt * G * 64, swb, sx + ch_tt * G, G, crow, sx[ch_tt], swr);
-      const int n = hb * 64 + crow;
-      if (a.dbg_a) a.dbg_a[(int64_t)(c0 + ch_tt) * H + n] = v;
-      atomicAdd(a.y + (int64_t)toks[ch_tt] * H + n, wts[ch_tt] * v);
+  const uint32_t q0 = nacts > 2 ? nacts - 2 : 0;
+  for (uint32_t dd = q0; dd < nacts; ++dd)
+    if (!mbar_wait(&R.afull[dd & 1], (dd >> 1) & 1)) {
+      wait_failed(status, kern, 4, dd & 1);
+      break;
     }
-    __syncthreads();
+}
+
+// ------------------------------------------------------------------ consumers
+// A chunk is consumed in blocks of 8 consecutive groups (int8: one block per chunk, int4:
+// two). Dots: warp w takes group w of the block for all 128 rows (lane l: rows l, l+32,
+// l+64, l+96), loads the block's activations once per token and writes each exact int32
+// dot to idot[buffer][w][token][row]. One consumer barrier later, thread (row, token set)
+// runs the ordered fp32 chain of its row over the block's 8 groups for its tokens
+// (tokens ts, ts+2, ... with ts = thread / 128). idot is double-buffered, so the barrier
+// after the next block's dots also orders this block's chain before the buffer is reused.
+template <int WBITS, bool WG32, bool AG32>
+__device__ __forceinline__ void block_dots(const uint8_t* stage, int j0, int gbase, int m, int tm,
+                                           const uint8_t* xs, int K, const int* xsum, int G, int* idot) {
+  constexpr int PPG = WBITS == 8 ? 2 : 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = gbase + j0 + warp;                     // this warp's group
+  const uint8_t* wp = stage + (j0 + warp) * PPG * kPiece + lane * 16;
+  uint4 w[4 * PPG];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    w[r * PPG] = *reinterpret_cast<const uint4*>(wp + r * 512);
+    if (WBITS == 8) w[r * PPG + 1] = *reinterpret_cast<const uint4*>(wp + kPiece + r * 512);
+  }
+  int* out = idot + warp * tm * kRows + lane;
+  for (int q = 0; q < m; ++q) {
+    const uint8_t* xg = xs + q * K + 32 * g;
+    const uint4 x0 = *reinterpret_cast<const uint4*>(xg);
+    const uint4 x1 = *reinterpret_cast<const uint4*>(xg + 16);
+    int xsg = 0;
+    if (WBITS == 4) xsg = xsum[q * G + g];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      int d;
+      if (WBITS == 8)
+        d = group_dot_i8(w[2 * r], w[2 * r + 1], x0, x1);
+      else
+        d = group_dot_i4(w[r], make_uint4(x0.x, x0.z, x1.x, x1.z), make_uint4(x0.y, x0.w, x1.y, x1.w), xsg);
+      out[q * kRows + r * 32] = d;
+    }
+  }
+}
+
+template <int WBITS, bool WG32, bool AG32>
+__device__ __forceinline__ void block_chain(const __half* sst, int j0, int gbase, int m, int tm, int G,
+                                            const int* idot, const __half* sxh, const float* sxf,
+                                            float acc[kTMP / 2], int isum[kTMP / 2]) {
+  const int row = threadIdx.x & 127, ts = threadIdx.x >> 7;
+  float sw[8];
+  if (WG32) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sw[j] = __half2float(sst[(j0 + j) * 128 + row]);
+  }
+#pragma unroll
+  for (int qq = 0; qq < kTMP / 2; ++qq) {
+    const int q = ts + 2 * qq;
+    if (q >= m) break;
+    int d[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) d[j] = idot[(j * tm + q) * kRows + row];
+    if (!WG32 && !AG32) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) isum[qq] += d[j];
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int g = gbase + j0 + j;
+        float sxg = 0.0f;
+        if (AG32) sxg = sxh ? __half2float(sxh[q * G + g]) : sxf[q * G + g];
+        float cg;
+        if (WG32 && AG32) cg = __fmul_rn(sw[j], sxg);
+        else if (WG32) cg = sw[j];
+        else cg = sxg;
+        acc[qq] = __fmaf_rn(__int2float_rn(d[j]), cg, acc[qq]);
+      }
+    }
+  }
+}
+
+// Consumes one pass (all chunks of the unit) and leaves the stage values of row
+// (thread & 127) for tokens ts + 2 qq in v[qq]. After a wait gives up (`abort` set by any
+// consumer), waits and compute are skipped but every stage is still released and every
+// barrier taken, so the producer is never left waiting.
+template <int WBITS, bool WG32, bool AG32>
+__device__ __forceinline__ void ring_consume(int K, int m, int tm, const Ring& R, uint32_t& c, uint32_t& nblk,
+                                             const uint8_t* xs, const __half* sxh, const float* sxf,
+                                             const int* xsum, int* idot, float sw_row,
+                                             float v[kTMP / 2], volatile int* abort, int* status,
+                                             int kernel) {
+  constexpr int PPG = WBITS == 8 ? 2 : 1;
+  const int lane = threadIdx.x & 31;
+  const int ts = threadIdx.x >> 7;
+  const bool chain_thread = ts < m;
+  const int KB = kbytes(K, WBITS), NP = KB / 16, G = K / 32;
+  float acc[kTMP / 2];
+  int isum[kTMP / 2];
+#pragma unroll
+  for (int q = 0; q < kTMP / 2; ++q) {
+    acc[q] = 0.0f;
+    isum[q] = 0;
+  }
+  for (int p0 = 0; p0 < NP; p0 += kSP, ++c) {
+    const int np = min(kSP, NP - p0);
+    const int st = c % kNS;
+    bool ok = *abort == 0;
+    if (ok && !mbar_wait(&R.full[st], (c / kNS) & 1)) {
+      *abort = 1;
+      if (lane == 0) wait_failed(status, kernel, 1, st);
+      ok = false;
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    const uint8_t* stage = R.ring + st * (kSP * kPiece);
+    const __half* sst = reinterpret_cast<const __half*>(R.sring + st * (kSP * 256));
+    const int gbase = p0 / PPG, ng = np / PPG;
+    // blocks of 8 groups; a short last chunk (K a multiple of 128 but not of 256 / 512)
+    // ends with a block of 4, handled by the first four warps and chain steps
+    for (int j0 = 0; j0 < ng; j0 += 8, ++nblk) {
+      const int nb = min(8, ng - j0);
+      int* ib = idot + (nblk & 1) * (8 * tm * kRows);
+      if (ok && (threadIdx.x >> 5) < nb) block_dots<WBITS, WG32, AG32>(stage, j0, gbase, m, tm, xs, K, xsum, G, ib);
+      named_bar(1, 32 * kCW);
+      if (ok && chain_thread) {
+        if (nb == 8) {
+          block_chain<WBITS, WG32, AG32>(sst, j0, gbase, m, tm, G, ib, sxh, sxf, acc, isum);
+        } else {
+          // 4-group tail: same chain, groups j0 .. j0+3 only
+          const int row = threadIdx.x & 127;
+          for (int qq = 0; qq < kTMP / 2; ++qq) {
+            const int q = ts + 2 * qq;
+            if (q >= m) break;
+            for (int j = 0; j < nb; ++j) {
+              const int g = gbase + j0 + j;
+              const int d = ib[(j * tm + q) * kRows + row];
+              if (!WG32 && !AG32) {
+                isum[qq] += d;
+              } else {
+                const float swg = WG32 ? __half2float(sst[(j0 + j) * 128 + row]) : 0.0f;
+                float sxg = 0.0f;
+                if (AG32) sxg = sxh ? __half2float(sxh[q * G + g]) : sxf[q * G + g];
+                float cg;
+                if (WG32 && AG32) cg = __fmul_rn(swg, sxg);
+                else if (WG32) cg = swg;
+                else cg = sxg;
+                acc[qq] = __fmaf_rn(__int2float_rn(d), cg, acc[qq]);
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&R.empty[st]);
+  }
+#pragma unroll
+  for (int qq = 0; qq < kTMP / 2; ++qq) {
+    const int q = ts + 2 * qq;
+    const float sxt = (!AG32 && q < m) ? sxf[q] : 0.0f;
+    if (WG32 && AG32) v[qq] = acc[qq];
+    else if (WG32) v[qq] = __fmul_rn(acc[qq], sxt);
+    else if (AG32) v[qq] = __fmul_rn(acc[qq], sw_row);
+    else v[qq] = __fmul_rn(__fmaf_rn(__int2float_rn(isum[qq]), sxt, 0.0f), sw_row);
+  }
+}
+
+// Down pass of one unit: the slab's 128-row blocks arrive a chunk at a time; thread t takes
+// rows t, t + 256, ... of the chunk (int8: 2 rows, int4: 4). Per (row, token) the two group
+// dots against the unit's 64 h codes give this unit's share of the row's down value
+// (fp32, any order), weighted and added into y (and, for inspection, into the pair's
+// down value). hx: the pass's h codes [tm][64] (int4 weights: each 8-byte word
+// de-interleaved), hxs: per-group code sums [tm][2] (int4), hs: h scales [tm][2].
+template <int WBITS, bool WG32, bool AG32>
+__device__ __forceinline__ void down_consume(int H, int m, const Ring& R, uint32_t& c, const uint8_t* hx,
+                                             const int* hxs, const float* hs, const int* toks,
+                                             const float* wts, float* y, float* dbg, int slot0,
+                                             volatile int* abort, int* status) {
+  constexpr int PPU = WBITS == 8 ? 4 : 2;
+  constexpr int NBC = kSP / PPU;
+  constexpr int RPT = NBC * kRows / (32 * kCW);   // rows per thread of a full chunk
+  const int lane = threadIdx.x & 31;
+  const int HB = H / kRows;
+  for (int hb0 = 0; hb0 < HB; hb0 += NBC, ++c) {
+    const int nb = min(NBC, HB - hb0);
+    const int st = c % kNS;
+    bool ok = *abort == 0;
+    if (ok && !mbar_wait(&R.full[st], (c / kNS) & 1)) {
+      *abort = 1;
+      if (lane == 0) wait_failed(status, 2, 1, st);
+      ok = false;
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      const uint8_t* stage = R.ring + st * (kSP * kPiece);
+      const uint8_t* sst = R.sring + st * (kSP * 256);
+      uint4 w[RPT][PPU];
+      float c0s[RPT], c1s[RPT];
+#pragma unroll
+      for (int k = 0; k < RPT; ++k) {
+        const int rr = threadIdx.x + 32 * kCW * k, b = rr >> 7, r = rr & 127;
+        if (b < nb) {
+#pragma unroll
+          for (int p = 0; p < PPU; ++p)
+            w[k][p] = *reinterpret_cast<const uint4*>(stage + ((b * PPU + p) * kRows + r) * 16);
+          if (WG32) {
+            const __half* sh = reinterpret_cast<const __half*>(sst);
+            c0s[k] = __half2float(sh[(b * 2) * kRows + r]);
+            c1s[k] = __half2float(sh[(b * 2 + 1) * kRows + r]);
+          } else {
+            c0s[k] = c1s[k] = reinterpret_cast<const float*>(sst)[b * kRows + r];
+          }
+        }
+      }
+      for (int q = 0; q < m; ++q) {
+        const uint4* xq = reinterpret_cast<const uint4*>(hx + q * 64);
+        const uint4 x0 = xq[0], x1 = xq[1], x2 = xq[2], x3 = xq[3];
+        const float hs0 = hs[2 * q], hs1 = hs[2 * q + 1];
+        const float wq = wts[q];
+        float* yq = y + (int64_t)toks[q] * H;
+        float* dq = dbg ? dbg + (int64_t)(slot0 + q) * H : nullptr;
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+          const int rr = threadIdx.x + 32 * kCW * k, b = rr >> 7, r = rr & 127;
+          if (b >= nb) break;
+          int d0, d1;
+          if (WBITS == 8) {
+            d0 = group_dot_i8(w[k][0], w[k][1], x0, x1);
+            d1 = group_dot_i8(w[k][2], w[k][3], x2, x3);
+          } else {
+            d0 = group_dot_i4(w[k][0], make_uint4(x0.x, x0.z, x1.x, x1.z), make_uint4(x0.y, x0.w, x1.y, x1.w),
+                              hxs[2 * q]);
+            d1 = group_dot_i4(w[k][1], make_uint4(x2.x, x2.z, x3.x, x3.z), make_uint4(x2.y, x2.w, x3.y, x3.w),
+                              hxs[2 * q + 1]);
+          }
+          float v;
+          if (WG32 && AG32)
+            v = __fmaf_rn(__int2float_rn(d1), __fmul_rn(c1s[k], hs1), __fmul_rn(__int2float_rn(d0), __fmul_rn(c0s[k], hs0)));
+          else if (WG32)
+            v = __fmul_rn(__fmaf_rn(__int2float_rn(d1), c1s[k], __fmul_rn(__int2float_rn(d0), c0s[k])), hs0);
+          else if (AG32)
+            v = __fmul_rn(__fmaf_rn(__int2float_rn(d1), hs1, __fmul_rn(__int2float_rn(d0), hs0)), c0s[k]);
+          else
+            v = __fmul_rn(__fmul_rn(__int2float_rn(d0 + d1), hs0), c0s[k]);
+          const int n = (hb0 + b) * kRows + r;
+          atomicAdd(yq + n, wq * v);
+          if (dq) atomicAdd(dq + n, v);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&R.empty[st]);
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+// Per unit and pass: the gate/up pass (consumer warps of ring_consume; after it the gate and
+// up stage values meet in shared memory and warps 0 and 1 apply SwiGLU and quantize h per
+// group of 32 -- one warp per group), then the down pass over the unit's slab with the
+// pass's h codes from shared memory (MODE 2) or from the workspace (MODE 1).
+template <int WBITS, bool WG32, bool AG32, int MODE>
+__global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ RingArgs A) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = align1024(smem_raw);
+  const RingPlan P = ring_plan(A.kmax, A.tm);
+  Ring R;
+  R.ring = base + P.ring;
+  R.sring = base + P.sring;
+  R.full = reinterpret_cast<uint64_t*>(base + P.bars);
+  R.empty = R.full + kNS;
+  R.afull = R.empty + kNS;
+  R.aempty = R.afull + 2;
+  R.abuf = base + P.abuf;
+  R.xsum = reinterpret_cast<int*>(base + P.xsum);
+  R.sxf = reinterpret_cast<float*>(base + P.sxf);
+  int* idot = reinterpret_cast<int*>(base + P.idot);
+  float* gbuf = reinterpret_cast<float*>(base + P.ubuf);
+  float* ubuf = gbuf + A.tm * 64;
+  uint8_t* hq = base + P.hq;                       // [tm][64] h codes of the pass
+  uint8_t* hqd = hq + A.tm * 64;                   // [tm][64] de-interleaved (int4 weights)
+  float* hs = reinterpret_cast<float*>(hqd + A.tm * 64);   // [tm][2] h scales
+  int* hxs = reinterpret_cast<int*>(hs + 2 * A.tm);        // [tm][2] code sums
+  int* toks = reinterpret_cast<int*>(base + P.info);
+  float* wts = reinterpret_cast<float*>(toks + kTMP);
+  volatile int* abort = toks + 3 * kTMP;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* status = A.x[0][0].status;
+
+  if (threadIdx.x == 0) {
+    *abort = 0;
+    for (int s = 0; s < kNS; ++s) {
+      mbar_init(&R.full[s], 1);
+      mbar_init(&R.empty[s], kCW);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&R.afull[b], 1);
+      mbar_init(&R.aempty[b], kCW);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == kCW) {
+    if (lane == 0) ring_producer<WBITS, WG32, AG32, MODE>(A, P, R);
+    return;
+  }
+
+  const int ctid = threadIdx.x;             // consumer thread index, [0, 256)
+  const int row = ctid & 127, ts = ctid >> 7;  // chain row, first token (tokens ts + 2 qq)
+  const int tm = A.tm;
+  uint32_t c = 0, pidx = 0, nblk = 0;       // chunks, gate/up passes, 8-group blocks consumed
+  for (int u = blockIdx.x; u < A.units; u += gridDim.x) {
+    Unit U;
+    if (!unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, ctid == 0)) continue;
+    const ExpertArgs& g = A.x[0][U.shd ? 1 : 0];
+    const ExpertArgs& d = A.x[1][U.shd ? 1 : 0];
+    const int I = g.b.I, IB = I / 32;
+    for (int c0 = U.s0; c0 < U.s1; c0 += tm) {
+      const int m = min(tm, U.s1 - c0);
+      named_bar(1, 32 * kCW);              // previous pass done with the per-pass arrays
+      if (ctid < m) {
+        const int slot = c0 + ctid;
+        if (MODE != 0) {
+          int p = U.shd ? slot : __ldcg(d.perm + slot);
+          if (p < 0 || p >= (U.shd ? d.T : d.T * d.k)) {
+            set_status(status, kStatusDeviceCheck);
+            p = 0;
+          }
+          toks[ctid] = U.shd ? slot : p / d.k;
+          wts[ctid] = U.shd ? 1.0f : d.wts[p];
+        }
+        if (MODE != 1 && !AG32) R.sxf[ctid] = reinterpret_cast<const float*>(g.sa)[act_row(g, true, U, slot)];
+      }
+      if (MODE == 1) {
+        // h of this unit's 64 columns, written by the gate/up and h-quantization kernels
+        if (ctid < 4 * m) {
+          const int q = ctid >> 2, part = ctid & 3;
+          reinterpret_cast<uint4*>(hq + q * 64)[part] =
+              *reinterpret_cast<const uint4*>(d.qa + (int64_t)(c0 + q) * I + U.sub * 64 + part * 16);
+        }
+        if (ctid < 2 * m) {
+          const int q = ctid >> 1, j = ctid & 1;
+          hs[ctid] = AG32 ? __half2float(reinterpret_cast<const __half*>(d.sa)[(int64_t)(c0 + q) * IB + 2 * U.sub + j])
+                          : reinterpret_cast<const float*>(d.sa)[c0 + q];
+        }
+      }
+      if (MODE != 1) {
+        const int K = g.b.H, G = K / 32;
+        const bool copy_scales = AG32 && (G % 8) == 0;
+        const int b = pidx & 1;
+        if (AG32 && !copy_scales)
+          for (int l = ctid; l < m * G; l += 32 * kCW) {
+            const int tt = l / G, gg = l - tt * G;
+            const int r = act_row(g, true, U, c0 + tt);
+            R.sxf[l] = __half2float(reinterpret_cast<const __half*>(g.sa)[(int64_t)r * G + gg]);
+          }
+        uint8_t* xs = R.abuf + b * P.abytes;
+        int* xsum = R.xsum + b * tm * G;
+        bool aok = *abort == 0;
+        if (aok && !mbar_wait(&R.afull[b], (pidx >> 1) & 1)) {
+          *abort = 1;
+          if (lane == 0) wait_failed(status, 1, 5, b);
+          aok = false;
+        }
+        if (WBITS == 4) {
+          // de-interleave each 8-byte word into even / odd elements; per-group sums
+          // (barriers taken by every consumer thread, whatever its wait returned)
+          if (aok)
+            for (int l = ctid; l < m * (K / 8); l += 32 * kCW) {
+              uint2* wp = reinterpret_cast<uint2*>(xs) + l;
+              const uint2 v = *wp;
+              uint2 o;
+              deinterleave8(v.x, v.y, o.x, o.y);
+              *wp = o;
+            }
+          named_bar(1, 32 * kCW);
+          if (aok)
+            for (int l = ctid; l < m * G; l += 32 * kCW) {
+              const uint4* q4 = reinterpret_cast<const uint4*>(xs + (l / G) * K + 32 * (l % G));
+              const uint4 a0 = q4[0], a1 = q4[1];
+              int sacc = __dp4a((int)a0.x, 0x01010101, 0);
+              sacc = __dp4a((int)a0.y, 0x01010101, sacc);
+              sacc = __dp4a((int)a0.z, 0x01010101, sacc);
+              sacc = __dp4a((int)a0.w, 0x01010101, sacc);
+              sacc = __dp4a((int)a1.x, 0x01010101, sacc);
+              sacc = __dp4a((int)a1.y, 0x01010101, sacc);
+              sacc = __dp4a((int)a1.z, 0x01010101, sacc);
+              sacc = __dp4a((int)a1.w, 0x01010101, sacc);
+              xsum[l] = sacc;
+            }
+        }
+        named_bar(1, 32 * kCW);
+        const __half* sxh = copy_scales ? reinterpret_cast<const __half*>(xs + P.ascale) : nullptr;
+        const int64_t blk = (int64_t)U.e * 2 * I + (int64_t)U.sub * kRows;
+        const float sw_row = WG32 ? 0.0f : reinterpret_cast<const float*>(g.b.gu_s)[blk + row];
+        float v[kTMP / 2];
+        ring_consume<WBITS, WG32, AG32>(K, m, tm, R, c, nblk, xs, sxh, R.sxf, xsum, idot, sw_row, v, abort,
+                                        status, 1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&R.aempty[b]);
+        ++pidx;
+        const bool is_up = row >= 64;
+#pragma unroll
+        for (int qq = 0; qq < kTMP / 2; ++qq) {
+          const int q = ts + 2 * qq;
+          if (q < m) {
+            if (g.dbg_a) (is_up ? g.dbg_b : g.dbg_a)[(int64_t)(c0 + q) * I + U.sub * 64 + (row & 63)] = v[qq];
+            (is_up ? ubuf : gbuf)[q * 64 + (row & 63)] = v[qq];
+          }
+        }
+        named_bar(1, 32 * kCW);
+        if (warp < 2) {
+          // SwiGLU and h quantization: warp w takes the group of 32 indices w * 32 ..
+          const int il = warp * 32 + lane, i = U.sub * 64 + il;
+          for (int q = 0; q < m; ++q) {
+            const int slot = c0 + q;
+            const float h = cswiglu(gbuf[q * 64 + il], ubuf[q * 64 + il]);
+            if (AG32) {
+              const float sc = f16_round(__fdiv_rn(warp_max(fabsf(h)), 127.0f));
+              const int code = quant_code(h, sc, 127.0f);
+              g.qh[(int64_t)slot * I + i] = (int8_t)code;
+              if (lane == 0) g.sh[(int64_t)slot * IB + i / 32] = __float2half_rn(sc);
+              if (MODE == 2) {
+                hq[q * 64 + il] = (uint8_t)(int8_t)code;
+                if (lane == 0) hs[2 * q + warp] = sc;
+              }
+            } else {
+              g.hbuf[(int64_t)slot * I + i] = h;
+            }
+          }
+        }
+      }
+      if (MODE != 0) {
+        named_bar(1, 32 * kCW);            // h codes / scales of the pass in shared memory
+        const uint8_t* hx = hq;
+        if (WBITS == 4) {
+          if (ctid < 8 * m) {
+            const uint2 v = reinterpret_cast<const uint2*>(hq)[ctid];
+            uint2 o;
+            deinterleave8(v.x, v.y, o.x, o.y);
+            reinterpret_cast<uint2*>(hqd)[ctid] = o;
+          }
+          if (ctid < 2 * m) {
+            const uint4* q4 = reinterpret_cast<const uint4*>(hq + ctid * 32);
+            const uint4 a0 = q4[0], a1 = q4[1];
+            int sacc = __dp4a((int)a0.x, 0x01010101, 0);
+            sacc = __dp4a((int)a0.y, 0x01010101, sacc);
+            sacc = __dp4a((int)a0.z, 0x01010101, sacc);
+            sacc = __dp4a((int)a0.w, 0x01010101, sacc);
+            sacc = __dp4a((int)a1.x, 0x01010101, sacc);
+            sacc = __dp4a((int)a1.y, 0x01010101, sacc);
+            sacc = __dp4a((int)a1.z, 0x01010101, sacc);
+            sacc = __dp4a((int)a1.w, 0x01010101, sacc);
+            hxs[ctid] = sacc;
+          }
+          named_bar(1, 32 * kCW);
+          hx = hqd;
+        }
+        down_consume<WBITS, WG32, AG32>(d.b.H, m, R, c, hx, hxs, hs, toks, wts, d.y, d.dbg_a, c0, abort, status);
+      }
+    }
   }
 }
 
 // ------------------------------------------------------------------ host side
 namespace {
 
-template <int WBITS, bool WG32, bool AG32>
-cudaError_t launch_gateup_t(const ExpertArgs& r, const ExpertArgs* s, cudaStream_t st) {
-  const int K = r.b.H;
-  const int tm = pass_tokens(K, r.T);
-  const SmemPlan P = smem_plan(K, tm, WG32);
+int sm_count() {
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (n[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 148;
+  }
+  return n[dev];
+}
+
+template <int WBITS, bool WG32, bool AG32, int MODE>
+cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
+  const RingPlan P = ring_plan(A.kmax, A.tm);
   static int attr_bytes = 0;
   if (P.total > attr_bytes) {
-    const cudaError_t e = cudaFuncSetAttribute(k_gateup_rows<WBITS, WG32, AG32>,
+    const cudaError_t e = cudaFuncSetAttribute(k_expert_ring<WBITS, WG32, AG32, MODE>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, P.total);
     if (e != cudaSuccess) return e;
     attr_bytes = P.total;
   }
-  const int routed = r.max_active * (r.b.I / 32);
-  const int grid = routed + (s ? s->b.I / 32 : 0);
-  return launch_pdl(k_gateup_rows<WBITS, WG32, AG32>, dim3(grid), dim3(NT), (size_t)P.total, st, r,
-                    s ? *s : r, s ? 1 : 0, routed, tm);
+  const int grid = A.units < sm_count() ? A.units : sm_count();
+  if (grid <= 0) return cudaSuccess;
+  return launch_pdl(k_expert_ring<WBITS, WG32, AG32, MODE>, dim3(grid), dim3(kNT), (size_t)P.total, st, A);
 }
 
 template <int WBITS, bool WG32, bool AG32>
-cudaError_t launch_down_t(const ExpertArgs& r, const ExpertArgs* s, cudaStream_t st) {
-  const int H = r.b.H;
-  const int Kmax = s && s->b.I > r.b.I ? s->b.I : r.b.I;
-  const int tm = pass_tokens(Kmax, r.T);
-  const SmemPlan P = smem_plan(Kmax, tm, WG32);
-  static int attr_bytes = 0;
-  if (P.total > attr_bytes) {
-    const cudaError_t e = cudaFuncSetAttribute(k_down_rows<WBITS, WG32, AG32>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, P.total);
-    if (e != cudaSuccess) return e;
-    attr_bytes = P.total;
-  }
-  const int routed = r.max_active * (H / 64);
-  const int grid = routed + (s ? H / 64 : 0);
-  return launch_pdl(k_down_rows<WBITS, WG32, AG32>, dim3(grid), dim3(NT), (size_t)P.total, st, r,
-                    s ? *s : r, s ? 1 : 0, routed, tm);
+cudaError_t launch_mode(int mode, const RingArgs& A, cudaStream_t st) {
+  if (mode == 0) return launch_ring_t<WBITS, WG32, AG32, 0>(A, st);
+  if (mode == 1) return launch_ring_t<WBITS, WG32, AG32, 1>(A, st);
+  if constexpr (AG32) return launch_ring_t<WBITS, WG32, AG32, 2>(A, st);
+  return cudaErrorInvalidValue;               // the fused mode needs group-32 activations
 }
 
 }  // namespace
 
-#define MOE_DISPATCH_TMA(FN, r, s, st)                                                        \
-  ([&]() -> cudaError_t {                                                                     \
-    const int sel = ((r).b.wbits == 8 ? 4 : 0) | ((r).b.wg32 ? 2 : 0) | ((r).ag32 ? 1 : 0); \
-    switch (sel) {                                                                            \
-      case 7: return FN<8, true, true>(r, s, st);                                             \
-      case 6: return FN<8, true, false>(r, s, st);                                            \
-      case 5: return FN<8, false, true>(r, s, st);                                            \
-      case 4: return FN<8, false, false>(r, s, st);                                           \
-      case 3: return FN<4, true, true>(r, s, st);                                             \
-      case 2: return FN<4, true, false>(r, s, st);                                            \
-      case 1: return FN<4, false, true>(r, s, st);                                            \
-      default: return FN<4, false, false>(r, s, st);                                          \
-    }                                                                                         \
-  }())
-
-cudaError_t launch_gateup_tma(const ExpertArgs& r, const ExpertArgs* s, cudaStream_t st) {
-  return MOE_DISPATCH_TMA(launch_gateup_t, r, s, st);
+bool experts_fusable(const ExpertArgs& r, const ExpertArgs* s) {
+  (void)s;
+  return r.ag32 != 0;
 }
 
-cudaError_t launch_down_tma(const ExpertArgs& r, const ExpertArgs* s, cudaStream_t st) {
-  return MOE_DISPATCH_TMA(launch_down_t, r, s, st);
+cudaError_t launch_experts(int mode, const ExpertArgs& gr, const ExpertArgs* gs, const ExpertArgs& dr,
+                           const ExpertArgs* ds, cudaStream_t st) {
+  RingArgs A;
+  std::memset(&A, 0, sizeof(A));
+  A.x[0][0] = gr;
+  A.x[0][1] = gs ? *gs : gr;
+  A.x[1][0] = dr;
+  A.x[1][1] = ds ? *ds : dr;
+  A.has_shared = gs != nullptr;
+  A.per = gr.b.I / 64;
+  A.routed = gr.max_active * A.per;
+  A.units = A.routed + (gs ? gs->b.I / 64 : 0);
+  A.kmax = mode == 1 ? 64 : gr.b.H;           // K of the staged activation rows
+  A.tm = ring_tokens(A.kmax, gr.T);
+  const int sel = (gr.b.wbits == 8 ? 4 : 0) | (gr.b.wg32 ? 2 : 0) | (gr.ag32 ? 1 : 0);
+  switch (sel) {
+    case 7: return launch_mode<8, true, true>(mode, A, st);
+    case 6: return launch_mode<8, true, false>(mode, A, st);
+    case 5: return launch_mode<8, false, true>(mode, A, st);
+    case 4: return launch_mode<8, false, false>(mode, A, st);
+    case 3: return launch_mode<4, true, true>(mode, A, st);
+    case 2: return launch_mode<4, true, false>(mode, A, st);
+    case 1: return launch_mode<4, false, true>(mode, A, st);
+    default: return launch_mode<4, false, false>(mode, A, st);
+  }
 }
 
 }  // namespace moe

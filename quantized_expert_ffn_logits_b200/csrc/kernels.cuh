@@ -28,6 +28,7 @@ struct Grouping {            // batch-union grouping outputs (all device pointer
   int32_t* n_active;         // [1]
   int32_t* act_expert;       // [E]
   int32_t* act_begin;        // [E+1]
+  int32_t* act_rows;         // [E][8] token of each active expert's first 8 slots (or null)
 };
 
 void launch_topk(const float* logits, const float* bias, int T, int E, int k, int score,
@@ -38,7 +39,7 @@ void launch_topk(const float* logits, const float* bias, int T, int E, int k, in
 void launch_permute(const int32_t* idx, int T, int k, int E, const Grouping& g, uint32_t* masks,
                     int32_t* base, int* status, int reset_status, cudaStream_t st);
 
-// ---- expert_gemv.cu
+// ---- expert_stream.cu (weight-streaming expert kernels)
 struct ExpertArgs {
   BlobView b;
   // activation rows: gate/up reads q_x rows (one per token); down reads q_h rows (one per slot)
@@ -51,6 +52,7 @@ struct ExpertArgs {
   const int32_t* act_expert;
   const int32_t* act_begin;
   const int32_t* perm;
+  const int32_t* act_rows;   // [E][8] tokens of the first 8 slots of each active expert
   const float* wts;          // routing weights [T*k] (down, routed)
   int T, k;
   int max_active;            // grid bound on active experts
@@ -64,9 +66,13 @@ struct ExpertArgs {
   int* status;
 };
 
-// ---- expert_stream.cu: routed experts `r` and (optional) shared expert `s` in one grid each
-cudaError_t launch_gateup_tma(const ExpertArgs& r, const ExpertArgs* s, cudaStream_t st);
-cudaError_t launch_down_tma(const ExpertArgs& r, const ExpertArgs* s, cudaStream_t st);
+// Routed experts and (optional) shared expert: gate/up args gr/gs, down args dr/ds. Work
+// unit = (expert, 64 intermediate indices). mode 0: gate/up pass of every unit (h to the
+// workspace), 1: down pass (h from the workspace), 2: both, h kept on chip -- needs
+// experts_fusable() (group-32 activations: h of a unit is quantized without the rest).
+bool experts_fusable(const ExpertArgs& r, const ExpertArgs* s);
+cudaError_t launch_experts(int mode, const ExpertArgs& gr, const ExpertArgs* gs, const ExpertArgs& dr,
+                           const ExpertArgs* ds, cudaStream_t st);
 
 // ---- route_fused.cu (T <= 32)
 struct RouteArgs {
@@ -111,6 +117,7 @@ inline cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cud
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// ---- expert_gemv.cu (debug entry point)
 void launch_group_dots(const BlobView& b, int which, int n, const int32_t* expert,
                        const int32_t* row, const int8_t* act, int32_t* dots, cudaStream_t st);
 

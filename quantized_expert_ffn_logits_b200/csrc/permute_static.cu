@@ -66,7 +66,7 @@ extern "C" moe_status moe_permute_no_alloc(const int32_t* idx, int32_t T, int32_
   o += al256(C * E * 4);
   int32_t* prefix = reinterpret_cast<int32_t*>(ws + o);
   o += al256(C * E * 4);
-  moe::Grouping g;
+  moe::Grouping g{};
   g.offsets = offsets;
   g.perm = perm;
   g.n_active = reinterpret_cast<int32_t*>(ws + o);

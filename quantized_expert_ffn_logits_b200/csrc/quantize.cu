@@ -12,7 +12,7 @@ namespace moe {
 
 // One warp per weight row. Rows [0, E*2I) are gate/up rows (logical [E][2I][H]),
 // rows [E*2I, E*2I + E*H) are down rows (logical [E][H][I]). Codes and scales are
-// written straight into the blob's tiled layout.
+// written straight into the blob's tiled layout (include/moe_b200.h).
 __global__ void __launch_bounds__(256) k_quantize_experts(const float* __restrict__ w_gu,
                                                           const float* __restrict__ w_dn,
                                                           BlobView b, uint8_t* gu_w, uint8_t* dn_w,
@@ -25,44 +25,56 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const float* __restric
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t R = warp0; R < n_rows; R += nwarps) {
     const float* src;
-    int K, rows_per_block, piece_stride;
-    uint8_t* dst;     // byte 0 of this row's piece 0 in the tiled code region
-    uint8_t* sdst;    // this row's scale slot (g32: group 0, next group at +rows_per_block)
+    int K;
+    bool down;
+    int64_t blk = 0;     // gate/up: first row of the row's 128-row block
+    int r = 0;           // row inside its block
+    int e = 0, hb = 0;   // down: expert, 128-row block of H
     if (R < n_gu) {
-      const int e = (int)(R / (2 * b.I));
+      e = (int)(R / (2 * b.I));
       const int lr = (int)(R % (2 * b.I));
       const int half = lr >= b.I;
       const int i = lr - half * b.I;
       K = b.H;
-      rows_per_block = 256;
-      const int kb = kbytes(K, b.wbits);
-      const int r = half * 128 + (i & 127);
-      const int64_t blk = (int64_t)e * 2 * b.I + (int64_t)(i >> 7) * 256;  // first row of block
+      down = false;
+      r = half * 64 + (i & 63);
+      blk = (int64_t)e * 2 * b.I + (int64_t)(i >> 6) * 128;
       src = w_gu + R * (int64_t)K;
-      dst = gu_w + blk * kb + (int64_t)r * 16;
-      sdst = b.wg32 ? gu_s + (blk * (K / 32) + r) * 2 : gu_s + (blk + r) * 4;
     } else {
       const int64_t R2 = R - n_gu;
-      const int e = (int)(R2 / b.H);
+      e = (int)(R2 / b.H);
       const int n = (int)(R2 % b.H);
       K = b.I;
-      rows_per_block = 128;
-      const int kb = kbytes(K, b.wbits);
-      const int r = n & 127;
-      const int64_t blk = (int64_t)e * b.H + (int64_t)(n >> 7) * 128;
+      down = true;
+      hb = n >> 7;
+      r = n & 127;
       src = w_dn + R2 * (int64_t)K;
-      dst = dn_w + blk * kb + (int64_t)r * 16;
-      sdst = b.wg32 ? dn_s + (blk * (K / 32) + r) * 2 : dn_s + (blk + r) * 4;
     }
-    piece_stride = rows_per_block * 16;
     const int G = K / 32;
+    const int kb = kbytes(K, b.wbits);
+    const int U = b.I / 64, HB = b.H / 128;
+    const int sb = b.wbits == 8 ? 64 : 32;            // bytes of 64 elements
+    // byte `byte` of this row's codes -> its place in the tiled region
+    auto code_at = [&](int byte) -> uint8_t* {
+      if (!down) return gu_w + blk * kb + (int64_t)(byte >> 4) * (128 * 16) + r * 16 + (byte & 15);
+      const int u = byte / sb, bb = byte - u * sb;
+      const int64_t slab = ((int64_t)e * U + u) * HB + hb;
+      return dn_w + ((slab * (sb / 16) + (bb >> 4)) * 128 + r) * 16 + (bb & 15);
+    };
+    // scale slot of group g (fp16) or of the row (fp32)
+    auto scale_at = [&](int g) -> uint8_t* {
+      if (!down) return b.wg32 ? gu_s + ((blk * G) + (int64_t)g * 128 + r) * 2 : gu_s + (blk + r) * 4;
+      if (!b.wg32) return dn_s + ((int64_t)e * b.H + hb * 128 + r) * 4;
+      const int64_t slab = ((int64_t)e * U + (g >> 1)) * HB + hb;
+      return dn_s + ((slab * 2 + (g & 1)) * 128 + r) * 2;
+    };
     float s_row = 0.0f;
     if (!b.wg32) {
       float amax = 0.0f;
       for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(src[k]));
       amax = warp_max(amax);
       s_row = __fdiv_rn(amax, qmax);
-      if (lane == 0) *reinterpret_cast<float*>(sdst) = s_row;
+      if (lane == 0) *reinterpret_cast<float*>(scale_at(0)) = s_row;
     }
     for (int g = 0; g < G; ++g) {
       const float v = src[32 * g + lane];
@@ -70,20 +82,14 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const float* __restric
       if (b.wg32) {
         const float amax = warp_max(fabsf(v));
         s = f16_round(__fdiv_rn(amax, qmax));
-        if (lane == 0)
-          reinterpret_cast<__half*>(sdst)[(int64_t)g * rows_per_block] = __float2half_rn(s);
+        if (lane == 0) *reinterpret_cast<__half*>(scale_at(g)) = __float2half_rn(s);
       }
       const int q = quant_code(v, s, qmax);
       if (b.wbits == 8) {
-        const int byte = 32 * g + lane;
-        dst[(int64_t)(byte >> 4) * piece_stride + (byte & 15)] = (uint8_t)(int8_t)q;
+        *code_at(32 * g + lane) = (uint8_t)(int8_t)q;
       } else {
         const int hi = __shfl_down_sync(0xffffffffu, q, 1);
-        if ((lane & 1) == 0) {
-          const int byte = 16 * g + (lane >> 1);
-          dst[(int64_t)(byte >> 4) * piece_stride + (byte & 15)] =
-              (uint8_t)((q & 15) | ((hi & 15) << 4));
-        }
+        if ((lane & 1) == 0) *code_at(16 * g + (lane >> 1)) = (uint8_t)((q & 15) | ((hi & 15) << 4));
       }
     }
   }

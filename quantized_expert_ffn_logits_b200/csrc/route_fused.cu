@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
   extern __shared__ float part[];                 // [T][C] chunk partials of this expert
   __shared__ uint32_t masks[1024];
   __shared__ int32_t offs[1024];
+  __shared__ int32_t aidx[1024];
   __shared__ int32_t sel[32 * 32];
   __shared__ int32_t wsum[8], fsum[8];
   __shared__ float red[8];
@@ -222,6 +223,7 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
     const int c = __popc(masks[x]);
     offs[x] = run;
     r.g.offsets[x] = run;
+    aidx[x] = frun;
     if (c > 0) {
       r.g.act_expert[frun] = x;
       r.g.act_begin[frun] = run;
@@ -239,7 +241,9 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
     const int ee = sel[p];
     if (ee < 0 || ee >= E) continue;
     const int t = p / k;
-    r.g.perm[offs[ee] + __popc(masks[ee] & ((1u << t) - 1u))] = p;
+    const int rank = __popc(masks[ee] & ((1u << t) - 1u));
+    r.g.perm[offs[ee] + rank] = p;
+    if (r.g.act_rows && rank < 8) r.g.act_rows[aidx[ee] * 8 + rank] = t;
   }
   if (tid == 0) *r.ticket = 0u;
 }

@@ -200,6 +200,7 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
                                                   int E, Grouping g, uint32_t* masks,
                                                   int32_t* base, int* status, int reset_status) {
   __shared__ int32_t off_s[1024];
+  __shared__ int32_t aidx_s[1024];
   __shared__ int32_t wsum[32], fsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
@@ -269,6 +270,7 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
     const int excl = incl - v;
     off_s[tid] = excl;
     g.offsets[tid] = excl;
+    aidx_s[tid] = inclf - 1;
     if (f) {
       g.act_expert[inclf - 1] = tid;
       g.act_begin[inclf - 1] = excl;
@@ -287,8 +289,9 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
       const int e = idx[(int64_t)t * k + j];
       if (e < 0 || e >= E) continue;
       const uint32_t m = __ldcg(masks + (int64_t)c * E + e);
-      const int pos = off_s[e] + __ldcg(base + (int64_t)c * E + e) + __popc(m & ((1u << lane) - 1u));
-      g.perm[pos] = t * k + j;
+      const int rank = __ldcg(base + (int64_t)c * E + e) + __popc(m & ((1u << lane) - 1u));
+      g.perm[off_s[e] + rank] = t * k + j;
+      if (g.act_rows && rank < 8) g.act_rows[aidx_s[e] * 8 + rank] = t;
     }
   }
 }

@@ -128,21 +128,29 @@ def test_blob_decodes_to_codes_and_scales(wbits, g32):
         return np.stack([((b & 15) ^ 8) - 8, (((b >> 4) & 15) ^ 8) - 8], -1).reshape(rows, K).astype(np.int8)
 
     kb_gu, kb_dn = (H, I) if wbits == 8 else (H // 2, I // 2)
-    got_gu = codes(blob[off[0]:off[0] + E * 2 * I * kb_gu], E * 2 * I, 256, kb_gu, H)
-    # row order inside each 256-row block: 128 gate rows then the matching 128 up rows
-    order = np.concatenate([np.concatenate([np.arange(128 * s, 128 * s + 128),
-                                            I + np.arange(128 * s, 128 * s + 128)])
-                            for s in range(I // 128)])
+    got_gu = codes(blob[off[0]:off[0] + E * 2 * I * kb_gu], E * 2 * I, 128, kb_gu, H)
+    # row order inside each 128-row block: 64 gate rows then the matching 64 up rows
+    order = np.concatenate([np.concatenate([np.arange(64 * s, 64 * s + 64),
+                                            I + np.arange(64 * s, 64 * s + 64)])
+                            for s in range(I // 64)])
     want_gu = ex.q_gu[:, order, :].reshape(E * 2 * I, H)
     assert np.array_equal(got_gu, want_gu)
-    got_dn = codes(blob[off[1]:off[1] + E * H * kb_dn], E * H, 128, kb_dn, I)
+    # down: slabs of 64 columns, each [128-row block][piece][row][16 bytes]
+    U, HB, sb = I // 64, H // 128, kb_dn // (I // 64)
+    dn = blob[off[1]:off[1] + E * H * kb_dn].reshape(E, U, HB, sb // 16, 128, 16)
+    dn = dn.transpose(0, 2, 4, 1, 3, 5).reshape(E * H, kb_dn)
+    if wbits == 8:
+        got_dn = dn.view(np.int8).reshape(E * H, I)
+    else:
+        b16 = dn.astype(np.int16)
+        got_dn = np.stack([((b16 & 15) ^ 8) - 8, (((b16 >> 4) & 15) ^ 8) - 8], -1).reshape(E * H, I)
     assert np.array_equal(got_dn, ex.q_dn.reshape(E * H, I))
     if g32:
         sg = blob[off[2]:off[2] + E * 2 * I * (H // 32) * 2].view(np.float16).astype(np.float32)
-        sg = sg.reshape(E * 2 * I // 256, H // 32, 256).transpose(0, 2, 1).reshape(E, 2 * I, H // 32)
+        sg = sg.reshape(E * 2 * I // 128, H // 32, 128).transpose(0, 2, 1).reshape(E, 2 * I, H // 32)
         assert np.array_equal(sg, ex.s_gu[:, order, :])
         sd = blob[off[3]:off[3] + E * H * (I // 32) * 2].view(np.float16).astype(np.float32)
-        sd = sd.reshape(E * H // 128, I // 32, 128).transpose(0, 2, 1).reshape(E, H, I // 32)
+        sd = sd.reshape(E, U, HB, 2, 128).transpose(0, 2, 4, 1, 3).reshape(E, H, I // 32)
         assert np.array_equal(sd, ex.s_dn)
     else:
         sg = blob[off[2]:off[2] + E * 2 * I * 4].view(np.float32).reshape(E, 2 * I)

@@ -106,8 +106,10 @@ def test_layer_forward_matches_oracle(name, T):
 
 
 @pytest.mark.parametrize("name,T", [("olmoe_int8", 8), ("glm_int4", 4), ("e512_int4", 64)])
-def test_down_stage_values_bit_exact(name, T):
-    """The down projection's per-row stage values follow the same canonical chain."""
+def test_down_stage_values_close(name, T):
+    """Per-pair down values: fp32 sums of the per-slab shares (any order) against the
+    oracle's fp64 down projection of the same quantized h (the int32 dots themselves are
+    pinned bit-exact through moe_expert_group_dots)."""
     m = M()
     case = S.Case.make(REDUCED[name], T)
     g, cfg, y, ws, v = _run_layer(case, m.MOE_FLAG_DEBUG)
@@ -115,7 +117,7 @@ def test_down_stage_values_bit_exact(name, T):
     P, H = T * case.cfg.top_k, case.cfg.H
     perm = _np(m.workspace_view(ws, v["perm"], torch.int32, (P,)))
     ye = _np(m.workspace_view(ws, v["y_pair"], torch.float32, (P, H)))
-    assert np.array_equal(ye, ref["ye32"][perm])
+    assert_close_y(ye, ref["ye"][perm], "per-pair down values")
 
 
 @pytest.mark.parametrize("name,T", [("olmoe_int8", 33), ("glm_int4", 4), ("e512_int4", 100)])
