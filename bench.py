@@ -82,6 +82,15 @@ def gateup_bytes(cfg, T, n_active):
     return b
 
 
+def expert_bytes(cfg, T, n_active):
+    """Algorithmic bytes of the expert kernel: the unique experts' blobs (gate/up and down,
+    codes and scales) and the shared expert's; activations and h stay on chip or in L2."""
+    b = n_active * (blob_row_bytes(cfg, cfg.H, 2 * cfg.I) + blob_row_bytes(cfg, cfg.I, cfg.H))
+    if cfg.shared_I:
+        b += blob_row_bytes(cfg, cfg.H, 2 * cfg.shared_I) + blob_row_bytes(cfg, cfg.shared_I, cfg.H)
+    return b
+
+
 def layer_bytes(cfg, T, n_active):
     """Algorithmic bytes of one layer forward: unique experts' blobs (gate/up and down), the
     shared expert, the router weight, x in and y out (fp32)."""
@@ -228,14 +237,15 @@ def oracle_sampler(cfg, T, seed_base=7_000_000):
     return run_units, desc, cores
 
 
-def time_oracle(cfg, T, budget_s=12.0):
+def time_oracle(cfg, T, budget_s=20.0):
     run_units, desc, cores = oracle_sampler(cfg, T)
     per_tok = cfg.top_k + (1 if cfg.shared_I else 0)
     t0 = time.perf_counter()
     run_units(per_tok)
     t1 = time.perf_counter() - t0
-    n = max(per_tok, int(budget_s / max(t1, 1e-3)) * per_tok)
-    n = min(n, 64 * per_tok)
+    # about budget_s of CPU work (the first, single-token call sizes it)
+    n = max(per_tok, int(budget_s / max(t1, 1e-4)) * per_tok)
+    n = min(n, 100_000 * per_tok)
     t0 = time.perf_counter()
     toks = run_units(n)
     el = time.perf_counter() - t0
@@ -436,15 +446,19 @@ def gpu_arm(args, cfg, T):
     value = world * T * args.steps / (ms_max / 1e3)
     peaks, peak_src = load_peaks()
     n_act = float(np.mean(n_active_of))
-    # dominant kernel: gate/up (weight streaming, HBM-bound)
+    # dominant kernel: the expert kernel (weight streaming, HBM-bound); with group-32
+    # activations one launch runs gate/up, SwiGLU, h quantization, down and the combine, and
+    # the gate/up stage events bracket it
+    fused = cfg.act == "g32_f16"
     gu_us = stage_us["gate_up"]
-    gu_bytes = float(np.mean([gateup_bytes(cfg, T, a) for a in n_active_of]))
+    gu_bytes = float(np.mean([(expert_bytes if fused else gateup_bytes)(cfg, T, a) for a in n_active_of]))
     roof = None
     if gu_us:
         ach = gu_bytes / (gu_us * 1e-6) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic_from_profiles(cfg, T),
-                "kernel": "k_gateup (gate/up + SwiGLU + h quantization)",
+                "kernel": ("k_expert_ring (gate/up, SwiGLU, h quantization, down, weighted combine)"
+                           if fused else "k_expert_ring (gate/up pass)"),
                 "bytes_per_launch": int(gu_bytes), "us_per_launch": round(gu_us, 3),
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6.65 TB/s"}
     lb = float(np.mean([layer_bytes(cfg, T, a) for a in n_active_of]))
@@ -518,11 +532,11 @@ def gpu_arm(args, cfg, T):
 
 
 def traffic_from_profiles(cfg, T):
-    """DRAM bytes per launch of the gate/up kernel from the committed ncu summary, if it was
-    taken on this workload with the current kernel source; else None."""
+    """DRAM bytes (read + write) per launch of the expert kernel from the committed ncu
+    summary, if it was taken on this workload with the current kernel source; else None."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "k_gateup_traffic.json")
-    src = os.path.join(ROOT, "quantized_expert_ffn_logits_b200", "csrc", "expert_gemv.cu")
+    path = os.path.join(ROOT, "profiles", "k_expert_ring_traffic.json")
+    src = os.path.join(ROOT, "quantized_expert_ffn_logits_b200", "csrc", "expert_stream.cu")
     try:
         with open(path) as f:
             d = json.load(f)

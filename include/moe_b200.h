@@ -222,10 +222,12 @@ MOE_API size_t moe_layer_workspace_bytes(int32_t T, const moe_expert_blob* exper
  * library leaves it consistent after every call. Calls that share a workspace must be ordered
  * on one stream.
  * Launch sequence: for T <= 32 one routing kernel (activation quantization, logits, top-k and
- * grouping; the last CTA to finish its logit does the selection), then one gate/up kernel and
- * one down kernel, each covering the routed and the shared experts; larger T routes through
- * four kernels. Kernels use programmatic dependent launch, so under stream capture the graph
- * gets programmatic edges. */
+ * grouping; the last CTA to finish its logit does the selection), larger T four; then, with
+ * group-32 activations, one expert kernel that covers the routed and the shared experts: per
+ * work unit (expert, 64 intermediate indices) gate/up, SwiGLU, h quantization and the unit's
+ * share of the down projection, added into y. With per-token activation scales h needs all of
+ * I first: gate/up, h quantization, then down as separate launches. Kernels use programmatic
+ * dependent launch, so under stream capture the graph gets programmatic edges. */
 MOE_API moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
                              const float* router_bias, const moe_expert_blob* experts,
                              const moe_expert_blob* shared, const moe_route_cfg* cfg, float* y,
@@ -237,9 +239,10 @@ enum {
   MOE_STAGE_ROUTER = 1,    /* router logits */
   MOE_STAGE_TOPK = 2,      /* top-k selection and weights (grouping too when T = 1) */
   MOE_STAGE_GROUP = 3,     /* batch-union grouping (T > 1) */
-  MOE_STAGE_GATE_UP = 4,   /* gate/up + SwiGLU (+ h quantization for group-32 activations) */
+  MOE_STAGE_GATE_UP = 4,   /* gate/up + SwiGLU (group-32 activations: the whole expert kernel,
+                              h quantization, down projection and combine included) */
   MOE_STAGE_QUANT_H = 5,   /* h quantization (per-token activation scales only) */
-  MOE_STAGE_DOWN = 6,      /* down projection + weighted combine */
+  MOE_STAGE_DOWN = 6,      /* down projection + weighted combine (per-token scales only) */
   MOE_STAGE_COUNT = 7
 };
 
@@ -303,8 +306,11 @@ MOE_API moe_status moe_expert_group_dots(const moe_expert_blob* blob, int32_t wh
                                  int32_t* dots, void* stream);
 
 /* The control block's int32 words [2] and [3] record the first bounded wait that gave up
- * during the last call (MOE_ERR_TIMEOUT): [2] = kernel (1 gate/up, 2 down) | role (1 producer,
- * 2 consumer) << 4 | pipeline stage << 8, [3] = the CTA index; both 0 otherwise.
+ * during the last call (MOE_ERR_TIMEOUT): [2] = pass (1 gate/up, 2 down) | wait << 4 | ring
+ * stage or buffer << 8, with wait 0 = producer waiting for a free stage, 1 = consumer waiting
+ * for a chunk, 2 / 4 = producer draining chunks / activation copies before exit, 3 = producer
+ * waiting for a free activation buffer, 5 = consumer waiting for activation rows;
+ * [3] = the CTA index; both 0 otherwise.
  * Reads and clears the device status word of a moe_layer_forward / moe_permute workspace.
  * Synchronizes `stream`. Returns MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT as
  * recorded by the kernels, or MOE_ERR_CUDA if the copy fails. */

@@ -2,6 +2,7 @@
 // the launch sequence of the layer forward.
 #include <cstdint>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 
 #include "../../include/moe_b200.h"

@@ -94,6 +94,12 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
+// y[0..3] += (a, b, c, d): one 16-byte reduction (sm_90+), p 16-byte aligned.
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 // --------------------------------------------------------------- integer dots
 // Signed x signed 4-way byte dot.
 __device__ __forceinline__ int dp4a_ss(uint32_t a, uint32_t b, int c) {

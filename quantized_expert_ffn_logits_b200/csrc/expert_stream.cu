@@ -162,6 +162,12 @@ __device__ __forceinline__ int act_row(const ExpertArgs& a, bool gateup, const U
   return t;
 }
 
+// First chunk of a unit's down pass: units start at different 128-row blocks, so the
+// CTAs' atomic adds into y spread over the output instead of meeting on the same lines.
+__device__ __forceinline__ int down_rotation(const Unit& U, int nch) {
+  return (int)(((unsigned)U.sub * 7u + (unsigned)U.ai * 3u) % (unsigned)nch);
+}
+
 // Record the first wait that gave up: word 2 = kernel | role << 4 | stage << 8, word 3 = CTA.
 __device__ __forceinline__ void wait_failed(int* status, int kernel, int role, int stage) {
   if (!status) return;
@@ -212,6 +218,7 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
   int* status = A.x[0][0].status;
   uint32_t c = 0, pidx = 0, nacts = 0;      // chunks, passes, activation copies issued
   bool ok = true;
+  const uint64_t once = policy_evict_first();
   auto push = [&](const uint8_t* w, uint32_t wbytes, const uint8_t* sc, uint32_t sbytes) -> bool {
     const int st = c % kNS;
     if (c >= (uint32_t)kNS && !mbar_wait(&R.empty[st], ((c / kNS) - 1) & 1)) {
@@ -219,8 +226,8 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
       return false;
     }
     mbar_arrive_expect_tx(&R.full[st], wbytes + sbytes);
-    bulk_load(R.ring + st * (kSP * kPiece), w, wbytes, &R.full[st]);
-    if (sbytes) bulk_load(R.sring + st * (kSP * 256), sc, sbytes, &R.full[st]);
+    bulk_load_hint(R.ring + st * (kSP * kPiece), w, wbytes, &R.full[st], once);
+    if (sbytes) bulk_load_hint(R.sring + st * (kSP * 256), sc, sbytes, &R.full[st], once);
     ++c;
     return true;
   };
@@ -268,7 +275,10 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
         const int64_t slab0 = ((int64_t)U.e * (d.b.I / 64) + U.sub) * HB;   // first 128-row block
         const uint8_t* wsrc = d.b.dn_w + slab0 * PPU * kPiece;
         const uint8_t* ssrc = WG32 ? d.b.dn_s + slab0 * 512 : d.b.dn_s + (int64_t)U.e * d.b.H * 4;
-        for (int hb0 = 0; hb0 < HB && ok; hb0 += NBC) {
+        const int nch = (HB + NBC - 1) / NBC;
+        const int rot = down_rotation(U, nch);
+        for (int j = 0; j < nch && ok; ++j) {
+          const int hb0 = ((j + rot) % nch) * NBC;
           const int nb = min(NBC, HB - hb0);
           ok = push(wsrc + (int64_t)hb0 * PPU * kPiece, (uint32_t)(nb * PPU * kPiece), ssrc + (int64_t)hb0 * 512,
                     (uint32_t)nb * 512);
@@ -459,7 +469,7 @@ __device__ __forceinline__ void ring_consume(int K, int m, int tm, const Ring& R
 // down value). hx: the pass's h codes [tm][64] (int4 weights: each 8-byte word
 // de-interleaved), hxs: per-group code sums [tm][2] (int4), hs: h scales [tm][2].
 template <int WBITS, bool WG32, bool AG32>
-__device__ __forceinline__ void down_consume(int H, int m, const Ring& R, uint32_t& c, const uint8_t* hx,
+__device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& R, uint32_t& c, const uint8_t* hx,
                                              const int* hxs, const float* hs, const int* toks,
                                              const float* wts, float* y, float* dbg, int slot0,
                                              volatile int* abort, int* status) {
@@ -468,7 +478,9 @@ __device__ __forceinline__ void down_consume(int H, int m, const Ring& R, uint32
   constexpr int RPT = NBC * kRows / (32 * kCW);   // rows per thread of a full chunk
   const int lane = threadIdx.x & 31;
   const int HB = H / kRows;
-  for (int hb0 = 0; hb0 < HB; hb0 += NBC, ++c) {
+  const int nch = (HB + NBC - 1) / NBC;
+  for (int j = 0; j < nch; ++j, ++c) {
+    const int hb0 = ((j + rot) % nch) * NBC;
     const int nb = min(NBC, HB - hb0);
     const int st = c % kNS;
     bool ok = *abort == 0;
@@ -530,7 +542,12 @@ __device__ __forceinline__ void down_consume(int H, int m, const Ring& R, uint32
           else
             v = __fmul_rn(__fmul_rn(__int2float_rn(d0 + d1), hs0), c0s[k]);
           const int n = (hb0 + b) * kRows + r;
-          atomicAdd(yq + n, wq * v);
+          // lanes 4j .. 4j+3 hold rows n .. n+3: one 16-byte reduction per four rows
+          const float wv = wq * v;
+          const float w1 = __shfl_down_sync(0xffffffffu, wv, 1);
+          const float w2 = __shfl_down_sync(0xffffffffu, wv, 2);
+          const float w3 = __shfl_down_sync(0xffffffffu, wv, 3);
+          if ((lane & 3) == 0) red_add_v4(yq + n, wv, w1, w2, w3);
           if (dq) atomicAdd(dq + n, v);
         }
       }
@@ -745,7 +762,9 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
           named_bar(1, 32 * kCW);
           hx = hqd;
         }
-        down_consume<WBITS, WG32, AG32>(d.b.H, m, R, c, hx, hxs, hs, toks, wts, d.y, d.dbg_a, c0, abort, status);
+        const int rot = down_rotation(U, (d.b.H / kRows + kSP / (WBITS == 8 ? 4 : 2) - 1) / (kSP / (WBITS == 8 ? 4 : 2)));
+        down_consume<WBITS, WG32, AG32>(d.b.H, m, rot, R, c, hx, hxs, hs, toks, wts, d.y, d.dbg_a, c0, abort,
+                                        status);
       }
     }
   }

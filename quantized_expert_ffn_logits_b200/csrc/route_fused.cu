@@ -134,8 +134,19 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
       const int t = i / E, x = i - t * E;
       const float kv = skey[i];
       const float* kt = skey + t * E;
-      int rank = 0;
-      for (int j = 0; j < E; ++j) {
+      int rank = 0, j = 0;
+      if ((E & 3) == 0) {
+        const float4* kt4 = reinterpret_cast<const float4*>(kt);
+#pragma unroll 4
+        for (; j < E; j += 4) {
+          const float4 q = kt4[j >> 2];
+          rank += (q.x > kv) | ((q.x == kv) & (j < x));
+          rank += (q.y > kv) | ((q.y == kv) & (j + 1 < x));
+          rank += (q.z > kv) | ((q.z == kv) & (j + 2 < x));
+          rank += (q.w > kv) | ((q.w == kv) & (j + 3 < x));
+        }
+      }
+      for (; j < E; ++j) {
         const float kj = kt[j];
         rank += (kj > kv) | ((kj == kv) & (j < x));
       }
@@ -176,6 +187,34 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
                                      r.rsf, r.idx + (int64_t)t * k, r.w + (int64_t)t * k, r.status);
       if (lane < k) sel[t * k + lane] = my_e;
     }
+  }
+  __syncthreads();
+  if (T == 1) {
+    // one token: the active experts are its k distinct selections, one slot each, in
+    // ascending expert order
+    if (tid < k) {
+      const int ee = sel[tid];
+      int pos = 0;
+      for (int j = 0; j < k; ++j) pos += sel[j] < ee;
+      if (ee >= 0 && ee < E) {
+        r.g.act_expert[pos] = ee;
+        r.g.act_begin[pos] = pos;
+        r.g.perm[pos] = tid;
+        if (r.g.act_rows) r.g.act_rows[pos * 8] = 0;
+      }
+    }
+    for (int x = tid; x < E; x += 256) {
+      int cnt = 0;
+      for (int j = 0; j < k; ++j) cnt += sel[j] < x;
+      r.g.offsets[x] = cnt;
+    }
+    if (tid == 0) {
+      r.g.offsets[E] = k;
+      *r.g.n_active = k;
+      r.g.act_begin[k] = k;
+      *r.ticket = 0u;
+    }
+    return;
   }
   for (int x = tid; x < E; x += 256) masks[x] = 0u;
   __syncthreads();
