@@ -26,7 +26,7 @@ MOE_W_INT8, MOE_W_INT4 = 0, 1
 MOE_SCALE_ROW_F32, MOE_SCALE_G32_F16 = 0, 1
 MOE_ACT_TOKEN_F32, MOE_ACT_G32_F16 = 0, 1
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID_NOAUX_TC = 0, 1
-MOE_FLAG_DEBUG, MOE_FLAG_FORCE_GEMV = 1, 2
+MOE_FLAG_DEBUG, MOE_FLAG_FORCE_GEMV, MOE_FLAG_FORCE_MMA = 1, 2, 4
 
 WTYPES = {"int8": MOE_W_INT8, "int4": MOE_W_INT4}
 WSCALES = {"row_f32": MOE_SCALE_ROW_F32, "g32_f16": MOE_SCALE_G32_F16}

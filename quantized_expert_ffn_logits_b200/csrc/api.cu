@@ -76,11 +76,14 @@ moe_status check_cfg(const moe_route_cfg* c, int32_t E) {
 struct Layout {
   int64_t status, qx, sx, logits, idx, w, offsets, perm, n_active, act_expert, act_begin, act_rows;
   int64_t masks, base, qh, sh, hbuf, dbg_gate, dbg_up, dbg_y, total;
+  // tensor-core path (T > 32, group-32 weights and activations)
+  int64_t mm_tiles, mm_ntiles, mm_xa, mm_xs, mm_xsum, mm_ha, mm_hs, mm_hsum;
+  int32_t mm_max_tiles, mm_min_tokens, mm_hk;
   int64_t qh_sh, sh_sh, hbuf_sh, dbg_gate_sh, dbg_up_sh, dbg_y_sh;   // shared-expert rows
 };
 
 Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k, int32_t ag32,
-              bool debug) {
+              bool debug, bool mma, bool force_mma) {
   Layout L;
   int64_t o = 0;
   auto take = [&](int64_t bytes) {
@@ -131,13 +134,39 @@ Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k,
     L.dbg_gate = L.dbg_up = L.dbg_y = -1;
     L.dbg_gate_sh = L.dbg_up_sh = L.dbg_y_sh = -1;
   }
+  L.mm_max_tiles = 0;
+  L.mm_min_tokens = force_mma ? 1 : moe::kMmaMinTokens;
+  L.mm_hk = std::max(I, Is);
+  L.mm_tiles = L.mm_ntiles = L.mm_xa = L.mm_xs = L.mm_xsum = L.mm_ha = L.mm_hs = L.mm_hsum = -1;
+  if (mma) {
+    // tiles of 128 slots: every qualifying expert wastes at most one partial tile
+    const int64_t n_exp = std::min<int64_t>(E, P / L.mm_min_tokens);
+    const int64_t mt = (P + 127) / 128 + n_exp + (Is ? (T + 127) / 128 : 0) + 1;
+    L.mm_max_tiles = (int32_t)mt;
+    L.mm_tiles = take(mt * 16);
+    L.mm_ntiles = take(4);
+    L.mm_xa = take(mt * 128 * H);
+    L.mm_xs = take(mt * (H / 32) * 128 * 2);
+    L.mm_xsum = take(mt * (H / 32) * 128 * 4);
+    L.mm_ha = take(mt * 128 * L.mm_hk);
+    L.mm_hs = take(mt * (L.mm_hk / 32) * 128 * 2);
+    L.mm_hsum = take(mt * (L.mm_hk / 32) * 128 * 4);
+  }
   L.total = o;
   return L;
+}
+
+// Calls with more than kFusedRouteMaxT tokens, group-32 weights and activations send experts
+// with many pairs to the tensor-core GEMMs.
+bool use_mma(int32_t T, const moe_expert_blob* experts, const moe_route_cfg* cfg) {
+  return T > kFusedRouteMaxT && cfg->act == MOE_ACT_G32_F16 && experts->wscale == MOE_SCALE_G32_F16 &&
+         (cfg->flags & MOE_FLAG_FORCE_GEMV) == 0;
 }
 
 struct LayerPlan {
   BlobOffsets eo, so;
   int32_t Is;
+  bool mma;      // experts with many tokens take the tensor-core path
   Layout L;
 };
 
@@ -157,8 +186,10 @@ moe_status plan_layer(int32_t T, const moe_expert_blob* experts, const moe_exper
       return MOE_ERR_UNSUPPORTED;
     p.Is = shared->inter;
   }
+  p.mma = use_mma(T, experts, cfg);
   p.L = layout(T, experts->n_experts, experts->hidden, experts->inter, p.Is, cfg->top_k,
-               cfg->act == MOE_ACT_G32_F16, (cfg->flags & MOE_FLAG_DEBUG) != 0);
+               cfg->act == MOE_ACT_G32_F16, (cfg->flags & MOE_FLAG_DEBUG) != 0, p.mma,
+               (cfg->flags & MOE_FLAG_FORCE_MMA) != 0);
   return MOE_OK;
 }
 
@@ -314,7 +345,8 @@ moe_status moe_layer_debug_views(int32_t T, const moe_expert_blob* experts,
   if (total == 0) return MOE_ERR_UNSUPPORTED;
   const int32_t Is = shared ? shared->inter : 0;
   const Layout L = layout(T, experts->n_experts, experts->hidden, experts->inter, Is, cfg->top_k,
-                          cfg->act == MOE_ACT_G32_F16, (cfg->flags & MOE_FLAG_DEBUG) != 0);
+                          cfg->act == MOE_ACT_G32_F16, (cfg->flags & MOE_FLAG_DEBUG) != 0,
+                          use_mma(T, experts, cfg), (cfg->flags & MOE_FLAG_FORCE_MMA) != 0);
   out->status = L.status;
   out->q_x = L.qx;
   out->s_x = L.sx;
@@ -511,19 +543,70 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   // the down kernels add each unit's share of a pair's down value into the pair's view
   if (L.dbg_y >= 0)
     keep(cudaMemsetAsync(ws + L.dbg_y, 0, (size_t)((int64_t)(T * k + T) * H * 4), st), "debug view reset");
+  // experts with many slots: tensor-core GEMMs (tile list, operand gather, gate/up, down)
+  const int mma_min = p.mma ? L.mm_min_tokens : 0x7fffffff;
+  auto launch_mma = [&](bool down) {
+    moe::MmaArgs m;
+    std::memset(&m, 0, sizeof(m));
+    m.b[0] = bv;
+    m.b[1] = shared ? sa.b : bv;
+    m.tiles = static_cast<const int4*>(at(L.mm_tiles));
+    m.n_tiles = static_cast<const int32_t*>(at(L.mm_ntiles));
+    m.max_tiles = L.mm_max_tiles;
+    m.a_ops = static_cast<const uint8_t*>(at(L.mm_xa));
+    m.a_scales = static_cast<const __half*>(at(L.mm_xs));
+    m.a_xsum = static_cast<const int32_t*>(at(L.mm_xsum));
+    m.h_xsum = static_cast<int32_t*>(at(L.mm_hsum));
+    m.h_ops = static_cast<uint8_t*>(at(L.mm_ha));
+    m.h_scales = static_cast<__half*>(at(L.mm_hs));
+    m.hk = L.mm_hk;
+    m.qh[0] = ra.qh;
+    m.qh[1] = shared ? sa.qh : ra.qh;
+    m.sh[0] = ra.sh;
+    m.sh[1] = shared ? sa.sh : ra.sh;
+    m.dbg_a[0] = ra.dbg_a;
+    m.dbg_a[1] = shared ? sa.dbg_a : nullptr;
+    m.dbg_b[0] = ra.dbg_b;
+    m.dbg_b[1] = shared ? sa.dbg_b : nullptr;
+    m.perm = g.perm;
+    m.wts = wts;
+    m.y = y;
+    m.dbg_y[0] = rd.dbg_a;
+    m.dbg_y[1] = shared ? sd.dbg_a : nullptr;
+    m.T = T;
+    m.k = k;
+    m.status = status;
+    if (!down) {
+      keep(moe::launch_mma_plan(g, E, T, shared ? 1 : 0, L.mm_min_tokens, L.mm_max_tiles,
+                                static_cast<int4*>(at(L.mm_tiles)), static_cast<int32_t*>(at(L.mm_ntiles)),
+                                status, st),
+           "tensor-core tile plan");
+      keep(moe::launch_mma_gather(static_cast<const int8_t*>(at(L.qx)), static_cast<const __half*>(at(L.sx)),
+                                  m.tiles, m.n_tiles, g.perm, k, T, H, L.mm_max_tiles,
+                                  static_cast<uint8_t*>(at(L.mm_xa)), static_cast<__half*>(at(L.mm_xs)),
+                                  static_cast<int32_t*>(at(L.mm_xsum)), status, st),
+           "tensor-core operand gather");
+      keep(moe::launch_expert_mma(true, m, st), "tensor-core gate/up kernel");
+    } else {
+      keep(moe::launch_expert_mma(false, m, st), "tensor-core down kernel");
+    }
+  };
   if (moe::experts_fusable(ra, sap)) {
     // 4+5 in one persistent grid: per unit (expert, 64 intermediate indices) the gate/up
     // pass, SwiGLU and h quantization, then the unit's share of the down projection
     mk.begin(MOE_STAGE_GATE_UP);
-    keep(moe::launch_experts(2, ra, sap, rd, sdp, st), "expert kernel");
+    if (p.mma) launch_mma(false);
+    keep(moe::launch_experts(2, ra, sap, rd, sdp, mma_min, st), "expert kernel");
     mk.end(MOE_STAGE_GATE_UP);
-    for (int sg = MOE_STAGE_QUANT_H; sg <= MOE_STAGE_DOWN; ++sg) {
-      mk.begin(sg);
-      mk.end(sg);
-    }
+    mk.begin(MOE_STAGE_DOWN);
+    if (p.mma) launch_mma(true);
+    mk.end(MOE_STAGE_DOWN);
+    mk.begin(MOE_STAGE_QUANT_H);
+    mk.end(MOE_STAGE_QUANT_H);
   } else {
     mk.begin(MOE_STAGE_GATE_UP);
-    keep(moe::launch_experts(0, ra, sap, rd, sdp, st), "gate/up kernel");
+    if (p.mma) launch_mma(false);
+    keep(moe::launch_experts(0, ra, sap, rd, sdp, mma_min, st), "gate/up kernel");
     mk.end(MOE_STAGE_GATE_UP);
     mk.begin(MOE_STAGE_QUANT_H);
     if (!ag32) {
@@ -536,7 +619,8 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     }
     mk.end(MOE_STAGE_QUANT_H);
     mk.begin(MOE_STAGE_DOWN);
-    keep(moe::launch_experts(1, ra, sap, rd, sdp, st), "down kernel");
+    keep(moe::launch_experts(1, ra, sap, rd, sdp, mma_min, st), "down kernel");
+    if (p.mma) launch_mma(true);
     mk.end(MOE_STAGE_DOWN);
   }
   if (err != cudaSuccess) return cuda_fail(err_where, err);
@@ -570,6 +654,7 @@ int32_t moe_layer_kernel_count(int32_t T, const moe_expert_blob* experts,
   if (moe_layer_workspace_bytes(T, experts, shared, cfg) == 0) return -1;
   if (T == 0) return 0;
   int n = T <= kFusedRouteMaxT ? 1 : 4;        // routing (fused, or quantize/logits/top-k/grouping)
+  if (use_mma(T, experts, cfg)) n += 4;                                     // tensor-core tile plan, gather, gate/up, down
   if (cfg->act == MOE_ACT_G32_F16) return n + 1;   // gate/up and down of all experts in one grid
   n += 1;                                       // gate/up, routed and shared experts in one grid
   if (cfg->act != MOE_ACT_G32_F16) n += 1 + (shared ? 1 : 0);   // h quantization

@@ -47,6 +47,22 @@ __device__ __forceinline__ float cswiglu(float g, float u) {
   return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, cexp(-g))), u);
 }
 
+// Exact int -> float for |v| < 2^22 with two full-rate operations: the bits of 1.5 * 2^23
+// plus v are the float 1.5 * 2^23 + v (the exponent stays 2^23, so the ulp is 1); subtracting
+// 1.5 * 2^23 leaves v exactly. Group dots stay below 32 * 127 * 127 < 2^19.
+__device__ __forceinline__ float exact_i2f(int v) {
+  return __fsub_rn(__int_as_float(0x4B400000 + v), 12582912.0f);
+}
+// The same with the bias folded in: (float)(a + bias_a) for kb = 0x4B400000 + bias_a.
+__device__ __forceinline__ float2 exact_i2f2k(int a, int b, int kb) {
+  return __fadd2_rn(make_float2(__int_as_float(kb + a), __int_as_float(kb + b)),
+                    make_float2(-12582912.0f, -12582912.0f));
+}
+__device__ __forceinline__ float2 exact_i2f2(int a, int b) {
+  return __fadd2_rn(make_float2(__int_as_float(0x4B400000 + a), __int_as_float(0x4B400000 + b)),
+                    make_float2(-12582912.0f, -12582912.0f));
+}
+
 // ---------------------------------------------------------------- quantization
 __device__ __forceinline__ float f16_round(float d) { return __half2float(__float2half_rn(d)); }
 
@@ -78,6 +94,16 @@ __device__ __forceinline__ int warp_sum_int(int v) {
 
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+// Record the first bounded wait that gave up: status word = timeout, word 2 = kernel | wait
+// << 4 | stage << 8, word 3 = the CTA.
+__device__ __forceinline__ void wait_failed(int* status, int kernel, int role, int stage) {
+  if (!status) return;
+  if (atomicCAS(status, 0, kStatusTimeout) == 0) {
+    status[2] = kernel | (role << 4) | (stage << 8);
+    status[3] = (int)blockIdx.x;
+  }
 }
 
 // Streaming 128-bit load of read-only data (no L1 allocation: weights are read once).

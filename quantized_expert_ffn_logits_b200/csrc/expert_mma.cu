@@ -1,0 +1,612 @@
+// expert_mma.cu -- tensor-core path for experts with many tokens (prefill, large batches).
+//
+// An expert that receives at least kMmaMinTokens (token, expert) pairs in a call is a dense
+// contraction: its pairs are cut into tiles of 128 slots and every (tile, 128-row weight
+// block) pair runs as an M = 128 (slots) x N = 128 (rows) integer GEMM on the sm_100a tensor
+// cores (tcgen05.mma kind::i8, int32 in tensor memory). One MMA with K = 32 is exactly one
+// quantization group, so its accumulator is the exact int32 dot I_g of every (slot, row) in
+// the tile; the epilogue then runs the ordered fp32 chain acc = fma((float)I_g, c_g, acc)
+// with c_g = s_w,g * s_x,g per element -- the same arithmetic as the weight-streaming path
+// and the oracle (GLM-5.2 colibri page, "Integer-dot kernels"; "Batch-union MoE": every
+// selected expert's weights are read once per tile of 128 of its tokens).
+//
+// Gate/up tiles (N = the 64 gate rows and 64 up rows of one block) end with SwiGLU and Q8_0
+// h quantization per group of 32 -- one thread holds a slot's 32 indices of a group -- and
+// write h in the operand layout the down GEMM reads; down tiles (N = 128 output rows) add
+// w * v into y with 16-byte reductions.
+//
+// The per-group epilogue (three fp32 operations per element per group against one 32-wide
+// MMA step) bounds this path, not the tensor cores: see the measurement notes.
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.cuh"
+#include "tma.cuh"
+#include "umma.cuh"
+
+namespace moe {
+
+// -------------------------------------------------------------------- tile plan
+// tiles[i] = {active expert index (-1: the shared expert), first slot, valid slots, expert}.
+// Routed experts with at least min_tokens slots, in active order, then the shared expert's
+// tokens (when has_shared and T >= min_tokens). One CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) k_mma_plan(const int32_t* __restrict__ n_active,
+                                                   const int32_t* __restrict__ act_expert,
+                                                   const int32_t* __restrict__ act_begin, int E, int T,
+                                                   int has_shared, int min_tokens, int max_tiles,
+                                                   int4* __restrict__ tiles, int32_t* __restrict__ n_tiles,
+                                                   int* status) {
+  __shared__ int wsum[32];
+  __shared__ int carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_wait();
+  pdl_trigger();
+  const int na = min(*n_active, E);
+  if (tid == 0) carry = 0;
+  __syncthreads();
+  for (int base = 0; base < na; base += 1024) {
+    const int ai = base + tid;
+    int cnt = 0, s0 = 0, n = 0, e = 0;
+    if (ai < na) {
+      s0 = act_begin[ai];
+      n = act_begin[ai + 1] - s0;
+      e = act_expert[ai];
+      if (n >= min_tokens) cnt = (n + 127) / 128;
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const int v = wsum[lane];
+      int iv = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int x = __shfl_up_sync(0xffffffffu, iv, o);
+        if (lane >= o) iv += x;
+      }
+      wsum[lane] = iv - v;
+    }
+    __syncthreads();
+    const int first = carry + wsum[warp] + incl - cnt;
+    for (int j = 0; j < cnt; ++j) {
+      if (first + j >= max_tiles) {
+        set_status(status, kStatusDeviceCheck);
+        break;
+      }
+      tiles[first + j] = make_int4(ai, s0 + 128 * j, min(128, n - 128 * j), e);
+    }
+    __syncthreads();
+    if (tid == 1023) carry = first + cnt;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    int total = carry;
+    if (has_shared && T >= min_tokens)
+      for (int s0 = 0; s0 < T; s0 += 128) {
+        if (total >= max_tiles) {
+          set_status(status, kStatusDeviceCheck);
+          break;
+        }
+        tiles[total++] = make_int4(-1, s0, min(128, T - s0), 0);
+      }
+    *n_tiles = min(total, max_tiles);
+  }
+}
+
+// -------------------------------------------------------------------- gather
+// Operand A of the gate/up GEMM: for tile i, the q_x rows of its slots' tokens in the
+// tensor-core operand layout [tile][K/16 pieces][128 slots][16 B], their fp16 group scales
+// [tile][K/32][128] and the sum of each group's codes [tile][K/32][128] (the correction
+// for unsigned int4 weight bytes); slots past the tile's valid count are zero. One thread
+// per (tile, slot, group).
+__global__ void __launch_bounds__(256) k_mma_gather(const int8_t* __restrict__ qx, const __half* __restrict__ sx,
+                                                    const int4* __restrict__ tiles,
+                                                    const int32_t* __restrict__ n_tiles,
+                                                    const int32_t* __restrict__ perm, int k, int T, int K,
+                                                    uint8_t* __restrict__ xa, __half* __restrict__ xs,
+                                                    int32_t* __restrict__ xsum, int* status) {
+  pdl_wait();
+  pdl_trigger();
+  const int G = K / 32;
+  const int nt = *n_tiles;
+  const int64_t per_tile = (int64_t)128 * G;
+  for (int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; id < (int64_t)nt * per_tile;
+       id += (int64_t)gridDim.x * blockDim.x) {
+    const int ti = (int)(id / per_tile);
+    const int rem = (int)(id - (int64_t)ti * per_tile);
+    const int g = rem >> 7, t = rem & 127;
+    const int4 tl = tiles[ti];
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    __half s = __float2half_rn(0.0f);
+    if (t < tl.z) {
+      const int slot = tl.y + t;
+      int tok = slot;
+      if (tl.x >= 0) {
+        const int pr = perm[slot];
+        tok = (pr >= 0 && pr < T * k) ? pr / k : -1;
+      }
+      if (tok >= 0 && tok < T) {
+        const uint4* src = reinterpret_cast<const uint4*>(qx + (int64_t)tok * K + 32 * g);
+        v0 = src[0];
+        v1 = src[1];
+        s = sx[(int64_t)tok * G + g];
+      } else if (g == 0) {
+        set_status(status, kStatusDeviceCheck);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(xa) + ((int64_t)ti * 2 * G + 2 * g) * 128 + t;
+    dst[0] = v0;
+    dst[128] = v1;
+    xs[((int64_t)ti * G + g) * 128 + t] = s;
+    int sum = __dp4a((int)v0.x, 0x01010101, 0);
+    sum = __dp4a((int)v0.y, 0x01010101, sum);
+    sum = __dp4a((int)v0.z, 0x01010101, sum);
+    sum = __dp4a((int)v0.w, 0x01010101, sum);
+    sum = __dp4a((int)v1.x, 0x01010101, sum);
+    sum = __dp4a((int)v1.y, 0x01010101, sum);
+    sum = __dp4a((int)v1.z, 0x01010101, sum);
+    sum = __dp4a((int)v1.w, 0x01010101, sum);
+    xsum[((int64_t)ti * G + g) * 128 + t] = sum;
+  }
+}
+
+// -------------------------------------------------------------------- GEMM kernel
+constexpr int kMmaKC = 4;                  // groups per pipeline stage
+constexpr int kMmaNS = 4;                  // pipeline stages
+constexpr int kMmaNB = 4;                  // tensor-memory accumulator buffers (128 columns each:
+                                           // all 512; one CTA per SM), so MMAs run 4 groups ahead
+constexpr int kMmaThreads = 20 * 32;       // producer, MMA, 2 prep, 16 epilogue warps
+constexpr int kMmaEpiWarps = 16;
+
+// One pipeline stage: operand A (128 slots x 4 groups, int8), operand B (128 rows x 4 groups,
+// int8), packed int4 B as copied, the fp16 scales of both and B's scales as fp32.
+struct MmaStage {
+  static constexpr int A = 0;              // [8 pieces][128][16]
+  static constexpr int B = 16384;          // [8 pieces][128][16]
+  static constexpr int BRAW = 32768;       // [4 pieces][128][16] (int4 weights)
+  static constexpr int AS = 40960;         // [4][128] fp16
+  static constexpr int BS = 41984;         // [4][128] fp16
+  static constexpr int BSF = 43008;        // [4][128] fp32
+  static constexpr int XS = 45056;         // [4][128] int32: code sums of A's groups (int4 B)
+  static constexpr int BYTES = 47104;
+};
+// + 32 KB of slack past the last stage: an operand descriptor's furthest byte stays inside
+// this CTA's shared memory whatever its strides.
+constexpr int kMmaSmem = kMmaNS * MmaStage::BYTES + 256 + 4096 + 1024 + 32 * 1024;
+
+
+// Stage s's producer side: every copy of the chunk (4 groups) of item (tile, block).
+template <int WBITS, bool GATEUP>
+__device__ __forceinline__ uint32_t mma_stage_bytes() {
+  constexpr uint32_t braw = WBITS == 8 ? 16384u : 8192u;
+  return 16384u + 1024u + braw + 1024u + (WBITS == 4 ? 2048u : 0u);
+}
+
+template <int WBITS, bool GATEUP>
+__global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_constant__ MmaArgs A) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kMmaNS * MmaStage::BYTES);
+  uint64_t* prep = full + kMmaNS;
+  uint64_t* empty = prep + kMmaNS;
+  uint64_t* acc_full = empty + kMmaNS;
+  uint64_t* acc_empty = acc_full + kMmaNB;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + kMmaNB);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* xchg = reinterpret_cast<int*>(tmem_slot + 4);   // [2][2][128] h amax, [2][2][128] h code sums
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int PPG = WBITS == 8 ? 2 : 1;  // 16-byte pieces of one group of packed weights
+  constexpr int PPU = 2 * PPG;             // pieces of a 64-column down slab row
+  constexpr int kKern = GATEUP ? 3 : 4;
+
+  if (threadIdx.x == 0) {
+    *abort = 0;
+    for (int s = 0; s < kMmaNS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&prep[s], 2);
+      mbar_init(&empty[s], 1 + kMmaEpiWarps);
+    }
+    for (int b = 0; b < kMmaNB; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kMmaEpiWarps);
+    }
+    fence_barrier_init();
+  }
+  for (int i = threadIdx.x; i < 4 * 2 * 128; i += kMmaThreads) xchg[i] = 0;
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kMmaNB * 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  const BlobView& b0 = A.b[0];
+  const int H = b0.H;
+  const int nt = min(*A.n_tiles, A.max_tiles);
+  // items = (tile, block): gate/up blocks of 64 intermediate indices, down blocks of 128 rows
+  const int I_r = b0.I, I_s = A.b[1].I;
+  const int per_r = GATEUP ? I_r / 64 : H / 128;
+  const int per_s = GATEUP ? I_s / 64 : H / 128;
+  const int per = max(per_r, per_s);        // items per tile (slots of a shorter tile idle)
+  const int n_items = nt * per;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      uint32_t c = 0;
+      bool ok = true;
+      const uint64_t once = policy_evict_first();
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const int ti = it / per, blkn = it - ti * per;
+        const int4 tl = A.tiles[ti];
+        const int sh = tl.x < 0;
+        const BlobView& bv = A.b[sh];
+        if (blkn >= (sh ? per_s : per_r)) continue;
+        const int K = GATEUP ? H : bv.I;
+        const int G = K / 32, KB = kbytes(K, WBITS);
+        const uint8_t* a_src = GATEUP ? A.a_ops + (int64_t)ti * 128 * K : A.h_ops + (int64_t)ti * 128 * A.hk;
+        const __half* as_src = GATEUP ? A.a_scales + (int64_t)ti * G * 128 : A.h_scales + (int64_t)ti * (A.hk / 32) * 128;
+        const int32_t* xs_src = GATEUP ? A.a_xsum + (int64_t)ti * G * 128 : A.h_xsum + (int64_t)ti * (A.hk / 32) * 128;
+        for (int g0 = 0; g0 < G && ok; g0 += kMmaKC, ++c) {
+          const int s = c % kMmaNS;
+          if (c >= (uint32_t)kMmaNS && !mbar_wait(&empty[s], ((c / kMmaNS) - 1) & 1)) {
+            wait_failed(A.status, kKern, 0, s);
+            ok = false;
+            break;
+          }
+          uint8_t* st = base + s * MmaStage::BYTES;
+          mbar_arrive_expect_tx(&full[s], mma_stage_bytes<WBITS, GATEUP>());
+          bulk_load(st + MmaStage::A, a_src + (int64_t)g0 * 2 * 2048, 16384, &full[s]);
+          bulk_load(st + MmaStage::AS, as_src + (int64_t)g0 * 128, 1024, &full[s]);
+          if (WBITS == 4) bulk_load(st + MmaStage::XS, xs_src + (int64_t)g0 * 128, 2048, &full[s]);
+          uint8_t* bdst = st + (WBITS == 8 ? MmaStage::B : MmaStage::BRAW);
+          if (GATEUP) {
+            const int64_t blk = (int64_t)tl.w * 2 * bv.I + (int64_t)blkn * 128;
+            bulk_load_hint(bdst, bv.gu_w + blk * KB + (int64_t)g0 * PPG * 2048, kMmaKC * PPG * 2048, &full[s], once);
+            bulk_load_hint(st + MmaStage::BS, bv.gu_s + (blk * G + (int64_t)g0 * 128) * 2, 1024, &full[s], once);
+          } else {
+            const int U = bv.I / 64, HB = bv.H / 128;
+            for (int h = 0; h < 2; ++h) {
+              const int64_t slab = ((int64_t)tl.w * U + g0 / 2 + h) * HB + blkn;
+              bulk_load_hint(bdst + h * PPU * 2048, bv.dn_w + slab * PPU * 2048, PPU * 2048, &full[s], once);
+              bulk_load_hint(st + MmaStage::BS + h * 512, bv.dn_s + slab * 512, 512, &full[s], once);
+            }
+          }
+        }
+      }
+      // drain the copies still in flight before the CTA may exit
+      const uint32_t c0 = c > (uint32_t)kMmaNS ? c - kMmaNS : 0;
+      for (uint32_t d = c0; d < c; ++d)
+        if (!mbar_wait(&full[d % kMmaNS], (d / kMmaNS) & 1)) {
+          wait_failed(A.status, kKern, 2, d % kMmaNS);
+          break;
+        }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      uint32_t c = 0, gi = 0;
+      // int4 weights enter as unsigned bytes n ^ 8 = w + 8 (the epilogue subtracts 8 * sum(a))
+      constexpr uint32_t idesc = idesc_i8(128, 128, WBITS == 8);
+      for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+        const int ti = it / per, blkn = it - ti * per;
+        const int4 tl = A.tiles[ti];
+        const int sh = tl.x < 0;
+        if (blkn >= (sh ? per_s : per_r)) continue;
+        const int K = GATEUP ? H : A.b[sh].I;
+        const int G = K / 32;
+        for (int g0 = 0; g0 < G; g0 += kMmaKC, ++c) {
+          const int s = c % kMmaNS;
+          bool ok = *abort == 0;
+          if (ok && !mbar_wait(&prep[s], (c / kMmaNS) & 1)) {
+            *abort = 1;
+            wait_failed(A.status, kKern, 1, s);
+            ok = false;
+          }
+          tc_fence_after();
+          const uint8_t* st = base + s * MmaStage::BYTES;
+          for (int j = 0; j < kMmaKC; ++j, ++gi) {
+            const int bb = gi % kMmaNB;
+            if (ok && gi >= (uint32_t)kMmaNB && !mbar_wait(&acc_empty[bb], ((gi / kMmaNB) - 1) & 1)) {
+              *abort = 1;
+              wait_failed(A.status, kKern, 3, bb);
+              ok = false;
+            }
+            tc_fence_after();
+            if (ok)
+              mma_i8(tmem + bb * 128, smem_desc(st + MmaStage::A + j * 4096, 2048, 128),
+                     smem_desc(st + MmaStage::B + j * 4096, 2048, 128), idesc, 0);
+            mma_commit(&acc_full[bb]);         // arrives (in order) even when skipped
+          }
+          mma_commit(&empty[s]);
+        }
+      }
+    }
+  } else if (warp < 4) {
+    // ---------------------------------------------------------------- prep: int4 -> int8, scales
+    uint32_t c = 0;
+    const int pt = threadIdx.x - 64;        // [0, 64)
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+      const int ti = it / per, blkn = it - ti * per;
+      const int4 tl = A.tiles[ti];
+      const int sh = tl.x < 0;
+      if (blkn >= (sh ? per_s : per_r)) continue;
+      const int K = GATEUP ? H : A.b[sh].I;
+      const int G = K / 32;
+      for (int g0 = 0; g0 < G; g0 += kMmaKC, ++c) {
+        const int s = c % kMmaNS;
+        bool ok = *abort == 0;
+        if (ok && !mbar_wait(&full[s], (c / kMmaNS) & 1)) {
+          *abort = 1;
+          if (lane == 0) wait_failed(A.status, kKern, 4, s);
+          ok = false;
+        }
+        uint8_t* st = base + s * MmaStage::BYTES;
+        if (ok) {
+          if (WBITS == 4) {
+            // group j of row r: 16 packed bytes -> pieces 2j, 2j+1 of unsigned bytes n ^ 8
+            for (int q = pt; q < kMmaKC * 128; q += 64) {
+              const int j = q >> 7, r = q & 127;
+              const uint4 w = *reinterpret_cast<const uint4*>(st + MmaStage::BRAW + (j * 128 + r) * 16);
+              const uint32_t wv[4] = {w.x ^ 0x88888888u, w.y ^ 0x88888888u, w.z ^ 0x88888888u, w.w ^ 0x88888888u};
+              uint32_t o[8];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const uint32_t lo = wv[u] & 0x0F0F0F0Fu, hi = (wv[u] >> 4) & 0x0F0F0F0Fu;
+                o[2 * u] = __byte_perm(lo, hi, 0x5140);
+                o[2 * u + 1] = __byte_perm(lo, hi, 0x7362);
+              }
+              *reinterpret_cast<uint4*>(st + MmaStage::B + ((2 * j) * 128 + r) * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+              *reinterpret_cast<uint4*>(st + MmaStage::B + ((2 * j + 1) * 128 + r) * 16) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            fence_async_smem();
+          }
+          const __half* bs = reinterpret_cast<const __half*>(st + MmaStage::BS);
+          float* bsf = reinterpret_cast<float*>(st + MmaStage::BSF);
+          for (int q = pt; q < kMmaKC * 128; q += 64) bsf[q] = __half2float(bs[q]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&prep[s]);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    // 16 warps: warp 4 + 4 c + q reads tensor-memory lane quadrant q (slots 32 q ..) and
+    // column slice c: gate/up -> gate columns 16 c .. 16 c + 15 and the matching up columns
+    // 64 + 16 c ..; down -> output rows 32 c .. 32 c + 31 of the block.
+    const int ew = warp - 4;                // [0, 16)
+    const int quad = warp & 3;              // tensor-memory lane quadrant of this warp
+    const int cs = ew >> 2;                 // column slice
+    const int t = quad * 32 + lane;         // slot of the tile = tensor-memory lane
+    const int colA = GATEUP ? 16 * cs : 32 * cs;
+    const int colB = GATEUP ? 64 + 16 * cs : 32 * cs + 16;
+    // gate/up: the two slices of one Q8_0 group of h meet here (per item parity, group, slot)
+    int* amax_s = xchg;                     // [item parity][group][slot]
+    int* hsum_s = xchg + 2 * 2 * 128;
+    uint32_t c = 0, gi = 0, nit = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+      const int ti = it / per, blkn = it - ti * per;
+      const int4 tl = A.tiles[ti];
+      const int sh = tl.x < 0;
+      if (blkn >= (sh ? per_s : per_r)) continue;
+      const int K = GATEUP ? H : A.b[sh].I;
+      const int G = K / 32;
+      float2 acc2[16];                       // columns colA .. +15 (acc2[0..7]), colB .. (acc2[8..15])
+#pragma unroll
+      for (int q = 0; q < 16; ++q) acc2[q] = make_float2(0.0f, 0.0f);
+      for (int g0 = 0; g0 < G; g0 += kMmaKC, ++c) {
+        const int s = c % kMmaNS;
+        bool ok = *abort == 0;
+        if (ok && !mbar_wait(&prep[s], (c / kMmaNS) & 1)) {
+          *abort = 1;
+          if (lane == 0) wait_failed(A.status, kKern, 5, s);
+          ok = false;
+        }
+        const uint8_t* st = base + s * MmaStage::BYTES;
+        const __half* as = reinterpret_cast<const __half*>(st + MmaStage::AS);
+        const float* bsf = reinterpret_cast<const float*>(st + MmaStage::BSF);
+        for (int j = 0; j < kMmaKC; ++j, ++gi) {
+          const int bb = gi % kMmaNB;
+          if (ok && !mbar_wait(&acc_full[bb], (gi / kMmaNB) & 1)) {
+            *abort = 1;
+            if (lane == 0) wait_failed(A.status, kKern, 6, bb);
+            ok = false;
+          }
+          ok = __all_sync(0xffffffffu, ok);
+          tc_fence_after();
+          uint32_t d0[16], d1[16];
+          if (ok) {
+            const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + bb * 128;
+            tmem_ld16(ta + colA, d0);
+            tmem_ld16(ta + colB, d1);
+            tmem_wait_ld();
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[bb]);
+          if (ok) {
+            // acc = fma((float)I_g, s_w * s_x, acc) per element, two elements per packed op;
+            // exact (float)I_g: bits of 1.5 * 2^23 + (D - 8 * sum(a)) minus 1.5 * 2^23
+            const float sx = __half2float(as[j * 128 + t]);
+            const float2 sx2 = make_float2(sx, sx);
+            const int kb = 0x4B400000 -
+                           (WBITS == 4 ? 8 * reinterpret_cast<const int32_t*>(st + MmaStage::XS)[j * 128 + t] : 0);
+            const float4* sa = reinterpret_cast<const float4*>(bsf + j * 128 + colA);
+            const float4* sb = reinterpret_cast<const float4*>(bsf + j * 128 + colB);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float4 wa = sa[q4], wb = sb[q4];
+              const int q = 4 * q4;
+              acc2[q / 2] = __ffma2_rn(exact_i2f2k((int)d0[q], (int)d0[q + 1], kb),
+                                       __fmul2_rn(make_float2(wa.x, wa.y), sx2), acc2[q / 2]);
+              acc2[q / 2 + 1] = __ffma2_rn(exact_i2f2k((int)d0[q + 2], (int)d0[q + 3], kb),
+                                           __fmul2_rn(make_float2(wa.z, wa.w), sx2), acc2[q / 2 + 1]);
+              acc2[8 + q / 2] = __ffma2_rn(exact_i2f2k((int)d1[q], (int)d1[q + 1], kb),
+                                           __fmul2_rn(make_float2(wb.x, wb.y), sx2), acc2[8 + q / 2]);
+              acc2[8 + q / 2 + 1] = __ffma2_rn(exact_i2f2k((int)d1[q + 2], (int)d1[q + 3], kb),
+                                               __fmul2_rn(make_float2(wb.z, wb.w), sx2), acc2[8 + q / 2 + 1]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      float acc[32];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        acc[2 * q] = acc2[q].x;
+        acc[2 * q + 1] = acc2[q].y;
+      }
+      const bool live = *abort == 0;
+      // ---- item output
+      const bool valid = t < tl.z;
+      const int slot = tl.y + t;
+      if (GATEUP) {
+        const int I = A.b[sh].I, IB = I / 32;
+        const int i0 = blkn * 64 + 16 * cs;  // the thread's 16 intermediate indices
+        const int par = nit & 1, gl = cs >> 1;
+        int* am = amax_s + (par * 2 + gl) * 128 + t;
+        int* hm = hsum_s + (par * 2 + gl) * 128 + t;
+        float h[16];
+        float amax = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          h[q] = cswiglu(acc[q], acc[16 + q]);
+          amax = fmaxf(amax, fabsf(h[q]));
+        }
+        atomicMax(am, __float_as_int(amax));             // non-negative: int order = float order
+        named_bar(2, 32 * kMmaEpiWarps);
+        const float sc = f16_round(__fdiv_rn(__int_as_float(*am), 127.0f));
+        uint32_t pk[4];
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) {
+          uint32_t v = 0;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) v |= (uint32_t)(uint8_t)(int8_t)quant_code(h[4 * w4 + u], sc, 127.0f) << (8 * u);
+          pk[w4] = v;
+        }
+        int hsum = 0;
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) hsum = __dp4a((int)pk[w4], 0x01010101, hsum);
+        atomicAdd(hm, hsum);
+        if (live) {
+          *reinterpret_cast<uint4*>(A.h_ops + ((int64_t)ti * (A.hk / 16) + i0 / 16) * 128 * 16 + t * 16) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          if (valid) {
+            *reinterpret_cast<uint4*>(A.qh[sh] + (int64_t)slot * I + i0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if (A.dbg_a[sh])
+              for (int q = 0; q < 16; ++q) {
+                A.dbg_a[sh][(int64_t)slot * I + i0 + q] = acc[q];
+                A.dbg_b[sh][(int64_t)slot * I + i0 + q] = acc[16 + q];
+              }
+          }
+        }
+        named_bar(2, 32 * kMmaEpiWarps);
+        if ((cs & 1) == 0) {
+          if (live) {
+            const int64_t hg = (int64_t)ti * (A.hk / 32) + i0 / 32;
+            A.h_scales[hg * 128 + t] = __float2half_rn(sc);
+            A.h_xsum[hg * 128 + t] = *hm;
+            if (valid) A.sh[sh][(int64_t)slot * IB + i0 / 32] = __float2half_rn(sc);
+          }
+          *am = 0;                           // this parity's entries are next used two items on
+          *hm = 0;
+        }
+      } else if (valid && live) {
+        int tok = slot;
+        float wt = 1.0f;
+        bool okp = true;
+        if (!sh) {
+          const int p = A.perm[slot];
+          okp = p >= 0 && p < A.T * A.k;
+          if (!okp) set_status(A.status, kStatusDeviceCheck);
+          tok = okp ? p / A.k : 0;
+          wt = okp ? A.wts[p] : 0.0f;
+        }
+        if (okp) {
+          const int n0 = blkn * 128 + 32 * cs;
+          float* yr = A.y + (int64_t)tok * H + n0;
+#pragma unroll
+          for (int q = 0; q < 32; q += 4)
+            red_add_v4(yr + q, wt * acc[q], wt * acc[q + 1], wt * acc[q + 2], wt * acc[q + 3]);
+          if (A.dbg_y[sh])
+            for (int q = 0; q < 32; ++q) atomicAdd(A.dbg_y[sh] + (int64_t)slot * H + n0 + q, acc[q]);
+        }
+      }
+      ++nit;
+    }
+  }
+  // all tensor-memory reads done before the allocating warp frees it
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kMmaNB * 128);
+}
+
+// -------------------------------------------------------------------- host side
+namespace {
+
+int sm_count_mma() {
+  static int n[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  if (n[dev] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 148;
+  }
+  return n[dev];
+}
+
+template <int WBITS, bool GATEUP>
+cudaError_t launch_mma_t(const MmaArgs& a, int max_items, cudaStream_t st) {
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(k_expert_mma<WBITS, GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = std::max(1, std::min(max_items, sm_count_mma()));
+  return launch_pdl(k_expert_mma<WBITS, GATEUP>, dim3(grid), dim3(kMmaThreads), (size_t)kMmaSmem, st, a);
+}
+
+}  // namespace
+
+cudaError_t launch_mma_plan(const Grouping& g, int E, int T, int has_shared, int min_tokens, int max_tiles,
+                            int4* tiles, int32_t* n_tiles, int* status, cudaStream_t st) {
+  return launch_pdl(k_mma_plan, dim3(1), dim3(1024), 0, st, (const int32_t*)g.n_active,
+                    (const int32_t*)g.act_expert, (const int32_t*)g.act_begin, E, T, has_shared, min_tokens,
+                    max_tiles, tiles, n_tiles, status);
+}
+
+cudaError_t launch_mma_gather(const int8_t* qx, const __half* sx, const int4* tiles, const int32_t* n_tiles,
+                              const int32_t* perm, int k, int T, int K, int max_tiles, uint8_t* xa, __half* xs,
+                              int32_t* xsum, int* status, cudaStream_t st) {
+  const int64_t work = (int64_t)max_tiles * 128 * (K / 32);
+  const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, (int64_t)sm_count_mma() * 8));
+  return launch_pdl(k_mma_gather, dim3(grid), dim3(256), 0, st, qx, sx, tiles, n_tiles, perm, k, T, K, xa, xs,
+                    xsum, status);
+}
+
+cudaError_t launch_expert_mma(bool gateup, const MmaArgs& a, cudaStream_t st) {
+  const int per_r = gateup ? a.b[0].I / 64 : a.b[0].H / 128;
+  const int per_s = gateup ? a.b[1].I / 64 : a.b[1].H / 128;
+  const int max_items = a.max_tiles * std::max(per_r, per_s);
+  if (a.b[0].wbits == 8)
+    return gateup ? launch_mma_t<8, true>(a, max_items, st) : launch_mma_t<8, false>(a, max_items, st);
+  return gateup ? launch_mma_t<4, true>(a, max_items, st) : launch_mma_t<4, false>(a, max_items, st);
+}
+
+}  // namespace moe

@@ -101,7 +101,7 @@ struct Unit {
 // load is issued before any is used, so resolving a unit costs one L2 round trip.
 __device__ __forceinline__ bool unit_of(const ExpertArgs& r, const ExpertArgs& s, int has_shared,
                                         int routed_units, int per_expert_r, int u, Unit& U,
-                                        bool want_rows, bool report) {
+                                        bool want_rows, bool report, int mma_min) {
   if (u < routed_units) {
     U.shd = false;
     U.ai = u / per_expert_r;
@@ -123,13 +123,14 @@ __device__ __forceinline__ bool unit_of(const ExpertArgs& r, const ExpertArgs& s
       U.rows8[7] = hi.w;
     }
     if (U.ai >= na) return false;
+    if (U.s1 - U.s0 >= mma_min) return false;     // on the tensor-core path
     if (U.e < 0 || U.e >= r.b.E || U.s0 < 0 || U.s0 > U.s1 || U.s1 > r.T * r.k) {
       if (report) set_status(r.status, kStatusDeviceCheck);
       return false;
     }
     return true;
   }
-  if (!has_shared) return false;
+  if (!has_shared || s.T >= mma_min) return false;
   U.shd = true;
   U.ai = 0;
   U.e = 0;
@@ -168,15 +169,6 @@ __device__ __forceinline__ int down_rotation(const Unit& U, int nch) {
   return (int)(((unsigned)U.sub * 7u + (unsigned)U.ai * 3u) % (unsigned)nch);
 }
 
-// Record the first wait that gave up: word 2 = kernel | role << 4 | stage << 8, word 3 = CTA.
-__device__ __forceinline__ void wait_failed(int* status, int kernel, int role, int stage) {
-  if (!status) return;
-  if (atomicCAS(status, 0, kStatusTimeout) == 0) {
-    status[2] = kernel | (role << 4) | (stage << 8);
-    status[3] = (int)blockIdx.x;
-  }
-}
-
 struct Ring {
   uint8_t* ring;
   uint8_t* sring;
@@ -200,6 +192,7 @@ struct RingArgs {
   int routed;              // routed units
   int per;                 // units per routed expert (I / 64)
   int tm, kmax;
+  int mma_min;             // experts with this many slots are left to the tensor-core path
 };
 
 // ------------------------------------------------------------------ producer
@@ -233,7 +226,8 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
   };
   for (int u = blockIdx.x; u < A.units && ok; u += gridDim.x) {
     Unit U;
-    if (!unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, false)) continue;
+    if (!unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, false, A.mma_min))
+      continue;
     const ExpertArgs& g = A.x[0][U.shd ? 1 : 0];
     const ExpertArgs& d = A.x[1][U.shd ? 1 : 0];
     for (int c0 = U.s0; c0 < U.s1 && ok; c0 += A.tm, ++pidx) {
@@ -371,7 +365,7 @@ __device__ __forceinline__ void block_chain(const __half* sst, int j0, int gbase
         if (WG32 && AG32) cg = __fmul_rn(sw[j], sxg);
         else if (WG32) cg = sw[j];
         else cg = sxg;
-        acc[qq] = __fmaf_rn(__int2float_rn(d[j]), cg, acc[qq]);
+        acc[qq] = __fmaf_rn(exact_i2f(d[j]), cg, acc[qq]);
       }
     }
   }
@@ -441,7 +435,7 @@ __device__ __forceinline__ void ring_consume(int K, int m, int tm, const Ring& R
                 if (WG32 && AG32) cg = __fmul_rn(swg, sxg);
                 else if (WG32) cg = swg;
                 else cg = sxg;
-                acc[qq] = __fmaf_rn(__int2float_rn(d), cg, acc[qq]);
+                acc[qq] = __fmaf_rn(exact_i2f(d), cg, acc[qq]);
               }
             }
           }
@@ -617,7 +611,8 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   uint32_t c = 0, pidx = 0, nblk = 0;       // chunks, gate/up passes, 8-group blocks consumed
   for (int u = blockIdx.x; u < A.units; u += gridDim.x) {
     Unit U;
-    if (!unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, ctid == 0)) continue;
+    if (!unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, ctid == 0, A.mma_min))
+      continue;
     const ExpertArgs& g = A.x[0][U.shd ? 1 : 0];
     const ExpertArgs& d = A.x[1][U.shd ? 1 : 0];
     const int I = g.b.I, IB = I / 32;
@@ -817,7 +812,7 @@ bool experts_fusable(const ExpertArgs& r, const ExpertArgs* s) {
 }
 
 cudaError_t launch_experts(int mode, const ExpertArgs& gr, const ExpertArgs* gs, const ExpertArgs& dr,
-                           const ExpertArgs* ds, cudaStream_t st) {
+                           const ExpertArgs* ds, int mma_min, cudaStream_t st) {
   RingArgs A;
   std::memset(&A, 0, sizeof(A));
   A.x[0][0] = gr;
@@ -830,6 +825,7 @@ cudaError_t launch_experts(int mode, const ExpertArgs& gr, const ExpertArgs* gs,
   A.units = A.routed + (gs ? gs->b.I / 64 : 0);
   A.kmax = mode == 1 ? 64 : gr.b.H;           // K of the staged activation rows
   A.tm = ring_tokens(A.kmax, gr.T);
+  A.mma_min = mma_min;
   const int sel = (gr.b.wbits == 8 ? 4 : 0) | (gr.b.wg32 ? 2 : 0) | (gr.ag32 ? 1 : 0);
   switch (sel) {
     case 7: return launch_mode<8, true, true>(mode, A, st);

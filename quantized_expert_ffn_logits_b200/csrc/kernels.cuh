@@ -71,8 +71,49 @@ struct ExpertArgs {
 // workspace), 1: down pass (h from the workspace), 2: both, h kept on chip -- needs
 // experts_fusable() (group-32 activations: h of a unit is quantized without the rest).
 bool experts_fusable(const ExpertArgs& r, const ExpertArgs* s);
+// Experts (the shared one: T) with mma_min or more slots are skipped (tensor-core path).
 cudaError_t launch_experts(int mode, const ExpertArgs& gr, const ExpertArgs* gs, const ExpertArgs& dr,
-                           const ExpertArgs* ds, cudaStream_t st);
+                           const ExpertArgs* ds, int mma_min, cudaStream_t st);
+
+// ---- expert_mma.cu: tensor-core GEMMs for experts with many tokens
+constexpr int kMmaMinTokens = 64;          // pairs an expert needs in a call to take this path
+
+struct MmaArgs {
+  BlobView b[2];                           // routed experts, shared expert
+  const int4* tiles;
+  const int32_t* n_tiles;
+  int max_tiles;
+  const uint8_t* a_ops;                    // operand A of every tile: [tile][K/16][128][16]
+  const __half* a_scales;                  // [tile][K/32][128]
+  const int32_t* a_xsum;                   // [tile][K/32][128] sum of a group's codes (int4 weights)
+  // gate/up outputs: h of every tile in operand layout for the down GEMM, and the per-slot
+  // views of the workspace (q_h, s_h; gate / up values when debugging)
+  uint8_t* h_ops;                          // [tile][hk/16][128][16]
+  __half* h_scales;                        // [tile][hk/32][128]
+  int32_t* h_xsum;                         // [tile][hk/32][128]
+  int hk;                                  // row length of a tile's h: max(I, I_shared)
+  int8_t* qh[2];
+  __half* sh[2];
+  float* dbg_a[2];
+  float* dbg_b[2];
+  // down outputs
+  const int32_t* perm;
+  const float* wts;
+  float* y;
+  float* dbg_y[2];
+  int T, k;
+  int* status;
+};
+
+// Tile list of the experts with >= min_tokens slots (+ the shared expert's tokens).
+cudaError_t launch_mma_plan(const Grouping& g, int E, int T, int has_shared, int min_tokens, int max_tiles,
+                            int4* tiles, int32_t* n_tiles, int* status, cudaStream_t st);
+// Operand A (q_x rows of each tile's tokens, [tile][K/16][128][16]) and its scales.
+cudaError_t launch_mma_gather(const int8_t* qx, const __half* sx, const int4* tiles, const int32_t* n_tiles,
+                              const int32_t* perm, int k, int T, int K, int max_tiles, uint8_t* xa, __half* xs,
+                              int32_t* xsum, int* status, cudaStream_t st);
+// Gate/up (+ SwiGLU, Q8_0 h) or down (+ weighted combine) of every tile x weight block.
+cudaError_t launch_expert_mma(bool gateup, const MmaArgs& a, cudaStream_t st);
 
 // ---- route_fused.cu (T <= 32)
 struct RouteArgs {

@@ -63,10 +63,26 @@ def _run_layer(case, flags):
 
 @pytest.mark.parametrize("name,T", CASES)
 def test_layer_forward_matches_oracle(name, T):
+    _check_layer(name, T, M().MOE_FLAG_DEBUG)
+
+
+# The tensor-core path (experts with >= 64 pairs at T > 32; every expert with the force flag):
+# the same bit-exact gate/up values, h codes and scales as the streaming path and the oracle.
+MMA_CASES = [("olmoe_int4", 300, False), ("olmoe_int4", 40, True), ("olmoe_int8", 70, True),
+             ("e512_int4", 100, True), ("glm_int4", 50, True)]
+
+
+@pytest.mark.parametrize("name,T,force", MMA_CASES)
+def test_tensor_core_path_matches_oracle(name, T, force):
+    m = M()
+    _check_layer(name, T, m.MOE_FLAG_DEBUG | (m.MOE_FLAG_FORCE_MMA if force else 0))
+
+
+def _check_layer(name, T, flags):
     m = M()
     c = REDUCED[name]
     case = S.Case.make(c, T)
-    g, cfg, y, ws, v = _run_layer(case, m.MOE_FLAG_DEBUG)
+    g, cfg, y, ws, v = _run_layer(case, flags)
     assert m.moe_read_device_status(ws) == m.MOE_OK
     ref = oracle_layer(case, union=True)
     k, E, H, I = c.top_k, c.E, c.H, c.I
