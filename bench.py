@@ -9,6 +9,9 @@ never left in L2 by the previous steps. The timed region replays a CUDA graph of
 the steps (launch overhead removed), bracketed by a barrier and a device
 synchronize on both sides; multi-GPU runs are weak-scaled (each rank its own
 tokens and replicas, no data-path collective) and report the max over ranks.
+The line also carries the metric's prefill half ("prefill"): the OLMoE-shaped
+packed-int4 layer on 4096 tokens per GPU, whose experts run as int8 tensor-core
+GEMMs, with its tensor roofline against the int8 peak.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload olmoe_int8:1]
   python bench.py --impl reference ...   (the CPU oracle as the reference arm)
@@ -237,7 +240,7 @@ def oracle_sampler(cfg, T, seed_base=7_000_000):
     return run_units, desc, cores
 
 
-def time_oracle(cfg, T, budget_s=20.0):
+def time_oracle(cfg, T, budget_s=45.0):
     run_units, desc, cores = oracle_sampler(cfg, T)
     per_tok = cfg.top_k + (1 if cfg.shared_I else 0)
     t0 = time.perf_counter()
@@ -290,6 +293,115 @@ def reference_arm(args, cfg, T):
 
 
 # --------------------------------------------------------------------- GPU arm
+PREFILL_WORKLOAD = "olmoe_int4:4096"
+
+
+def rank_seeds(rank: int, replicas: int, batches: int):
+    """Weak scaling: every rank its own layer replicas (expert weights) and token batches --
+    seeds disjoint across ranks, so no rank's inputs repeat another's."""
+    return ([1000 * rank + r for r in range(replicas)],
+            [90_000_000 + 1_000_000 * rank + s for s in range(batches)])
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The timed duration of the slowest rank (every rank calls this, in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank_step: int, world: int, steps: int, ms_max: float) -> float:
+    """Tokens per second of all ranks together over the slowest rank's timed region."""
+    return world * tokens_per_rank_step * steps / (ms_max / 1e3)
+
+
+def prefill_arm(args, dev, world, M, torch, dist):
+    """The metric's "prefill 4k" half: the OLMoE-shaped packed-int4 layer (group-32 scales) on
+    T = 4096 fresh tokens per GPU (every expert > 64 pairs: the tensor-core GEMMs). Eager steps
+    timed with CUDA events (max over ranks); the GEMM kernels' share from stage events."""
+    cfg, T = parse_workload(args.prefill_workload)
+    rank = int(os.environ.get("RANK", "0"))
+    rcfg = M.RouteCfg(score=cfg.score, top_k=cfg.top_k, renormalize=cfg.renormalize,
+                      routed_scaling_factor=cfg.rsf, act=cfg.act)
+    case = S.Case.make(cfg, T, replica=1000 * rank + 7)
+    gu = torch.empty((cfg.E, 2 * cfg.I, cfg.H), dtype=torch.float32, device=dev)
+    case.gate_up_gpu(gu)
+    dn = torch.empty((cfg.E, cfg.H, cfg.I), dtype=torch.float32, device=dev)
+    case.down_gpu(dn)
+    blob = M.ExpertBlob.quantize(gu, dn, cfg.wtype, cfg.wscale)
+    del gu, dn
+    shared = None
+    if cfg.shared_I:
+        sgu = torch.empty((1, 2 * cfg.shared_I, cfg.H), dtype=torch.float32, device=dev)
+        sdn = torch.empty((1, cfg.H, cfg.shared_I), dtype=torch.float32, device=dev)
+        case.shared_gate_up_gpu(sgu)
+        case.shared_down_gpu(sdn)
+        shared = M.ExpertBlob.quantize(sgu, sdn, cfg.wtype, cfg.wscale)
+        del sgu, sdn
+    wr = torch.from_numpy(case.router_w()).to(dev)
+    b = case.bias()
+    bias = torch.from_numpy(b).to(dev) if b is not None else None
+    lay = M.Layer(T, blob, shared, rcfg, wr, bias)
+    xs = [torch.from_numpy(S.Case.make(cfg, T, seed=80_000_000 + 1_000_000 * rank + s).x()).to(dev)
+          for s in range(2)]
+    y = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    steps = max(1, args.prefill_steps)
+    nst = len(M.MOE_STAGES)
+    ev = M.moe_stage_events()
+    pairs = []
+    with torch.cuda.stream(stream):
+        for i in range(nst):
+            b_ev = torch.cuda.Event(enable_timing=True, external=True)
+            e_ev = torch.cuda.Event(enable_timing=True, external=True)
+            b_ev.record(stream)
+            e_ev.record(stream)
+            ev.begin[i], ev.end[i] = b_ev.cuda_event, e_ev.cuda_event
+            pairs.append((b_ev, e_ev))
+        for s in range(3):
+            lay(xs[s % 2], y, stream)
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for s in range(steps):
+            lay(xs[s % 2], y, stream)
+        e1.record(stream)
+    stream.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / steps
+    # stage times of one more step: gate/up stage = tile plan + gather + gate/up GEMM (+ the
+    # streaming kernel, idle here), down stage = the down GEMM
+    with torch.cuda.stream(stream):
+        lay(xs[0], y, stream, events=ev)
+    stream.synchronize()
+    stage = {n: pairs[i][0].elapsed_time(pairs[i][1]) * 1e3 for i, n in enumerate(M.MOE_STAGES)}
+    peaks, _ = load_peaks()
+    int8_peak = 2.0 * peaks["bf16_tflops"]           # nominal int8 : bf16 dense ratio 2
+    ops = layer_int_ops(cfg, T)
+    gemm_us = stage["gate_up"] + stage["down"]
+    ach = ops / (gemm_us * 1e-6) / 1e12
+    return {
+        "workload": workload_desc(cfg, T), "T": T, "value": round(world * T / (ms / 1e3), 1),
+        "unit": "tok/s", "ms_per_step": round(ms, 4), "steps": steps,
+        "stage_us": {k: round(v, 1) for k, v in stage.items()},
+        "roofline": {"bound": "tensor", "achieved": round(ach, 1), "peak": round(int8_peak, 1),
+                     "unit": "TOPS", "frac": round(ach / int8_peak, 4),
+                     "kernel": "k_expert_mma gate/up + down (int8 tcgen05.mma, per-group fp32 epilogue)",
+                     "ops_per_step": int(ops),
+                     "peak_source": "measured bf16 TFLOP/s (MEASURED_PEAKS.json) x 2, the nominal int8 / bf16 dense ratio"},
+        "note": "the per-group fp32 epilogue (3 fp32 ops per element per quantization group) bounds the tensor-core path",
+    }
+
+
 def gpu_arm(args, cfg, T):
     import torch
     import torch.distributed as dist
@@ -312,11 +424,12 @@ def gpu_arm(args, cfg, T):
             dist.barrier(device_ids=[local])
 
     R = args.replicas
+    rep_seeds, x_seeds = rank_seeds(rank, R, max(1, min(args.steps, args.period)))
     rcfg = M.RouteCfg(score=cfg.score, top_k=cfg.top_k, renormalize=cfg.renormalize,
                       routed_scaling_factor=cfg.rsf, act=cfg.act)
     layers, n_active_of = [], []
     for r in range(R):
-        case = S.Case.make(cfg, T, replica=1000 * rank + r)
+        case = S.Case.make(cfg, T, replica=rep_seeds[r])
         gu = torch.empty((cfg.E, 2 * cfg.I, cfg.H), dtype=torch.float32, device=dev)
         case.gate_up_gpu(gu)
         dn = torch.empty((cfg.E, cfg.H, cfg.I), dtype=torch.float32, device=dev)
@@ -340,7 +453,7 @@ def gpu_arm(args, cfg, T):
     G = max(1, min(args.steps, args.period))
     xs = []
     for s in range(G):
-        xc = S.Case.make(cfg, T, seed=90_000_000 + 1_000_000 * rank + s)
+        xc = S.Case.make(cfg, T, seed=x_seeds[s])
         xs.append(torch.from_numpy(xc.x()).to(dev))
     y = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
     # distinct experts per step (for the algorithmic byte counts)
@@ -428,11 +541,7 @@ def gpu_arm(args, cfg, T):
     barrier()
     clocks.mark(w0, w1)
     clk = clocks.stop()
-    ms = start.elapsed_time(end)
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(start.elapsed_time(end), world, dev)
 
     # per-stage device times of the last graph period (inside the timed region)
     stage_ms = {n: [] for n in M.MOE_STAGES}
@@ -443,7 +552,7 @@ def gpu_arm(args, cfg, T):
                 stage_ms[n].append(b_ev.elapsed_time(e_ev))
     stage_us = {n: (1e3 * statistics.mean(v) if v else None) for n, v in stage_ms.items()}
 
-    value = world * T * args.steps / (ms_max / 1e3)
+    value = whole_job_rate(T, world, args.steps, ms_max)
     peaks, peak_src = load_peaks()
     n_act = float(np.mean(n_active_of))
     # dominant kernel: the expert kernel (weight streaming, HBM-bound); with group-32
@@ -501,6 +610,10 @@ def gpu_arm(args, cfg, T):
                "h2d_bytes_per_step": T * cfg.H * 4, "d2h_bytes_per_step": T * cfg.H * 4,
                "steps": ne, "path": "Layer.__call__ (moe_layer_forward) eager, pinned host x in / y out"}
 
+    prefill = None
+    if not args.no_prefill:
+        prefill = prefill_arm(args, dev, world, M, torch, dist)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = time_oracle(cfg, T)
@@ -518,6 +631,7 @@ def gpu_arm(args, cfg, T):
                    "parallelism": f"dp{world} (weak: independent tokens per GPU)"},
         "roofline": roof,
         "layer": layer,
+        "prefill": prefill,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches,
@@ -561,6 +675,9 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (4k tokens) measurement")
+    ap.add_argument("--prefill-workload", default=PREFILL_WORKLOAD)
+    ap.add_argument("--prefill-steps", type=int, default=20)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

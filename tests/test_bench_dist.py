@@ -1,0 +1,57 @@
+"""Multi-rank logic of bench.py on CPU: two gloo ranks (spawned processes) take the max of
+their timed regions, draw disjoint inputs (weak scaling), and the whole-job rate counts every
+rank's tokens over the slowest rank's time; the reference arm does no work off rank 0."""
+import datetime
+import multiprocessing as mp
+import os
+import socket
+import types
+
+import bench
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        got = bench.max_over_ranks(10.0 + 5.0 * rank, world, "cpu")
+        seeds = bench.rank_seeds(rank, 8, 16)
+    finally:
+        dist.destroy_process_group()
+    q.put((rank, got, seeds))
+
+
+def test_two_gloo_ranks_max_time_and_disjoint_inputs():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    assert [got for _, got, _ in res] == [15.0, 15.0]           # both see the slowest rank
+    (_, _, (rep0, x0)), (_, _, (rep1, x1)) = res
+    assert not set(rep0) & set(rep1) and not set(x0) & set(x1)
+    assert len(set(rep0)) == 8 and len(set(x0)) == 16
+
+
+def test_whole_job_rate_counts_all_ranks_over_the_slowest():
+    assert bench.whole_job_rate(1, 2, 100, 15.0) == 2 * 100 / 0.015
+    assert bench.whole_job_rate(4096, 1, 20, 58.0) == 4096 * 20 / 0.058
+
+
+def test_reference_arm_idle_off_rank_zero(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    args = types.SimpleNamespace(steps=1, warmup=0)
+    assert bench.reference_arm(args, None, 1) == 0
