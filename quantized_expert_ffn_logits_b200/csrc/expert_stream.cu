@@ -303,7 +303,7 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
 // runs the ordered fp32 chain of its row over the block's 8 groups for its tokens
 // (tokens ts, ts+2, ... with ts = thread / 128). idot is double-buffered, so the barrier
 // after the next block's dots also orders this block's chain before the buffer is reused.
-template <int WBITS, bool WG32, bool AG32>
+template <int WBITS, bool WG32, bool AG32, int TM>
 __device__ __forceinline__ void block_dots(const uint8_t* stage, int j0, int gbase, int m, int tm,
                                            const uint8_t* xs, int K, const int* xsum, int G, int* idot) {
   constexpr int PPG = WBITS == 8 ? 2 : 1;
@@ -317,7 +317,8 @@ __device__ __forceinline__ void block_dots(const uint8_t* stage, int j0, int gba
     if (WBITS == 8) w[r * PPG + 1] = *reinterpret_cast<const uint4*>(wp + kPiece + r * 512);
   }
   int* out = idot + warp * tm * kRows + lane;
-  for (int q = 0; q < m; ++q) {
+  const int mq = TM == 1 ? 1 : m;          // TM: compile-time bound on the pass's tokens
+  for (int q = 0; q < mq; ++q) {
     const uint8_t* xg = xs + q * K + 32 * g;
     const uint4 x0 = *reinterpret_cast<const uint4*>(xg);
     const uint4 x1 = *reinterpret_cast<const uint4*>(xg + 16);
@@ -335,7 +336,7 @@ __device__ __forceinline__ void block_dots(const uint8_t* stage, int j0, int gba
   }
 }
 
-template <int WBITS, bool WG32, bool AG32>
+template <int WBITS, bool WG32, bool AG32, int TM>
 __device__ __forceinline__ void block_chain(const __half* sst, int j0, int gbase, int m, int tm, int G,
                                             const int* idot, const __half* sxh, const float* sxf,
                                             float acc[kTMP / 2], int isum[kTMP / 2]) {
@@ -346,9 +347,9 @@ __device__ __forceinline__ void block_chain(const __half* sst, int j0, int gbase
     for (int j = 0; j < 8; ++j) sw[j] = __half2float(sst[(j0 + j) * 128 + row]);
   }
 #pragma unroll
-  for (int qq = 0; qq < kTMP / 2; ++qq) {
+  for (int qq = 0; qq < (TM == 1 ? 1 : kTMP / 2); ++qq) {
     const int q = ts + 2 * qq;
-    if (q >= m) break;
+    if (TM != 1 && q >= m) break;
     int d[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) d[j] = idot[(j * tm + q) * kRows + row];
@@ -375,7 +376,7 @@ __device__ __forceinline__ void block_chain(const __half* sst, int j0, int gbase
 // (thread & 127) for tokens ts + 2 qq in v[qq]. After a wait gives up (`abort` set by any
 // consumer), waits and compute are skipped but every stage is still released and every
 // barrier taken, so the producer is never left waiting.
-template <int WBITS, bool WG32, bool AG32>
+template <int WBITS, bool WG32, bool AG32, int TM>
 __device__ __forceinline__ void ring_consume(int K, int m, int tm, const Ring& R, uint32_t& c, uint32_t& nblk,
                                              const uint8_t* xs, const __half* sxh, const float* sxf,
                                              const int* xsum, int* idot, float sw_row,
@@ -411,11 +412,11 @@ __device__ __forceinline__ void ring_consume(int K, int m, int tm, const Ring& R
     for (int j0 = 0; j0 < ng; j0 += 8, ++nblk) {
       const int nb = min(8, ng - j0);
       int* ib = idot + (nblk & 1) * (8 * tm * kRows);
-      if (ok && (threadIdx.x >> 5) < nb) block_dots<WBITS, WG32, AG32>(stage, j0, gbase, m, tm, xs, K, xsum, G, ib);
+      if (ok && (threadIdx.x >> 5) < nb) block_dots<WBITS, WG32, AG32, TM>(stage, j0, gbase, m, tm, xs, K, xsum, G, ib);
       named_bar(1, 32 * kCW);
       if (ok && chain_thread) {
         if (nb == 8) {
-          block_chain<WBITS, WG32, AG32>(sst, j0, gbase, m, tm, G, ib, sxh, sxf, acc, isum);
+          block_chain<WBITS, WG32, AG32, TM>(sst, j0, gbase, m, tm, G, ib, sxh, sxf, acc, isum);
         } else {
           // 4-group tail: same chain, groups j0 .. j0+3 only
           const int row = threadIdx.x & 127;
@@ -462,7 +463,7 @@ __device__ __forceinline__ void ring_consume(int K, int m, int tm, const Ring& R
 // (fp32, any order), weighted and added into y (and, for inspection, into the pair's
 // down value). hx: the pass's h codes [tm][64] (int4 weights: each 8-byte word
 // de-interleaved), hxs: per-group code sums [tm][2] (int4), hs: h scales [tm][2].
-template <int WBITS, bool WG32, bool AG32>
+template <int WBITS, bool WG32, bool AG32, int TM>
 __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& R, uint32_t& c, const uint8_t* hx,
                                              const int* hxs, const float* hs, const int* toks,
                                              const float* wts, float* y, float* dbg, int slot0,
@@ -505,7 +506,7 @@ __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& 
           }
         }
       }
-      for (int q = 0; q < m; ++q) {
+      for (int q = 0; q < (TM == 1 ? 1 : m); ++q) {
         const uint4* xq = reinterpret_cast<const uint4*>(hx + q * 64);
         const uint4 x0 = xq[0], x1 = xq[1], x2 = xq[2], x3 = xq[3];
         const float hs0 = hs[2 * q], hs1 = hs[2 * q + 1];
@@ -556,7 +557,7 @@ __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& 
 // up stage values meet in shared memory and warps 0 and 1 apply SwiGLU and quantize h per
 // group of 32 -- one warp per group), then the down pass over the unit's slab with the
 // pass's h codes from shared memory (MODE 2) or from the workspace (MODE 1).
-template <int WBITS, bool WG32, bool AG32, int MODE>
+template <int WBITS, bool WG32, bool AG32, int MODE, int TM>
 __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ RingArgs A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
@@ -695,7 +696,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
         const int64_t blk = (int64_t)U.e * 2 * I + (int64_t)U.sub * kRows;
         const float sw_row = WG32 ? 0.0f : reinterpret_cast<const float*>(g.b.gu_s)[blk + row];
         float v[kTMP / 2];
-        ring_consume<WBITS, WG32, AG32>(K, m, tm, R, c, nblk, xs, sxh, R.sxf, xsum, idot, sw_row, v, abort,
+        ring_consume<WBITS, WG32, AG32, TM>(K, m, tm, R, c, nblk, xs, sxh, R.sxf, xsum, idot, sw_row, v, abort,
                                         status, 1);
         __syncwarp();
         if (lane == 0) mbar_arrive(&R.aempty[b]);
@@ -758,7 +759,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
           hx = hqd;
         }
         const int rot = down_rotation(U, (d.b.H / kRows + kSP / (WBITS == 8 ? 4 : 2) - 1) / (kSP / (WBITS == 8 ? 4 : 2)));
-        down_consume<WBITS, WG32, AG32>(d.b.H, m, rot, R, c, hx, hxs, hs, toks, wts, d.y, d.dbg_a, c0, abort,
+        down_consume<WBITS, WG32, AG32, TM>(d.b.H, m, rot, R, c, hx, hxs, hs, toks, wts, d.y, d.dbg_a, c0, abort,
                                         status);
       }
     }
@@ -781,27 +782,34 @@ int sm_count() {
   return n[dev];
 }
 
-template <int WBITS, bool WG32, bool AG32, int MODE>
+template <int WBITS, bool WG32, bool AG32, int MODE, int TM>
 cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
   const RingPlan P = ring_plan(A.kmax, A.tm);
   static int attr_bytes = 0;
   if (P.total > attr_bytes) {
-    const cudaError_t e = cudaFuncSetAttribute(k_expert_ring<WBITS, WG32, AG32, MODE>,
+    const cudaError_t e = cudaFuncSetAttribute(k_expert_ring<WBITS, WG32, AG32, MODE, TM>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, P.total);
     if (e != cudaSuccess) return e;
     attr_bytes = P.total;
   }
   const int grid = A.units < sm_count() ? A.units : sm_count();
   if (grid <= 0) return cudaSuccess;
-  return launch_pdl(k_expert_ring<WBITS, WG32, AG32, MODE>, dim3(grid), dim3(kNT), (size_t)P.total, st, A);
+  return launch_pdl(k_expert_ring<WBITS, WG32, AG32, MODE, TM>, dim3(grid), dim3(kNT), (size_t)P.total, st, A);
 }
 
+template <int WBITS, bool WG32, bool AG32, int TM>
+cudaError_t launch_mode_tm(int mode, const RingArgs& A, cudaStream_t st) {
+  if (mode == 0) return launch_ring_t<WBITS, WG32, AG32, 0, TM>(A, st);
+  if (mode == 1) return launch_ring_t<WBITS, WG32, AG32, 1, TM>(A, st);
+  if constexpr (AG32) return launch_ring_t<WBITS, WG32, AG32, 2, TM>(A, st);
+  return cudaErrorInvalidValue;               // the fused mode needs group-32 activations
+}
+
+// One token per pass (decode) gets consumers compiled for exactly one token.
 template <int WBITS, bool WG32, bool AG32>
 cudaError_t launch_mode(int mode, const RingArgs& A, cudaStream_t st) {
-  if (mode == 0) return launch_ring_t<WBITS, WG32, AG32, 0>(A, st);
-  if (mode == 1) return launch_ring_t<WBITS, WG32, AG32, 1>(A, st);
-  if constexpr (AG32) return launch_ring_t<WBITS, WG32, AG32, 2>(A, st);
-  return cudaErrorInvalidValue;               // the fused mode needs group-32 activations
+  return A.tm == 1 ? launch_mode_tm<WBITS, WG32, AG32, 1>(mode, A, st)
+                   : launch_mode_tm<WBITS, WG32, AG32, kTMP>(mode, A, st);
 }
 
 }  // namespace

@@ -56,56 +56,106 @@ __global__ void __launch_bounds__(256) k_router_small(const float* __restrict__ 
   }
 }
 
-// Large T: 64x64 output tile per CTA, each thread a 4x4 register tile. The K loop
-// walks the 32-element chunks in order; within a chunk every output runs its own
-// fma chain from +0 and is then added to the output's running total.
+// Large T: a TT x 64 (tokens x experts) output tile per CTA, each thread a (TT/16) x 4
+// register tile. The K loop walks the 32-element chunks in order; within a chunk every output
+// runs its own fma chain from +0, which is then added to the output's running total. The
+// next chunk's x and W_r slices are loaded (float4) into registers while the current one is
+// computed, then stored into the other shared-memory buffer: one barrier per chunk.
+template <int TT>
 __global__ void __launch_bounds__(256) k_router_tiled(const float* __restrict__ x,
                                                       const float* __restrict__ wr, int T, int E,
                                                       int H, float* __restrict__ logits) {
-  __shared__ __align__(16) float xs[32][68];
-  __shared__ __align__(16) float ws[32][68];
+  constexpr int RT = TT / 16;                      // token rows per thread
+  constexpr int XV = TT * 8 / 256;                 // float4 of x per thread per chunk
+  __shared__ __align__(16) float xs[2][32][TT + 4];
+  __shared__ __align__(16) float ws[2][32][64 + 4];
   pdl_wait();
   pdl_trigger();
-  const int tb = blockIdx.y * 64, eb = blockIdx.x * 64;
+  const int tb = blockIdx.y * TT, eb = blockIdx.x * 64;
   const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
-  float total[4][4];
+  const int C = H / 32;
+  float4 xr[XV], wrg[2];
+  auto load = [&](int c) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int v = 0; v < XV; ++v) {
+      const int l = threadIdx.x + 256 * v, rr = l >> 3, k4 = l & 7;
+      const int t = tb + rr;
+      xr[v] = t < T ? __ldg(reinterpret_cast<const float4*>(x + (int64_t)t * H + 32 * c) + k4)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int l = threadIdx.x + 256 * v, rr = l >> 3, k4 = l & 7;
+      const int e = eb + rr;
+      wrg[v] = e < E ? __ldg(reinterpret_cast<const float4*>(wr + (int64_t)e * H + 32 * c) + k4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto store = [&](int b) {
+#pragma unroll
+    for (int v = 0; v < XV; ++v) {
+      const int l = threadIdx.x + 256 * v, rr = l >> 3, k = 4 * (l & 7);
+      xs[b][k][rr] = xr[v].x;
+      xs[b][k + 1][rr] = xr[v].y;
+      xs[b][k + 2][rr] = xr[v].z;
+      xs[b][k + 3][rr] = xr[v].w;
+    }
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int l = threadIdx.x + 256 * v, rr = l >> 3, k = 4 * (l & 7);
+      ws[b][k][rr] = wrg[v].x;
+      ws[b][k + 1][rr] = wrg[v].y;
+      ws[b][k + 2][rr] = wrg[v].z;
+      ws[b][k + 3][rr] = wrg[v].w;
+    }
+  };
+  float total[RT][4];
+#pragma unroll
+  for (int i = 0; i < RT; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) total[i][j] = 0.0f;
-  for (int c = 0; c < H / 32; ++c) {
-    for (int l = threadIdx.x; l < 64 * 32; l += 256) {
-      const int rr = l >> 5, kk = l & 31;
-      const int t = tb + rr, e = eb + rr;
-      xs[kk][rr] = t < T ? x[(int64_t)t * H + 32 * c + kk] : 0.0f;
-      ws[kk][rr] = e < E ? wr[(int64_t)e * H + 32 * c + kk] : 0.0f;
-    }
-    __syncthreads();
-    float part[4][4];
+  load(0);
+  store(0);
+  __syncthreads();
+  for (int c = 0; c < C; ++c) {
+    const int b = c & 1;
+    if (c + 1 < C) load(c + 1);
+    float part[RT][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < RT; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) part[i][j] = 0.0f;
 #pragma unroll 8
     for (int kk = 0; kk < 32; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[4] = {b.x, b.y, b.z, b.w};
+      float av[RT];
+      if constexpr (RT == 4) {
+        const float4 a = *reinterpret_cast<const float4*>(&xs[b][kk][ty * 4]);
+        av[0] = a.x;
+        av[1] = a.y;
+        av[2] = a.z;
+        av[3] = a.w;
+      } else {
+        const float2 a = *reinterpret_cast<const float2*>(&xs[b][kk][ty * 2]);
+        av[0] = a.x;
+        av[1] = a.y;
+      }
+      const float4 bw = *reinterpret_cast<const float4*>(&ws[b][kk][tx * 4]);
+      const float bv[4] = {bw.x, bw.y, bw.z, bw.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < RT; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) part[i][j] = __fmaf_rn(av[i], bv[j], part[i][j]);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < RT; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) total[i][j] = __fadd_rn(total[i][j], part[i][j]);
+    if (c + 1 < C) store(b ^ 1);
     __syncthreads();
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = tb + ty * 4 + i;
+  for (int i = 0; i < RT; ++i) {
+    const int t = tb + ty * RT + i;
     if (t >= T) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -126,8 +176,15 @@ void launch_router_logits(const float* x, const float* wr, int T, int E, int H, 
     launch_pdl(k_router_small<TT>, grid, dim3(threads), TT * C * sizeof(float), st, x, wr, T, E, H,
                logits);
   } else {
-    dim3 grid((E + 63) / 64, (T + 63) / 64);
-    launch_pdl(k_router_tiled, grid, dim3(256), 0, st, x, wr, T, E, H, logits);
+    // 32-token tiles when 64-token ones would leave SMs idle
+    const int64_t tiles64 = (int64_t)((E + 63) / 64) * ((T + 63) / 64);
+    if (tiles64 < 2 * 148) {
+      dim3 grid((E + 63) / 64, (T + 31) / 32);
+      launch_pdl(k_router_tiled<32>, grid, dim3(256), 0, st, x, wr, T, E, H, logits);
+    } else {
+      dim3 grid((E + 63) / 64, (T + 63) / 64);
+      launch_pdl(k_router_tiled<64>, grid, dim3(256), 0, st, x, wr, T, E, H, logits);
+    }
   }
 }
 

@@ -6,8 +6,10 @@
 
 namespace moe {
 
-// Poll limit of a bounded mbarrier wait (with nanosleep back-off: well over 100 ms).
-constexpr uint32_t kWaitLimit = 1u << 22;
+// A bounded mbarrier wait: up to kWaitTries suspending tests of kWaitSuspendNs each (the
+// thread sleeps until the phase completes or the suspension ends), about a second in all.
+constexpr uint32_t kWaitTries = 1000;
+constexpr uint32_t kWaitSuspendNs = 1000000;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -44,12 +46,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of `bar` to complete; false if the poll limit ran out.
+// Test for completion of phase `parity`, suspending the thread up to `ns` nanoseconds while
+// the phase is still open (it resumes as soon as the phase completes).
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete; false if the bound ran out.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (i >= 32) __nanosleep(64);
-  }
+  for (uint32_t i = 0; i < kWaitTries; ++i)
+    if (mbar_try_wait_suspend(bar, parity, kWaitSuspendNs)) return true;
   return false;
 }
 
