@@ -191,7 +191,7 @@ __device__ __forceinline__ uint32_t mma_stage_bytes() {
 template <int WBITS, bool GATEUP>
 __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_constant__ MmaArgs A) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* base = smem_align1024(smem_raw);
   uint64_t* full = reinterpret_cast<uint64_t*>(base + kMmaNS * MmaStage::BYTES);
   uint64_t* prep = full + kMmaNS;
   uint64_t* empty = prep + kMmaNS;

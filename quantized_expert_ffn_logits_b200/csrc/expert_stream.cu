@@ -82,9 +82,6 @@ inline int ring_tokens(int K, int max_tokens) {
   return tm;
 }
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
 
 // One work unit as the kernel sees it.
 struct Unit {
@@ -560,7 +557,7 @@ __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& 
 template <int WBITS, bool WG32, bool AG32, int MODE, int TM>
 __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ RingArgs A) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* base = align1024(smem_raw);
+  uint8_t* base = smem_align1024(smem_raw);
   const RingPlan P = ring_plan(A.kmax, A.tm);
   Ring R;
   R.ring = base + P.ring;

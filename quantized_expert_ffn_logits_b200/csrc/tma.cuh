@@ -15,6 +15,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte boundary at or after the start of a shared-memory array, by pointer
+// arithmetic on the array itself (no round trip through an integer), so the compiler still
+// knows every pointer derived from it is shared memory and emits shared-memory loads.
+__device__ __forceinline__ uint8_t* smem_align1024(uint8_t* smem) {
+  return smem + ((1024u - (smem_u32(smem) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
