@@ -219,17 +219,23 @@ MOE_API size_t moe_layer_workspace_bytes(int32_t T, const moe_expert_blob* exper
  *   hidden size, wtype and wscale as `experts` and its own intermediate size.
  * workspace: device buffer of ws_bytes >= moe_layer_workspace_bytes(); it holds every
  * intermediate (quantized x, logits, routing, grouping, quantized h) and, in its first 256
- * bytes, a control block (device status word, routing ticket counter). The control block must
- * be zero before the workspace is first used (allocate it zeroed, e.g. cudaMemset once); the
- * library leaves it consistent after every call. Calls that share a workspace must be ordered
- * on one stream.
- * Launch sequence: for T <= 32 one routing kernel (activation quantization, logits, top-k and
- * grouping; the last CTA to finish its logit does the selection), larger T four; then, with
- * group-32 activations, one expert kernel that covers the routed and the shared experts: per
- * work unit (expert, 64 intermediate indices) gate/up, SwiGLU, h quantization and the unit's
- * share of the down projection, added into y. With per-token activation scales h needs all of
- * I first: gate/up, h quantization, then down as separate launches. Kernels use programmatic
- * dependent launch, so under stream capture the graph gets programmatic edges. */
+ * bytes, a control block (device status word, routing ticket, wait record, and at bytes 16-23
+ * the single-token grid-barrier counter). The control block must be zero before the workspace
+ * is first used (allocate it zeroed, e.g. cudaMemset once); the library leaves it consistent
+ * after every call. Calls that share a workspace must be ordered on one stream.
+ * Launch sequence: one token with group-32 activations (decode) is ONE launch: every CTA of
+ * the expert kernel quantizes the token, computes the router logits of a share of the
+ * experts and zeroes a share of y; after a grid barrier (all CTAs resident: the grid is at
+ * most one CTA per SM) every CTA selects the same top-k and streams its work units. Other
+ * calls: for T <= 32 one routing kernel (activation quantization, logits, top-k and grouping;
+ * the last CTA to finish its logit does the selection), larger T four; then, with group-32
+ * activations, one expert kernel that covers the routed and the shared experts: per work unit
+ * (expert, 64 intermediate indices) gate/up, SwiGLU, h quantization and the unit's share of
+ * the down projection, added into y. With per-token activation scales h needs all of I first:
+ * gate/up, h quantization, then down as separate launches. Kernels use programmatic dependent
+ * launch, so under stream capture the graph gets programmatic edges; router_w and the expert
+ * blobs are model parameters, read (the single-token kernel: router rows staged) before a
+ * kernel waits for its predecessor in the stream, so they must not be written by it. */
 MOE_API moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
                              const float* router_bias, const moe_expert_blob* experts,
                              const moe_expert_blob* shared, const moe_route_cfg* cfg, float* y,
@@ -311,8 +317,10 @@ MOE_API moe_status moe_expert_group_dots(const moe_expert_blob* blob, int32_t wh
  * during the last call (MOE_ERR_TIMEOUT): [2] = pass (1 gate/up, 2 down) | wait << 4 | ring
  * stage or buffer << 8, with wait 0 = producer waiting for a free stage, 1 = consumer waiting
  * for a chunk, 2 / 4 = producer draining chunks / activation copies before exit, 3 = producer
- * waiting for a free activation buffer, 5 = consumer waiting for activation rows;
- * [3] = the CTA index; both 0 otherwise.
+ * waiting for a free activation buffer, 5 = consumer waiting for activation rows, 6 = the
+ * single-token kernel's grid barrier, 7 = its staged router rows;
+ * [3] = the CTA index; both 0 otherwise. After MOE_ERR_TIMEOUT the routing ticket and the
+ * grid-barrier counter may be mid-call: reading the status resets them (not words 2-3).
  * Reads and clears the device status word of a moe_layer_forward / moe_permute workspace.
  * Synchronizes `stream`. Returns MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT as
  * recorded by the kernels, or MOE_ERR_CUDA if the copy fails. */

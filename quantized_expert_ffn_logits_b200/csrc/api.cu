@@ -17,6 +17,9 @@ inline int64_t al256(int64_t v) { return (v + 255) & ~int64_t(255); }
 
 // Batches up to this many tokens take the single-launch routing kernel.
 constexpr int32_t kFusedRouteMaxT = 32;
+// Control block at the start of a layer workspace: status word, routing ticket, wait record
+// (words 0-3), single-token grid-barrier counter (bytes 16-23).
+constexpr int64_t kControlBytes = 256;
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 struct BlobOffsets {
@@ -93,7 +96,7 @@ Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k,
   };
   const int64_t P = (int64_t)T * k;
   const int64_t C = (T + 31) / 32;
-  L.status = take(256);
+  L.status = take(kControlBytes);
   L.qx = take((int64_t)T * H);
   L.sx = take(ag32 ? (int64_t)T * (H / 32) * 2 : (int64_t)T * 4);
   L.logits = take((int64_t)T * E * 4);
@@ -161,6 +164,12 @@ Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k,
 bool use_mma(int32_t T, const moe_expert_blob* experts, const moe_route_cfg* cfg) {
   return T > kFusedRouteMaxT && cfg->act == MOE_ACT_G32_F16 && experts->wscale == MOE_SCALE_G32_F16 &&
          (cfg->flags & MOE_FLAG_FORCE_GEMV) == 0;
+}
+
+// One token with group-32 activations: routing and every expert in one launch (the expert
+// kernel routes the token itself before a grid barrier).
+bool use_decode(int32_t T, const moe_expert_blob* experts, const moe_route_cfg* cfg) {
+  return T == 1 && cfg->act == MOE_ACT_G32_F16 && experts->n_experts <= 512 && experts->hidden % 128 == 0;
 }
 
 struct LayerPlan {
@@ -434,9 +443,12 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     }
   };
 
+  moe::RouteArgs r;
+  std::memset(&r, 0, sizeof(r));
+  const bool decode = use_decode(T, experts, cfg);
   if (T <= kFusedRouteMaxT) {
-    // 1-3. activation quantization, router logits, top-k and grouping in one launch
-    moe::RouteArgs r;
+    // 1-3. activation quantization, router logits, top-k and grouping in one launch (one
+    //      token: inside the expert kernel, launched below)
     r.x = x;
     r.wr = router_w;
     r.bias = bias;
@@ -457,8 +469,9 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     r.g = g;
     r.status = status;
     r.ticket = reinterpret_cast<unsigned*>(ws + L.status + 4);
+    r.gbar = reinterpret_cast<unsigned long long*>(ws + L.status + 16);
     mk.begin(MOE_STAGE_QUANT_X);
-    keep(moe::launch_route_fused(r, st), "routing kernel");
+    if (!decode) keep(moe::launch_route_fused(r, st), "routing kernel");
     mk.end(MOE_STAGE_QUANT_X);
     for (int sg = MOE_STAGE_ROUTER; sg <= MOE_STAGE_GROUP; ++sg) {
       mk.begin(sg);
@@ -591,7 +604,16 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
       keep(moe::launch_expert_mma(false, m, st), "tensor-core down kernel");
     }
   };
-  if (moe::experts_fusable(ra, sap)) {
+  if (decode) {
+    // one token: routing (1-3) and 4+5 in one persistent grid
+    mk.begin(MOE_STAGE_GATE_UP);
+    keep(moe::launch_decode(r, ra, sap, rd, sdp, st), "decode kernel");
+    mk.end(MOE_STAGE_GATE_UP);
+    for (int sg : {MOE_STAGE_DOWN, MOE_STAGE_QUANT_H}) {
+      mk.begin(sg);
+      mk.end(sg);
+    }
+  } else if (moe::experts_fusable(ra, sap)) {
     // 4+5 in one persistent grid: per unit (expert, 64 intermediate indices) the gate/up
     // pass, SwiGLU and h quantization, then the unit's share of the down projection
     mk.begin(MOE_STAGE_GATE_UP);
@@ -653,6 +675,7 @@ int32_t moe_layer_kernel_count(int32_t T, const moe_expert_blob* experts,
                                const moe_expert_blob* shared, const moe_route_cfg* cfg) {
   if (moe_layer_workspace_bytes(T, experts, shared, cfg) == 0) return -1;
   if (T == 0) return 0;
+  if (use_decode(T, experts, cfg)) return 1;   // routing and experts in one grid
   int n = T <= kFusedRouteMaxT ? 1 : 4;        // routing (fused, or quantize/logits/top-k/grouping)
   if (use_mma(T, experts, cfg)) n += 4;                                     // tensor-core tile plan, gather, gate/up, down
   if (cfg->act == MOE_ACT_G32_F16) return n + 1;   // gate/up and down of all experts in one grid
@@ -686,6 +709,13 @@ moe_status moe_read_device_status(void* workspace, size_t ws_bytes, void* stream
   if (e != cudaSuccess) return cuda_fail("status synchronize", e);
   e = cudaMemsetAsync(workspace, 0, 4, st);
   if (e != cudaSuccess) return cuda_fail("status clear", e);
+  if (h == MOE_ERR_TIMEOUT && ws_bytes >= (size_t)kControlBytes) {
+    // a wait gave up: the routing ticket (word 1) and the grid-barrier counter (bytes 16-23)
+    // may be left mid-call; the wait record (words 2-3) stays readable
+    e = cudaMemsetAsync(static_cast<uint8_t*>(workspace) + 4, 0, 4, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(static_cast<uint8_t*>(workspace) + 16, 0, kControlBytes - 16, st);
+    if (e != cudaSuccess) return cuda_fail("control block reset", e);
+  }
   return static_cast<moe_status>(h);
 }
 

@@ -45,8 +45,12 @@ constexpr int kSmemMax = 227 * 1024;
 
 // Shared-memory plan (offsets from a 1024-aligned base). Activation buffer b holds tm rows
 // of K codes, then (g32 activations) tm rows of G fp16 scales.
+// Single-token routing scratch (RingPlan::route): se, swt, sj, sidx, sw [32] each, then
+// flag words.
+constexpr int kRouteBytes = 5 * 32 * 4 + 16;
+
 struct RingPlan {
-  int ring, sring, bars, abuf, abytes, ascale, xsum, sxf, idot, ubuf, hq, info, total;
+  int ring, sring, bars, abuf, abytes, ascale, xsum, sxf, idot, ubuf, hq, info, route, total;
 };
 
 __host__ __device__ inline RingPlan ring_plan(int K, int tm) {
@@ -71,6 +75,7 @@ __host__ __device__ inline RingPlan ring_plan(int K, int tm) {
   p.ubuf = take(2 * tm * 64 * 4);               // gate / up stage values of a pass
   p.hq = take(2 * tm * 64 + 2 * tm * 4 + 2 * tm * 4);   // h codes (+ de-interleaved), scales, sums
   p.info = take(3 * kTMP * 4 + 16);             // tokens, weights, abort flag
+  p.route = take(kRouteBytes);                 // single-token routing (in-kernel selection)
   p.total = o + 1024;                           // slack for aligning the base
   return p;
 }
@@ -190,7 +195,317 @@ struct RingArgs {
   int per;                 // units per routed expert (I / 64)
   int tm, kmax;
   int mma_min;             // experts with this many slots are left to the tensor-core path
+  RouteArgs r;             // MODE 3 (one token): the routing done inside the kernel
 };
+
+// int4 weights: each 8-byte word of the activation rows de-interleaved into its even, then
+// its odd elements (the order of a packed weight word's low and high nibbles), and the sum
+// of every group's 32 codes (the unsigned-nibble correction of the int4 dot).
+__device__ __forceinline__ void act_deinterleave(uint8_t* xs, int words, int tid, int nt) {
+  for (int l = tid; l < words; l += nt) {
+    uint2* wp = reinterpret_cast<uint2*>(xs) + l;
+    const uint2 v = *wp;
+    uint2 o;
+    deinterleave8(v.x, v.y, o.x, o.y);
+    *wp = o;
+  }
+}
+__device__ __forceinline__ void act_group_sums(const uint8_t* xs, int* xsum, int m, int K, int tid, int nt) {
+  const int G = K / 32;
+  for (int l = tid; l < m * G; l += nt) {
+    const uint4* q4 = reinterpret_cast<const uint4*>(xs + (l / G) * K + 32 * (l % G));
+    const uint4 a0 = q4[0], a1 = q4[1];
+    int sacc = __dp4a((int)a0.x, 0x01010101, 0);
+    sacc = __dp4a((int)a0.y, 0x01010101, sacc);
+    sacc = __dp4a((int)a0.z, 0x01010101, sacc);
+    sacc = __dp4a((int)a0.w, 0x01010101, sacc);
+    sacc = __dp4a((int)a1.x, 0x01010101, sacc);
+    sacc = __dp4a((int)a1.y, 0x01010101, sacc);
+    sacc = __dp4a((int)a1.z, 0x01010101, sacc);
+    sacc = __dp4a((int)a1.w, 0x01010101, sacc);
+    xsum[l] = sacc;
+  }
+}
+
+// ------------------------------------------------------------------ single-token routing
+// MODE 3 (one token, group-32 activations) begins with the routing that other calls run as a
+// separate kernel, so a decode step is one launch. Every CTA quantizes the token's
+// activations (groups of 32: scale = fp16(max|x| / 127), code = x / scale rounded and
+// clamped; GLM-5.2 colibri page, "Quantization kernels") straight into its activation
+// buffer 0, computes the router logits of experts blockIdx.x, blockIdx.x + grid, ... in the
+// fixed fp32 order (32-element fma chunks from +0, chunk partials added in chunk order) and
+// zeroes its share of y. After a grid barrier every CTA reads the E logits and makes the
+// same top-k selection (all keys ranked in parallel; softmax or sigmoid weights as in
+// topk.cuh); CTA 0 also writes the routing and grouping views of the workspace.
+struct RouteSmem {
+  int* se;        // [k] selected experts, ascending (active-expert order)
+  float* swt;     // [k] their routing weights
+  int* sj;        // [k] their positions in the token's top-k list (pair index)
+  int* sidx;      // [k] the top-k list in selection order
+  float* sw;      // [k] its weights
+  volatile int* flag;
+};
+
+// Bound of the grid-barrier wait: 2^22 polls (each an L2 round trip: seconds in all).
+constexpr uint32_t kGridWaitTries = 1u << 22;
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Thread 0 of every CTA, after a CTA barrier: arrive, then wait until every CTA of the grid
+// has arrived. The counter is a multiple of 1024 when a call starts (grids are <= 1024
+// CTAs); this call's arrivals take base .. base + grid - 1 and the last one moves the
+// counter on to base + 1024 for the next call. False if the wait gave up.
+__device__ __forceinline__ bool grid_barrier(unsigned long long* ctr) {
+  __threadfence();
+  const unsigned long long old = atomicAdd(ctr, 1ull);
+  const unsigned long long target = (old & ~1023ull) + gridDim.x;
+  if (old + 1 == target) atomicAdd(ctr, 1024ull - gridDim.x);
+  for (uint32_t i = 0; i < kGridWaitTries; ++i)
+    if (ld_acquire_u64(ctr) >= target) return true;
+  return false;
+}
+
+// Scratch use of the (still idle) ring during the routing: the router rows of the CTA's
+// experts at 0 (when they fit kRowBytes; copied before the wait for the preceding kernel),
+// logit chunk partials at kRowBytes.
+constexpr int kRowBytes = 96 * 1024;
+constexpr int kPartFloats = (kNS * kSP * kPiece - kRowBytes) / 4;
+
+__device__ __forceinline__ int route_experts_of_cta(int E) {
+  return (int)blockIdx.x < E ? (E - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+}
+
+// Thread 0, before the wait for the preceding kernel: stage this CTA's router rows (model
+// parameters, not written by the preceding kernel) into the ring; completes on `bar`.
+// False if they do not fit (the logits then read them from global memory).
+__device__ __forceinline__ bool stage_router_rows(const RouteArgs& r, uint8_t* ring, uint64_t* bar) {
+  const int ne = route_experts_of_cta(r.E);
+  const uint32_t row = (uint32_t)r.H * 4;
+  if (ne == 0 || ne * row > (uint32_t)kRowBytes) return false;
+  mbar_arrive_expect_tx(bar, ne * row);
+  for (int j = 0; j < ne; ++j)
+    bulk_load(ring + j * row, r.wr + (int64_t)(blockIdx.x + j * gridDim.x) * r.H, row, bar);
+  return true;
+}
+
+// Every thread of the CTA. False when a wait gave up (status recorded). rows_bar: the
+// router rows were staged by stage_router_rows and complete on it.
+__device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Ring& R, const RouteSmem& S,
+                                uint64_t* rows_bar) {
+  volatile int* flag = S.flag;
+  const int tid = threadIdx.x, H = r.H, G = H / 32, C = H / 32, E = r.E, k = r.k;
+  const bool cta0 = blockIdx.x == 0;
+  if (cta0 && tid == 0) {
+    r.status[0] = 0;
+    r.status[2] = 0;
+    r.status[3] = 0;
+  }
+  // 1. activation codes and group scales: 8 threads per group, 4 elements each (8 G is a
+  //    multiple of 32, so a warp's lanes are all in range or all out)
+  uint8_t* xs = R.abuf;
+  __half* sxs = reinterpret_cast<__half*>(xs + P.ascale);
+  for (int l = tid; l < 8 * G; l += kNT) {
+    const int g = l >> 3;
+    const float4 v = __ldg(reinterpret_cast<const float4*>(r.x) + l);
+    float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+    const float sc = f16_round(__fdiv_rn(m, 127.0f));
+    const uint32_t word = (uint32_t)(uint8_t)(int8_t)quant_code(v.x, sc, 127.0f) |
+                          (uint32_t)(uint8_t)(int8_t)quant_code(v.y, sc, 127.0f) << 8 |
+                          (uint32_t)(uint8_t)(int8_t)quant_code(v.z, sc, 127.0f) << 16 |
+                          (uint32_t)(uint8_t)(int8_t)quant_code(v.w, sc, 127.0f) << 24;
+    reinterpret_cast<uint32_t*>(xs)[l] = word;
+    if ((l & 7) == 0) sxs[g] = __float2half_rn(sc);
+    if (cta0) {
+      reinterpret_cast<uint32_t*>(r.qx)[l] = word;
+      if ((l & 7) == 0) reinterpret_cast<__half*>(r.sx)[g] = __float2half_rn(sc);
+    }
+  }
+  // 2. this CTA's share of y = 0 (ordered before every CTA's adds by the grid barrier)
+  float4* y4 = reinterpret_cast<float4*>(r.y);
+  for (int l = blockIdx.x * kNT + tid; l < H / 4; l += gridDim.x * kNT) y4[l] = make_float4(0.f, 0.f, 0.f, 0.f);
+  // 3. logits of this CTA's experts, as many at a time as their chunk partials fit the ring
+  //    (idle until the barrier): partials first, then each expert's added in chunk order
+  float* part = reinterpret_cast<float*>(R.ring + kRowBytes);
+  const int ne = route_experts_of_cta(E);
+  const int nb = kPartFloats / C;
+  if (rows_bar) {
+    // the router rows (copied while the preceding kernel finished)
+    const bool ok = mbar_wait(rows_bar, 0);
+    if (tid == 0) *flag = ok;
+    __syncthreads();
+    if (!*flag) {
+      if (tid == 0) wait_failed(r.status, 1, 7, 0);
+      return false;
+    }
+  }
+  for (int j0 = 0; j0 < ne; j0 += nb) {
+    const int nj = min(nb, ne - j0);
+    for (int l = tid; l < nj * C; l += kNT) {
+      const int j = l / C, c = l - j * C;
+      const int e = blockIdx.x + (j0 + j) * gridDim.x;
+      const float4* w4 = rows_bar ? reinterpret_cast<const float4*>(R.ring + (int64_t)(j0 + j) * H * 4) + 8 * c
+                                  : reinterpret_cast<const float4*>(r.wr + (int64_t)e * H + 32 * c);
+      const float4* x4 = reinterpret_cast<const float4*>(r.x + 32 * c);
+      float4 wv[8];
+#pragma unroll
+      for (int v = 0; v < 8; ++v) wv[v] = rows_bar ? w4[v] : __ldg(w4 + v);
+      float acc = 0.0f;
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {
+        const float4 xv = __ldg(x4 + v);
+        acc = __fmaf_rn(xv.x, wv[v].x, acc);
+        acc = __fmaf_rn(xv.y, wv[v].y, acc);
+        acc = __fmaf_rn(xv.z, wv[v].z, acc);
+        acc = __fmaf_rn(xv.w, wv[v].w, acc);
+      }
+      part[l] = acc;
+    }
+    __syncthreads();
+    for (int j = tid; j < nj; j += kNT) {
+      const float* pj = part + j * C;
+      float total = 0.0f;
+      int c = 0;
+      for (; c + 8 <= C; c += 8) {
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) v[q] = pj[c + q];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) total = __fadd_rn(total, v[q]);
+      }
+      for (; c < C; ++c) total = __fadd_rn(total, pj[c]);
+      r.logits[blockIdx.x + (j0 + j) * gridDim.x] = total;
+    }
+    __syncthreads();
+  }
+  __syncthreads();
+  if (tid == 0) *flag = grid_barrier(r.gbar) ? 1 : 0;
+  __syncthreads();
+  if (!*flag) {
+    if (tid == 0) wait_failed(r.status, 1, 6, 0);
+    return false;
+  }
+  // 5. top-k (every CTA, same result): every key ranks itself against all E keys in
+  //    parallel (rank = keys larger, or equal with a lower expert index: descending, ties
+  //    to the lower expert); then warp 0 forms the routing weights of the k selected
+  float* slog = reinterpret_cast<float*>(R.ring);           // scratch again: [E] logits
+  float* skey = slog + 512;                                  //                [E] selection keys
+  if (tid < 32) S.sidx[tid] = -1;
+  for (int i = tid; i < E; i += kNT) {
+    const float L = __ldcg(r.logits + i);
+    slog[i] = L;
+    skey[i] = r.score == 0 ? L : __fadd_rn(csigmoid(L), r.bias ? r.bias[i] : 0.0f);
+  }
+  __syncthreads();
+  for (int i = tid; i < E; i += kNT) {
+    const float kv = skey[i];
+    int rank = 0, j = 0;
+    if ((E & 3) == 0) {
+      const float4* k4 = reinterpret_cast<const float4*>(skey);
+#pragma unroll 4
+      for (; j < E; j += 4) {
+        const float4 q = k4[j >> 2];
+        rank += (q.x > kv) | ((q.x == kv) & (j < i));
+        rank += (q.y > kv) | ((q.y == kv) & (j + 1 < i));
+        rank += (q.z > kv) | ((q.z == kv) & (j + 2 < i));
+        rank += (q.w > kv) | ((q.w == kv) & (j + 3 < i));
+      }
+    }
+    for (; j < E; ++j) rank += (skey[j] > kv) | ((skey[j] == kv) & (j < i));
+    if (rank < k) S.sidx[rank] = i;
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const int lane = tid;
+    const bool on = lane < k;
+    const int my_e = on ? S.sidx[lane] : 0;
+    const float myl = (my_e >= 0 && my_e < E) ? slog[my_e] : 0.0f;
+    float wv;
+    if (r.score == 0) {
+      const float lmax = __shfl_sync(0xffffffffu, myl, 0);
+      const float ex = on ? cexp(myl - lmax) : 0.0f;
+      float den;
+      if (r.renorm) {
+        den = warp_sum(ex);
+      } else {
+        float sacc = 0.0f;
+        for (int x = lane; x < E; x += 32) sacc += cexp(slog[x] - lmax);
+        den = warp_sum(sacc);
+      }
+      wv = ex / den * r.rsf;
+    } else {
+      const float sg = on ? csigmoid(myl) : 0.0f;
+      const float den = r.renorm ? warp_sum(sg) : 1.0f;
+      wv = sg / den * r.rsf;
+    }
+    if (on) S.sw[lane] = wv;
+  }
+  __syncthreads();
+  if (tid < k) {
+    const int ee = S.sidx[tid];
+    int pos = 0;
+    for (int j = 0; j < k; ++j) pos += S.sidx[j] < ee;
+    S.se[pos] = ee;
+    S.sj[pos] = tid;
+    S.swt[pos] = S.sw[tid];
+    if (cta0) {
+      r.idx[tid] = ee;
+      r.w[tid] = S.sw[tid];
+      r.g.act_expert[pos] = ee;
+      r.g.act_begin[pos] = pos;
+      r.g.perm[pos] = tid;
+      if (r.g.act_rows) r.g.act_rows[pos * 8] = 0;
+    }
+  }
+  if (cta0) {
+    for (int x = tid; x < E; x += kNT) {
+      int cnt = 0;
+      for (int j = 0; j < k; ++j) cnt += S.sidx[j] < x;
+      r.g.offsets[x] = cnt;
+    }
+    if (tid == 0) {
+      r.g.offsets[E] = k;
+      *r.g.n_active = k;
+      r.g.act_begin[k] = k;
+    }
+  }
+  __syncthreads();
+  return true;
+}
+
+// Work unit u of a MODE 3 grid: routed units (the token's k experts, ascending) first, then
+// the shared expert's. Slot of the routed pair = its active-expert index.
+__device__ __forceinline__ bool unit_of_token(const RingArgs& A, const RouteSmem& S, int u, Unit& U, bool report) {
+  if (u < A.routed) {
+    U.shd = false;
+    U.ai = u / A.per;
+    U.sub = u - U.ai * A.per;
+    U.e = S.se[U.ai];
+    U.s0 = U.ai;
+    U.s1 = U.ai + 1;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) U.rows8[q] = 0;
+    if (U.ai >= A.r.k || U.e < 0 || U.e >= A.r.E) {
+      if (report) set_status(A.r.status, kStatusDeviceCheck);
+      return false;
+    }
+    return true;
+  }
+  if (!A.has_shared) return false;
+  U.shd = true;
+  U.ai = 0;
+  U.e = 0;
+  U.s0 = 0;
+  U.s1 = 1;
+  U.sub = u - A.routed;
+  return true;
+}
 
 // ------------------------------------------------------------------ producer
 // Lane 0 of the producer warp: every chunk of every pass of every unit of this CTA, in the
@@ -200,7 +515,7 @@ struct RingArgs {
 // (all H rows x its 64 columns) in chunks of whole 128-row blocks, with their scales
 // (fp16 [block][2][128] or fp32 per row).
 template <int WBITS, bool WG32, bool AG32, int MODE>
-__device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& R) {
+__device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& R, const RouteSmem& S) {
   constexpr int PPG = WBITS == 8 ? 2 : 1;
   constexpr int PPU = WBITS == 8 ? 4 : 2;   // pieces of a row's 64-column down slice
   constexpr int NBC = kSP / PPU;            // 128-row down blocks per chunk
@@ -223,7 +538,9 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
   };
   for (int u = blockIdx.x; u < A.units && ok; u += gridDim.x) {
     Unit U;
-    if (!unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, false, A.mma_min))
+    if (MODE == 3 ? !unit_of_token(A, S, u, U, false)
+                  : !unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, false,
+                             A.mma_min))
       continue;
     const ExpertArgs& g = A.x[0][U.shd ? 1 : 0];
     const ExpertArgs& d = A.x[1][U.shd ? 1 : 0];
@@ -240,6 +557,7 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
           ok = push(wsrc + (int64_t)p0 * kPiece, (uint32_t)np * kPiece,
                     ssrc + (int64_t)(p0 / PPG) * 256, WG32 ? (uint32_t)(np / PPG) * 256 : 0u);
           if (!ok || p0 != 0) continue;
+          if (MODE == 3) continue;   // the CTA quantized the token's activations itself
           // this pass's activation rows, behind its first chunk
           const int b = pidx & 1;
           if (pidx >= 2 && !mbar_wait(&R.aempty[b], ((pidx >> 1) - 1) & 1)) {
@@ -594,12 +912,40 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
     }
     fence_barrier_init();
   }
+  RouteSmem S;
+  S.se = reinterpret_cast<int*>(base + P.route);
+  S.swt = reinterpret_cast<float*>(S.se + 32);
+  S.sj = S.se + 64;
+  S.sidx = S.se + 96;
+  S.sw = S.swt + 96;
+  S.flag = reinterpret_cast<volatile int*>(S.se + 160);
+  volatile int* rows_flag = S.se + 161;
   __syncthreads();
+  bool rows = false;
+  if (MODE == 3) {
+    if (threadIdx.x == 0) *rows_flag = stage_router_rows(A.r, R.ring, &R.afull[0]);
+    __syncthreads();
+    rows = *rows_flag != 0;
+  }
   pdl_wait();
+  if (MODE == 3) {
+    // one token: routing first. Its grid barrier also means every CTA of this grid is
+    // resident before any CTA lets the next kernel launch (and take SMs).
+    if (!route_one_token(A.r, P, R, S, rows ? &R.afull[0] : nullptr)) return;
+    if (WBITS == 4) {
+      act_deinterleave(R.abuf, A.kmax / 8, threadIdx.x, kNT);
+      __syncthreads();
+      act_group_sums(R.abuf, R.xsum, 1, A.kmax, threadIdx.x, kNT);
+      __syncthreads();
+    }
+    // the ring held the logit partials (generic stores); the bulk copies refill it
+    fence_async_smem();
+    __syncthreads();
+  }
   pdl_trigger();
 
   if (warp == kCW) {
-    if (lane == 0) ring_producer<WBITS, WG32, AG32, MODE>(A, P, R);
+    if (lane == 0) ring_producer<WBITS, WG32, AG32, MODE>(A, P, R, S);
     return;
   }
 
@@ -609,7 +955,9 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   uint32_t c = 0, pidx = 0, nblk = 0;       // chunks, gate/up passes, 8-group blocks consumed
   for (int u = blockIdx.x; u < A.units; u += gridDim.x) {
     Unit U;
-    if (!unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, ctid == 0, A.mma_min))
+    if (MODE == 3 ? !unit_of_token(A, S, u, U, ctid == 0)
+                  : !unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, ctid == 0,
+                             A.mma_min))
       continue;
     const ExpertArgs& g = A.x[0][U.shd ? 1 : 0];
     const ExpertArgs& d = A.x[1][U.shd ? 1 : 0];
@@ -619,7 +967,10 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
       named_bar(1, 32 * kCW);              // previous pass done with the per-pass arrays
       if (ctid < m) {
         const int slot = c0 + ctid;
-        if (MODE != 0) {
+        if (MODE == 3) {
+          toks[ctid] = 0;
+          wts[ctid] = U.shd ? 1.0f : S.swt[U.ai];
+        } else if (MODE != 0) {
           int p = U.shd ? slot : __ldcg(d.perm + slot);
           if (p < 0 || p >= (U.shd ? d.T : d.T * d.k)) {
             set_status(status, kStatusDeviceCheck);
@@ -645,8 +996,9 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
       }
       if (MODE != 1) {
         const int K = g.b.H, G = K / 32;
-        const bool copy_scales = AG32 && (G % 8) == 0;
-        const int b = pidx & 1;
+        // MODE 3: buffer 0 holds the token's codes and fp16 scales (and int4 prep) already
+        const bool copy_scales = MODE == 3 || (AG32 && (G % 8) == 0);
+        const int b = MODE == 3 ? 0 : pidx & 1;
         if (AG32 && !copy_scales)
           for (int l = ctid; l < m * G; l += 32 * kCW) {
             const int tt = l / G, gg = l - tt * G;
@@ -656,37 +1008,17 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
         uint8_t* xs = R.abuf + b * P.abytes;
         int* xsum = R.xsum + b * tm * G;
         bool aok = *abort == 0;
-        if (aok && !mbar_wait(&R.afull[b], (pidx >> 1) & 1)) {
+        if (MODE != 3 && aok && !mbar_wait(&R.afull[b], (pidx >> 1) & 1)) {
           *abort = 1;
           if (lane == 0) wait_failed(status, 1, 5, b);
           aok = false;
         }
-        if (WBITS == 4) {
+        if (WBITS == 4 && MODE != 3) {
           // de-interleave each 8-byte word into even / odd elements; per-group sums
           // (barriers taken by every consumer thread, whatever its wait returned)
-          if (aok)
-            for (int l = ctid; l < m * (K / 8); l += 32 * kCW) {
-              uint2* wp = reinterpret_cast<uint2*>(xs) + l;
-              const uint2 v = *wp;
-              uint2 o;
-              deinterleave8(v.x, v.y, o.x, o.y);
-              *wp = o;
-            }
+          if (aok) act_deinterleave(xs, m * (K / 8), ctid, 32 * kCW);
           named_bar(1, 32 * kCW);
-          if (aok)
-            for (int l = ctid; l < m * G; l += 32 * kCW) {
-              const uint4* q4 = reinterpret_cast<const uint4*>(xs + (l / G) * K + 32 * (l % G));
-              const uint4 a0 = q4[0], a1 = q4[1];
-              int sacc = __dp4a((int)a0.x, 0x01010101, 0);
-              sacc = __dp4a((int)a0.y, 0x01010101, sacc);
-              sacc = __dp4a((int)a0.z, 0x01010101, sacc);
-              sacc = __dp4a((int)a0.w, 0x01010101, sacc);
-              sacc = __dp4a((int)a1.x, 0x01010101, sacc);
-              sacc = __dp4a((int)a1.y, 0x01010101, sacc);
-              sacc = __dp4a((int)a1.z, 0x01010101, sacc);
-              sacc = __dp4a((int)a1.w, 0x01010101, sacc);
-              xsum[l] = sacc;
-            }
+          if (aok) act_group_sums(xs, xsum, m, K, ctid, 32 * kCW);
         }
         named_bar(1, 32 * kCW);
         const __half* sxh = copy_scales ? reinterpret_cast<const __half*>(xs + P.ascale) : nullptr;
@@ -696,7 +1028,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
         ring_consume<WBITS, WG32, AG32, TM>(K, m, tm, R, c, nblk, xs, sxh, R.sxf, xsum, idot, sw_row, v, abort,
                                         status, 1);
         __syncwarp();
-        if (lane == 0) mbar_arrive(&R.aempty[b]);
+        if (MODE != 3 && lane == 0) mbar_arrive(&R.aempty[b]);
         ++pidx;
         const bool is_up = row >= 64;
 #pragma unroll
@@ -719,7 +1051,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
               const int code = quant_code(h, sc, 127.0f);
               g.qh[(int64_t)slot * I + i] = (int8_t)code;
               if (lane == 0) g.sh[(int64_t)slot * IB + i / 32] = __float2half_rn(sc);
-              if (MODE == 2) {
+              if (MODE >= 2) {              // h stays on chip for the down pass
                 hq[q * 64 + il] = (uint8_t)(int8_t)code;
                 if (lane == 0) hs[2 * q + warp] = sc;
               }
@@ -779,6 +1111,10 @@ int sm_count() {
   return n[dev];
 }
 
+// MODE 3 grid: every unit its CTA, and at least one CTA per expert for the router logits (up
+// to one CTA per SM: the grid barrier needs all of them resident at once).
+int decode_grid(int units, int E) { return std::min(sm_count(), std::max(units, E)); }
+
 template <int WBITS, bool WG32, bool AG32, int MODE, int TM>
 cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
   const RingPlan P = ring_plan(A.kmax, A.tm);
@@ -789,7 +1125,7 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_bytes = P.total;
   }
-  const int grid = A.units < sm_count() ? A.units : sm_count();
+  const int grid = MODE == 3 ? decode_grid(A.units, A.r.E) : std::min(A.units, sm_count());
   if (grid <= 0) return cudaSuccess;
   return launch_pdl(k_expert_ring<WBITS, WG32, AG32, MODE, TM>, dim3(grid), dim3(kNT), (size_t)P.total, st, A);
 }
@@ -807,6 +1143,11 @@ template <int WBITS, bool WG32, bool AG32>
 cudaError_t launch_mode(int mode, const RingArgs& A, cudaStream_t st) {
   return A.tm == 1 ? launch_mode_tm<WBITS, WG32, AG32, 1>(mode, A, st)
                    : launch_mode_tm<WBITS, WG32, AG32, kTMP>(mode, A, st);
+}
+
+template <int WBITS, bool WG32>
+cudaError_t launch_decode_t(const RingArgs& A, cudaStream_t st) {
+  return launch_ring_t<WBITS, WG32, true, 3, 1>(A, st);
 }
 
 }  // namespace
@@ -841,6 +1182,39 @@ cudaError_t launch_experts(int mode, const ExpertArgs& gr, const ExpertArgs* gs,
     case 2: return launch_mode<4, true, false>(mode, A, st);
     case 1: return launch_mode<4, false, true>(mode, A, st);
     default: return launch_mode<4, false, false>(mode, A, st);
+  }
+}
+
+bool decode_fusable(const RouteArgs& r, const ExpertArgs& gr, const ExpertArgs* gs) {
+  if (r.T != 1 || !experts_fusable(gr, gs) || !r.ag32 || r.E > 512 || r.k > 32 || r.H != gr.b.H ||
+      r.H % 128 != 0 || !r.gbar)
+    return false;
+  return r.H / 32 <= kPartFloats;   // one expert's chunk partials fit the ring scratch
+}
+
+cudaError_t launch_decode(const RouteArgs& r, const ExpertArgs& gr, const ExpertArgs* gs, const ExpertArgs& dr,
+                          const ExpertArgs* ds, cudaStream_t st) {
+  if (!decode_fusable(r, gr, gs)) return cudaErrorInvalidValue;
+  RingArgs A;
+  std::memset(&A, 0, sizeof(A));
+  A.x[0][0] = gr;
+  A.x[0][1] = gs ? *gs : gr;
+  A.x[1][0] = dr;
+  A.x[1][1] = ds ? *ds : dr;
+  A.has_shared = gs != nullptr;
+  A.per = gr.b.I / 64;
+  A.routed = r.k * A.per;
+  A.units = A.routed + (gs ? gs->b.I / 64 : 0);
+  A.kmax = gr.b.H;
+  A.tm = 1;
+  A.mma_min = 0x7fffffff;
+  A.r = r;
+  const int sel = (gr.b.wbits == 8 ? 2 : 0) | (gr.b.wg32 ? 1 : 0);
+  switch (sel) {
+    case 3: return launch_decode_t<8, true>(A, st);
+    case 2: return launch_decode_t<8, false>(A, st);
+    case 1: return launch_decode_t<4, true>(A, st);
+    default: return launch_decode_t<4, false>(A, st);
   }
 }
 

@@ -131,8 +131,19 @@ struct RouteArgs {
   Grouping g;
   int* status;
   unsigned* ticket;       // zero between calls; the last CTA resets it
+  // grid barrier of the single-token expert kernel: a multiple of 1024 between calls (each
+  // call's CTAs arrive at base .. base + grid - 1, the last one moves it to base + 1024)
+  unsigned long long* gbar;
 };
 cudaError_t launch_route_fused(const RouteArgs& r, cudaStream_t st);
+
+// One token, group-32 activations: the routing (activation quantization, router logits, top-k,
+// grouping) runs inside the expert kernel -- every CTA computes some experts' logits, then
+// a grid barrier -- so the whole layer is one launch. decode_fusable() says whether
+// the call qualifies (T == 1, E <= 512, fused mode).
+bool decode_fusable(const RouteArgs& r, const ExpertArgs& gr, const ExpertArgs* gs);
+cudaError_t launch_decode(const RouteArgs& r, const ExpertArgs& gr, const ExpertArgs* gs, const ExpertArgs& dr,
+                          const ExpertArgs* ds, cudaStream_t st);
 
 #ifdef MOE_NO_PDL
 constexpr bool kUsePdl = false;

@@ -6,6 +6,12 @@
 
 namespace moe {
 
+// Orders this thread's generic-proxy shared-memory accesses before later async-proxy ones
+// (bulk copies, tensor-core operand reads) of the CTA.
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // A bounded mbarrier wait: up to kWaitTries suspending tests of kWaitSuspendNs each (the
 // thread sleeps until the phase completes or the suspension ends), about a second in all.
 constexpr uint32_t kWaitTries = 1000;
@@ -100,6 +106,13 @@ __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint3
       "%4;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// Bulk prefetch of global memory into L2 (16-byte aligned address, size a multiple of 16):
+// no shared-memory destination and no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
 }
 
 // Ampere-style asynchronous 16-byte copies global -> shared (L2 only), grouped by commit.

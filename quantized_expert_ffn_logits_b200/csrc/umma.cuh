@@ -30,11 +30,6 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Generic-proxy writes to shared memory made visible to the tensor core (async proxy).
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ MMA
 // D[tmem] (=|+=) A[smem] x B[smem]^T, 8-bit operands (signedness in the instruction
 // descriptor), int32 accumulator; issued by one thread.
