@@ -169,7 +169,8 @@ bool use_mma(int32_t T, const moe_expert_blob* experts, const moe_route_cfg* cfg
 // One token with group-32 activations: routing and every expert in one launch (the expert
 // kernel routes the token itself before a grid barrier).
 bool use_decode(int32_t T, const moe_expert_blob* experts, const moe_route_cfg* cfg) {
-  return T == 1 && cfg->act == MOE_ACT_G32_F16 && experts->n_experts <= 512 && experts->hidden % 128 == 0;
+  return T == 1 && cfg->act == MOE_ACT_G32_F16 && experts->n_experts <= 512 && experts->hidden % 128 == 0 &&
+         4 * experts->n_experts <= experts->hidden;
 }
 
 struct LayerPlan {

@@ -45,9 +45,9 @@ constexpr int kSmemMax = 227 * 1024;
 
 // Shared-memory plan (offsets from a 1024-aligned base). Activation buffer b holds tm rows
 // of K codes, then (g32 activations) tm rows of G fp16 scales.
-// Single-token routing scratch (RingPlan::route): se, swt, sj, sidx, sw [32] each, then
-// flag words.
-constexpr int kRouteBytes = 5 * 32 * 4 + 16;
+// Single-token routing scratch (RingPlan::route): se, swt, sj, sidx, sw, own [32] each,
+// then two flag words and the y-zero barrier target (8 bytes).
+constexpr int kRouteBytes = 6 * 32 * 4 + 16;
 
 struct RingPlan {
   int ring, sring, bars, abuf, abytes, ascale, xsum, sxf, idot, ubuf, hq, info, route, total;
@@ -196,6 +196,7 @@ struct RingArgs {
   int tm, kmax;
   int mma_min;             // experts with this many slots are left to the tensor-core path
   RouteArgs r;             // MODE 3 (one token): the routing done inside the kernel
+  int cluster;             // MODE 3: logits shared per cluster of this many CTAs (0: grid barrier)
 };
 
 // int4 weights: each 8-byte word of the activation rows de-interleaved into its even, then
@@ -243,7 +244,9 @@ struct RouteSmem {
   int* sj;        // [k] their positions in the token's top-k list (pair index)
   int* sidx;      // [k] the top-k list in selection order
   float* sw;      // [k] its weights
+  float* own;     // [32] logits of this CTA's experts (cluster exchange)
   volatile int* flag;
+  volatile unsigned long long* ytarget;   // y-zero barrier target (cluster exchange)
 };
 
 // Bound of the grid-barrier wait: 2^22 polls (each an L2 round trip: seconds in all).
@@ -259,9 +262,14 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
 // has arrived. The counter is a multiple of 1024 when a call starts (grids are <= 1024
 // CTAs); this call's arrivals take base .. base + grid - 1 and the last one moves the
 // counter on to base + 1024 for the next call. False if the wait gave up.
+__device__ __forceinline__ unsigned long long atom_add_release(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.release.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
+  return old;
+}
+
 __device__ __forceinline__ bool grid_barrier(unsigned long long* ctr) {
-  __threadfence();
-  const unsigned long long old = atomicAdd(ctr, 1ull);
+  const unsigned long long old = atom_add_release(ctr, 1ull);   // the CTA's writes before it
   const unsigned long long target = (old & ~1023ull) + gridDim.x;
   if (old + 1 == target) atomicAdd(ctr, 1024ull - gridDim.x);
   for (uint32_t i = 0; i < kGridWaitTries; ++i)
@@ -269,36 +277,64 @@ __device__ __forceinline__ bool grid_barrier(unsigned long long* ctr) {
   return false;
 }
 
-// Scratch use of the (still idle) ring during the routing: the router rows of the CTA's
-// experts at 0 (when they fit kRowBytes; copied before the wait for the preceding kernel),
-// logit chunk partials at kRowBytes.
-constexpr int kRowBytes = 96 * 1024;
-constexpr int kPartFloats = (kNS * kSP * kPiece - kRowBytes) / 4;
+// Scratch use of the (still idle) ring during the routing. The logit of a 32-element chunk
+// is one thread's fma chain, so threads read chunks 128 bytes apart; stored with a 144-byte
+// chunk pitch instead, the eight lanes of a quarter warp hit eight different bank groups.
+// [0, kRowBytes): the router rows of the CTA's experts, chunk pitch 144 (when they fit;
+// copied before the wait for the preceding kernel); [kRowBytes, + kXBytes): the token's x,
+// same pitch (when it fits); then the chunk partials.
+constexpr int kChunkPitch = 144;
+constexpr int kRowBytes = 80 * 1024;
+constexpr int kXBytes = 28 * 1024;
+constexpr int kPartFloats = (kNS * kSP * kPiece - kRowBytes - kXBytes) / 4;
 
-__device__ __forceinline__ int route_experts_of_cta(int E) {
-  return (int)blockIdx.x < E ? (E - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+// Who computes which logits. Grid exchange: CTA b owns experts b, b + grid, ...; cluster
+// exchange: cluster rank c owns experts c, c + cluster size, ... (every cluster computes all
+// E logits and its CTAs share them through distributed shared memory).
+struct Owners {
+  int first, stride;
+};
+__device__ __forceinline__ Owners route_owners(bool cl) {
+  Owners o;
+  o.first = cl ? (int)cluster_rank() : (int)blockIdx.x;
+  o.stride = cl ? (int)cluster_size() : (int)gridDim.x;
+  return o;
+}
+__device__ __forceinline__ int owned_experts(int E, Owners o) {
+  return o.first < E ? (E - 1 - o.first) / o.stride + 1 : 0;
 }
 
-// Thread 0, before the wait for the preceding kernel: stage this CTA's router rows (model
-// parameters, not written by the preceding kernel) into the ring; completes on `bar`.
-// False if they do not fit (the logits then read them from global memory).
-__device__ __forceinline__ bool stage_router_rows(const RouteArgs& r, uint8_t* ring, uint64_t* bar) {
-  const int ne = route_experts_of_cta(r.E);
-  const uint32_t row = (uint32_t)r.H * 4;
-  if (ne == 0 || ne * row > (uint32_t)kRowBytes) return false;
-  mbar_arrive_expect_tx(bar, ne * row);
-  for (int j = 0; j < ne; ++j)
-    bulk_load(ring + j * row, r.wr + (int64_t)(blockIdx.x + j * gridDim.x) * r.H, row, bar);
-  return true;
+// Every thread, before the wait for the preceding kernel: stage this CTA's router rows
+// (model parameters, not written by the preceding kernel) into the ring, a 128-byte chunk
+// per copy at the 144-byte pitch, completing on `bar`. Returns (to every thread) whether
+// they fit; if not, the logits read them from global memory.
+__device__ __forceinline__ bool stage_router_rows(const RouteArgs& r, bool cl, uint8_t* ring, uint64_t* bar,
+                                                  volatile int* flag) {
+  const Owners o = route_owners(cl);
+  const int ne = owned_experts(r.E, o), C = r.H / 32;
+  const bool fit = ne > 0 && (int64_t)ne * C * kChunkPitch <= kRowBytes;
+  if (threadIdx.x == 0) {
+    if (fit) mbar_arrive_expect_tx(bar, (uint32_t)(ne * C * 128));
+    *flag = fit;
+  }
+  __syncthreads();                          // the expected bytes are set before any copy lands
+  if (fit)
+    for (int t = threadIdx.x; t < ne * C; t += kNT) {
+      const int j = t / C, c = t - j * C;
+      bulk_load(ring + (int64_t)t * kChunkPitch, r.wr + (int64_t)(o.first + j * o.stride) * r.H + 32 * c, 128, bar);
+    }
+  return fit;
 }
 
-// Every thread of the CTA. False when a wait gave up (status recorded). rows_bar: the
-// router rows were staged by stage_router_rows and complete on it.
+// Every thread of the CTA. False when a wait gave up (status recorded; with the cluster
+// exchange the CTA has still taken both cluster-barrier arrivals, and must wait on the
+// second before it exits). rows_bar: the router rows were staged and complete on it.
 __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Ring& R, const RouteSmem& S,
-                                uint64_t* rows_bar) {
+                                uint64_t* rows_bar, bool cl) {
   volatile int* flag = S.flag;
   const int tid = threadIdx.x, H = r.H, G = H / 32, C = H / 32, E = r.E, k = r.k;
   const bool cta0 = blockIdx.x == 0;
+  const Owners own = route_owners(cl);
   if (cta0 && tid == 0) {
     r.status[0] = 0;
     r.status[2] = 0;
@@ -308,6 +344,7 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
   //    multiple of 32, so a warp's lanes are all in range or all out)
   uint8_t* xs = R.abuf;
   __half* sxs = reinterpret_cast<__half*>(xs + P.ascale);
+  uint8_t* xpad = C * kChunkPitch <= kXBytes ? R.ring + kRowBytes : nullptr;
   for (int l = tid; l < 8 * G; l += kNT) {
     const int g = l >> 3;
     const float4 v = __ldg(reinterpret_cast<const float4*>(r.x) + l);
@@ -322,44 +359,51 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
                           (uint32_t)(uint8_t)(int8_t)quant_code(v.w, sc, 127.0f) << 24;
     reinterpret_cast<uint32_t*>(xs)[l] = word;
     if ((l & 7) == 0) sxs[g] = __float2half_rn(sc);
+    if (xpad) *reinterpret_cast<float4*>(xpad + (l >> 3) * kChunkPitch + (l & 7) * 16) = v;
     if (cta0) {
       reinterpret_cast<uint32_t*>(r.qx)[l] = word;
       if ((l & 7) == 0) reinterpret_cast<__half*>(r.sx)[g] = __float2half_rn(sc);
     }
   }
-  // 2. this CTA's share of y = 0 (ordered before every CTA's adds by the grid barrier)
+  // 2. this CTA's share of y = 0 (ordered before every CTA's adds by a grid barrier: the
+  //    routing's, or with the cluster exchange one whose wait comes before the first add)
   float4* y4 = reinterpret_cast<float4*>(r.y);
   for (int l = blockIdx.x * kNT + tid; l < H / 4; l += gridDim.x * kNT) y4[l] = make_float4(0.f, 0.f, 0.f, 0.f);
   // 3. logits of this CTA's experts, as many at a time as their chunk partials fit the ring
-  //    (idle until the barrier): partials first, then each expert's added in chunk order
-  float* part = reinterpret_cast<float*>(R.ring + kRowBytes);
-  const int ne = route_experts_of_cta(E);
+  //    (idle until the selection): partials first, then each expert's added in chunk order
+  float* part = reinterpret_cast<float*>(R.ring + kRowBytes + kXBytes);
+  const int ne = owned_experts(E, own);
   const int nb = kPartFloats / C;
+  bool good = true;
   if (rows_bar) {
     // the router rows (copied while the preceding kernel finished)
     const bool ok = mbar_wait(rows_bar, 0);
     if (tid == 0) *flag = ok;
-    __syncthreads();
-    if (!*flag) {
-      if (tid == 0) wait_failed(r.status, 1, 7, 0);
-      return false;
-    }
   }
-  for (int j0 = 0; j0 < ne; j0 += nb) {
+  __syncthreads();                          // x at the chunk pitch, the rows' wait result
+  if (rows_bar) {
+    good = *flag != 0;
+    if (!good && tid == 0) wait_failed(r.status, 1, 7, 0);
+  }
+  for (int j0 = 0; good && j0 < ne; j0 += nb) {
     const int nj = min(nb, ne - j0);
     for (int l = tid; l < nj * C; l += kNT) {
       const int j = l / C, c = l - j * C;
-      const int e = blockIdx.x + (j0 + j) * gridDim.x;
-      const float4* w4 = rows_bar ? reinterpret_cast<const float4*>(R.ring + (int64_t)(j0 + j) * H * 4) + 8 * c
+      const int e = own.first + (j0 + j) * own.stride;
+      const float4* w4 = rows_bar ? reinterpret_cast<const float4*>(R.ring + (int64_t)((j0 + j) * C + c) * kChunkPitch)
                                   : reinterpret_cast<const float4*>(r.wr + (int64_t)e * H + 32 * c);
-      const float4* x4 = reinterpret_cast<const float4*>(r.x + 32 * c);
-      float4 wv[8];
+      const float4* x4 = xpad ? reinterpret_cast<const float4*>(xpad + c * kChunkPitch)
+                              : reinterpret_cast<const float4*>(r.x + 32 * c);
+      float4 wv[8], xv4[8];
 #pragma unroll
-      for (int v = 0; v < 8; ++v) wv[v] = rows_bar ? w4[v] : __ldg(w4 + v);
+      for (int v = 0; v < 8; ++v) {
+        wv[v] = rows_bar ? w4[v] : __ldg(w4 + v);
+        xv4[v] = xpad ? x4[v] : __ldg(x4 + v);
+      }
       float acc = 0.0f;
 #pragma unroll
       for (int v = 0; v < 8; ++v) {
-        const float4 xv = __ldg(x4 + v);
+        const float4 xv = xv4[v];
         acc = __fmaf_rn(xv.x, wv[v].x, acc);
         acc = __fmaf_rn(xv.y, wv[v].y, acc);
         acc = __fmaf_rn(xv.z, wv[v].z, acc);
@@ -380,26 +424,50 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
         for (int q = 0; q < 8; ++q) total = __fadd_rn(total, v[q]);
       }
       for (; c < C; ++c) total = __fadd_rn(total, pj[c]);
-      r.logits[blockIdx.x + (j0 + j) * gridDim.x] = total;
+      const int e = own.first + (j0 + j) * own.stride;
+      if (!cl || (int)blockIdx.x < own.stride) r.logits[e] = total;   // the fp32 logit view
+      if (cl) S.own[j0 + j] = total;
     }
     __syncthreads();
   }
   __syncthreads();
-  if (tid == 0) *flag = grid_barrier(r.gbar) ? 1 : 0;
-  __syncthreads();
-  if (!*flag) {
-    if (tid == 0) wait_failed(r.status, 1, 6, 0);
-    return false;
-  }
-  // 5. top-k (every CTA, same result): every key ranks itself against all E keys in
-  //    parallel (rank = keys larger, or equal with a lower expert index: descending, ties
-  //    to the lower expert); then warp 0 forms the routing weights of the k selected
+  // 4. every logit into this CTA's shared memory
   float* slog = reinterpret_cast<float*>(R.ring);           // scratch again: [E] logits
   float* skey = slog + 512;                                  //                [E] selection keys
+  if (!cl) {
+    if (tid == 0) *flag = grid_barrier(r.gbar) ? 1 : 0;
+    __syncthreads();
+    if (!*flag) {
+      if (tid == 0) wait_failed(r.status, 1, 6, 0);
+      return false;
+    }
+    if (!good) return false;
+    for (int i = tid; i < E; i += kNT) slog[i] = __ldcg(r.logits + i);
+  } else {
+    if (tid == 0) {
+      // y-zero barrier, first half: this CTA's share of y is zero; the wait is taken before
+      // the CTA's first add into y
+      __threadfence();
+      const unsigned long long old = atomicAdd(r.gbar, 1ull);
+      const unsigned long long target = (old & ~1023ull) + gridDim.x;
+      if (old + 1 == target) atomicAdd(r.gbar, 1024ull - gridDim.x);
+      *S.ytarget = target;
+    }
+    cluster_arrive();
+    cluster_wait();
+    for (int i = tid; i < E; i += kNT) slog[i] = ld_dsmem_f32(S.own + i / own.stride, (uint32_t)(i % own.stride));
+    cluster_arrive();                                       // this CTA's remote reads are done
+    if (!good) return false;
+  }
   if (tid < 32) S.sidx[tid] = -1;
+  // 5. top-k (every CTA, same result): every key ranks itself against all E keys in
+  //    parallel (rank = keys larger, or equal with a lower expert index: descending, ties
+  //    to the lower expert). The logits also go to activation buffer 1 (idle in this mode):
+  //    the routing weights are formed there after the producer has started.
+  float* slogk = reinterpret_cast<float*>(R.abuf + P.abytes);
   for (int i = tid; i < E; i += kNT) {
-    const float L = __ldcg(r.logits + i);
-    slog[i] = L;
+    const float L = slog[i];
+    slogk[i] = L;
     skey[i] = r.score == 0 ? L : __fadd_rn(csigmoid(L), r.bias ? r.bias[i] : 0.0f);
   }
   __syncthreads();
@@ -420,43 +488,17 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
     for (; j < E; ++j) rank += (skey[j] > kv) | ((skey[j] == kv) & (j < i));
     if (rank < k) S.sidx[rank] = i;
   }
+  fence_async_smem();                       // this thread's ring accesses precede the bulk copies
   __syncthreads();
-  if (tid < 32) {
-    const int lane = tid;
-    const bool on = lane < k;
-    const int my_e = on ? S.sidx[lane] : 0;
-    const float myl = (my_e >= 0 && my_e < E) ? slog[my_e] : 0.0f;
-    float wv;
-    if (r.score == 0) {
-      const float lmax = __shfl_sync(0xffffffffu, myl, 0);
-      const float ex = on ? cexp(myl - lmax) : 0.0f;
-      float den;
-      if (r.renorm) {
-        den = warp_sum(ex);
-      } else {
-        float sacc = 0.0f;
-        for (int x = lane; x < E; x += 32) sacc += cexp(slog[x] - lmax);
-        den = warp_sum(sacc);
-      }
-      wv = ex / den * r.rsf;
-    } else {
-      const float sg = on ? csigmoid(myl) : 0.0f;
-      const float den = r.renorm ? warp_sum(sg) : 1.0f;
-      wv = sg / den * r.rsf;
-    }
-    if (on) S.sw[lane] = wv;
-  }
-  __syncthreads();
+  // 6. the selection in ascending expert order (all the producer needs)
   if (tid < k) {
     const int ee = S.sidx[tid];
     int pos = 0;
     for (int j = 0; j < k; ++j) pos += S.sidx[j] < ee;
     S.se[pos] = ee;
     S.sj[pos] = tid;
-    S.swt[pos] = S.sw[tid];
     if (cta0) {
       r.idx[tid] = ee;
-      r.w[tid] = S.sw[tid];
       r.g.act_expert[pos] = ee;
       r.g.act_begin[pos] = pos;
       r.g.perm[pos] = tid;
@@ -477,6 +519,45 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
   }
   __syncthreads();
   return true;
+}
+
+// Warp 0 of the consumers, after route_one_token: routing weights of the k selected experts
+// from the logits kept in activation buffer 1 -- softmax over the selected (renormalized) or
+// over all E, or sigmoid scores (normalized over the selected), times the routed scaling
+// factor (as in topk.cuh) -- into S.sw (selection order) and S.swt (ascending order).
+__device__ __forceinline__ void route_weights(const RouteArgs& r, const RingPlan& P, const Ring& R,
+                                              const RouteSmem& S) {
+  const float* slogk = reinterpret_cast<const float*>(R.abuf + P.abytes);
+  const int lane = threadIdx.x & 31, E = r.E, k = r.k;
+  const bool on = lane < k;
+  const int my_e = on ? S.sidx[lane] : 0;
+  const float myl = (my_e >= 0 && my_e < E) ? slogk[my_e] : 0.0f;
+  float wv;
+  if (r.score == 0) {
+    const float lmax = __shfl_sync(0xffffffffu, myl, 0);
+    const float ex = on ? cexp(myl - lmax) : 0.0f;
+    float den;
+    if (r.renorm) {
+      den = warp_sum(ex);
+    } else {
+      float sacc = 0.0f;
+      for (int x = lane; x < E; x += 32) sacc += cexp(slogk[x] - lmax);
+      den = warp_sum(sacc);
+    }
+    wv = ex / den * r.rsf;
+  } else {
+    const float sg = on ? csigmoid(myl) : 0.0f;
+    const float den = r.renorm ? warp_sum(sg) : 1.0f;
+    wv = sg / den * r.rsf;
+  }
+  if (on) {
+    int pos = 0;
+    for (int j = 0; j < k; ++j) pos += S.sidx[j] < my_e;
+    S.sw[lane] = wv;
+    S.swt[pos] = wv;
+    if (blockIdx.x == 0) r.w[lane] = wv;
+  }
+  __syncwarp();
 }
 
 // Work unit u of a MODE 3 grid: routed units (the token's k experts, ascending) first, then
@@ -918,34 +999,34 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   S.sj = S.se + 64;
   S.sidx = S.se + 96;
   S.sw = S.swt + 96;
-  S.flag = reinterpret_cast<volatile int*>(S.se + 160);
-  volatile int* rows_flag = S.se + 161;
+  S.own = S.swt + 128;
+  S.flag = reinterpret_cast<volatile int*>(S.se + 192);
+  volatile int* rows_flag = S.se + 193;
+  S.ytarget = reinterpret_cast<volatile unsigned long long*>(S.se + 194);
   __syncthreads();
   bool rows = false;
   if (MODE == 3) {
-    if (threadIdx.x == 0) *rows_flag = stage_router_rows(A.r, R.ring, &R.afull[0]);
-    __syncthreads();
-    rows = *rows_flag != 0;
+    rows = stage_router_rows(A.r, A.cluster != 0, R.ring, &R.afull[0], rows_flag);
   }
   pdl_wait();
   if (MODE == 3) {
     // one token: routing first. Its grid barrier also means every CTA of this grid is
     // resident before any CTA lets the next kernel launch (and take SMs).
-    if (!route_one_token(A.r, P, R, S, rows ? &R.afull[0] : nullptr)) return;
-    if (WBITS == 4) {
-      act_deinterleave(R.abuf, A.kmax / 8, threadIdx.x, kNT);
-      __syncthreads();
-      act_group_sums(R.abuf, R.xsum, 1, A.kmax, threadIdx.x, kNT);
-      __syncthreads();
+    if (!route_one_token(A.r, P, R, S, rows ? &R.afull[0] : nullptr, A.cluster != 0)) {
+      if (A.cluster) cluster_wait();
+      return;
     }
-    // the ring held the logit partials (generic stores); the bulk copies refill it
-    fence_async_smem();
-    __syncthreads();
   }
-  pdl_trigger();
+  // the next kernel may launch once every CTA of this grid is resident: after the routing's
+  // grid barrier, or with the cluster exchange after the y-zero barrier (consumers, below)
+  if (!(MODE == 3 && A.cluster)) pdl_trigger();
 
   if (warp == kCW) {
     if (lane == 0) ring_producer<WBITS, WG32, AG32, MODE>(A, P, R, S);
+    if (MODE == 3 && A.cluster) {
+      __syncwarp();
+      cluster_wait();                      // peers are done reading this CTA's logits
+    }
     return;
   }
 
@@ -953,6 +1034,17 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   const int row = ctid & 127, ts = ctid >> 7;  // chain row, first token (tokens ts + 2 qq)
   const int tm = A.tm;
   uint32_t c = 0, pidx = 0, nblk = 0;       // chunks, gate/up passes, 8-group blocks consumed
+  bool ywait = !(MODE == 3 && A.cluster);   // cluster exchange: y-zero barrier still to wait on
+  if (MODE == 3) {
+    // off the path to the first weight copy: the routing weights (read only by this warp's
+    // ctid 0) and, int4 weights, the token's de-interleaved codes and group sums
+    if (warp == 0) route_weights(A.r, P, R, S);
+    if (WBITS == 4) {
+      act_deinterleave(R.abuf, A.kmax / 8, ctid, 32 * kCW);
+      named_bar(1, 32 * kCW);
+      act_group_sums(R.abuf, R.xsum, 1, A.kmax, ctid, 32 * kCW);
+    }
+  }
   for (int u = blockIdx.x; u < A.units; u += gridDim.x) {
     Unit U;
     if (MODE == 3 ? !unit_of_token(A, S, u, U, ctid == 0)
@@ -1062,6 +1154,21 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
         }
       }
       if (MODE != 0) {
+        if (!ywait) {
+          // y-zero barrier, second half, before this CTA's first add into y (long done by now:
+          // every CTA arrived right after zeroing its share, before its first gate/up pass)
+          if (ctid == 0) {
+            bool ok = false;
+            for (uint32_t i = 0; i < kGridWaitTries && !ok; ++i) ok = ld_acquire_u64(A.r.gbar) >= *S.ytarget;
+            if (!ok) {
+              *abort = 1;
+              wait_failed(status, 1, 8, 0);
+            }
+          }
+          ywait = true;
+          named_bar(1, 32 * kCW);
+          pdl_trigger();
+        }
         named_bar(1, 32 * kCW);            // h codes / scales of the pass in shared memory
         const uint8_t* hx = hq;
         if (WBITS == 4) {
@@ -1093,6 +1200,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
       }
     }
   }
+  if (MODE == 3 && A.cluster) cluster_wait();   // peers are done reading this CTA's logits
 }
 
 // ------------------------------------------------------------------ host side
@@ -1125,9 +1233,71 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     attr_bytes = P.total;
   }
-  const int grid = MODE == 3 ? decode_grid(A.units, A.r.E) : std::min(A.units, sm_count());
-  if (grid <= 0) return cudaSuccess;
-  return launch_pdl(k_expert_ring<WBITS, WG32, AG32, MODE, TM>, dim3(grid), dim3(kNT), (size_t)P.total, st, A);
+  if constexpr (MODE == 3) {
+    // one token: the logits shared per cluster (16 CTAs, else 8) when a CTA's share of the
+    // router rows fits its staging area and every cluster of the grid can be resident at
+    // once (the y-zero barrier waits on all CTAs) with no fewer CTAs than the grid exchange
+    // would use; else every CTA computes some logits and a grid barrier follows
+    auto kern = k_expert_ring<WBITS, WG32, AG32, MODE, TM>;
+    static int max_clusters[2] = {-1, -1}, max_clusters_smem = -1;
+    if (max_clusters_smem != P.total) {
+      (void)cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      for (int i = 0; i < 2; ++i) {
+        const int cs = i == 0 ? 16 : 8;
+        cudaLaunchConfig_t q = {};
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = cs;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        q.gridDim = dim3(cs * 8);
+        q.blockDim = dim3(kNT);
+        q.dynamicSmemBytes = (size_t)P.total;
+        q.attrs = qa;
+        q.numAttrs = 1;
+        int n = 0;
+        max_clusters[i] = cudaOccupancyMaxActiveClusters(&n, kern, &q) == cudaSuccess ? n : 0;
+      }
+      max_clusters_smem = P.total;
+      (void)cudaGetLastError();
+    }
+    const int grid_x = decode_grid(A.units, A.r.E);          // grid exchange
+    const int need = std::min(std::max(A.units, 1), sm_count());
+    int cs_best = 0, cgrid = 0;
+    for (int i = 0; i < 2; ++i) {
+      const int cs = i == 0 ? 16 : 8;
+      const int per = (A.r.E + cs - 1) / cs;
+      if ((int64_t)per * (A.r.H / 32) * kChunkPitch > kRowBytes || per > 32) continue;
+      const int want = (std::max(A.units, 1) + cs - 1) / cs;
+      const int g = cs * std::min({want, max_clusters[i], sm_count() / cs});
+      if (g >= need && (cs_best == 0 || g < cgrid)) {
+        cs_best = cs;
+        cgrid = g;
+      }
+    }
+    RingArgs B = A;
+    B.cluster = cs_best;
+    if (!B.cluster) return launch_pdl(kern, dim3(grid_x), dim3(kNT), (size_t)P.total, st, B);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = cs_best;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(cgrid);
+    cfg.blockDim = dim3(kNT);
+    cfg.dynamicSmemBytes = (size_t)P.total;
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = kUsePdl ? 2 : 1;
+    return cudaLaunchKernelEx(&cfg, kern, B);
+  } else {
+    const int grid = std::min(A.units, sm_count());
+    if (grid <= 0) return cudaSuccess;
+    return launch_pdl(k_expert_ring<WBITS, WG32, AG32, MODE, TM>, dim3(grid), dim3(kNT), (size_t)P.total, st, A);
+  }
 }
 
 template <int WBITS, bool WG32, bool AG32, int TM>
@@ -1187,7 +1357,7 @@ cudaError_t launch_experts(int mode, const ExpertArgs& gr, const ExpertArgs* gs,
 
 bool decode_fusable(const RouteArgs& r, const ExpertArgs& gr, const ExpertArgs* gs) {
   if (r.T != 1 || !experts_fusable(gr, gs) || !r.ag32 || r.E > 512 || r.k > 32 || r.H != gr.b.H ||
-      r.H % 128 != 0 || !r.gbar)
+      r.H % 128 != 0 || 4 * r.E > r.H || !r.gbar)   // the logits also fit activation buffer 1
     return false;
   return r.H / 32 <= kPartFloats;   // one expert's chunk partials fit the ring scratch
 }
