@@ -470,15 +470,17 @@ def gpu_arm(args, cfg, T):
             layers[s % R](xs[s % G], y, stream)
     stream.synchronize()
 
-    # Graphs: `graph_ev` = one period of G steps with every stage bracketed by CUDA events
-    # (external event nodes; they cut the programmatic edges around them, so this period
-    # runs slower), `graph` = G steps without events, `graph_rem` = the remainder. The timed
-    # region replays `graph` for the first K - G steps and `graph_ev` for the last G, so the
-    # per-launch stage durations are read live from inside the timed region.
+    # Graphs: `graph_ev` = the last Ge steps with every stage bracketed by CUDA events
+    # (external event nodes; they cut the programmatic edges around them, so these steps run
+    # slower), `graph` = G steps without events, `graph_rem` = the remainder. The timed region
+    # replays `graph` for the first K - Ge steps (an event between the two parts times them)
+    # and `graph_ev` for the last Ge, so the per-launch stage durations are read live from
+    # inside the timed region.
+    Ge = max(1, min(G, args.event_steps))
     nst = len(M.MOE_STAGES)
     evs = []
     with torch.cuda.stream(stream):
-        for s in range(G):
+        for s in range(Ge):
             e = M.moe_stage_events()
             pair = []
             for i in range(nst):
@@ -493,13 +495,13 @@ def gpu_arm(args, cfg, T):
     stream.synchronize()
     graph_ev = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph_ev, stream=stream):
-        for s in range(G):
+        for s in range(Ge):
             layers[s % R](xs[s], y, stream, events=evs[s][0])
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for s in range(G):
             layers[s % R](xs[s], y, stream)
-    n_main, rem = divmod(args.steps - G, G)
+    n_main, rem = divmod(args.steps - Ge, G)
     graph_rem = None
     if rem:
         graph_rem = torch.cuda.CUDAGraph()
@@ -523,6 +525,7 @@ def gpu_arm(args, cfg, T):
     clocks = ClockSampler(gpu_id)
     time.sleep(0.1)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    mid = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_push("timed")
@@ -533,6 +536,7 @@ def gpu_arm(args, cfg, T):
             graph.replay()
         if graph_rem is not None:
             graph_rem.replay()
+        mid.record(stream)
         graph_ev.replay()
         end.record(stream)
     stream.synchronize()
@@ -542,11 +546,13 @@ def gpu_arm(args, cfg, T):
     clocks.mark(w0, w1)
     clk = clocks.stop()
     ms_max = max_over_ranks(start.elapsed_time(end), world, dev)
+    main_steps = args.steps - Ge
+    ms_main = max_over_ranks(start.elapsed_time(mid), world, dev) if main_steps > 0 else None
 
     # per-stage device times of the last graph period (inside the timed region)
     stage_ms = {n: [] for n in M.MOE_STAGES}
     if True:
-        for s in range(G):
+        for s in range(Ge):
             for i, n in enumerate(M.MOE_STAGES):
                 b_ev, e_ev = evs[s][1][i]
                 stage_ms[n].append(b_ev.elapsed_time(e_ev))
@@ -561,14 +567,26 @@ def gpu_arm(args, cfg, T):
     fused = cfg.act == "g32_f16"
     gu_us = stage_us["gate_up"]
     gu_bytes = float(np.mean([(expert_bytes if fused else gateup_bytes)(cfg, T, a) for a in n_active_of]))
+    one_launch = layers[0].kernels == 1
+    how = "gate/up stage events (the last Ge steps)"
+    if one_launch:
+        # the kernel also reads the router weight and x and writes y
+        gu_bytes = float(np.mean([layer_bytes(cfg, T, a) for a in n_active_of]))
+    if one_launch and ms_main:
+        # one kernel per step (single-token routing inside it): its average launch duration
+        # is the event-timed region without stage events over its launches
+        gu_us = ms_main * 1e3 / main_steps
+        how = f"one launch per step: events around the first {main_steps} timed steps / launches"
     roof = None
     if gu_us:
         ach = gu_bytes / (gu_us * 1e-6) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic_from_profiles(cfg, T),
-                "kernel": ("k_expert_ring (gate/up, SwiGLU, h quantization, down, weighted combine)"
+                "kernel": (("k_expert_ring (single token: routing, gate/up, SwiGLU, h quantization, down, "
+                            "weighted combine)" if one_launch else
+                            "k_expert_ring (gate/up, SwiGLU, h quantization, down, weighted combine)")
                            if fused else "k_expert_ring (gate/up pass)"),
-                "bytes_per_launch": int(gu_bytes), "us_per_launch": round(gu_us, 3),
+                "bytes_per_launch": int(gu_bytes), "us_per_launch": round(gu_us, 3), "timing": how,
                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else "fallback 6.65 TB/s"}
     lb = float(np.mean([layer_bytes(cfg, T, a) for a in n_active_of]))
     step_s = ms_max / 1e3 / args.steps
@@ -584,12 +602,9 @@ def gpu_arm(args, cfg, T):
         ne = min(args.steps, args.e2e_steps)
         xh = [torch.from_numpy(S.Case.make(cfg, T, seed=95_000_000 + s).x()).pin_memory() for s in range(min(ne, 64))]
         yh = torch.empty((T, cfg.H), dtype=torch.float32).pin_memory()
-        xd = torch.empty((T, cfg.H), dtype=torch.float32, device=dev)
         with torch.cuda.stream(stream):
             for s in range(3):
-                xd.copy_(xh[s % len(xh)], non_blocking=True)
-                layers[s % R](xd, y, stream)
-                yh.copy_(y, non_blocking=True)
+                layers[s % R].forward_host(xh[s % len(xh)], yh, stream)
         stream.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier()
@@ -597,9 +612,7 @@ def gpu_arm(args, cfg, T):
         with torch.cuda.stream(stream):
             e0.record(stream)
             for s in range(ne):
-                xd.copy_(xh[s % len(xh)], non_blocking=True)
-                layers[s % R](xd, y, stream)
-                yh.copy_(y, non_blocking=True)
+                layers[s % R].forward_host(xh[s % len(xh)], yh, stream)
             e1.record(stream)
         stream.synchronize()
         barrier()
@@ -608,7 +621,8 @@ def gpu_arm(args, cfg, T):
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
         e2e = {"value": world * T * ne / (float(te.item()) / 1e3), "unit": "tok/s",
                "h2d_bytes_per_step": T * cfg.H * 4, "d2h_bytes_per_step": T * cfg.H * 4,
-               "steps": ne, "path": "Layer.__call__ (moe_layer_forward) eager, pinned host x in / y out"}
+               "steps": ne, "path": "Layer.forward_host -> moe_layer_forward_host (C ABI, one call per step: "
+                       "pinned host x copied in, the layer, y copied out), eager"}
 
     prefill = None
     if not args.no_prefill:
@@ -627,7 +641,7 @@ def gpu_arm(args, cfg, T):
         "config": {"workload": workload_desc(cfg, T), "T": T, "replicas": R,
                    "l2": f"inputs larger than L2: {R} layer replicas rotate "
                          f"({R * layers[0].experts.nbytes / 1e9:.2f} GB of expert blobs)",
-                   "graph": f"CUDA graphs of {G} steps; the last {G} timed steps carry per-stage event nodes", "accumulate": "int32 dots, fp32 scales",
+                   "graph": f"CUDA graphs of {G} steps; the last {Ge} timed steps carry per-stage event nodes", "accumulate": "int32 dots, fp32 scales",
                    "parallelism": f"dp{world} (weak: independent tokens per GPU)"},
         "roofline": roof,
         "layer": layer,
@@ -672,6 +686,8 @@ def main(argv=None):
                     help="config[:T], config one of " + ", ".join(S.CONFIG_ORDER))
     ap.add_argument("--replicas", type=int, default=8, help="layer replicas rotated per step")
     ap.add_argument("--period", type=int, default=256, help="steps per captured graph")
+    ap.add_argument("--event-steps", type=int, default=32,
+                    help="timed steps (the last ones) with per-stage event records")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

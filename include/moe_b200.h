@@ -272,6 +272,18 @@ MOE_API moe_status moe_layer_forward_timed(const float* x, int32_t T, const floa
                                            size_t ws_bytes, void* stream,
                                            const moe_stage_events* events);
 
+/* moe_layer_forward with x and y in host memory: enqueues on `stream` the copy of x_host
+ * [T][H] into x_dev, the layer (y_dev [T][H]) and the copy of y_dev into y_host, and returns
+ * (synchronize `stream` before reading y_host). x_host / y_host should be page-locked
+ * (cudaHostAlloc) for the copies to be asynchronous; x_dev / y_dev are device buffers of
+ * T * H floats, 16-byte aligned, owned by the caller. Errors as moe_layer_forward, plus
+ * INVALID_ARG for a null buffer and CUDA for a failed copy. */
+MOE_API moe_status moe_layer_forward_host(const float* x_host, int32_t T, const float* router_w,
+                                          const float* router_bias, const moe_expert_blob* experts,
+                                          const moe_expert_blob* shared, const moe_route_cfg* cfg,
+                                          float* x_dev, float* y_dev, float* y_host, void* workspace,
+                                          size_t ws_bytes, void* stream);
+
 /* Number of kernels one moe_layer_forward call with these arguments launches. */
 MOE_API int32_t moe_layer_kernel_count(int32_t T, const moe_expert_blob* experts,
                                        const moe_expert_blob* shared, const moe_route_cfg* cfg);

@@ -74,6 +74,7 @@ _SIGS = {
     "moe_permute_no_alloc": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_layer_workspace_bytes": (_sz, [_i32, _PB, _PB, _PC]),
     "moe_layer_forward": (_i32, [_vp, _i32, _vp, _vp, _PB, _PB, _PC, _vp, _vp, _sz, _vp]),
+    "moe_layer_forward_host": (_i32, [_vp, _i32, _vp, _vp, _PB, _PB, _PC, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_layer_forward_timed": (_i32, [_vp, _i32, _vp, _vp, _PB, _PB, _PC, _vp, _vp, _sz, _vp,
                                        C.POINTER(moe_stage_events)]),
     "moe_layer_kernel_count": (_i32, [_i32, _PB, _PB, _PC]),
@@ -331,6 +332,23 @@ class Layer:
                                               C.byref(events))
         _check(rc, "moe_layer_forward")
         return y
+
+    def forward_host(self, x_host, y_host, stream=None):
+        """The layer on host buffers (page-locked CPU tensors [T][H] fp32): one call into
+        moe_layer_forward_host, which enqueues the copy in, the layer and the copy out on
+        `stream` (synchronize it before reading y_host). Device staging buffers are the
+        layer's own."""
+        import torch
+        if getattr(self, "_xd", None) is None:
+            H = self.experts.hidden
+            self._xd = torch.empty((self.T, H), dtype=torch.float32, device=self.router_w.device)
+            self._yd = torch.empty((self.T, H), dtype=torch.float32, device=self.router_w.device)
+        rw, rb, e, s, c = self._args
+        rc = _lib.moe_layer_forward_host(x_host.data_ptr(), self.T, rw, rb, e, s, c, self._xd.data_ptr(),
+                                         self._yd.data_ptr(), y_host.data_ptr(), self.workspace.data_ptr(),
+                                         self.workspace.numel(), _stream(stream))
+        _check(rc, "moe_layer_forward_host")
+        return y_host
 
 
 def moe_layer_debug_views(T: int, experts: ExpertBlob, shared: ExpertBlob | None,

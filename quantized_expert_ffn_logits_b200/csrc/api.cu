@@ -663,6 +663,26 @@ moe_status moe_layer_forward(const float* x, int32_t T, const float* router_w,
                       stream, nullptr);
 }
 
+moe_status moe_layer_forward_host(const float* x_host, int32_t T, const float* router_w,
+                                  const float* router_bias, const moe_expert_blob* experts,
+                                  const moe_expert_blob* shared, const moe_route_cfg* cfg, float* x_dev,
+                                  float* y_dev, float* y_host, void* workspace, size_t ws_bytes, void* stream) {
+  if (T < 0 || !experts) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return forward_impl(x_dev, T, router_w, router_bias, experts, shared, cfg, y_dev, workspace,
+                                  ws_bytes, stream, nullptr);
+  if (!x_host || !y_host || !x_dev || !y_dev) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = (size_t)T * (size_t)experts->hidden * sizeof(float);
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail("x host-to-device copy", e);
+  const moe_status s = forward_impl(x_dev, T, router_w, router_bias, experts, shared, cfg, y_dev, workspace,
+                                    ws_bytes, stream, nullptr);
+  if (s != MOE_OK) return s;
+  e = cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return cuda_fail("y device-to-host copy", e);
+  return MOE_OK;
+}
+
 moe_status moe_layer_forward_timed(const float* x, int32_t T, const float* router_w,
                                    const float* router_bias, const moe_expert_blob* experts,
                                    const moe_expert_blob* shared, const moe_route_cfg* cfg,

@@ -345,24 +345,33 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
   uint8_t* xs = R.abuf;
   __half* sxs = reinterpret_cast<__half*>(xs + P.ascale);
   uint8_t* xpad = C * kChunkPitch <= kXBytes ? R.ring + kRowBytes : nullptr;
-  for (int l = tid; l < 8 * G; l += kNT) {
-    const int g = l >> 3;
-    const float4 v = __ldg(reinterpret_cast<const float4*>(r.x) + l);
-    float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-    const float sc = f16_round(__fdiv_rn(m, 127.0f));
-    const uint32_t word = (uint32_t)(uint8_t)(int8_t)quant_code(v.x, sc, 127.0f) |
-                          (uint32_t)(uint8_t)(int8_t)quant_code(v.y, sc, 127.0f) << 8 |
-                          (uint32_t)(uint8_t)(int8_t)quant_code(v.z, sc, 127.0f) << 16 |
-                          (uint32_t)(uint8_t)(int8_t)quant_code(v.w, sc, 127.0f) << 24;
-    reinterpret_cast<uint32_t*>(xs)[l] = word;
-    if ((l & 7) == 0) sxs[g] = __float2half_rn(sc);
-    if (xpad) *reinterpret_cast<float4*>(xpad + (l >> 3) * kChunkPitch + (l & 7) * 16) = v;
-    if (cta0) {
-      reinterpret_cast<uint32_t*>(r.qx)[l] = word;
-      if ((l & 7) == 0) reinterpret_cast<__half*>(r.sx)[g] = __float2half_rn(sc);
+  for (int l0 = tid; l0 < 8 * G; l0 += 4 * kNT) {
+    float4 xv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)                // every load of the round in flight at once
+      if (l0 + u * kNT < 8 * G) xv[u] = __ldg(reinterpret_cast<const float4*>(r.x) + l0 + u * kNT);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int l = l0 + u * kNT;
+      if (l >= 8 * G) break;                   // warp-uniform (8 G and kNT are multiples of 32)
+      const int g = l >> 3;
+      const float4 v = xv[u];
+      float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      const float sc = f16_round(__fdiv_rn(m, 127.0f));
+      const uint32_t word = (uint32_t)(uint8_t)(int8_t)quant_code(v.x, sc, 127.0f) |
+                            (uint32_t)(uint8_t)(int8_t)quant_code(v.y, sc, 127.0f) << 8 |
+                            (uint32_t)(uint8_t)(int8_t)quant_code(v.z, sc, 127.0f) << 16 |
+                            (uint32_t)(uint8_t)(int8_t)quant_code(v.w, sc, 127.0f) << 24;
+      reinterpret_cast<uint32_t*>(xs)[l] = word;
+      if ((l & 7) == 0) sxs[g] = __float2half_rn(sc);
+      if (xpad) *reinterpret_cast<float4*>(xpad + (l >> 3) * kChunkPitch + (l & 7) * 16) = v;
+      if (cta0) {
+        reinterpret_cast<uint32_t*>(r.qx)[l] = word;
+        if ((l & 7) == 0) reinterpret_cast<__half*>(r.sx)[g] = __float2half_rn(sc);
+      }
     }
   }
   // 2. this CTA's share of y = 0 (ordered before every CTA's adds by a grid barrier: the
@@ -376,8 +385,9 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
   const int nb = kPartFloats / C;
   bool good = true;
   if (rows_bar) {
-    // the router rows (copied while the preceding kernel finished)
-    const bool ok = mbar_wait(rows_bar, 0);
+    // the router rows (copied while the preceding kernel finished): polled, not suspended on
+    bool ok = false;
+    for (uint32_t i = 0; i < (1u << 24) && !ok; ++i) ok = mbar_try_wait(rows_bar, 0);
     if (tid == 0) *flag = ok;
   }
   __syncthreads();                          // x at the chunk pitch, the rows' wait result
@@ -390,15 +400,24 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
     for (int l = tid; l < nj * C; l += kNT) {
       const int j = l / C, c = l - j * C;
       const int e = own.first + (j0 + j) * own.stride;
-      const float4* w4 = rows_bar ? reinterpret_cast<const float4*>(R.ring + (int64_t)((j0 + j) * C + c) * kChunkPitch)
-                                  : reinterpret_cast<const float4*>(r.wr + (int64_t)e * H + 32 * c);
-      const float4* x4 = xpad ? reinterpret_cast<const float4*>(xpad + c * kChunkPitch)
-                              : reinterpret_cast<const float4*>(r.x + 32 * c);
       float4 wv[8], xv4[8];
+      if (rows_bar) {
+        const float4* w4 = reinterpret_cast<const float4*>(R.ring + ((j0 + j) * C + c) * kChunkPitch);
 #pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        wv[v] = rows_bar ? w4[v] : __ldg(w4 + v);
-        xv4[v] = xpad ? x4[v] : __ldg(x4 + v);
+        for (int v = 0; v < 8; ++v) wv[v] = w4[v];
+      } else {
+        const float4* w4 = reinterpret_cast<const float4*>(r.wr + (int64_t)e * H + 32 * c);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) wv[v] = __ldg(w4 + v);
+      }
+      if (xpad) {
+        const float4* x4 = reinterpret_cast<const float4*>(xpad + c * kChunkPitch);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) xv4[v] = x4[v];
+      } else {
+        const float4* x4 = reinterpret_cast<const float4*>(r.x + 32 * c);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) xv4[v] = __ldg(x4 + v);
       }
       float acc = 0.0f;
 #pragma unroll

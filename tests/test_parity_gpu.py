@@ -151,6 +151,29 @@ def test_forward_without_debug_equals_debug(name, T):
     assert_close_y(_np(y0), ref["y"])
 
 
+@pytest.mark.parametrize("name,T", [("olmoe_int8", 1), ("glm_int4", 3), ("olmoe_int4", 40)])
+def test_forward_host_buffers_equal_device_path(name, T):
+    """moe_layer_forward_host (pinned host x in, y out, one C call) gives the y of
+    moe_layer_forward on device buffers -- to the layer tolerance, the combine into y being
+    fp32 adds in arrival order -- repeated calls included (the single-token grid barrier
+    counter moves on between calls)."""
+    m = M()
+    case = S.Case.make(REDUCED[name], T)
+    g = gpu_layer(case)
+    c = case.cfg
+    lay = m.Layer(T, g["blob"], g["shared"], route_cfg(c), g["wr"], g["bias"])
+    yd = torch.empty((T, c.H), dtype=torch.float32, device="cuda")
+    lay(g["x"], yd)
+    xh = g["x"].cpu().pin_memory()
+    yh = torch.full((T, c.H), float("nan"), dtype=torch.float32).pin_memory()
+    for _ in range(3):
+        lay.forward_host(xh, yh)
+    torch.cuda.synchronize()
+    assert m.moe_read_device_status(lay.workspace) == m.MOE_OK
+    assert_close_y(yh.numpy(), _np(yd).astype(np.float64))
+    assert_close_y(yh.numpy(), oracle_layer(case)["y"])
+
+
 def test_synth_device_generator_matches_host():
     t = torch.empty(1_000_003, dtype=torch.float32, device="cuda")
     S.normal_gpu_(t, 12345, 777, 0.02)
