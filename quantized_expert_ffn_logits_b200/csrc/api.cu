@@ -672,13 +672,24 @@ moe_status moe_layer_forward_host(const float* x_host, int32_t T, const float* r
                                   ws_bytes, stream, nullptr);
   if (!x_host || !y_host || !x_dev || !y_dev) return MOE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t bytes = (size_t)T * (size_t)experts->hidden * sizeof(float);
-  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st);
+  const int64_t n = (int64_t)T * experts->hidden;
+  const size_t bytes = (size_t)n * sizeof(float);
+  // page-locked host buffers with device-mapped addresses: the SMs move x and y (kernels
+  // chained to the layer's); otherwise copy-engine copies
+  void* xm = nullptr;
+  void* ym = nullptr;
+  const bool mapped = aligned(x_host, 16) && aligned(y_host, 16) && aligned(x_dev, 16) && aligned(y_dev, 16) &&
+                      cudaHostGetDevicePointer(&xm, const_cast<float*>(x_host), 0) == cudaSuccess &&
+                      cudaHostGetDevicePointer(&ym, y_host, 0) == cudaSuccess;
+  if (!mapped) (void)cudaGetLastError();   // the lookup's error is not the call's
+  cudaError_t e = mapped ? moe::launch_copy_in(static_cast<const float*>(xm), x_dev, n, st)
+                         : cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return cuda_fail("x host-to-device copy", e);
   const moe_status s = forward_impl(x_dev, T, router_w, router_bias, experts, shared, cfg, y_dev, workspace,
                                     ws_bytes, stream, nullptr);
   if (s != MOE_OK) return s;
-  e = cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st);
+  e = mapped ? moe::launch_copy_out(y_dev, static_cast<float*>(ym), n, st)
+             : cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st);
   if (e != cudaSuccess) return cuda_fail("y device-to-host copy", e);
   return MOE_OK;
 }

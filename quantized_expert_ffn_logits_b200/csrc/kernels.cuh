@@ -169,6 +169,11 @@ inline cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cud
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// ---- host_io.cu: n floats between page-locked host memory (device-mapped address) and the
+// device, as programmatically chained kernels (n a multiple of 4, both addresses 16-aligned).
+cudaError_t launch_copy_in(const float* x_host_mapped, float* x_dev, int64_t n, cudaStream_t st);
+cudaError_t launch_copy_out(const float* y_dev, float* y_host_mapped, int64_t n, cudaStream_t st);
+
 // ---- expert_gemv.cu (debug entry point)
 void launch_group_dots(const BlobView& b, int which, int n, const int32_t* expert,
                        const int32_t* row, const int8_t* act, int32_t* dots, cudaStream_t st);
