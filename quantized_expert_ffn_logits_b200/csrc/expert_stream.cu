@@ -5,26 +5,26 @@
 // "Quantization kernels: ... dequant-on-use"; "Batch-union MoE": every selected expert's
 // weights are streamed once per call, whatever the number of tokens routed to it).
 //
-// Work unit = one selected expert x one 128-row block of the blob: gate/up blocks hold 64
-// gate rows and the 64 matching up rows, down blocks 128 output rows. A block's whole K
-// range is one contiguous run in the blob ([piece][128 rows][16 B], 2 KB per piece), so it
-// streams as a handful of large bulk copies. Grid = one persistent CTA per SM (at most
-// one per unit), units taken round-robin; a unit with more tokens than fit one pass is
-// streamed once per pass.
+// Work unit = one selected expert x 64 intermediate indices: its gate/up block (64 gate rows
+// and the 64 matching up rows, the whole K range contiguous in the blob as [piece][128
+// rows][16 B]) and its down slab (all H output rows x those 64 columns). Grid = one
+// persistent CTA per SM (at most one per unit), units round-robin; a unit with more tokens
+// than fit one pass is streamed once per pass.
 //
 // CTA = one producer warp + eight consumer warps. The producer's lane 0 walks the CTA's
-// passes and pushes 32 KB chunks (16 pieces) plus the matching group scales into a
-// four-stage shared-memory ring with cp.async.bulk ("full" mbarrier per stage, released
-// on an "empty" mbarrier), and the pass's activation rows into one of two activation
-// buffers right behind the pass's first chunk, so they arrive in stream order instead of
-// queueing behind the weights. A consumer thread owns one row of the block for a set of
-// tokens: per chunk it loads all 16 pieces of its row, forms every group's exact int32 dot
-// (independent dp4a chains) and then runs the ordered fp32 chain over the chunk's groups,
-// acc = fma((float)I_g, c_g, acc) -- groups arrive in ascending order, so nothing is
-// parked. Up to four chunks (128 KB) per SM are in flight. Every wait is bounded: a wait
-// that gives up sets the status word, the consumers skip the rest of their work but keep
-// releasing stages (all warps take the same barriers), and the producer drains its copies
-// before the CTA exits.
+// passes and pushes 32 KB chunks (16 pieces) plus the matching scales into a four-stage
+// shared-memory ring with cp.async.bulk ("full" mbarrier per stage, released on an "empty"
+// mbarrier), and the pass's activation rows into one of two activation buffers right behind
+// the pass's first chunk. Consumers, per block of 8 groups: warp w forms the exact int32 dots
+// of group w for all 128 rows, a consumer barrier, then one thread per (row, token) runs the
+// ordered fp32 chain acc = fma((float)I_g, c_g, acc). After the gate/up pass the gate and up
+// values meet in shared memory, two warps apply SwiGLU and quantize h per group of 32, and
+// the unit's down slab is consumed against those codes, each row's share added into y with
+// 16-byte reductions. With one token and group-32 activations (MODE 3) the kernel also does
+// the routing (route_one_token): the whole layer is one launch. Every wait is bounded: a
+// wait that gives up sets the status word, the consumers skip the rest of their work but
+// keep releasing stages (all warps take the same barriers), and the producer drains its
+// copies before the CTA exits.
 #include <algorithm>
 #include <cstring>
 
