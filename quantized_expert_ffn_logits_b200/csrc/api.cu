@@ -80,7 +80,7 @@ struct Layout {
   int64_t status, qx, sx, logits, idx, w, offsets, perm, n_active, act_expert, act_begin, act_rows;
   int64_t masks, base, qh, sh, hbuf, dbg_gate, dbg_up, dbg_y, total;
   // tensor-core path (T > 32, group-32 weights and activations)
-  int64_t mm_tiles, mm_ntiles, mm_xa, mm_xs, mm_xsum, mm_ha, mm_hs, mm_hsum;
+  int64_t mm_tiles, mm_ntiles, mm_xa, mm_xs, mm_ha, mm_hs;
   int32_t mm_max_tiles, mm_min_tokens, mm_hk;
   int64_t qh_sh, sh_sh, hbuf_sh, dbg_gate_sh, dbg_up_sh, dbg_y_sh;   // shared-expert rows
 };
@@ -140,7 +140,7 @@ Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k,
   L.mm_max_tiles = 0;
   L.mm_min_tokens = force_mma ? 1 : moe::kMmaMinTokens;
   L.mm_hk = std::max(I, Is);
-  L.mm_tiles = L.mm_ntiles = L.mm_xa = L.mm_xs = L.mm_xsum = L.mm_ha = L.mm_hs = L.mm_hsum = -1;
+  L.mm_tiles = L.mm_ntiles = L.mm_xa = L.mm_xs = L.mm_ha = L.mm_hs = -1;
   if (mma) {
     // tiles of 128 slots: every qualifying expert wastes at most one partial tile
     const int64_t n_exp = std::min<int64_t>(E, P / L.mm_min_tokens);
@@ -148,12 +148,10 @@ Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k,
     L.mm_max_tiles = (int32_t)mt;
     L.mm_tiles = take(mt * 16);
     L.mm_ntiles = take(4);
-    L.mm_xa = take(mt * 128 * H);
+    L.mm_xa = take(mt * 128 * H * 2);                     // fp16 operands
     L.mm_xs = take(mt * (H / 32) * 128 * 2);
-    L.mm_xsum = take(mt * (H / 32) * 128 * 4);
-    L.mm_ha = take(mt * 128 * L.mm_hk);
+    L.mm_ha = take(mt * 128 * L.mm_hk * 2);
     L.mm_hs = take(mt * (L.mm_hk / 32) * 128 * 2);
-    L.mm_hsum = take(mt * (L.mm_hk / 32) * 128 * 4);
   }
   L.total = o;
   return L;
@@ -569,8 +567,6 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     m.max_tiles = L.mm_max_tiles;
     m.a_ops = static_cast<const uint8_t*>(at(L.mm_xa));
     m.a_scales = static_cast<const __half*>(at(L.mm_xs));
-    m.a_xsum = static_cast<const int32_t*>(at(L.mm_xsum));
-    m.h_xsum = static_cast<int32_t*>(at(L.mm_hsum));
     m.h_ops = static_cast<uint8_t*>(at(L.mm_ha));
     m.h_scales = static_cast<__half*>(at(L.mm_hs));
     m.hk = L.mm_hk;
@@ -598,7 +594,7 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
       keep(moe::launch_mma_gather(static_cast<const int8_t*>(at(L.qx)), static_cast<const __half*>(at(L.sx)),
                                   m.tiles, m.n_tiles, g.perm, k, T, H, L.mm_max_tiles,
                                   static_cast<uint8_t*>(at(L.mm_xa)), static_cast<__half*>(at(L.mm_xs)),
-                                  static_cast<int32_t*>(at(L.mm_xsum)), status, st),
+                                  status, st),
            "tensor-core operand gather");
       keep(moe::launch_expert_mma(true, m, st), "tensor-core gate/up kernel");
     } else {

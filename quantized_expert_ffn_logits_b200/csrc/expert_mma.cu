@@ -2,21 +2,23 @@
 //
 // An expert that receives at least kMmaMinTokens (token, expert) pairs in a call is a dense
 // contraction: its pairs are cut into tiles of 128 slots and every (tile, 128-row weight
-// block) pair runs as an M = 128 (slots) x N = 128 (rows) integer GEMM on the sm_100a tensor
-// cores (tcgen05.mma kind::i8, int32 in tensor memory). One MMA with K = 32 is exactly one
-// quantization group, so its accumulator is the exact int32 dot I_g of every (slot, row) in
-// the tile; the epilogue then runs the ordered fp32 chain acc = fma((float)I_g, c_g, acc)
-// with c_g = s_w,g * s_x,g per element -- the same arithmetic as the weight-streaming path
-// and the oracle (GLM-5.2 colibri page, "Integer-dot kernels"; "Batch-union MoE": every
-// selected expert's weights are read once per tile of 128 of its tokens).
+// block) pair runs as an M = 128 (slots) x N = 128 (rows) GEMM on the sm_100a tensor cores.
+// The codes enter as fp16 (exact: they are integers of at most 8 bits) and two tcgen05.mma
+// kind::f16 with K = 16 and an fp32 accumulator cover one quantization group of 32: every
+// product is an integer below 2^14 and every partial sum below 2^19, so the accumulator holds
+// the exact group dot I_g as an fp32 value -- no integer-to-float step is left. The epilogue
+// runs the ordered fp32 chain acc = fma((float)I_g, c_g, acc) with c_g = s_w,g * s_x,g per
+// element, the same arithmetic as the weight-streaming path and the oracle (GLM-5.2 colibri
+// page, "Integer-dot kernels"; "Batch-union MoE": every selected expert's weights are read once
+// per tile of 128 of its tokens).
 //
 // Gate/up tiles (N = the 64 gate rows and 64 up rows of one block) end with SwiGLU and Q8_0
 // h quantization per group of 32 -- one thread holds a slot's 32 indices of a group -- and
-// write h in the operand layout the down GEMM reads; down tiles (N = 128 output rows) add
-// w * v into y with 16-byte reductions.
+// write h (as fp16 codes) in the operand layout the down GEMM reads; down tiles (N = 128
+// output rows) add w * v into y with 16-byte reductions.
 //
-// The per-group epilogue (three fp32 operations per element per group against one 32-wide
-// MMA step) bounds this path, not the tensor cores: see the measurement notes.
+// The per-group epilogue (two fp32 operations per element per group against one 32-wide
+// step of the tensor cores) bounds this path, not the tensor cores: see the measurement notes.
 #include <algorithm>
 #include <cstring>
 
@@ -99,18 +101,35 @@ __global__ void __launch_bounds__(1024) k_mma_plan(const int32_t* __restrict__ n
   }
 }
 
+// Four signed int8 codes -> four exact fp16 values (two words): the bytes x ^ 0x80 = x + 128
+// become the low mantissa bytes of fp16 1024 + (x + 128), then 1152 is subtracted (exact).
+__device__ __forceinline__ void cvt_i8x4_f16(uint32_t w, uint32_t& o0, uint32_t& o1) {
+  const uint32_t x = w ^ 0x80808080u;
+  uint32_t h0 = __byte_perm(x, 0x64646464u, 0x5140), h1 = __byte_perm(x, 0x64646464u, 0x7362);
+  const __half2 k = __halves2half2(__float2half_rn(1152.0f), __float2half_rn(1152.0f));
+  __half2 r0 = __hsub2(*reinterpret_cast<__half2*>(&h0), k), r1 = __hsub2(*reinterpret_cast<__half2*>(&h1), k);
+  o0 = *reinterpret_cast<uint32_t*>(&r0);
+  o1 = *reinterpret_cast<uint32_t*>(&r1);
+}
+// Four bytes holding v = n + 8 (n a signed 4-bit code) -> the four fp16 values n.
+__device__ __forceinline__ void cvt_u4x4_f16(uint32_t v, uint32_t& o0, uint32_t& o1) {
+  uint32_t h0 = __byte_perm(v, 0x64646464u, 0x5140), h1 = __byte_perm(v, 0x64646464u, 0x7362);
+  const __half2 k = __halves2half2(__float2half_rn(1032.0f), __float2half_rn(1032.0f));
+  __half2 r0 = __hsub2(*reinterpret_cast<__half2*>(&h0), k), r1 = __hsub2(*reinterpret_cast<__half2*>(&h1), k);
+  o0 = *reinterpret_cast<uint32_t*>(&r0);
+  o1 = *reinterpret_cast<uint32_t*>(&r1);
+}
+
 // -------------------------------------------------------------------- gather
-// Operand A of the gate/up GEMM: for tile i, the q_x rows of its slots' tokens in the
-// tensor-core operand layout [tile][K/16 pieces][128 slots][16 B], their fp16 group scales
-// [tile][K/32][128] and the sum of each group's codes [tile][K/32][128] (the correction
-// for unsigned int4 weight bytes); slots past the tile's valid count are zero. One thread
-// per (tile, slot, group).
+// Operand A of the gate/up GEMM: for tile i, the q_x rows of its slots' tokens as fp16 (exact:
+// the codes are integers) in the tensor-core operand layout [tile][K/8 pieces][128 slots][16 B],
+// and their fp16 group scales [tile][K/32][128]; slots past the tile's valid count are zero.
+// One thread per (tile, slot, group).
 __global__ void __launch_bounds__(256) k_mma_gather(const int8_t* __restrict__ qx, const __half* __restrict__ sx,
                                                     const int4* __restrict__ tiles,
                                                     const int32_t* __restrict__ n_tiles,
                                                     const int32_t* __restrict__ perm, int k, int T, int K,
-                                                    uint8_t* __restrict__ xa, __half* __restrict__ xs,
-                                                    int32_t* __restrict__ xsum, int* status) {
+                                                    uint8_t* __restrict__ xa, __half* __restrict__ xs, int* status) {
   pdl_wait();
   pdl_trigger();
   const int G = K / 32;
@@ -122,7 +141,9 @@ __global__ void __launch_bounds__(256) k_mma_gather(const int8_t* __restrict__ q
     const int rem = (int)(id - (int64_t)ti * per_tile);
     const int g = rem >> 7, t = rem & 127;
     const int4 tl = tiles[ti];
-    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    uint4 o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) o[u] = make_uint4(0, 0, 0, 0);
     __half s = __float2half_rn(0.0f);
     if (t < tl.z) {
       const int slot = tl.y + t;
@@ -133,59 +154,57 @@ __global__ void __launch_bounds__(256) k_mma_gather(const int8_t* __restrict__ q
       }
       if (tok >= 0 && tok < T) {
         const uint4* src = reinterpret_cast<const uint4*>(qx + (int64_t)tok * K + 32 * g);
-        v0 = src[0];
-        v1 = src[1];
+        const uint4 v0 = src[0], v1 = src[1];
+        cvt_i8x4_f16(v0.x, o[0].x, o[0].y);
+        cvt_i8x4_f16(v0.y, o[0].z, o[0].w);
+        cvt_i8x4_f16(v0.z, o[1].x, o[1].y);
+        cvt_i8x4_f16(v0.w, o[1].z, o[1].w);
+        cvt_i8x4_f16(v1.x, o[2].x, o[2].y);
+        cvt_i8x4_f16(v1.y, o[2].z, o[2].w);
+        cvt_i8x4_f16(v1.z, o[3].x, o[3].y);
+        cvt_i8x4_f16(v1.w, o[3].z, o[3].w);
         s = sx[(int64_t)tok * G + g];
       } else if (g == 0) {
         set_status(status, kStatusDeviceCheck);
       }
     }
-    uint4* dst = reinterpret_cast<uint4*>(xa) + ((int64_t)ti * 2 * G + 2 * g) * 128 + t;
-    dst[0] = v0;
-    dst[128] = v1;
+    uint4* dst = reinterpret_cast<uint4*>(xa) + ((int64_t)ti * 4 * G + 4 * g) * 128 + t;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) dst[u * 128] = o[u];
     xs[((int64_t)ti * G + g) * 128 + t] = s;
-    int sum = __dp4a((int)v0.x, 0x01010101, 0);
-    sum = __dp4a((int)v0.y, 0x01010101, sum);
-    sum = __dp4a((int)v0.z, 0x01010101, sum);
-    sum = __dp4a((int)v0.w, 0x01010101, sum);
-    sum = __dp4a((int)v1.x, 0x01010101, sum);
-    sum = __dp4a((int)v1.y, 0x01010101, sum);
-    sum = __dp4a((int)v1.z, 0x01010101, sum);
-    sum = __dp4a((int)v1.w, 0x01010101, sum);
-    xsum[((int64_t)ti * G + g) * 128 + t] = sum;
   }
 }
 
 // -------------------------------------------------------------------- GEMM kernel
-constexpr int kMmaKC = 4;                  // groups per pipeline stage
+constexpr int kMmaKC = 2;                  // quantization groups per pipeline stage
 constexpr int kMmaNS = 4;                  // pipeline stages
-constexpr int kMmaNB = 4;                  // tensor-memory accumulator buffers (128 columns each:
+constexpr int kMmaNB = 4;                  // tensor-memory accumulators (128 fp32 columns each:
                                            // all 512; one CTA per SM), so MMAs run 4 groups ahead
-constexpr int kMmaThreads = 20 * 32;       // producer, MMA, 2 prep, 16 epilogue warps
+constexpr int kMmaPrepWarps = 2;
 constexpr int kMmaEpiWarps = 16;
+constexpr int kMmaEpi0 = 2 + kMmaPrepWarps;                       // first epilogue warp
+constexpr int kMmaThreads = (kMmaEpi0 + kMmaEpiWarps) * 32;       // producer, MMA, prep, epilogue
 
-// One pipeline stage: operand A (128 slots x 4 groups, int8), operand B (128 rows x 4 groups,
-// int8), packed int4 B as copied, the fp16 scales of both and B's scales as fp32.
+// One pipeline stage (two groups): operand A (the 128 slots' codes, already fp16 in the
+// workspace), operand B as copied (the int8 or packed int4 codes of 128 weight rows) and as
+// fp16 for the tensor cores, the fp16 scales of both and B's as fp32. Operand layout: K-major
+// canonical without swizzle, [16-byte piece along K][128 rows][16 B].
 struct MmaStage {
-  static constexpr int A = 0;              // [8 pieces][128][16]
-  static constexpr int B = 16384;          // [8 pieces][128][16]
-  static constexpr int BRAW = 32768;       // [4 pieces][128][16] (int4 weights)
-  static constexpr int AS = 40960;         // [4][128] fp16
-  static constexpr int BS = 41984;         // [4][128] fp16
-  static constexpr int BSF = 43008;        // [4][128] fp32
-  static constexpr int XS = 45056;         // [4][128] int32: code sums of A's groups (int4 B)
-  static constexpr int BYTES = 47104;
+  static constexpr int AH = 0;             // [8 pieces][128][16] fp16
+  static constexpr int BH = 16384;         // [8 pieces][128][16] fp16
+  static constexpr int B8 = 32768;         // [4 pieces][128][16] int8 (int4: 2 pieces)
+  static constexpr int AS = 40960;         // [2][128] fp16
+  static constexpr int BS = 41472;         // [2][128] fp16
+  static constexpr int BSF = 41984;        // [2][128] fp32
+  static constexpr int BYTES = 43008;      // a multiple of 1024
 };
-// + 32 KB of slack past the last stage: an operand descriptor's furthest byte stays inside
-// this CTA's shared memory whatever its strides.
-constexpr int kMmaSmem = kMmaNS * MmaStage::BYTES + 256 + 4096 + 1024 + 32 * 1024;
+// the stages, barriers (256 B), the h exchange (2 KB), 1 KB for aligning the base
+constexpr int kMmaSmem = kMmaNS * MmaStage::BYTES + 256 + 2048 + 1024;
 
-
-// Stage s's producer side: every copy of the chunk (4 groups) of item (tile, block).
-template <int WBITS, bool GATEUP>
+// Stage bytes the producer copies (A codes and scales, B codes and scales).
+template <int WBITS>
 __device__ __forceinline__ uint32_t mma_stage_bytes() {
-  constexpr uint32_t braw = WBITS == 8 ? 16384u : 8192u;
-  return 16384u + 1024u + braw + 1024u + (WBITS == 4 ? 2048u : 0u);
+  return 16384u + 512u + (WBITS == 8 ? 8192u : 4096u) + 512u;
 }
 
 template <int WBITS, bool GATEUP>
@@ -199,17 +218,18 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
   uint64_t* acc_empty = acc_full + kMmaNB;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + kMmaNB);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* xchg = reinterpret_cast<int*>(tmem_slot + 4);   // [2][2][128] h amax, [2][2][128] h code sums
+  int* xchg = reinterpret_cast<int*>(base + kMmaNS * MmaStage::BYTES + 256);   // [2][2][128] h amax
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int PPG = WBITS == 8 ? 2 : 1;  // 16-byte pieces of one group of packed weights
+  constexpr int PPG = WBITS == 8 ? 2 : 1;  // 16-byte pieces of one group of weight codes
   constexpr int PPU = 2 * PPG;             // pieces of a 64-column down slab row
   constexpr int kKern = GATEUP ? 3 : 4;
+  static_assert(kMmaKC == 2, "a stage is one 64-column down slab");
 
   if (threadIdx.x == 0) {
     *abort = 0;
     for (int s = 0; s < kMmaNS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&prep[s], 2);
+      mbar_init(&prep[s], kMmaPrepWarps);
       mbar_init(&empty[s], 1 + kMmaEpiWarps);
     }
     for (int b = 0; b < kMmaNB; ++b) {
@@ -218,7 +238,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
     }
     fence_barrier_init();
   }
-  for (int i = threadIdx.x; i < 4 * 2 * 128; i += kMmaThreads) xchg[i] = 0;
+  for (int i = threadIdx.x; i < 2 * 2 * 128; i += kMmaThreads) xchg[i] = 0;
   if (warp == 1) {
     tmem_alloc(tmem_slot, kMmaNB * 128);
     tmem_relinquish();
@@ -254,9 +274,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
         if (blkn >= (sh ? per_s : per_r)) continue;
         const int K = GATEUP ? H : bv.I;
         const int G = K / 32, KB = kbytes(K, WBITS);
-        const uint8_t* a_src = GATEUP ? A.a_ops + (int64_t)ti * 128 * K : A.h_ops + (int64_t)ti * 128 * A.hk;
+        const uint8_t* a_src = GATEUP ? A.a_ops + (int64_t)ti * 128 * K * 2 : A.h_ops + (int64_t)ti * 128 * A.hk * 2;
         const __half* as_src = GATEUP ? A.a_scales + (int64_t)ti * G * 128 : A.h_scales + (int64_t)ti * (A.hk / 32) * 128;
-        const int32_t* xs_src = GATEUP ? A.a_xsum + (int64_t)ti * G * 128 : A.h_xsum + (int64_t)ti * (A.hk / 32) * 128;
         for (int g0 = 0; g0 < G && ok; g0 += kMmaKC, ++c) {
           const int s = c % kMmaNS;
           if (c >= (uint32_t)kMmaNS && !mbar_wait(&empty[s], ((c / kMmaNS) - 1) & 1)) {
@@ -265,22 +284,19 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
             break;
           }
           uint8_t* st = base + s * MmaStage::BYTES;
-          mbar_arrive_expect_tx(&full[s], mma_stage_bytes<WBITS, GATEUP>());
-          bulk_load(st + MmaStage::A, a_src + (int64_t)g0 * 2 * 2048, 16384, &full[s]);
-          bulk_load(st + MmaStage::AS, as_src + (int64_t)g0 * 128, 1024, &full[s]);
-          if (WBITS == 4) bulk_load(st + MmaStage::XS, xs_src + (int64_t)g0 * 128, 2048, &full[s]);
-          uint8_t* bdst = st + (WBITS == 8 ? MmaStage::B : MmaStage::BRAW);
+          mbar_arrive_expect_tx(&full[s], mma_stage_bytes<WBITS>());
+          bulk_load(st + MmaStage::AH, a_src + (int64_t)g0 * 4 * 2048, 16384, &full[s]);
+          bulk_load(st + MmaStage::AS, as_src + (int64_t)g0 * 128, 512, &full[s]);
           if (GATEUP) {
             const int64_t blk = (int64_t)tl.w * 2 * bv.I + (int64_t)blkn * 128;
-            bulk_load_hint(bdst, bv.gu_w + blk * KB + (int64_t)g0 * PPG * 2048, kMmaKC * PPG * 2048, &full[s], once);
-            bulk_load_hint(st + MmaStage::BS, bv.gu_s + (blk * G + (int64_t)g0 * 128) * 2, 1024, &full[s], once);
+            bulk_load_hint(st + MmaStage::B8, bv.gu_w + blk * KB + (int64_t)g0 * PPG * 2048, kMmaKC * PPG * 2048,
+                           &full[s], once);
+            bulk_load_hint(st + MmaStage::BS, bv.gu_s + (blk * G + (int64_t)g0 * 128) * 2, 512, &full[s], once);
           } else {
             const int U = bv.I / 64, HB = bv.H / 128;
-            for (int h = 0; h < 2; ++h) {
-              const int64_t slab = ((int64_t)tl.w * U + g0 / 2 + h) * HB + blkn;
-              bulk_load_hint(bdst + h * PPU * 2048, bv.dn_w + slab * PPU * 2048, PPU * 2048, &full[s], once);
-              bulk_load_hint(st + MmaStage::BS + h * 512, bv.dn_s + slab * 512, 512, &full[s], once);
-            }
+            const int64_t slab = ((int64_t)tl.w * U + g0 / 2) * HB + blkn;
+            bulk_load_hint(st + MmaStage::B8, bv.dn_w + slab * PPU * 2048, PPU * 2048, &full[s], once);
+            bulk_load_hint(st + MmaStage::BS, bv.dn_s + slab * 512, 512, &full[s], once);
           }
         }
       }
@@ -296,8 +312,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
       uint32_t c = 0, gi = 0;
-      // int4 weights enter as unsigned bytes n ^ 8 = w + 8 (the epilogue subtracts 8 * sum(a))
-      constexpr uint32_t idesc = idesc_i8(128, 128, WBITS == 8);
+      constexpr uint32_t idesc = idesc_f16(128, 128);
       for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
         const int ti = it / per, blkn = it - ti * per;
         const int4 tl = A.tiles[ti];
@@ -323,19 +338,24 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
               ok = false;
             }
             tc_fence_after();
-            if (ok)
-              mma_i8(tmem + bb * 128, smem_desc(st + MmaStage::A + j * 4096, 2048, 128),
-                     smem_desc(st + MmaStage::B + j * 4096, 2048, 128), idesc, 0);
+            if (ok) {
+              // group j: fp16 pieces 4j .. 4j + 3, two MMAs of K = 16 (exact integer dot)
+              const uint8_t* a = st + MmaStage::AH + j * 8192;
+              const uint8_t* b = st + MmaStage::BH + j * 8192;
+              mma_f16(tmem + bb * 128, smem_desc(a, 2048, 128), smem_desc(b, 2048, 128), idesc, 0);
+              mma_f16(tmem + bb * 128, smem_desc(a + 4096, 2048, 128), smem_desc(b + 4096, 2048, 128), idesc, 1);
+            }
             mma_commit(&acc_full[bb]);         // arrives (in order) even when skipped
           }
           mma_commit(&empty[s]);
         }
       }
     }
-  } else if (warp < 4) {
-    // ---------------------------------------------------------------- prep: int4 -> int8, scales
+  } else if (warp < kMmaEpi0) {
+    // ---------------------------------------------------------------- prep: weight codes -> fp16, scales
     uint32_t c = 0;
-    const int pt = threadIdx.x - 64;        // [0, 64)
+    const int pt = threadIdx.x - 64;        // [0, 32 * kMmaPrepWarps)
+    constexpr int NPT = 32 * kMmaPrepWarps;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
       const int ti = it / per, blkn = it - ti * per;
       const int4 tl = A.tiles[ti];
@@ -353,27 +373,51 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
         }
         uint8_t* st = base + s * MmaStage::BYTES;
         if (ok) {
+          if (WBITS == 8) {
+            // int8 piece p (16 codes of a row) -> fp16 pieces 2p, 2p + 1; every load of the
+            // thread's share first (independent chains)
+            constexpr int NQ = 4 * 128 / NPT;
+            uint4 w[NQ];
+#pragma unroll
+            for (int u = 0; u < NQ; ++u) w[u] = *reinterpret_cast<const uint4*>(st + MmaStage::B8 + (pt + u * NPT) * 16);
+#pragma unroll
+            for (int u = 0; u < NQ; ++u) {
+              const int q = pt + u * NPT, p = q >> 7, r = q & 127;
+              uint4 lo, hi;
+              cvt_i8x4_f16(w[u].x, lo.x, lo.y);
+              cvt_i8x4_f16(w[u].y, lo.z, lo.w);
+              cvt_i8x4_f16(w[u].z, hi.x, hi.y);
+              cvt_i8x4_f16(w[u].w, hi.z, hi.w);
+              *reinterpret_cast<uint4*>(st + MmaStage::BH + ((2 * p) * 128 + r) * 16) = lo;
+              *reinterpret_cast<uint4*>(st + MmaStage::BH + ((2 * p + 1) * 128 + r) * 16) = hi;
+            }
+          }
           if (WBITS == 4) {
-            // group j of row r: 16 packed bytes -> pieces 2j, 2j+1 of unsigned bytes n ^ 8
-            for (int q = pt; q < kMmaKC * 128; q += 64) {
-              const int j = q >> 7, r = q & 127;
-              const uint4 w = *reinterpret_cast<const uint4*>(st + MmaStage::BRAW + (j * 128 + r) * 16);
-              const uint32_t wv[4] = {w.x ^ 0x88888888u, w.y ^ 0x88888888u, w.z ^ 0x88888888u, w.w ^ 0x88888888u};
-              uint32_t o[8];
+            // packed int4 piece j (the 32 codes of group j of a row, element 2b in the low nibble
+            // of byte b) -> fp16 pieces 4j .. 4j + 3
+            constexpr int NQ = 2 * 128 / NPT;
+            uint4 w[NQ];
+#pragma unroll
+            for (int v = 0; v < NQ; ++v) w[v] = *reinterpret_cast<const uint4*>(st + MmaStage::B8 + (pt + v * NPT) * 16);
+#pragma unroll
+            for (int v = 0; v < NQ; ++v) {
+              const int q = pt + v * NPT, j = q >> 7, r = q & 127;
+              const uint32_t wv[4] = {w[v].x, w[v].y, w[v].z, w[v].w};
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
-                const uint32_t lo = wv[u] & 0x0F0F0F0Fu, hi = (wv[u] >> 4) & 0x0F0F0F0Fu;
-                o[2 * u] = __byte_perm(lo, hi, 0x5140);
-                o[2 * u + 1] = __byte_perm(lo, hi, 0x7362);
+                const uint32_t x = wv[u] ^ 0x88888888u;            // nibbles n + 8
+                const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
+                uint4 o;
+                cvt_u4x4_f16(__byte_perm(lo, hi, 0x5140), o.x, o.y);   // elements 8u .. 8u + 3
+                cvt_u4x4_f16(__byte_perm(lo, hi, 0x7362), o.z, o.w);   // elements 8u + 4 .. 8u + 7
+                *reinterpret_cast<uint4*>(st + MmaStage::BH + ((4 * j + u) * 128 + r) * 16) = o;
               }
-              *reinterpret_cast<uint4*>(st + MmaStage::B + ((2 * j) * 128 + r) * 16) = make_uint4(o[0], o[1], o[2], o[3]);
-              *reinterpret_cast<uint4*>(st + MmaStage::B + ((2 * j + 1) * 128 + r) * 16) = make_uint4(o[4], o[5], o[6], o[7]);
             }
-            fence_async_smem();
           }
+          fence_async_smem();
           const __half* bs = reinterpret_cast<const __half*>(st + MmaStage::BS);
           float* bsf = reinterpret_cast<float*>(st + MmaStage::BSF);
-          for (int q = pt; q < kMmaKC * 128; q += 64) bsf[q] = __half2float(bs[q]);
+          for (int q = pt; q < kMmaKC * 128; q += NPT) bsf[q] = __half2float(bs[q]);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&prep[s]);
@@ -381,18 +425,18 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
     }
   } else {
     // ---------------------------------------------------------------- epilogue
-    // 16 warps: warp 4 + 4 c + q reads tensor-memory lane quadrant q (slots 32 q ..) and
-    // column slice c: gate/up -> gate columns 16 c .. 16 c + 15 and the matching up columns
+    // 16 warps: epilogue warp e reads tensor-memory lane quadrant warp % 4 (slots 32 q ..) and
+    // column slice e / 4: gate/up -> gate columns 16 c .. 16 c + 15 and the matching up columns
     // 64 + 16 c ..; down -> output rows 32 c .. 32 c + 31 of the block.
-    const int ew = warp - 4;                // [0, 16)
+    const int ew = warp - kMmaEpi0;         // [0, 16)
     const int quad = warp & 3;              // tensor-memory lane quadrant of this warp
     const int cs = ew >> 2;                 // column slice
     const int t = quad * 32 + lane;         // slot of the tile = tensor-memory lane
     const int colA = GATEUP ? 16 * cs : 32 * cs;
     const int colB = GATEUP ? 64 + 16 * cs : 32 * cs + 16;
+    const uint32_t tq = tmem + ((uint32_t)(quad * 32) << 16);
     // gate/up: the two slices of one Q8_0 group of h meet here (per item parity, group, slot)
     int* amax_s = xchg;                     // [item parity][group][slot]
-    int* hsum_s = xchg + 2 * 2 * 128;
     uint32_t c = 0, gi = 0, nit = 0;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
       const int ti = it / per, blkn = it - ti * per;
@@ -415,6 +459,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
         const uint8_t* st = base + s * MmaStage::BYTES;
         const __half* as = reinterpret_cast<const __half*>(st + MmaStage::AS);
         const float* bsf = reinterpret_cast<const float*>(st + MmaStage::BSF);
+#pragma unroll
         for (int j = 0; j < kMmaKC; ++j, ++gi) {
           const int bb = gi % kMmaNB;
           if (ok && !mbar_wait(&acc_full[bb], (gi / kMmaNB) & 1)) {
@@ -426,34 +471,31 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
           tc_fence_after();
           uint32_t d0[16], d1[16];
           if (ok) {
-            const uint32_t ta = tmem + ((uint32_t)(quad * 32) << 16) + bb * 128;
-            tmem_ld16(ta + colA, d0);
-            tmem_ld16(ta + colB, d1);
+            tmem_ld16(tq + bb * 128 + colA, d0);
+            tmem_ld16(tq + bb * 128 + colB, d1);
             tmem_wait_ld();
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[bb]);
           if (ok) {
-            // acc = fma((float)I_g, s_w * s_x, acc) per element, two elements per packed op;
-            // exact (float)I_g: bits of 1.5 * 2^23 + (D - 8 * sum(a)) minus 1.5 * 2^23
+            // acc = fma((float)I_g, s_w * s_x, acc) per element, two elements per packed op; the
+            // tensor cores already produced (float)I_g exactly
             const float sx = __half2float(as[j * 128 + t]);
             const float2 sx2 = make_float2(sx, sx);
-            const int kb = 0x4B400000 -
-                           (WBITS == 4 ? 8 * reinterpret_cast<const int32_t*>(st + MmaStage::XS)[j * 128 + t] : 0);
             const float4* sa = reinterpret_cast<const float4*>(bsf + j * 128 + colA);
             const float4* sb = reinterpret_cast<const float4*>(bsf + j * 128 + colB);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
               const float4 wa = sa[q4], wb = sb[q4];
               const int q = 4 * q4;
-              acc2[q / 2] = __ffma2_rn(exact_i2f2k((int)d0[q], (int)d0[q + 1], kb),
+              acc2[q / 2] = __ffma2_rn(make_float2(__uint_as_float(d0[q]), __uint_as_float(d0[q + 1])),
                                        __fmul2_rn(make_float2(wa.x, wa.y), sx2), acc2[q / 2]);
-              acc2[q / 2 + 1] = __ffma2_rn(exact_i2f2k((int)d0[q + 2], (int)d0[q + 3], kb),
+              acc2[q / 2 + 1] = __ffma2_rn(make_float2(__uint_as_float(d0[q + 2]), __uint_as_float(d0[q + 3])),
                                            __fmul2_rn(make_float2(wa.z, wa.w), sx2), acc2[q / 2 + 1]);
-              acc2[8 + q / 2] = __ffma2_rn(exact_i2f2k((int)d1[q], (int)d1[q + 1], kb),
+              acc2[8 + q / 2] = __ffma2_rn(make_float2(__uint_as_float(d1[q]), __uint_as_float(d1[q + 1])),
                                            __fmul2_rn(make_float2(wb.x, wb.y), sx2), acc2[8 + q / 2]);
-              acc2[8 + q / 2 + 1] = __ffma2_rn(exact_i2f2k((int)d1[q + 2], (int)d1[q + 3], kb),
+              acc2[8 + q / 2 + 1] = __ffma2_rn(make_float2(__uint_as_float(d1[q + 2]), __uint_as_float(d1[q + 3])),
                                                __fmul2_rn(make_float2(wb.z, wb.w), sx2), acc2[8 + q / 2 + 1]);
             }
           }
@@ -476,7 +518,6 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
         const int i0 = blkn * 64 + 16 * cs;  // the thread's 16 intermediate indices
         const int par = nit & 1, gl = cs >> 1;
         int* am = amax_s + (par * 2 + gl) * 128 + t;
-        int* hm = hsum_s + (par * 2 + gl) * 128 + t;
         float h[16];
         float amax = 0.0f;
 #pragma unroll
@@ -495,13 +536,16 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
           for (int u = 0; u < 4; ++u) v |= (uint32_t)(uint8_t)(int8_t)quant_code(h[4 * w4 + u], sc, 127.0f) << (8 * u);
           pk[w4] = v;
         }
-        int hsum = 0;
-#pragma unroll
-        for (int w4 = 0; w4 < 4; ++w4) hsum = __dp4a((int)pk[w4], 0x01010101, hsum);
-        atomicAdd(hm, hsum);
         if (live) {
-          *reinterpret_cast<uint4*>(A.h_ops + ((int64_t)ti * (A.hk / 16) + i0 / 16) * 128 * 16 + t * 16) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          // the down GEMM's operand A: the 16 codes as fp16, pieces i0 / 8 and i0 / 8 + 1
+          uint4 f0, f1;
+          cvt_i8x4_f16(pk[0], f0.x, f0.y);
+          cvt_i8x4_f16(pk[1], f0.z, f0.w);
+          cvt_i8x4_f16(pk[2], f1.x, f1.y);
+          cvt_i8x4_f16(pk[3], f1.z, f1.w);
+          uint4* hd = reinterpret_cast<uint4*>(A.h_ops) + ((int64_t)ti * (A.hk / 8) + i0 / 8) * 128 + t;
+          hd[0] = f0;
+          hd[128] = f1;
           if (valid) {
             *reinterpret_cast<uint4*>(A.qh[sh] + (int64_t)slot * I + i0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             if (A.dbg_a[sh])
@@ -516,11 +560,9 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
           if (live) {
             const int64_t hg = (int64_t)ti * (A.hk / 32) + i0 / 32;
             A.h_scales[hg * 128 + t] = __float2half_rn(sc);
-            A.h_xsum[hg * 128 + t] = *hm;
             if (valid) A.sh[sh][(int64_t)slot * IB + i0 / 32] = __float2half_rn(sc);
           }
-          *am = 0;                           // this parity's entries are next used two items on
-          *hm = 0;
+          *am = 0;                           // this parity's entry is next used two items on
         }
       } else if (valid && live) {
         int tok = slot;
@@ -593,11 +635,11 @@ cudaError_t launch_mma_plan(const Grouping& g, int E, int T, int has_shared, int
 
 cudaError_t launch_mma_gather(const int8_t* qx, const __half* sx, const int4* tiles, const int32_t* n_tiles,
                               const int32_t* perm, int k, int T, int K, int max_tiles, uint8_t* xa, __half* xs,
-                              int32_t* xsum, int* status, cudaStream_t st) {
+                              int* status, cudaStream_t st) {
   const int64_t work = (int64_t)max_tiles * 128 * (K / 32);
   const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, (int64_t)sm_count_mma() * 8));
   return launch_pdl(k_mma_gather, dim3(grid), dim3(256), 0, st, qx, sx, tiles, n_tiles, perm, k, T, K, xa, xs,
-                    xsum, status);
+                    status);
 }
 
 cudaError_t launch_expert_mma(bool gateup, const MmaArgs& a, cudaStream_t st) {

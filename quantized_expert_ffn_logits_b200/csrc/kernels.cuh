@@ -83,14 +83,12 @@ struct MmaArgs {
   const int4* tiles;
   const int32_t* n_tiles;
   int max_tiles;
-  const uint8_t* a_ops;                    // operand A of every tile: [tile][K/16][128][16]
+  const uint8_t* a_ops;                    // operand A of every tile, fp16: [tile][K/8][128][16]
   const __half* a_scales;                  // [tile][K/32][128]
-  const int32_t* a_xsum;                   // [tile][K/32][128] sum of a group's codes (int4 weights)
   // gate/up outputs: h of every tile in operand layout for the down GEMM, and the per-slot
   // views of the workspace (q_h, s_h; gate / up values when debugging)
-  uint8_t* h_ops;                          // [tile][hk/16][128][16]
+  uint8_t* h_ops;                          // fp16: [tile][hk/8][128][16]
   __half* h_scales;                        // [tile][hk/32][128]
-  int32_t* h_xsum;                         // [tile][hk/32][128]
   int hk;                                  // row length of a tile's h: max(I, I_shared)
   int8_t* qh[2];
   __half* sh[2];
@@ -111,7 +109,7 @@ cudaError_t launch_mma_plan(const Grouping& g, int E, int T, int has_shared, int
 // Operand A (q_x rows of each tile's tokens, [tile][K/16][128][16]) and its scales.
 cudaError_t launch_mma_gather(const int8_t* qx, const __half* sx, const int4* tiles, const int32_t* n_tiles,
                               const int32_t* perm, int k, int T, int K, int max_tiles, uint8_t* xa, __half* xs,
-                              int32_t* xsum, int* status, cudaStream_t st);
+                              int* status, cudaStream_t st);
 // Gate/up (+ SwiGLU, Q8_0 h) or down (+ weighted combine) of every tile x weight block.
 cudaError_t launch_expert_mma(bool gateup, const MmaArgs& a, cudaStream_t st);
 
