@@ -322,3 +322,42 @@ def test_extreme_top_k(k):
     g = gpu_layer(case)
     y, ws = m.moe_layer_forward(g["x"], g["wr"], None, g["blob"], None, route_cfg(c))
     assert_close_y(_np(y), oracle_layer(case)["y"])
+
+
+@pytest.mark.parametrize("wtype", ["int8", "int4"])
+def test_tensor_core_dots_exact_at_extreme_codes(wtype):
+    """The tensor-core path forms each group's dot with fp16 operands and an fp32
+    accumulator; that is exact only because every partial sum is an integer below 2^24. Pin it
+    where the sums are largest: x and every weight are +-1, so every activation code is +-127
+    and every weight code +-127 (int8) or +-7 (int4), and half of the weight rows copy the sign
+    pattern of token 0 (group dots up to 32 * 127 * 127). Gate/up stage values must equal the
+    oracle's bit for bit."""
+    m = M()
+    rng = np.random.default_rng(77)
+    E, H, I, T, k = 2, 256, 128, 40, 2
+    x = np.where(rng.random((T, H)) < 0.5, -1.0, 1.0).astype(np.float32)
+    gu = np.where(rng.random((E, 2 * I, H)) < 0.5, -1.0, 1.0).astype(np.float32)
+    gu[:, ::2, :] = x[0]                       # rows whose dots with token 0 are maximal
+    dn = np.where(rng.random((E, H, I)) < 0.5, -1.0, 1.0).astype(np.float32)
+    wr = rng.normal(0.0, 1.0 / np.sqrt(H), (E, H)).astype(np.float32)
+    wb = 8 if wtype == "int8" else 4
+    ex = O.QExperts.quantize(gu, dn, wb, True)
+    ref = O.layer_forward(x, wr, None, ex, None, "softmax", k, True, 1.0, True, union=True)
+    blob = m.ExpertBlob.quantize(torch.from_numpy(gu).cuda(), torch.from_numpy(dn).cuda(), wtype, "g32_f16")
+    cfg = m.RouteCfg(score="softmax", top_k=k, renormalize=True, routed_scaling_factor=1.0, act="g32_f16",
+                     flags=m.MOE_FLAG_DEBUG | m.MOE_FLAG_FORCE_MMA)
+    y, ws = m.moe_layer_forward(torch.from_numpy(x).cuda(), torch.from_numpy(wr).cuda(), None, blob, None, cfg)
+    torch.cuda.synchronize()
+    assert m.moe_read_device_status(ws) == m.MOE_OK
+    v = m.moe_layer_debug_views(T, blob, None, cfg)
+    view = lambda off, dt, shape: _np(m.workspace_view(ws, off, dt, shape))
+    P = T * k
+    perm = view(v["perm"], torch.int32, (P,))
+    assert np.array_equal(perm, ref["perm"])
+    gate = view(v["gate"], torch.float32, (P, I))
+    up = view(v["up"], torch.float32, (P, I))
+    assert np.abs(gate).max() > 0
+    assert np.array_equal(gate, ref["gate"][perm]), "gate stage values"
+    assert np.array_equal(up, ref["up"][perm]), "up stage values"
+    assert np.array_equal(view(v["q_h"], torch.int8, (P, I)), ref["qh"][perm])
+    assert_close_y(_np(y), ref["y"])
