@@ -181,6 +181,7 @@ constexpr int kMmaNS = 4;                  // pipeline stages
 constexpr int kMmaNB = 4;                  // tensor-memory accumulators (128 fp32 columns each:
                                            // all 512; one CTA per SM), so MMAs run 4 groups ahead
 constexpr int kMmaPrepWarps = 2;
+constexpr uint32_t kMmaSleepNs = 200;      // backoff of the roles that run ahead of the epilogue
 constexpr int kMmaEpiWarps = 16;
 constexpr int kMmaEpi0 = 2 + kMmaPrepWarps;                       // first epilogue warp
 constexpr int kMmaThreads = (kMmaEpi0 + kMmaEpiWarps) * 32;       // producer, MMA, prep, epilogue
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
         const __half* as_src = GATEUP ? A.a_scales + (int64_t)ti * G * 128 : A.h_scales + (int64_t)ti * (A.hk / 32) * 128;
         for (int g0 = 0; g0 < G && ok; g0 += kMmaKC, ++c) {
           const int s = c % kMmaNS;
-          if (c >= (uint32_t)kMmaNS && !mbar_wait(&empty[s], ((c / kMmaNS) - 1) & 1)) {
+          if (c >= (uint32_t)kMmaNS && !mbar_wait_sleep(&empty[s], ((c / kMmaNS) - 1) & 1, kMmaSleepNs)) {
             wait_failed(A.status, kKern, 0, s);
             ok = false;
             break;
@@ -323,7 +324,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
         for (int g0 = 0; g0 < G; g0 += kMmaKC, ++c) {
           const int s = c % kMmaNS;
           bool ok = *abort == 0;
-          if (ok && !mbar_wait(&prep[s], (c / kMmaNS) & 1)) {
+          if (ok && !mbar_wait_sleep(&prep[s], (c / kMmaNS) & 1, kMmaSleepNs)) {
             *abort = 1;
             wait_failed(A.status, kKern, 1, s);
             ok = false;
@@ -332,7 +333,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
           const uint8_t* st = base + s * MmaStage::BYTES;
           for (int j = 0; j < kMmaKC; ++j, ++gi) {
             const int bb = gi % kMmaNB;
-            if (ok && gi >= (uint32_t)kMmaNB && !mbar_wait(&acc_empty[bb], ((gi / kMmaNB) - 1) & 1)) {
+            if (ok && gi >= (uint32_t)kMmaNB && !mbar_wait_sleep(&acc_empty[bb], ((gi / kMmaNB) - 1) & 1, kMmaSleepNs)) {
               *abort = 1;
               wait_failed(A.status, kKern, 3, bb);
               ok = false;
@@ -366,7 +367,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
       for (int g0 = 0; g0 < G; g0 += kMmaKC, ++c) {
         const int s = c % kMmaNS;
         bool ok = *abort == 0;
-        if (ok && !mbar_wait(&full[s], (c / kMmaNS) & 1)) {
+        if (ok && !mbar_wait_sleep(&full[s], (c / kMmaNS) & 1, kMmaSleepNs)) {
           *abort = 1;
           if (lane == 0) wait_failed(A.status, kKern, 4, s);
           ok = false;
