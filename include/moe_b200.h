@@ -276,8 +276,11 @@ MOE_API moe_status moe_layer_forward_timed(const float* x, int32_t T, const floa
  * [T][H] into x_dev, the layer (y_dev [T][H]) and the copy of y_dev into y_host, and returns
  * (synchronize `stream` before reading y_host). x_host / y_host should be page-locked
  * (cudaHostAlloc) for the copies to be asynchronous; x_dev / y_dev are device buffers of
- * T * H floats, 16-byte aligned, owned by the caller. Errors as moe_layer_forward, plus
- * INVALID_ARG for a null buffer and CUDA for a failed copy. */
+ * T * H floats, 16-byte aligned, owned by the caller, used as this call's staging: with
+ * page-locked (device-mapped) host buffers the SMs move x and y in kernels chained to the
+ * layer's, and x_dev may be written before work enqueued earlier on `stream` has finished, so
+ * such work must not read x_dev. Errors as moe_layer_forward, plus INVALID_ARG for a null
+ * buffer and CUDA for a failed copy. */
 MOE_API moe_status moe_layer_forward_host(const float* x_host, int32_t T, const float* router_w,
                                           const float* router_bias, const moe_expert_blob* experts,
                                           const moe_expert_blob* shared, const moe_route_cfg* cfg,
