@@ -236,7 +236,7 @@ __device__ __forceinline__ void act_group_sums(const uint8_t* xs, int* xsum, int
 // buffer 0, computes the router logits of experts blockIdx.x, blockIdx.x + grid, ... in the
 // fixed fp32 order (32-element fma chunks from +0, chunk partials added in chunk order) and
 // zeroes its share of y. After a grid barrier every CTA reads the E logits and makes the
-// same top-k selection (all keys ranked in parallel; softmax or sigmoid weights as in
+// same top-k selection (a chunked parallel rank; softmax or sigmoid weights as in
 // topk.cuh); CTA 0 also writes the routing and grouping views of the workspace.
 struct RouteSmem {
   int* se;        // [k] selected experts, ascending (active-expert order)
@@ -332,7 +332,8 @@ __device__ __forceinline__ bool stage_router_rows(const RouteArgs& r, bool cl, u
 __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Ring& R, const RouteSmem& S,
                                 uint64_t* rows_bar, bool cl) {
   volatile int* flag = S.flag;
-  const int tid = threadIdx.x, H = r.H, G = H / 32, C = H / 32, E = r.E, k = r.k;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = r.H, G = H / 32, C = H / 32, E = r.E, k = r.k;
   const bool cta0 = blockIdx.x == 0;
   const Owners own = route_owners(cl);
   if (cta0 && tid == 0) {
@@ -479,33 +480,67 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
     if (!good) return false;
   }
   if (tid < 32) S.sidx[tid] = -1;
-  // 5. top-k (every CTA, same result): every key ranks itself against all E keys in
-  //    parallel (rank = keys larger, or equal with a lower expert index: descending, ties
-  //    to the lower expert). The logits also go to activation buffer 1 (idle in this mode):
-  //    the routing weights are formed there after the producer has started.
+  // 5. top-k (every CTA, same result): keys ranked by (keys larger, or equal with a lower
+  //    expert index): descending, ties to the lower expert. The logits also go to activation
+  //    buffer 1 (idle in this mode): the routing weights are formed there after the producer
+  //    has started.
   float* slogk = reinterpret_cast<float*>(R.abuf + P.abytes);
+  float* ckey = skey + 512;                                 // [E / 64 * k] candidate keys
+  int* cidx = reinterpret_cast<int*>(ckey + 512);           //              their experts
   for (int i = tid; i < E; i += kNT) {
     const float L = slog[i];
     slogk[i] = L;
     skey[i] = r.score == 0 ? L : __fadd_rn(csigmoid(L), r.bias ? r.bias[i] : 0.0f);
   }
+  const int nch = (E + 63) / 64, ncand = nch * k;
+  for (int t = tid; t < ncand; t += kNT) cidx[t] = -1;     // chunks with fewer than k keys
   __syncthreads();
+  // Two phases, O(64 E + (k E / 64)^2) comparisons instead of O(E^2): (a) every key ranks
+  // itself within its chunk of 64 keys (one thread per key); with one chunk that is the
+  // answer, else a key of chunk rank < k is a candidate, kept (key and expert) at slot
+  // chunk * k + rank; (b) every candidate ranks itself against all candidates. A key of the
+  // global top k is among its chunk's top k, and every key ranked above it is too, so its rank
+  // among the candidates is its global rank (same tie rule throughout).
   for (int i = tid; i < E; i += kNT) {
+    const int base = i & ~63, n = min(64, E - base);
     const float kv = skey[i];
     int rank = 0, j = 0;
-    if ((E & 3) == 0) {
-      const float4* k4 = reinterpret_cast<const float4*>(skey);
+    if ((n & 3) == 0) {
+      const float4* k4 = reinterpret_cast<const float4*>(skey + base);
 #pragma unroll 4
-      for (; j < E; j += 4) {
+      for (; j < n; j += 4) {
         const float4 q = k4[j >> 2];
-        rank += (q.x > kv) | ((q.x == kv) & (j < i));
-        rank += (q.y > kv) | ((q.y == kv) & (j + 1 < i));
-        rank += (q.z > kv) | ((q.z == kv) & (j + 2 < i));
-        rank += (q.w > kv) | ((q.w == kv) & (j + 3 < i));
+        const int jj = base + j;
+        rank += (q.x > kv) | ((q.x == kv) & (jj < i));
+        rank += (q.y > kv) | ((q.y == kv) & (jj + 1 < i));
+        rank += (q.z > kv) | ((q.z == kv) & (jj + 2 < i));
+        rank += (q.w > kv) | ((q.w == kv) & (jj + 3 < i));
       }
     }
-    for (; j < E; ++j) rank += (skey[j] > kv) | ((skey[j] == kv) & (j < i));
-    if (rank < k) S.sidx[rank] = i;
+    for (; j < n; ++j) rank += (skey[base + j] > kv) | ((skey[base + j] == kv) & (base + j < i));
+    if (rank < k) {
+      if (nch == 1) {
+        S.sidx[rank] = i;
+      } else {
+        ckey[(i >> 6) * k + rank] = kv;
+        cidx[(i >> 6) * k + rank] = i;
+      }
+    }
+  }
+  if (nch > 1) {
+    __syncthreads();
+    for (int t = tid; t < ncand; t += kNT) {
+      const int i = cidx[t];
+      if (i < 0) continue;
+      const float kv = ckey[t];
+      int rank = 0;
+      for (int u = 0; u < ncand; ++u) {
+        const float q = ckey[u];
+        const int j = cidx[u];
+        rank += (j >= 0) & ((q > kv) | ((q == kv) & (j < i)));
+      }
+      if (rank < k) S.sidx[rank] = i;
+    }
   }
   fence_async_smem();                       // this thread's ring accesses precede the bulk copies
   __syncthreads();

@@ -361,3 +361,29 @@ def test_tensor_core_dots_exact_at_extreme_codes(wtype):
     assert np.array_equal(up, ref["up"][perm]), "up stage values"
     assert np.array_equal(view(v["q_h"], torch.int8, (P, I)), ref["qh"][perm])
     assert_close_y(_np(y), ref["y"])
+
+
+def test_single_token_selection_ties_go_to_lower_experts():
+    """x = 0 makes every router logit 0: the in-kernel selection of the single-token path
+    (here 256 experts: four 64-expert chunks, then the candidates ranked against each other)
+    must return experts 0 .. k-1 in that order, with equal softmax weights."""
+    m = M()
+    E, H, I, k = 256, 1024, 64, 8
+    rng = np.random.default_rng(5)
+    gu = rng.normal(0.0, 0.02, (E, 2 * I, H)).astype(np.float32)
+    dn = rng.normal(0.0, 0.02, (E, H, I)).astype(np.float32)
+    wr = rng.normal(0.0, 1.0 / np.sqrt(H), (E, H)).astype(np.float32)
+    blob = m.ExpertBlob.quantize(torch.from_numpy(gu).cuda(), torch.from_numpy(dn).cuda(), "int8", "g32_f16")
+    cfg = m.RouteCfg(score="softmax", top_k=k, renormalize=True, routed_scaling_factor=1.0, act="g32_f16",
+                     flags=m.MOE_FLAG_DEBUG)
+    assert m.moe_layer_kernel_count(1, blob, None, cfg) == 1          # the single-token kernel
+    x = torch.zeros((1, H), dtype=torch.float32, device="cuda")
+    y, ws = m.moe_layer_forward(x, torch.from_numpy(wr).cuda(), None, blob, None, cfg)
+    torch.cuda.synchronize()
+    assert m.moe_read_device_status(ws) == m.MOE_OK
+    v = m.moe_layer_debug_views(1, blob, None, cfg)
+    idx = _np(m.workspace_view(ws, v["idx"], torch.int32, (1, k)))
+    w = _np(m.workspace_view(ws, v["w"], torch.float32, (1, k)))
+    assert idx.tolist() == [list(range(k))]
+    assert np.allclose(w, 1.0 / k, rtol=1e-6)
+    assert np.array_equal(_np(y), np.zeros((1, H), np.float32))
