@@ -368,7 +368,7 @@ def test_single_token_selection_ties_go_to_lower_experts():
     (here 256 experts: four 64-expert chunks, then the candidates ranked against each other)
     must return experts 0 .. k-1 in that order, with equal softmax weights."""
     m = M()
-    E, H, I, k = 256, 1024, 64, 8
+    E, H, I, k = 256, 1024, 128, 8
     rng = np.random.default_rng(5)
     gu = rng.normal(0.0, 0.02, (E, 2 * I, H)).astype(np.float32)
     dn = rng.normal(0.0, 0.02, (E, H, I)).astype(np.float32)
