@@ -97,7 +97,7 @@ enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID_NOAUX_TC = 1 };
                                       in the workspace (see moe_layer_debug_views) */
 #define MOE_FLAG_FORCE_GEMV 2u     /* run every expert on the weight-streaming (GEMV) path */
 #define MOE_FLAG_FORCE_MMA 4u      /* T > 32: run every expert (shared one included) with at least
-                                      one pair on the tensor-core path (normally: >= 64 pairs) */
+                                      one pair on the tensor-core path (normally: >= 16 pairs) */
 
 /* A set of E quantized experts of one layer (or the single shared expert, E = 1).
  *

@@ -76,7 +76,11 @@ cudaError_t launch_experts(int mode, const ExpertArgs& gr, const ExpertArgs* gs,
                            const ExpertArgs* ds, int mma_min, cudaStream_t st);
 
 // ---- expert_mma.cu: tensor-core GEMMs for experts with many tokens
-constexpr int kMmaMinTokens = 64;          // pairs an expert needs in a call to take this path
+// Pairs an expert needs in a call to take this path. A tensor-core call costs about the same
+// whatever its tiles' fill (~510 us for the 64 OLMoE-shaped int4 experts at one tile each),
+// while streaming an expert costs in proportion to its pairs: measured, streaming wins below
+// ~12-16 pairs per expert.
+constexpr int kMmaMinTokens = 16;
 
 struct MmaArgs {
   BlobView b[2];                           // routed experts, shared expert

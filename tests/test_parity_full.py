@@ -23,7 +23,7 @@ FULL = [
     ("glm_int4", 4, 2),
     ("e512_int4", 1, None),
     ("e512_int4", 64, 8),
-    ("olmoe_int4", 512, 6),        # tensor-core path (experts with >= 64 pairs)
+    ("olmoe_int4", 512, 6),        # tensor-core path (experts with >= 16 pairs)
     ("olmoe_int4", 4096, 4),
     ("e512_int4", 4096, 4),        # Zipf-skewed: tensor cores for hot experts, streaming for the rest
 ]

@@ -66,7 +66,7 @@ def test_layer_forward_matches_oracle(name, T):
     _check_layer(name, T, M().MOE_FLAG_DEBUG)
 
 
-# The tensor-core path (experts with >= 64 pairs at T > 32; every expert with the force flag):
+# The tensor-core path (experts with >= 16 pairs at T > 32; every expert with the force flag):
 # the same bit-exact gate/up values, h codes and scales as the streaming path and the oracle.
 MMA_CASES = [("olmoe_int4", 300, False), ("olmoe_int4", 40, True), ("olmoe_int8", 70, True),
              ("e512_int4", 100, True), ("glm_int4", 50, True)]
