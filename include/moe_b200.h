@@ -341,6 +341,24 @@ MOE_API moe_status moe_expert_group_dots(const moe_expert_blob* blob, int32_t wh
  * recorded by the kernels, or MOE_ERR_CUDA if the copy fails. */
 MOE_API moe_status moe_read_device_status(void* workspace, size_t ws_bytes, void* stream);
 
+/* moe_read_device_status for a workspace of at least its 256-byte control block (every
+ * moe_layer_forward and moe_permute workspace): the status query without a size. Synchronizes
+ * `stream`; same returns. */
+MOE_API moe_status moe_get_device_status(void* workspace, void* stream);
+
+/* moe_layer_forward with MOE_FLAG_DEBUG added to cfg->flags (so the workspace must hold
+ * moe_layer_workspace_bytes() of that configuration), and `views` filled as
+ * moe_layer_debug_views() fills it: byte offsets, inside `workspace`, of the call's
+ * intermediates (quantized x, logits, idx, w, grouping, quantized h, gate/up stage values and
+ * per-pair down values). Sampled int32 group dots come from moe_expert_group_dots. Errors as
+ * moe_layer_forward, plus INVALID_ARG for a null cfg or views; views is written only when the
+ * call returns MOE_OK with T > 0. */
+MOE_API moe_status moe_layer_forward_debug(const float* x, int32_t T, const float* router_w,
+                                           const float* router_bias, const moe_expert_blob* experts,
+                                           const moe_expert_blob* shared, const moe_route_cfg* cfg,
+                                           float* y, void* workspace, size_t ws_bytes, void* stream,
+                                           moe_debug_views* views);
+
 #ifdef __cplusplus
 }
 #endif

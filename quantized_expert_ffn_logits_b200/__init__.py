@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import ctypes as C
 import os
+import dataclasses
 from dataclasses import dataclass
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -81,6 +82,9 @@ _SIGS = {
     "moe_layer_debug_views": (_i32, [_i32, _PB, _PB, _PC, C.POINTER(moe_debug_views)]),
     "moe_expert_group_dots": (_i32, [_PB, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "moe_read_device_status": (_i32, [_vp, _sz, _vp]),
+    "moe_get_device_status": (_i32, [_vp, _vp]),
+    "moe_layer_forward_debug": (_i32, [_vp, _i32, _vp, _vp, _PB, _PB, _PC, _vp, _vp, _sz, _vp,
+                                       C.POINTER(moe_debug_views)]),
 }
 EXPORTS = tuple(_SIGS)
 for _name, (_res, _args) in _SIGS.items():
@@ -377,6 +381,41 @@ def moe_expert_group_dots(blob: ExpertBlob, which: int, expert, row, act, stream
 
 def moe_read_device_status(workspace, stream=None) -> int:
     return int(_lib.moe_read_device_status(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_get_device_status(workspace, stream=None) -> int:
+    return int(_lib.moe_get_device_status(_ptr(workspace), _stream(stream)))
+
+
+def moe_layer_forward_debug(x, router_w, router_bias, experts: ExpertBlob,
+                            shared: ExpertBlob | None, cfg: RouteCfg, y=None, workspace=None,
+                            stream=None):
+    """moe_layer_forward with the debug intermediates kept: returns (y, workspace, views), views
+    being the byte offsets of moe_layer_debug_views (read them with workspace_view)."""
+    import torch
+    T, H = x.shape
+    dbg = dataclasses.replace(cfg, flags=cfg.flags | MOE_FLAG_DEBUG)
+    _dev(x, torch.float32, "x")
+    _dev(router_w, torch.float32, "router_w")
+    _dev(router_bias, torch.float32, "router_bias")
+    if y is None:
+        y = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    _dev(y, torch.float32, "y")
+    nb = moe_layer_workspace_bytes(T, experts, shared, dbg)
+    if nb == 0:
+        raise MoeError(MOE_ERR_UNSUPPORTED, "moe_layer_workspace_bytes")
+    if workspace is None:
+        workspace = torch.zeros(nb, dtype=torch.uint8, device=x.device)   # control block zeroed
+    _dev(workspace, torch.uint8, "workspace")
+    e = experts.struct()
+    s = shared.struct() if shared is not None else None
+    c = cfg.struct()
+    v = moe_debug_views()
+    _check(_lib.moe_layer_forward_debug(_ptr(x), T, _ptr(router_w), _ptr(router_bias), C.byref(e),
+                                        C.byref(s) if s else None, C.byref(c), _ptr(y), _ptr(workspace),
+                                        workspace.numel(), _stream(stream), C.byref(v)),
+           "moe_layer_forward_debug")
+    return y, workspace, {n: getattr(v, n) for n, _ in moe_debug_views._fields_}
 
 
 def workspace_view(workspace, offset: int, dtype, shape):

@@ -747,4 +747,21 @@ moe_status moe_read_device_status(void* workspace, size_t ws_bytes, void* stream
   return static_cast<moe_status>(h);
 }
 
+moe_status moe_get_device_status(void* workspace, void* stream) {
+  return moe_read_device_status(workspace, (size_t)kControlBytes, stream);
+}
+
+moe_status moe_layer_forward_debug(const float* x, int32_t T, const float* router_w,
+                                   const float* router_bias, const moe_expert_blob* experts,
+                                   const moe_expert_blob* shared, const moe_route_cfg* cfg, float* y,
+                                   void* workspace, size_t ws_bytes, void* stream, moe_debug_views* views) {
+  if (!cfg || !views) return MOE_ERR_INVALID_ARG;
+  moe_route_cfg c = *cfg;
+  c.flags |= MOE_FLAG_DEBUG;
+  const moe_status s = moe_layer_forward(x, T, router_w, router_bias, experts, shared, &c, y, workspace,
+                                         ws_bytes, stream);
+  if (s != MOE_OK || T == 0) return s;
+  return moe_layer_debug_views(T, experts, shared, &c, views);
+}
+
 }  // extern "C"

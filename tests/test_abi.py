@@ -114,3 +114,12 @@ def test_other_entry_points_reject_bad_arguments():
     assert v.gate > 0 and v.up > 0 and v.y_pair > 0 and v.total == L.moe_layer_workspace_bytes(4, C.byref(b), None, C.byref(_cfg(flags=1)))
     assert L.moe_layer_debug_views(4, C.byref(b), None, C.byref(_cfg()), C.byref(v)) == M.MOE_OK
     assert v.gate == -1
+    assert L.moe_get_device_status(None, None) == M.MOE_ERR_INVALID_ARG
+    # the debug forward sizes its workspace for the debug layout and leaves views alone on errors
+    f = L.moe_layer_forward_debug
+    plain = L.moe_layer_workspace_bytes(4, C.byref(b), None, C.byref(_cfg()))
+    v.gate = 12345
+    assert f(fake, 4, fake, None, C.byref(b), None, None, fake, fake, plain, None, C.byref(v)) == M.MOE_ERR_INVALID_ARG
+    assert f(fake, 4, fake, None, C.byref(b), None, C.byref(_cfg()), fake, fake, plain, None, None) == M.MOE_ERR_INVALID_ARG
+    assert f(fake, 4, fake, None, C.byref(b), None, C.byref(_cfg()), fake, fake, plain, None, C.byref(v)) == M.MOE_ERR_WORKSPACE
+    assert v.gate == 12345

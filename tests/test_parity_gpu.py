@@ -151,6 +151,26 @@ def test_forward_without_debug_equals_debug(name, T):
     assert_close_y(_np(y0), ref["y"])
 
 
+@pytest.mark.parametrize("name,T", [("olmoe_int8", 1), ("e512_int4", 64)])
+def test_forward_debug_entry_point(name, T):
+    """moe_layer_forward_debug: the forward with the debug intermediates kept, and their offsets
+    returned in the same call (routing indices and h codes equal to the oracle's; y within the
+    layer tolerance); moe_get_device_status reads the clean status word."""
+    m = M()
+    case = S.Case.make(REDUCED[name], T)
+    g = gpu_layer(case)
+    c = case.cfg
+    y, ws, v = m.moe_layer_forward_debug(g["x"], g["wr"], g["bias"], g["blob"], g["shared"], route_cfg(c))
+    torch.cuda.synchronize()
+    assert m.moe_get_device_status(ws) == m.MOE_OK
+    assert v == m.moe_layer_debug_views(T, g["blob"], g["shared"], route_cfg(c, m.MOE_FLAG_DEBUG))
+    assert v["gate"] >= 0 and v["y_pair"] >= 0
+    ref = oracle_layer(case)
+    idx = _np(m.workspace_view(ws, v["idx"], torch.int32, (T, c.top_k)))
+    assert np.array_equal(idx, ref["idx"])
+    assert_close_y(_np(y), ref["y"])
+
+
 @pytest.mark.parametrize("name,T", [("olmoe_int8", 1), ("glm_int4", 3), ("olmoe_int4", 40)])
 def test_forward_host_buffers_equal_device_path(name, T):
     """moe_layer_forward_host (pinned host x in, y out, one C call) gives the y of
