@@ -27,7 +27,7 @@ class LayerIn(C.Structure):
     _fields_ = [("T", C.c_int32), ("score", C.c_int32), ("top_k", C.c_int32),
                 ("renorm", C.c_int32), ("act_g32", C.c_int32), ("rsf", C.c_float),
                 ("x", C.c_void_p), ("Wr", C.c_void_p), ("bias", C.c_void_p),
-                ("ex", C.POINTER(Experts)), ("sh", C.POINTER(Experts))]
+                ("ex", C.POINTER(Experts)), ("sh", C.POINTER(Experts)), ("top_p", C.c_float)]
 
 
 class LayerOut(C.Structure):
@@ -53,7 +53,7 @@ def lib():
             "orc_blob_layout": (i32, [i32, i32, i32, i32, i32, vp]),
             "orc_pack_blob": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
             "orc_router_logits": (None, [vp, vp, i32, i32, i32, vp]),
-            "orc_route": (i32, [vp, vp, i32, i32, i32, i32, i32, f32, vp, vp]),
+            "orc_route": (i32, [vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp]),
             "orc_permute": (i32, [vp, i32, i32, i32, vp, vp]),
             "orc_stage": (C.c_float, [vp, vp, i32, i32, vp, vp, i32, vp]),
             "orc_stage_f64": (C.c_double, [vp, vp, i32, i32, vp, vp, i32]),
@@ -189,13 +189,14 @@ def router_logits(x, Wr):
     return L
 
 
-def route(L, bias, score: str, k: int, renorm: bool, rsf: float):
+def route(L, bias, score: str, k: int, renorm: bool, rsf: float, top_p: float = 0.0):
     L = _c(L, np.float32)
     T, E = L.shape
     b = None if bias is None else _c(bias, np.float32)
     idx = np.empty((T, k), np.int32)
     w = np.empty((T, k), np.float64)
-    if lib().orc_route(_p(L), _p(b), T, E, SCORES[score], k, int(renorm), float(rsf), _p(idx), _p(w)):
+    if lib().orc_route(_p(L), _p(b), T, E, SCORES[score], k, int(renorm), float(rsf), float(top_p),
+                       _p(idx), _p(w)):
         raise ValueError("orc_route: bad k")
     return idx, w
 
@@ -207,7 +208,7 @@ def permute(idx, E: int):
     perm = np.empty(T * k, np.int32)
     if lib().orc_permute(_p(idx), T, k, E, _p(offsets), _p(perm)):
         raise ValueError("expert index out of range")
-    return offsets, perm
+    return offsets, perm[: offsets[E]]       # slots with expert -1 (dropped) are left out
 
 
 # ---------------------------------------------------------------- expert math
@@ -246,7 +247,7 @@ def expert_ffn(ex: QExperts, e: int, qx, sx, ag32: bool):
 
 def layer_forward(x, Wr, bias, ex: QExperts, sh: QExperts | None, score: str, k: int,
                   renorm: bool, rsf: float, act_g32: bool, union: bool = False,
-                  nthreads: int = 1, debug: bool = True):
+                  nthreads: int = 1, debug: bool = True, top_p: float = 0.0):
     """Whole layer. Returns dict with y (fp64 [T][H]) and, if debug, every intermediate."""
     x = _c(x, np.float32)
     Wr = _c(Wr, np.float32)
@@ -268,7 +269,7 @@ def layer_forward(x, Wr, bias, ex: QExperts, sh: QExperts | None, score: str, k:
     st = ex.struct()
     sst = sh.struct() if sh is not None else None
     lin = LayerIn(T, SCORES[score], k, int(renorm), int(act_g32), float(rsf), _p(x), _p(Wr), _p(b),
-                  C.pointer(st), C.pointer(sst) if sst is not None else None)
+                  C.pointer(st), C.pointer(sst) if sst is not None else None, float(top_p))
     lout = LayerOut(*[_p(o.get(n)) for n, _ in LayerOut._fields_])
     if union:
         rc = lib().orc_layer_forward_union(C.byref(lin), C.byref(lout))

@@ -43,7 +43,15 @@
  *   - SwiGLU: h = (g / (1 + cexp(-g))) * u;
  *   - cexp: own fp32 exp (Cody-Waite two-constant reduction by ln 2, degree-7
  *     Taylor polynomial in Horner form, exponent scaling), input clamped to
- *     [-87, 88].
+ *     [-87, 88];
+ *   - adaptive expert top-p (the GLM page's "--topp" knob, "adaptive expert
+ *     top-p", which it credits with 30-40% less expert reading): the mass of
+ *     slot j of a token's top-k list is v_j = cexp(L_j - L_0) (softmax; slot 0
+ *     holds the largest logit) or sigmoid(L_j); D = v_0 + ... + v_{k-1} and
+ *     C_m = v_0 + ... + v_{m-1} are fp32 sums in slot order; the kept count m is
+ *     the first m with C_m >= top_p * D (fp32 product). Dropped slots get
+ *     expert -1 and weight 0; with renormalisation the kept weights are
+ *     renormalised over the kept experts.
  */
 #include <math.h>
 #include <stdint.h>
@@ -273,9 +281,26 @@ static int by_key_desc(const void* a, const void* b) {
   return p->e < q->e ? -1 : (p->e > q->e ? 1 : 0);
 }
 
-/* score 0 = softmax, 1 = sigmoid noaux_tc. idx [T][k], w [T][k] (fp64). */
+/* Adaptive top-p cut of one token's top-k list (slot order): the number of slots kept. */
+static int topp_keep(const float* Lt, const keyed* ks, int score, int k, float top_p) {
+  float v[1024];
+  for (int j = 0; j < k; ++j)
+    v[j] = score == 0 ? orc_cexp(Lt[ks[j].e] - Lt[ks[0].e]) : orc_sigmoid(Lt[ks[j].e]);
+  float D = 0.0f;
+  for (int j = 0; j < k; ++j) D = D + v[j];
+  const float thr = top_p * D;
+  float c = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    c = c + v[j];
+    if (c >= thr) return j + 1;
+  }
+  return k;
+}
+
+/* score 0 = softmax, 1 = sigmoid noaux_tc. idx [T][k], w [T][k] (fp64). top_p in (0, 1):
+ * adaptive top-p (dropped slots: idx -1, w 0); other values: off. */
 int orc_route(const float* L, const float* bias, int T, int E, int score, int k, int renorm,
-              float rsf, int32_t* idx, double* w) {
+              float rsf, float top_p, int32_t* idx, double* w) {
   if (k <= 0 || k > E) return 1;
   keyed* ks = (keyed*)malloc(sizeof(keyed) * (size_t)E);
   for (int t = 0; t < T; ++t) {
@@ -286,19 +311,25 @@ int orc_route(const float* L, const float* bias, int T, int E, int score, int k,
       else ks[e].key = orc_sigmoid(Lt[e]) + (bias ? bias[e] : 0.0f);
     }
     qsort(ks, (size_t)E, sizeof(keyed), by_key_desc);
-    for (int j = 0; j < k; ++j) idx[(int64_t)t * k + j] = ks[j].e;
+    /* kept slots: all k, or the adaptive top-p prefix; the renormalised weights are taken
+       over the kept slots */
+    const int m = (top_p > 0.0f && top_p < 1.0f) ? topp_keep(Lt, ks, score, k, top_p) : k;
+    for (int j = 0; j < k; ++j) {
+      idx[(int64_t)t * k + j] = j < m ? ks[j].e : -1;
+      w[(int64_t)t * k + j] = 0.0;
+    }
     if (score == 0) {
       double M = -INFINITY;
       for (int e = 0; e < E; ++e) if ((double)Lt[e] > M) M = (double)Lt[e];
       double den = 0.0;
-      if (renorm) for (int j = 0; j < k; ++j) den += exp((double)Lt[ks[j].e] - M);
+      if (renorm) for (int j = 0; j < m; ++j) den += exp((double)Lt[ks[j].e] - M);
       else for (int e = 0; e < E; ++e) den += exp((double)Lt[e] - M);
-      for (int j = 0; j < k; ++j)
+      for (int j = 0; j < m; ++j)
         w[(int64_t)t * k + j] = exp((double)Lt[ks[j].e] - M) / den * (double)rsf;
     } else {
       double den = 0.0;
-      for (int j = 0; j < k; ++j) den += 1.0 / (1.0 + exp(-(double)Lt[ks[j].e]));
-      for (int j = 0; j < k; ++j) {
+      for (int j = 0; j < m; ++j) den += 1.0 / (1.0 + exp(-(double)Lt[ks[j].e]));
+      for (int j = 0; j < m; ++j) {
         double s = 1.0 / (1.0 + exp(-(double)Lt[ks[j].e]));
         w[(int64_t)t * k + j] = (renorm ? s / den : s) * (double)rsf;
       }
@@ -308,12 +339,14 @@ int orc_route(const float* L, const float* bias, int T, int E, int score, int k,
   return 0;
 }
 
-/* Batch-union grouping: offsets [E+1], perm [T*k] holds t*k+j sorted by (expert, t). */
+/* Batch-union grouping: offsets [E+1], perm [offsets[E]] holds t*k+j sorted by (expert, t).
+ * Slots with expert -1 (dropped by adaptive top-p) are left out. */
 int orc_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32_t* perm) {
   int32_t* fill = (int32_t*)calloc((size_t)E + 1, sizeof(int32_t));
   for (int e = 0; e <= E; ++e) offsets[e] = 0;
   for (int64_t p = 0; p < (int64_t)T * k; ++p) {
     int e = idx[p];
+    if (e == -1) continue;
     if (e < 0 || e >= E) { free(fill); return 1; }
     offsets[e + 1] += 1;
   }
@@ -322,7 +355,7 @@ int orc_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32
   for (int t = 0; t < T; ++t)
     for (int j = 0; j < k; ++j) {
       int e = idx[(int64_t)t * k + j];
-      perm[fill[e]++] = t * k + j;
+      if (e >= 0) perm[fill[e]++] = t * k + j;
     }
   free(fill);
   return 0;
@@ -417,6 +450,7 @@ typedef struct {
   const float* bias;     /* [E] or NULL */
   const orc_experts* ex;
   const orc_experts* sh; /* NULL = no shared expert */
+  float top_p;           /* adaptive top-p in (0, 1); other values: off */
 } orc_layer_in;
 
 typedef struct {
@@ -450,7 +484,7 @@ static int layer_common(const orc_layer_in* in, orc_layer_out* out, float** Lp, 
   int8_t* qx = out->qx ? out->qx : (int8_t*)malloc((size_t)T * H + 1);
   float* sx = out->sx ? out->sx : (float*)malloc(sizeof(float) * (size_t)T * sxn + 4);
   orc_router_logits(in->x, in->Wr, T, E, H, L);
-  if (orc_route(L, in->bias, T, E, in->score, k, in->renorm, in->rsf, idx, w)) return 1;
+  if (orc_route(L, in->bias, T, E, in->score, k, in->renorm, in->rsf, in->top_p, idx, w)) return 1;
   orc_quantize_rows(in->x, T, H, 127, in->act_g32, qx, sx);
   *Lp = L; *idxp = idx; *wp = w; *qxp = qx; *sxp = sx;
   return 0;
@@ -480,8 +514,10 @@ static void shared_and_combine(const orc_layer_in* in, orc_layer_out* out, int t
   const int H = in->ex->H, k = in->top_k;
   double* yt = out->y + (int64_t)t * H;
   for (int n = 0; n < H; ++n) yt[n] = 0.0;
-  for (int j = 0; j < k; ++j)
+  for (int j = 0; j < k; ++j) {
+    if (!ye_rows[j]) continue;           /* a slot dropped by adaptive top-p */
     for (int n = 0; n < H; ++n) yt[n] += w[(int64_t)t * k + j] * ye_rows[j][n];
+  }
   if (in->sh) {
     double* ys = (double*)malloc(sizeof(double) * (size_t)H);
     orc_expert_ffn(in->sh, 0, qxt, sxt, in->act_g32, ys, NULL, NULL, NULL, NULL, NULL);
@@ -505,6 +541,8 @@ int orc_layer_forward(const orc_layer_in* in, orc_layer_out* out, int nthreads) 
     for (int j = 0; j < k && j < 64; ++j) {
       int64_t row = (int64_t)t * k + j;
       double* yr = out->ye ? out->ye + row * H : ye + (int64_t)j * H;
+      rows[j] = NULL;
+      if (idx[row] < 0) continue;        /* dropped by adaptive top-p */
       pair_ffn(in, out, row, idx[row], qx + (int64_t)t * H, sx + (int64_t)t * sxn, yr);
       rows[j] = yr;
     }
@@ -536,7 +574,8 @@ int orc_layer_forward_union(const orc_layer_in* in, orc_layer_out* out) {
     }
   for (int t = 0; t < T; ++t) {
     const double* rows[64];
-    for (int j = 0; j < k; ++j) rows[j] = ye + ((int64_t)t * k + j) * H;
+    for (int j = 0; j < k; ++j)
+      rows[j] = idx[(int64_t)t * k + j] < 0 ? NULL : ye + ((int64_t)t * k + j) * H;
     shared_and_combine(in, out, t, qx + (int64_t)t * H, sx + (int64_t)t * sxn, w, rows);
   }
   if (!out->ye) free(ye);

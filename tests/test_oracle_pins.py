@@ -443,3 +443,122 @@ def test_shared_expert_adds_with_weight_one():
         ys = O.expert_ffn(sh, 0, with_sh["qx"][t], with_sh["sx"][t], True)["ye"]
         assert np.allclose(with_sh["y"][t], no_sh["y"][t] + ys, rtol=1e-14, atol=1e-18)
         assert np.allclose(with_sh["w"][t].sum(), 2.5)
+
+
+# ------------------------------------------------------- adaptive expert top-p
+# The GLM page's "--topp" knob ("adaptive expert top-p"): per token, keep the shortest prefix
+# of the sorted top-k list whose share of the list's mass reaches p.
+def _topp_masses(L_t, sel, score):
+    """fp64 masses of a token's top-k list (slot order), computed here from the logits."""
+    Lt = L_t.astype(np.float64)
+    return np.exp(Lt[sel] - Lt[sel[0]]) if score == "softmax" else 1.0 / (1.0 + np.exp(-Lt[sel]))
+
+
+@pytest.mark.parametrize("score,renorm", [("softmax", True), ("softmax", False), ("sigmoid", True)])
+@pytest.mark.parametrize("p", [0.3, 0.5, 0.7, 0.9])
+def test_topp_keeps_shortest_prefix_reaching_p(score, renorm, p):
+    r = rng(40 + int(100 * p))
+    T, E, k = 300, 64, 8
+    rsf = 2.5 if score == "sigmoid" else 1.0
+    L = r.normal(0, 1, (T, E)).astype(np.float32)
+    b = r.normal(0, 0.05, E).astype(np.float32) if score == "sigmoid" else None
+    idx0, w0 = O.route(L, b, score, k, renorm, rsf)
+    idx, w = O.route(L, b, score, k, renorm, rsf, top_p=p)
+    decided = 0
+    for t in range(T):
+        m = int((idx[t] >= 0).sum())
+        assert 1 <= m <= k
+        assert np.array_equal(idx[t, :m], idx0[t, :m]) and np.all(idx[t, m:] == -1)
+        assert np.all(w[t, m:] == 0.0)
+        v = _topp_masses(L[t], idx0[t], score)
+        share = np.cumsum(v) / v.sum()
+        want = int(np.argmax(share >= p)) + 1
+        # the cut is taken on fp32 sums: only a share within rounding of p may land either side
+        if all(abs(share[j] - p) > 1e-5 for j in range(k)):
+            assert m == want, (t, m, want)
+            decided += 1
+        if renorm:
+            assert np.allclose(w[t, :m], v[:m] / v[:m].sum() * rsf, rtol=1e-12, atol=0)
+            assert abs(w[t, :m].sum() - rsf) < 1e-12
+        else:
+            assert np.array_equal(w[t, :m], w0[t, :m])
+    assert decided > 0.9 * T
+
+
+@pytest.mark.parametrize("p", [0.0, 1.0, 1.5, -0.0])
+def test_topp_off_values_give_plain_topk(p):
+    r = rng(50)
+    L = r.normal(0, 1, (20, 32)).astype(np.float32)
+    for score in ("softmax", "sigmoid"):
+        a = O.route(L, None, score, 6, True, 1.0)
+        b = O.route(L, None, score, 6, True, 1.0, top_p=p)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("score", ["softmax", "sigmoid"])
+def test_topp_equal_logits_keep_ceil_pk(score):
+    """All logits equal: every slot has the same mass (exactly 1, or 1/2 for the sigmoid), so
+    the kept count is ceil(p k) -- p k computed as the fp32 product, exact for k = 8."""
+    L = np.zeros((1, 16), np.float32)
+    for p in (0.05, 0.125, 0.2, 0.3, 0.5, 0.51, 0.75, 0.99):
+        idx, w = O.route(L, None, score, 8, True, 1.0, top_p=p)
+        m = math.ceil(float(np.float32(p)) * 8)
+        assert idx[0].tolist() == list(range(m)) + [-1] * (8 - m), p
+        assert np.allclose(w[0, :m], 1.0 / m, rtol=1e-15)
+
+
+def test_topp_kept_count_grows_with_p():
+    r = rng(51)
+    L = r.normal(0, 1, (100, 64)).astype(np.float32)
+    prev = np.zeros(100, np.int64)
+    for p in np.linspace(0.05, 0.95, 19):
+        idx, _ = O.route(L, None, "softmax", 8, True, 1.0, top_p=float(p))
+        m = (idx >= 0).sum(1)
+        assert np.all(m >= prev)
+        prev = m
+    assert prev.min() >= 1 and prev.max() <= 8
+
+
+def test_topp_permute_leaves_out_dropped_slots():
+    idx = np.array([[3, 1, -1], [1, -1, -1], [0, 3, 2]], np.int32)
+    offsets, perm = O.permute(idx, 4)
+    assert offsets.tolist() == [0, 1, 3, 4, 6]
+    assert perm.tolist() == [6, 1, 3, 8, 0, 7]
+    with pytest.raises(ValueError):
+        O.permute(np.array([[0, -2]], np.int32), 4)
+
+
+@pytest.mark.parametrize("name,p", [("olmoe_int8", 0.6), ("glm_int4", 0.7), ("e512_int4", 0.5)])
+def test_topp_layer_equals_kept_expert_composition(name, p):
+    """The layer with top-p equals a composition built here from single-expert FFN calls: each
+    token's kept experts weighted by the renormalised (or plain) routing weights, plus the
+    shared expert; the batch-union path gives the same bits."""
+    cfg = S.CONFIGS[name].with_(H=256, I=128, E=16, top_k=4)
+    if cfg.shared_I:
+        cfg = cfg.with_(shared_I=128)
+    case = S.Case.make(cfg, 7)
+    x, Wr = case.x(), case.router_w()
+    wb, g32 = (8 if cfg.wtype == "int8" else 4), cfg.wscale == "g32_f16"
+    ex = O.QExperts.quantize(np.stack([case.gate_up(e) for e in range(cfg.E)]),
+                             np.stack([case.down(e) for e in range(cfg.E)]), wb, g32)
+    sh = None
+    if cfg.shared_I:
+        sh = O.QExperts.quantize(case.shared_gate_up()[None], case.shared_down()[None], wb, g32)
+    ag32 = cfg.act == "g32_f16"
+    args = (x, Wr, case.bias(), ex, sh, cfg.score, cfg.top_k, cfg.renormalize, cfg.rsf, ag32)
+    a = O.layer_forward(*args, top_p=p)
+    u = O.layer_forward(*args, union=True, top_p=p)
+    assert np.array_equal(a["y"], u["y"]) and np.array_equal(a["idx"], u["idx"])
+    assert u["offsets"][-1] == int((a["idx"] >= 0).sum()) < 7 * cfg.top_k
+    L = O.router_logits(x, Wr)
+    idx, w = O.route(L, case.bias(), cfg.score, cfg.top_k, cfg.renormalize, cfg.rsf, top_p=p)
+    assert np.array_equal(idx, a["idx"])
+    qx, sx = O.quantize_act(x, ag32)
+    for t in range(7):
+        want = np.zeros(cfg.H)
+        for j in range(cfg.top_k):
+            if idx[t, j] >= 0:
+                want += w[t, j] * O.expert_ffn(ex, int(idx[t, j]), qx[t], sx[t], ag32)["ye"]
+        if sh is not None:
+            want += O.expert_ffn(sh, 0, qx[t], sx[t], ag32)["ye"]
+        assert np.allclose(a["y"][t], want, rtol=1e-12, atol=1e-15)
