@@ -48,9 +48,10 @@ def parse_workload(spec: str):
     return cfg, T
 
 
-def workload_desc(cfg, T):
+def workload_desc(cfg, T, top_p=0.0):
     return (f"{cfg.name} T={T}: H{cfg.H} E{cfg.E} I{cfg.I} top-{cfg.top_k} {cfg.score}"
-            f"{' renorm' if cfg.renormalize else ''}{f' rsf {cfg.rsf}' if cfg.rsf != 1 else ''}, "
+            f"{' renorm' if cfg.renormalize else ''}{f' rsf {cfg.rsf}' if cfg.rsf != 1 else ''}"
+            f"{f' adaptive top-p {top_p:g}' if 0 < top_p < 1 else ''}, "
             f"{cfg.wtype} {cfg.wscale} experts, {cfg.act} activations"
             f"{f', shared I{cfg.shared_I}' if cfg.shared_I else ''}")
 
@@ -104,8 +105,10 @@ def layer_bytes(cfg, T, n_active):
     return b
 
 
-def layer_int_ops(cfg, T):
-    return 2 * (T * cfg.top_k * 3 * cfg.H * cfg.I + T * 3 * cfg.H * cfg.shared_I)
+def layer_int_ops(cfg, T, pairs=None):
+    """pairs: routed (token, expert) pairs computed (T * k, or fewer with adaptive top-p)."""
+    pairs = T * cfg.top_k if pairs is None else pairs
+    return 2 * (pairs * 3 * cfg.H * cfg.I + T * 3 * cfg.H * cfg.shared_I)
 
 
 class ClockSampler:
@@ -172,7 +175,7 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------- oracle
-def oracle_sampler(cfg, T, seed_base=7_000_000):
+def oracle_sampler(cfg, T, top_p=0.0, seed_base=7_000_000):
     """Prepare the oracle for timing on host cores: experts of a token sample, pre-quantized.
     Returns (run_units(n_units) -> tokens processed, unit description, cores)."""
     import oracle as O
@@ -187,7 +190,7 @@ def oracle_sampler(cfg, T, seed_base=7_000_000):
     x = case.x()
     Wr, bias = case.router_w(), case.bias()
     L = O.router_logits(x, Wr)
-    idx, _ = O.route(L, bias, cfg.score, cfg.top_k, cfg.renormalize, cfg.rsf)
+    idx, _ = O.route(L, bias, cfg.score, cfg.top_k, cfg.renormalize, cfg.rsf, top_p=top_p)
     experts = {}
     shared = None
     if cfg.shared_I:
@@ -201,7 +204,7 @@ def oracle_sampler(cfg, T, seed_base=7_000_000):
         return experts[e]
 
     # pre-quantize the experts of the first tokens (input preparation, not timed)
-    for e in sorted(set(int(v) for v in idx[:16].reshape(-1))):
+    for e in sorted(set(int(v) for v in idx[:16].reshape(-1)) - {-1}):
         ensure(e)
     cursor = [0]
 
@@ -216,7 +219,7 @@ def oracle_sampler(cfg, T, seed_base=7_000_000):
             cursor[0] += 1
         toks = sorted(set(t for t, _ in units))
         Lt = O.router_logits(x[toks], Wr)
-        it, wt = O.route(Lt, bias, cfg.score, cfg.top_k, cfg.renormalize, cfg.rsf)
+        it, wt = O.route(Lt, bias, cfg.score, cfg.top_k, cfg.renormalize, cfg.rsf, top_p=top_p)
         qx, sx = O.quantize_act(x[toks], ag32)
         pos = {t: i for i, t in enumerate(toks)}
 
@@ -224,6 +227,8 @@ def oracle_sampler(cfg, T, seed_base=7_000_000):
             t, u = tu
             i = pos[t]
             if u < cfg.top_k:
+                if it[i, u] < 0:                 # slot dropped by adaptive top-p
+                    return i, 0.0
                 r = O.expert_ffn(experts[int(it[i, u])], 0, qx[i], sx[i], ag32)
                 return i, wt[i, u] * r["ye"]
             r = O.expert_ffn(shared, 0, qx[i], sx[i], ag32)
@@ -240,8 +245,8 @@ def oracle_sampler(cfg, T, seed_base=7_000_000):
     return run_units, desc, cores
 
 
-def time_oracle(cfg, T, budget_s=45.0):
-    run_units, desc, cores = oracle_sampler(cfg, T)
+def time_oracle(cfg, T, top_p=0.0, budget_s=45.0):
+    run_units, desc, cores = oracle_sampler(cfg, T, top_p)
     per_tok = cfg.top_k + (1 if cfg.shared_I else 0)
     t0 = time.perf_counter()
     run_units(per_tok)
@@ -262,7 +267,7 @@ def reference_arm(args, cfg, T):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    run_units, desc, cores = oracle_sampler(cfg, T)
+    run_units, desc, cores = oracle_sampler(cfg, T, args.top_p)
     per_tok = cfg.top_k + (1 if cfg.shared_I else 0)
     t0 = time.perf_counter()
     run_units(1)
@@ -282,7 +287,7 @@ def reference_arm(args, cfg, T):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(cfg, T), "T": T,
+        "config": {"workload": workload_desc(cfg, T, args.top_p), "T": T,
                    "step": f"{units} (token, expert) units per step = {units / per_tok:g} tokens"},
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
                          "sample": f"{args.steps} steps of {units} {desc}"},
@@ -431,8 +436,8 @@ def gpu_arm(args, cfg, T):
     R = args.replicas
     rep_seeds, x_seeds = rank_seeds(rank, R, max(1, min(args.steps, args.period)))
     rcfg = M.RouteCfg(score=cfg.score, top_k=cfg.top_k, renormalize=cfg.renormalize,
-                      routed_scaling_factor=cfg.rsf, act=cfg.act)
-    layers, n_active_of = [], []
+                      routed_scaling_factor=cfg.rsf, act=cfg.act, top_p=args.top_p)
+    layers, n_active_of, kept_of = [], [], []
     for r in range(R):
         case = S.Case.make(cfg, T, replica=rep_seeds[r])
         gu = torch.empty((cfg.E, 2 * cfg.I, cfg.H), dtype=torch.float32, device=dev)
@@ -465,7 +470,8 @@ def gpu_arm(args, cfg, T):
     for s in range(G):
         lay = layers[s % R]
         idx, _ = M.moe_route_topk(M.moe_router_logits(xs[s], lay.router_w), lay.router_bias, rcfg)
-        n_active_of.append(int(torch.unique(idx).numel()))
+        n_active_of.append(int(torch.unique(idx[idx >= 0]).numel()))   # -1: dropped by top-p
+        kept_of.append(int((idx >= 0).sum()))
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
@@ -597,7 +603,8 @@ def gpu_arm(args, cfg, T):
     step_s = ms_max / 1e3 / args.steps
     layer = {"bytes_per_step": int(lb), "gbs": round(lb / step_s / 1e9, 1),
              "frac_hbm": round(lb / step_s / 1e9 / peaks["hbm_gbs"], 4),
-             "int8_tops": round(layer_int_ops(cfg, T) / step_s / 1e12, 2),
+             "int8_tops": round(layer_int_ops(cfg, T, float(np.mean(kept_of))) / step_s / 1e12, 2),
+             "routed_pairs_per_step": round(float(np.mean(kept_of)), 2),
              "distinct_experts_per_step": round(n_act, 2),
              "stage_us": {k: (round(v, 3) if v is not None else None) for k, v in stage_us.items()}}
 
@@ -635,7 +642,7 @@ def gpu_arm(args, cfg, T):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = time_oracle(cfg, T)
+        cpu = time_oracle(cfg, T, args.top_p)
 
     launches = layers[0].kernels * args.steps
     line = {
@@ -643,7 +650,7 @@ def gpu_arm(args, cfg, T):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
-        "config": {"workload": workload_desc(cfg, T), "T": T, "replicas": R,
+        "config": {"workload": workload_desc(cfg, T, args.top_p), "T": T, "replicas": R,
                    "l2": f"inputs larger than L2: {R} layer replicas rotate "
                          f"({R * layers[0].experts.nbytes / 1e9:.2f} GB of expert blobs)",
                    "graph": f"CUDA graphs of {G} steps; the last {Ge} timed steps carry per-stage event nodes", "accumulate": "int32 dots, fp32 scales",
@@ -699,6 +706,9 @@ def main(argv=None):
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (4k tokens) measurement")
     ap.add_argument("--prefill-workload", default=PREFILL_WORKLOAD)
     ap.add_argument("--prefill-steps", type=int, default=20)
+    ap.add_argument("--top-p", type=float, default=0.0,
+                    help="adaptive expert top-p of the main workload (0 = off; the prefill half "
+                         "is measured without it)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -65,7 +65,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -138,6 +138,16 @@ typedef struct {
   float routed_scaling_factor;  /* multiplies every routing weight (1.0 for plain softmax) */
   int32_t act;                  /* MOE_ACT_* (applies to x and to h) */
   uint32_t flags;               /* MOE_FLAG_* */
+  float top_p;                  /* adaptive expert top-p (the GLM-5.2 colibri page's "--topp"):
+                                   0 or >= 1 = off (every token keeps its k experts). In (0, 1):
+                                   per token, slot j of the top-k list (descending key) has mass
+                                   v_j = exp(L_j - L_0) (softmax) or sigmoid(L_j); D = v_0 + ... +
+                                   v_{k-1} and C_m = v_0 + ... + v_{m-1} are fp32 sums in slot
+                                   order, and the first m slots are kept for the first m with
+                                   C_m >= top_p * D. Dropped slots get idx -1 and weight 0 and
+                                   their experts are not read for that token; with renormalize
+                                   the kept weights are renormalized over the kept experts.
+                                   Must be finite and >= 0 (else MOE_ERR_INVALID_ARG). */
 } moe_route_cfg;
 
 /* Version of this ABI (MOE_ABI_VERSION). */

@@ -277,4 +277,6 @@ def layer_forward(x, Wr, bias, ex: QExperts, sh: QExperts | None, score: str, k:
         rc = lib().orc_layer_forward(C.byref(lin), C.byref(lout), int(nthreads))
     if rc:
         raise ValueError("oracle layer forward failed")
+    if "perm" in o:
+        o["perm"] = o["perm"][: o["offsets"][E]]   # slots dropped by adaptive top-p are left out
     return o

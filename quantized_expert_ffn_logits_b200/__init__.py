@@ -43,7 +43,8 @@ class moe_expert_blob(C.Structure):
 
 class moe_route_cfg(C.Structure):
     _fields_ = [("score", C.c_int32), ("top_k", C.c_int32), ("renormalize", C.c_int32),
-                ("routed_scaling_factor", C.c_float), ("act", C.c_int32), ("flags", C.c_uint32)]
+                ("routed_scaling_factor", C.c_float), ("act", C.c_int32), ("flags", C.c_uint32),
+                ("top_p", C.c_float)]
 
 
 class moe_debug_views(C.Structure):
@@ -91,6 +92,10 @@ for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
     _fn.argtypes = _args
+ABI_VERSION = 2          # the struct layouts above (moe_route_cfg with top_p)
+if _lib.moe_abi_version() != ABI_VERSION:
+    raise ImportError(f"{LIB_PATH}: ABI version {_lib.moe_abi_version()}, this binding needs "
+                      f"{ABI_VERSION}: rebuild the library")
 
 
 class MoeError(RuntimeError):
@@ -136,10 +141,12 @@ class RouteCfg:
     routed_scaling_factor: float = 1.0
     act: str = "g32_f16"
     flags: int = 0
+    top_p: float = 0.0      # adaptive expert top-p; 0 (or >= 1) = off
 
     def struct(self) -> moe_route_cfg:
         return moe_route_cfg(SCORES[self.score], self.top_k, int(self.renormalize),
-                             float(self.routed_scaling_factor), ACTS[self.act], self.flags)
+                             float(self.routed_scaling_factor), ACTS[self.act], self.flags,
+                             float(self.top_p))
 
 
 class ExpertBlob:

@@ -1,5 +1,6 @@
 // api.cu -- the C ABI (include/moe_b200.h): argument checks, workspace layout and
 // the launch sequence of the layer forward.
+#include <cmath>
 #include <cstdint>
 #include <cstdio>
 #include <algorithm>
@@ -72,8 +73,12 @@ moe_status check_cfg(const moe_route_cfg* c, int32_t E) {
   if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID_NOAUX_TC) return MOE_ERR_INVALID_ARG;
   if (c->act != MOE_ACT_TOKEN_F32 && c->act != MOE_ACT_G32_F16) return MOE_ERR_INVALID_ARG;
   if (c->top_k < 1 || c->top_k > 32 || c->top_k > E) return MOE_ERR_UNSUPPORTED;
+  if (!(c->top_p >= 0.0f) || !std::isfinite(c->top_p)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
+
+// The adaptive top-p threshold the kernels take: 0 when off.
+float topp_of(const moe_route_cfg* c) { return (c->top_p > 0.0f && c->top_p < 1.0f) ? c->top_p : 0.0f; }
 
 // Workspace of one layer forward: every region starts at a multiple of 256 bytes.
 struct Layout {
@@ -287,8 +292,8 @@ moe_status moe_route_topk(const float* logits, const float* bias, int32_t T, int
   if (T == 0) return MOE_OK;
   if (!logits || !idx || !w) return MOE_ERR_INVALID_ARG;
   moe::launch_topk(logits, cfg->score == MOE_SCORE_SIGMOID_NOAUX_TC ? bias : nullptr, T, E,
-                   cfg->top_k, cfg->score, cfg->renormalize != 0, cfg->routed_scaling_factor, idx,
-                   w, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+                   cfg->top_k, cfg->score, cfg->renormalize != 0, cfg->routed_scaling_factor,
+                   topp_of(cfg), idx, w, nullptr, nullptr, static_cast<cudaStream_t>(stream));
   return launch_status();
 }
 
@@ -459,6 +464,7 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     r.renorm = cfg->renormalize != 0;
     r.ag32 = ag32;
     r.rsf = cfg->routed_scaling_factor;
+    r.top_p = topp_of(cfg);
     r.qx = static_cast<int8_t*>(at(L.qx));
     r.sx = at(L.sx);
     r.y = y;
@@ -488,7 +494,7 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     // 3. top-k selection and weights, batch-union grouping
     mk.begin(MOE_STAGE_TOPK);
     moe::launch_topk(logits, bias, T, E, k, cfg->score, cfg->renormalize != 0,
-                     cfg->routed_scaling_factor, idx, wts, nullptr, status, st);
+                     cfg->routed_scaling_factor, topp_of(cfg), idx, wts, nullptr, status, st);
     mk.end(MOE_STAGE_TOPK);
     mk.begin(MOE_STAGE_GROUP);
     moe::launch_permute(idx, T, k, E, g, static_cast<uint32_t*>(at(L.masks)),

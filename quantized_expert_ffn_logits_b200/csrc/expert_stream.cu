@@ -31,6 +31,7 @@
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tma.cuh"
+#include "topk.cuh"
 
 namespace moe {
 
@@ -47,7 +48,7 @@ constexpr int kSmemMax = 227 * 1024;
 // of K codes, then (g32 activations) tm rows of G fp16 scales.
 // Single-token routing scratch (RingPlan::route): se, swt, sj, sidx, sw, own [32] each,
 // then two flag words and the y-zero barrier target (8 bytes).
-constexpr int kRouteBytes = 6 * 32 * 4 + 16;
+constexpr int kRouteBytes = 6 * 32 * 4 + 32;
 
 struct RingPlan {
   int ring, sring, bars, abuf, abytes, ascale, xsum, sxf, idot, ubuf, hq, info, route, total;
@@ -247,6 +248,7 @@ struct RouteSmem {
   float* own;     // [32] logits of this CTA's experts (cluster exchange)
   volatile int* flag;
   volatile unsigned long long* ytarget;   // y-zero barrier target (cluster exchange)
+  volatile int* nk;                       // slots kept: k, or the adaptive top-p prefix
 };
 
 // Bound of the grid-barrier wait: 2^22 polls (each an L2 round trip: seconds in all).
@@ -329,6 +331,7 @@ __device__ __forceinline__ bool stage_router_rows(const RouteArgs& r, bool cl, u
 // Every thread of the CTA. False when a wait gave up (status recorded; with the cluster
 // exchange the CTA has still taken both cluster-barrier arrivals, and must wait on the
 // second before it exits). rows_bar: the router rows were staged and complete on it.
+template <bool TOPP>
 __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Ring& R, const RouteSmem& S,
                                 uint64_t* rows_bar, bool cl) {
   volatile int* flag = S.flag;
@@ -480,6 +483,7 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
     if (!good) return false;
   }
   if (tid < 32) S.sidx[tid] = -1;
+  if (TOPP && tid == 0) *S.nk = k;
   // 5. top-k (every CTA, same result): keys ranked by (keys larger, or equal with a lower
   //    expert index): descending, ties to the lower expert. The logits also go to activation
   //    buffer 1 (idle in this mode): the routing weights are formed there after the producer
@@ -544,31 +548,53 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
   }
   fence_async_smem();                       // this thread's ring accesses precede the bulk copies
   __syncthreads();
-  // 6. the selection in ascending expert order (all the producer needs)
+  // 5b. adaptive top-p: the kept prefix of the list (topk.cuh's rule; every CTA, same result)
+  if constexpr (TOPP) {
+    if (warp == 0) {
+      const bool on = lane < k;
+      const int ee = on ? S.sidx[lane] : 0;
+      const float myl = (ee >= 0 && ee < E) ? slog[ee] : 0.0f;
+      float v;
+      if (r.score == 0) {
+        const float lmax = __shfl_sync(0xffffffffu, myl, 0);
+        v = on ? cexp(myl - lmax) : 0.0f;
+      } else {
+        v = on ? csigmoid(myl) : 0.0f;
+      }
+      float cm;
+      const int m = topp_keep(v, k, r.top_p, cm);
+      if (lane == 0) *S.nk = m;
+    }
+    __syncthreads();
+  }
+  // 6. the kept selection in ascending expert order (all the producer needs)
+  const int nk = TOPP ? *S.nk : k;
   if (tid < k) {
     const int ee = S.sidx[tid];
-    int pos = 0;
-    for (int j = 0; j < k; ++j) pos += S.sidx[j] < ee;
-    S.se[pos] = ee;
-    S.sj[pos] = tid;
-    if (cta0) {
-      r.idx[tid] = ee;
-      r.g.act_expert[pos] = ee;
-      r.g.act_begin[pos] = pos;
-      r.g.perm[pos] = tid;
-      if (r.g.act_rows) r.g.act_rows[pos * 8] = 0;
+    if (tid < nk) {
+      int pos = 0;
+      for (int j = 0; j < nk; ++j) pos += S.sidx[j] < ee;
+      S.se[pos] = ee;
+      S.sj[pos] = tid;
+      if (cta0) {
+        r.g.act_expert[pos] = ee;
+        r.g.act_begin[pos] = pos;
+        r.g.perm[pos] = tid;
+        if (r.g.act_rows) r.g.act_rows[pos * 8] = 0;
+      }
     }
+    if (cta0) r.idx[tid] = tid < nk ? ee : -1;
   }
   if (cta0) {
     for (int x = tid; x < E; x += kNT) {
       int cnt = 0;
-      for (int j = 0; j < k; ++j) cnt += S.sidx[j] < x;
+      for (int j = 0; j < nk; ++j) cnt += S.sidx[j] < x;
       r.g.offsets[x] = cnt;
     }
     if (tid == 0) {
-      r.g.offsets[E] = k;
-      *r.g.n_active = k;
-      r.g.act_begin[k] = k;
+      r.g.offsets[E] = nk;
+      *r.g.n_active = nk;
+      r.g.act_begin[nk] = nk;
     }
   }
   __syncthreads();
@@ -579,6 +605,7 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
 // from the logits kept in activation buffer 1 -- softmax over the selected (renormalized) or
 // over all E, or sigmoid scores (normalized over the selected), times the routed scaling
 // factor (as in topk.cuh) -- into S.sw (selection order) and S.swt (ascending order).
+template <bool TOPP>
 __device__ __forceinline__ void route_weights(const RouteArgs& r, const RingPlan& P, const Ring& R,
                                               const RouteSmem& S) {
   const float* slogk = reinterpret_cast<const float*>(R.abuf + P.abytes);
@@ -586,40 +613,48 @@ __device__ __forceinline__ void route_weights(const RouteArgs& r, const RingPlan
   const bool on = lane < k;
   const int my_e = on ? S.sidx[lane] : 0;
   const float myl = (my_e >= 0 && my_e < E) ? slogk[my_e] : 0.0f;
-  float wv;
+  float v, den;                             // slot mass, weight denominator
   if (r.score == 0) {
     const float lmax = __shfl_sync(0xffffffffu, myl, 0);
-    const float ex = on ? cexp(myl - lmax) : 0.0f;
-    float den;
+    v = on ? cexp(myl - lmax) : 0.0f;
     if (r.renorm) {
-      den = warp_sum(ex);
+      den = warp_sum(v);
     } else {
       float sacc = 0.0f;
       for (int x = lane; x < E; x += 32) sacc += cexp(slogk[x] - lmax);
       den = warp_sum(sacc);
     }
-    wv = ex / den * r.rsf;
   } else {
-    const float sg = on ? csigmoid(myl) : 0.0f;
-    const float den = r.renorm ? warp_sum(sg) : 1.0f;
-    wv = sg / den * r.rsf;
+    v = on ? csigmoid(myl) : 0.0f;
+    den = r.renorm ? warp_sum(v) : 1.0f;
   }
-  if (on) {
+  float wv = v / den * r.rsf;
+  const int nk = TOPP ? *S.nk : k;          // adaptive top-p: the kept prefix (route_one_token)
+  if (TOPP && r.renorm) {
+    float cm;
+    topp_keep(v, k, r.top_p, cm);
+    wv = v / cm * r.rsf;
+  }
+  if (lane < nk) {
     int pos = 0;
-    for (int j = 0; j < k; ++j) pos += S.sidx[j] < my_e;
+    for (int j = 0; j < nk; ++j) pos += S.sidx[j] < my_e;
     S.sw[lane] = wv;
     S.swt[pos] = wv;
-    if (blockIdx.x == 0) r.w[lane] = wv;
   }
+  if (on && blockIdx.x == 0) r.w[lane] = lane < nk ? wv : 0.0f;
   __syncwarp();
 }
 
 // Work unit u of a MODE 3 grid: routed units (the token's k experts, ascending) first, then
 // the shared expert's. Slot of the routed pair = its active-expert index.
-__device__ __forceinline__ bool unit_of_token(const RingArgs& A, const RouteSmem& S, int u, Unit& U, bool report) {
+// nk (TOPP): the token's kept slots, the adaptive top-p prefix; units of dropped slots are none.
+template <bool TOPP>
+__device__ __forceinline__ bool unit_of_token(const RingArgs& A, const RouteSmem& S, int nk, int u, Unit& U,
+                                              bool report) {
   if (u < A.routed) {
     U.shd = false;
     U.ai = u / A.per;
+    if (TOPP && U.ai < A.r.k && U.ai >= nk) return false;   // a slot dropped by adaptive top-p
     U.sub = u - U.ai * A.per;
     U.e = S.se[U.ai];
     U.s0 = U.ai;
@@ -649,7 +684,7 @@ __device__ __forceinline__ bool unit_of_token(const RingArgs& A, const RouteSmem
 // with the pass's activation rows right after the first chunk. Down pass: the unit's slab
 // (all H rows x its 64 columns) in chunks of whole 128-row blocks, with their scales
 // (fp16 [block][2][128] or fp32 per row).
-template <int WBITS, bool WG32, bool AG32, int MODE>
+template <int WBITS, bool WG32, bool AG32, int MODE, bool TOPP>
 __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& R, const RouteSmem& S) {
   constexpr int PPG = WBITS == 8 ? 2 : 1;
   constexpr int PPU = WBITS == 8 ? 4 : 2;   // pieces of a row's 64-column down slice
@@ -671,9 +706,10 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
     ++c;
     return true;
   };
+  const int nk = (MODE == 3 && TOPP) ? *S.nk : 0;
   for (int u = blockIdx.x; u < A.units && ok; u += gridDim.x) {
     Unit U;
-    if (MODE == 3 ? !unit_of_token(A, S, u, U, false)
+    if (MODE == 3 ? !unit_of_token<TOPP>(A, S, nk, u, U, false)
                   : !unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, false,
                              A.mma_min))
       continue;
@@ -1007,7 +1043,7 @@ __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& 
 // up stage values meet in shared memory and warps 0 and 1 apply SwiGLU and quantize h per
 // group of 32 -- one warp per group), then the down pass over the unit's slab with the
 // pass's h codes from shared memory (MODE 2) or from the workspace (MODE 1).
-template <int WBITS, bool WG32, bool AG32, int MODE, int TM>
+template <int WBITS, bool WG32, bool AG32, int MODE, int TM, bool TOPP>
 __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ RingArgs A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_align1024(smem_raw);
@@ -1057,6 +1093,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   S.flag = reinterpret_cast<volatile int*>(S.se + 192);
   volatile int* rows_flag = S.se + 193;
   S.ytarget = reinterpret_cast<volatile unsigned long long*>(S.se + 194);
+  S.nk = S.se + 196;
   __syncthreads();
   bool rows = false;
   if (MODE == 3) {
@@ -1066,7 +1103,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   if (MODE == 3) {
     // one token: routing first. Its grid barrier also means every CTA of this grid is
     // resident before any CTA lets the next kernel launch (and take SMs).
-    if (!route_one_token(A.r, P, R, S, rows ? &R.afull[0] : nullptr, A.cluster != 0)) {
+    if (!route_one_token<TOPP>(A.r, P, R, S, rows ? &R.afull[0] : nullptr, A.cluster != 0)) {
       if (A.cluster) cluster_wait();
       return;
     }
@@ -1076,7 +1113,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   if (!(MODE == 3 && A.cluster)) pdl_trigger();
 
   if (warp == kCW) {
-    if (lane == 0) ring_producer<WBITS, WG32, AG32, MODE>(A, P, R, S);
+    if (lane == 0) ring_producer<WBITS, WG32, AG32, MODE, TOPP>(A, P, R, S);
     if (MODE == 3 && A.cluster) {
       __syncwarp();
       cluster_wait();                      // peers are done reading this CTA's logits
@@ -1092,16 +1129,17 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   if (MODE == 3) {
     // off the path to the first weight copy: the routing weights (read only by this warp's
     // ctid 0) and, int4 weights, the token's de-interleaved codes and group sums
-    if (warp == 0) route_weights(A.r, P, R, S);
+    if (warp == 0) route_weights<TOPP>(A.r, P, R, S);
     if (WBITS == 4) {
       act_deinterleave(R.abuf, A.kmax / 8, ctid, 32 * kCW);
       named_bar(1, 32 * kCW);
       act_group_sums(R.abuf, R.xsum, 1, A.kmax, ctid, 32 * kCW);
     }
   }
+  const int nk = (MODE == 3 && TOPP) ? *S.nk : 0;
   for (int u = blockIdx.x; u < A.units; u += gridDim.x) {
     Unit U;
-    if (MODE == 3 ? !unit_of_token(A, S, u, U, ctid == 0)
+    if (MODE == 3 ? !unit_of_token<TOPP>(A, S, nk, u, U, ctid == 0)
                   : !unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, ctid == 0,
                              A.mma_min))
       continue;
@@ -1277,12 +1315,12 @@ int sm_count() {
 // to one CTA per SM: the grid barrier needs all of them resident at once).
 int decode_grid(int units, int E) { return std::min(sm_count(), std::max(units, E)); }
 
-template <int WBITS, bool WG32, bool AG32, int MODE, int TM>
+template <int WBITS, bool WG32, bool AG32, int MODE, int TM, bool TOPP = false>
 cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
   const RingPlan P = ring_plan(A.kmax, A.tm);
   static int attr_bytes = 0;
   if (P.total > attr_bytes) {
-    const cudaError_t e = cudaFuncSetAttribute(k_expert_ring<WBITS, WG32, AG32, MODE, TM>,
+    const cudaError_t e = cudaFuncSetAttribute(k_expert_ring<WBITS, WG32, AG32, MODE, TM, TOPP>,
                                                cudaFuncAttributeMaxDynamicSharedMemorySize, P.total);
     if (e != cudaSuccess) return e;
     attr_bytes = P.total;
@@ -1292,7 +1330,7 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
     // router rows fits its staging area and every cluster of the grid can be resident at
     // once (the y-zero barrier waits on all CTAs) with no fewer CTAs than the grid exchange
     // would use; else every CTA computes some logits and a grid barrier follows
-    auto kern = k_expert_ring<WBITS, WG32, AG32, MODE, TM>;
+    auto kern = k_expert_ring<WBITS, WG32, AG32, MODE, TM, TOPP>;
     static int max_clusters[2] = {-1, -1}, max_clusters_smem = -1;
     if (max_clusters_smem != P.total) {
       (void)cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -1350,7 +1388,8 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
   } else {
     const int grid = std::min(A.units, sm_count());
     if (grid <= 0) return cudaSuccess;
-    return launch_pdl(k_expert_ring<WBITS, WG32, AG32, MODE, TM>, dim3(grid), dim3(kNT), (size_t)P.total, st, A);
+    return launch_pdl(k_expert_ring<WBITS, WG32, AG32, MODE, TM, TOPP>, dim3(grid), dim3(kNT), (size_t)P.total, st,
+                      A);
   }
 }
 
@@ -1369,9 +1408,11 @@ cudaError_t launch_mode(int mode, const RingArgs& A, cudaStream_t st) {
                    : launch_mode_tm<WBITS, WG32, AG32, kTMP>(mode, A, st);
 }
 
+// Adaptive top-p gets its own instantiation, so the plain single-token kernel carries none of it.
 template <int WBITS, bool WG32>
 cudaError_t launch_decode_t(const RingArgs& A, cudaStream_t st) {
-  return launch_ring_t<WBITS, WG32, true, 3, 1>(A, st);
+  return A.r.top_p > 0.0f ? launch_ring_t<WBITS, WG32, true, 3, 1, true>(A, st)
+                          : launch_ring_t<WBITS, WG32, true, 3, 1, false>(A, st);
 }
 
 }  // namespace

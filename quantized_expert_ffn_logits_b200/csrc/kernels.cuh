@@ -31,9 +31,11 @@ struct Grouping {            // batch-union grouping outputs (all device pointer
   int32_t* act_rows;         // [E][8] token of each active expert's first 8 slots (or null)
 };
 
+// top_p: adaptive expert top-p threshold in (0, 1), 0 = off (dropped slots: idx -1, w 0).
 void launch_topk(const float* logits, const float* bias, int T, int E, int k, int score,
-                 int renorm, float rsf, int32_t* idx, float* w, const Grouping* single_token,
+                 int renorm, float rsf, float top_p, int32_t* idx, float* w, const Grouping* single_token,
                  int* status, cudaStream_t st);
+// Pairs with expert -1 (dropped by adaptive top-p) are left out of the grouping.
 // masks/base: scratch [ceil(T/32)][E] each.
 // reset_status: clear the status word first (stand-alone use).
 void launch_permute(const int32_t* idx, int T, int k, int E, const Grouping& g, uint32_t* masks,
@@ -124,6 +126,7 @@ struct RouteArgs {
   const float* bias;      // sigmoid mode only, may be null
   int T, E, H, k, score, renorm, ag32;
   float rsf;
+  float top_p;            // adaptive expert top-p in (0, 1); 0 = off
   int8_t* qx;
   void* sx;
   float* y;               // zeroed here

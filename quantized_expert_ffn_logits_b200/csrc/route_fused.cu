@@ -155,27 +155,36 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
     __syncthreads();
     for (int t = warp; t < T; t += 8) {
       const bool on = lane < k;
-      const int my_e = on ? sel[t * k + lane] : 0;
+      int my_e = on ? sel[t * k + lane] : 0;
       const float myl = slog[t * E + my_e];
-      float wv;
+      float v, den;                      // slot mass, weight denominator (as topk.cuh)
       if (r.score == 0) {
         const float lmax = __shfl_sync(0xffffffffu, myl, 0);
-        const float ex = on ? cexp(myl - lmax) : 0.0f;
-        float den;
+        v = on ? cexp(myl - lmax) : 0.0f;
         if (r.renorm) {
-          den = warp_sum(ex);
+          den = warp_sum(v);
         } else {
           float sacc = 0.0f;
           for (int x = lane; x < E; x += 32) sacc += cexp(slog[t * E + x] - lmax);
           den = warp_sum(sacc);
         }
-        wv = ex / den * r.rsf;
       } else {
-        const float sg = on ? csigmoid(myl) : 0.0f;
-        const float den = r.renorm ? warp_sum(sg) : 1.0f;
-        wv = sg / den * r.rsf;
+        v = on ? csigmoid(myl) : 0.0f;
+        den = r.renorm ? warp_sum(v) : 1.0f;
+      }
+      float wv = v / den * r.rsf;
+      if (r.top_p > 0.0f) {
+        float cm;
+        const int m = topp_keep(v, k, r.top_p, cm);
+        if (lane >= m) {
+          my_e = -1;
+          wv = 0.0f;
+        } else if (r.renorm) {
+          wv = v / cm * r.rsf;
+        }
       }
       if (on) {
+        sel[t * k + lane] = my_e;
         r.idx[(int64_t)t * k + lane] = my_e;
         r.w[(int64_t)t * k + lane] = wv;
       }
@@ -184,18 +193,21 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
     // one warp per token
     for (int t = warp; t < T; t += 8) {
       const int my_e = warp_topk<NE>(r.logits + (int64_t)t * E, r.bias, E, k, r.score, r.renorm,
-                                     r.rsf, r.idx + (int64_t)t * k, r.w + (int64_t)t * k, r.status);
+                                     r.rsf, r.top_p, r.idx + (int64_t)t * k, r.w + (int64_t)t * k,
+                                     r.status);
       if (lane < k) sel[t * k + lane] = my_e;
     }
   }
   __syncthreads();
   if (T == 1) {
-    // one token: the active experts are its k distinct selections, one slot each, in
-    // ascending expert order
+    // one token: the active experts are its kept selections (all k, or the adaptive top-p
+    // prefix; dropped slots hold -1), one slot each, in ascending expert order
+    int nk = 0;
+    for (int j = 0; j < k; ++j) nk += sel[j] >= 0;
     if (tid < k) {
       const int ee = sel[tid];
       int pos = 0;
-      for (int j = 0; j < k; ++j) pos += sel[j] < ee;
+      for (int j = 0; j < k; ++j) pos += (sel[j] >= 0) & (sel[j] < ee);
       if (ee >= 0 && ee < E) {
         r.g.act_expert[pos] = ee;
         r.g.act_begin[pos] = pos;
@@ -205,13 +217,13 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
     }
     for (int x = tid; x < E; x += 256) {
       int cnt = 0;
-      for (int j = 0; j < k; ++j) cnt += sel[j] < x;
+      for (int j = 0; j < k; ++j) cnt += (sel[j] >= 0) & (sel[j] < x);
       r.g.offsets[x] = cnt;
     }
     if (tid == 0) {
-      r.g.offsets[E] = k;
-      *r.g.n_active = k;
-      r.g.act_begin[k] = k;
+      r.g.offsets[E] = nk;
+      *r.g.n_active = nk;
+      r.g.act_begin[nk] = nk;
       *r.ticket = 0u;
     }
     return;

@@ -193,7 +193,7 @@ void launch_router_logits(const float* x, const float* wr, int T, int E, int H, 
 template <int NE>
 __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits,
                                               const float* __restrict__ bias, int T, int E, int k,
-                                              int score, int renorm, float rsf,
+                                              int score, int renorm, float rsf, float top_p,
                                               int32_t* __restrict__ idx, float* __restrict__ w,
                                               Grouping g1, int single, int* status) {
   pdl_wait();
@@ -201,34 +201,41 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits,
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  const int my_e = warp_topk<NE>(logits + (int64_t)t * E, bias, E, k, score, renorm, rsf,
+  const int my_e = warp_topk<NE>(logits + (int64_t)t * E, bias, E, k, score, renorm, rsf, top_p,
                                  idx + (int64_t)t * k, w + (int64_t)t * k, status);
-  const bool sel = lane < k;
   if (single) {
-    // One token: the grouping is the k selected experts in ascending order.
-    int rank = 0;
-    for (int i = 0; i < k; ++i) rank += __shfl_sync(0xffffffffu, my_e, i) < my_e;
-    if (sel) {
+    // One token: the grouping is the kept selected experts (all k, or the top-p prefix: slots
+    // with expert -1 are dropped) in ascending order.
+    int rank = 0, nk = 0;
+    for (int i = 0; i < k; ++i) {
+      const int o = __shfl_sync(0xffffffffu, my_e, i);
+      nk += o >= 0;
+      rank += (o >= 0) & (o < my_e);
+    }
+    if (lane < k && my_e >= 0) {
       g1.act_expert[rank] = my_e;
       g1.act_begin[rank] = rank;
       g1.perm[rank] = lane;
     }
     if (lane == 0) {
-      g1.act_begin[k] = k;
-      *g1.n_active = k;
-      g1.offsets[E] = k;
+      g1.act_begin[nk] = nk;
+      *g1.n_active = nk;
+      g1.offsets[E] = nk;
     }
     for (int e0 = 0; e0 < E; e0 += 32) {
       const int e = e0 + lane;
       int cnt = 0;
-      for (int i = 0; i < k; ++i) cnt += __shfl_sync(0xffffffffu, my_e, i) < e;
+      for (int i = 0; i < k; ++i) {
+        const int o = __shfl_sync(0xffffffffu, my_e, i);
+        cnt += (o >= 0) & (o < e);
+      }
       if (e < E) g1.offsets[e] = cnt;
     }
   }
 }
 
 void launch_topk(const float* logits, const float* bias, int T, int E, int k, int score,
-                 int renorm, float rsf, int32_t* idx, float* w, const Grouping* single_token,
+                 int renorm, float rsf, float top_p, int32_t* idx, float* w, const Grouping* single_token,
                  int* status, cudaStream_t st) {
   if (T <= 0) return;
   const int blocks = (T + 7) / 8;
@@ -237,7 +244,7 @@ void launch_topk(const float* logits, const float* bias, int T, int E, int k, in
   const int single = single_token != nullptr;
 #define MOE_TOPK_CASE(N)                                                                     \
   launch_pdl(k_topk<N>, dim3(blocks), dim3(256), 0, st, logits, bias, T, E, k, score, renorm, rsf, \
-             idx, w, g, single, status)
+             top_p, idx, w, g, single, status)
   if (E <= 32) MOE_TOPK_CASE(1);
   else if (E <= 64) MOE_TOPK_CASE(2);
   else if (E <= 128) MOE_TOPK_CASE(4);
@@ -273,6 +280,7 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
     if (t < T) {
       for (int j = 0; j < k; ++j) {
         const int e = idx[(int64_t)t * k + j];
+        if (e == -1) continue;               // a slot dropped by adaptive top-p
         if (e < 0 || e >= E) set_status(status, kStatusDeviceCheck);
         else atomicOr(&mrow[e], 1u << lane);
       }

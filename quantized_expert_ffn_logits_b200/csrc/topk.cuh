@@ -5,6 +5,9 @@
 // weights s / sum_sel(s) * routed_scaling_factor (GLM-5.2 colibri page, "What's
 // implemented"). Lane l holds the keys of experts l, l+32, ... (NE per lane); k
 // rounds of a warp arg-max pick the largest key, equal keys going to the lower expert.
+//
+// Adaptive expert top-p (the colibri page's "--topp" knob): a token keeps only the shortest
+// prefix of its top-k list whose share of the list's mass reaches top_p (topp_keep).
 #pragma once
 
 #include <cfloat>
@@ -13,11 +16,34 @@
 
 namespace moe {
 
+// Adaptive top-p cut, called by every lane of a warp in which lane j < k holds the mass v of
+// slot j of a token's top-k list (v = exp(L_j - L_0) for softmax, sigmoid(L_j) for the sigmoid
+// router; lanes >= k pass anything). Every lane runs the same fp32 sums in slot order:
+// D = v_0 + ... + v_{k-1}, C_m = v_0 + ... + v_{m-1}; the result is the first m with
+// C_m >= top_p * D (k if none), and cm = C_m, the kept mass (the renormalized weights' sum).
+__device__ __forceinline__ int topp_keep(float v, int k, float top_p, float& cm) {
+  float d = 0.0f;
+  for (int j = 0; j < k; ++j) d = __fadd_rn(d, __shfl_sync(0xffffffffu, v, j));
+  const float thr = __fmul_rn(top_p, d);
+  float c = 0.0f;
+  int m = k;
+  for (int j = 0; j < k; ++j) {
+    c = __fadd_rn(c, __shfl_sync(0xffffffffu, v, j));
+    if (c >= thr) {                          // the same on every lane
+      m = j + 1;
+      break;
+    }
+  }
+  cm = c;
+  return m;
+}
+
 // Lt: the token's logits [E] (read through L2: they may have been written by other CTAs
-// of the same grid). Writes idx_out[j], w_out[j] for j < k; returns lane j's expert.
+// of the same grid). Writes idx_out[j], w_out[j] for j < k; returns lane j's expert (-1 for a
+// slot that adaptive top-p drops: top_p in (0, 1), else 0 = off).
 template <int NE>
 __device__ __forceinline__ int warp_topk(const float* Lt, const float* __restrict__ bias, int E,
-                                         int k, int score, int renorm, float rsf,
+                                         int k, int score, int renorm, float rsf, float top_p,
                                          int32_t* idx_out, float* w_out, int* status) {
   const int lane = threadIdx.x & 31;
   float key[NE], lg[NE];
@@ -63,13 +89,12 @@ __device__ __forceinline__ int warp_topk(const float* Lt, const float* __restric
   }
   const bool sel = lane < k;
   if (sel && (my_e < 0 || my_e >= E)) set_status(status, kStatusDeviceCheck);
-  float wv;
+  float v, den;                            // slot mass, weight denominator
   if (score == 0) {
     const float lmax = __shfl_sync(0xffffffffu, my_l, 0);
-    const float ex = sel ? cexp(my_l - lmax) : 0.0f;
-    float den;
+    v = sel ? cexp(my_l - lmax) : 0.0f;
     if (renorm) {
-      den = warp_sum(ex);
+      den = warp_sum(v);
     } else {
       float s = 0.0f;
 #pragma unroll
@@ -77,11 +102,20 @@ __device__ __forceinline__ int warp_topk(const float* Lt, const float* __restric
         if (lane + 32 * m < E) s += cexp(lg[m] - lmax);
       den = warp_sum(s);
     }
-    wv = ex / den * rsf;
   } else {
-    const float s = sel ? csigmoid(my_l) : 0.0f;
-    const float den = renorm ? warp_sum(s) : 1.0f;
-    wv = s / den * rsf;
+    v = sel ? csigmoid(my_l) : 0.0f;
+    den = renorm ? warp_sum(v) : 1.0f;
+  }
+  float wv = v / den * rsf;
+  if (top_p > 0.0f) {
+    float cm;
+    const int m = topp_keep(v, k, top_p, cm);
+    if (lane >= m) {
+      my_e = -1;
+      wv = 0.0f;
+    } else if (renorm) {
+      wv = v / cm * rsf;
+    }
   }
   if (sel) {
     idx_out[lane] = my_e;

@@ -23,10 +23,10 @@ def ag32(cfg):
     return cfg.act == "g32_f16"
 
 
-def route_cfg(cfg, flags=0):
+def route_cfg(cfg, flags=0, top_p=0.0):
     import quantized_expert_ffn_logits_b200 as M
     return M.RouteCfg(score=cfg.score, top_k=cfg.top_k, renormalize=cfg.renormalize,
-                      routed_scaling_factor=cfg.rsf, act=cfg.act, flags=flags)
+                      routed_scaling_factor=cfg.rsf, act=cfg.act, flags=flags, top_p=top_p)
 
 
 def gpu_layer(case: S.Case, device="cuda"):
@@ -67,11 +67,11 @@ def oracle_experts(case: S.Case, experts=None):
     return ex, sh
 
 
-def oracle_layer(case: S.Case, union=False):
+def oracle_layer(case: S.Case, union=False, top_p=0.0):
     c = case.cfg
     ex, sh = oracle_experts(case)
     return O.layer_forward(case.x(), case.router_w(), case.bias(), ex, sh, c.score, c.top_k,
-                           c.renormalize, c.rsf, ag32(c), union=union)
+                           c.renormalize, c.rsf, ag32(c), union=union, top_p=top_p)
 
 
 def oracle_tokens(case: S.Case, tokens):

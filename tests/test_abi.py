@@ -31,7 +31,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_status_strings():
-    assert M.moe_abi_version() == 1
+    assert M.moe_abi_version() == 2
     for s in range(7):
         assert M.moe_status_string(s).startswith("MOE_")
     assert M.moe_status_string(99) == "MOE_ERR_UNKNOWN"
@@ -56,8 +56,8 @@ def _blob(E=8, H=256, I=128, wtype=0, wscale=1, data=256, nbytes=None):
     return b
 
 
-def _cfg(k=2, score=0, act=1, flags=0):
-    return M.moe_route_cfg(score, k, 1, 1.0, act, flags)
+def _cfg(k=2, score=0, act=1, flags=0, top_p=0.0):
+    return M.moe_route_cfg(score, k, 1, 1.0, act, flags, top_p)
 
 
 def test_workspace_bytes_grow_with_tokens():
@@ -79,6 +79,9 @@ def test_forward_argument_errors_return_before_launch():
     assert f(fake, 4, fake, None, C.byref(b), None, C.byref(_cfg(k=9)), fake, fake, ws_need, None) == M.MOE_ERR_UNSUPPORTED
     assert f(fake, 4, fake, None, C.byref(b), None, C.byref(_cfg(k=0)), fake, fake, ws_need, None) == M.MOE_ERR_UNSUPPORTED
     assert f(fake, 4, fake, None, C.byref(b), None, C.byref(_cfg(score=7)), fake, fake, ws_need, None) == M.MOE_ERR_INVALID_ARG
+    for bad_p in (float("nan"), -0.25, float("inf")):     # adaptive top-p: finite and >= 0
+        assert f(fake, 4, fake, None, C.byref(b), None, C.byref(_cfg(top_p=bad_p)), fake, fake, ws_need, None) == M.MOE_ERR_INVALID_ARG
+        assert M._lib.moe_route_topk(fake, None, 4, 8, C.byref(_cfg(top_p=bad_p)), fake, fake, None) == M.MOE_ERR_INVALID_ARG
     assert f(fake, -1, fake, None, C.byref(b), None, C.byref(c), fake, fake, ws_need, None) == M.MOE_ERR_INVALID_ARG
     assert f(fake + 4, 4, fake, None, C.byref(b), None, C.byref(c), fake, fake, ws_need, None) == M.MOE_ERR_INVALID_ARG
     small = _blob(nbytes=1024)

@@ -50,11 +50,11 @@ def _np(t):
     return t.detach().cpu().numpy()
 
 
-def _run_layer(case, flags):
+def _run_layer(case, flags, top_p=0.0):
     m = M()
     c = case.cfg
     g = gpu_layer(case)
-    cfg = route_cfg(c, flags=flags)
+    cfg = route_cfg(c, flags=flags, top_p=top_p)
     y, ws = m.moe_layer_forward(g["x"], g["wr"], g["bias"], g["blob"], g["shared"], cfg)
     torch.cuda.synchronize()
     views = m.moe_layer_debug_views(case.T, g["blob"], g["shared"], cfg)
@@ -78,15 +78,53 @@ def test_tensor_core_path_matches_oracle(name, T, force):
     _check_layer(name, T, m.MOE_FLAG_DEBUG | (m.MOE_FLAG_FORCE_MMA if force else 0))
 
 
-def _check_layer(name, T, flags):
+# Adaptive expert top-p (the GLM page's "--topp"): every routing path -- the single-launch
+# decode kernel (T = 1, group-32 activations), the fused routing kernel (rank-based and warp
+# top-k, and its one-token grouping with per-token scales), the four-launch routing with the
+# tensor-core GEMMs -- drops the same slots as the oracle, bit for bit, and the layer output
+# leaves their experts out.
+TOPP_CASES = [("olmoe_int8", 1, 0.5), ("glm_int4", 1, 0.7), ("e512_int4", 1, 0.6),
+              ("tiny", 1, 0.3), ("tiny", 4, 0.3), ("glm_int4", 4, 0.7), ("olmoe_int8", 8, 0.5),
+              ("e512_int4", 30, 0.4), ("olmoe_int4", 130, 0.6), ("e512_int4", 100, 0.5)]
+
+
+@pytest.mark.parametrize("name,T,p", TOPP_CASES)
+def test_adaptive_top_p_matches_oracle(name, T, p):
+    _check_layer(name, T, M().MOE_FLAG_DEBUG, top_p=p)
+
+
+@pytest.mark.parametrize("score,renorm,E,k", [("softmax", True, 64, 8), ("softmax", False, 512, 10),
+                                              ("sigmoid", True, 256, 8)])
+def test_route_topk_adaptive_top_p(score, renorm, E, k):
+    m = M()
+    r = np.random.default_rng(E + k)
+    T = 200
+    L = r.normal(0, 1, (T, E)).astype(np.float32)
+    b = r.normal(0, 0.05, E).astype(np.float32) if score == "sigmoid" else None
+    rsf = 2.5 if score == "sigmoid" else 1.0
+    for p in (0.3, 0.6, 0.9):
+        want_idx, want_w = O.route(L, b, score, k, renorm, rsf, top_p=p)
+        cfg = m.RouteCfg(score=score, top_k=k, renormalize=renorm, routed_scaling_factor=rsf, top_p=p)
+        idx, w = m.moe_route_topk(torch.from_numpy(L).cuda(), torch.from_numpy(b).cuda() if b is not None else None,
+                                  cfg)
+        torch.cuda.synchronize()
+        assert np.array_equal(_np(idx), want_idx)
+        assert np.allclose(_np(w), want_w, rtol=2e-6, atol=1e-7)
+        if p < 0.8:          # (sigmoid masses of a top-8 are near equal: 0.9 keeps all 8)
+            assert (want_idx < 0).any()
+
+
+def _check_layer(name, T, flags, top_p=0.0):
     m = M()
     c = REDUCED[name]
     case = S.Case.make(c, T)
-    g, cfg, y, ws, v = _run_layer(case, flags)
+    g, cfg, y, ws, v = _run_layer(case, flags, top_p)
     assert m.moe_read_device_status(ws) == m.MOE_OK
-    ref = oracle_layer(case, union=True)
+    ref = oracle_layer(case, union=True, top_p=top_p)
     k, E, H, I = c.top_k, c.E, c.H, c.I
-    P = T * k
+    if top_p:
+        assert (ref["idx"] < 0).any(), "no slot dropped: the case does not exercise top-p"
+    P = int((ref["idx"] >= 0).sum())             # kept (token, slot) pairs
     view = lambda off, dt, shape: _np(m.workspace_view(ws, off, dt, shape))
     # routing: bit-exact logits and indices, weights to fp32 rounding
     assert np.array_equal(view(v["logits"], torch.float32, (T, E)), ref["logits"])
@@ -103,7 +141,7 @@ def _check_layer(name, T, flags):
     perm = view(v["perm"], torch.int32, (P,))
     assert np.array_equal(perm, ref["perm"])
     n_active = int(view(v["n_active"], torch.int32, (1,))[0])
-    assert n_active == len(set(ref["idx"].reshape(-1).tolist()))
+    assert n_active == len(set(ref["idx"].reshape(-1).tolist()) - {-1})
     # per-pair stage values (grouped row r holds pair perm[r]) and quantized h
     gate = view(v["gate"], torch.float32, (P, I))
     up = view(v["up"], torch.float32, (P, I))
