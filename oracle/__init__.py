@@ -53,6 +53,8 @@ def lib():
             "orc_blob_layout": (i32, [i32, i32, i32, i32, i32, vp]),
             "orc_pack_blob": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
             "orc_router_logits": (None, [vp, vp, i32, i32, i32, vp]),
+            "orc_fp8_e4m3_to_f32": (C.c_float, [C.c_uint8]),
+            "orc_dequant_fp8": (None, [vp, vp, C.c_int64, C.c_int64, vp]),
             "orc_route": (i32, [vp, vp, i32, i32, i32, i32, i32, f32, f32, vp, vp]),
             "orc_permute": (i32, [vp, i32, i32, i32, vp, vp]),
             "orc_stage": (C.c_float, [vp, vp, i32, i32, vp, vp, i32, vp]),
@@ -177,6 +179,30 @@ class QExperts:
 
 # ------------------------------------------------------------------ routing
 SCORES = {"softmax": 0, "sigmoid": 1}
+
+
+def fp8_e4m3_decode(codes):
+    """float8 E4M3 codes (uint8) as fp32, from the format's definition."""
+    codes = np.asarray(codes, np.uint8)
+    f = lib().orc_fp8_e4m3_to_f32
+    return np.array([f(int(c)) for c in codes.reshape(-1)], np.float32).reshape(codes.shape)
+
+
+def dequant_fp8(w8, s_inv):
+    """FP8 weights [..., N, K] (uint8 E4M3 codes) with fp32 inverse scales per 128 x 128 block
+    [..., ceil(N/128), ceil(K/128)] -> fp32 [..., N, K] (decode, then one fp32 product)."""
+    w8 = _c(w8, np.uint8)
+    s_inv = _c(s_inv, np.float32)
+    N, K = w8.shape[-2:]
+    lead = w8.shape[:-2]
+    out = np.empty(w8.shape, np.float32)
+    w2 = w8.reshape(-1, N, K)
+    s2 = s_inv.reshape(-1, (N + 127) // 128, (K + 127) // 128)
+    o2 = out.reshape(-1, N, K)
+    for i in range(w2.shape[0]):
+        wi, si, oi = w2[i], np.ascontiguousarray(s2[i]), o2[i]
+        lib().orc_dequant_fp8(_p(wi), _p(si), N, K, _p(oi))
+    return out.reshape(*lead, N, K)
 
 
 def router_logits(x, Wr):

@@ -361,6 +361,30 @@ int orc_permute(const int32_t* idx, int T, int k, int E, int32_t* offsets, int32
   return 0;
 }
 
+/* ---------------------------------------------- FP8 checkpoint conversion */
+
+/* One float8 E4M3 ("fn": no infinities) code as fp32, from the format's
+ * definition: sign bit 7, exponent bits 6-3 with bias 7, mantissa bits 2-0;
+ * exponent 0 is subnormal (m * 2^-9), else (8 + m) * 2^(e - 10); exponent 15
+ * with mantissa 7 is NaN. Every value is exact in fp32. */
+float orc_fp8_e4m3_to_f32(uint8_t v) {
+  const int s = v >> 7, e = (v >> 3) & 15, m = v & 7;
+  if (e == 15 && m == 7) return NAN;
+  const float mag = e == 0 ? ldexpf((float)m, -9) : ldexpf((float)(8 + m), e - 10);
+  return s ? -mag : mag;
+}
+
+/* The GLM page's FP8 -> int4 converter step, dequantizing side: an FP8 matrix
+ * [N][K] with one fp32 inverse scale per 128 x 128 block ([ceil(N/128)][ceil(K/128)],
+ * the DeepSeek-V3-style checkpoint layout) to fp32: w = decode(code) * scale, one
+ * fp32 rounding. The codes are then quantized like any fp32 weight. */
+void orc_dequant_fp8(const uint8_t* w8, const float* s_inv, int64_t N, int64_t K, float* out) {
+  const int64_t KB = (K + 127) / 128;
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k)
+      out[n * K + k] = orc_fp8_e4m3_to_f32(w8[n * K + k]) * s_inv[(n / 128) * KB + k / 128];
+}
+
 /* -------------------------------------------------------- expert arithmetic */
 
 /* Canonical fp32 stage value of one weight row against one activation vector.

@@ -562,3 +562,38 @@ def test_topp_layer_equals_kept_expert_composition(name, p):
         if sh is not None:
             want += O.expert_ffn(sh, 0, qx[t], sx[t], ag32)["ye"]
         assert np.allclose(a["y"][t], want, rtol=1e-12, atol=1e-15)
+
+
+# ----------------------------------------------------- FP8 checkpoint conversion
+# The GLM page's FP8 -> int4 converter: FP8 (E4M3) weights with one inverse scale per
+# 128 x 128 block are dequantized, then quantized like any fp32 weight.
+def test_fp8_e4m3_decode_matches_library_for_all_codes():
+    torch = pytest.importorskip("torch")
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).float().numpy()
+    got = O.fp8_e4m3_decode(codes)
+    nan = np.isnan(want)
+    assert nan.sum() == 2 and np.array_equal(np.isnan(got), nan)      # 0x7f, 0xff
+    assert np.array_equal(got[~nan].view(np.uint32), want[~nan].view(np.uint32))   # -0 included
+
+
+def test_fp8_e4m3_closed_forms():
+    """Values fixed by the E4M3 definition (bias 7, 3 mantissa bits, no infinities)."""
+    cases = {0x38: 1.0, 0x30: 0.5, 0xC0: -2.0, 0x7E: 448.0, 0x08: 2.0 ** -6, 0x01: 2.0 ** -9,
+             0x07: 7 * 2.0 ** -9, 0x3F: 1.875, 0x00: 0.0}
+    got = O.fp8_e4m3_decode(np.array(list(cases), np.uint8))
+    assert got.tolist() == list(cases.values())
+
+
+def test_fp8_block_scales_cover_ragged_blocks():
+    torch = pytest.importorskip("torch")
+    r = rng(60)
+    E, N, K = 2, 300, 200                                  # ragged last blocks in both dims
+    w8 = r.integers(0, 256, (E, N, K), dtype=np.uint8)
+    w8[(w8 & 0x7F) == 0x7F] = 0x38                         # no NaN codes
+    s = (2.0 ** r.integers(-12, -2, (E, 3, 2))).astype(np.float32) * r.uniform(1, 2, (E, 3, 2)).astype(np.float32)
+    got = O.dequant_fp8(w8, s)
+    dec = torch.from_numpy(w8.reshape(-1).copy()).view(torch.float8_e4m3fn).float().numpy().reshape(E, N, K)
+    full = np.repeat(np.repeat(s, 128, axis=1), 128, axis=2)[:, :N, :K]
+    assert np.array_equal(got, (dec * full).astype(np.float32))
+    assert got[1, 299, 199] == dec[1, 299, 199] * s[1, 2, 1]
