@@ -688,6 +688,54 @@ def traffic_from_profiles(cfg, T):
         return None
 
 
+def fp8_convert_arm(args):
+    """The FP8 checkpoint converter (GLM page, FP8 -> int4): moe_quantize_experts_fp8 on the
+    OLMoE-shaped expert set (E4M3 codes with 128 x 128 block scales -> packed int4, group-32
+    fp16 scales), device-resident input, CUDA events over K conversions. Bound: HBM (read the
+    codes and scales once, write the blob once)."""
+    import torch
+    import quantized_expert_ffn_logits_b200 as M
+    cfg = S.CONFIGS["olmoe_int4"]
+    E, H, I = cfg.E, cfg.H, cfg.I
+    cdiv = lambda a: (a + 127) // 128
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(8)
+    def codes(shape):
+        c = torch.randint(0, 256, shape, dtype=torch.uint8, device=dev, generator=g)
+        return torch.where((c & 0x7F) == 0x7F, torch.full_like(c, 0x3A), c)   # no NaN codes
+    gu8, dn8 = codes((E, 2 * I, H)), codes((E, H, I))
+    sgu = torch.rand((E, cdiv(2 * I), cdiv(H)), device=dev, generator=g) * 2 ** -8 + 2 ** -9
+    sdn = torch.rand((E, cdiv(H), cdiv(I)), device=dev, generator=g) * 2 ** -8 + 2 ** -9
+    blob = M.ExpertBlob(cfg.wtype, cfg.wscale, E, H, I, device=dev)
+    for _ in range(args.warmup):
+        M.moe_quantize_experts_fp8(gu8, sgu, dn8, sdn, blob)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        M.moe_quantize_experts_fp8(gu8, sgu, dn8, sdn, blob)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    nbytes = gu8.numel() + dn8.numel() + 4 * (sgu.numel() + sdn.numel()) + blob.nbytes
+    peaks, src = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line = {"metric": "FP8 checkpoint -> int4 blob conversion (moe_quantize_experts_fp8)",
+            "value": round(gbs, 1), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp8->int4", "data": "synthetic",
+            "config": {"workload": f"OLMoE-shaped experts E{E} H{H} I{I}: E4M3 codes + 128x128 block "
+                                   f"scales -> {cfg.wtype} {cfg.wscale} blob",
+                       "bytes_per_step": int(nbytes), "experts_per_s": round(E / (ms * 1e-3), 1)},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                         "peak_source": src},
+            "gpu_launches": 2 * args.steps}     # a blob memset and the conversion kernel per step
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -706,6 +754,8 @@ def main(argv=None):
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (4k tokens) measurement")
     ap.add_argument("--prefill-workload", default=PREFILL_WORKLOAD)
     ap.add_argument("--prefill-steps", type=int, default=20)
+    ap.add_argument("--fp8-convert", action="store_true",
+                    help="time the FP8 checkpoint converter instead of the layer (one JSON line)")
     ap.add_argument("--top-p", type=float, default=0.0,
                     help="adaptive expert top-p of the main workload (0 = off; the prefill half "
                          "is measured without it)")
@@ -713,6 +763,8 @@ def main(argv=None):
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     cfg, T = parse_workload(args.workload)
+    if args.fp8_convert:
+        return fp8_convert_arm(args)
     if args.impl == "reference":
         return reference_arm(args, cfg, T)
     return gpu_arm(args, cfg, T)

@@ -177,6 +177,20 @@ MOE_API moe_status moe_quantize_experts(const float* w_gate_up, const float* w_d
 /* Q8_0-style activation quantization (GLM page, "Integer-dot kernels (Q8_0-style int8
  * activations ...)").  x [T][H] fp32 -> q [T][H] int8 and `scales`: fp16 [T][H/32]
  * (MOE_ACT_G32_F16) or fp32 [T] (MOE_ACT_TOKEN_F32). H multiple of 32. */
+/* The GLM-5.2 colibri page's FP8 -> int4 converter step, on the GPU: FP8 checkpoint weights
+ * (float8 E4M3 codes, "fn" variant: no infinities) with one fp32 inverse scale per 128 x 128
+ * block of each expert's matrix (the DeepSeek-V3-style layout) are dequantized -- value =
+ * code (exact in fp32) * its block's scale, one fp32 rounding -- and quantized into `out`
+ * exactly as moe_quantize_experts quantizes fp32 weights (any wtype / wscale).
+ *   w_gate_up: uint8 [E][2I][H] (gate rows then up rows per expert), s_gate_up: fp32
+ *   [E][ceil(2I/128)][ceil(H/128)]; w_down: uint8 [E][H][I], s_down: fp32
+ *   [E][ceil(H/128)][ceil(I/128)]. All device memory, caller-owned, read only.
+ * NaN codes (0x7f, 0xff) are invalid input (the blob is then undefined). Errors as
+ * moe_quantize_experts. */
+MOE_API moe_status moe_quantize_experts_fp8(const uint8_t* w_gate_up, const float* s_gate_up,
+                                            const uint8_t* w_down, const float* s_down,
+                                            const moe_expert_blob* out, void* stream);
+
 MOE_API moe_status moe_quantize_activations(const float* x, int32_t T, int32_t H, int32_t act,
                                     int8_t* q, void* scales, void* stream);
 

@@ -68,6 +68,7 @@ _SIGS = {
     "moe_last_error": (C.c_char_p, []),
     "moe_expert_blob_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "moe_quantize_experts": (_i32, [_vp, _vp, _PB, _vp]),
+    "moe_quantize_experts_fp8": (_i32, [_vp, _vp, _vp, _vp, _PB, _vp]),
     "moe_quantize_activations": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_router_logits": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp]),
     "moe_route_topk": (_i32, [_vp, _vp, _i32, _i32, _PC, _vp, _vp, _vp]),
@@ -179,6 +180,17 @@ class ExpertBlob:
         moe_quantize_experts(w_gate_up, w_down, b, stream)
         return b
 
+    @classmethod
+    def quantize_fp8(cls, w_gate_up, s_gate_up, w_down, s_down, wtype: str, wscale: str,
+                     stream=None) -> "ExpertBlob":
+        """FP8 checkpoint weights -> blob: w_gate_up [E][2I][H] and w_down [E][H][I] E4M3 codes
+        (torch.uint8 or torch.float8_e4m3fn CUDA tensors), s_gate_up / s_down fp32 inverse
+        scales per 128 x 128 block ([E][ceil(2I/128)][ceil(H/128)], [E][ceil(H/128)][ceil(I/128)])."""
+        E, twoI, H = w_gate_up.shape
+        b = cls(wtype, wscale, E, H, twoI // 2, device=w_gate_up.device)
+        moe_quantize_experts_fp8(w_gate_up, s_gate_up, w_down, s_down, b, stream)
+        return b
+
 
 # ---------------------------------------------------------------- entry points
 def moe_abi_version() -> int:
@@ -191,6 +203,23 @@ def moe_status_string(status: int) -> str:
 
 def moe_expert_blob_bytes(wtype: int, wscale: int, n_experts: int, hidden: int, inter: int) -> int:
     return int(_lib.moe_expert_blob_bytes(wtype, wscale, n_experts, hidden, inter))
+
+
+def moe_quantize_experts_fp8(w_gate_up, s_gate_up, w_down, s_down, blob: ExpertBlob, stream=None) -> None:
+    import torch
+    E, I, H = blob.n_experts, blob.inter, blob.hidden
+    cdiv = lambda a: (a + 127) // 128
+    for t, name, shape in ((w_gate_up, "w_gate_up", (E, 2 * I, H)), (w_down, "w_down", (E, H, I))):
+        if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or tuple(t.shape) != shape:
+            raise ValueError(f"{name}: want uint8/float8_e4m3fn {shape}, got {t.dtype} {tuple(t.shape)}")
+        _dev(t, t.dtype, name)
+    _dev(s_gate_up, torch.float32, "s_gate_up")
+    _dev(s_down, torch.float32, "s_down")
+    if tuple(s_gate_up.shape) != (E, cdiv(2 * I), cdiv(H)) or tuple(s_down.shape) != (E, cdiv(H), cdiv(I)):
+        raise ValueError("block scales: want [E][ceil(2I/128)][ceil(H/128)] and [E][ceil(H/128)][ceil(I/128)]")
+    st = blob.struct()
+    _check(_lib.moe_quantize_experts_fp8(_ptr(w_gate_up), _ptr(s_gate_up), _ptr(w_down), _ptr(s_down),
+                                         C.byref(st), _stream(stream)), "moe_quantize_experts_fp8")
 
 
 def moe_quantize_experts(w_gate_up, w_down, blob: ExpertBlob, stream=None) -> None:

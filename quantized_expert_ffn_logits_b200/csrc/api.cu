@@ -262,6 +262,23 @@ moe_status moe_quantize_experts(const float* w_gate_up, const float* w_down,
   return launch_status();
 }
 
+moe_status moe_quantize_experts_fp8(const uint8_t* w_gate_up, const float* s_gate_up,
+                                    const uint8_t* w_down, const float* s_down,
+                                    const moe_expert_blob* out, void* stream) {
+  if (!w_gate_up || !s_gate_up || !w_down || !s_down) return MOE_ERR_INVALID_ARG;
+  BlobOffsets o;
+  const moe_status s = check_blob(out, o);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t me = cudaMemsetAsync(out->data, 0, (size_t)o.total, st);
+  if (me != cudaSuccess) return cuda_fail("blob memset", me);
+  const BlobView b = view(out, o);
+  uint8_t* d = static_cast<uint8_t*>(out->data);
+  moe::launch_quantize_experts_fp8(w_gate_up, s_gate_up, w_down, s_down, b, d + o.gu_w, d + o.dn_w,
+                                   d + o.gu_s, d + o.dn_s, st);
+  return launch_status();
+}
+
 moe_status moe_quantize_activations(const float* x, int32_t T, int32_t H, int32_t act, int8_t* q,
                                     void* scales, void* stream) {
   if (T < 0 || H <= 0 || H % 32) return T < 0 ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED;

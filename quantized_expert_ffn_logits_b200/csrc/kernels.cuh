@@ -12,6 +12,11 @@ namespace moe {
 void launch_quantize_experts(const float* w_gu, const float* w_dn, const BlobView& b,
                              uint8_t* gu_w, uint8_t* dn_w, uint8_t* gu_s, uint8_t* dn_s,
                              cudaStream_t st);
+// FP8 checkpoint weights: E4M3 codes [E][2I][H] / [E][H][I] with fp32 inverse scales per
+// 128 x 128 block, [E][ceil(2I/128)][ceil(H/128)] / [E][ceil(H/128)][ceil(I/128)].
+void launch_quantize_experts_fp8(const uint8_t* w_gu, const float* s_gu, const uint8_t* w_dn,
+                                 const float* s_dn, const BlobView& b, uint8_t* gu_w, uint8_t* dn_w,
+                                 uint8_t* gu_s, uint8_t* dn_s, cudaStream_t st);
 // y_zero (optional): output rows to zero; status (optional): status word to reset.
 void launch_quantize_act(const float* x, int T, int H, int g32, int8_t* q, void* scales,
                          float* y_zero, int* status, cudaStream_t st);

@@ -4,19 +4,42 @@
 // implemented": "Quantization kernels: int8 / packed int4 / packed int2,
 // per-row scales, dequant-on-use"; Q8_0-style int8 activations from the same
 // section; group size 32 from the mtlm-7m-base card, "Files").
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.cuh"
 #include "tma.cuh"
 
 namespace moe {
 
+// A float8 E4M3 code ("fn": no infinities) as fp32, from the format's bit layout: sign bit 7,
+// exponent bits 6-3 (bias 7), mantissa bits 2-0; exponent 0 is subnormal (m * 2^-9);
+// exponent 15 with mantissa 7 is NaN. Exact.
+__device__ __forceinline__ float fp8_e4m3(uint32_t v) {
+  const uint32_t e = (v >> 3) & 15u, m = v & 7u;
+  float mag = e == 0 ? (float)m * 0x1p-9f : __uint_as_float(((e + 120u) << 23) | (m << 20));
+  if (e == 15u && m == 7u) mag = __uint_as_float(0x7fc00000u);
+  return (v & 0x80u) ? -mag : mag;
+}
+
+// Weight values to quantize: fp32 rows, or FP8 checkpoint rows (the GLM page's FP8 -> int4
+// converter): E4M3 codes with one fp32 inverse scale per 128 x 128 block of each expert's
+// matrix, value = code * scale (one fp32 rounding).
+struct WSource {
+  const float* gu;          // fp32 [E][2I][H]
+  const float* dn;          // fp32 [E][H][I]
+  const uint8_t* gu8;       // E4M3 [E][2I][H]
+  const float* gu_s;        //   [E][ceil(2I/128)][ceil(H/128)]
+  const uint8_t* dn8;       // E4M3 [E][H][I]
+  const float* dn_s;        //   [E][ceil(H/128)][ceil(I/128)]
+};
+
 // One warp per weight row. Rows [0, E*2I) are gate/up rows (logical [E][2I][H]),
 // rows [E*2I, E*2I + E*H) are down rows (logical [E][H][I]). Codes and scales are
 // written straight into the blob's tiled layout (include/moe_b200.h).
-__global__ void __launch_bounds__(256) k_quantize_experts(const float* __restrict__ w_gu,
-                                                          const float* __restrict__ w_dn,
-                                                          BlobView b, uint8_t* gu_w, uint8_t* dn_w,
-                                                          uint8_t* gu_s, uint8_t* dn_s) {
+template <bool FP8>
+__global__ void __launch_bounds__(256) k_quantize_experts(const WSource w, BlobView b, uint8_t* gu_w,
+                                                          uint8_t* dn_w, uint8_t* gu_s, uint8_t* dn_s) {
   const int lane = threadIdx.x & 31;
   const int64_t n_gu = (int64_t)b.E * 2 * b.I;
   const int64_t n_rows = n_gu + (int64_t)b.E * b.H;
@@ -24,7 +47,9 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const float* __restric
   const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t R = warp0; R < n_rows; R += nwarps) {
-    const float* src;
+    const float* src = nullptr;             // fp32 source row
+    const uint8_t* src8 = nullptr;          // FP8 source row and its blocks' scales
+    const float* srow = nullptr;
     int K;
     bool down;
     int64_t blk = 0;     // gate/up: first row of the row's 128-row block
@@ -39,7 +64,12 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const float* __restric
       down = false;
       r = half * 64 + (i & 63);
       blk = (int64_t)e * 2 * b.I + (int64_t)(i >> 6) * 128;
-      src = w_gu + R * (int64_t)K;
+      if constexpr (FP8) {
+        src8 = w.gu8 + R * (int64_t)K;
+        srow = w.gu_s + ((int64_t)e * ((2 * b.I + 127) / 128) + lr / 128) * ((K + 127) / 128);
+      } else {
+        src = w.gu + R * (int64_t)K;
+      }
     } else {
       const int64_t R2 = R - n_gu;
       e = (int)(R2 / b.H);
@@ -48,8 +78,17 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const float* __restric
       down = true;
       hb = n >> 7;
       r = n & 127;
-      src = w_dn + R2 * (int64_t)K;
+      if constexpr (FP8) {
+        src8 = w.dn8 + R2 * (int64_t)K;
+        srow = w.dn_s + ((int64_t)e * ((b.H + 127) / 128) + n / 128) * ((K + 127) / 128);
+      } else {
+        src = w.dn + R2 * (int64_t)K;
+      }
     }
+    auto value = [&](int k) -> float {
+      if constexpr (FP8) return __fmul_rn(fp8_e4m3(src8[k]), srow[k >> 7]);
+      else return src[k];
+    };
     const int G = K / 32;
     const int kb = kbytes(K, b.wbits);
     const int U = b.I / 64, HB = b.H / 128;
@@ -71,13 +110,13 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const float* __restric
     float s_row = 0.0f;
     if (!b.wg32) {
       float amax = 0.0f;
-      for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(src[k]));
+      for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(value(k)));
       amax = warp_max(amax);
       s_row = __fdiv_rn(amax, qmax);
       if (lane == 0) *reinterpret_cast<float*>(scale_at(0)) = s_row;
     }
     for (int g = 0; g < G; ++g) {
-      const float v = src[32 * g + lane];
+      const float v = value(32 * g + lane);
       float s = s_row;
       if (b.wg32) {
         const float amax = warp_max(fabsf(v));
@@ -170,13 +209,31 @@ __global__ void __launch_bounds__(256) k_quantize_rows_token(const float* __rest
   if (threadIdx.x == 0) scales[r] = s;
 }
 
+namespace {
+int64_t quantize_blocks(const BlobView& b) {
+  const int64_t rows = (int64_t)b.E * (2 * b.I + b.H);
+  return std::min<int64_t>((rows + 7) / 8, 148 * 64);
+}
+}  // namespace
+
 void launch_quantize_experts(const float* w_gu, const float* w_dn, const BlobView& b,
                              uint8_t* gu_w, uint8_t* dn_w, uint8_t* gu_s, uint8_t* dn_s,
                              cudaStream_t st) {
-  const int64_t rows = (int64_t)b.E * (2 * b.I + b.H);
-  int64_t blocks = (rows + 7) / 8;
-  if (blocks > 148 * 64) blocks = 148 * 64;
-  k_quantize_experts<<<(unsigned)blocks, 256, 0, st>>>(w_gu, w_dn, b, gu_w, dn_w, gu_s, dn_s);
+  WSource w{};
+  w.gu = w_gu;
+  w.dn = w_dn;
+  k_quantize_experts<false><<<(unsigned)quantize_blocks(b), 256, 0, st>>>(w, b, gu_w, dn_w, gu_s, dn_s);
+}
+
+void launch_quantize_experts_fp8(const uint8_t* w_gu, const float* s_gu, const uint8_t* w_dn,
+                                 const float* s_dn, const BlobView& b, uint8_t* gu_w, uint8_t* dn_w,
+                                 uint8_t* gu_s, uint8_t* dn_s, cudaStream_t st) {
+  WSource w{};
+  w.gu8 = w_gu;
+  w.gu_s = s_gu;
+  w.dn8 = w_dn;
+  w.dn_s = s_dn;
+  k_quantize_experts<true><<<(unsigned)quantize_blocks(b), 256, 0, st>>>(w, b, gu_w, dn_w, gu_s, dn_s);
 }
 
 void launch_quantize_act(const float* x, int T, int H, int g32, int8_t* q, void* scales,

@@ -102,6 +102,8 @@ def test_other_entry_points_reject_bad_arguments():
     b = _blob()
     assert L.moe_quantize_experts(None, fake, C.byref(b), None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_quantize_experts(fake, fake, C.byref(_blob(nbytes=10)), None) == M.MOE_ERR_WORKSPACE
+    assert L.moe_quantize_experts_fp8(fake, None, fake, fake, C.byref(b), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_experts_fp8(fake, fake, fake, fake, C.byref(_blob(nbytes=10)), None) == M.MOE_ERR_WORKSPACE
     assert L.moe_quantize_activations(fake, 4, 100, 1, fake, fake, None) == M.MOE_ERR_UNSUPPORTED
     assert L.moe_quantize_activations(fake, 4, 128, 5, fake, fake, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_router_logits(fake, fake, 4, 8, 100, fake, None) == M.MOE_ERR_UNSUPPORTED

@@ -259,6 +259,33 @@ def test_quantize_experts_blob_bytes_identical(wtype, wscale, E, H, I):
     assert diff.size == 0, f"{diff.size} bytes differ, first at {diff[:8]}"
 
 
+@pytest.mark.parametrize("wtype,wscale", [("int8", "row_f32"), ("int8", "g32_f16"),
+                                          ("int4", "row_f32"), ("int4", "g32_f16")])
+@pytest.mark.parametrize("E,H,I", [(3, 256, 128), (2, 384, 256)])
+def test_quantize_experts_fp8_blob_bytes_identical(wtype, wscale, E, H, I):
+    """The FP8 checkpoint converter (GLM page): E4M3 codes with 128 x 128 block scales give the
+    oracle's blob byte for byte (every code but the two NaNs, scales varying per block)."""
+    m = M()
+    r = np.random.default_rng(E * H + I)
+    cdiv = lambda a: (a + 127) // 128
+    gu8 = r.integers(0, 256, (E, 2 * I, H), dtype=np.uint8)
+    dn8 = r.integers(0, 256, (E, H, I), dtype=np.uint8)
+    for a in (gu8, dn8):
+        a[(a & 0x7F) == 0x7F] = 0x3A                      # no NaN codes
+    gu8[0, 5, :32] = 0                                     # an all-zero group
+    sgu = (r.uniform(0.5, 2.0, (E, cdiv(2 * I), cdiv(H))) * 2.0 ** -8).astype(np.float32)
+    sdn = (r.uniform(0.5, 2.0, (E, cdiv(H), cdiv(I))) * 2.0 ** -8).astype(np.float32)
+    blob = m.ExpertBlob.quantize_fp8(torch.from_numpy(gu8).cuda(), torch.from_numpy(sgu).cuda(),
+                                     torch.from_numpy(dn8).cuda(), torch.from_numpy(sdn).cuda(), wtype, wscale)
+    ex = O.QExperts.quantize(O.dequant_fp8(gu8, sgu), O.dequant_fp8(dn8, sdn), 8 if wtype == "int8" else 4,
+                             wscale == "g32_f16")
+    got = _np(blob.data)
+    want = ex.pack_blob()
+    assert got.size == want.size
+    diff = np.nonzero(got != want)[0]
+    assert diff.size == 0, f"{diff.size} bytes differ, first at {diff[:8]}"
+
+
 @pytest.mark.parametrize("act", ["g32_f16", "token_f32"])
 @pytest.mark.parametrize("T,H,sigma", [(1, 2048, 1.0), (7, 256, 0.02), (65, 6144, 3.0)])
 def test_quantize_activations_bit_exact(act, T, H, sigma):
