@@ -202,7 +202,8 @@ MOE_API moe_status moe_router_logits(const float* x, const float* router_w, int3
  * sigmoid router (noaux_tc, routed_scaling_factor)"; OLMoE page: "top-8 of 64").
  * bias [E] (sigmoid mode only, may be NULL = zeros) shifts the selection key, never the
  * weights. idx [T][k] int32 in descending key order (ties: lower expert index first),
- * w [T][k] fp32. */
+ * w [T][k] fp32. With cfg->top_p in (0, 1) (adaptive top-p, see moe_route_cfg) the slots
+ * after each token's kept prefix hold idx -1 and w 0. */
 MOE_API moe_status moe_route_topk(const float* logits, const float* bias, int32_t T, int32_t E,
                           const moe_route_cfg* cfg, int32_t* idx, float* w, void* stream);
 
@@ -210,9 +211,10 @@ MOE_API moe_status moe_route_topk(const float* logits, const float* bias, int32_
 MOE_API size_t moe_permute_workspace_bytes(int32_t T, int32_t k, int32_t E);
 
 /* Batch-union grouping (GLM page, "Batch-union MoE"): offsets [E+1] (offsets[e] = first
- * position of expert e) and perm [T*k], the pair indices t*k+j sorted by (expert, t).
- * idx values must lie in [0, E); out-of-range values set MOE_ERR_DEVICE_CHECK in the
- * workspace status word and are dropped. */
+ * position of expert e) and perm [offsets[E]], the pair indices t*k+j sorted by (expert, t).
+ * idx values must lie in [0, E) or be -1 (a slot dropped by adaptive top-p: left out, so
+ * offsets[E] = the kept pairs); other values set MOE_ERR_DEVICE_CHECK in the workspace
+ * status word and are dropped. */
 MOE_API moe_status moe_permute(const int32_t* idx, int32_t T, int32_t k, int32_t E, int32_t* offsets,
                        int32_t* perm, void* workspace, size_t ws_bytes, void* stream);
 
