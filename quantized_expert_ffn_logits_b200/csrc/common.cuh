@@ -53,15 +53,6 @@ __device__ __forceinline__ float cswiglu(float g, float u) {
 __device__ __forceinline__ float exact_i2f(int v) {
   return __fsub_rn(__int_as_float(0x4B400000 + v), 12582912.0f);
 }
-// The same with the bias folded in: (float)(a + bias_a) for kb = 0x4B400000 + bias_a.
-__device__ __forceinline__ float2 exact_i2f2k(int a, int b, int kb) {
-  return __fadd2_rn(make_float2(__int_as_float(kb + a), __int_as_float(kb + b)),
-                    make_float2(-12582912.0f, -12582912.0f));
-}
-__device__ __forceinline__ float2 exact_i2f2(int a, int b) {
-  return __fadd2_rn(make_float2(__int_as_float(0x4B400000 + a), __int_as_float(0x4B400000 + b)),
-                    make_float2(-12582912.0f, -12582912.0f));
-}
 
 // ---------------------------------------------------------------- quantization
 __device__ __forceinline__ float f16_round(float d) { return __half2float(__float2half_rn(d)); }
@@ -86,12 +77,6 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-__device__ __forceinline__ int warp_sum_int(int v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
@@ -104,20 +89,6 @@ __device__ __forceinline__ void wait_failed(int* status, int kernel, int role, i
     status[2] = kernel | (role << 4) | (stage << 8);
     status[3] = (int)blockIdx.x;
   }
-}
-
-// Streaming 128-bit load of read-only data (no L1 allocation: weights are read once).
-__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
-  uint4 v;
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-      : "l"(p));
-  return v;
-}
-
-// Fire-and-forget prefetch of the line holding p into L2.
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // y[0..3] += (a, b, c, d): one 16-byte reduction (sm_90+), p 16-byte aligned.
