@@ -128,3 +128,15 @@ def test_other_entry_points_reject_bad_arguments():
     assert f(fake, 4, fake, None, C.byref(b), None, C.byref(_cfg()), fake, fake, plain, None, None) == M.MOE_ERR_INVALID_ARG
     assert f(fake, 4, fake, None, C.byref(b), None, C.byref(_cfg()), fake, fake, plain, None, C.byref(v)) == M.MOE_ERR_WORKSPACE
     assert v.gate == 12345
+
+
+def test_build_entry_point_builds_and_checks_the_library():
+    """__graft_entry__.build(): compiles what is stale (nothing, normally) and checks the
+    library it loads (ABI version, exports)."""
+    import importlib
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    if root not in sys.path:
+        sys.path.insert(0, root)
+    g = importlib.import_module("__graft_entry__")
+    g.build()
