@@ -50,6 +50,7 @@ def lib():
             "orc_swiglu_n": (None, [vp, vp, i64, vp]),
             "orc_quantize_rows": (i32, [vp, i64, i32, i32, i32, vp, vp]),
             "orc_pack_int4": (i32, [vp, i64, i32, vp]),
+            "orc_pack_int2": (i32, [vp, i64, i32, vp]),
             "orc_blob_layout": (i32, [i32, i32, i32, i32, i32, vp]),
             "orc_pack_blob": (i32, [i32, i32, i32, i32, i32, vp, vp, vp, vp, vp]),
             "orc_router_logits": (None, [vp, vp, i32, i32, i32, vp]),
@@ -128,6 +129,18 @@ def pack_int4(q):
     return out
 
 
+def pack_int2(q):
+    q = _c(q, np.int8)
+    N, K = q.shape
+    out = np.empty((N, K // 4), np.uint8)
+    if lib().orc_pack_int2(_p(q), N, K, _p(out)):
+        raise ValueError("K not a multiple of 4")
+    return out
+
+
+QMAX = {8: 127, 4: 7, 2: 1}      # symmetric codes: 2^(bits-1) - 1
+
+
 def blob_layout(E, H, I, wbits, g32):
     off = np.zeros(5, np.uint64)
     if lib().orc_blob_layout(E, H, I, wbits, int(g32), _p(off)):
@@ -152,7 +165,7 @@ class QExperts:
         down = np.asarray(down, np.float32)
         E, twoI, H = gate_up.shape
         I = twoI // 2
-        qmax = 127 if wbits == 8 else 7
+        qmax = QMAX[wbits]
         qg, sg = quantize_rows(gate_up.reshape(E * twoI, H), qmax, wg32)
         qd, sd = quantize_rows(down.reshape(E * H, I), qmax, wg32)
         return cls(qg.reshape(E, twoI, H), sg.reshape((E, twoI, H // 32) if wg32 else (E, twoI)),

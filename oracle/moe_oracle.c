@@ -160,6 +160,22 @@ int orc_pack_int4(const int8_t* q, int64_t N, int K, uint8_t* out) {
   return 0;
 }
 
+/* Pack int2 codes four per byte (the GLM page's "packed int2"): element 4j + i in bits
+ * 2i .. 2i + 1 of byte j, two's complement (codes -1, 0, 1 under the symmetric rule). */
+int orc_pack_int2(const int8_t* q, int64_t N, int K, uint8_t* out) {
+  if (K % 4) return 1;
+  for (int64_t n = 0; n < N; ++n)
+    for (int j = 0; j < K / 4; ++j) {
+      uint8_t b = 0;
+      for (int i = 0; i < 4; ++i) b |= (uint8_t)(((uint8_t)q[n * K + 4 * j + i] & 3u) << (2 * i));
+      out[n * (K / 4) + j] = b;
+    }
+  return 0;
+}
+
+/* Code bytes of K elements of a row. */
+static uint64_t code_bytes(uint64_t K, int wbits) { return K * (uint64_t)wbits / 8; }
+
 /* ------------------------------------------------------ expert blob layout */
 /* The blob byte layout is the one the library's public header documents:
  * four regions (gate/up codes, down codes, gate/up scales, down scales), each
@@ -173,9 +189,9 @@ int orc_pack_int4(const int8_t* q, int64_t N, int K, uint8_t* out) {
 static uint64_t al256(uint64_t v) { return (v + 255) & ~(uint64_t)255; }
 
 int orc_blob_layout(int E, int H, int I, int wbits, int g32, uint64_t* off /* [5] */) {
-  if (E <= 0 || H <= 0 || I <= 0 || H % 128 || I % 128 || (wbits != 8 && wbits != 4)) return 1;
-  uint64_t kb_gu = wbits == 8 ? (uint64_t)H : (uint64_t)H / 2;
-  uint64_t kb_dn = wbits == 8 ? (uint64_t)I : (uint64_t)I / 2;
+  if (E <= 0 || H <= 0 || I <= 0 || H % 128 || I % 128 || (wbits != 8 && wbits != 4 && wbits != 2)) return 1;
+  uint64_t kb_gu = code_bytes((uint64_t)H, wbits);
+  uint64_t kb_dn = code_bytes((uint64_t)I, wbits);
   uint64_t s_gu = g32 ? (uint64_t)(H / 32) * 2 : 4;
   uint64_t s_dn = g32 ? (uint64_t)(I / 32) * 2 : 4;
   off[0] = 0;
@@ -196,8 +212,10 @@ static void put_row(uint8_t* region, int rows_per_block, uint64_t kb, int64_t bl
 static void row_bytes(const int8_t* q, int K, int wbits, uint8_t* out) {
   if (wbits == 8) {
     for (int k = 0; k < K; ++k) out[k] = (uint8_t)q[k];
-  } else {
+  } else if (wbits == 4) {
     orc_pack_int4(q, 1, K, out);
+  } else {
+    orc_pack_int2(q, 1, K, out);
   }
 }
 
@@ -207,8 +225,8 @@ int orc_pack_blob(int E, int H, int I, int wbits, int g32, const int8_t* q_gu, c
   uint64_t off[5];
   if (orc_blob_layout(E, H, I, wbits, g32, off)) return 1;
   memset(blob, 0, off[4]);
-  uint64_t kb_gu = wbits == 8 ? (uint64_t)H : (uint64_t)H / 2;
-  uint64_t kb_dn = wbits == 8 ? (uint64_t)I : (uint64_t)I / 2;
+  uint64_t kb_gu = code_bytes((uint64_t)H, wbits);
+  uint64_t kb_dn = code_bytes((uint64_t)I, wbits);
   int Gg = H / 32, Gd = I / 32;
   uint8_t* rb = (uint8_t*)malloc(kb_gu > kb_dn ? kb_gu : kb_dn);
   for (int e = 0; e < E; ++e) {
@@ -231,7 +249,7 @@ int orc_pack_blob(int E, int H, int I, int wbits, int g32, const int8_t* q_gu, c
        128-row blocks [hb][piece][row][16 bytes]; g32 scales [slab][hb][2][row] */
     {
       const int U = I / 64, HB = H / 128;
-      const uint64_t sbytes = kb_dn / U;     /* code bytes of 64 elements: 64 or 32 */
+      const uint64_t sbytes = kb_dn / U;     /* code bytes of 64 elements: 64, 32 or 16 */
       for (int n = 0; n < H; ++n) {
         int64_t grow = (int64_t)e * H + n;
         int hb = n / 128, r = n % 128;

@@ -76,7 +76,16 @@ def test_int4_golden_group_and_packing():
     assert O.pack_int4(q)[0].tolist() == g["packed"]
 
 
-@pytest.mark.parametrize("qmax,g32", [(127, True), (127, False), (7, True), (7, False)])
+def test_int2_golden_group_and_packing():
+    g = gold("int2_group_example.json")
+    w = (np.array(g["m"], np.float64) * 2.0 ** -3).astype(np.float32)[None, :]
+    q, s = O.quantize_rows(w, O.QMAX[2], g32=True)
+    assert s[0, 0] == np.float32(g["scale"])
+    assert q[0].tolist() == g["q"]
+    assert O.pack_int2(q)[0].tolist() == g["packed"]
+
+
+@pytest.mark.parametrize("qmax,g32", [(127, True), (127, False), (7, True), (7, False), (1, True), (1, False)])
 def test_quantization_roundtrip_bound(qmax, g32):
     """|w - q*d| <= d/2 for every element, |q| <= Q, and each group's largest |w| maps to +-Q."""
     w = rng(qmax + g32).normal(0, 0.02, (64, 256)).astype(np.float32)
@@ -108,7 +117,22 @@ def test_int4_packing_bit_identical_to_int8_container():
     assert np.array_equal(un.astype(np.int64) @ a, q.astype(np.int64) @ a)
 
 
-@pytest.mark.parametrize("wbits,g32", [(8, True), (8, False), (4, True), (4, False)])
+def _unpack_int2(p):
+    p = p.astype(np.int16)
+    return np.stack([(((p >> (2 * i)) & 3) ^ 2) - 2 for i in range(4)], -1).reshape(p.shape[0], -1)
+
+
+def test_int2_packing_bit_identical_to_int8_container():
+    w = rng(7).normal(0, 0.02, (32, 512)).astype(np.float32)
+    q, _ = O.quantize_rows(w, O.QMAX[2], True)
+    assert set(np.unique(q).tolist()) == {-1, 0, 1}
+    un = _unpack_int2(O.pack_int2(q))
+    assert np.array_equal(un.astype(np.int8), q)
+    a = rng(8).integers(-127, 128, 512).astype(np.int64)
+    assert np.array_equal(un.astype(np.int64) @ a, q.astype(np.int64) @ a)
+
+
+@pytest.mark.parametrize("wbits,g32", [(8, True), (8, False), (4, True), (4, False), (2, True), (2, False)])
 def test_blob_decodes_to_codes_and_scales(wbits, g32):
     """The oracle's blob decodes (by reshapes) back to the logical codes and scales."""
     E, H, I = 2, 256, 128
@@ -124,10 +148,12 @@ def test_blob_decodes_to_codes_and_scales(wbits, g32):
         a = region.reshape(rows // block, kb // 16, block, 16).transpose(0, 2, 1, 3).reshape(rows, kb)
         if wbits == 8:
             return a.view(np.int8).reshape(rows, K)
+        if wbits == 2:
+            return _unpack_int2(a).reshape(rows, K).astype(np.int8)
         b = a.astype(np.int16)
         return np.stack([((b & 15) ^ 8) - 8, (((b >> 4) & 15) ^ 8) - 8], -1).reshape(rows, K).astype(np.int8)
 
-    kb_gu, kb_dn = (H, I) if wbits == 8 else (H // 2, I // 2)
+    kb_gu, kb_dn = H * wbits // 8, I * wbits // 8
     got_gu = codes(blob[off[0]:off[0] + E * 2 * I * kb_gu], E * 2 * I, 128, kb_gu, H)
     # row order inside each 128-row block: 64 gate rows then the matching 64 up rows
     order = np.concatenate([np.concatenate([np.arange(64 * s, 64 * s + 64),
@@ -141,6 +167,8 @@ def test_blob_decodes_to_codes_and_scales(wbits, g32):
     dn = dn.transpose(0, 2, 4, 1, 3, 5).reshape(E * H, kb_dn)
     if wbits == 8:
         got_dn = dn.view(np.int8).reshape(E * H, I)
+    elif wbits == 2:
+        got_dn = _unpack_int2(dn).reshape(E * H, I)
     else:
         b16 = dn.astype(np.int16)
         got_dn = np.stack([((b16 & 15) ^ 8) - 8, (((b16 >> 4) & 15) ^ 8) - 8], -1).reshape(E * H, I)
@@ -341,7 +369,8 @@ def _check_ffn_against_numpy(ex, e, qx, sx, ag32, got):
     assert np.allclose(got["ye"], wd @ hq, rtol=1e-12, atol=1e-18)
 
 
-@pytest.mark.parametrize("wbits,wg32,ag32", [(8, False, False), (8, True, True), (4, True, True), (4, False, True)])
+@pytest.mark.parametrize("wbits,wg32,ag32", [(8, False, False), (8, True, True), (4, True, True), (4, False, True),
+                                             (2, True, True), (2, False, True)])
 def test_single_expert_reproduces_dense_swiglu_ffn(wbits, wg32, ag32):
     """E = 1, k = 1, weight 1: the layer is one dense SwiGLU FFN on the quantized operands."""
     cfg = S.CONFIGS["olmoe_int8"].with_(H=256, I=128, E=1, top_k=1)
