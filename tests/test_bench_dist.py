@@ -55,3 +55,31 @@ def test_reference_arm_idle_off_rank_zero(monkeypatch):
     monkeypatch.setenv("RANK", "1")
     args = types.SimpleNamespace(steps=1, warmup=0)
     assert bench.reference_arm(args, None, 1) == 0
+
+
+def _reference_line(capsys, monkeypatch, *extra):
+    import json
+    monkeypatch.setenv("RANK", "0")
+    assert bench.main(["--impl", "reference", "--workload", "tiny:4", "--steps", "2", "--warmup", "3",
+                       *extra]) == 0
+    return json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+
+
+def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
+    """The oracle as the reference arm: one JSON line with the keys the benchmark contract
+    asks for, its cpu_baseline and e2e describing this run."""
+    d = _reference_line(capsys, monkeypatch)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["unit"] == "tok/s" and d["value"] > 0
+    assert d["higher_is_better"] is True and d["steps"] == 2 and d["warmup"] == 3
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert "workload" in d["config"] and "top-p" not in d["config"]["workload"]
+
+
+def test_reference_arm_with_adaptive_top_p(capsys, monkeypatch):
+    d = _reference_line(capsys, monkeypatch, "--top-p", "0.3")
+    assert d["value"] > 0 and "adaptive top-p 0.3" in d["config"]["workload"]
