@@ -483,7 +483,8 @@ def _topp_masses(L_t, sel, score):
     return np.exp(Lt[sel] - Lt[sel[0]]) if score == "softmax" else 1.0 / (1.0 + np.exp(-Lt[sel]))
 
 
-@pytest.mark.parametrize("score,renorm", [("softmax", True), ("softmax", False), ("sigmoid", True)])
+@pytest.mark.parametrize("score,renorm", [("softmax", True), ("softmax", False), ("sigmoid", True),
+                                          ("sigmoid", False)])
 @pytest.mark.parametrize("p", [0.3, 0.5, 0.7, 0.9])
 def test_topp_keeps_shortest_prefix_reaching_p(score, renorm, p):
     r = rng(40 + int(100 * p))
