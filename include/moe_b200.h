@@ -252,7 +252,8 @@ MOE_API size_t moe_layer_workspace_bytes(int32_t T, const moe_expert_blob* exper
  * Launch sequence: one token with group-32 activations (decode) is ONE launch: every CTA of
  * the expert kernel quantizes the token, computes the router logits of a share of the
  * experts and zeroes a share of y; after a grid barrier (all CTAs resident: the grid is at
- * most one CTA per SM) every CTA selects the same top-k and streams its work units. Other
+ * most one CTA per SM) every CTA selects the same top-k (with adaptive top-p: the same kept
+ * prefix, in a separate instantiation of that kernel) and streams its work units. Other
  * calls: for T <= 32 one routing kernel (activation quantization, logits, top-k and grouping;
  * the last CTA to finish its logit does the selection), larger T four; then, with group-32
  * activations, one expert kernel that covers the routed and the shared experts: per work unit
