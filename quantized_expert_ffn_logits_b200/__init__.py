@@ -209,14 +209,16 @@ def moe_quantize_experts_fp8(w_gate_up, s_gate_up, w_down, s_down, blob: ExpertB
     import torch
     E, I, H = blob.n_experts, blob.inter, blob.hidden
     cdiv = lambda a: (a + 127) // 128
-    for t, name, shape in ((w_gate_up, "w_gate_up", (E, 2 * I, H)), (w_down, "w_down", (E, H, I))):
+    codes = ((w_gate_up, "w_gate_up", (E, 2 * I, H)), (w_down, "w_down", (E, H, I)))
+    for t, name, shape in codes:
         if t.dtype not in (torch.uint8, torch.float8_e4m3fn) or tuple(t.shape) != shape:
             raise ValueError(f"{name}: want uint8/float8_e4m3fn {shape}, got {t.dtype} {tuple(t.shape)}")
+    if tuple(s_gate_up.shape) != (E, cdiv(2 * I), cdiv(H)) or tuple(s_down.shape) != (E, cdiv(H), cdiv(I)):
+        raise ValueError("block scales: want [E][ceil(2I/128)][ceil(H/128)] and [E][ceil(H/128)][ceil(I/128)]")
+    for t, name, _ in codes:
         _dev(t, t.dtype, name)
     _dev(s_gate_up, torch.float32, "s_gate_up")
     _dev(s_down, torch.float32, "s_down")
-    if tuple(s_gate_up.shape) != (E, cdiv(2 * I), cdiv(H)) or tuple(s_down.shape) != (E, cdiv(H), cdiv(I)):
-        raise ValueError("block scales: want [E][ceil(2I/128)][ceil(H/128)] and [E][ceil(H/128)][ceil(I/128)]")
     st = blob.struct()
     _check(_lib.moe_quantize_experts_fp8(_ptr(w_gate_up), _ptr(s_gate_up), _ptr(w_down), _ptr(s_down),
                                          C.byref(st), _stream(stream)), "moe_quantize_experts_fp8")

@@ -140,3 +140,23 @@ def test_build_entry_point_builds_and_checks_the_library():
         sys.path.insert(0, root)
     g = importlib.import_module("__graft_entry__")
     g.build()
+
+
+def test_fp8_binding_checks_shapes_and_devices():
+    """ExpertBlob.quantize_fp8's argument checks run on the host, before any launch."""
+    torch = pytest.importorskip("torch")
+
+    class _Blob:                                     # shape fields only: nothing is launched
+        n_experts, inter, hidden = 2, 128, 256
+    gu = torch.zeros((2, 256, 256), dtype=torch.uint8)
+    dn = torch.zeros((2, 256, 128), dtype=torch.uint8)
+    sgu = torch.ones((2, 2, 2))
+    sdn = torch.ones((2, 2, 1))
+    with pytest.raises(ValueError, match="w_gate_up"):
+        M.moe_quantize_experts_fp8(gu[:, :128], sgu, dn, sdn, _Blob())
+    with pytest.raises(ValueError, match="w_down"):
+        M.moe_quantize_experts_fp8(gu, sgu, dn.float(), sdn, _Blob())
+    with pytest.raises(ValueError, match="block scales"):
+        M.moe_quantize_experts_fp8(gu, sgu[:, :1], dn, sdn, _Blob())
+    with pytest.raises(ValueError, match="CUDA"):  # right shapes, but host tensors
+        M.moe_quantize_experts_fp8(gu, sgu, dn, sdn, _Blob())
