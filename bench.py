@@ -111,6 +111,52 @@ def layer_int_ops(cfg, T, pairs=None):
     return 2 * (pairs * 3 * cfg.H * cfg.I + T * 3 * cfg.H * cfg.shared_I)
 
 
+def step_plan(steps: int, period: int, event_steps: int):
+    """How the timed steps are replayed: CUDA graphs of G steps with no event nodes, n_main
+    replays of the G-step graph and then one graph of the rem remaining steps (n_main * G + rem
+    = steps). The Ge steps with per-stage event nodes (which cut the programmatic edges and add
+    ~3 us per stage) are a separate graph replayed after the timed region, never inside it."""
+    if steps < 1 or period < 1:
+        raise ValueError("steps and period must be >= 1")
+    G = min(steps, period)
+    n_main, rem = divmod(steps, G)
+    Ge = max(1, min(G, event_steps))
+    return G, n_main, rem, Ge
+
+
+def timed_replays(steps: int, period: int, event_steps: int):
+    """The graph replays of the timed region, in order: (graph, steps it runs, instrumented).
+    None of them carries event nodes, whatever the step counts."""
+    G, n_main, rem, _ = step_plan(steps, period, event_steps)
+    plan = [("graph", G, False)] * n_main
+    if rem:
+        plan.append(("graph_rem", rem, False))
+    return plan
+
+
+def expert_set_bytes(cfg) -> int:
+    """Blob bytes of one layer's experts (routed and shared: codes and scales)."""
+    b = cfg.E * (blob_row_bytes(cfg, cfg.H, 2 * cfg.I) + blob_row_bytes(cfg, cfg.I, cfg.H))
+    if cfg.shared_I:
+        b += blob_row_bytes(cfg, cfg.H, 2 * cfg.shared_I) + blob_row_bytes(cfg, cfg.shared_I, cfg.H)
+    return b
+
+
+def line_config(cfg, T, args, world=1):
+    """The `config` object of the JSON line: the workload and how it is stepped. Both arms
+    print the same object for the same arguments."""
+    G, n_main, rem, Ge = step_plan(args.steps, args.period, args.event_steps)
+    R = args.replicas
+    return {"workload": workload_desc(cfg, T, args.top_p), "T": T, "replicas": R,
+            "l2": f"inputs larger than L2: {R} layer replicas rotate "
+                  f"({R * expert_set_bytes(cfg) / 1e9:.2f} GB of expert blobs)",
+            "graph": f"timed steps replayed as CUDA graphs of {G} steps ({n_main} x {G}"
+                     f"{f' + {rem}' if rem else ''}) with no event nodes; per-stage events come "
+                     f"from {Ge} further steps replayed after the timed region",
+            "accumulate": "int32 dots, fp32 scales",
+            "parallelism": f"dp{world} (weak: independent tokens per GPU)"}
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 20 ms while running."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -287,10 +333,10 @@ def reference_arm(args, cfg, T):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(cfg, T, args.top_p), "T": T,
-                   "step": f"{units} (token, expert) units per step = {units / per_tok:g} tokens"},
+        "config": line_config(cfg, T, args, args.gpus),
         "cpu_baseline": {"value": value, "unit": "tok/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{args.steps} steps of {units} {desc}"},
+                         "sample": f"{args.steps} steps, each {units} {desc} "
+                                   f"({units / per_tok:g} tokens per step)"},
         "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -434,7 +480,8 @@ def gpu_arm(args, cfg, T):
             dist.barrier(device_ids=[local])
 
     R = args.replicas
-    rep_seeds, x_seeds = rank_seeds(rank, R, max(1, min(args.steps, args.period)))
+    G = step_plan(args.steps, args.period, args.event_steps)[0]
+    rep_seeds, x_seeds = rank_seeds(rank, R, G)
     rcfg = M.RouteCfg(score=cfg.score, top_k=cfg.top_k, renormalize=cfg.renormalize,
                       routed_scaling_factor=cfg.rsf, act=cfg.act, top_p=args.top_p)
     layers, n_active_of, kept_of = [], [], []
@@ -459,8 +506,7 @@ def gpu_arm(args, cfg, T):
         bias = torch.from_numpy(b).to(dev) if b is not None else None
         layers.append(M.Layer(T, blob, shared, rcfg, wr, bias))
     torch.cuda.synchronize()
-    # distinct token batches, resident in HBM before timing
-    G = max(1, min(args.steps, args.period))
+    # distinct token batches (one per step of a graph), resident in HBM before timing
     xs = []
     for s in range(G):
         xc = S.Case.make(cfg, T, seed=x_seeds[s])
@@ -481,13 +527,11 @@ def gpu_arm(args, cfg, T):
             layers[s % R](xs[s % G], y, stream)
     stream.synchronize()
 
-    # Graphs: `graph_ev` = the last Ge steps with every stage bracketed by CUDA events
-    # (external event nodes; they cut the programmatic edges around them, so these steps run
-    # slower), `graph` = G steps without events, `graph_rem` = the remainder. The timed region
-    # replays `graph` for the first K - Ge steps (an event between the two parts times them)
-    # and `graph_ev` for the last Ge, so the per-launch stage durations are read live from
-    # inside the timed region.
-    Ge = max(1, min(G, args.event_steps))
+    # Graphs (step_plan): `graph` = G steps and `graph_rem` = the remainder, neither with event
+    # nodes, are the timed region; `graph_ev` = Ge steps with every stage bracketed by CUDA
+    # events (external event nodes, which cut the programmatic edges around them) is replayed
+    # once after the timed region for the per-stage durations.
+    G, n_main, rem, Ge = step_plan(args.steps, args.period, args.event_steps)
     nst = len(M.MOE_STAGES)
     evs = []
     with torch.cuda.stream(stream):
@@ -512,7 +556,6 @@ def gpu_arm(args, cfg, T):
     with torch.cuda.graph(graph, stream=stream):
         for s in range(G):
             layers[s % R](xs[s], y, stream)
-    n_main, rem = divmod(args.steps - Ge, G)
     graph_rem = None
     if rem:
         graph_rem = torch.cuda.CUDAGraph()
@@ -536,19 +579,15 @@ def gpu_arm(args, cfg, T):
     clocks = ClockSampler(gpu_id)
     time.sleep(0.1)
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    mid = torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_push("timed")
     w0 = time.perf_counter()
+    graphs = {"graph": graph, "graph_rem": graph_rem}
     with torch.cuda.stream(stream):
         start.record(stream)
-        for _ in range(n_main):
-            graph.replay()
-        if graph_rem is not None:
-            graph_rem.replay()
-        mid.record(stream)
-        graph_ev.replay()
+        for name, _, _ in timed_replays(args.steps, args.period, args.event_steps):
+            graphs[name].replay()
         end.record(stream)
     stream.synchronize()
     w1 = time.perf_counter()
@@ -557,16 +596,16 @@ def gpu_arm(args, cfg, T):
     clocks.mark(w0, w1)
     clk = clocks.stop()
     ms_max = max_over_ranks(start.elapsed_time(end), world, dev)
-    main_steps = args.steps - Ge
-    ms_main = max_over_ranks(start.elapsed_time(mid), world, dev) if main_steps > 0 else None
 
-    # per-stage device times of the last graph period (inside the timed region)
+    # per-stage device times: the instrumented graph, replayed after the timed region
+    with torch.cuda.stream(stream):
+        graph_ev.replay()
+    stream.synchronize()
     stage_ms = {n: [] for n in M.MOE_STAGES}
-    if True:
-        for s in range(Ge):
-            for i, n in enumerate(M.MOE_STAGES):
-                b_ev, e_ev = evs[s][1][i]
-                stage_ms[n].append(b_ev.elapsed_time(e_ev))
+    for s in range(Ge):
+        for i, n in enumerate(M.MOE_STAGES):
+            b_ev, e_ev = evs[s][1][i]
+            stage_ms[n].append(b_ev.elapsed_time(e_ev))
     stage_us = {n: (1e3 * statistics.mean(v) if v else None) for n, v in stage_ms.items()}
 
     value = whole_job_rate(T, world, args.steps, ms_max)
@@ -579,15 +618,15 @@ def gpu_arm(args, cfg, T):
     gu_us = stage_us["gate_up"]
     gu_bytes = float(np.mean([(expert_bytes if fused else gateup_bytes)(cfg, T, a) for a in n_active_of]))
     one_launch = layers[0].kernels == 1
-    how = "gate/up stage events (the last Ge steps)"
+    how = (f"gate/up stage events of {Ge} instrumented steps replayed after the timed region "
+           f"(event nodes around the expert kernel: the duration includes its launch latency)")
     if one_launch:
-        # the kernel also reads the router weight and x and writes y
+        # one kernel per step (single-token routing inside it): it also reads the router weight
+        # and x and writes y, and its average launch duration is the event-free timed region
+        # over its launches
         gu_bytes = float(np.mean([layer_bytes(cfg, T, a) for a in n_active_of]))
-    if one_launch and ms_main:
-        # one kernel per step (single-token routing inside it): its average launch duration
-        # is the event-timed region without stage events over its launches
-        gu_us = ms_main * 1e3 / main_steps
-        how = f"one launch per step: events around the first {main_steps} timed steps / launches"
+        gu_us = ms_max * 1e3 / args.steps
+        how = f"one launch per step: CUDA events around the {args.steps} event-free timed steps / launches"
     roof = None
     if gu_us:
         ach = gu_bytes / (gu_us * 1e-6) / 1e9
@@ -650,11 +689,7 @@ def gpu_arm(args, cfg, T):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic",
-        "config": {"workload": workload_desc(cfg, T, args.top_p), "T": T, "replicas": R,
-                   "l2": f"inputs larger than L2: {R} layer replicas rotate "
-                         f"({R * layers[0].experts.nbytes / 1e9:.2f} GB of expert blobs)",
-                   "graph": f"CUDA graphs of {G} steps; the last {Ge} timed steps carry per-stage event nodes", "accumulate": "int32 dots, fp32 scales",
-                   "parallelism": f"dp{world} (weak: independent tokens per GPU)"},
+        "config": line_config(cfg, T, args, world),
         "roofline": roof,
         "layer": layer,
         "prefill": prefill,
@@ -747,7 +782,7 @@ def main(argv=None):
     ap.add_argument("--replicas", type=int, default=8, help="layer replicas rotated per step")
     ap.add_argument("--period", type=int, default=256, help="steps per captured graph")
     ap.add_argument("--event-steps", type=int, default=32,
-                    help="timed steps (the last ones) with per-stage event records")
+                    help="steps with per-stage event records, replayed after the timed region")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

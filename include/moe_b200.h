@@ -174,9 +174,6 @@ MOE_API size_t moe_expert_blob_bytes(int32_t wtype, int32_t wscale, int32_t n_ex
 MOE_API moe_status moe_quantize_experts(const float* w_gate_up, const float* w_down,
                                 const moe_expert_blob* out, void* stream);
 
-/* Q8_0-style activation quantization (GLM page, "Integer-dot kernels (Q8_0-style int8
- * activations ...)").  x [T][H] fp32 -> q [T][H] int8 and `scales`: fp16 [T][H/32]
- * (MOE_ACT_G32_F16) or fp32 [T] (MOE_ACT_TOKEN_F32). H multiple of 32. */
 /* The GLM-5.2 colibri page's FP8 -> int4 converter step, on the GPU: FP8 checkpoint weights
  * (float8 E4M3 codes, "fn" variant: no infinities) with one fp32 inverse scale per 128 x 128
  * block of each expert's matrix (the DeepSeek-V3-style layout) are dequantized -- value =
@@ -191,6 +188,9 @@ MOE_API moe_status moe_quantize_experts_fp8(const uint8_t* w_gate_up, const floa
                                             const uint8_t* w_down, const float* s_down,
                                             const moe_expert_blob* out, void* stream);
 
+/* Q8_0-style activation quantization (GLM page, "Integer-dot kernels (Q8_0-style int8
+ * activations ...)").  x [T][H] fp32 -> q [T][H] int8 and `scales`: fp16 [T][H/32]
+ * (MOE_ACT_G32_F16) or fp32 [T] (MOE_ACT_TOKEN_F32). H multiple of 32. */
 MOE_API moe_status moe_quantize_activations(const float* x, int32_t T, int32_t H, int32_t act,
                                     int8_t* q, void* scales, void* stream);
 

@@ -599,27 +599,13 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
 // -------------------------------------------------------------------- host side
 namespace {
 
-int sm_count_mma() {
-  static int n[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (n[dev] == 0) {
-    int v = 0;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    n[dev] = v > 0 ? v : 148;
-  }
-  return n[dev];
-}
+int sm_count_mma() { return device_sm_count(); }
 
 template <int WBITS, bool GATEUP>
 cudaError_t launch_mma_t(const MmaArgs& a, int max_items, cudaStream_t st) {
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(k_expert_mma<WBITS, GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMmaSmem);
+  {
+    const cudaError_t e = ensure_smem_attr((const void*)k_expert_mma<WBITS, GATEUP>, kMmaSmem);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   const int grid = std::max(1, std::min(max_items, sm_count_mma()));
   return launch_pdl(k_expert_mma<WBITS, GATEUP>, dim3(grid), dim3(kMmaThreads), (size_t)kMmaSmem, st, a);

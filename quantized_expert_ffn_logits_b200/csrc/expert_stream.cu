@@ -1298,18 +1298,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
 // ------------------------------------------------------------------ host side
 namespace {
 
-int sm_count() {
-  static int n[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (n[dev] == 0) {
-    int v = 0;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    n[dev] = v > 0 ? v : 148;
-  }
-  return n[dev];
-}
+int sm_count() { return device_sm_count(); }
 
 // MODE 3 grid: every unit its CTA, and at least one CTA per expert for the router logits (up
 // to one CTA per SM: the grid barrier needs all of them resident at once).
@@ -1318,12 +1307,9 @@ int decode_grid(int units, int E) { return std::min(sm_count(), std::max(units, 
 template <int WBITS, bool WG32, bool AG32, int MODE, int TM, bool TOPP = false>
 cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
   const RingPlan P = ring_plan(A.kmax, A.tm);
-  static int attr_bytes = 0;
-  if (P.total > attr_bytes) {
-    const cudaError_t e = cudaFuncSetAttribute(k_expert_ring<WBITS, WG32, AG32, MODE, TM, TOPP>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize, P.total);
+  {
+    const cudaError_t e = ensure_smem_attr((const void*)k_expert_ring<WBITS, WG32, AG32, MODE, TM, TOPP>, P.total);
     if (e != cudaSuccess) return e;
-    attr_bytes = P.total;
   }
   if constexpr (MODE == 3) {
     // one token: the logits shared per cluster (16 CTAs, else 8) when a CTA's share of the
@@ -1331,27 +1317,36 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
     // once (the y-zero barrier waits on all CTAs) with no fewer CTAs than the grid exchange
     // would use; else every CTA computes some logits and a grid barrier follows
     auto kern = k_expert_ring<WBITS, WG32, AG32, MODE, TM, TOPP>;
-    static int max_clusters[2] = {-1, -1}, max_clusters_smem = -1;
-    if (max_clusters_smem != P.total) {
-      (void)cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      for (int i = 0; i < 2; ++i) {
-        const int cs = i == 0 ? 16 : 8;
-        cudaLaunchConfig_t q = {};
-        cudaLaunchAttribute qa[1];
-        qa[0].id = cudaLaunchAttributeClusterDimension;
-        qa[0].val.clusterDim.x = cs;
-        qa[0].val.clusterDim.y = 1;
-        qa[0].val.clusterDim.z = 1;
-        q.gridDim = dim3(cs * 8);
-        q.blockDim = dim3(kNT);
-        q.dynamicSmemBytes = (size_t)P.total;
-        q.attrs = qa;
-        q.numAttrs = 1;
-        int n = 0;
-        max_clusters[i] = cudaOccupancyMaxActiveClusters(&n, kern, &q) == cudaSuccess ? n : 0;
+    const int dev = current_device();
+    if (dev < 0) return cudaErrorInvalidDevice;
+    // most co-resident clusters of 16 and of 8 CTAs, per device (for this shared-memory size)
+    static int cached_clusters[kMaxDevices][2], cached_smem[kMaxDevices];
+    int max_clusters[2];
+    {
+      std::lock_guard<std::mutex> lk(setup_mutex());     // released before sm_count() below
+      if (cached_smem[dev] != P.total) {
+        (void)cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        for (int i = 0; i < 2; ++i) {
+          const int cs = i == 0 ? 16 : 8;
+          cudaLaunchConfig_t q = {};
+          cudaLaunchAttribute qa[1];
+          qa[0].id = cudaLaunchAttributeClusterDimension;
+          qa[0].val.clusterDim.x = cs;
+          qa[0].val.clusterDim.y = 1;
+          qa[0].val.clusterDim.z = 1;
+          q.gridDim = dim3(cs * 8);
+          q.blockDim = dim3(kNT);
+          q.dynamicSmemBytes = (size_t)P.total;
+          q.attrs = qa;
+          q.numAttrs = 1;
+          int n = 0;
+          cached_clusters[dev][i] = cudaOccupancyMaxActiveClusters(&n, kern, &q) == cudaSuccess ? n : 0;
+        }
+        cached_smem[dev] = P.total;
+        (void)cudaGetLastError();
       }
-      max_clusters_smem = P.total;
-      (void)cudaGetLastError();
+      max_clusters[0] = cached_clusters[dev][0];
+      max_clusters[1] = cached_clusters[dev][1];
     }
     const int grid_x = decode_grid(A.units, A.r.E);          // grid exchange
     const int need = std::min(std::max(A.units, 1), sm_count());

@@ -2,11 +2,20 @@
 #pragma once
 
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
 
 namespace moe {
+
+// ---- host_setup.cu: per-device host-side setup (attributes and properties are per device;
+// the caches are keyed by the current device and guarded by setup_mutex())
+constexpr int kMaxDevices = 64;
+int current_device();                                   // -1 if unknown or >= kMaxDevices
+int device_sm_count();                                  // SMs of the current device
+cudaError_t ensure_smem_attr(const void* kernel, int bytes);   // dynamic smem limit >= bytes
+std::mutex& setup_mutex();
 
 // ---- quantize.cu
 void launch_quantize_experts(const float* w_gu, const float* w_dn, const BlobView& b,

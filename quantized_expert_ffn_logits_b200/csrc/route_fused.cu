@@ -304,12 +304,9 @@ cudaError_t launch_route_fused(const RouteArgs& r, cudaStream_t st) {
   int E = r.E;
 #define MOE_ROUTE_CASE(N)                                                                  \
   do {                                                                                     \
-    static size_t attr_bytes = 48 * 1024;                                                  \
-    if (smem > attr_bytes) {                                                               \
-      const cudaError_t e = cudaFuncSetAttribute(                                          \
-          k_route_fused<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);       \
+    if (smem > 48 * 1024) {                                                                \
+      const cudaError_t e = ensure_smem_attr((const void*)k_route_fused<N>, (int)smem);    \
       if (e != cudaSuccess) return e;                                                      \
-      attr_bytes = smem;                                                                   \
     }                                                                                      \
     return launch_pdl(k_route_fused<N>, dim3(E), dim3(256), smem, st, r);                              \
   } while (0)

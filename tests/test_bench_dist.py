@@ -83,3 +83,27 @@ def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
 def test_reference_arm_with_adaptive_top_p(capsys, monkeypatch):
     d = _reference_line(capsys, monkeypatch, "--top-p", "0.3")
     assert d["value"] > 0 and "adaptive top-p 0.3" in d["config"]["workload"]
+
+
+def test_timed_region_has_no_instrumented_step():
+    """Every timed step is an event-free graph replay, whatever --steps, --period and
+    --event-steps are (the driver's --steps 20 is below the default --event-steps 32), and the
+    replays add up to exactly --steps."""
+    for steps in (1, 3, 19, 20, 31, 32, 33, 255, 256, 257, 5000):
+        for period in (1, 16, 20, 64, 256):
+            for ev in (1, 16, 20, 32, 64):
+                G, n_main, rem, Ge = bench.step_plan(steps, period, ev)
+                assert n_main * G + rem == steps and 0 <= rem < G and 1 <= Ge <= G
+                plan = bench.timed_replays(steps, period, ev)
+                assert sum(n for _, n, _ in plan) == steps
+                assert not any(inst for _, _, inst in plan), (steps, period, ev)
+                assert {name for name, _, _ in plan} <= {"graph", "graph_rem"}
+
+
+def test_both_arms_print_the_same_config(capsys, monkeypatch):
+    """The reference arm's config object is the one the GPU arm prints for the same arguments."""
+    d = _reference_line(capsys, monkeypatch)
+    cfg, T = bench.parse_workload("tiny:4")
+    ns = types.SimpleNamespace(steps=2, warmup=3, period=256, event_steps=32, replicas=8, top_p=0.0)
+    assert d["config"] == bench.line_config(cfg, T, ns, 1)
+    assert "no event nodes" in d["config"]["graph"]
