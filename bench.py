@@ -585,6 +585,10 @@ def gpu_arm(args, cfg, T):
     w0 = time.perf_counter()
     graphs = {"graph": graph, "graph_rem": graph_rem}
     with torch.cuda.stream(stream):
+        # a ~50 us spin ahead of the start event keeps the GPU busy while the host submits
+        # the graph replays, so the timed region holds device time only (no submission
+        # latency between the start event and the first step)
+        torch.cuda._sleep(100_000)
         start.record(stream)
         for name, _, _ in timed_replays(args.steps, args.period, args.event_steps):
             graphs[name].replay()

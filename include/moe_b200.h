@@ -65,7 +65,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 2
+#define MOE_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -93,11 +93,15 @@ enum { MOE_ACT_TOKEN_F32 = 0, MOE_ACT_G32_F16 = 1 };
 enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID_NOAUX_TC = 1 };
 
 /* moe_route_cfg.flags */
-#define MOE_FLAG_DEBUG 1u          /* also keep gate/up stage values and per-pair down values
-                                      in the workspace (see moe_layer_debug_views) */
+#define MOE_FLAG_DEBUG 1u          /* also keep gate/up stage values, per-pair down values and
+                                      the down projection's int32 group dots in the workspace
+                                      (see moe_layer_debug_views) */
 #define MOE_FLAG_FORCE_GEMV 2u     /* run every expert on the weight-streaming (GEMV) path */
 #define MOE_FLAG_FORCE_MMA 4u      /* T > 32: run every expert (shared one included) with at least
                                       one pair on the tensor-core path (normally: >= 16 pairs) */
+#define MOE_FLAG_SHORT_WAITS 8u    /* the single-token kernel's waits on other CTAs (its grid
+                                      barrier) give up after about 2 ms instead of about a second
+                                      (MOE_ERR_TIMEOUT): for testing the timeout path */
 
 /* A set of E quantized experts of one layer (or the single shared expert, E = 1).
  *
@@ -339,6 +343,11 @@ typedef struct {
   int64_t up;           /* MOE_FLAG_DEBUG: fp32, same shape */
   int64_t y_pair;       /* MOE_FLAG_DEBUG: fp32 [T*k][H] then [T][H]: expert outputs before
                            the combine */
+  int64_t dn_dots;      /* MOE_FLAG_DEBUG: int32 [T*k][H][I/32] then [T][H][I_shared/32]: the
+                           exact int32 group dots of the down projection (row n of the down
+                           matrix against the pair's q_h, per group of 32), as the expert kernel
+                           that ran the pair formed them; entries of dropped slots are 0. Size
+                           4 * H * (T*k*I + T*I_shared) / 32 bytes. */
   int64_t total;        /* == moe_layer_workspace_bytes() */
 } moe_debug_views;
 
@@ -360,7 +369,8 @@ MOE_API moe_status moe_expert_group_dots(const moe_expert_blob* blob, int32_t wh
  * stage or buffer << 8, with wait 0 = producer waiting for a free stage, 1 = consumer waiting
  * for a chunk, 2 / 4 = producer draining chunks / activation copies before exit, 3 = producer
  * waiting for a free activation buffer, 5 = consumer waiting for activation rows, 6 = the
- * single-token kernel's grid barrier, 7 = its staged router rows;
+ * single-token kernel's grid barrier, 7 = its staged router rows, 8 = the y-zero barrier of its
+ * cluster variant (logits exchanged within clusters of CTAs, y zeroed before any CTA adds);
  * [3] = the CTA index; both 0 otherwise. After MOE_ERR_TIMEOUT the routing ticket and the
  * grid-barrier counter may be mid-call: reading the status resets them (not words 2-3).
  * Reads and clears the device status word of a moe_layer_forward / moe_permute workspace.
@@ -376,8 +386,8 @@ MOE_API moe_status moe_get_device_status(void* workspace, void* stream);
 /* moe_layer_forward with MOE_FLAG_DEBUG added to cfg->flags (so the workspace must hold
  * moe_layer_workspace_bytes() of that configuration), and `views` filled as
  * moe_layer_debug_views() fills it: byte offsets, inside `workspace`, of the call's
- * intermediates (quantized x, logits, idx, w, grouping, quantized h, gate/up stage values and
- * per-pair down values). Sampled int32 group dots come from moe_expert_group_dots. Errors as
+ * intermediates (quantized x, logits, idx, w, grouping, quantized h, gate/up stage values,
+ * per-pair down values and the down projection's int32 group dots). Errors as
  * moe_layer_forward, plus INVALID_ARG for a null cfg or views; views is written only when the
  * call returns MOE_OK with T > 0. */
 MOE_API moe_status moe_layer_forward_debug(const float* x, int32_t T, const float* router_w,

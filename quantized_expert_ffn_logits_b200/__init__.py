@@ -27,7 +27,7 @@ MOE_W_INT8, MOE_W_INT4 = 0, 1
 MOE_SCALE_ROW_F32, MOE_SCALE_G32_F16 = 0, 1
 MOE_ACT_TOKEN_F32, MOE_ACT_G32_F16 = 0, 1
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID_NOAUX_TC = 0, 1
-MOE_FLAG_DEBUG, MOE_FLAG_FORCE_GEMV, MOE_FLAG_FORCE_MMA = 1, 2, 4
+MOE_FLAG_DEBUG, MOE_FLAG_FORCE_GEMV, MOE_FLAG_FORCE_MMA, MOE_FLAG_SHORT_WAITS = 1, 2, 4, 8
 
 WTYPES = {"int8": MOE_W_INT8, "int4": MOE_W_INT4}
 WSCALES = {"row_f32": MOE_SCALE_ROW_F32, "g32_f16": MOE_SCALE_G32_F16}
@@ -50,7 +50,7 @@ class moe_route_cfg(C.Structure):
 class moe_debug_views(C.Structure):
     _fields_ = [(n, C.c_int64) for n in ("status", "q_x", "s_x", "logits", "idx", "w", "offsets",
                                           "perm", "n_active", "act_expert", "q_h", "s_h", "gate",
-                                          "up", "y_pair", "total")]
+                                          "up", "y_pair", "dn_dots", "total")]
 
 
 MOE_STAGES = ("quant_x", "router", "topk", "group", "gate_up", "quant_h", "down")
@@ -93,7 +93,7 @@ for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
     _fn.argtypes = _args
-ABI_VERSION = 2          # the struct layouts above (moe_route_cfg with top_p)
+ABI_VERSION = 3          # the struct layouts above (moe_route_cfg with top_p, moe_debug_views with dn_dots)
 if _lib.moe_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH}: ABI version {_lib.moe_abi_version()}, this binding needs "
                       f"{ABI_VERSION}: rebuild the library")

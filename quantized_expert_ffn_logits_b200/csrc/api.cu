@@ -16,6 +16,11 @@ using moe::BlobView;
 
 inline int64_t al256(int64_t v) { return (v + 255) & ~int64_t(255); }
 
+// Bounds of the single-token kernel's cross-CTA waits (grid barrier, y-zero barrier): about
+// a second, or 2 ms with MOE_FLAG_SHORT_WAITS.
+constexpr unsigned long long kWaitNs = 1000000000ull;
+constexpr unsigned long long kShortWaitNs = 2000000ull;
+
 // Batches up to this many tokens take the single-launch routing kernel.
 constexpr int32_t kFusedRouteMaxT = 32;
 // Control block at the start of a layer workspace: status word, routing ticket, wait record
@@ -83,11 +88,11 @@ float topp_of(const moe_route_cfg* c) { return (c->top_p > 0.0f && c->top_p < 1.
 // Workspace of one layer forward: every region starts at a multiple of 256 bytes.
 struct Layout {
   int64_t status, qx, sx, logits, idx, w, offsets, perm, n_active, act_expert, act_begin, act_rows;
-  int64_t masks, base, qh, sh, hbuf, dbg_gate, dbg_up, dbg_y, total;
+  int64_t masks, base, qh, sh, hbuf, dbg_gate, dbg_up, dbg_y, dbg_dots, total;
   // tensor-core path (T > 32, group-32 weights and activations)
   int64_t mm_tiles, mm_ntiles, mm_xa, mm_xs, mm_ha, mm_hs;
   int32_t mm_max_tiles, mm_min_tokens, mm_hk;
-  int64_t qh_sh, sh_sh, hbuf_sh, dbg_gate_sh, dbg_up_sh, dbg_y_sh;   // shared-expert rows
+  int64_t qh_sh, sh_sh, hbuf_sh, dbg_gate_sh, dbg_up_sh, dbg_y_sh, dbg_dots_sh;   // shared-expert rows
 };
 
 Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k, int32_t ag32,
@@ -138,9 +143,11 @@ Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k,
     L.dbg_up_sh = L.dbg_up + P * I * 4;
     L.dbg_y = take((P + T) * H * 4);
     L.dbg_y_sh = L.dbg_y + P * H * 4;
+    L.dbg_dots = take((P * (I / 32) + (int64_t)T * (Is / 32)) * H * 4);
+    L.dbg_dots_sh = L.dbg_dots + P * H * (I / 32) * 4;
   } else {
-    L.dbg_gate = L.dbg_up = L.dbg_y = -1;
-    L.dbg_gate_sh = L.dbg_up_sh = L.dbg_y_sh = -1;
+    L.dbg_gate = L.dbg_up = L.dbg_y = L.dbg_dots = -1;
+    L.dbg_gate_sh = L.dbg_up_sh = L.dbg_y_sh = L.dbg_dots_sh = -1;
   }
   L.mm_max_tiles = 0;
   L.mm_min_tokens = force_mma ? 1 : moe::kMmaMinTokens;
@@ -392,6 +399,7 @@ moe_status moe_layer_debug_views(int32_t T, const moe_expert_blob* experts,
   out->gate = L.dbg_gate;
   out->up = L.dbg_up;
   out->y_pair = L.dbg_y;
+  out->dn_dots = L.dbg_dots;
   out->total = L.total;
   return MOE_OK;
 }
@@ -492,6 +500,7 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     r.status = status;
     r.ticket = reinterpret_cast<unsigned*>(ws + L.status + 4);
     r.gbar = reinterpret_cast<unsigned long long*>(ws + L.status + 16);
+    r.wait_ns = (cfg->flags & MOE_FLAG_SHORT_WAITS) ? kShortWaitNs : kWaitNs;
     mk.begin(MOE_STAGE_QUANT_X);
     if (!decode) keep(moe::launch_route_fused(r, st), "routing kernel");
     mk.end(MOE_STAGE_QUANT_X);
@@ -566,18 +575,23 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   rd.sa = at(L.sh);
   rd.dbg_a = static_cast<float*>(at(L.dbg_y));
   rd.dbg_b = nullptr;
+  rd.dbg_dots = static_cast<int32_t*>(at(L.dbg_dots));
   moe::ExpertArgs sd = sa;
   if (shared) {
     sd.qa = static_cast<const int8_t*>(at(L.qh_sh));
     sd.sa = at(L.sh_sh);
     sd.dbg_a = static_cast<float*>(at(L.dbg_y_sh));
     sd.dbg_b = nullptr;
+    sd.dbg_dots = static_cast<int32_t*>(at(L.dbg_dots_sh));
   }
   const moe::ExpertArgs* sap = shared ? &sa : nullptr;
   const moe::ExpertArgs* sdp = shared ? &sd : nullptr;
   // the down kernels add each unit's share of a pair's down value into the pair's view
   if (L.dbg_y >= 0)
     keep(cudaMemsetAsync(ws + L.dbg_y, 0, (size_t)((int64_t)(T * k + T) * H * 4), st), "debug view reset");
+  if (L.dbg_dots >= 0)
+    keep(cudaMemsetAsync(ws + L.dbg_dots, 0, (size_t)(((int64_t)T * k * (I / 32) + (int64_t)T * (p.Is / 32)) * H * 4), st),
+         "debug dots reset");
   // experts with many slots: tensor-core GEMMs (tile list, operand gather, gate/up, down)
   const int mma_min = p.mma ? L.mm_min_tokens : 0x7fffffff;
   auto launch_mma = [&](bool down) {
@@ -606,6 +620,8 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     m.y = y;
     m.dbg_y[0] = rd.dbg_a;
     m.dbg_y[1] = shared ? sd.dbg_a : nullptr;
+    m.dbg_dots[0] = rd.dbg_dots;
+    m.dbg_dots[1] = shared ? sd.dbg_dots : nullptr;
     m.T = T;
     m.k = k;
     m.status = status;

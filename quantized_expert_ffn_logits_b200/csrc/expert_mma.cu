@@ -182,6 +182,12 @@ constexpr int kMmaNB = 4;                  // tensor-memory accumulators (128 fp
                                            // all 512; one CTA per SM), so MMAs run 4 groups ahead
 constexpr int kMmaPrepWarps = 2;
 constexpr uint32_t kMmaSleepNs = 200;      // backoff of the roles that run ahead of the epilogue
+// One accumulator hand-off per 2-group stage: the MMA issuer fills a pair of accumulators
+// (groups 2i, 2i + 1) and commits once; the epilogue waits once, drains both, releases once.
+constexpr bool kMmaPairCommit = true;
+// Weight blocks are re-read by every tile of their expert: normal L2 policy, not evict-first
+// (measured: the same time either way at 4096 tokens).
+constexpr bool kMmaWeightsEvictFirst = false;
 constexpr int kMmaEpiWarps = 16;
 constexpr int kMmaEpi0 = 2 + kMmaPrepWarps;                       // first epilogue warp
 constexpr int kMmaThreads = (kMmaEpi0 + kMmaEpiWarps) * 32;       // producer, MMA, prep, epilogue
@@ -288,16 +294,19 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
           mbar_arrive_expect_tx(&full[s], mma_stage_bytes<WBITS>());
           bulk_load(st + MmaStage::AH, a_src + (int64_t)g0 * 4 * 2048, 16384, &full[s]);
           bulk_load(st + MmaStage::AS, as_src + (int64_t)g0 * 128, 512, &full[s]);
+          auto load_w = [&](void* dst, const void* src, uint32_t bytes) {
+            if (kMmaWeightsEvictFirst) bulk_load_hint(dst, src, bytes, &full[s], once);
+            else bulk_load(dst, src, bytes, &full[s]);
+          };
           if (GATEUP) {
             const int64_t blk = (int64_t)tl.w * 2 * bv.I + (int64_t)blkn * 128;
-            bulk_load_hint(st + MmaStage::B8, bv.gu_w + blk * KB + (int64_t)g0 * PPG * 2048, kMmaKC * PPG * 2048,
-                           &full[s], once);
-            bulk_load_hint(st + MmaStage::BS, bv.gu_s + (blk * G + (int64_t)g0 * 128) * 2, 512, &full[s], once);
+            load_w(st + MmaStage::B8, bv.gu_w + blk * KB + (int64_t)g0 * PPG * 2048, kMmaKC * PPG * 2048);
+            load_w(st + MmaStage::BS, bv.gu_s + (blk * G + (int64_t)g0 * 128) * 2, 512);
           } else {
             const int U = bv.I / 64, HB = bv.H / 128;
             const int64_t slab = ((int64_t)tl.w * U + g0 / 2) * HB + blkn;
-            bulk_load_hint(st + MmaStage::B8, bv.dn_w + slab * PPU * 2048, PPU * 2048, &full[s], once);
-            bulk_load_hint(st + MmaStage::BS, bv.dn_s + slab * 512, 512, &full[s], once);
+            load_w(st + MmaStage::B8, bv.dn_w + slab * PPU * 2048, PPU * 2048);
+            load_w(st + MmaStage::BS, bv.dn_s + slab * 512, 512);
           }
         }
       }
@@ -331,22 +340,43 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
           }
           tc_fence_after();
           const uint8_t* st = base + s * MmaStage::BYTES;
-          for (int j = 0; j < kMmaKC; ++j, ++gi) {
-            const int bb = gi % kMmaNB;
-            if (ok && gi >= (uint32_t)kMmaNB && !mbar_wait_sleep(&acc_empty[bb], ((gi / kMmaNB) - 1) & 1, kMmaSleepNs)) {
+          if constexpr (kMmaPairCommit) {
+            // the stage's two groups into accumulator pair pr (buffers 2 pr, 2 pr + 1)
+            const uint32_t pr = c & 1;
+            if (ok && c >= 2 && !mbar_wait_sleep(&acc_empty[pr], ((c >> 1) - 1) & 1, kMmaSleepNs)) {
               *abort = 1;
-              wait_failed(A.status, kKern, 3, bb);
+              wait_failed(A.status, kKern, 3, pr);
               ok = false;
             }
             tc_fence_after();
-            if (ok) {
-              // group j: fp16 pieces 4j .. 4j + 3, two MMAs of K = 16 (exact integer dot)
-              const uint8_t* a = st + MmaStage::AH + j * 8192;
-              const uint8_t* b = st + MmaStage::BH + j * 8192;
-              mma_f16(tmem + bb * 128, smem_desc(a, 2048, 128), smem_desc(b, 2048, 128), idesc, 0);
-              mma_f16(tmem + bb * 128, smem_desc(a + 4096, 2048, 128), smem_desc(b + 4096, 2048, 128), idesc, 1);
+            if (ok)
+              for (int j = 0; j < kMmaKC; ++j) {
+                const uint8_t* a = st + MmaStage::AH + j * 8192;
+                const uint8_t* b = st + MmaStage::BH + j * 8192;
+                const uint32_t d = tmem + (2 * pr + j) * 128;
+                mma_f16(d, smem_desc(a, 2048, 128), smem_desc(b, 2048, 128), idesc, 0);
+                mma_f16(d, smem_desc(a + 4096, 2048, 128), smem_desc(b + 4096, 2048, 128), idesc, 1);
+              }
+            mma_commit(&acc_full[pr]);           // arrives (in order) even when skipped
+            gi += kMmaKC;
+          } else {
+            for (int j = 0; j < kMmaKC; ++j, ++gi) {
+              const int bb = gi % kMmaNB;
+              if (ok && gi >= (uint32_t)kMmaNB && !mbar_wait_sleep(&acc_empty[bb], ((gi / kMmaNB) - 1) & 1, kMmaSleepNs)) {
+                *abort = 1;
+                wait_failed(A.status, kKern, 3, bb);
+                ok = false;
+              }
+              tc_fence_after();
+              if (ok) {
+                // group j: fp16 pieces 4j .. 4j + 3, two MMAs of K = 16 (exact integer dot)
+                const uint8_t* a = st + MmaStage::AH + j * 8192;
+                const uint8_t* b = st + MmaStage::BH + j * 8192;
+                mma_f16(tmem + bb * 128, smem_desc(a, 2048, 128), smem_desc(b, 2048, 128), idesc, 0);
+                mma_f16(tmem + bb * 128, smem_desc(a + 4096, 2048, 128), smem_desc(b + 4096, 2048, 128), idesc, 1);
+              }
+              mma_commit(&acc_full[bb]);         // arrives (in order) even when skipped
             }
-            mma_commit(&acc_full[bb]);         // arrives (in order) even when skipped
           }
           mma_commit(&empty[s]);
         }
@@ -460,25 +490,50 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
         const uint8_t* st = base + s * MmaStage::BYTES;
         const __half* as = reinterpret_cast<const __half*>(st + MmaStage::AS);
         const float* bsf = reinterpret_cast<const float*>(st + MmaStage::BSF);
-#pragma unroll
-        for (int j = 0; j < kMmaKC; ++j, ++gi) {
-          const int bb = gi % kMmaNB;
-          if (ok && !mbar_wait(&acc_full[bb], (gi / kMmaNB) & 1)) {
+        const uint32_t pr = c & 1;            // pair mode: the stage's accumulator pair
+        if (kMmaPairCommit) {
+          if (ok && !mbar_wait(&acc_full[pr], (c >> 1) & 1)) {
             *abort = 1;
-            if (lane == 0) wait_failed(A.status, kKern, 6, bb);
+            if (lane == 0) wait_failed(A.status, kKern, 6, pr);
             ok = false;
           }
           ok = __all_sync(0xffffffffu, ok);
           tc_fence_after();
+        }
+#pragma unroll
+        for (int j = 0; j < kMmaKC; ++j, ++gi) {
+          const int bb = kMmaPairCommit ? (int)(2 * pr + j) : (int)(gi % kMmaNB);
+          if (!kMmaPairCommit) {
+            if (ok && !mbar_wait(&acc_full[bb], (gi / kMmaNB) & 1)) {
+              *abort = 1;
+              if (lane == 0) wait_failed(A.status, kKern, 6, bb);
+              ok = false;
+            }
+            ok = __all_sync(0xffffffffu, ok);
+            tc_fence_after();
+          }
           uint32_t d0[16], d1[16];
           if (ok) {
             tmem_ld16(tq + bb * 128 + colA, d0);
             tmem_ld16(tq + bb * 128 + colB, d1);
             tmem_wait_ld();
           }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[bb]);
+          if (!kMmaPairCommit || j == kMmaKC - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[kMmaPairCommit ? (int)pr : bb]);
+          }
+          if (!GATEUP && A.dbg_dots[sh] && ok && t < tl.z) {
+            // debug: the down GEMM's exact group dots (fp32 integers) of output rows
+            // n0 .. n0 + 31 for this slot, group g0 + j
+            const int GI = K / 32, n0 = blkn * 128 + 32 * cs;
+            int32_t* dd = A.dbg_dots[sh] + ((int64_t)(tl.y + t) * H + n0) * GI + g0 + j;
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              dd[(int64_t)q * GI] = (int32_t)__uint_as_float(d0[q]);
+              dd[(int64_t)(16 + q) * GI] = (int32_t)__uint_as_float(d1[q]);
+            }
+          }
           if (ok) {
             // acc = fma((float)I_g, s_w * s_x, acc) per element, two elements per packed op; the
             // tensor cores already produced (float)I_g exactly

@@ -251,8 +251,16 @@ struct RouteSmem {
   volatile int* nk;                       // slots kept: k, or the adaptive top-p prefix
 };
 
-// Bound of the grid-barrier wait: 2^22 polls (each an L2 round trip: seconds in all).
+// Bounds of the cross-CTA waits (grid barrier, y-zero barrier): RouteArgs::wait_ns of
+// %globaltimer time (about a second by default), and at most 2^22 polls (each an L2 round
+// trip) whatever the timer reads.
 constexpr uint32_t kGridWaitTries = 1u << 22;
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
   unsigned long long v;
@@ -260,23 +268,33 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   return v;
 }
 
-// Thread 0 of every CTA, after a CTA barrier: arrive, then wait until every CTA of the grid
-// has arrived. The counter is a multiple of 1024 when a call starts (grids are <= 1024
-// CTAs); this call's arrivals take base .. base + grid - 1 and the last one moves the
-// counter on to base + 1024 for the next call. False if the wait gave up.
 __device__ __forceinline__ unsigned long long atom_add_release(unsigned long long* p, unsigned long long v) {
   unsigned long long old;
   asm volatile("atom.release.gpu.global.add.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
   return old;
 }
 
-__device__ __forceinline__ bool grid_barrier(unsigned long long* ctr) {
+// Poll until *p >= target; false once wait_ns have passed (checked every 32 polls) or the
+// poll bound ran out.
+__device__ __forceinline__ bool wait_counter(const unsigned long long* p, unsigned long long target,
+                                             unsigned long long wait_ns) {
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t i = 0; i < kGridWaitTries; ++i) {
+    if (ld_acquire_u64(p) >= target) return true;
+    if ((i & 31u) == 31u && globaltimer_ns() - t0 > wait_ns) return false;
+  }
+  return false;
+}
+
+// Thread 0 of every CTA, after a CTA barrier: arrive, then wait until every CTA of the grid
+// has arrived. The counter is a multiple of 1024 when a call starts (grids are <= 1024
+// CTAs); this call's arrivals take base .. base + grid - 1 and the last one moves the
+// counter on to base + 1024 for the next call. False if the wait gave up.
+__device__ __forceinline__ bool grid_barrier(unsigned long long* ctr, unsigned long long wait_ns) {
   const unsigned long long old = atom_add_release(ctr, 1ull);   // the CTA's writes before it
   const unsigned long long target = (old & ~1023ull) + gridDim.x;
   if (old + 1 == target) atomicAdd(ctr, 1024ull - gridDim.x);
-  for (uint32_t i = 0; i < kGridWaitTries; ++i)
-    if (ld_acquire_u64(ctr) >= target) return true;
-  return false;
+  return wait_counter(ctr, target, wait_ns);
 }
 
 // Scratch use of the (still idle) ring during the routing. The logit of a 32-element chunk
@@ -458,7 +476,7 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
   float* slog = reinterpret_cast<float*>(R.ring);           // scratch again: [E] logits
   float* skey = slog + 512;                                  //                [E] selection keys
   if (!cl) {
-    if (tid == 0) *flag = grid_barrier(r.gbar) ? 1 : 0;
+    if (tid == 0) *flag = grid_barrier(r.gbar, r.wait_ns) ? 1 : 0;
     __syncthreads();
     if (!*flag) {
       if (tid == 0) wait_failed(r.status, 1, 6, 0);
@@ -947,13 +965,14 @@ __device__ __forceinline__ void ring_consume(int K, int m, int tm, const Ring& R
 // rows t, t + 256, ... of the chunk (int8: 2 rows, int4: 4). Per (row, token) the two group
 // dots against the unit's 64 h codes give this unit's share of the row's down value
 // (fp32, any order), weighted and added into y (and, for inspection, into the pair's
-// down value). hx: the pass's h codes [tm][64] (int4 weights: each 8-byte word
+// down value, and its two exact group dots into the debug view [slot][H][I/32] at groups
+// 2 sub, 2 sub + 1). hx: the pass's h codes [tm][64] (int4 weights: each 8-byte word
 // de-interleaved), hxs: per-group code sums [tm][2] (int4), hs: h scales [tm][2].
 template <int WBITS, bool WG32, bool AG32, int TM>
 __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& R, uint32_t& c, const uint8_t* hx,
                                              const int* hxs, const float* hs, const int* toks,
-                                             const float* wts, float* y, float* dbg, int slot0,
-                                             volatile int* abort, int* status) {
+                                             const float* wts, float* y, float* dbg, int32_t* ddots, int GI,
+                                             int sub, int slot0, volatile int* abort, int* status) {
   constexpr int PPU = WBITS == 8 ? 4 : 2;
   constexpr int NBC = kSP / PPU;
   constexpr int RPT = NBC * kRows / (32 * kCW);   // rows per thread of a full chunk
@@ -999,6 +1018,7 @@ __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& 
         const float wq = wts[q];
         float* yq = y + (int64_t)toks[q] * H;
         float* dq = dbg ? dbg + (int64_t)(slot0 + q) * H : nullptr;
+        int32_t* tq = ddots ? ddots + (int64_t)(slot0 + q) * H * GI + 2 * sub : nullptr;
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
           const int rr = threadIdx.x + 32 * kCW * k, b = rr >> 7, r = rr & 127;
@@ -1030,6 +1050,10 @@ __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& 
           const float w3 = __shfl_down_sync(0xffffffffu, wv, 3);
           if ((lane & 3) == 0) red_add_v4(yq + n, wv, w1, w2, w3);
           if (dq) atomicAdd(dq + n, v);
+          if (tq) {
+            tq[(int64_t)n * GI] = d0;
+            tq[(int64_t)n * GI + 1] = d1;
+          }
         }
       }
     }
@@ -1250,8 +1274,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
           // y-zero barrier, second half, before this CTA's first add into y (long done by now:
           // every CTA arrived right after zeroing its share, before its first gate/up pass)
           if (ctid == 0) {
-            bool ok = false;
-            for (uint32_t i = 0; i < kGridWaitTries && !ok; ++i) ok = ld_acquire_u64(A.r.gbar) >= *S.ytarget;
+            const bool ok = wait_counter(A.r.gbar, *S.ytarget, A.r.wait_ns);
             if (!ok) {
               *abort = 1;
               wait_failed(status, 1, 8, 0);
@@ -1287,8 +1310,8 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
           hx = hqd;
         }
         const int rot = down_rotation(U, (d.b.H / kRows + kSP / (WBITS == 8 ? 4 : 2) - 1) / (kSP / (WBITS == 8 ? 4 : 2)));
-        down_consume<WBITS, WG32, AG32, TM>(d.b.H, m, rot, R, c, hx, hxs, hs, toks, wts, d.y, d.dbg_a, c0, abort,
-                                        status);
+        down_consume<WBITS, WG32, AG32, TM>(d.b.H, m, rot, R, c, hx, hxs, hs, toks, wts, d.y, d.dbg_a, d.dbg_dots,
+                                            d.b.I / 32, U.sub, c0, abort, status);
       }
     }
   }
@@ -1364,7 +1387,24 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
     }
     RingArgs B = A;
     B.cluster = cs_best;
-    if (!B.cluster) return launch_pdl(kern, dim3(grid_x), dim3(kNT), (size_t)P.total, st, B);
+    if (!B.cluster) {
+      // cooperative launch: the grid barrier needs every CTA resident at once, which the
+      // runtime then guarantees (it refuses a grid that cannot be co-resident instead of
+      // leaving CTAs to wait for SMs held by CTAs that spin on the barrier)
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute at[2];
+      at[0].id = cudaLaunchAttributeCooperative;
+      at[0].val.cooperative = 1;
+      at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      at[1].val.programmaticStreamSerializationAllowed = 1;
+      cfg.gridDim = dim3(grid_x);
+      cfg.blockDim = dim3(kNT);
+      cfg.dynamicSmemBytes = (size_t)P.total;
+      cfg.stream = st;
+      cfg.attrs = at;
+      cfg.numAttrs = kUsePdl ? 2 : 1;
+      return cudaLaunchKernelEx(&cfg, kern, B);
+    }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;

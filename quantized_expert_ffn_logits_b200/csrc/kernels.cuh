@@ -78,6 +78,7 @@ struct ExpertArgs {
   float* hbuf;               // gate/up, token act: [slots][I] fp32 h
   float* dbg_a;              // gate/up: gate values [slots][I]; down: pair values [slots][H]
   float* dbg_b;              // gate/up: up values
+  int32_t* dbg_dots;         // down: int32 group dots [slots][H][I/32] (debug)
   float* y;                  // down: [T][H] accumulated
   int* status;
 };
@@ -119,6 +120,7 @@ struct MmaArgs {
   const float* wts;
   float* y;
   float* dbg_y[2];
+  int32_t* dbg_dots[2];                    // down: int32 group dots [slot][H][K/32] (debug)
   int T, k;
   int* status;
 };
@@ -153,6 +155,7 @@ struct RouteArgs {
   // grid barrier of the single-token expert kernel: a multiple of 1024 between calls (each
   // call's CTAs arrive at base .. base + grid - 1, the last one moves it to base + 1024)
   unsigned long long* gbar;
+  unsigned long long wait_ns;   // bound of the single-token kernel's cross-CTA waits (ns)
 };
 cudaError_t launch_route_fused(const RouteArgs& r, cudaStream_t st);
 

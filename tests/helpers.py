@@ -67,11 +67,47 @@ def oracle_experts(case: S.Case, experts=None):
     return ex, sh
 
 
-def oracle_layer(case: S.Case, union=False, top_p=0.0):
+def oracle_layer(case: S.Case, union=False, top_p=0.0, x=None):
+    """The oracle's layer on the case's inputs (or on another x with the case's weights);
+    the result also carries the oracle-quantized experts under "experts" (routed, shared)."""
     c = case.cfg
     ex, sh = oracle_experts(case)
-    return O.layer_forward(case.x(), case.router_w(), case.bias(), ex, sh, c.score, c.top_k,
-                           c.renormalize, c.rsf, ag32(c), union=union, top_p=top_p)
+    o = O.layer_forward(case.x() if x is None else x, case.router_w(), case.bias(), ex, sh, c.score,
+                        c.top_k, c.renormalize, c.rsf, ag32(c), union=union, top_p=top_p)
+    o["experts"] = (ex, sh)
+    return o
+
+
+def group_dots(qw, qa):
+    """Exact per-group integer dots: qw [N][K] int8 codes, qa [n][K] int8 -> int64 [n][N][K/32]
+    (products and sums of integers below 2^53 are exact in fp64)."""
+    qw = np.asarray(qw)
+    N, K = qw.shape
+    G = K // 32
+    w = qw.astype(np.float64).reshape(N, G, 32)
+    a = np.asarray(qa).astype(np.float64).reshape(-1, G, 32)
+    return np.einsum("ngi,hgi->nhg", a, w).astype(np.int64)
+
+
+def expected_down_dots(ref, case: S.Case, perm):
+    """The down projection's exact group dots of every kept pair (grouped row r = pair
+    perm[r]) and, with a shared expert, of every token against it: from the oracle's q_h and
+    down codes. Returns (routed [P][H][I/32], shared [T][H][I_s/32] or None)."""
+    c = case.cfg
+    ex, sh = ref["experts"]
+    k = c.top_k
+    perm = np.asarray(perm)
+    e_of = ref["idx"].reshape(-1)[perm]
+    out = np.zeros((len(perm), c.H, c.I // 32), np.int64)
+    for e in np.unique(e_of):
+        rows = np.nonzero(e_of == e)[0]
+        out[rows] = group_dots(ex.q_dn[e], ref["qh"][perm[rows]])
+    shd = None
+    if sh is not None:
+        qh_sh = np.stack([O.expert_ffn(sh, 0, ref["qx"][t], ref["sx"][t], ag32(c))["qh"]
+                          for t in range(case.T)])
+        shd = group_dots(sh.q_dn[0], qh_sh)
+    return out, shd
 
 
 def oracle_tokens(case: S.Case, tokens):

@@ -31,7 +31,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_status_strings():
-    assert M.moe_abi_version() == 2
+    assert M.moe_abi_version() == 3
     for s in range(7):
         assert M.moe_status_string(s).startswith("MOE_")
     assert M.moe_status_string(99) == "MOE_ERR_UNKNOWN"
@@ -117,8 +117,10 @@ def test_other_entry_points_reject_bad_arguments():
     v = M.moe_debug_views()
     assert L.moe_layer_debug_views(4, C.byref(b), None, C.byref(_cfg(flags=1)), C.byref(v)) == M.MOE_OK
     assert v.gate > 0 and v.up > 0 and v.y_pair > 0 and v.total == L.moe_layer_workspace_bytes(4, C.byref(b), None, C.byref(_cfg(flags=1)))
+    # the down projection's group dots: int32 [T*k][H][I/32], the last region of the debug layout
+    assert v.dn_dots > v.y_pair and v.dn_dots + 4 * 2 * 256 * (128 // 32) * 4 <= v.total
     assert L.moe_layer_debug_views(4, C.byref(b), None, C.byref(_cfg()), C.byref(v)) == M.MOE_OK
-    assert v.gate == -1
+    assert v.gate == -1 and v.dn_dots == -1
     assert L.moe_get_device_status(None, None) == M.MOE_ERR_INVALID_ARG
     # the debug forward sizes its workspace for the debug layout and leaves views alone on errors
     f = L.moe_layer_forward_debug

@@ -1,9 +1,11 @@
 """GPU parity at the five workloads' full sizes, in the launch configuration bench.py times
 (one moe_layer_forward call over the whole batch, no debug copies): every output row of the
 decode batches; for the larger batches a seeded sample of tokens, which the oracle computes
-one by one, regenerating only the experts those tokens use. Routing indices of the compared
-tokens are bit-exact; their output rows meet the layer tolerance (rel-L2 1e-5, max-abs
-1e-4 * max|y|)."""
+one by one, regenerating only the experts those tokens use. Where some experts of the batch
+run on the tensor cores (at least 16 pairs) and others are streamed, half of the sample is
+drawn from the tokens routed to a streamed expert, so both paths are compared at their
+full-size tile counts. Routing indices of the compared tokens are bit-exact; their output
+rows meet the layer tolerance (rel-L2 1e-5, max-abs 1e-4 * max|y|)."""
 import numpy as np
 import pytest
 
@@ -22,11 +24,24 @@ FULL = [
     ("glm_int4", 1, None),
     ("glm_int4", 4, 2),
     ("e512_int4", 1, None),
-    ("e512_int4", 64, 8),
-    ("olmoe_int4", 512, 6),        # tensor-core path (experts with >= 16 pairs)
-    ("olmoe_int4", 4096, 4),
-    ("e512_int4", 4096, 4),        # Zipf-skewed: tensor cores for hot experts, streaming for the rest
+    ("e512_int4", 64, None),       # Zipf-skewed: the hottest experts on the tensor cores
+    ("olmoe_int4", 512, 32),       # tensor-core path (experts with >= 16 pairs)
+    ("olmoe_int4", 4096, 64),
+    ("e512_int4", 4096, 64),       # Zipf-skewed: tensor cores for hot experts, streaming for the rest
 ]
+MMA_MIN_PAIRS = 16                 # pairs an expert needs in a call for the tensor-core path
+
+
+def _sample(idx, T, n, seed):
+    """n tokens: half (when there are any) routed to an expert with fewer than MMA_MIN_PAIRS
+    pairs in the batch (the streaming path), the rest at random."""
+    rng = np.random.default_rng(seed)
+    counts = np.bincount(idx[idx >= 0].reshape(-1), minlength=int(idx.max()) + 1)
+    cold = np.nonzero(np.isin(idx, np.nonzero(counts < MMA_MIN_PAIRS)[0]).any(axis=1))[0]
+    pick = set(rng.choice(cold, size=min(n // 2, len(cold)), replace=False).tolist()) if len(cold) else set()
+    rest = [t for t in rng.permutation(T).tolist() if t not in pick]
+    pick.update(rest[: n - len(pick)])
+    return sorted(pick), len(cold), int((counts >= MMA_MIN_PAIRS).sum())
 
 
 @pytest.mark.parametrize("name,T,sample", FULL)
@@ -41,11 +56,17 @@ def test_full_size_layer(name, T, sample):
     assert M.moe_read_device_status(ws) == M.MOE_OK
     yg = y.cpu().numpy()
     assert np.isfinite(yg).all()
-    rng = np.random.default_rng(1234 + T)
-    toks = list(range(T)) if sample is None else sorted(rng.choice(T, size=sample, replace=False).tolist())
-    ref = oracle_tokens(case, toks)
     v = M.moe_layer_debug_views(T, g["blob"], g["shared"], cfg)
     idx = M.workspace_view(ws, v["idx"], torch.int32, (T, c.top_k)).cpu().numpy()
+    if sample is None:
+        toks = list(range(T))
+    else:
+        toks, n_cold, n_hot = _sample(idx, T, sample, 1234 + T)
+        if name == "e512_int4" and T == 4096:       # the mixed case must reach both paths
+            assert n_cold > 0 and n_hot > 0
+            assert any(np.isin(idx[t], np.nonzero(np.bincount(idx.reshape(-1)) < MMA_MIN_PAIRS)[0]).any()
+                       for t in toks)
+    ref = oracle_tokens(case, toks)
     assert np.array_equal(idx[toks], ref["idx"])
     assert_close_y(yg[toks], ref["y"])
     del g, y, ws

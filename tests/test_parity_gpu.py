@@ -7,7 +7,8 @@ import pytest
 
 import oracle as O
 import synth as S
-from helpers import (ag32, assert_close_y, gpu_layer, oracle_layer, route_cfg, wbits, wg32)
+from helpers import (ag32, assert_close_y, expected_down_dots, gpu_layer, oracle_layer, route_cfg, wbits,
+                     wg32)
 
 pytestmark = pytest.mark.gpu
 
@@ -156,7 +157,36 @@ def _check_layer(name, T, flags, top_p=0.0):
     assert np.array_equal(sh, ref["sh"][perm])
     ye = view(v["y_pair"], torch.float32, (P, H))
     assert_close_y(ye, ref["ye"][perm], "per-pair expert outputs")
+    _check_down_dots(m, ws, v, case, ref, perm)
     assert_close_y(_np(y), ref["y"])
+
+
+def _check_down_dots(m, ws, v, case, ref, perm):
+    """The down projection's int32 group dots, as the expert kernels formed them (streaming
+    and tensor-core paths alike), equal the exact integer dots of the oracle's h codes with the
+    oracle's down codes, for every kept pair and every shared-expert row; dropped slots stay 0.
+    Two entries are also checked against the oracle's own stage routine."""
+    c = case.cfg
+    T, k, H, I, Is = case.T, c.top_k, c.H, c.I, c.shared_I
+    P = len(perm)
+    got = _np(m.workspace_view(ws, v["dn_dots"], torch.int32, (T * k, H, I // 32)))
+    want, want_sh = expected_down_dots(ref, case, perm)
+    bad = np.argwhere(got[:P] != want)
+    assert bad.size == 0, f"{len(bad)} down group dots differ, first (row, n, g) {bad[:4].tolist()}"
+    assert not got[P:].any(), "dropped slots' dots must stay 0"
+    ex, sh = ref["experts"]
+    for r in (0, P - 1):
+        pair = int(perm[r])
+        e = int(ref["idx"].reshape(-1)[pair])
+        n = (7 * r + 3) % H
+        _, dots = O.stage(ex.q_dn[e, n], ex.s_dn[e, n], wg32(c), ref["qh"][pair], ref["sh"][pair], ag32(c))
+        # (per-row weights with per-token activations: the stage routine's one whole-row dot)
+        mine = got[r, n] if dots.size > 1 else got[r, n].sum(keepdims=True)
+        assert np.array_equal(mine, dots), (r, n)
+    if Is:
+        off = v["dn_dots"] + T * k * H * (I // 32) * 4
+        got_sh = _np(m.workspace_view(ws, off, torch.int32, (T, H, Is // 32)))
+        assert np.array_equal(got_sh, want_sh), "shared-expert down group dots"
 
 
 @pytest.mark.parametrize("name,T", [("olmoe_int8", 8), ("glm_int4", 4), ("e512_int4", 64)])
@@ -211,25 +241,30 @@ def test_forward_debug_entry_point(name, T):
 
 @pytest.mark.parametrize("name,T", [("olmoe_int8", 1), ("glm_int4", 3), ("olmoe_int4", 40)])
 def test_forward_host_buffers_equal_device_path(name, T):
-    """moe_layer_forward_host (pinned host x in, y out, one C call) gives the y of
-    moe_layer_forward on device buffers -- to the layer tolerance, the combine into y being
-    fp32 adds in arrival order -- repeated calls included (the single-token grid barrier
-    counter moves on between calls)."""
+    """moe_layer_forward_host (pinned host x in, y out, one C call per step) on four different
+    inputs enqueued back to back with no synchronization between them, each into its own host
+    output: every call's y matches the oracle on its own x (to the layer tolerance). The calls
+    share the device staging buffer of x, which the next call's input copy overwrites while the
+    previous call's kernels may still be running; a copy that overtook a reader of x would
+    show up here as a wrong y. The first call's y also matches moe_layer_forward on device
+    buffers."""
     m = M()
     case = S.Case.make(REDUCED[name], T)
     g = gpu_layer(case)
     c = case.cfg
     lay = m.Layer(T, g["blob"], g["shared"], route_cfg(c), g["wr"], g["bias"])
+    xs = [case.x()] + [S.normal_cpu(T * c.H, 4242 + i, 0, c.x_sigma).reshape(T, c.H) for i in range(3)]
+    xh = [torch.from_numpy(x).pin_memory() for x in xs]
+    yh = [torch.full((T, c.H), float("nan"), dtype=torch.float32).pin_memory() for _ in xs]
     yd = torch.empty((T, c.H), dtype=torch.float32, device="cuda")
     lay(g["x"], yd)
-    xh = g["x"].cpu().pin_memory()
-    yh = torch.full((T, c.H), float("nan"), dtype=torch.float32).pin_memory()
-    for _ in range(3):
-        lay.forward_host(xh, yh)
+    for a, b in zip(xh, yh):
+        lay.forward_host(a, b)
     torch.cuda.synchronize()
     assert m.moe_read_device_status(lay.workspace) == m.MOE_OK
-    assert_close_y(yh.numpy(), _np(yd).astype(np.float64))
-    assert_close_y(yh.numpy(), oracle_layer(case)["y"])
+    assert_close_y(yh[0].numpy(), _np(yd).astype(np.float64))
+    for i, x in enumerate(xs):
+        assert_close_y(yh[i].numpy(), oracle_layer(case, x=x)["y"], f"call {i}")
 
 
 def test_synth_device_generator_matches_host():
@@ -445,6 +480,52 @@ def test_tensor_core_dots_exact_at_extreme_codes(wtype):
     assert np.array_equal(gate, ref["gate"][perm]), "gate stage values"
     assert np.array_equal(up, ref["up"][perm]), "up stage values"
     assert np.array_equal(view(v["q_h"], torch.int8, (P, I)), ref["qh"][perm])
+    ref["experts"] = (ex, None)
+    _check_down_dots(m, ws, v, S.Case(S.CONFIGS["olmoe_int8"].with_(E=E, H=H, I=I, top_k=k, shared_I=0), T, 0),
+                     ref, perm)
+    assert_close_y(_np(y), ref["y"])
+
+
+@pytest.mark.parametrize("wtype", ["int8", "int4"])
+@pytest.mark.parametrize("path", ["mma", "stream"])
+def test_down_dots_exact_at_extreme_codes(wtype, path):
+    """The down projection at its largest group dots, on both expert paths: every gate and up
+    row is the same +-1 pattern and every token agrees with it in most signs, so for each token
+    all of its h values are equal and positive and every h code is +127; half of the down rows
+    are all +1 (codes +127 / +7), the rest random
+    signs, so group dots reach 32 * 127 * 127 (int8) or 32 * 127 * 7 (int4) -- partial sums far
+    above fp16's integer range, exact only in the fp32 accumulator. The down group dots must
+    equal the exact integer dots bit for bit, and y must meet the layer tolerance."""
+    m = M()
+    rng = np.random.default_rng(91)
+    E, H, I, T, k = 2, 256, 128, 40, 2
+    pat = np.where(rng.random(H) < 0.5, -1.0, 1.0).astype(np.float32)
+    x = pat * np.where(rng.random((T, H)) < 0.3, -1.0, 1.0).astype(np.float32)   # gate values > 0
+    x[0] = pat
+    gu = np.broadcast_to(pat, (E, 2 * I, H)).copy()
+    dn = np.where(rng.random((E, H, I)) < 0.5, -1.0, 1.0).astype(np.float32)
+    dn[:, ::2, :] = 1.0
+    wr = rng.normal(0.0, 1.0 / np.sqrt(H), (E, H)).astype(np.float32)
+    wb = 8 if wtype == "int8" else 4
+    ex = O.QExperts.quantize(gu, dn, wb, True)
+    ref = O.layer_forward(x, wr, None, ex, None, "softmax", k, True, 1.0, True, union=True)
+    ref["experts"] = (ex, None)
+    assert (ref["qh"] == 127).all()
+    blob = m.ExpertBlob.quantize(torch.from_numpy(gu).cuda(), torch.from_numpy(dn).cuda(), wtype, "g32_f16")
+    force = m.MOE_FLAG_FORCE_MMA if path == "mma" else m.MOE_FLAG_FORCE_GEMV
+    cfg = m.RouteCfg(score="softmax", top_k=k, renormalize=True, routed_scaling_factor=1.0, act="g32_f16",
+                     flags=m.MOE_FLAG_DEBUG | force)
+    y, ws = m.moe_layer_forward(torch.from_numpy(x).cuda(), torch.from_numpy(wr).cuda(), None, blob, None, cfg)
+    torch.cuda.synchronize()
+    assert m.moe_read_device_status(ws) == m.MOE_OK
+    v = m.moe_layer_debug_views(T, blob, None, cfg)
+    perm = _np(m.workspace_view(ws, v["perm"], torch.int32, (T * k,)))
+    assert np.array_equal(perm, ref["perm"])
+    assert np.array_equal(_np(m.workspace_view(ws, v["q_h"], torch.int8, (T * k, I))), ref["qh"][perm])
+    case = S.Case(S.CONFIGS["olmoe_int8"].with_(E=E, H=H, I=I, top_k=k, shared_I=0), T, 0)
+    _check_down_dots(m, ws, v, case, ref, perm)
+    got = _np(m.workspace_view(ws, v["dn_dots"], torch.int32, (T * k, H, I // 32)))
+    assert np.abs(got).max() == 32 * 127 * (127 if wtype == "int8" else 7)
     assert_close_y(_np(y), ref["y"])
 
 
