@@ -67,7 +67,7 @@ def load_peaks():
 
 
 def blob_row_bytes(cfg, K, I_rows):
-    kb = K if cfg.wtype == "int8" else K // 2
+    kb = K * {"int8": 8, "int4": 4, "int2": 2}[cfg.wtype] // 8
     sb = (K // 32) * 2 if cfg.wscale == "g32_f16" else 4
     return I_rows * (kb + sb)
 
@@ -228,7 +228,7 @@ def oracle_sampler(cfg, T, top_p=0.0, seed_base=7_000_000):
     from concurrent.futures import ThreadPoolExecutor
 
     cores = os.cpu_count() or 1
-    wbits = 8 if cfg.wtype == "int8" else 4
+    wbits = {"int8": 8, "int4": 4, "int2": 2}[cfg.wtype]
     wg32 = cfg.wscale == "g32_f16"
     ag32 = cfg.act == "g32_f16"
     n_tok = 64

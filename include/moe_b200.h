@@ -38,7 +38,7 @@
  * Numerics. Every step that decides an integer (quantized codes, top-k
  * selection) runs a fixed fp32 operation sequence, so results are bit-exact
  * across runs and against a CPU implementation of the same sequence:
- *   - quantization: d = amax / Q (fp32 division, Q = 127 int8 or 7 int4),
+ *   - quantization: d = amax / Q (fp32 division, Q = 127 int8, 7 int4 or 1 int2),
  *     stored as fp32 (per row / per token) or rounded to fp16 (group of 32);
  *     q = clamp(round_half_away(v / stored_d), -Q, Q); q = 0 if stored_d = 0;
  *   - router logits: per 32-element chunk an fma chain from +0 in ascending
@@ -83,8 +83,12 @@ typedef enum {
   MOE_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up */
 } moe_status;
 
-/* Expert weight code type. Packed int4: two's-complement nibbles, two per byte. */
-enum { MOE_W_INT8 = 0, MOE_W_INT4 = 1 };
+/* Expert weight code type (the GLM-5.2 colibri page, "What's implemented": int8 / packed int4 /
+ * packed int2). Packed int4: two's-complement nibbles, two per byte (element 2j in the low
+ * nibble of byte j), codes -7..7. Packed int2: two's-complement 2-bit fields, four per byte
+ * (element 4j + i in bits 2i..2i+1 of byte j), codes -1, 0, 1 (the symmetric rule with
+ * Q = 1: d = amax, -2 never produced). */
+enum { MOE_W_INT8 = 0, MOE_W_INT4 = 1, MOE_W_INT2 = 2 };
 /* Weight scale granularity: one fp32 per row, or one fp16 per 32 values of a row. */
 enum { MOE_SCALE_ROW_F32 = 0, MOE_SCALE_G32_F16 = 1 };
 /* Activation quantization: one fp32 scale per token, or Q8_0-style fp16 per 32. */
@@ -110,21 +114,21 @@ enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID_NOAUX_TC = 1 };
  *   R0 gate/up codes: for each expert e, for each s in [0, I/64): a block of
  *      128 rows -- rows 0..63 are gate rows 64s..64s+63, rows 64..127 the up
  *      rows of the same intermediate indices -- stored as [KB/16][128][16]:
- *      16-byte piece p of row r at (p * 128 + r) * 16. KB = H (int8) or H/2
- *      (int4; element 2j in the low nibble of byte j). One block's K range is
- *      one contiguous run, one piece of it 2 KB.
+ *      16-byte piece p of row r at (p * 128 + r) * 16. KB = H (int8), H/2
+ *      (int4) or H/4 (int2) code bytes per row. One block's K range is one
+ *      contiguous run, one piece of it 2 KB.
  *   R1 down codes: the [H][I] matrix of expert e cut along I into slabs of 64
  *      intermediate indices: for each e, each u in [0, I/64), each b in
  *      [0, H/128): rows 128b..128b+127, columns 64u..64u+63, stored
- *      [SB/16][128][16] (SB = 64 bytes int8, 32 bytes int4). One slab (all H
- *      rows of 64 columns) is one contiguous run.
+ *      [SB/16][128][16] (SB = 64 bytes int8, 32 bytes int4, 16 bytes int2). One
+ *      slab (all H rows of 64 columns) is one contiguous run.
  *   R2 gate/up scales: for each e, each 128-row block: fp16 [H/32][128]
  *      (group-major) or fp32 [128].
  *   R3 down scales: fp16: for each e, u, b as in R1: [2][128] (the two groups
  *      of the slab); fp32: [E][H], one per row.
  * Padding bytes between regions are zero. */
 typedef struct {
-  int32_t wtype;      /* MOE_W_INT8 | MOE_W_INT4 */
+  int32_t wtype;      /* MOE_W_INT8 | MOE_W_INT4 | MOE_W_INT2 */
   int32_t wscale;     /* MOE_SCALE_ROW_F32 | MOE_SCALE_G32_F16 */
   int32_t n_experts;  /* E */
   int32_t hidden;     /* H */

@@ -23,13 +23,13 @@ _lib = C.CDLL(LIB_PATH)
 # ---------------------------------------------------------------- constants
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE = 0, 1, 2, 3
 MOE_ERR_CUDA, MOE_ERR_DEVICE_CHECK, MOE_ERR_TIMEOUT = 4, 5, 6
-MOE_W_INT8, MOE_W_INT4 = 0, 1
+MOE_W_INT8, MOE_W_INT4, MOE_W_INT2 = 0, 1, 2
 MOE_SCALE_ROW_F32, MOE_SCALE_G32_F16 = 0, 1
 MOE_ACT_TOKEN_F32, MOE_ACT_G32_F16 = 0, 1
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID_NOAUX_TC = 0, 1
 MOE_FLAG_DEBUG, MOE_FLAG_FORCE_GEMV, MOE_FLAG_FORCE_MMA, MOE_FLAG_SHORT_WAITS = 1, 2, 4, 8
 
-WTYPES = {"int8": MOE_W_INT8, "int4": MOE_W_INT4}
+WTYPES = {"int8": MOE_W_INT8, "int4": MOE_W_INT4, "int2": MOE_W_INT2}
 WSCALES = {"row_f32": MOE_SCALE_ROW_F32, "g32_f16": MOE_SCALE_G32_F16}
 ACTS = {"token_f32": MOE_ACT_TOKEN_F32, "g32_f16": MOE_ACT_G32_F16}
 SCORES = {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID_NOAUX_TC}

@@ -33,12 +33,12 @@ struct BlobOffsets {
 };
 
 bool blob_offsets(int32_t wtype, int32_t wscale, int32_t E, int32_t H, int32_t I, BlobOffsets& o) {
-  if ((wtype != MOE_W_INT8 && wtype != MOE_W_INT4) ||
+  if ((wtype != MOE_W_INT8 && wtype != MOE_W_INT4 && wtype != MOE_W_INT2) ||
       (wscale != MOE_SCALE_ROW_F32 && wscale != MOE_SCALE_G32_F16))
     return false;
   if (E < 1 || E > 1024 || H < 128 || I < 128 || H % 128 || I % 128) return false;
-  const int64_t kb_gu = wtype == MOE_W_INT8 ? H : H / 2;
-  const int64_t kb_dn = wtype == MOE_W_INT8 ? I : I / 2;
+  const int64_t bits = wtype == MOE_W_INT8 ? 8 : wtype == MOE_W_INT4 ? 4 : 2;
+  const int64_t kb_gu = H * bits / 8, kb_dn = I * bits / 8;
   const int64_t s_gu = wscale == MOE_SCALE_G32_F16 ? (int64_t)(H / 32) * 2 : 4;
   const int64_t s_dn = wscale == MOE_SCALE_G32_F16 ? (int64_t)(I / 32) * 2 : 4;
   o.gu_w = 0;
@@ -68,7 +68,7 @@ BlobView view(const moe_expert_blob* b, const BlobOffsets& o) {
   v.E = b->n_experts;
   v.H = b->hidden;
   v.I = b->inter;
-  v.wbits = b->wtype == MOE_W_INT8 ? 8 : 4;
+  v.wbits = b->wtype == MOE_W_INT8 ? 8 : b->wtype == MOE_W_INT4 ? 4 : 2;
   v.wg32 = b->wscale == MOE_SCALE_G32_F16;
   return v;
 }

@@ -145,6 +145,46 @@ __device__ __forceinline__ int group_dot_i4(const uint4& w, const uint4& xe, con
   return d - 8 * xsum;
 }
 
+// One group of 32 packed int2 weights (8 bytes: w.x holds elements 0..15, w.y 16..31; element
+// 4j + i in bits 2i .. 2i + 1 of byte j) against activations stored de-interleaved per 16
+// elements: xa.{x,y,z,w} hold elements {0,4,8,12}, {1,5,9,13}, {2,6,10,14}, {3,7,11,15} of the
+// group's first 16, xb the same of its last 16. Each 2-bit field is read as unsigned
+// f ^ 2 = q + 2 (two's complement q in -2..1), so the dot is corrected by 2 * xsum.
+__device__ __forceinline__ int group_dot_i2(const uint2& w, const uint4& xa, const uint4& xb, int xsum) {
+  const uint32_t m = 0x03030303u;
+  const uint32_t v0 = w.x ^ 0xAAAAAAAAu, v1 = w.y ^ 0xAAAAAAAAu;
+  int d = dp4a_us(v0 & m, xa.x, 0);
+  d = dp4a_us((v0 >> 2) & m, xa.y, d);
+  d = dp4a_us((v0 >> 4) & m, xa.z, d);
+  d = dp4a_us((v0 >> 6) & m, xa.w, d);
+  d = dp4a_us(v1 & m, xb.x, d);
+  d = dp4a_us((v1 >> 2) & m, xb.y, d);
+  d = dp4a_us((v1 >> 4) & m, xb.z, d);
+  d = dp4a_us((v1 >> 6) & m, xb.w, d);
+  return d - 2 * xsum;
+}
+
+// 16 activation bytes (words a = x0..x3, x4..x7, x8..x11, x12..x15) -> (x0 x4 x8 x12),
+// (x1 x5 x9 x13), (x2 x6 x10 x14), (x3 x7 x11 x15): the order of a packed int2 word's fields.
+__device__ __forceinline__ uint4 deinterleave16(const uint4& a) {
+  const uint32_t t0 = __byte_perm(a.x, a.y, 0x5140), t1 = __byte_perm(a.z, a.w, 0x5140);
+  const uint32_t t2 = __byte_perm(a.x, a.y, 0x7362), t3 = __byte_perm(a.z, a.w, 0x7362);
+  return make_uint4(__byte_perm(t0, t1, 0x5410), __byte_perm(t0, t1, 0x7632), __byte_perm(t2, t3, 0x5410),
+                    __byte_perm(t2, t3, 0x7632));
+}
+
+// Sum of the 32 signed codes of a group (two 16-byte words).
+__device__ __forceinline__ int code_sum32(const uint4& a0, const uint4& a1) {
+  int s = __dp4a((int)a0.x, 0x01010101, 0);
+  s = __dp4a((int)a0.y, 0x01010101, s);
+  s = __dp4a((int)a0.z, 0x01010101, s);
+  s = __dp4a((int)a0.w, 0x01010101, s);
+  s = __dp4a((int)a1.x, 0x01010101, s);
+  s = __dp4a((int)a1.y, 0x01010101, s);
+  s = __dp4a((int)a1.z, 0x01010101, s);
+  return __dp4a((int)a1.w, 0x01010101, s);
+}
+
 // 8 activation bytes x0..x7 -> (x0 x2 x4 x6), (x1 x3 x5 x7).
 __device__ __forceinline__ void deinterleave8(uint32_t lo, uint32_t hi, uint32_t& even,
                                               uint32_t& odd) {
@@ -160,10 +200,10 @@ struct BlobView {
   const uint8_t* gu_s;  // R2 gate/up scales
   const uint8_t* dn_s;  // R3 down scales
   int E, H, I;
-  int wbits;            // 8 or 4
+  int wbits;            // 8, 4 or 2
   int wg32;             // 1: fp16 group-32 scales, 0: fp32 per row
 };
 
-__host__ __device__ __forceinline__ int kbytes(int K, int wbits) { return wbits == 8 ? K : K / 2; }
+__host__ __device__ __forceinline__ int kbytes(int K, int wbits) { return K * wbits / 8; }
 
 }  // namespace moe

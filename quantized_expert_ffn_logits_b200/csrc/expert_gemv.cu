@@ -20,19 +20,20 @@ __global__ void k_group_dots(BlobView b, int which, int n, const int32_t* __rest
   const int smp = (int)(id / G), g = (int)(id % G);
   const int e = expert[smp], r = row[smp];
   const int KB = kbytes(K, b.wbits);
-  const int gbytes = b.wbits == 8 ? 32 : 16;     // code bytes of one group
-  const uint8_t* p0;                             // the group's first 16-byte piece
+  const int gbytes = 4 * b.wbits;                // code bytes of one group: 32, 16 or 8
+  const uint8_t* p0;                             // the group's first code byte
   if (which == 0) {
     const int half = r >= b.I;
     const int i = r - half * b.I;
     const int64_t blk = (int64_t)e * 2 * b.I + (int64_t)(i >> 6) * 128;
     const int byte = g * gbytes;
-    p0 = b.gu_w + blk * KB + ((int64_t)(byte >> 4) * 128 + half * 64 + (i & 63)) * 16;
+    p0 = b.gu_w + blk * KB + ((int64_t)(byte >> 4) * 128 + half * 64 + (i & 63)) * 16 + (byte & 15);
   } else {
     // slab of the group's 64 columns; the group starts at byte (g % 2) * gbytes of it
     const int U = b.I / 64, HB = b.H / 128, sbytes = 2 * gbytes;
     const int64_t slab = ((int64_t)e * U + g / 2) * HB + (r >> 7);
-    p0 = b.dn_w + ((slab * (sbytes / 16) + (g & 1) * (gbytes / 16)) * 128 + (r & 127)) * 16;
+    const int byte = (g & 1) * gbytes;
+    p0 = b.dn_w + ((slab * (sbytes / 16) + (byte >> 4)) * 128 + (r & 127)) * 16 + (byte & 15);
   }
   const uint8_t* xg = reinterpret_cast<const uint8_t*>(act) + (int64_t)smp * K + 32 * g;
   const uint4 x0 = *reinterpret_cast<const uint4*>(xg);
@@ -42,6 +43,9 @@ __global__ void k_group_dots(BlobView b, int which, int n, const int32_t* __rest
     const uint4 w0 = *reinterpret_cast<const uint4*>(p0);
     const uint4 w1 = *reinterpret_cast<const uint4*>(p0 + 128 * 16);
     d = group_dot_i8(w0, w1, x0, x1);
+  } else if (b.wbits == 2) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p0);
+    d = group_dot_i2(w, deinterleave16(x0), deinterleave16(x1), code_sum32(x0, x1));
   } else {
     const uint4 w = *reinterpret_cast<const uint4*>(p0);
     uint32_t e0, o0, e1, o1, e2, o2, e3, o3;

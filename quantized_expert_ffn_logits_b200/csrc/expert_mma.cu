@@ -111,10 +111,13 @@ __device__ __forceinline__ void cvt_i8x4_f16(uint32_t w, uint32_t& o0, uint32_t&
   o0 = *reinterpret_cast<uint32_t*>(&r0);
   o1 = *reinterpret_cast<uint32_t*>(&r1);
 }
-// Four bytes holding v = n + 8 (n a signed 4-bit code) -> the four fp16 values n.
+// Four bytes holding v = n + BIAS (n a signed code: BIAS 8 for 4-bit, 2 for 2-bit codes) ->
+// the four fp16 values n: the bytes become the low mantissa bytes of fp16 1024 + v, then
+// 1024 + BIAS is subtracted (exact).
+template <int BIAS = 8>
 __device__ __forceinline__ void cvt_u4x4_f16(uint32_t v, uint32_t& o0, uint32_t& o1) {
   uint32_t h0 = __byte_perm(v, 0x64646464u, 0x5140), h1 = __byte_perm(v, 0x64646464u, 0x7362);
-  const __half2 k = __halves2half2(__float2half_rn(1032.0f), __float2half_rn(1032.0f));
+  const __half2 k = __halves2half2(__float2half_rn(1024.0f + BIAS), __float2half_rn(1024.0f + BIAS));
   __half2 r0 = __hsub2(*reinterpret_cast<__half2*>(&h0), k), r1 = __hsub2(*reinterpret_cast<__half2*>(&h1), k);
   o0 = *reinterpret_cast<uint32_t*>(&r0);
   o1 = *reinterpret_cast<uint32_t*>(&r1);
@@ -182,7 +185,11 @@ constexpr int kMmaNB = 4;                  // tensor-memory accumulators (128 fp
                                            // all 512; one CTA per SM), so MMAs run 4 groups ahead
 constexpr int kMmaPrepWarps = 2;
 constexpr uint32_t kMmaSleepNs = 200;      // backoff of the roles that run ahead of the epilogue
-// One accumulator hand-off per 2-group stage: the MMA issuer fills a pair of accumulators
+// The roles that run ahead (producer, MMA issuer, prep) poll with short sleeps (measured: the
+// same time as suspending waits, which free issue slots the epilogue does not need).
+__device__ __forceinline__ bool mma_wait_ahead(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_sleep(bar, parity, kMmaSleepNs);
+}// One accumulator hand-off per 2-group stage: the MMA issuer fills a pair of accumulators
 // (groups 2i, 2i + 1) and commits once; the epilogue waits once, drains both, releases once.
 constexpr bool kMmaPairCommit = true;
 // Weight blocks are re-read by every tile of their expert: normal L2 policy, not evict-first
@@ -211,7 +218,7 @@ constexpr int kMmaSmem = kMmaNS * MmaStage::BYTES + 256 + 2048 + 1024;
 // Stage bytes the producer copies (A codes and scales, B codes and scales).
 template <int WBITS>
 __device__ __forceinline__ uint32_t mma_stage_bytes() {
-  return 16384u + 512u + (WBITS == 8 ? 8192u : 4096u) + 512u;
+  return 16384u + 512u + 1024u * WBITS + 512u;   // B: 2 groups x 128 rows x 32 codes
 }
 
 template <int WBITS, bool GATEUP>
@@ -227,8 +234,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* xchg = reinterpret_cast<int*>(base + kMmaNS * MmaStage::BYTES + 256);   // [2][2][128] h amax
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int PPG = WBITS == 8 ? 2 : 1;  // 16-byte pieces of one group of weight codes
-  constexpr int PPU = 2 * PPG;             // pieces of a 64-column down slab row
+  constexpr int PPU = WBITS / 2;           // 16-byte pieces of a 64-column down slab row
   constexpr int kKern = GATEUP ? 3 : 4;
   static_assert(kMmaKC == 2, "a stage is one 64-column down slab");
 
@@ -285,7 +291,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
         const __half* as_src = GATEUP ? A.a_scales + (int64_t)ti * G * 128 : A.h_scales + (int64_t)ti * (A.hk / 32) * 128;
         for (int g0 = 0; g0 < G && ok; g0 += kMmaKC, ++c) {
           const int s = c % kMmaNS;
-          if (c >= (uint32_t)kMmaNS && !mbar_wait_sleep(&empty[s], ((c / kMmaNS) - 1) & 1, kMmaSleepNs)) {
+          if (c >= (uint32_t)kMmaNS && !mma_wait_ahead(&empty[s], ((c / kMmaNS) - 1) & 1)) {
             wait_failed(A.status, kKern, 0, s);
             ok = false;
             break;
@@ -300,7 +306,8 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
           };
           if (GATEUP) {
             const int64_t blk = (int64_t)tl.w * 2 * bv.I + (int64_t)blkn * 128;
-            load_w(st + MmaStage::B8, bv.gu_w + blk * KB + (int64_t)g0 * PPG * 2048, kMmaKC * PPG * 2048);
+            // the stage's 2 groups: code bytes 4 WBITS g0 .. of each row = pieces WBITS g0 / 4 ..
+            load_w(st + MmaStage::B8, bv.gu_w + blk * KB + (int64_t)g0 * WBITS / 4 * 2048, 1024u * WBITS);
             load_w(st + MmaStage::BS, bv.gu_s + (blk * G + (int64_t)g0 * 128) * 2, 512);
           } else {
             const int U = bv.I / 64, HB = bv.H / 128;
@@ -333,7 +340,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
         for (int g0 = 0; g0 < G; g0 += kMmaKC, ++c) {
           const int s = c % kMmaNS;
           bool ok = *abort == 0;
-          if (ok && !mbar_wait_sleep(&prep[s], (c / kMmaNS) & 1, kMmaSleepNs)) {
+          if (ok && !mma_wait_ahead(&prep[s], (c / kMmaNS) & 1)) {
             *abort = 1;
             wait_failed(A.status, kKern, 1, s);
             ok = false;
@@ -343,7 +350,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
           if constexpr (kMmaPairCommit) {
             // the stage's two groups into accumulator pair pr (buffers 2 pr, 2 pr + 1)
             const uint32_t pr = c & 1;
-            if (ok && c >= 2 && !mbar_wait_sleep(&acc_empty[pr], ((c >> 1) - 1) & 1, kMmaSleepNs)) {
+            if (ok && c >= 2 && !mma_wait_ahead(&acc_empty[pr], ((c >> 1) - 1) & 1)) {
               *abort = 1;
               wait_failed(A.status, kKern, 3, pr);
               ok = false;
@@ -362,7 +369,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
           } else {
             for (int j = 0; j < kMmaKC; ++j, ++gi) {
               const int bb = gi % kMmaNB;
-              if (ok && gi >= (uint32_t)kMmaNB && !mbar_wait_sleep(&acc_empty[bb], ((gi / kMmaNB) - 1) & 1, kMmaSleepNs)) {
+              if (ok && gi >= (uint32_t)kMmaNB && !mma_wait_ahead(&acc_empty[bb], ((gi / kMmaNB) - 1) & 1)) {
                 *abort = 1;
                 wait_failed(A.status, kKern, 3, bb);
                 ok = false;
@@ -397,7 +404,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
       for (int g0 = 0; g0 < G; g0 += kMmaKC, ++c) {
         const int s = c % kMmaNS;
         bool ok = *abort == 0;
-        if (ok && !mbar_wait_sleep(&full[s], (c / kMmaNS) & 1, kMmaSleepNs)) {
+        if (ok && !mma_wait_ahead(&full[s], (c / kMmaNS) & 1)) {
           *abort = 1;
           if (lane == 0) wait_failed(A.status, kKern, 4, s);
           ok = false;
@@ -421,6 +428,34 @@ __global__ void __launch_bounds__(kMmaThreads, 1) k_expert_mma(const __grid_cons
               cvt_i8x4_f16(w[u].w, hi.z, hi.w);
               *reinterpret_cast<uint4*>(st + MmaStage::BH + ((2 * p) * 128 + r) * 16) = lo;
               *reinterpret_cast<uint4*>(st + MmaStage::BH + ((2 * p + 1) * 128 + r) * 16) = hi;
+            }
+          }
+          if (WBITS == 2) {
+            // the packed int2 piece of a row (its 64 codes of the stage, element 4b + i in bits
+            // 2i .. 2i + 1 of byte b) -> fp16 pieces 0 .. 7
+            constexpr int NQ = 128 / NPT;
+            uint4 w[NQ];
+#pragma unroll
+            for (int v = 0; v < NQ; ++v) w[v] = *reinterpret_cast<const uint4*>(st + MmaStage::B8 + (pt + v * NPT) * 16);
+#pragma unroll
+            for (int v = 0; v < NQ; ++v) {
+              const int r = pt + v * NPT;
+              const uint32_t wv[4] = {w[v].x, w[v].y, w[v].z, w[v].w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {                          // elements 16 u .. 16 u + 15
+                const uint32_t x = wv[u] ^ 0xAAAAAAAAu;               // fields n + 2
+                const uint32_t m2 = 0x03030303u;
+                const uint32_t f0 = x & m2, f1 = (x >> 2) & m2, f2 = (x >> 4) & m2, f3 = (x >> 6) & m2;
+                const uint32_t a = __byte_perm(f0, f1, 0x5140), b = __byte_perm(f2, f3, 0x5140);   // 0 1 4 5, 2 3 6 7
+                const uint32_t c = __byte_perm(f0, f1, 0x7362), d = __byte_perm(f2, f3, 0x7362);   // 8 9 12 13, 10 11 14 15
+                uint4 o0, o1;
+                cvt_u4x4_f16<2>(__byte_perm(a, b, 0x5410), o0.x, o0.y);
+                cvt_u4x4_f16<2>(__byte_perm(a, b, 0x7632), o0.z, o0.w);
+                cvt_u4x4_f16<2>(__byte_perm(c, d, 0x5410), o1.x, o1.y);
+                cvt_u4x4_f16<2>(__byte_perm(c, d, 0x7632), o1.z, o1.w);
+                *reinterpret_cast<uint4*>(st + MmaStage::BH + ((2 * u) * 128 + r) * 16) = o0;
+                *reinterpret_cast<uint4*>(st + MmaStage::BH + ((2 * u + 1) * 128 + r) * 16) = o1;
+              }
             }
           }
           if (WBITS == 4) {
@@ -690,6 +725,8 @@ cudaError_t launch_expert_mma(bool gateup, const MmaArgs& a, cudaStream_t st) {
   const int max_items = a.max_tiles * std::max(per_r, per_s);
   if (a.b[0].wbits == 8)
     return gateup ? launch_mma_t<8, true>(a, max_items, st) : launch_mma_t<8, false>(a, max_items, st);
+  if (a.b[0].wbits == 2)
+    return gateup ? launch_mma_t<2, true>(a, max_items, st) : launch_mma_t<2, false>(a, max_items, st);
   return gateup ? launch_mma_t<4, true>(a, max_items, st) : launch_mma_t<4, false>(a, max_items, st);
 }
 

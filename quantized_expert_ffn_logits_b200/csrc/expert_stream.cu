@@ -51,10 +51,14 @@ constexpr int kSmemMax = 227 * 1024;
 constexpr int kRouteBytes = 6 * 32 * 4 + 32;
 
 struct RingPlan {
-  int ring, sring, bars, abuf, abytes, ascale, xsum, sxf, idot, ubuf, hq, info, route, total;
+  int ring, sring, sstage, bars, abuf, abytes, ascale, xsum, sxf, idot, ubuf, hq, info, route, total;
 };
 
-__host__ __device__ inline RingPlan ring_plan(int K, int tm) {
+// Bytes of one stage's scales: a chunk's fp16 group scales (16 pieces of codes hold 8, 16 or
+// 32 groups of 128 rows for int8, int4, int2) or its down blocks' scales.
+__host__ __device__ inline int ring_sstage(int wbits) { return wbits >= 4 ? 4096 : 16384 / wbits; }
+
+__host__ __device__ inline RingPlan ring_plan(int K, int tm, int wbits) {
   RingPlan p;
   const int G = K / 32;
   int o = 0;
@@ -65,7 +69,8 @@ __host__ __device__ inline RingPlan ring_plan(int K, int tm) {
     return at;
   };
   p.ring = take(kNS * kSP * kPiece);            // 128 KB
-  p.sring = take(kNS * kSP * 128 * 2);          // group / row scales of a stage
+  p.sstage = ring_sstage(wbits);
+  p.sring = take(kNS * p.sstage);               // group / row scales of a stage
   p.bars = take((2 * kNS + 4) * 8);
   p.ascale = tm * K;                            // offset of the scales inside a buffer
   p.abytes = (tm * K + tm * G * 2 + 127) & ~127;
@@ -82,9 +87,9 @@ __host__ __device__ inline RingPlan ring_plan(int K, int tm) {
 }
 
 // Tokens per pass: up to kTMP, as many as shared memory allows.
-inline int ring_tokens(int K, int max_tokens) {
+inline int ring_tokens(int K, int max_tokens, int wbits) {
   int tm = max_tokens < 1 ? 1 : (max_tokens > kTMP ? kTMP : max_tokens);
-  while (tm > 1 && ring_plan(K, tm).total > kSmemMax) --tm;
+  while (tm > 1 && ring_plan(K, tm, wbits).total > kSmemMax) --tm;
   return tm;
 }
 
@@ -174,7 +179,8 @@ __device__ __forceinline__ int down_rotation(const Unit& U, int nch) {
 
 struct Ring {
   uint8_t* ring;
-  uint8_t* sring;
+  uint8_t* sring;     // [kNS][sstage]
+  int sstage;
   uint64_t* full;     // [kNS]
   uint64_t* empty;    // [kNS]
   uint64_t* afull;    // [2]
@@ -210,6 +216,14 @@ __device__ __forceinline__ void act_deinterleave(uint8_t* xs, int words, int tid
     uint2 o;
     deinterleave8(v.x, v.y, o.x, o.y);
     *wp = o;
+  }
+}
+// int2 weights: each 16-byte word of the activation rows de-interleaved into the order of a
+// packed int2 word's fields (elements i, i + 4, i + 8, i + 12 for i = 0 .. 3).
+__device__ __forceinline__ void act_deinterleave16(uint8_t* xs, int words, int tid, int nt) {
+  for (int l = tid; l < words; l += nt) {
+    uint4* wp = reinterpret_cast<uint4*>(xs) + l;
+    *wp = deinterleave16(*wp);
   }
 }
 __device__ __forceinline__ void act_group_sums(const uint8_t* xs, int* xsum, int m, int K, int tid, int nt) {
@@ -704,8 +718,8 @@ __device__ __forceinline__ bool unit_of_token(const RingArgs& A, const RouteSmem
 // (fp16 [block][2][128] or fp32 per row).
 template <int WBITS, bool WG32, bool AG32, int MODE, bool TOPP>
 __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& R, const RouteSmem& S) {
-  constexpr int PPG = WBITS == 8 ? 2 : 1;
-  constexpr int PPU = WBITS == 8 ? 4 : 2;   // pieces of a row's 64-column down slice
+  constexpr int GPP4 = 16 / WBITS;          // 4 x groups per 16-byte piece (int8 2, int4 4, int2 8)
+  constexpr int PPU = WBITS / 2;            // pieces of a row's 64-column down slice
   constexpr int NBC = kSP / PPU;            // 128-row down blocks per chunk
   constexpr int kern = MODE == 1 ? 2 : 1;
   int* status = A.x[0][0].status;
@@ -720,7 +734,7 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
     }
     mbar_arrive_expect_tx(&R.full[st], wbytes + sbytes);
     bulk_load_hint(R.ring + st * (kSP * kPiece), w, wbytes, &R.full[st], once);
-    if (sbytes) bulk_load_hint(R.sring + st * (kSP * 256), sc, sbytes, &R.full[st], once);
+    if (sbytes) bulk_load_hint(R.sring + st * R.sstage, sc, sbytes, &R.full[st], once);
     ++c;
     return true;
   };
@@ -744,7 +758,7 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
         for (int p0 = 0; p0 < NP && ok; p0 += kSP) {
           const int np = min(kSP, NP - p0);
           ok = push(wsrc + (int64_t)p0 * kPiece, (uint32_t)np * kPiece,
-                    ssrc + (int64_t)(p0 / PPG) * 256, WG32 ? (uint32_t)(np / PPG) * 256 : 0u);
+                    ssrc + (int64_t)(p0 * GPP4 / 4) * 256, WG32 ? (uint32_t)(np * GPP4 / 4) * 256 : 0u);
           if (!ok || p0 != 0) continue;
           if (MODE == 3) continue;   // the CTA quantized the token's activations itself
           // this pass's activation rows, behind its first chunk
@@ -812,13 +826,21 @@ __device__ __forceinline__ void block_dots(const uint8_t* stage, int j0, int gba
                                            const uint8_t* xs, int K, const int* xsum, int G, int* idot) {
   constexpr int PPG = WBITS == 8 ? 2 : 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = gbase + j0 + warp;                     // this warp's group
-  const uint8_t* wp = stage + (j0 + warp) * PPG * kPiece + lane * 16;
+  const int gg = j0 + warp;                            // this warp's group inside the chunk
+  const int g = gbase + gg;                            // ... and inside the row
+  // int8: two pieces per group, int4: one, int2: 8 bytes (half of one) of each row
+  const uint8_t* wp = WBITS == 2 ? stage + (gg >> 1) * kPiece + lane * 16 + (gg & 1) * 8
+                                 : stage + gg * PPG * kPiece + lane * 16;
   uint4 w[4 * PPG];
+  uint2 w2[4];
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    w[r * PPG] = *reinterpret_cast<const uint4*>(wp + r * 512);
-    if (WBITS == 8) w[r * PPG + 1] = *reinterpret_cast<const uint4*>(wp + kPiece + r * 512);
+    if (WBITS == 2) {
+      w2[r] = *reinterpret_cast<const uint2*>(wp + r * 512);
+    } else {
+      w[r * PPG] = *reinterpret_cast<const uint4*>(wp + r * 512);
+      if (WBITS == 8) w[r * PPG + 1] = *reinterpret_cast<const uint4*>(wp + kPiece + r * 512);
+    }
   }
   int* out = idot + warp * tm * kRows + lane;
   const int mq = TM == 1 ? 1 : m;          // TM: compile-time bound on the pass's tokens
@@ -827,14 +849,16 @@ __device__ __forceinline__ void block_dots(const uint8_t* stage, int j0, int gba
     const uint4 x0 = *reinterpret_cast<const uint4*>(xg);
     const uint4 x1 = *reinterpret_cast<const uint4*>(xg + 16);
     int xsg = 0;
-    if (WBITS == 4) xsg = xsum[q * G + g];
+    if (WBITS != 8) xsg = xsum[q * G + g];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       int d;
       if (WBITS == 8)
         d = group_dot_i8(w[2 * r], w[2 * r + 1], x0, x1);
-      else
+      else if (WBITS == 4)
         d = group_dot_i4(w[r], make_uint4(x0.x, x0.z, x1.x, x1.z), make_uint4(x0.y, x0.w, x1.y, x1.w), xsg);
+      else
+        d = group_dot_i2(w2[r], x0, x1, xsg);   // activations de-interleaved per 16
       out[q * kRows + r * 32] = d;
     }
   }
@@ -886,7 +910,7 @@ __device__ __forceinline__ void ring_consume(int K, int m, int tm, const Ring& R
                                              const int* xsum, int* idot, float sw_row,
                                              float v[kTMP / 2], volatile int* abort, int* status,
                                              int kernel) {
-  constexpr int PPG = WBITS == 8 ? 2 : 1;
+  constexpr int GPP4 = 16 / WBITS;          // 4 x groups per 16-byte piece
   const int lane = threadIdx.x & 31;
   const int ts = threadIdx.x >> 7;
   const bool chain_thread = ts < m;
@@ -909,8 +933,8 @@ __device__ __forceinline__ void ring_consume(int K, int m, int tm, const Ring& R
     }
     ok = __all_sync(0xffffffffu, ok);
     const uint8_t* stage = R.ring + st * (kSP * kPiece);
-    const __half* sst = reinterpret_cast<const __half*>(R.sring + st * (kSP * 256));
-    const int gbase = p0 / PPG, ng = np / PPG;
+    const __half* sst = reinterpret_cast<const __half*>(R.sring + st * R.sstage);
+    const int gbase = p0 * GPP4 / 4, ng = np * GPP4 / 4;
     // blocks of 8 groups; a short last chunk (K a multiple of 128 but not of 256 / 512)
     // ends with a block of 4, handled by the first four warps and chain steps
     for (int j0 = 0; j0 < ng; j0 += 8, ++nblk) {
@@ -973,7 +997,7 @@ __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& 
                                              const int* hxs, const float* hs, const int* toks,
                                              const float* wts, float* y, float* dbg, int32_t* ddots, int GI,
                                              int sub, int slot0, volatile int* abort, int* status) {
-  constexpr int PPU = WBITS == 8 ? 4 : 2;
+  constexpr int PPU = WBITS / 2;                  // pieces of a row's 64 columns
   constexpr int NBC = kSP / PPU;
   constexpr int RPT = NBC * kRows / (32 * kCW);   // rows per thread of a full chunk
   const int lane = threadIdx.x & 31;
@@ -992,7 +1016,7 @@ __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& 
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       const uint8_t* stage = R.ring + st * (kSP * kPiece);
-      const uint8_t* sst = R.sring + st * (kSP * 256);
+      const uint8_t* sst = R.sring + st * R.sstage;
       uint4 w[RPT][PPU];
       float c0s[RPT], c1s[RPT];
 #pragma unroll
@@ -1027,11 +1051,15 @@ __device__ __forceinline__ void down_consume(int H, int m, int rot, const Ring& 
           if (WBITS == 8) {
             d0 = group_dot_i8(w[k][0], w[k][1], x0, x1);
             d1 = group_dot_i8(w[k][2], w[k][3], x2, x3);
-          } else {
+          } else if (WBITS == 4) {
             d0 = group_dot_i4(w[k][0], make_uint4(x0.x, x0.z, x1.x, x1.z), make_uint4(x0.y, x0.w, x1.y, x1.w),
                               hxs[2 * q]);
             d1 = group_dot_i4(w[k][1], make_uint4(x2.x, x2.z, x3.x, x3.z), make_uint4(x2.y, x2.w, x3.y, x3.w),
                               hxs[2 * q + 1]);
+          } else {
+            // int2: the row's 64 codes are one piece, h de-interleaved per 16
+            d0 = group_dot_i2(make_uint2(w[k][0].x, w[k][0].y), x0, x1, hxs[2 * q]);
+            d1 = group_dot_i2(make_uint2(w[k][0].z, w[k][0].w), x2, x3, hxs[2 * q + 1]);
           }
           float v;
           if (WG32 && AG32)
@@ -1071,10 +1099,11 @@ template <int WBITS, bool WG32, bool AG32, int MODE, int TM, bool TOPP>
 __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ RingArgs A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_align1024(smem_raw);
-  const RingPlan P = ring_plan(A.kmax, A.tm);
+  const RingPlan P = ring_plan(A.kmax, A.tm, WBITS);
   Ring R;
   R.ring = base + P.ring;
   R.sring = base + P.sring;
+  R.sstage = P.sstage;
   R.full = reinterpret_cast<uint64_t*>(base + P.bars);
   R.empty = R.full + kNS;
   R.afull = R.empty + kNS;
@@ -1152,10 +1181,11 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   bool ywait = !(MODE == 3 && A.cluster);   // cluster exchange: y-zero barrier still to wait on
   if (MODE == 3) {
     // off the path to the first weight copy: the routing weights (read only by this warp's
-    // ctid 0) and, int4 weights, the token's de-interleaved codes and group sums
+    // ctid 0) and, int4 / int2 weights, the token's de-interleaved codes and group sums
     if (warp == 0) route_weights<TOPP>(A.r, P, R, S);
-    if (WBITS == 4) {
-      act_deinterleave(R.abuf, A.kmax / 8, ctid, 32 * kCW);
+    if (WBITS != 8) {
+      if (WBITS == 4) act_deinterleave(R.abuf, A.kmax / 8, ctid, 32 * kCW);
+      else act_deinterleave16(R.abuf, A.kmax / 16, ctid, 32 * kCW);
       named_bar(1, 32 * kCW);
       act_group_sums(R.abuf, R.xsum, 1, A.kmax, ctid, 32 * kCW);
     }
@@ -1221,10 +1251,14 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
           if (lane == 0) wait_failed(status, 1, 5, b);
           aok = false;
         }
-        if (WBITS == 4 && MODE != 3) {
-          // de-interleave each 8-byte word into even / odd elements; per-group sums
-          // (barriers taken by every consumer thread, whatever its wait returned)
-          if (aok) act_deinterleave(xs, m * (K / 8), ctid, 32 * kCW);
+        if (WBITS != 8 && MODE != 3) {
+          // de-interleave each 8-byte word into even / odd elements (int4) or each 16-byte
+          // word by fours (int2); per-group sums (barriers taken by every consumer thread,
+          // whatever its wait returned)
+          if (aok) {
+            if (WBITS == 4) act_deinterleave(xs, m * (K / 8), ctid, 32 * kCW);
+            else act_deinterleave16(xs, m * (K / 16), ctid, 32 * kCW);
+          }
           named_bar(1, 32 * kCW);
           if (aok) act_group_sums(xs, xsum, m, K, ctid, 32 * kCW);
         }
@@ -1286,30 +1320,25 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
         }
         named_bar(1, 32 * kCW);            // h codes / scales of the pass in shared memory
         const uint8_t* hx = hq;
-        if (WBITS == 4) {
-          if (ctid < 8 * m) {
+        if (WBITS != 8) {
+          // the h codes in the order of the packed weights' fields, and their group sums
+          if (WBITS == 4 && ctid < 8 * m) {
             const uint2 v = reinterpret_cast<const uint2*>(hq)[ctid];
             uint2 o;
             deinterleave8(v.x, v.y, o.x, o.y);
             reinterpret_cast<uint2*>(hqd)[ctid] = o;
           }
+          if (WBITS == 2 && ctid < 4 * m)
+            reinterpret_cast<uint4*>(hqd)[ctid] = deinterleave16(reinterpret_cast<const uint4*>(hq)[ctid]);
           if (ctid < 2 * m) {
             const uint4* q4 = reinterpret_cast<const uint4*>(hq + ctid * 32);
-            const uint4 a0 = q4[0], a1 = q4[1];
-            int sacc = __dp4a((int)a0.x, 0x01010101, 0);
-            sacc = __dp4a((int)a0.y, 0x01010101, sacc);
-            sacc = __dp4a((int)a0.z, 0x01010101, sacc);
-            sacc = __dp4a((int)a0.w, 0x01010101, sacc);
-            sacc = __dp4a((int)a1.x, 0x01010101, sacc);
-            sacc = __dp4a((int)a1.y, 0x01010101, sacc);
-            sacc = __dp4a((int)a1.z, 0x01010101, sacc);
-            sacc = __dp4a((int)a1.w, 0x01010101, sacc);
-            hxs[ctid] = sacc;
+            hxs[ctid] = code_sum32(q4[0], q4[1]);
           }
           named_bar(1, 32 * kCW);
           hx = hqd;
         }
-        const int rot = down_rotation(U, (d.b.H / kRows + kSP / (WBITS == 8 ? 4 : 2) - 1) / (kSP / (WBITS == 8 ? 4 : 2)));
+        constexpr int NBC = kSP / (WBITS / 2);   // 128-row down blocks per chunk
+        const int rot = down_rotation(U, (d.b.H / kRows + NBC - 1) / NBC);
         down_consume<WBITS, WG32, AG32, TM>(d.b.H, m, rot, R, c, hx, hxs, hs, toks, wts, d.y, d.dbg_a, d.dbg_dots,
                                             d.b.I / 32, U.sub, c0, abort, status);
       }
@@ -1329,7 +1358,7 @@ int decode_grid(int units, int E) { return std::min(sm_count(), std::max(units, 
 
 template <int WBITS, bool WG32, bool AG32, int MODE, int TM, bool TOPP = false>
 cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
-  const RingPlan P = ring_plan(A.kmax, A.tm);
+  const RingPlan P = ring_plan(A.kmax, A.tm, WBITS);
   {
     const cudaError_t e = ensure_smem_attr((const void*)k_expert_ring<WBITS, WG32, AG32, MODE, TM, TOPP>, P.total);
     if (e != cudaSuccess) return e;
@@ -1470,10 +1499,14 @@ cudaError_t launch_experts(int mode, const ExpertArgs& gr, const ExpertArgs* gs,
   A.routed = gr.max_active * A.per;
   A.units = A.routed + (gs ? gs->b.I / 64 : 0);
   A.kmax = mode == 1 ? 64 : gr.b.H;           // K of the staged activation rows
-  A.tm = ring_tokens(A.kmax, gr.T);
+  A.tm = ring_tokens(A.kmax, gr.T, gr.b.wbits);
   A.mma_min = mma_min;
-  const int sel = (gr.b.wbits == 8 ? 4 : 0) | (gr.b.wg32 ? 2 : 0) | (gr.ag32 ? 1 : 0);
+  const int sel = (gr.b.wbits == 8 ? 4 : gr.b.wbits == 2 ? 8 : 0) | (gr.b.wg32 ? 2 : 0) | (gr.ag32 ? 1 : 0);
   switch (sel) {
+    case 11: return launch_mode<2, true, true>(mode, A, st);
+    case 10: return launch_mode<2, true, false>(mode, A, st);
+    case 9: return launch_mode<2, false, true>(mode, A, st);
+    case 8: return launch_mode<2, false, false>(mode, A, st);
     case 7: return launch_mode<8, true, true>(mode, A, st);
     case 6: return launch_mode<8, true, false>(mode, A, st);
     case 5: return launch_mode<8, false, true>(mode, A, st);
@@ -1509,8 +1542,10 @@ cudaError_t launch_decode(const RouteArgs& r, const ExpertArgs& gr, const Expert
   A.tm = 1;
   A.mma_min = 0x7fffffff;
   A.r = r;
-  const int sel = (gr.b.wbits == 8 ? 2 : 0) | (gr.b.wg32 ? 1 : 0);
+  const int sel = (gr.b.wbits == 8 ? 2 : gr.b.wbits == 2 ? 4 : 0) | (gr.b.wg32 ? 1 : 0);
   switch (sel) {
+    case 5: return launch_decode_t<2, true>(A, st);
+    case 4: return launch_decode_t<2, false>(A, st);
     case 3: return launch_decode_t<8, true>(A, st);
     case 2: return launch_decode_t<8, false>(A, st);
     case 1: return launch_decode_t<4, true>(A, st);

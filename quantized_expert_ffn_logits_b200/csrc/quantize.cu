@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const WSource w, BlobV
   const int lane = threadIdx.x & 31;
   const int64_t n_gu = (int64_t)b.E * 2 * b.I;
   const int64_t n_rows = n_gu + (int64_t)b.E * b.H;
-  const float qmax = b.wbits == 8 ? 127.0f : 7.0f;
+  const float qmax = b.wbits == 8 ? 127.0f : b.wbits == 4 ? 7.0f : 1.0f;   // 2^(bits-1) - 1
   const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t R = warp0; R < n_rows; R += nwarps) {
@@ -92,7 +92,7 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const WSource w, BlobV
     const int G = K / 32;
     const int kb = kbytes(K, b.wbits);
     const int U = b.I / 64, HB = b.H / 128;
-    const int sb = b.wbits == 8 ? 64 : 32;            // bytes of 64 elements
+    const int sb = 8 * b.wbits;                       // bytes of 64 elements
     // byte `byte` of this row's codes -> its place in the tiled region
     auto code_at = [&](int byte) -> uint8_t* {
       if (!down) return gu_w + blk * kb + (int64_t)(byte >> 4) * (128 * 16) + r * 16 + (byte & 15);
@@ -126,9 +126,16 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const WSource w, BlobV
       const int q = quant_code(v, s, qmax);
       if (b.wbits == 8) {
         *code_at(32 * g + lane) = (uint8_t)(int8_t)q;
-      } else {
+      } else if (b.wbits == 4) {
         const int hi = __shfl_down_sync(0xffffffffu, q, 1);
         if ((lane & 1) == 0) *code_at(16 * g + (lane >> 1)) = (uint8_t)((q & 15) | ((hi & 15) << 4));
+      } else {
+        // four 2-bit fields per byte: element 4j + i in bits 2i .. 2i + 1
+        const int q1 = __shfl_down_sync(0xffffffffu, q, 1);
+        const int q2 = __shfl_down_sync(0xffffffffu, q, 2);
+        const int q3 = __shfl_down_sync(0xffffffffu, q, 3);
+        if ((lane & 3) == 0)
+          *code_at(8 * g + (lane >> 2)) = (uint8_t)((q & 3) | ((q1 & 3) << 2) | ((q2 & 3) << 4) | ((q3 & 3) << 6));
       }
     }
   }

@@ -103,7 +103,7 @@ class LayerConfig:
     score: str                  # "softmax" | "sigmoid"
     renormalize: bool
     rsf: float                  # routed_scaling_factor (1.0 for softmax models)
-    wtype: str                  # "int8" | "int4"
+    wtype: str                  # "int8" | "int4" | "int2"
     wscale: str                 # "row_f32" | "g32_f16"
     act: str                    # "token_f32" | "g32_f16"
     shared_I: int = 0           # 0 = no shared expert
@@ -145,8 +145,13 @@ CONFIGS = {
     "e512_int4": LayerConfig("e512_int4", H=2048, E=512, I=512, top_k=10, score="softmax",
                              renormalize=False, rsf=1.0, wtype="int4", wscale="g32_f16",
                              act="g32_f16", shared_I=512, tokens=(1, 64, 4096), zipf=1.1),
+    # the OLMoE-shaped decode layer with packed int2 experts (group-32 scales): the third code
+    # container of the GLM page's quantization kernels
+    "olmoe_int2": LayerConfig("olmoe_int2", H=2048, E=64, I=1024, top_k=8, score="softmax",
+                              renormalize=True, rsf=1.0, wtype="int2", wscale="g32_f16",
+                              act="g32_f16", tokens=(1, 8)),
 }
-CONFIG_ORDER = ["tiny", "olmoe_int8", "olmoe_int4", "glm_int4", "e512_int4"]
+CONFIG_ORDER = ["tiny", "olmoe_int8", "olmoe_int4", "glm_int4", "e512_int4", "olmoe_int2"]
 
 
 def case_seed(cfg: LayerConfig, T: int, replica: int = 0) -> int:

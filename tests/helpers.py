@@ -12,7 +12,7 @@ MAX_ABS = 1e-4     # layer output: max |error| relative to max |y_ref|
 
 
 def wbits(cfg):
-    return 8 if cfg.wtype == "int8" else 4
+    return {"int8": 8, "int4": 4, "int2": 2}[cfg.wtype]
 
 
 def wg32(cfg):

@@ -37,14 +37,14 @@ def test_version_and_status_strings():
     assert M.moe_status_string(99) == "MOE_ERR_UNKNOWN"
 
 
-@pytest.mark.parametrize("wtype,wscale", [(0, 0), (0, 1), (1, 0), (1, 1)])
+@pytest.mark.parametrize("wtype,wscale", [(0, 0), (0, 1), (1, 0), (1, 1), (2, 0), (2, 1)])
 @pytest.mark.parametrize("E,H,I", [(8, 256, 128), (64, 2048, 1024), (256, 6144, 2048), (1, 2048, 512)])
 def test_blob_bytes_match_documented_layout(wtype, wscale, E, H, I):
     got = M.moe_expert_blob_bytes(wtype, wscale, E, H, I)
-    assert got == O.blob_layout(E, H, I, 8 if wtype == 0 else 4, wscale == 1)[4]
+    assert got == O.blob_layout(E, H, I, {0: 8, 1: 4, 2: 2}[wtype], wscale == 1)[4]
 
 
-@pytest.mark.parametrize("args", [(0, 0, 8, 96, 128), (0, 0, 8, 256, 100), (2, 0, 8, 256, 128),
+@pytest.mark.parametrize("args", [(0, 0, 8, 96, 128), (0, 0, 8, 256, 100), (3, 0, 8, 256, 128),
                                   (0, 3, 8, 256, 128), (0, 0, 0, 256, 128), (0, 0, 2000, 256, 128)])
 def test_blob_bytes_reject_unsupported(args):
     assert M.moe_expert_blob_bytes(*args) == 0

@@ -28,6 +28,8 @@ FULL = [
     ("olmoe_int4", 512, 32),       # tensor-core path (experts with >= 16 pairs)
     ("olmoe_int4", 4096, 64),
     ("e512_int4", 4096, 64),       # Zipf-skewed: tensor cores for hot experts, streaming for the rest
+    ("olmoe_int2", 1, None),       # packed int2 experts: the single-token kernel
+    ("olmoe_int2", 8, None),
 ]
 MMA_MIN_PAIRS = 16                 # pairs an expert needs in a call for the tensor-core path
 

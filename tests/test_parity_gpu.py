@@ -38,13 +38,19 @@ REDUCED = {
                                        renormalize=True),
     "int4_row_tok": BASE["glm_int4"].with_(name="int4_row_tok", H=256, E=16, I=128, top_k=4,
                                            act="token_f32", shared_I=256),
+    # packed int2 experts (the GLM page's third container): group-32 scales and activations,
+    # and per-row scales with per-token activations and a shared expert
+    "int2_g32": BASE["olmoe_int2"].with_(name="int2_g32", H=512, E=16, I=256, top_k=4),
+    "int2_row_tok": BASE["olmoe_int2"].with_(name="int2_row_tok", H=384, E=8, I=128, top_k=3,
+                                             wscale="row_f32", act="token_f32", shared_I=128),
 }
 CASES = [("tiny", 1), ("tiny", 4), ("tiny", 37),
          ("olmoe_int8", 1), ("olmoe_int8", 8), ("olmoe_int8", 33), ("olmoe_int8", 70),
          ("olmoe_int4", 1), ("olmoe_int4", 40), ("olmoe_int4", 130),
          ("glm_int4", 1), ("glm_int4", 4), ("glm_int4", 50),
          ("e512_int4", 1), ("e512_int4", 64), ("e512_int4", 100),
-         ("int8_g32_tok", 5), ("int4_g32_tok", 9), ("int8_row_g32", 6), ("int4_row_tok", 3)]
+         ("int8_g32_tok", 5), ("int4_g32_tok", 9), ("int8_row_g32", 6), ("int4_row_tok", 3),
+         ("int2_g32", 1), ("int2_g32", 8), ("int2_g32", 37), ("int2_row_tok", 1), ("int2_row_tok", 5)]
 
 
 def _np(t):
@@ -70,7 +76,7 @@ def test_layer_forward_matches_oracle(name, T):
 # The tensor-core path (experts with >= 16 pairs at T > 32; every expert with the force flag):
 # the same bit-exact gate/up values, h codes and scales as the streaming path and the oracle.
 MMA_CASES = [("olmoe_int4", 300, False), ("olmoe_int4", 40, True), ("olmoe_int8", 70, True),
-             ("e512_int4", 100, True), ("glm_int4", 50, True)]
+             ("e512_int4", 100, True), ("glm_int4", 50, True), ("int2_g32", 300, False), ("int2_g32", 40, True)]
 
 
 @pytest.mark.parametrize("name,T,force", MMA_CASES)
@@ -274,7 +280,8 @@ def test_synth_device_generator_matches_host():
 
 
 @pytest.mark.parametrize("wtype,wscale", [("int8", "row_f32"), ("int8", "g32_f16"),
-                                          ("int4", "row_f32"), ("int4", "g32_f16")])
+                                          ("int4", "row_f32"), ("int4", "g32_f16"),
+                                          ("int2", "row_f32"), ("int2", "g32_f16")])
 @pytest.mark.parametrize("E,H,I", [(3, 256, 128), (2, 384, 256)])
 def test_quantize_experts_blob_bytes_identical(wtype, wscale, E, H, I):
     m = M()
@@ -385,7 +392,8 @@ def test_permute_flags_out_of_range_expert():
     assert m.moe_read_device_status(ws) == m.MOE_OK
 
 
-@pytest.mark.parametrize("wtype,wscale", [("int8", "g32_f16"), ("int4", "g32_f16"), ("int4", "row_f32")])
+@pytest.mark.parametrize("wtype,wscale", [("int8", "g32_f16"), ("int4", "g32_f16"), ("int4", "row_f32"),
+                                          ("int2", "g32_f16"), ("int2", "row_f32")])
 def test_expert_group_dots_bit_exact(wtype, wscale):
     m = M()
     c = S.CONFIGS["olmoe_int8"].with_(E=4, H=512, I=256, wtype=wtype, wscale=wscale)
@@ -486,15 +494,16 @@ def test_tensor_core_dots_exact_at_extreme_codes(wtype):
     assert_close_y(_np(y), ref["y"])
 
 
-@pytest.mark.parametrize("wtype", ["int8", "int4"])
+@pytest.mark.parametrize("wtype", ["int8", "int4", "int2"])
 @pytest.mark.parametrize("path", ["mma", "stream"])
 def test_down_dots_exact_at_extreme_codes(wtype, path):
     """The down projection at its largest group dots, on both expert paths: every gate and up
     row is the same +-1 pattern and every token agrees with it in most signs, so for each token
     all of its h values are equal and positive and every h code is +127; half of the down rows
     are all +1 (codes +127 / +7), the rest random
-    signs, so group dots reach 32 * 127 * 127 (int8) or 32 * 127 * 7 (int4) -- partial sums far
-    above fp16's integer range, exact only in the fp32 accumulator. The down group dots must
+    signs, so group dots reach 32 * 127 * 127 (int8), 32 * 127 * 7 (int4) or 32 * 127 (int2) --
+    partial sums far above fp16's integer range, exact only in the fp32 accumulator. The down
+    group dots must
     equal the exact integer dots bit for bit, and y must meet the layer tolerance."""
     m = M()
     rng = np.random.default_rng(91)
@@ -506,7 +515,7 @@ def test_down_dots_exact_at_extreme_codes(wtype, path):
     dn = np.where(rng.random((E, H, I)) < 0.5, -1.0, 1.0).astype(np.float32)
     dn[:, ::2, :] = 1.0
     wr = rng.normal(0.0, 1.0 / np.sqrt(H), (E, H)).astype(np.float32)
-    wb = 8 if wtype == "int8" else 4
+    wb = {"int8": 8, "int4": 4, "int2": 2}[wtype]
     ex = O.QExperts.quantize(gu, dn, wb, True)
     ref = O.layer_forward(x, wr, None, ex, None, "softmax", k, True, 1.0, True, union=True)
     ref["experts"] = (ex, None)
@@ -525,7 +534,7 @@ def test_down_dots_exact_at_extreme_codes(wtype, path):
     case = S.Case(S.CONFIGS["olmoe_int8"].with_(E=E, H=H, I=I, top_k=k, shared_I=0), T, 0)
     _check_down_dots(m, ws, v, case, ref, perm)
     got = _np(m.workspace_view(ws, v["dn_dots"], torch.int32, (T * k, H, I // 32)))
-    assert np.abs(got).max() == 32 * 127 * (127 if wtype == "int8" else 7)
+    assert np.abs(got).max() == 32 * 127 * O.QMAX[wb]
     assert_close_y(_np(y), ref["y"])
 
 
