@@ -65,7 +65,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 3
+#define MOE_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define MOE_API __attribute__((visibility("default")))
@@ -156,6 +156,20 @@ typedef struct {
                                    their experts are not read for that token; with renormalize
                                    the kept weights are renormalized over the kept experts.
                                    Must be finite and >= 0 (else MOE_ERR_INVALID_ARG). */
+  int32_t n_experts_total;      /* expert parallelism (the GLM-5.2 colibri page, "Experimental
+                                   resident CUDA backend": whole experts placed on devices). 0 = the
+                                   layer holds every expert (E = experts->n_experts). Otherwise the
+                                   router has n_experts_total experts (router_w [n_experts_total][H],
+                                   router_bias [n_experts_total]) and `experts` holds the contiguous
+                                   range expert_begin .. expert_begin + experts->n_experts - 1 of
+                                   them: every token is routed over all n_experts_total experts
+                                   (idx and w hold global ids and weights, the same on every
+                                   device), and only pairs whose expert is in the range are computed
+                                   and added into y. Summing y over devices that hold disjoint ranges
+                                   covering all experts (the shared expert on one of them) gives the
+                                   layer. Requires expert_begin >= 0, expert_begin + n_experts <=
+                                   n_experts_total <= 1024 (else MOE_ERR_UNSUPPORTED). */
+  int32_t expert_begin;         /* first global expert id held by `experts` (0 without EP) */
 } moe_route_cfg;
 
 /* Version of this ABI (MOE_ABI_VERSION). */

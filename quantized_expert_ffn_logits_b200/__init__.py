@@ -44,7 +44,7 @@ class moe_expert_blob(C.Structure):
 class moe_route_cfg(C.Structure):
     _fields_ = [("score", C.c_int32), ("top_k", C.c_int32), ("renormalize", C.c_int32),
                 ("routed_scaling_factor", C.c_float), ("act", C.c_int32), ("flags", C.c_uint32),
-                ("top_p", C.c_float)]
+                ("top_p", C.c_float), ("n_experts_total", C.c_int32), ("expert_begin", C.c_int32)]
 
 
 class moe_debug_views(C.Structure):
@@ -93,7 +93,8 @@ for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
     _fn.argtypes = _args
-ABI_VERSION = 3          # the struct layouts above (moe_route_cfg with top_p, moe_debug_views with dn_dots)
+ABI_VERSION = 4          # the struct layouts above (moe_route_cfg with top_p and the expert range,
+                         # moe_debug_views with dn_dots)
 if _lib.moe_abi_version() != ABI_VERSION:
     raise ImportError(f"{LIB_PATH}: ABI version {_lib.moe_abi_version()}, this binding needs "
                       f"{ABI_VERSION}: rebuild the library")
@@ -143,11 +144,13 @@ class RouteCfg:
     act: str = "g32_f16"
     flags: int = 0
     top_p: float = 0.0      # adaptive expert top-p; 0 (or >= 1) = off
+    n_experts_total: int = 0   # expert parallelism: the router's experts (0 = the blob's)
+    expert_begin: int = 0      # ... and the first global expert id the blob holds
 
     def struct(self) -> moe_route_cfg:
         return moe_route_cfg(SCORES[self.score], self.top_k, int(self.renormalize),
                              float(self.routed_scaling_factor), ACTS[self.act], self.flags,
-                             float(self.top_p))
+                             float(self.top_p), int(self.n_experts_total), int(self.expert_begin))
 
 
 class ExpertBlob:

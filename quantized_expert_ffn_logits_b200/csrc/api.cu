@@ -73,10 +73,18 @@ BlobView view(const moe_expert_blob* b, const BlobOffsets& o) {
   return v;
 }
 
-moe_status check_cfg(const moe_route_cfg* c, int32_t E) {
+// The router's experts: all of them (n_experts_total, or the blob's when 0).
+int32_t experts_total(const moe_route_cfg* c, int32_t E_local) {
+  return c->n_experts_total > 0 ? c->n_experts_total : E_local;
+}
+
+moe_status check_cfg(const moe_route_cfg* c, int32_t E_local) {
   if (!c) return MOE_ERR_INVALID_ARG;
   if (c->score != MOE_SCORE_SOFTMAX && c->score != MOE_SCORE_SIGMOID_NOAUX_TC) return MOE_ERR_INVALID_ARG;
   if (c->act != MOE_ACT_TOKEN_F32 && c->act != MOE_ACT_G32_F16) return MOE_ERR_INVALID_ARG;
+  if (c->n_experts_total < 0 || c->expert_begin < 0) return MOE_ERR_UNSUPPORTED;
+  const int32_t E = experts_total(c, E_local);
+  if (E > 1024 || (int64_t)c->expert_begin + E_local > E) return MOE_ERR_UNSUPPORTED;
   if (c->top_k < 1 || c->top_k > 32 || c->top_k > E) return MOE_ERR_UNSUPPORTED;
   if (!(c->top_p >= 0.0f) || !std::isfinite(c->top_p)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
@@ -95,7 +103,8 @@ struct Layout {
   int64_t qh_sh, sh_sh, hbuf_sh, dbg_gate_sh, dbg_up_sh, dbg_y_sh, dbg_dots_sh;   // shared-expert rows
 };
 
-Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k, int32_t ag32,
+// E: experts held here (grouping), E_total: the router's experts (logits).
+Layout layout(int32_t T, int32_t E, int32_t E_total, int32_t H, int32_t I, int32_t Is, int32_t k, int32_t ag32,
               bool debug, bool mma, bool force_mma) {
   Layout L;
   int64_t o = 0;
@@ -109,7 +118,7 @@ Layout layout(int32_t T, int32_t E, int32_t H, int32_t I, int32_t Is, int32_t k,
   L.status = take(kControlBytes);
   L.qx = take((int64_t)T * H);
   L.sx = take(ag32 ? (int64_t)T * (H / 32) * 2 : (int64_t)T * 4);
-  L.logits = take((int64_t)T * E * 4);
+  L.logits = take((int64_t)T * E_total * 4);
   L.idx = take(P * 4);
   L.w = take(P * 4);
   L.offsets = take((int64_t)(E + 1) * 4);
@@ -179,8 +188,9 @@ bool use_mma(int32_t T, const moe_expert_blob* experts, const moe_route_cfg* cfg
 // One token with group-32 activations: routing and every expert in one launch (the expert
 // kernel routes the token itself before a grid barrier).
 bool use_decode(int32_t T, const moe_expert_blob* experts, const moe_route_cfg* cfg) {
-  return T == 1 && cfg->act == MOE_ACT_G32_F16 && experts->n_experts <= 512 && experts->hidden % 128 == 0 &&
-         4 * experts->n_experts <= experts->hidden;
+  const int32_t E = experts_total(cfg, experts->n_experts);
+  return T == 1 && cfg->act == MOE_ACT_G32_F16 && E <= 512 && experts->hidden % 128 == 0 &&
+         4 * E <= experts->hidden;
 }
 
 struct LayerPlan {
@@ -207,7 +217,8 @@ moe_status plan_layer(int32_t T, const moe_expert_blob* experts, const moe_exper
     p.Is = shared->inter;
   }
   p.mma = use_mma(T, experts, cfg);
-  p.L = layout(T, experts->n_experts, experts->hidden, experts->inter, p.Is, cfg->top_k,
+  p.L = layout(T, experts->n_experts, experts_total(cfg, experts->n_experts), experts->hidden,
+               experts->inter, p.Is, cfg->top_k,
                cfg->act == MOE_ACT_G32_F16, (cfg->flags & MOE_FLAG_DEBUG) != 0, p.mma,
                (cfg->flags & MOE_FLAG_FORCE_MMA) != 0);
   return MOE_OK;
@@ -311,7 +322,11 @@ moe_status moe_router_logits(const float* x, const float* router_w, int32_t T, i
 moe_status moe_route_topk(const float* logits, const float* bias, int32_t T, int32_t E,
                           const moe_route_cfg* cfg, int32_t* idx, float* w, void* stream) {
   if (T < 0 || E < 1 || E > 1024) return E > 1024 ? MOE_ERR_UNSUPPORTED : MOE_ERR_INVALID_ARG;
-  const moe_status s = check_cfg(cfg, E);
+  if (!cfg) return MOE_ERR_INVALID_ARG;
+  moe_route_cfg c = *cfg;                 // selection over the E logits given: no expert range
+  c.n_experts_total = 0;
+  c.expert_begin = 0;
+  const moe_status s = check_cfg(&c, E);
   if (s != MOE_OK) return s;
   if (T == 0) return MOE_OK;
   if (!logits || !idx || !w) return MOE_ERR_INVALID_ARG;
@@ -351,7 +366,7 @@ moe_status moe_permute(const int32_t* idx, int32_t T, int32_t k, int32_t E, int3
   g.act_expert = reinterpret_cast<int32_t*>(ws + o);
   o += al256((int64_t)(E + 1) * 4);
   g.act_begin = reinterpret_cast<int32_t*>(ws + o);
-  moe::launch_permute(idx, T, k, E, g, masks, base, reinterpret_cast<int*>(ws), 1,
+  moe::launch_permute(idx, T, k, E, 0, E, g, masks, base, reinterpret_cast<int*>(ws), 1,
                       static_cast<cudaStream_t>(stream));
   return launch_status();
 }
@@ -381,7 +396,8 @@ moe_status moe_layer_debug_views(int32_t T, const moe_expert_blob* experts,
   const size_t total = moe_layer_workspace_bytes(T, experts, shared, cfg);
   if (total == 0) return MOE_ERR_UNSUPPORTED;
   const int32_t Is = shared ? shared->inter : 0;
-  const Layout L = layout(T, experts->n_experts, experts->hidden, experts->inter, Is, cfg->top_k,
+  const Layout L = layout(T, experts->n_experts, experts_total(cfg, experts->n_experts), experts->hidden,
+                          experts->inter, Is, cfg->top_k,
                           cfg->act == MOE_ACT_G32_F16, (cfg->flags & MOE_FLAG_DEBUG) != 0,
                           use_mma(T, experts, cfg), (cfg->flags & MOE_FLAG_FORCE_MMA) != 0);
   out->status = L.status;
@@ -447,7 +463,9 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   const Layout& L = p.L;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   auto at = [&](int64_t off) -> void* { return off < 0 ? nullptr : ws + off; };
+  // E: experts held here (grouping, blob), E_total: the router's (logits, top-k)
   const int32_t E = experts->n_experts, H = experts->hidden, I = experts->inter, k = cfg->top_k;
+  const int32_t E_total = experts_total(cfg, E), e0 = cfg->expert_begin;
   const int ag32 = cfg->act == MOE_ACT_G32_F16;
   int* status = static_cast<int*>(at(L.status));
   const BlobView bv = view(experts, p.eo);
@@ -482,7 +500,9 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     r.wr = router_w;
     r.bias = bias;
     r.T = T;
-    r.E = E;
+    r.E = E_total;
+    r.e0 = e0;
+    r.EL = E;
     r.H = H;
     r.k = k;
     r.score = cfg->score;
@@ -515,15 +535,15 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
     mk.end(MOE_STAGE_QUANT_X);
     // 2. router logits
     mk.begin(MOE_STAGE_ROUTER);
-    moe::launch_router_logits(x, router_w, T, E, H, logits, st);
+    moe::launch_router_logits(x, router_w, T, E_total, H, logits, st);
     mk.end(MOE_STAGE_ROUTER);
     // 3. top-k selection and weights, batch-union grouping
     mk.begin(MOE_STAGE_TOPK);
-    moe::launch_topk(logits, bias, T, E, k, cfg->score, cfg->renormalize != 0,
+    moe::launch_topk(logits, bias, T, E_total, k, cfg->score, cfg->renormalize != 0,
                      cfg->routed_scaling_factor, topp_of(cfg), idx, wts, nullptr, status, st);
     mk.end(MOE_STAGE_TOPK);
     mk.begin(MOE_STAGE_GROUP);
-    moe::launch_permute(idx, T, k, E, g, static_cast<uint32_t*>(at(L.masks)),
+    moe::launch_permute(idx, T, k, E, e0, E_total, g, static_cast<uint32_t*>(at(L.masks)),
                         static_cast<int32_t*>(at(L.base)), status, 0, st);
     mk.end(MOE_STAGE_GROUP);
   }

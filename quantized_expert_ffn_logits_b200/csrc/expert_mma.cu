@@ -189,7 +189,8 @@ constexpr uint32_t kMmaSleepNs = 200;      // backoff of the roles that run ahea
 // same time as suspending waits, which free issue slots the epilogue does not need).
 __device__ __forceinline__ bool mma_wait_ahead(uint64_t* bar, uint32_t parity) {
   return mbar_wait_sleep(bar, parity, kMmaSleepNs);
-}// One accumulator hand-off per 2-group stage: the MMA issuer fills a pair of accumulators
+}
+// One accumulator hand-off per 2-group stage: the MMA issuer fills a pair of accumulators
 // (groups 2i, 2i + 1) and commits once; the epilogue waits once, drains both, releases once.
 constexpr bool kMmaPairCommit = true;
 // Weight blocks are re-read by every tile of their expert: normal L2 policy, not evict-first

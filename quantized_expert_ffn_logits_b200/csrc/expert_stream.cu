@@ -263,6 +263,7 @@ struct RouteSmem {
   volatile int* flag;
   volatile unsigned long long* ytarget;   // y-zero barrier target (cluster exchange)
   volatile int* nk;                       // slots kept: k, or the adaptive top-p prefix
+  volatile int* nl;                       // kept slots whose expert is held here (units)
 };
 
 // Bounds of the cross-CTA waits (grid barrier, y-zero barrier): RouteArgs::wait_ns of
@@ -358,6 +359,27 @@ __device__ __forceinline__ bool stage_router_rows(const RouteArgs& r, bool cl, u
       bulk_load(ring + (int64_t)t * kChunkPitch, r.wr + (int64_t)(o.first + j * o.stride) * r.H + 32 * c, 128, bar);
     }
   return fit;
+}
+
+// Slot j of the token's top-k list (S.sidx, global ids): its local expert id if the slot is
+// kept (j < nk: adaptive top-p) and its expert held here (expert parallelism), else -1.
+__device__ __forceinline__ int kept_local(const RouteArgs& r, const RouteSmem& S, int nk, int j) {
+  const int ee = S.sidx[j];
+  return (j < nk && ee >= r.e0 && ee < r.e0 + r.EL) ? ee - r.e0 : -1;
+}
+// Kept local slots with a local id below le (the position of le in ascending order).
+__device__ __forceinline__ int kept_local_rank(const RouteArgs& r, const RouteSmem& S, int nk, int le) {
+  int pos = 0;
+  for (int j = 0; j < r.k; ++j) {
+    const int o = kept_local(r, S, nk, j);
+    pos += (o >= 0) & (o < le);
+  }
+  return pos;
+}
+__device__ __forceinline__ int kept_local_count(const RouteArgs& r, const RouteSmem& S, int nk) {
+  int n = 0;
+  for (int j = 0; j < r.k; ++j) n += kept_local(r, S, nk, j) >= 0;
+  return n;
 }
 
 // Every thread of the CTA. False when a wait gave up (status recorded; with the cluster
@@ -599,17 +621,19 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
     }
     __syncthreads();
   }
-  // 6. the kept selection in ascending expert order (all the producer needs)
+  // 6. the kept selection whose experts are held here (all of them without expert
+  //    parallelism), by local id, in ascending order (all the producer needs)
   const int nk = TOPP ? *S.nk : k;
+  const int nl = kept_local_count(r, S, nk);
   if (tid < k) {
     const int ee = S.sidx[tid];
-    if (tid < nk) {
-      int pos = 0;
-      for (int j = 0; j < nk; ++j) pos += S.sidx[j] < ee;
-      S.se[pos] = ee;
+    const int le = kept_local(r, S, nk, tid);
+    if (le >= 0) {
+      const int pos = kept_local_rank(r, S, nk, le);
+      S.se[pos] = le;
       S.sj[pos] = tid;
       if (cta0) {
-        r.g.act_expert[pos] = ee;
+        r.g.act_expert[pos] = le;
         r.g.act_begin[pos] = pos;
         r.g.perm[pos] = tid;
         if (r.g.act_rows) r.g.act_rows[pos * 8] = 0;
@@ -617,16 +641,13 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
     }
     if (cta0) r.idx[tid] = tid < nk ? ee : -1;
   }
+  if (tid == 0) *S.nl = nl;
   if (cta0) {
-    for (int x = tid; x < E; x += kNT) {
-      int cnt = 0;
-      for (int j = 0; j < nk; ++j) cnt += S.sidx[j] < x;
-      r.g.offsets[x] = cnt;
-    }
+    for (int x = tid; x < r.EL; x += kNT) r.g.offsets[x] = kept_local_rank(r, S, nk, x);
     if (tid == 0) {
-      r.g.offsets[E] = nk;
-      *r.g.n_active = nk;
-      r.g.act_begin[nk] = nk;
+      r.g.offsets[r.EL] = nl;
+      *r.g.n_active = nl;
+      r.g.act_begin[nl] = nl;
     }
   }
   __syncthreads();
@@ -668,10 +689,9 @@ __device__ __forceinline__ void route_weights(const RouteArgs& r, const RingPlan
     wv = v / cm * r.rsf;
   }
   if (lane < nk) {
-    int pos = 0;
-    for (int j = 0; j < nk; ++j) pos += S.sidx[j] < my_e;
     S.sw[lane] = wv;
-    S.swt[pos] = wv;
+    const int le = kept_local(r, S, nk, lane);   // its weight goes with its unit (held here)
+    if (le >= 0) S.swt[kept_local_rank(r, S, nk, le)] = wv;
   }
   if (on && blockIdx.x == 0) r.w[lane] = lane < nk ? wv : 0.0f;
   __syncwarp();
@@ -679,21 +699,22 @@ __device__ __forceinline__ void route_weights(const RouteArgs& r, const RingPlan
 
 // Work unit u of a MODE 3 grid: routed units (the token's k experts, ascending) first, then
 // the shared expert's. Slot of the routed pair = its active-expert index.
-// nk (TOPP): the token's kept slots, the adaptive top-p prefix; units of dropped slots are none.
+// nl: the token's kept slots whose experts are held here (all k without adaptive top-p or
+// expert parallelism); units of the others are none.
 template <bool TOPP>
-__device__ __forceinline__ bool unit_of_token(const RingArgs& A, const RouteSmem& S, int nk, int u, Unit& U,
+__device__ __forceinline__ bool unit_of_token(const RingArgs& A, const RouteSmem& S, int nl, int u, Unit& U,
                                               bool report) {
   if (u < A.routed) {
     U.shd = false;
     U.ai = u / A.per;
-    if (TOPP && U.ai < A.r.k && U.ai >= nk) return false;   // a slot dropped by adaptive top-p
+    if (U.ai < A.r.k && U.ai >= nl) return false;   // dropped by top-p, or held elsewhere
     U.sub = u - U.ai * A.per;
     U.e = S.se[U.ai];
     U.s0 = U.ai;
     U.s1 = U.ai + 1;
 #pragma unroll
     for (int q = 0; q < 8; ++q) U.rows8[q] = 0;
-    if (U.ai >= A.r.k || U.e < 0 || U.e >= A.r.E) {
+    if (U.ai >= A.r.k || U.e < 0 || U.e >= A.r.EL) {
       if (report) set_status(A.r.status, kStatusDeviceCheck);
       return false;
     }
@@ -738,10 +759,10 @@ __device__ void ring_producer(const RingArgs& A, const RingPlan& P, const Ring& 
     ++c;
     return true;
   };
-  const int nk = (MODE == 3 && TOPP) ? *S.nk : 0;
+  const int nl = MODE == 3 ? *S.nl : 0;
   for (int u = blockIdx.x; u < A.units && ok; u += gridDim.x) {
     Unit U;
-    if (MODE == 3 ? !unit_of_token<TOPP>(A, S, nk, u, U, false)
+    if (MODE == 3 ? !unit_of_token<TOPP>(A, S, nl, u, U, false)
                   : !unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, false,
                              A.mma_min))
       continue;
@@ -1147,6 +1168,7 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   volatile int* rows_flag = S.se + 193;
   S.ytarget = reinterpret_cast<volatile unsigned long long*>(S.se + 194);
   S.nk = S.se + 196;
+  S.nl = S.se + 197;
   __syncthreads();
   bool rows = false;
   if (MODE == 3) {
@@ -1190,10 +1212,10 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
       act_group_sums(R.abuf, R.xsum, 1, A.kmax, ctid, 32 * kCW);
     }
   }
-  const int nk = (MODE == 3 && TOPP) ? *S.nk : 0;
+  const int nl = MODE == 3 ? *S.nl : 0;
   for (int u = blockIdx.x; u < A.units; u += gridDim.x) {
     Unit U;
-    if (MODE == 3 ? !unit_of_token<TOPP>(A, S, nk, u, U, ctid == 0)
+    if (MODE == 3 ? !unit_of_token<TOPP>(A, S, nl, u, U, ctid == 0)
                   : !unit_of(A.x[0][0], A.x[0][1], A.has_shared, A.routed, A.per, u, U, MODE != 1, ctid == 0,
                              A.mma_min))
       continue;

@@ -49,11 +49,13 @@ struct Grouping {            // batch-union grouping outputs (all device pointer
 void launch_topk(const float* logits, const float* bias, int T, int E, int k, int score,
                  int renorm, float rsf, float top_p, int32_t* idx, float* w, const Grouping* single_token,
                  int* status, cudaStream_t st);
-// Pairs with expert -1 (dropped by adaptive top-p) are left out of the grouping.
-// masks/base: scratch [ceil(T/32)][E] each.
+// Pairs with expert -1 (dropped by adaptive top-p) are left out of the grouping, and so are
+// pairs whose global expert id lies outside e0 .. e0 + E - 1 (held elsewhere: expert
+// parallelism); the grouping uses local ids (global - e0). Ids outside [0, e_total) are
+// reported (device check) and dropped. masks/base: scratch [ceil(T/32)][E] each.
 // reset_status: clear the status word first (stand-alone use).
-void launch_permute(const int32_t* idx, int T, int k, int E, const Grouping& g, uint32_t* masks,
-                    int32_t* base, int* status, int reset_status, cudaStream_t st);
+void launch_permute(const int32_t* idx, int T, int k, int E, int e0, int e_total, const Grouping& g,
+                    uint32_t* masks, int32_t* base, int* status, int reset_status, cudaStream_t st);
 
 // ---- expert_stream.cu (weight-streaming expert kernels)
 struct ExpertArgs {
@@ -140,7 +142,9 @@ struct RouteArgs {
   const float* x;
   const float* wr;
   const float* bias;      // sigmoid mode only, may be null
-  int T, E, H, k, score, renorm, ag32;
+  int T, E, H, k, score, renorm, ag32;     // E: the router's experts (all of them)
+  int e0, EL;             // experts held here: global ids e0 .. e0 + EL - 1 (local 0 .. EL - 1);
+                          // the grouping keeps only pairs in that range, with local ids
   float rsf;
   float top_p;            // adaptive expert top-p in (0, 1); 0 = off
   int8_t* qx;

@@ -76,7 +76,7 @@ extern "C" moe_status moe_permute_no_alloc(const int32_t* idx, int32_t T, int32_
   g.act_begin = reinterpret_cast<int32_t*>(ws + o);
   // The kernel zeroes its mask rows before use and resets the status word, so
   // nothing left in the array by an earlier call leaks into this one.
-  moe::launch_permute(idx, T, k, E, g, masks, prefix, reinterpret_cast<int*>(ws), 1,
+  moe::launch_permute(idx, T, k, E, 0, E, g, masks, prefix, reinterpret_cast<int*>(ws), 1,
                       static_cast<cudaStream_t>(stream));
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

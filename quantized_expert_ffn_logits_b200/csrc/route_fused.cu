@@ -199,6 +199,16 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
     }
   }
   __syncthreads();
+  // expert parallelism: the grouping keeps the pairs whose expert is held here (global ids
+  // e0 .. e0 + EL - 1), by local id; the idx / w views keep the global selection
+  const int EL = r.EL;
+  if (r.e0 != 0 || EL != E) {
+    for (int p = tid; p < T * k; p += 256) {
+      const int ee = sel[p];
+      sel[p] = (ee >= r.e0 && ee < r.e0 + EL) ? ee - r.e0 : -1;
+    }
+    __syncthreads();
+  }
   if (T == 1) {
     // one token: the active experts are its kept selections (all k, or the adaptive top-p
     // prefix; dropped slots hold -1), one slot each, in ascending expert order
@@ -208,37 +218,37 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
       const int ee = sel[tid];
       int pos = 0;
       for (int j = 0; j < k; ++j) pos += (sel[j] >= 0) & (sel[j] < ee);
-      if (ee >= 0 && ee < E) {
+      if (ee >= 0 && ee < EL) {
         r.g.act_expert[pos] = ee;
         r.g.act_begin[pos] = pos;
         r.g.perm[pos] = tid;
         if (r.g.act_rows) r.g.act_rows[pos * 8] = 0;
       }
     }
-    for (int x = tid; x < E; x += 256) {
+    for (int x = tid; x < EL; x += 256) {
       int cnt = 0;
       for (int j = 0; j < k; ++j) cnt += (sel[j] >= 0) & (sel[j] < x);
       r.g.offsets[x] = cnt;
     }
     if (tid == 0) {
-      r.g.offsets[E] = nk;
+      r.g.offsets[EL] = nk;
       *r.g.n_active = nk;
       r.g.act_begin[nk] = nk;
       *r.ticket = 0u;
     }
     return;
   }
-  for (int x = tid; x < E; x += 256) masks[x] = 0u;
+  for (int x = tid; x < EL; x += 256) masks[x] = 0u;
   __syncthreads();
 
   // 6. grouping: bit t of masks[e] = token t routes to e; pairs sorted by (expert, token)
   for (int p = tid; p < T * k; p += 256) {
     const int ee = sel[p];
-    if (ee >= 0 && ee < E) atomicOr(&masks[ee], 1u << (p / k));
+    if (ee >= 0 && ee < EL) atomicOr(&masks[ee], 1u << (p / k));
   }
   __syncthreads();
-  const int per = (E + 255) / 256;
-  const int lo = min(tid * per, E), hi = min(lo + per, E);
+  const int per = (EL + 255) / 256;
+  const int lo = min(tid * per, EL), hi = min(lo + per, EL);
   int cnt = 0, nf = 0;
   for (int x = lo; x < hi; ++x) {
     const int c = __popc(masks[x]);
@@ -283,14 +293,14 @@ __global__ void __launch_bounds__(256, 1) k_route_fused(const __grid_constant__ 
     run += c;
   }
   if (tid == 0) {
-    r.g.offsets[E] = total;
+    r.g.offsets[EL] = total;
     *r.g.n_active = ftotal;
     r.g.act_begin[ftotal] = total;
   }
   __syncthreads();
   for (int p = tid; p < T * k; p += 256) {
     const int ee = sel[p];
-    if (ee < 0 || ee >= E) continue;
+    if (ee < 0 || ee >= EL) continue;
     const int t = p / k;
     const int rank = __popc(masks[ee] & ((1u << t) - 1u));
     r.g.perm[offs[ee] + rank] = p;

@@ -261,7 +261,7 @@ void launch_topk(const float* logits, const float* bias, int T, int E, int k, in
 //   C: exclusive scan over experts -> offsets, list of distinct experts;
 //   D: pos = offsets[e] + base[c][e] + (tokens of the chunk before this one routed to e).
 __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ idx, int T, int k,
-                                                  int E, Grouping g, uint32_t* masks,
+                                                  int E, int e0, int e_total, Grouping g, uint32_t* masks,
                                                   int32_t* base, int* status, int reset_status) {
   __shared__ int32_t off_s[1024];
   __shared__ int32_t aidx_s[1024];
@@ -279,10 +279,14 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
     const int t = 32 * c + lane;
     if (t < T) {
       for (int j = 0; j < k; ++j) {
-        const int e = idx[(int64_t)t * k + j];
-        if (e == -1) continue;               // a slot dropped by adaptive top-p
-        if (e < 0 || e >= E) set_status(status, kStatusDeviceCheck);
-        else atomicOr(&mrow[e], 1u << lane);
+        const int eg = idx[(int64_t)t * k + j];
+        if (eg == -1) continue;              // a slot dropped by adaptive top-p
+        if (eg < 0 || eg >= e_total) {
+          set_status(status, kStatusDeviceCheck);
+          continue;
+        }
+        const int e = eg - e0;               // local id; outside [0, E): held elsewhere
+        if (e >= 0 && e < E) atomicOr(&mrow[e], 1u << lane);
       }
     }
   }
@@ -351,8 +355,9 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
     const int t = 32 * c + lane;
     if (t >= T) continue;
     for (int j = 0; j < k; ++j) {
-      const int e = idx[(int64_t)t * k + j];
-      if (e < 0 || e >= E) continue;
+      const int eg = idx[(int64_t)t * k + j];
+      const int e = eg - e0;
+      if (eg < 0 || eg >= e_total || e < 0 || e >= E) continue;
       const uint32_t m = __ldcg(masks + (int64_t)c * E + e);
       const int rank = __ldcg(base + (int64_t)c * E + e) + __popc(m & ((1u << lane) - 1u));
       g.perm[off_s[e] + rank] = t * k + j;
@@ -361,10 +366,10 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
   }
 }
 
-void launch_permute(const int32_t* idx, int T, int k, int E, const Grouping& g, uint32_t* masks,
-                    int32_t* base, int* status, int reset_status, cudaStream_t st) {
+void launch_permute(const int32_t* idx, int T, int k, int E, int e0, int e_total, const Grouping& g,
+                    uint32_t* masks, int32_t* base, int* status, int reset_status, cudaStream_t st) {
   if (T <= 0) return;
-  launch_pdl(k_permute, dim3(1), dim3(1024), 0, st, idx, T, k, E, g, masks, base, status,
+  launch_pdl(k_permute, dim3(1), dim3(1024), 0, st, idx, T, k, E, e0, e_total, g, masks, base, status,
              reset_status);
 }
 

@@ -31,7 +31,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_version_and_status_strings():
-    assert M.moe_abi_version() == 3
+    assert M.moe_abi_version() == 4
     for s in range(7):
         assert M.moe_status_string(s).startswith("MOE_")
     assert M.moe_status_string(99) == "MOE_ERR_UNKNOWN"
@@ -162,3 +162,17 @@ def test_fp8_binding_checks_shapes_and_devices():
         M.moe_quantize_experts_fp8(gu, sgu[:, :1], dn, sdn, _Blob())
     with pytest.raises(ValueError, match="CUDA"):  # right shapes, but host tensors
         M.moe_quantize_experts_fp8(gu, sgu, dn, sdn, _Blob())
+
+
+def test_expert_range_arguments_are_checked():
+    """Expert parallelism's range (moe_route_cfg.n_experts_total, expert_begin) is checked on
+    the host: the size query returns 0 for a range the router cannot hold."""
+    b = M.moe_expert_blob(0, 1, 8, 256, 128, 0, 256, M.moe_expert_blob_bytes(0, 1, 8, 256, 128))
+    ok = M.moe_route_cfg(0, 2, 1, 1.0, 1, 0, 0.0, 16, 8)
+    bad = [M.moe_route_cfg(0, 2, 1, 1.0, 1, 0, 0.0, 16, 9),       # range past the router's experts
+           M.moe_route_cfg(0, 2, 1, 1.0, 1, 0, 0.0, 4, 0),        # fewer router experts than held
+           M.moe_route_cfg(0, 2, 1, 1.0, 1, 0, 0.0, 2000, 0),     # > 1024
+           M.moe_route_cfg(0, 2, 1, 1.0, 1, 0, 0.0, 16, -1)]
+    assert M._lib.moe_layer_workspace_bytes(4, C.byref(b), None, C.byref(ok)) > 0
+    for c in bad:
+        assert M._lib.moe_layer_workspace_bytes(4, C.byref(b), None, C.byref(c)) == 0
