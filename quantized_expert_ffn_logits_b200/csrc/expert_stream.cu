@@ -48,7 +48,7 @@ constexpr int kSmemMax = 227 * 1024;
 // of K codes, then (g32 activations) tm rows of G fp16 scales.
 // Single-token routing scratch (RingPlan::route): se, swt, sj, sidx, sw, own [32] each,
 // then two flag words and the y-zero barrier target (8 bytes).
-constexpr int kRouteBytes = 6 * 32 * 4 + 32;
+constexpr int kRouteBytes = 8 * 32 * 4;
 
 struct RingPlan {
   int ring, sring, sstage, bars, abuf, abytes, ascale, xsum, sxf, idot, ubuf, hq, info, route, total;
@@ -58,7 +58,8 @@ struct RingPlan {
 // 32 groups of 128 rows for int8, int4, int2) or its down blocks' scales.
 __host__ __device__ inline int ring_sstage(int wbits) { return wbits >= 4 ? 4096 : 16384 / wbits; }
 
-__host__ __device__ inline RingPlan ring_plan(int K, int tm, int wbits) {
+// ring_min: bytes the ring region must at least have (the single-token routing scratch).
+__host__ __device__ inline RingPlan ring_plan(int K, int tm, int wbits, int ring_min = 0) {
   RingPlan p;
   const int G = K / 32;
   int o = 0;
@@ -68,7 +69,7 @@ __host__ __device__ inline RingPlan ring_plan(int K, int tm, int wbits) {
     o = (o + bytes + 127) & ~127;
     return at;
   };
-  p.ring = take(kNS * kSP * kPiece);            // 128 KB
+  p.ring = take(kNS * kSP * kPiece > ring_min ? kNS * kSP * kPiece : ring_min);   // 128 KB or more
   p.sstage = ring_sstage(wbits);
   p.sring = take(kNS * p.sstage);               // group / row scales of a stage
   p.bars = take((2 * kNS + 4) * 8);
@@ -190,6 +191,14 @@ struct Ring {
   float* sxf;         // [tm][G] (or [tm] per-token scales)
 };
 
+// Single-token routing scratch in the (still idle) ring region: the router rows of the CTA's
+// experts at a 144-byte chunk pitch (staged before the wait for the preceding kernel), the
+// token's x at the same pitch, then the chunk partials (bytes; rows / x 0 = not staged).
+struct RouteScratch {
+  int rows, x, part;
+};
+__host__ __device__ inline int rs_total(const RouteScratch& s) { return s.rows + s.x + s.part; }
+
 // Launch arguments. x[0][*] = gate/up (q_x activations, writes h), x[1][*] = down (reads h,
 // adds into y); [*][0] routed experts, [*][1] the shared expert. Units are (expert,
 // 64 intermediate indices) in every mode: MODE 0 runs the gate/up pass of each unit,
@@ -204,6 +213,7 @@ struct RingArgs {
   int mma_min;             // experts with this many slots are left to the tensor-core path
   RouteArgs r;             // MODE 3 (one token): the routing done inside the kernel
   int cluster;             // MODE 3: logits shared per cluster of this many CTAs (0: grid barrier)
+  RouteScratch rs;         // MODE 3: the routing scratch layout
 };
 
 // int4 weights: each 8-byte word of the activation rows de-interleaved into its even, then
@@ -264,6 +274,7 @@ struct RouteSmem {
   volatile unsigned long long* ytarget;   // y-zero barrier target (cluster exchange)
   volatile int* nk;                       // slots kept: k, or the adaptive top-p prefix
   volatile int* nl;                       // kept slots whose expert is held here (units)
+  int* lsel;                              // [32] local id of each slot of the list, or -1
 };
 
 // Bounds of the cross-CTA waits (grid barrier, y-zero barrier): RouteArgs::wait_ns of
@@ -301,27 +312,36 @@ __device__ __forceinline__ bool wait_counter(const unsigned long long* p, unsign
   return false;
 }
 
-// Thread 0 of every CTA, after a CTA barrier: arrive, then wait until every CTA of the grid
-// has arrived. The counter is a multiple of 1024 when a call starts (grids are <= 1024
-// CTAs); this call's arrivals take base .. base + grid - 1 and the last one moves the
-// counter on to base + 1024 for the next call. False if the wait gave up.
-__device__ __forceinline__ bool grid_barrier(unsigned long long* ctr, unsigned long long wait_ns) {
+// Grid barrier (thread 0 of every CTA, after a CTA barrier) in two halves: arrive, returning
+// the target every CTA then waits for with wait_counter. The counter is a multiple of 1024
+// when a call starts (grids are <= 1024 CTAs); this call's arrivals take base .. base + grid - 1
+// and the last one moves the counter on to base + 1024 for the next call.
+__device__ __forceinline__ unsigned long long grid_arrive(unsigned long long* ctr) {
   const unsigned long long old = atom_add_release(ctr, 1ull);   // the CTA's writes before it
   const unsigned long long target = (old & ~1023ull) + gridDim.x;
   if (old + 1 == target) atomicAdd(ctr, 1024ull - gridDim.x);
-  return wait_counter(ctr, target, wait_ns);
+  return target;
 }
 
-// Scratch use of the (still idle) ring during the routing. The logit of a 32-element chunk
-// is one thread's fma chain, so threads read chunks 128 bytes apart; stored with a 144-byte
-// chunk pitch instead, the eight lanes of a quarter warp hit eight different bank groups.
-// [0, kRowBytes): the router rows of the CTA's experts, chunk pitch 144 (when they fit;
-// copied before the wait for the preceding kernel); [kRowBytes, + kXBytes): the token's x,
-// same pitch (when it fits); then the chunk partials.
+
+// Scratch use of the (still idle) ring during the routing (RouteScratch). The logit of a
+// 32-element chunk is one thread's fma chain, so threads read chunks 128 bytes apart; stored
+// with a 144-byte chunk pitch instead, the eight lanes of a quarter warp hit eight different
+// bank groups. Grid exchange: the 128 KB ring as [80 KB rows][28 KB x][20 KB partials], rows
+// staged when they fit; cluster exchange: sized for the ne experts a CTA owns.
 constexpr int kChunkPitch = 144;
 constexpr int kRowBytes = 80 * 1024;
 constexpr int kXBytes = 28 * 1024;
 constexpr int kPartFloats = (kNS * kSP * kPiece - kRowBytes - kXBytes) / 4;
+__host__ __device__ inline RouteScratch grid_scratch() { return RouteScratch{kRowBytes, kXBytes, kPartFloats * 4}; }
+__host__ __device__ inline RouteScratch cluster_scratch(int ne, int C) {
+  auto r128 = [](int v) { return (v + 127) & ~127; };
+  RouteScratch s;
+  s.rows = r128(ne * C * kChunkPitch);
+  s.x = C * kChunkPitch <= kXBytes ? r128(C * kChunkPitch) : 0;
+  s.part = r128((ne > 0 ? ne : 1) * C * 4);
+  return s;
+}
 
 // Who computes which logits. Grid exchange: CTA b owns experts b, b + grid, ...; cluster
 // exchange: cluster rank c owns experts c, c + cluster size, ... (every cluster computes all
@@ -344,10 +364,10 @@ __device__ __forceinline__ int owned_experts(int E, Owners o) {
 // per copy at the 144-byte pitch, completing on `bar`. Returns (to every thread) whether
 // they fit; if not, the logits read them from global memory.
 __device__ __forceinline__ bool stage_router_rows(const RouteArgs& r, bool cl, uint8_t* ring, uint64_t* bar,
-                                                  volatile int* flag) {
+                                                  volatile int* flag, int rows_bytes) {
   const Owners o = route_owners(cl);
   const int ne = owned_experts(r.E, o), C = r.H / 32;
-  const bool fit = ne > 0 && (int64_t)ne * C * kChunkPitch <= kRowBytes;
+  const bool fit = ne > 0 && (int64_t)ne * C * kChunkPitch <= rows_bytes;
   if (threadIdx.x == 0) {
     if (fit) mbar_arrive_expect_tx(bar, (uint32_t)(ne * C * 128));
     *flag = fit;
@@ -376,42 +396,59 @@ __device__ __forceinline__ int kept_local_rank(const RouteArgs& r, const RouteSm
   }
   return pos;
 }
-__device__ __forceinline__ int kept_local_count(const RouteArgs& r, const RouteSmem& S, int nk) {
-  int n = 0;
-  for (int j = 0; j < r.k; ++j) n += kept_local(r, S, nk, j) >= 0;
-  return n;
+
+// Grid exchange: 32-element chunk c (= the thread index) of the router rows of this CTA's
+// first two experts, loaded into registers before the wait for the preceding kernel (model
+// parameters, not written by it), so their latency overlaps the kernel's start.
+struct RowChunks {
+  float4 w[2][8];
+};
+__device__ __forceinline__ void prefetch_router_chunks(const RouteArgs& r, RowChunks& pf) {
+  const int C = r.H / 32, c = threadIdx.x;
+  const Owners o = route_owners(false);
+  const int ne = owned_experts(r.E, o);
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    if (c < C && j < ne) {
+      const float4* w4 = reinterpret_cast<const float4*>(r.wr + (int64_t)(o.first + j * o.stride) * r.H + 32 * c);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) pf.w[j][v] = __ldg(w4 + v);
+    }
 }
 
-// Every thread of the CTA. False when a wait gave up (status recorded; with the cluster
-// exchange the CTA has still taken both cluster-barrier arrivals, and must wait on the
-// second before it exits). rows_bar: the router rows were staged and complete on it.
-template <bool TOPP>
-__device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Ring& R, const RouteSmem& S,
-                                uint64_t* rows_bar, bool cl) {
-  volatile int* flag = S.flag;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int H = r.H, G = H / 32, C = H / 32, E = r.E, k = r.k;
-  const bool cta0 = blockIdx.x == 0;
-  const Owners own = route_owners(cl);
-  if (cta0 && tid == 0) {
-    r.status[0] = 0;
-    r.status[2] = 0;
-    r.status[3] = 0;
+// One 32-element router chunk against the token's same chunk: the fma chain from +0 in
+// ascending index.
+__device__ __forceinline__ float chunk_logit(const float4 (&xv)[8], const float4 (&wv)[8]) {
+  float acc = 0.0f;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    acc = __fmaf_rn(xv[v].x, wv[v].x, acc);
+    acc = __fmaf_rn(xv[v].y, wv[v].y, acc);
+    acc = __fmaf_rn(xv[v].z, wv[v].z, acc);
+    acc = __fmaf_rn(xv[v].w, wv[v].w, acc);
   }
-  // 1. activation codes and group scales: 8 threads per group, 4 elements each (8 G is a
-  //    multiple of 32, so a warp's lanes are all in range or all out)
+  return acc;
+}
+
+// Q8_0 codes and group scales of the token into activation buffer 0 (and, CTA 0, the q_x /
+// s_x views): 8 threads per group, 4 elements each, every load of a round in flight at once
+// (8 G is a multiple of 32, so a warp's lanes are all in range or all out). xpad (optional):
+// x also stored at the routing scratch's chunk pitch.
+__device__ __forceinline__ void quantize_token(const RouteArgs& r, const RingPlan& P, const Ring& R,
+                                               uint8_t* xpad, int tid, int nt) {
+  const int G = r.H / 32;
+  const bool cta0 = blockIdx.x == 0;
   uint8_t* xs = R.abuf;
   __half* sxs = reinterpret_cast<__half*>(xs + P.ascale);
-  uint8_t* xpad = C * kChunkPitch <= kXBytes ? R.ring + kRowBytes : nullptr;
-  for (int l0 = tid; l0 < 8 * G; l0 += 4 * kNT) {
+  for (int l0 = tid; l0 < 8 * G; l0 += 4 * nt) {
     float4 xv[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)                // every load of the round in flight at once
-      if (l0 + u * kNT < 8 * G) xv[u] = __ldg(reinterpret_cast<const float4*>(r.x) + l0 + u * kNT);
+    for (int u = 0; u < 4; ++u)
+      if (l0 + u * nt < 8 * G) xv[u] = __ldg(reinterpret_cast<const float4*>(r.x) + l0 + u * nt);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int l = l0 + u * kNT;
-      if (l >= 8 * G) break;                   // warp-uniform (8 G and kNT are multiples of 32)
+      const int l = l0 + u * nt;
+      if (l >= 8 * G) break;                   // warp-uniform (nt a multiple of 32)
       const int g = l >> 3;
       const float4 v = xv[u];
       float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
@@ -432,16 +469,106 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
       }
     }
   }
+}
+
+// Grid exchange, the logits (step 3 of route_one_token) first: thread c loads the token's
+// chunk c and forms the chunk partials of every expert this CTA owns (the first two from the
+// prefetched registers); the partials are added in chunk order per expert, and the CTA's
+// share of y is zeroed. Ends with a CTA barrier.
+__device__ __forceinline__ void grid_logits(const RouteArgs& r, const Ring& R, const RowChunks& pf) {
+  const int tid = threadIdx.x, H = r.H, C = H / 32;
+  const Owners own = route_owners(false);
+  const int ne = owned_experts(r.E, own);
+  float* part = reinterpret_cast<float*>(R.ring);          // [ne][C]
+  for (int c = tid; c < C && ne > 0; c += kNT) {
+    float4 xv[8];
+    const float4* x4 = reinterpret_cast<const float4*>(r.x + 32 * c);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) xv[v] = __ldg(x4 + v);
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      if (j < ne) {
+        float4 wv[8];
+        if (c == tid) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) wv[v] = pf.w[j][v];
+        } else {
+          const float4* w4 = reinterpret_cast<const float4*>(r.wr + (int64_t)(own.first + j * own.stride) * H + 32 * c);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) wv[v] = __ldg(w4 + v);
+        }
+        part[j * C + c] = chunk_logit(xv, wv);
+      }
+    for (int j = 2; j < ne; ++j) {
+      float4 wv[8];
+      const float4* w4 = reinterpret_cast<const float4*>(r.wr + (int64_t)(own.first + j * own.stride) * H + 32 * c);
+#pragma unroll
+      for (int v = 0; v < 8; ++v) wv[v] = __ldg(w4 + v);
+      part[j * C + c] = chunk_logit(xv, wv);
+    }
+  }
+  // this CTA's share of y = 0 (ordered before every CTA's adds by the grid barrier)
+  float4* y4 = reinterpret_cast<float4*>(r.y);
+  for (int l = blockIdx.x * kNT + tid; l < H / 4; l += gridDim.x * kNT) y4[l] = make_float4(0.f, 0.f, 0.f, 0.f);
+  __syncthreads();
+  for (int j = tid; j < ne; j += kNT) {
+    const float* pj = part + j * C;
+    float total = 0.0f;
+    int c = 0;
+    for (; c + 8 <= C; c += 8) {
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = pj[c + q];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) total = __fadd_rn(total, v[q]);
+    }
+    for (; c < C; ++c) total = __fadd_rn(total, pj[c]);
+    r.logits[own.first + j * own.stride] = total;
+  }
+  __syncthreads();
+}
+
+// Every thread of the CTA. False when a wait gave up (status recorded; with the cluster
+// exchange the CTA has still taken both cluster-barrier arrivals, and must wait on the
+// second before it exits). reg_rows: grid exchange with the router chunks prefetched in pf;
+// else the router rows were staged and complete on rows_bar (or, null, are read from global
+// memory).
+template <bool TOPP>
+__device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Ring& R, const RouteSmem& S,
+                                uint64_t* rows_bar, bool cl, const RouteScratch& rs, const RowChunks& pf,
+                                bool reg_rows) {
+  volatile int* flag = S.flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = r.H, G = H / 32, C = H / 32, E = r.E, k = r.k;
+  const bool cta0 = blockIdx.x == 0;
+  const Owners own = route_owners(cl);
+  if (cta0 && tid == 0) {
+    r.status[0] = 0;
+    r.status[2] = 0;
+    r.status[3] = 0;
+  }
+  bool good = true;
+  unsigned long long gtarget = 0;
+  if (reg_rows) {
+    // logits, y share zeroed, then warp 0 arrives at the grid barrier and waits (below) while
+    // the other warps quantize the token
+    grid_logits(r, R, pf);
+    if (tid == 0) gtarget = grid_arrive(r.gbar);
+    if (warp > 0) quantize_token(r, P, R, nullptr, tid - 32, kNT - 32);
+  } else {
+  // 1. the token's Q8_0 codes, and x at the chunk pitch for the staged logits (cluster
+  //    exchange, or grid exchange with more than two experts per CTA)
+  uint8_t* xpad = (rs.x && C * kChunkPitch <= rs.x) ? R.ring + rs.rows : nullptr;
+  quantize_token(r, P, R, xpad, tid, kNT);
   // 2. this CTA's share of y = 0 (ordered before every CTA's adds by a grid barrier: the
   //    routing's, or with the cluster exchange one whose wait comes before the first add)
   float4* y4 = reinterpret_cast<float4*>(r.y);
   for (int l = blockIdx.x * kNT + tid; l < H / 4; l += gridDim.x * kNT) y4[l] = make_float4(0.f, 0.f, 0.f, 0.f);
   // 3. logits of this CTA's experts, as many at a time as their chunk partials fit the ring
   //    (idle until the selection): partials first, then each expert's added in chunk order
-  float* part = reinterpret_cast<float*>(R.ring + kRowBytes + kXBytes);
+  float* part = reinterpret_cast<float*>(R.ring + rs.rows + rs.x);
   const int ne = owned_experts(E, own);
-  const int nb = kPartFloats / C;
-  bool good = true;
+  const int nb = rs.part / 4 / C;
   if (rows_bar) {
     // the router rows (copied while the preceding kernel finished): polled, not suspended on
     bool ok = false;
@@ -508,11 +635,15 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
     __syncthreads();
   }
   __syncthreads();
+  }   // cluster exchange: steps 1-3 from the staged router rows
   // 4. every logit into this CTA's shared memory
   float* slog = reinterpret_cast<float*>(R.ring);           // scratch again: [E] logits
   float* skey = slog + 512;                                  //                [E] selection keys
   if (!cl) {
-    if (tid == 0) *flag = grid_barrier(r.gbar, r.wait_ns) ? 1 : 0;
+    if (tid == 0) {
+      if (!reg_rows) gtarget = grid_arrive(r.gbar);
+      *flag = wait_counter(r.gbar, gtarget, r.wait_ns) ? 1 : 0;
+    }
     __syncthreads();
     if (!*flag) {
       if (tid == 0) wait_failed(r.status, 1, 6, 0);
@@ -563,7 +694,7 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
     const int base = i & ~63, n = min(64, E - base);
     const float kv = skey[i];
     int rank = 0, j = 0;
-    if ((n & 3) == 0) {
+    if ((n & 3) == 0) {   // (a fully unrolled 64-key version measured slower: run-once code)
       const float4* k4 = reinterpret_cast<const float4*>(skey + base);
 #pragma unroll 4
       for (; j < n; j += 4) {
@@ -622,32 +753,46 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
     __syncthreads();
   }
   // 6. the kept selection whose experts are held here (all of them without expert
-  //    parallelism), by local id, in ascending order (all the producer needs)
+  //    parallelism), by local id, in ascending order (all the producer needs): warp 0, one
+  //    lane per slot of the list
   const int nk = TOPP ? *S.nk : k;
-  const int nl = kept_local_count(r, S, nk);
-  if (tid < k) {
-    const int ee = S.sidx[tid];
-    const int le = kept_local(r, S, nk, tid);
+  if (warp == 0) {
+    const int ee = lane < k ? S.sidx[lane] : -1;
+    const int le = (lane < nk && ee >= r.e0 && ee < r.e0 + r.EL) ? ee - r.e0 : -1;
+    int pos = 0;
+    for (int i = 0; i < k; ++i) {
+      const int o = __shfl_sync(0xffffffffu, le, i);
+      pos += (o >= 0) & (o < le);
+    }
+    const int nl = __popc(__ballot_sync(0xffffffffu, le >= 0));
+    S.lsel[lane] = le;
     if (le >= 0) {
-      const int pos = kept_local_rank(r, S, nk, le);
       S.se[pos] = le;
-      S.sj[pos] = tid;
+      S.sj[pos] = lane;
       if (cta0) {
         r.g.act_expert[pos] = le;
         r.g.act_begin[pos] = pos;
-        r.g.perm[pos] = tid;
+        r.g.perm[pos] = lane;
         if (r.g.act_rows) r.g.act_rows[pos * 8] = 0;
       }
     }
-    if (cta0) r.idx[tid] = tid < nk ? ee : -1;
-  }
-  if (tid == 0) *S.nl = nl;
-  if (cta0) {
-    for (int x = tid; x < r.EL; x += kNT) r.g.offsets[x] = kept_local_rank(r, S, nk, x);
-    if (tid == 0) {
-      r.g.offsets[r.EL] = nl;
-      *r.g.n_active = nl;
-      r.g.act_begin[nl] = nl;
+    if (cta0 && lane < k) r.idx[lane] = lane < nk ? ee : -1;
+    if (lane == 0) *S.nl = nl;
+    __syncwarp();
+    if (cta0) {
+      for (int x = lane; x < r.EL; x += 32) {
+        int cnt = 0;
+        for (int i = 0; i < k; ++i) {
+          const int o = S.lsel[i];
+          cnt += (o >= 0) & (o < x);
+        }
+        r.g.offsets[x] = cnt;
+      }
+      if (lane == 0) {
+        r.g.offsets[r.EL] = nl;
+        *r.g.n_active = nl;
+        r.g.act_begin[nl] = nl;
+      }
     }
   }
   __syncthreads();
@@ -1120,7 +1265,7 @@ template <int WBITS, bool WG32, bool AG32, int MODE, int TM, bool TOPP>
 __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ RingArgs A) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_align1024(smem_raw);
-  const RingPlan P = ring_plan(A.kmax, A.tm, WBITS);
+  const RingPlan P = ring_plan(A.kmax, A.tm, WBITS, MODE == 3 ? rs_total(A.rs) : 0);
   Ring R;
   R.ring = base + P.ring;
   R.sring = base + P.sring;
@@ -1145,6 +1290,11 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* status = A.x[0][0].status;
 
+  // single-token routing, grid exchange with at most two experts per CTA: the CTA's router
+  // chunks straight into registers; else (cluster exchange, or more experts) staged rows
+  RowChunks pf;
+  const bool reg_rows = MODE == 3 && !A.cluster && owned_experts(A.r.E, route_owners(false)) <= 2;
+  if (reg_rows) prefetch_router_chunks(A.r, pf);   // in flight during the start-up
   if (threadIdx.x == 0) {
     *abort = 0;
     for (int s = 0; s < kNS; ++s) {
@@ -1169,16 +1319,17 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   S.ytarget = reinterpret_cast<volatile unsigned long long*>(S.se + 194);
   S.nk = S.se + 196;
   S.nl = S.se + 197;
+  S.lsel = S.se + 200;
   __syncthreads();
   bool rows = false;
   if (MODE == 3) {
-    rows = stage_router_rows(A.r, A.cluster != 0, R.ring, &R.afull[0], rows_flag);
+    if (!reg_rows) rows = stage_router_rows(A.r, A.cluster != 0, R.ring, &R.afull[0], rows_flag, A.rs.rows);
   }
   pdl_wait();
   if (MODE == 3) {
     // one token: routing first. Its grid barrier also means every CTA of this grid is
     // resident before any CTA lets the next kernel launch (and take SMs).
-    if (!route_one_token<TOPP>(A.r, P, R, S, rows ? &R.afull[0] : nullptr, A.cluster != 0)) {
+    if (!route_one_token<TOPP>(A.r, P, R, S, rows ? &R.afull[0] : nullptr, A.cluster != 0, A.rs, pf, reg_rows)) {
       if (A.cluster) cluster_wait();
       return;
     }
@@ -1381,59 +1532,39 @@ int decode_grid(int units, int E) { return std::min(sm_count(), std::max(units, 
 template <int WBITS, bool WG32, bool AG32, int MODE, int TM, bool TOPP = false>
 cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
   const RingPlan P = ring_plan(A.kmax, A.tm, WBITS);
-  {
+  if constexpr (MODE != 3) {
     const cudaError_t e = ensure_smem_attr((const void*)k_expert_ring<WBITS, WG32, AG32, MODE, TM, TOPP>, P.total);
     if (e != cudaSuccess) return e;
   }
   if constexpr (MODE == 3) {
-    // one token: the logits shared per cluster (16 CTAs, else 8) when a CTA's share of the
-    // router rows fits its staging area and every cluster of the grid can be resident at
+    // one token: the logits shared per cluster (of 16 or 8 CTAs, every CTA staging the router
+    // rows of E / cluster experts) when every cluster of the grid can be resident at
     // once (the y-zero barrier waits on all CTAs) with no fewer CTAs than the grid exchange
     // would use; else every CTA computes some logits and a grid barrier follows
     auto kern = k_expert_ring<WBITS, WG32, AG32, MODE, TM, TOPP>;
     const int dev = current_device();
     if (dev < 0) return cudaErrorInvalidDevice;
-    // most co-resident clusters of 16 and of 8 CTAs, per device (for this shared-memory size)
-    static int cached_clusters[kMaxDevices][2], cached_smem[kMaxDevices];
-    int max_clusters[2];
-    {
-      std::lock_guard<std::mutex> lk(setup_mutex());     // released before sm_count() below
-      if (cached_smem[dev] != P.total) {
-        (void)cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        for (int i = 0; i < 2; ++i) {
-          const int cs = i == 0 ? 16 : 8;
-          cudaLaunchConfig_t q = {};
-          cudaLaunchAttribute qa[1];
-          qa[0].id = cudaLaunchAttributeClusterDimension;
-          qa[0].val.clusterDim.x = cs;
-          qa[0].val.clusterDim.y = 1;
-          qa[0].val.clusterDim.z = 1;
-          q.gridDim = dim3(cs * 8);
-          q.blockDim = dim3(kNT);
-          q.dynamicSmemBytes = (size_t)P.total;
-          q.attrs = qa;
-          q.numAttrs = 1;
-          int n = 0;
-          cached_clusters[dev][i] = cudaOccupancyMaxActiveClusters(&n, kern, &q) == cudaSuccess ? n : 0;
-        }
-        cached_smem[dev] = P.total;
-        (void)cudaGetLastError();
-      }
-      max_clusters[0] = cached_clusters[dev][0];
-      max_clusters[1] = cached_clusters[dev][1];
-    }
+    const int C = A.r.H / 32, sms = sm_count();
     const int grid_x = decode_grid(A.units, A.r.E);          // grid exchange
-    const int need = std::min(std::max(A.units, 1), sm_count());
-    int cs_best = 0, cgrid = 0;
-    for (int i = 0; i < 2; ++i) {
-      const int cs = i == 0 ? 16 : 8;
-      const int per = (A.r.E + cs - 1) / cs;
-      if ((int64_t)per * (A.r.H / 32) * kChunkPitch > kRowBytes || per > 32) continue;
+    const int need = std::min(std::max(A.units, 1), sms);
+    int cs_best = 0, cgrid = 0, csmem = 0;
+    RouteScratch crs{};
+    // (clusters of 4 were measured slower at the OLMoE shape: staging 16 experts' router rows
+    // as 128-byte copies takes ~5 us of copy issue per CTA)
+    for (int cs : {16, 8}) {
+      const int ne = (A.r.E + cs - 1) / cs;
+      if (ne > 32) continue;                                   // S.own holds 32 logits
+      const RouteScratch rs = cluster_scratch(ne, C);
+      const int smem = ring_plan(A.kmax, A.tm, WBITS, rs_total(rs)).total;
+      if (smem > kSmemMax) continue;
+      const int mc = max_active_clusters((const void*)kern, dev, cs, smem, kNT);
       const int want = (std::max(A.units, 1) + cs - 1) / cs;
-      const int g = cs * std::min({want, max_clusters[i], sm_count() / cs});
+      const int g = cs * std::min({want, mc, sms / cs});
       if (g >= need && (cs_best == 0 || g < cgrid)) {
         cs_best = cs;
         cgrid = g;
+        csmem = smem;
+        crs = rs;
       }
     }
     RingArgs B = A;
@@ -1442,6 +1573,10 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
       // cooperative launch: the grid barrier needs every CTA resident at once, which the
       // runtime then guarantees (it refuses a grid that cannot be co-resident instead of
       // leaving CTAs to wait for SMs held by CTAs that spin on the barrier)
+      B.rs = grid_scratch();
+      const int smem = ring_plan(A.kmax, A.tm, WBITS, rs_total(B.rs)).total;
+      const cudaError_t e = ensure_smem_attr((const void*)kern, smem);
+      if (e != cudaSuccess) return e;
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute at[2];
       at[0].id = cudaLaunchAttributeCooperative;
@@ -1450,11 +1585,16 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
       at[1].val.programmaticStreamSerializationAllowed = 1;
       cfg.gridDim = dim3(grid_x);
       cfg.blockDim = dim3(kNT);
-      cfg.dynamicSmemBytes = (size_t)P.total;
+      cfg.dynamicSmemBytes = (size_t)smem;
       cfg.stream = st;
       cfg.attrs = at;
       cfg.numAttrs = kUsePdl ? 2 : 1;
       return cudaLaunchKernelEx(&cfg, kern, B);
+    }
+    B.rs = crs;
+    {
+      const cudaError_t e = ensure_smem_attr((const void*)kern, csmem);
+      if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[2];
@@ -1466,7 +1606,7 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
     at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.gridDim = dim3(cgrid);
     cfg.blockDim = dim3(kNT);
-    cfg.dynamicSmemBytes = (size_t)P.total;
+    cfg.dynamicSmemBytes = (size_t)csmem;
     cfg.stream = st;
     cfg.attrs = at;
     cfg.numAttrs = kUsePdl ? 2 : 1;

@@ -4,6 +4,7 @@
 // several GPUs, from several host threads.
 #include <map>
 #include <mutex>
+#include <tuple>
 #include <utility>
 
 #include "kernels.cuh"
@@ -48,6 +49,35 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes) {
   const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess) have = bytes;
   return e;
+}
+
+int max_active_clusters(const void* kernel, int dev, int cluster, int smem, int threads) {
+  if (ensure_smem_attr(kernel, smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 0;
+  }
+  std::lock_guard<std::mutex> lk(g_setup_mu);
+  static std::map<std::tuple<const void*, int, int, int>, int> done;
+  const auto key = std::make_tuple(kernel, dev, cluster, smem);
+  const auto it = done.find(key);
+  if (it != done.end()) return it->second;
+  if (cluster > 8) (void)cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaLaunchConfig_t q = {};
+  cudaLaunchAttribute qa[1];
+  qa[0].id = cudaLaunchAttributeClusterDimension;
+  qa[0].val.clusterDim.x = cluster;
+  qa[0].val.clusterDim.y = 1;
+  qa[0].val.clusterDim.z = 1;
+  q.gridDim = dim3(cluster * 8);
+  q.blockDim = dim3(threads);
+  q.dynamicSmemBytes = (size_t)smem;
+  q.attrs = qa;
+  q.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &q) != cudaSuccess) n = 0;
+  (void)cudaGetLastError();
+  done[key] = n;
+  return n;
 }
 
 }  // namespace moe

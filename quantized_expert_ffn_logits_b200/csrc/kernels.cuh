@@ -15,6 +15,8 @@ constexpr int kMaxDevices = 64;
 int current_device();                                   // -1 if unknown or >= kMaxDevices
 int device_sm_count();                                  // SMs of the current device
 cudaError_t ensure_smem_attr(const void* kernel, int bytes);   // dynamic smem limit >= bytes
+// Most co-resident clusters of `cluster` CTAs of `threads` threads and `smem` bytes (cached).
+int max_active_clusters(const void* kernel, int dev, int cluster, int smem, int threads);
 std::mutex& setup_mutex();
 
 // ---- quantize.cu
