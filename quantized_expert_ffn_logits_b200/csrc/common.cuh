@@ -65,6 +65,24 @@ __device__ __forceinline__ int quant_code(float v, float s, float qmax) {
   return (int)r;
 }
 
+// quant_code(v, s, qmax) with one multiplication by rs = fl(1 / s) instead of the division:
+// fl(v * rs) and fl(v / s) both lie within 2 ulp of v / s (|v / s| <= qmax + 1 < 2^7), so they
+// round to different integers only when v / s is that close to a half-integer; such values
+// (fractional part within 2^-16 * max(|q|, 1) of 0.5) take the exact division, and so does
+// any product that is not a plausible code (1 / s overflowed for a tiny s). Bit-identical to
+// quant_code.
+__device__ __forceinline__ int quant_code_rcp(float v, float s, float rs, float qmax) {
+  if (s == 0.0f) return 0;
+  const float r = __fmul_rn(v, rs);
+  const float a = fabsf(r);
+  const float f = a - truncf(a);
+  float q;
+  if (!(a < 256.0f) || fabsf(f - 0.5f) <= 0x1p-16f * fmaxf(a, 1.0f)) q = roundf(__fdiv_rn(v, s));
+  else q = roundf(r);
+  q = fminf(fmaxf(q, -qmax), qmax);
+  return (int)q;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -1570,26 +1570,16 @@ cudaError_t launch_ring_t(const RingArgs& A, cudaStream_t st) {
     RingArgs B = A;
     B.cluster = cs_best;
     if (!B.cluster) {
-      // cooperative launch: the grid barrier needs every CTA resident at once, which the
-      // runtime then guarantees (it refuses a grid that cannot be co-resident instead of
-      // leaving CTAs to wait for SMs held by CTAs that spin on the barrier)
+      // Plain (programmatic) launch: the grid is at most one CTA per SM and one CTA fits an SM,
+      // so on an otherwise idle GPU every CTA is resident; if other work holds SMs, the
+      // bounded grid-barrier wait returns MOE_ERR_TIMEOUT rather than hanging. (A cooperative
+      // launch would guarantee residency, but measured it cannot start while the host path's
+      // input-copy kernel still holds SMs: 3 us more per step there.)
       B.rs = grid_scratch();
       const int smem = ring_plan(A.kmax, A.tm, WBITS, rs_total(B.rs)).total;
       const cudaError_t e = ensure_smem_attr((const void*)kern, smem);
       if (e != cudaSuccess) return e;
-      cudaLaunchConfig_t cfg = {};
-      cudaLaunchAttribute at[2];
-      at[0].id = cudaLaunchAttributeCooperative;
-      at[0].val.cooperative = 1;
-      at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-      at[1].val.programmaticStreamSerializationAllowed = 1;
-      cfg.gridDim = dim3(grid_x);
-      cfg.blockDim = dim3(kNT);
-      cfg.dynamicSmemBytes = (size_t)smem;
-      cfg.stream = st;
-      cfg.attrs = at;
-      cfg.numAttrs = kUsePdl ? 2 : 1;
-      return cudaLaunchKernelEx(&cfg, kern, B);
+      return launch_pdl(kern, dim3(grid_x), dim3(kNT), (size_t)smem, st, B);
     }
     B.rs = crs;
     {

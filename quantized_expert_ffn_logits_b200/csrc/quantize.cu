@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(256) k_quantize_act(const float* __restrict__ 
     for (int g = warp; g < H / 32; g += nw) {
       const float v = xr[32 * g + lane];
       const float s = f16_round(__fdiv_rn(warp_max(fabsf(v)), 127.0f));
-      qr[32 * g + lane] = (int8_t)quant_code(v, s, 127.0f);
+      qr[32 * g + lane] = (int8_t)quant_code_rcp(v, s, __frcp_rn(s), 127.0f);
       if (lane == 0) sr[g] = __float2half_rn(s);
     }
   } else {
@@ -184,7 +184,8 @@ __global__ void __launch_bounds__(256) k_quantize_act(const float* __restrict__ 
     }
     __syncthreads();
     const float s = __fdiv_rn(red[0], 127.0f);
-    for (int k = threadIdx.x; k < H; k += blockDim.x) qr[k] = (int8_t)quant_code(xr[k], s, 127.0f);
+    const float rs = __frcp_rn(s);
+    for (int k = threadIdx.x; k < H; k += blockDim.x) qr[k] = (int8_t)quant_code_rcp(xr[k], s, rs, 127.0f);
     if (threadIdx.x == 0) reinterpret_cast<float*>(scales)[t] = s;
   }
 }

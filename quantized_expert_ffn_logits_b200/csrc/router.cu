@@ -257,7 +257,8 @@ void launch_topk(const float* logits, const float* bias, int T, int E, int k, in
 // ----------------------------------------------------------------- grouping
 // Stable counting sort of the T*k (token, slot) pairs by expert, one CTA.
 //   A: per 32-token chunk c, masks[c][e] = bit set of the chunk's tokens routed to e;
-//   B: per expert, base[c][e] = pairs of e in chunks before c;
+//   B: per expert, base[c][e] = pairs of e in chunks before c (the chunks cut into
+//      1024 / E parts, summed in parallel, then each part's sums scanned);
 //   C: exclusive scan over experts -> offsets, list of distinct experts;
 //   D: pos = offsets[e] + base[c][e] + (tokens of the chunk before this one routed to e).
 __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ idx, int T, int k,
@@ -265,6 +266,7 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
                                                   int32_t* base, int* status, int reset_status) {
   __shared__ int32_t off_s[1024];
   __shared__ int32_t aidx_s[1024];
+  __shared__ int32_t psum[1024];            // [part][expert] pair counts
   __shared__ int32_t wsum[32], fsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
@@ -291,16 +293,29 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
     }
   }
   __syncthreads();
-  int v = 0;
-  if (tid < E) {
-    int run = 0;
-    for (int c = 0; c < C; ++c) {
-      const uint32_t m = __ldcg(masks + (int64_t)c * E + tid);
-      base[(int64_t)c * E + tid] = run;
-      run += __popc(m);
-    }
-    v = run;
+  // B: thread (part, e) counts its part's chunks, then writes their bases from the counts of
+  //    the parts before it
+  const int NP = E >= 1024 ? 1 : 1024 / E;  // parts per expert
+  const int per = (C + NP - 1) / NP;         // chunks per part
+  const int pe = tid % E, pp = tid / E;
+  const int c0 = min(pp * per, C), c1 = min(c0 + per, C);
+  if (pp < NP) {
+    int cnt = 0;
+    for (int c = c0; c < c1; ++c) cnt += __popc(__ldcg(masks + (int64_t)c * E + pe));
+    psum[pp * E + pe] = cnt;
   }
+  __syncthreads();
+  int v = 0;
+  if (pp < NP) {
+    int run = 0;
+    for (int q = 0; q < pp; ++q) run += psum[q * E + pe];
+    for (int c = c0; c < c1; ++c) {
+      base[(int64_t)c * E + pe] = run;
+      run += __popc(__ldcg(masks + (int64_t)c * E + pe));
+    }
+  }
+  if (tid < E)
+    for (int q = 0; q < NP; ++q) v += psum[q * E + tid];
   const int f = (tid < E && v > 0) ? 1 : 0;
   int incl = v, inclf = f;
 #pragma unroll

@@ -562,3 +562,31 @@ def test_single_token_selection_ties_go_to_lower_experts():
     assert idx.tolist() == [list(range(k))]
     assert np.allclose(w, 1.0 / k, rtol=1e-6)
     assert np.array_equal(_np(y), np.zeros((1, H), np.float32))
+
+
+@pytest.mark.parametrize("act", ["g32_f16", "token_f32"])
+def test_quantize_activations_at_rounding_ties(act):
+    """Codes decided at half-integers: every group's maximum is 127 * 2^-7 (so the scale is
+    exactly 2^-7) and the other values are (j + 0.5) * 2^-7 -- exact ties, rounded half away
+    from zero -- or one ulp either side of them. The kernel's reciprocal fast path must hand
+    all of these to the exact division and match the oracle bit for bit."""
+    m = M()
+    H = 256
+    rows = []
+    for sign in (1.0, -1.0):
+        for shift in (0, 1, -1):
+            r = np.empty(H, np.float32)
+            for g in range(H // 32):
+                vals = np.array([(j % 126 + 0.5) * 2.0 ** -7 for j in range(g, g + 31)], np.float32) * sign
+                if shift:
+                    vals = np.nextafter(vals, np.float32(np.inf * shift)).astype(np.float32)
+                r[32 * g] = 127 * 2.0 ** -7
+                r[32 * g + 1:32 * g + 32] = vals
+            rows.append(r)
+    x = np.stack(rows)
+    q, s = m.moe_quantize_activations(torch.from_numpy(x).cuda(), act)
+    rq, rs = O.quantize_act(x, act == "g32_f16")
+    assert np.array_equal(_np(q), rq)
+    assert np.array_equal(_np(s).astype(np.float32), rs)
+    if act == "g32_f16":
+        assert (np.abs(rq[:2]) % 1 == 0).all() and np.any(np.abs(rq[0]) == 127)
