@@ -212,11 +212,13 @@ MOE_API moe_status moe_quantize_experts_fp8(const uint8_t* w_gate_up, const floa
 
 /* Q8_0-style activation quantization (GLM page, "Integer-dot kernels (Q8_0-style int8
  * activations ...)").  x [T][H] fp32 -> q [T][H] int8 and `scales`: fp16 [T][H/32]
- * (MOE_ACT_G32_F16) or fp32 [T] (MOE_ACT_TOKEN_F32). H multiple of 32. */
+ * (MOE_ACT_G32_F16) or fp32 [T] (MOE_ACT_TOKEN_F32). H multiple of 32; x 16-byte, q and
+ * scales 4-byte aligned (MOE_ERR_INVALID_ARG otherwise). */
 MOE_API moe_status moe_quantize_activations(const float* x, int32_t T, int32_t H, int32_t act,
                                     int8_t* q, void* scales, void* stream);
 
-/* Router logits [T][E] = x [T][H] . router_w [E][H]^T in the fixed fp32 order above. */
+/* Router logits [T][E] = x [T][H] . router_w [E][H]^T in the fixed fp32 order above. x and
+ * router_w 16-byte aligned (MOE_ERR_INVALID_ARG otherwise). */
 MOE_API moe_status moe_router_logits(const float* x, const float* router_w, int32_t T, int32_t E,
                              int32_t H, float* logits, void* stream);
 
@@ -261,7 +263,8 @@ MOE_API moe_status moe_permute_no_alloc(const int32_t* idx, int32_t T, int32_t k
 MOE_API size_t moe_layer_workspace_bytes(int32_t T, const moe_expert_blob* experts,
                                  const moe_expert_blob* shared, const moe_route_cfg* cfg);
 
-/* The whole layer: y [T][H] fp32 (overwritten) from x [T][H] fp32.
+/* The whole layer: y [T][H] fp32 (overwritten) from x [T][H] fp32 (x, y and router_w 16-byte
+ * aligned, the workspace 256-byte aligned: MOE_ERR_INVALID_ARG otherwise).
  *   router_w [E][H] fp32; router_bias [E] fp32 or NULL (sigmoid mode only);
  *   experts: the routed experts; shared: NULL or one expert (n_experts = 1) with the same
  *   hidden size, wtype and wscale as `experts` and its own intermediate size.

@@ -302,7 +302,8 @@ moe_status moe_quantize_activations(const float* x, int32_t T, int32_t H, int32_
   if (T < 0 || H <= 0 || H % 32) return T < 0 ? MOE_ERR_INVALID_ARG : MOE_ERR_UNSUPPORTED;
   if (act != MOE_ACT_TOKEN_F32 && act != MOE_ACT_G32_F16) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
-  if (!x || !q || !scales) return MOE_ERR_INVALID_ARG;
+  if (!x || !q || !scales || !aligned(x, 16) || !aligned(q, 4) || !aligned(scales, 4))
+    return MOE_ERR_INVALID_ARG;
   moe::launch_quantize_act(x, T, H, act == MOE_ACT_G32_F16, q, scales, nullptr, nullptr,
                            static_cast<cudaStream_t>(stream));
   return launch_status();

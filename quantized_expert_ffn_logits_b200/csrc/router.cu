@@ -261,34 +261,59 @@ void launch_topk(const float* logits, const float* bias, int T, int E, int k, in
 //      1024 / E parts, summed in parallel, then each part's sums scanned);
 //   C: exclusive scan over experts -> offsets, list of distinct experts;
 //   D: pos = offsets[e] + base[c][e] + (tokens of the chunk before this one routed to e).
+// SM: masks and base live in dynamic shared memory (2 * C * E words) instead of the
+// workspace. A token's k slots are read in batches of eight independent loads.
+template <bool SM>
 __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ idx, int T, int k,
-                                                  int E, int e0, int e_total, Grouping g, uint32_t* masks,
-                                                  int32_t* base, int* status, int reset_status) {
+                                                  int E, int e0, int e_total, Grouping g,
+                                                  uint32_t* masks_g, int32_t* base_g, int* status,
+                                                  int reset_status) {
+  extern __shared__ uint32_t dyn_s[];
   __shared__ int32_t off_s[1024];
   __shared__ int32_t aidx_s[1024];
   __shared__ int32_t psum[1024];            // [part][expert] pair counts
   __shared__ int32_t wsum[32], fsum[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = (T + 31) / 32;
+  uint32_t* masks = SM ? dyn_s : masks_g;
+  int32_t* base = SM ? reinterpret_cast<int32_t*>(dyn_s + (int64_t)C * E) : base_g;
+  auto ldm = [&](int64_t i) -> uint32_t {
+    if constexpr (SM) return masks[i];
+    else return __ldcg(masks + i);
+  };
+  auto ldb = [&](int64_t i) -> int32_t {
+    if constexpr (SM) return base[i];
+    else return __ldcg(base + i);
+  };
   pdl_wait();
   pdl_trigger();
   if (reset_status && tid == 0 && status) *status = 0;
+  if (SM)
+    for (int i = tid; i < C * E; i += 1024) masks[i] = 0u;
   __syncthreads();
-  const int C = (T + 31) / 32;
   for (int c = warp; c < C; c += 32) {
     uint32_t* mrow = masks + (int64_t)c * E;
-    for (int e = lane; e < E; e += 32) mrow[e] = 0u;
-    __syncwarp();
+    if (!SM) {
+      for (int e = lane; e < E; e += 32) mrow[e] = 0u;
+      __syncwarp();
+    }
     const int t = 32 * c + lane;
     if (t < T) {
-      for (int j = 0; j < k; ++j) {
-        const int eg = idx[(int64_t)t * k + j];
-        if (eg == -1) continue;              // a slot dropped by adaptive top-p
-        if (eg < 0 || eg >= e_total) {
-          set_status(status, kStatusDeviceCheck);
-          continue;
+      for (int j0 = 0; j0 < k; j0 += 8) {
+        int ev[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) ev[u] = j0 + u < k ? __ldg(idx + (int64_t)t * k + j0 + u) : -1;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int eg = ev[u];
+          if (eg == -1) continue;            // a slot dropped by adaptive top-p (or past k)
+          if (eg < 0 || eg >= e_total) {
+            set_status(status, kStatusDeviceCheck);
+            continue;
+          }
+          const int e = eg - e0;             // local id; outside [0, E): held elsewhere
+          if (e >= 0 && e < E) atomicOr(&mrow[e], 1u << lane);
         }
-        const int e = eg - e0;               // local id; outside [0, E): held elsewhere
-        if (e >= 0 && e < E) atomicOr(&mrow[e], 1u << lane);
       }
     }
   }
@@ -301,7 +326,7 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
   const int c0 = min(pp * per, C), c1 = min(c0 + per, C);
   if (pp < NP) {
     int cnt = 0;
-    for (int c = c0; c < c1; ++c) cnt += __popc(__ldcg(masks + (int64_t)c * E + pe));
+    for (int c = c0; c < c1; ++c) cnt += __popc(ldm((int64_t)c * E + pe));
     psum[pp * E + pe] = cnt;
   }
   __syncthreads();
@@ -311,7 +336,7 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
     for (int q = 0; q < pp; ++q) run += psum[q * E + pe];
     for (int c = c0; c < c1; ++c) {
       base[(int64_t)c * E + pe] = run;
-      run += __popc(__ldcg(masks + (int64_t)c * E + pe));
+      run += __popc(ldm((int64_t)c * E + pe));
     }
   }
   if (tid < E)
@@ -369,23 +394,40 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
   for (int c = warp; c < C; c += 32) {
     const int t = 32 * c + lane;
     if (t >= T) continue;
-    for (int j = 0; j < k; ++j) {
-      const int eg = idx[(int64_t)t * k + j];
-      const int e = eg - e0;
-      if (eg < 0 || eg >= e_total || e < 0 || e >= E) continue;
-      const uint32_t m = __ldcg(masks + (int64_t)c * E + e);
-      const int rank = __ldcg(base + (int64_t)c * E + e) + __popc(m & ((1u << lane) - 1u));
-      g.perm[off_s[e] + rank] = t * k + j;
-      if (g.act_rows && rank < 8) g.act_rows[aidx_s[e] * 8 + rank] = t;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int ev[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ev[u] = j0 + u < k ? __ldg(idx + (int64_t)t * k + j0 + u) : -1;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int eg = ev[u];
+        const int e = eg - e0;
+        if (eg < 0 || eg >= e_total || e < 0 || e >= E) continue;
+        const uint32_t m = ldm((int64_t)c * E + e);
+        const int rank = ldb((int64_t)c * E + e) + __popc(m & below);
+        g.perm[off_s[e] + rank] = t * k + j0 + u;
+        if (g.act_rows && rank < 8) g.act_rows[aidx_s[e] * 8 + rank] = t;
+      }
     }
   }
 }
 
+// Masks and bases in shared memory up to this many bytes (4096 tokens x 64 experts: 64 KB)
+constexpr int64_t kPermuteSmemMax = 160 * 1024;
+
 void launch_permute(const int32_t* idx, int T, int k, int E, int e0, int e_total, const Grouping& g,
                     uint32_t* masks, int32_t* base, int* status, int reset_status, cudaStream_t st) {
   if (T <= 0) return;
-  launch_pdl(k_permute, dim3(1), dim3(1024), 0, st, idx, T, k, E, e0, e_total, g, masks, base, status,
-             reset_status);
+  const int64_t smem = 2 * (int64_t)((T + 31) / 32) * E * 4;
+  if (smem <= kPermuteSmemMax &&
+      ensure_smem_attr(reinterpret_cast<const void*>(k_permute<true>), (int)smem) == cudaSuccess) {
+    launch_pdl(k_permute<true>, dim3(1), dim3(1024), (size_t)smem, st, idx, T, k, E, e0, e_total,
+               g, masks, base, status, reset_status);
+    return;
+  }
+  launch_pdl(k_permute<false>, dim3(1), dim3(1024), 0, st, idx, T, k, E, e0, e_total, g, masks,
+             base, status, reset_status);
 }
 
 }  // namespace moe

@@ -106,6 +106,9 @@ def test_other_entry_points_reject_bad_arguments():
     assert L.moe_quantize_experts_fp8(fake, fake, fake, fake, C.byref(_blob(nbytes=10)), None) == M.MOE_ERR_WORKSPACE
     assert L.moe_quantize_activations(fake, 4, 100, 1, fake, fake, None) == M.MOE_ERR_UNSUPPORTED
     assert L.moe_quantize_activations(fake, 4, 128, 5, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_activations(fake + 4, 4, 128, 1, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize_activations(fake, 4, 128, 1, fake + 2, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_router_logits(fake + 8, fake, 4, 8, 128, fake, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_router_logits(fake, fake, 4, 8, 100, fake, None) == M.MOE_ERR_UNSUPPORTED
     assert L.moe_route_topk(fake, None, 4, 8, C.byref(_cfg(k=9)), fake, fake, None) == M.MOE_ERR_UNSUPPORTED
     assert L.moe_route_topk(fake, None, 4, 2000, C.byref(_cfg()), fake, fake, None) == M.MOE_ERR_UNSUPPORTED
