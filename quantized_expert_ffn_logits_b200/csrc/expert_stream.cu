@@ -690,24 +690,34 @@ __device__ bool route_one_token(const RouteArgs& r, const RingPlan& P, const Rin
   // chunk * k + rank; (b) every candidate ranks itself against all candidates. A key of the
   // global top k is among its chunk's top k, and every key ranked above it is too, so its rank
   // among the candidates is its global rank (same tie rule throughout).
-  for (int i = tid; i < E; i += kNT) {
-    const int base = i & ~63, n = min(64, E - base);
-    const float kv = skey[i];
-    int rank = 0, j = 0;
-    if ((n & 3) == 0) {   // (a fully unrolled 64-key version measured slower: run-once code)
-      const float4* k4 = reinterpret_cast<const float4*>(skey + base);
-#pragma unroll 4
-      for (; j < n; j += 4) {
-        const float4 q = k4[j >> 2];
-        const int jj = base + j;
-        rank += (q.x > kv) | ((q.x == kv) & (jj < i));
-        rank += (q.y > kv) | ((q.y == kv) & (jj + 1 < i));
-        rank += (q.z > kv) | ((q.z == kv) & (jj + 2 < i));
-        rank += (q.w > kv) | ((q.w == kv) & (jj + 3 < i));
+  // (a): four adjacent lanes per key, each counting one quarter (16 keys) of the key's chunk
+  // with four independent counters; two xor-shuffles add the quarters. Warps step through the
+  // (key, quarter) pairs together so every shuffle has its whole warp.
+  for (int l0 = warp * 32; l0 < 4 * E; l0 += kNT) {
+    const int l = l0 + lane, i = l >> 2, qt = l & 3;
+    const bool on = l < 4 * E;
+    const int base = i & ~63, n = on ? min(64, E - base) : 0;
+    const float kv = on ? skey[i] : 0.0f;
+    const int j0 = 16 * qt, j1 = min(j0 + 16, n);
+    int r0 = 0, r1 = 0, r2 = 0, r3 = 0, j = j0;
+    if (j1 - j0 == 16) {
+      const float4* k4 = reinterpret_cast<const float4*>(skey + base + j0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 q = k4[u];
+        const int jj = base + j0 + 4 * u;
+        r0 += (q.x > kv) | ((q.x == kv) & (jj < i));
+        r1 += (q.y > kv) | ((q.y == kv) & (jj + 1 < i));
+        r2 += (q.z > kv) | ((q.z == kv) & (jj + 2 < i));
+        r3 += (q.w > kv) | ((q.w == kv) & (jj + 3 < i));
       }
+      j = j1;
     }
-    for (; j < n; ++j) rank += (skey[base + j] > kv) | ((skey[base + j] == kv) & (base + j < i));
-    if (rank < k) {
+    for (; j < j1; ++j) r0 += (skey[base + j] > kv) | ((skey[base + j] == kv) & (base + j < i));
+    int rank = (r0 + r1) + (r2 + r3);
+    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+    rank += __shfl_xor_sync(0xffffffffu, rank, 2);
+    if (on && qt == 0 && rank < k) {
       if (nch == 1) {
         S.sidx[rank] = i;
       } else {
