@@ -110,11 +110,12 @@ def expected_down_dots(ref, case: S.Case, perm):
     return out, shd
 
 
-def oracle_tokens(case: S.Case, tokens):
-    """Per-token oracle for selected tokens only, regenerating just the experts they use.
+def oracle_tokens(case: S.Case, tokens, x=None):
+    """Per-token oracle for selected tokens only (of the case's x, or of another x [T][H]),
+    regenerating just the experts they use.
     Returns dict(y [n][H], idx, w, ye {(t, j): fp64 [H]}, qh/sh/gate/up per pair)."""
     c = case.cfg
-    x = case.x()
+    x = case.x() if x is None else np.asarray(x)
     L = O.router_logits(x[tokens], case.router_w())
     idx, w = O.route(L, case.bias(), c.score, c.top_k, c.renormalize, c.rsf)
     qx, sx = O.quantize_act(x[tokens], ag32(c))

@@ -73,3 +73,26 @@ def test_full_size_layer(name, T, sample):
     assert_close_y(yg[toks], ref["y"])
     del g, y, ws
     torch.cuda.empty_cache()
+
+
+def test_full_size_host_buffers_single_token():
+    """moe_layer_forward_host at the full OLMoE int8 size with one token (the single-token
+    kernel with the grid barrier between the input and output copy kernels): four different
+    tokens enqueued back to back, each into its own page-locked output, against the oracle on
+    its own x."""
+    import quantized_expert_ffn_logits_b200 as M
+    c = S.CONFIGS["olmoe_int8"]
+    case = S.Case.make(c, 1)
+    g = gpu_layer(case)
+    lay = M.Layer(1, g["blob"], g["shared"], route_cfg(c), g["wr"], g["bias"])
+    xs = [case.x()] + [S.normal_cpu(c.H, 5151 + i, 0, c.x_sigma).reshape(1, c.H) for i in range(3)]
+    xh = [torch.from_numpy(x).pin_memory() for x in xs]
+    yh = [torch.full((1, c.H), float("nan"), dtype=torch.float32).pin_memory() for _ in xs]
+    for a, b in zip(xh, yh):
+        lay.forward_host(a, b)
+    torch.cuda.synchronize()
+    assert M.moe_read_device_status(lay.workspace) == M.MOE_OK
+    for i, x in enumerate(xs):
+        assert_close_y(yh[i].numpy(), oracle_tokens(case, [0], x=x)["y"], f"call {i}")
+    del g, lay
+    torch.cuda.empty_cache()
