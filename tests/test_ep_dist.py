@@ -129,3 +129,105 @@ def test_least_loaded_placement():
     rw = np.arange(12, dtype=np.float32).reshape(6, 2)
     rw2, _ = ep.renumber(order, rw)
     assert np.array_equal(rw2[1], rw[0]) and np.array_equal(rw2[0], rw[3])
+
+
+# all-to-all exchange: three ranks with different token counts (one with a single token)
+T_A2A = [4, 1, 6]
+
+
+def _oracle_x(x):
+    """The oracle's whole layer on rows x with the weights of one fixed case."""
+    import oracle as O
+    case = S.Case.make(CFG, 1)
+    ex = O.QExperts.quantize(np.stack([case.gate_up(e) for e in range(CFG.E)]),
+                             np.stack([case.down(e) for e in range(CFG.E)]), 8, True)
+    sh = O.QExperts.quantize(case.shared_gate_up()[None], case.shared_down()[None], 8, True)
+    return O.layer_forward(x, case.router_w(), case.bias(), ex, sh, CFG.score, CFG.top_k,
+                           CFG.renormalize, CFG.rsf, True)
+
+
+def _worker_a2a(rank, world, port, q):
+    import torch
+    import torch.distributed as dist
+    from quantized_expert_ffn_logits_b200 import ep
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ranges = ep.expert_ranges(CFG.E, world)
+        begin, count = ranges[rank]
+        x_local = torch.from_numpy(S.normal_cpu(T_A2A[rank] * CFG.H, 700 + rank, 0, 1.0).reshape(T_A2A[rank], CFG.H))
+        npairs = [0, 0]
+
+        def local_sum(x, with_shared):
+            o = _oracle_x(x.numpy())
+            T, k = o["idx"].shape
+            y = np.zeros((T, CFG.H))
+            for t in range(T):
+                for j in range(k):
+                    e = int(o["idx"][t, j])
+                    if begin <= e < begin + count:
+                        y[t] += o["w"][t, j] * o["ye"][t * k + j]
+                        npairs[0] += 1
+                if with_shared:
+                    y[t] += o["ysh"][t]
+                    npairs[1] += 1
+            return torch.from_numpy(y), torch.from_numpy(o["idx"].astype(np.int64))
+
+        def partial(x):
+            if x.shape[0] == 0:
+                return x.new_zeros((0, CFG.H))
+            return local_sum(x, False)[0]
+
+        y = ep.ep_step_a2a(x_local.double(), ranges, lambda x: local_sum(x, True), partial)
+        xs = [None] * world
+        dist.all_gather_object(xs, x_local.numpy())
+        counts = [None] * world
+        dist.all_gather_object(counts, npairs)
+    finally:
+        dist.destroy_process_group()
+    q.put((rank, y.numpy(), counts, np.concatenate(xs)))
+
+
+def test_three_rank_all_to_all_step_equals_the_whole_layer():
+    """ep_step_a2a on three gloo ranks holding 4, 1 and 6 tokens (uneven splits, some of them
+    empty): every rank's rows equal the oracle's whole layer on all tokens, every routed pair
+    is computed exactly once over all ranks (on the rank holding its expert), and the shared
+    expert once per token (on the token's rank)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    world = len(T_A2A)
+    procs = [ctx.Process(target=_worker_a2a, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=240) for _ in procs)
+    for p in procs:
+        p.join(60)
+        assert p.exitcode == 0
+    x_all = res[0][3]
+    ref = _oracle_x(x_all)
+    st = np.cumsum([0] + T_A2A)
+    for rank, y, _, _ in res:
+        want = ref["y"][st[rank]:st[rank + 1]]
+        assert np.allclose(y, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+    counts = res[0][2]
+    assert sum(c[0] for c in counts) == sum(T_A2A) * CFG.top_k
+    assert [c[1] for c in counts] == T_A2A
+
+
+def test_dispatch_plan_and_combine():
+    """a2a_plan on a hand-made routing: a token goes once to each other rank holding one of its
+    experts (dropped slots -1 go nowhere), grouped by rank in ascending token order;
+    a2a_combine adds the returned rows in that order."""
+    import torch
+    from quantized_expert_ffn_logits_b200 import ep
+    ranges = [(0, 3), (3, 3), (6, 2)]
+    idx = torch.tensor([[0, 4], [6, -1], [1, 2], [3, 7], [-1, -1]])
+    send, counts = ep.a2a_plan(idx, ranges, 0)
+    assert counts == [0, 2, 2] and send.tolist() == [0, 3, 1, 3]
+    send1, counts1 = ep.a2a_plan(idx, ranges, 1)
+    assert counts1 == [2, 0, 2] and send1.tolist() == [0, 2, 1, 3]
+    y = torch.zeros(5, 2, dtype=torch.float64)
+    back = torch.arange(8, dtype=torch.float64).reshape(4, 2)
+    ep.a2a_combine(y, send, counts, back)
+    assert y.tolist() == [[0, 1], [4, 5], [0, 0], [8, 10], [0, 0]]
