@@ -141,66 +141,11 @@ __global__ void __launch_bounds__(256) k_quantize_experts(const WSource w, BlobV
   }
 }
 
-// Group-32 activations, one warp per token: lane l holds the float4 pieces l, l + 32, ... of
-// the row, so the eight pieces of a group sit on eight adjacent lanes (the group maximum is
-// three xor-shuffles). A lane loads eight pieces before converting any: eight 16-byte loads
-// in flight per thread. Optionally zeroes the token's output row (the layer accumulates y);
-// block 0 clears the status words.
-constexpr int kActPieces = 8;
-__global__ void __launch_bounds__(256) k_quantize_act_g32(const float* __restrict__ x, int T, int H,
-                                                          int8_t* __restrict__ q,
-                                                          __half* __restrict__ sq,
-                                                          float* __restrict__ y_zero, int* status) {
-  pdl_wait();
-  pdl_trigger();
-  if (status && blockIdx.x == 0 && threadIdx.x == 0) {
-    status[0] = 0;
-    status[2] = 0;
-    status[3] = 0;
-  }
-  const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;                                   // whole warps leave together
-  const int np = H / 4;                                 // float4 pieces in the row
-  const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)t * H);
-  for (int p0 = 0; p0 * 32 < np; p0 += kActPieces) {
-    float4 v[kActPieces];
-#pragma unroll
-    for (int u = 0; u < kActPieces; ++u) {
-      const int P = lane + 32 * (p0 + u);
-      v[u] = P < np ? __ldcs(xr + P) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kActPieces; ++u) {
-      if ((p0 + u) * 32 >= np) break;                   // warp-uniform
-      const int P = lane + 32 * (p0 + u);
-      const float4 a = v[u];
-      float m = fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w)));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      if (P < np) {                                     // groups are whole: np is a multiple of 8
-        const float s = f16_round(__fdiv_rn(m, 127.0f));
-        const float rs = __frcp_rn(s);
-        char4 c;
-        c.x = (signed char)quant_code_rcp(a.x, s, rs, 127.0f);
-        c.y = (signed char)quant_code_rcp(a.y, s, rs, 127.0f);
-        c.z = (signed char)quant_code_rcp(a.z, s, rs, 127.0f);
-        c.w = (signed char)quant_code_rcp(a.w, s, rs, 127.0f);
-        reinterpret_cast<char4*>(q + (int64_t)t * H)[P] = c;
-        if ((lane & 7) == 0) sq[(int64_t)t * (H / 32) + P / 8] = __float2half_rn(s);
-        if (y_zero) reinterpret_cast<float4*>(y_zero + (int64_t)t * H)[P] = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-  }
-}
-
-// Token mode: one CTA per token, one fp32 scale over the row. Optionally zeroes the token's
-// output row; block 0 clears the status words.
-__global__ void __launch_bounds__(256) k_quantize_act_token(const float* __restrict__ x, int T,
-                                                            int H, int8_t* __restrict__ q,
-                                                            float* __restrict__ scales,
-                                                            float* __restrict__ y_zero, int* status) {
+// One CTA per token. g32: a warp per group of 32; token mode: one fp32 scale over
+// the row. Optionally zeroes the token's output row (the layer accumulates y).
+__global__ void __launch_bounds__(256) k_quantize_act(const float* __restrict__ x, int T, int H,
+                                                      int g32, int8_t* __restrict__ q,
+                                                      void* scales, float* y_zero, int* status) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;
@@ -217,22 +162,32 @@ __global__ void __launch_bounds__(256) k_quantize_act_token(const float* __restr
     float4* yr = reinterpret_cast<float4*>(y_zero + (int64_t)t * H);
     for (int k = threadIdx.x; k < H / 4; k += blockDim.x) yr[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  __shared__ float red[32];
-  float amax = 0.0f;
-  for (int k = threadIdx.x; k < H; k += blockDim.x) amax = fmaxf(amax, fabsf(xr[k]));
-  amax = warp_max(amax);
-  if (lane == 0) red[warp] = amax;
-  __syncthreads();
-  if (warp == 0) {
-    float v = lane < nw ? red[lane] : 0.0f;
-    v = warp_max(v);
-    if (lane == 0) red[0] = v;
+  if (g32) {
+    __half* sr = reinterpret_cast<__half*>(scales) + (int64_t)t * (H / 32);
+    for (int g = warp; g < H / 32; g += nw) {
+      const float v = xr[32 * g + lane];
+      const float s = f16_round(__fdiv_rn(warp_max(fabsf(v)), 127.0f));
+      qr[32 * g + lane] = (int8_t)quant_code_rcp(v, s, __frcp_rn(s), 127.0f);
+      if (lane == 0) sr[g] = __float2half_rn(s);
+    }
+  } else {
+    __shared__ float red[32];
+    float amax = 0.0f;
+    for (int k = threadIdx.x; k < H; k += blockDim.x) amax = fmaxf(amax, fabsf(xr[k]));
+    amax = warp_max(amax);
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    if (warp == 0) {
+      float v = lane < nw ? red[lane] : 0.0f;
+      v = warp_max(v);
+      if (lane == 0) red[0] = v;
+    }
+    __syncthreads();
+    const float s = __fdiv_rn(red[0], 127.0f);
+    const float rs = __frcp_rn(s);
+    for (int k = threadIdx.x; k < H; k += blockDim.x) qr[k] = (int8_t)quant_code_rcp(xr[k], s, rs, 127.0f);
+    if (threadIdx.x == 0) reinterpret_cast<float*>(scales)[t] = s;
   }
-  __syncthreads();
-  const float s = __fdiv_rn(red[0], 127.0f);
-  const float rs = __frcp_rn(s);
-  for (int k = threadIdx.x; k < H; k += blockDim.x) qr[k] = (int8_t)quant_code_rcp(xr[k], s, rs, 127.0f);
-  if (threadIdx.x == 0) scales[t] = s;
 }
 
 // Token-mode quantization of h (one fp32 scale per (token, expert) over I).
@@ -292,12 +247,7 @@ void launch_quantize_experts_fp8(const uint8_t* w_gu, const float* s_gu, const u
 void launch_quantize_act(const float* x, int T, int H, int g32, int8_t* q, void* scales,
                          float* y_zero, int* status, cudaStream_t st) {
   if (T <= 0) return;
-  if (g32)
-    launch_pdl(k_quantize_act_g32, dim3((T + 7) / 8), dim3(256), 0, st, x, T, H, q,
-               static_cast<__half*>(scales), y_zero, status);
-  else
-    launch_pdl(k_quantize_act_token, dim3(T), dim3(256), 0, st, x, T, H, q,
-               static_cast<float*>(scales), y_zero, status);
+  launch_pdl(k_quantize_act, dim3(T), dim3(256), 0, st, x, T, H, g32, q, scales, y_zero, status);
 }
 
 void launch_quantize_rows_token(const float* h, int rows, int K, int8_t* q, float* scales,

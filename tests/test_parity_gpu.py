@@ -329,7 +329,7 @@ def test_quantize_experts_fp8_blob_bytes_identical(wtype, wscale, E, H, I):
 
 
 @pytest.mark.parametrize("act", ["g32_f16", "token_f32"])
-# (H = 32, 96, 160: rows whose float4 pieces fill a warp once, partly, or once and a quarter)
+# (H = 32, 96, 160: fewer groups than a CTA has warps, and groups that do not divide among them)
 @pytest.mark.parametrize("T,H,sigma", [(1, 2048, 1.0), (7, 256, 0.02), (65, 6144, 3.0), (3, 32, 1.0),
                                        (9, 96, 1.0), (17, 160, 0.5)])
 def test_quantize_activations_bit_exact(act, T, H, sigma):
