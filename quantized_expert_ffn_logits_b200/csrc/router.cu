@@ -165,6 +165,136 @@ __global__ void __launch_bounds__(256) k_router_tiled(const float* __restrict__ 
   }
 }
 
+// The 32-token tile with the K loop split over two warp groups (512 threads): group g takes
+// the chunks c = g (mod 2), each with the same thread tile as k_router_tiled, its own double
+// buffer and one chunk of loads in flight. After each step (chunks 2s and 2s + 1) group 1 hands
+// its chunk partials to group 0 through shared memory, and group 0 adds chunk 2s's partial and
+// then chunk 2s + 1's to its running totals: the same chains and the same order of additions,
+// with twice the warps per SM to cover the shared-memory load latency.
+constexpr int kRouterKsTT = 32;
+struct RouterKsSmem {
+  float xs[2][2][32][kRouterKsTT + 4];   // [group][buffer][k][token]
+  float ws[2][2][32][64 + 4];            // [group][buffer][k][expert]
+  float pb[2][256][8];                   // [step parity][group-1 thread][output]
+};
+
+__global__ void __launch_bounds__(512) k_router_tiled_ks(const float* __restrict__ x,
+                                                         const float* __restrict__ wr, int T,
+                                                         int E, int H, float* __restrict__ logits) {
+  constexpr int TT = kRouterKsTT, RT = TT / 16, XV = TT * 8 / 256;
+  extern __shared__ __align__(16) uint8_t ks_raw[];
+  RouterKsSmem& S = *reinterpret_cast<RouterKsSmem*>(ks_raw);
+  pdl_wait();
+  pdl_trigger();
+  const int grp = threadIdx.x >> 8, gt = threadIdx.x & 255;
+  const int tb = blockIdx.y * TT, eb = blockIdx.x * 64;
+  const int ty = gt >> 4, tx = gt & 15;
+  const int C = H / 32;
+  float4 xr[XV], wrg[2];
+  auto load = [&](int c) {
+#pragma unroll
+    for (int v = 0; v < XV; ++v) {
+      const int l = gt + 256 * v, rr = l >> 3, k4 = l & 7;
+      const int t = tb + rr;
+      xr[v] = t < T ? __ldg(reinterpret_cast<const float4*>(x + (int64_t)t * H + 32 * c) + k4)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int l = gt + 256 * v, rr = l >> 3, k4 = l & 7;
+      const int e = eb + rr;
+      wrg[v] = e < E ? __ldg(reinterpret_cast<const float4*>(wr + (int64_t)e * H + 32 * c) + k4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto store = [&](int b) {
+#pragma unroll
+    for (int v = 0; v < XV; ++v) {
+      const int l = gt + 256 * v, rr = l >> 3, k = 4 * (l & 7);
+      S.xs[grp][b][k][rr] = xr[v].x;
+      S.xs[grp][b][k + 1][rr] = xr[v].y;
+      S.xs[grp][b][k + 2][rr] = xr[v].z;
+      S.xs[grp][b][k + 3][rr] = xr[v].w;
+    }
+#pragma unroll
+    for (int v = 0; v < 2; ++v) {
+      const int l = gt + 256 * v, rr = l >> 3, k = 4 * (l & 7);
+      S.ws[grp][b][k][rr] = wrg[v].x;
+      S.ws[grp][b][k + 1][rr] = wrg[v].y;
+      S.ws[grp][b][k + 2][rr] = wrg[v].z;
+      S.ws[grp][b][k + 3][rr] = wrg[v].w;
+    }
+  };
+  float total[RT][4];
+#pragma unroll
+  for (int i = 0; i < RT; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) total[i][j] = 0.0f;
+  if (grp < C) {
+    load(grp);
+    store(0);
+  }
+  __syncthreads();
+  const int steps = (C + 1) / 2;
+  for (int s = 0; s < steps; ++s) {
+    const int b = s & 1;
+    const int c = 2 * s + grp;                 // this group's chunk of the step
+    const bool mine = c < C;
+    if (c + 2 < C) load(c + 2);
+    float part[RT][4];
+#pragma unroll
+    for (int i = 0; i < RT; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) part[i][j] = 0.0f;
+    if (mine) {
+#pragma unroll 8
+      for (int kk = 0; kk < 32; ++kk) {
+        const float2 a = *reinterpret_cast<const float2*>(&S.xs[grp][b][kk][ty * 2]);
+        const float av[RT] = {a.x, a.y};
+        const float4 bw = *reinterpret_cast<const float4*>(&S.ws[grp][b][kk][tx * 4]);
+        const float bv[4] = {bw.x, bw.y, bw.z, bw.w};
+#pragma unroll
+        for (int i = 0; i < RT; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) part[i][j] = __fmaf_rn(av[i], bv[j], part[i][j]);
+      }
+    }
+    if (grp == 1 && mine) {
+      float4* pb = reinterpret_cast<float4*>(S.pb[b][gt]);
+      pb[0] = make_float4(part[0][0], part[0][1], part[0][2], part[0][3]);
+      pb[1] = make_float4(part[1][0], part[1][1], part[1][2], part[1][3]);
+    }
+    if (c + 2 < C) store(b ^ 1);
+    __syncthreads();
+    if (grp == 0) {
+#pragma unroll
+      for (int i = 0; i < RT; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) total[i][j] = __fadd_rn(total[i][j], part[i][j]);
+      if (2 * s + 1 < C) {
+        const float4* pb = reinterpret_cast<const float4*>(S.pb[b][gt]);
+        const float4 p0 = pb[0], p1 = pb[1];
+        const float q[RT][4] = {{p0.x, p0.y, p0.z, p0.w}, {p1.x, p1.y, p1.z, p1.w}};
+#pragma unroll
+        for (int i = 0; i < RT; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) total[i][j] = __fadd_rn(total[i][j], q[i][j]);
+      }
+    }
+  }
+  if (grp != 0) return;
+#pragma unroll
+  for (int i = 0; i < RT; ++i) {
+    const int t = tb + ty * RT + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = eb + tx * 4 + j;
+      if (e < E) logits[(int64_t)t * E + e] = total[i][j];
+    }
+  }
+}
+
 void launch_router_logits(const float* x, const float* wr, int T, int E, int H, float* logits,
                           cudaStream_t st) {
   if (T <= 0) return;
@@ -180,7 +310,12 @@ void launch_router_logits(const float* x, const float* wr, int T, int E, int H, 
     const int64_t tiles64 = (int64_t)((E + 63) / 64) * ((T + 63) / 64);
     if (tiles64 < 2 * 148) {
       dim3 grid((E + 63) / 64, (T + 31) / 32);
-      launch_pdl(k_router_tiled<32>, grid, dim3(256), 0, st, x, wr, T, E, H, logits);
+      // the K-split tile (68 KB of shared memory); the plain tile if that cannot be granted
+      constexpr int smem = (int)sizeof(RouterKsSmem);
+      if (ensure_smem_attr(reinterpret_cast<const void*>(k_router_tiled_ks), smem) == cudaSuccess)
+        launch_pdl(k_router_tiled_ks, grid, dim3(512), (size_t)smem, st, x, wr, T, E, H, logits);
+      else
+        launch_pdl(k_router_tiled<32>, grid, dim3(256), 0, st, x, wr, T, E, H, logits);
     } else {
       dim3 grid((E + 63) / 64, (T + 63) / 64);
       launch_pdl(k_router_tiled<64>, grid, dim3(256), 0, st, x, wr, T, E, H, logits);
