@@ -43,7 +43,6 @@ __global__ void __launch_bounds__(1024) k_mma_plan(const int32_t* __restrict__ n
   __shared__ int carry;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_wait();
-  pdl_trigger();
   const int na = min(*n_active, E);
   if (tid == 0) carry = 0;
   __syncthreads();
@@ -134,7 +133,6 @@ __global__ void __launch_bounds__(256) k_mma_gather(const int8_t* __restrict__ q
                                                     const int32_t* __restrict__ perm, int k, int T, int K,
                                                     uint8_t* __restrict__ xa, __half* __restrict__ xs, int* status) {
   pdl_wait();
-  pdl_trigger();
   const int G = K / 32;
   const int nt = *n_tiles;
   const int64_t per_tile = (int64_t)128 * G;

@@ -147,7 +147,6 @@ __global__ void __launch_bounds__(256) k_quantize_act(const float* __restrict__ 
                                                       int g32, int8_t* __restrict__ q,
                                                       void* scales, float* y_zero, int* status) {
   pdl_wait();
-  pdl_trigger();
   const int t = blockIdx.x;
   if (t >= T) return;
   if (status && t == 0 && threadIdx.x == 0) {

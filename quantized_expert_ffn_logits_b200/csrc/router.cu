@@ -24,7 +24,6 @@ __global__ void __launch_bounds__(256) k_router_small(const float* __restrict__ 
                                                       int H, float* __restrict__ logits) {
   extern __shared__ float part[];  // [TT][C]
   pdl_wait();
-  pdl_trigger();
   const int e = blockIdx.x;
   const int t0 = blockIdx.y * TT;
   const int C = H / 32;
@@ -70,7 +69,6 @@ __global__ void __launch_bounds__(256) k_router_tiled(const float* __restrict__ 
   __shared__ __align__(16) float xs[2][32][TT + 4];
   __shared__ __align__(16) float ws[2][32][64 + 4];
   pdl_wait();
-  pdl_trigger();
   const int tb = blockIdx.y * TT, eb = blockIdx.x * 64;
   const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
   const int C = H / 32;
@@ -185,7 +183,6 @@ __global__ void __launch_bounds__(512) k_router_tiled_ks(const float* __restrict
   extern __shared__ __align__(16) uint8_t ks_raw[];
   RouterKsSmem& S = *reinterpret_cast<RouterKsSmem*>(ks_raw);
   pdl_wait();
-  pdl_trigger();
   const int grp = threadIdx.x >> 8, gt = threadIdx.x & 255;
   const int tb = blockIdx.y * TT, eb = blockIdx.x * 64;
   const int ty = gt >> 4, tx = gt & 15;
@@ -332,7 +329,6 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ logits,
                                               int32_t* __restrict__ idx, float* __restrict__ w,
                                               Grouping g1, int single, int* status) {
   pdl_wait();
-  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -421,7 +417,6 @@ __global__ void __launch_bounds__(1024) k_permute(const int32_t* __restrict__ id
     else return __ldcg(base + i);
   };
   pdl_wait();
-  pdl_trigger();
   if (reset_status && tid == 0 && status) *status = 0;
   if (SM)
     for (int i = tid; i < C * E; i += 1024) masks[i] = 0u;
