@@ -147,8 +147,8 @@ __device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint3
 
 // Programmatic dependent launch: wait for the preceding grid (and its memory), and let the
 // next grid in the stream start its prologue. The batch routing kernels (activation
-// quantization, router logits, top-k, grouping, tile plan, operand gather) do not trigger
-// early: their successors launch when they complete. Launched early, a successor's CTAs take
+// quantization, router logits, top-k, grouping, tile plan, operand gather) and the streaming
+// expert kernel's batch modes do not trigger early: their successors launch when they complete. Launched early, a successor's CTAs take
 // the SMs that the rest of the running grid still needs (measured on the graph-replayed
 // prefill step: the single-wave activation quantization lost ~100 us to it; with no early
 // triggers in these kernels the step is ~6 us shorter than with them).
