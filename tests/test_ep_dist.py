@@ -131,8 +131,8 @@ def test_least_loaded_placement():
     assert np.array_equal(rw2[1], rw[0]) and np.array_equal(rw2[0], rw[3])
 
 
-# all-to-all exchange: three ranks with different token counts (one with a single token)
-T_A2A = [4, 1, 6]
+# all-to-all exchange: ranks with different token counts (one with a single token, one with none)
+A2A_SPLITS = [[4, 1, 6], [3, 0, 5, 2]]
 
 
 def _oracle_x(x):
@@ -146,7 +146,7 @@ def _oracle_x(x):
                            CFG.renormalize, CFG.rsf, True)
 
 
-def _worker_a2a(rank, world, port, q):
+def _worker_a2a(rank, world, port, q, t_a2a):
     import torch
     import torch.distributed as dist
     from quantized_expert_ffn_logits_b200 import ep
@@ -155,10 +155,13 @@ def _worker_a2a(rank, world, port, q):
     try:
         ranges = ep.expert_ranges(CFG.E, world)
         begin, count = ranges[rank]
-        x_local = torch.from_numpy(S.normal_cpu(T_A2A[rank] * CFG.H, 700 + rank, 0, 1.0).reshape(T_A2A[rank], CFG.H))
+        n = t_a2a[rank]
+        x_local = torch.from_numpy(S.normal_cpu(max(n, 1) * CFG.H, 700 + rank, 0, 1.0).reshape(max(n, 1), CFG.H)[:n])
         npairs = [0, 0]
 
         def local_sum(x, with_shared):
+            if x.shape[0] == 0:
+                return x.new_zeros((0, CFG.H)), torch.zeros((0, CFG.top_k), dtype=torch.int64)
             o = _oracle_x(x.numpy())
             T, k = o["idx"].shape
             y = np.zeros((T, CFG.H))
@@ -188,16 +191,17 @@ def _worker_a2a(rank, world, port, q):
     q.put((rank, y.numpy(), counts, np.concatenate(xs)))
 
 
-def test_three_rank_all_to_all_step_equals_the_whole_layer():
-    """ep_step_a2a on three gloo ranks holding 4, 1 and 6 tokens (uneven splits, some of them
-    empty): every rank's rows equal the oracle's whole layer on all tokens, every routed pair
-    is computed exactly once over all ranks (on the rank holding its expert), and the shared
-    expert once per token (on the token's rank)."""
+@pytest.mark.parametrize("t_a2a", A2A_SPLITS)
+def test_all_to_all_step_equals_the_whole_layer(t_a2a):
+    """ep_step_a2a on gloo ranks holding 4, 1 and 6 tokens, or 3, 0, 5 and 2 (uneven splits,
+    empty ones, a rank with no tokens at all): every rank's rows equal the oracle's whole layer
+    on all tokens, every routed pair is computed exactly once over all ranks (on the rank holding
+    its expert), and the shared expert once per token (on the token's rank)."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    world = len(T_A2A)
-    procs = [ctx.Process(target=_worker_a2a, args=(r, world, port, q)) for r in range(world)]
+    world = len(t_a2a)
+    procs = [ctx.Process(target=_worker_a2a, args=(r, world, port, q, t_a2a)) for r in range(world)]
     for p in procs:
         p.start()
     res = sorted(q.get(timeout=240) for _ in procs)
@@ -206,13 +210,15 @@ def test_three_rank_all_to_all_step_equals_the_whole_layer():
         assert p.exitcode == 0
     x_all = res[0][3]
     ref = _oracle_x(x_all)
-    st = np.cumsum([0] + T_A2A)
+    st = np.cumsum([0] + t_a2a)
     for rank, y, _, _ in res:
         want = ref["y"][st[rank]:st[rank + 1]]
-        assert np.allclose(y, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+        assert y.shape == want.shape
+        if want.size:
+            assert np.allclose(y, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
     counts = res[0][2]
-    assert sum(c[0] for c in counts) == sum(T_A2A) * CFG.top_k
-    assert [c[1] for c in counts] == T_A2A
+    assert sum(c[0] for c in counts) == sum(t_a2a) * CFG.top_k
+    assert [c[1] for c in counts] == t_a2a
 
 
 def test_dispatch_plan_and_combine():
