@@ -440,10 +440,11 @@ struct StageMarks {
   void end(int s) { if (ev) mark(ev->end[s]); }
 };
 
+// host_copy: the host-buffer entry, whose output copy kernel follows the layer's last kernel.
 moe_status forward_impl(const float* x, int32_t T, const float* router_w, const float* router_bias,
                         const moe_expert_blob* experts, const moe_expert_blob* shared,
                         const moe_route_cfg* cfg, float* y, void* workspace, size_t ws_bytes,
-                        void* stream, const moe_stage_events* events) {
+                        void* stream, const moe_stage_events* events, bool host_copy = false) {
   LayerPlan p;
   moe_status s = plan_layer(T, experts, shared, cfg, p);
   if (s != MOE_OK) return s;
@@ -553,6 +554,7 @@ moe_status forward_impl(const float* x, int32_t T, const float* router_w, const 
   //    experts in one grid
   moe::ExpertArgs ra;
   std::memset(&ra, 0, sizeof(ra));
+  ra.early_trigger = host_copy ? 1 : 0;
   ra.b = bv;
   ra.qa = static_cast<const int8_t*>(at(L.qx));
   ra.sa = at(L.sx);
@@ -742,7 +744,7 @@ moe_status moe_layer_forward_host(const float* x_host, int32_t T, const float* r
                          : cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st);
   if (e != cudaSuccess) return cuda_fail("x host-to-device copy", e);
   const moe_status s = forward_impl(x_dev, T, router_w, router_bias, experts, shared, cfg, y_dev, workspace,
-                                    ws_bytes, stream, nullptr);
+                                    ws_bytes, stream, nullptr, true);
   if (s != MOE_OK) return s;
   e = mapped ? moe::launch_copy_out(y_dev, static_cast<float*>(ym), n, st)
              : cudaMemcpyAsync(y_host, y_dev, bytes, cudaMemcpyDeviceToHost, st);

@@ -1348,8 +1348,9 @@ __global__ void __launch_bounds__(kNT, 1) k_expert_ring(const __grid_constant__ 
   // the routing's grid barrier (with the cluster exchange after the y-zero barrier, consumers,
   // below). The batch modes let it launch when this grid completes: launched early, its CTAs
   // took SMs this grid still needed (measured on graph-replayed steps: -2.1 % at OLMoE int8
-  // T = 8, -2.6 % at GLM int4 T = 4, no change at T = 4096)
-  if (MODE == 3 && !A.cluster) pdl_trigger();
+  // T = 8, -2.6 % at GLM int4 T = 4, no change at T = 4096) -- except before the host-buffer
+  // path's small output copy, which is better launched early
+  if (MODE == 3 ? !A.cluster : A.x[0][0].early_trigger != 0) pdl_trigger();
 
   if (warp == kCW) {
     if (lane == 0) ring_producer<WBITS, WG32, AG32, MODE, TOPP>(A, P, R, S);

@@ -85,6 +85,8 @@ struct ExpertArgs {
   int32_t* dbg_dots;         // down: int32 group dots [slots][H][I/32] (debug)
   float* y;                  // down: [T][H] accumulated
   int* status;
+  int early_trigger;         // streaming kernel, batch modes: let the next kernel launch early
+                             // (the host-buffer path, where a small output copy follows)
 };
 
 // Routed experts and (optional) shared expert: gate/up args gr/gs, down args dr/ds. Work
