@@ -105,18 +105,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
-// The same for a thread that runs ahead of its consumers (a producer or issuer): between
-// non-blocking tests it sleeps ~ns nanoseconds, so its waiting takes few issue slots from the
-// warps that set the pace. Bounded at about a second.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
-  const uint32_t tries = 1000000000u / (ns + 64u);
-  for (uint32_t i = 0; i < tries; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    __nanosleep(ns);
-  }
-  return false;
-}
-
 // Untiled bulk copy global -> this CTA's shared memory (16-byte aligned addresses, size a
 // multiple of 16), completing on `bar` (transaction bytes).
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
